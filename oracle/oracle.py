@@ -1,0 +1,295 @@
+"""ctypes front end of the FP64 oracle (fc_oracle.c).
+
+TEST INFRASTRUCTURE ONLY.  Inputs are promoted to float64 and made
+contiguous here; every computation happens in the C source, which follows
+the FlashCart pages (arXiv 2610.06409) as cited there.
+"""
+import ctypes as ct
+import os
+
+import numpy as np
+
+from . import build as _build
+
+_lib = None
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        path = _build.build()
+        L = ct.CDLL(path)
+        d = ct.POINTER(ct.c_double)
+        i32 = ct.POINTER(ct.c_int32)
+        ip = ct.POINTER(ct.c_int)
+        u8 = ct.POINTER(ct.c_ubyte)
+        sig = {
+            "orc_permavg": (None, [ct.c_int, d, d]),
+            "orc_detrace": (None, [ct.c_int, d, d]),
+            "orc_stf_dense": (None, [ct.c_int, d, d]),
+            "orc_stf_extract": (None, [ct.c_int, d, d]),
+            "orc_comp_pxyz": (None, [ct.c_int, ct.c_int, ip, ip, ip]),
+            "orc_direction_dense": (None, [ct.c_int, d, d]),
+            "orc_direction": (None, [ct.c_int, d, d]),
+            "orc_direction_jac": (None, [ct.c_int, d, d]),
+            "orc_admissible": (ct.c_int, [ct.c_int] * 3),
+            "orc_path_norm": (ct.c_double, [ct.c_int] * 3),
+            "orc_product_dense": (ct.c_int, [ct.c_int] * 3 + [d, d, d, ct.c_int]),
+            "orc_product": (ct.c_int, [ct.c_int] * 3 + [d, d, d]),
+            "orc_path_coeffs": (None, [ct.c_int] * 3 + [d]),
+            "orc_paths": (ct.c_int, [ct.c_int] * 3 + [ip, ip, ip]),
+            "orc_edge_conv": (ct.c_int, [ct.c_int] * 7 + [i32, i32, d, d, d, u8, d]),
+            "orc_edge_conv_vjp": (ct.c_int, [ct.c_int] * 7 + [i32, i32, d, d, d, d, u8, d, d, d]),
+            "orc_ladder": (ct.c_int, [ct.c_int] * 4 + [d, d, d, u8, d, d]),
+            "orc_ladder_vjp": (ct.c_int, [ct.c_int] * 4 + [d, d, d, d, u8, d, d, d]),
+            "orc_max_rank": (ct.c_int, []),
+            "orc_num_threads": (ct.c_int, []),
+        }
+        for name, (res, args) in sig.items():
+            f = getattr(L, name)
+            f.restype = res
+            f.argtypes = args
+        _lib = L
+    return _lib
+
+
+def _d(a):
+    return np.ascontiguousarray(a, dtype=np.float64)
+
+
+def _pd(a):
+    if a is None:
+        return None
+    return a.ctypes.data_as(ct.POINTER(ct.c_double))
+
+
+def _pi32(a):
+    return a.ctypes.data_as(ct.POINTER(ct.c_int32))
+
+
+def _pu8(a):
+    if a is None:
+        return None
+    return a.ctypes.data_as(ct.POINTER(ct.c_ubyte))
+
+
+def _mask(m, n):
+    if m is None:
+        return None
+    m = np.ascontiguousarray(np.asarray(m, dtype=np.uint8))
+    assert m.shape == (n,)
+    return m
+
+
+# --------------------------------------------------------------------------
+# tensors
+# --------------------------------------------------------------------------
+
+def permavg(l, t):
+    t = _d(t).reshape(-1)
+    out = np.empty(3 ** l)
+    lib().orc_permavg(l, _pd(t), _pd(out))
+    return out.reshape((3,) * l)
+
+
+def detrace(l, t):
+    t = _d(t).reshape(-1)
+    out = np.empty(3 ** l)
+    lib().orc_detrace(l, _pd(t), _pd(out))
+    return out.reshape((3,) * l)
+
+
+def stf_dense(l, comps):
+    c = _d(comps)
+    assert c.shape == (2 * l + 1,)
+    out = np.empty(3 ** l)
+    lib().orc_stf_dense(l, _pd(c), _pd(out))
+    return out.reshape((3,) * l)
+
+
+def stf_extract(l, dense):
+    t = _d(dense).reshape(-1)
+    out = np.empty(2 * l + 1)
+    lib().orc_stf_extract(l, _pd(t), _pd(out))
+    return out
+
+
+def comp_pxyz(l, c):
+    a, b, z = ct.c_int(), ct.c_int(), ct.c_int()
+    lib().orc_comp_pxyz(l, c, ct.byref(a), ct.byref(b), ct.byref(z))
+    return a.value, b.value, z.value
+
+
+def direction_dense(l, r):
+    r = _d(r)
+    out = np.empty(3 ** l)
+    lib().orc_direction_dense(l, _pd(r), _pd(out))
+    return out.reshape((3,) * l)
+
+
+def direction(l, r):
+    r = _d(r)
+    out = np.empty(2 * l + 1)
+    lib().orc_direction(l, _pd(r), _pd(out))
+    return out
+
+
+def direction_jac(l, r):
+    r = _d(r)
+    out = np.empty((2 * l + 1) * 3)
+    lib().orc_direction_jac(l, _pd(r), _pd(out))
+    return out.reshape(2 * l + 1, 3)
+
+
+def admissible(l1, l2, l3):
+    return bool(lib().orc_admissible(l1, l2, l3))
+
+
+def path_norm(l1, l2, l3):
+    return lib().orc_path_norm(l1, l2, l3)
+
+
+def product_dense(l1, l2, l3, x, y, route=0):
+    x, y = _d(x), _d(y)
+    out = np.empty(3 ** l3)
+    rc = lib().orc_product_dense(l1, l2, l3, _pd(x), _pd(y), _pd(out), route)
+    if rc:
+        raise ValueError("path (%d,%d)->%d not admissible" % (l1, l2, l3))
+    return out.reshape((3,) * l3)
+
+
+def product(l1, l2, l3, x, y):
+    x, y = _d(x), _d(y)
+    out = np.empty(2 * l3 + 1)
+    rc = lib().orc_product(l1, l2, l3, _pd(x), _pd(y), _pd(out))
+    if rc:
+        raise ValueError("path (%d,%d)->%d not admissible" % (l1, l2, l3))
+    return out
+
+
+def path_coeffs(l1, l2, l3):
+    out = np.empty((2 * l3 + 1) * (2 * l1 + 1) * (2 * l2 + 1))
+    lib().orc_path_coeffs(l1, l2, l3, _pd(out))
+    return out.reshape(2 * l3 + 1, 2 * l1 + 1, 2 * l2 + 1)
+
+
+def paths(lin, ledge, lout):
+    n = lib().orc_paths(lin, ledge, lout, None, None, None)
+    a = (ct.c_int * max(n, 1))()
+    b = (ct.c_int * max(n, 1))()
+    c = (ct.c_int * max(n, 1))()
+    lib().orc_paths(lin, ledge, lout, a, b, c)
+    return [(a[i], b[i], c[i]) for i in range(n)]
+
+
+def num_threads():
+    return lib().orc_num_threads()
+
+
+# --------------------------------------------------------------------------
+# edge convolution (Sec. 4 Eq. 1) and its VJP (App. C Eq. C1)
+# --------------------------------------------------------------------------
+
+def zrow(lin, ledge, lout, sum_paths=False):
+    """Output row length / C for the edge convolution."""
+    ps = paths(lin, ledge, lout)
+    if sum_paths:
+        return (lout + 1) ** 2
+    return sum(2 * l3 + 1 for (_, _, l3) in ps)
+
+
+def edge_conv(lin, ledge, lout, C, edge_index, edge_vec, x, w, n_nodes,
+              sum_paths=False, recv_mask=None):
+    """z = Eq. (1).  With recv_mask, only the listed receivers' rows are
+    computed (their edges are selected here; other rows stay zero)."""
+    ei = np.asarray(edge_index)
+    P = len(paths(lin, ledge, lout))
+    if recv_mask is not None:
+        m = _mask(recv_mask, n_nodes)
+        sel = np.nonzero(m[ei[0]])[0]
+        ei, edge_vec, w = ei[:, sel], np.asarray(edge_vec)[sel], np.asarray(w)[sel]
+    ei = np.ascontiguousarray(ei, dtype=np.int32)
+    E = ei.shape[1]
+    recv = np.ascontiguousarray(ei[0])
+    send = np.ascontiguousarray(ei[1])
+    vec = _d(edge_vec).reshape(E, 3)
+    x = _d(x)
+    w = _d(w).reshape(E, P, C)
+    assert x.shape == (n_nodes, (lin + 1) ** 2 * C)
+    zr = zrow(lin, ledge, lout, sum_paths)
+    z = np.empty((n_nodes, zr * C))
+    rc = lib().orc_edge_conv(lin, ledge, lout, C, int(sum_paths), n_nodes, E,
+                             _pi32(recv), _pi32(send), _pd(vec), _pd(x), _pd(w),
+                             None, _pd(z))
+    assert rc == 0
+    return z
+
+
+def edge_conv_vjp(lin, ledge, lout, C, edge_index, edge_vec, x, w, g, n_nodes,
+                  sum_paths=False, edge_mask=None, want=("x", "w", "r")):
+    """Eq. (C1) summed over edges.  With edge_mask, only the listed edges
+    contribute (they are selected here); w_bar / r_bar rows of the other
+    edges are zero."""
+    ei_full = np.asarray(edge_index)
+    E_full = ei_full.shape[1]
+    P = len(paths(lin, ledge, lout))
+    sel = None
+    ei, ev, ww = ei_full, np.asarray(edge_vec), np.asarray(w)
+    if edge_mask is not None:
+        sel = np.nonzero(_mask(edge_mask, E_full))[0]
+        ei, ev, ww = ei[:, sel], ev[sel], ww[sel]
+    ei = np.ascontiguousarray(ei, dtype=np.int32)
+    E = ei.shape[1]
+    recv = np.ascontiguousarray(ei[0])
+    send = np.ascontiguousarray(ei[1])
+    vec = _d(ev).reshape(E, 3)
+    x, ww, g = _d(x), _d(ww).reshape(E, P, C), _d(g)
+    xb = np.empty(((n_nodes, (lin + 1) ** 2 * C))) if "x" in want else None
+    wb = np.empty((E, P, C)) if "w" in want else None
+    rb = np.empty((E, 3)) if "r" in want else None
+    rc = lib().orc_edge_conv_vjp(lin, ledge, lout, C, int(sum_paths), n_nodes, E,
+                                 _pi32(recv), _pi32(send), _pd(vec), _pd(x),
+                                 _pd(ww), _pd(g), None, _pd(xb), _pd(wb), _pd(rb))
+    assert rc == 0
+    if sel is not None:
+        if wb is not None:
+            full = np.zeros((E_full, P, C)); full[sel] = wb; wb = full
+        if rb is not None:
+            full = np.zeros((E_full, 3)); full[sel] = rb; rb = full
+    return xb, wb, rb
+
+
+# --------------------------------------------------------------------------
+# node-local ladder (Sec. 5 Eq. 2, path-reduced products + per-rank mixing)
+# --------------------------------------------------------------------------
+
+def ladder(L, C, order, A1, path_w, mix_w, node_mask=None):
+    A1 = _d(A1)
+    N = A1.shape[0]
+    P = len(paths(L, L, L))
+    path_w = _d(path_w).reshape(max(order - 1, 0), P, C)
+    mix_w = _d(mix_w).reshape(max(order - 1, 0), L + 1, C, C)
+    states = np.empty((max(order - 1, 0), N, (L + 1) ** 2 * C))
+    z = np.empty((N, (L + 1) ** 2 * C))
+    m = _mask(node_mask, N)
+    rc = lib().orc_ladder(L, C, order, N, _pd(A1), _pd(path_w), _pd(mix_w),
+                          _pu8(m), _pd(states), _pd(z))
+    assert rc == 0
+    return states, z
+
+
+def ladder_vjp(L, C, order, A1, path_w, mix_w, gz, node_mask=None):
+    A1 = _d(A1)
+    N = A1.shape[0]
+    P = len(paths(L, L, L))
+    path_w = _d(path_w).reshape(max(order - 1, 0), P, C)
+    mix_w = _d(mix_w).reshape(max(order - 1, 0), L + 1, C, C)
+    gz = _d(gz)
+    A1b = np.empty_like(A1)
+    pwb = np.zeros_like(path_w)
+    mxb = np.zeros_like(mix_w)
+    m = _mask(node_mask, N)
+    rc = lib().orc_ladder_vjp(L, C, order, N, _pd(A1), _pd(path_w), _pd(mix_w),
+                              _pd(gz), _pu8(m), _pd(A1b), _pd(pwb), _pd(mxb))
+    assert rc == 0
+    return A1b, pwb, mxb
