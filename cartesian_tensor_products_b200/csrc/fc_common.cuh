@@ -1,0 +1,53 @@
+// Host-side helpers shared by the libflashcart translation units.
+#pragma once
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "flashcart.h"
+
+namespace fc {
+
+template <int L, int G, int g>
+struct FwdGroup;
+template <int L>
+struct FwdMeta;
+
+inline bool aligned16(const void* p) {
+  return (reinterpret_cast<uintptr_t>(p) & 15u) == 0;
+}
+inline bool aligned4(const void* p) {
+  return (reinterpret_cast<uintptr_t>(p) & 3u) == 0;
+}
+
+// number of paths / output row length for lmax_in = lmax_edge = lmax_out = L
+inline int num_paths(int L) {
+  int n = 0;
+  for (int l3 = 0; l3 <= L; ++l3)
+    for (int l1 = 0; l1 <= L; ++l1)
+      for (int l2 = 0; l2 <= L; ++l2)
+        if (l3 >= (l1 > l2 ? l1 - l2 : l2 - l1) && l3 <= l1 + l2 &&
+            ((l1 + l2 + l3) & 1) == 0)
+          ++n;
+  return n;
+}
+
+inline int out_row(int L, int sum_paths) {
+  if (sum_paths) return (L + 1) * (L + 1);
+  int n = 0;
+  for (int l3 = 0; l3 <= L; ++l3)
+    for (int l1 = 0; l1 <= L; ++l1)
+      for (int l2 = 0; l2 <= L; ++l2)
+        if (l3 >= (l1 > l2 ? l1 - l2 : l2 - l1) && l3 <= l1 + l2 &&
+            ((l1 + l2 + l3) & 1) == 0)
+          n += 2 * l3 + 1;
+  return n;
+}
+
+// SM count and occupancy are cached per device
+int device_sm_count();
+
+// validates the parts of a convolution descriptor this build supports
+int check_conv_desc(const fc_conv_desc* d);
+
+}  // namespace fc

@@ -1,0 +1,166 @@
+"""Thin ctypes binding of libflashcart (C ABI in include/flashcart.h).
+
+Argument marshalling only: tensors are checked for device, dtype and shape,
+their device pointers and the current CUDA stream are handed to the C entry
+points, and a non-zero status becomes a FlashCartError.  Every step of the
+computation runs in the library's CUDA kernels; there is no fallback.  If the
+library has not been built this module raises on import.
+
+Conventions (layouts, path order, component order) are those of the header.
+"""
+import ctypes as ct
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libflashcart.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        "libflashcart.so is not built (expected at %s); run "
+        "`python -m cartesian_tensor_products_b200.build`" % LIB_PATH)
+
+_lib = ct.CDLL(LIB_PATH)
+
+FC_OK = 0
+
+
+class FlashCartError(RuntimeError):
+    def __init__(self, status, where):
+        self.status = status
+        super().__init__("%s: %s (status %d)" % (
+            where, _lib.fc_status_string(status).decode(), status))
+
+
+class ConvDesc(ct.Structure):
+    _fields_ = [("lmax_in", ct.c_int), ("lmax_edge", ct.c_int),
+                ("lmax_out", ct.c_int), ("channels", ct.c_int),
+                ("sum_paths", ct.c_int)]
+
+
+class LadderDesc(ct.Structure):
+    _fields_ = [("lmax", ct.c_int), ("channels", ct.c_int), ("order", ct.c_int)]
+
+
+_vp = ct.c_void_p
+_SIGS = {
+    "fc_status_string": (ct.c_char_p, [ct.c_int]),
+    "fc_version": (ct.c_int, []),
+    "fc_conv_num_paths": (ct.c_int, [ct.POINTER(ConvDesc)]),
+    "fc_conv_out_row": (ct.c_int, [ct.POINTER(ConvDesc)]),
+    "fc_conv_path": (ct.c_int, [ct.POINTER(ConvDesc), ct.c_int, ct.POINTER(ct.c_int),
+                                ct.POINTER(ct.c_int), ct.POINTER(ct.c_int)]),
+    "fc_build_rowptr": (ct.c_int, [ct.c_int, ct.c_int, _vp, _vp, _vp, _vp, _vp]),
+    "fc_edge_conv": (ct.c_int, [ct.POINTER(ConvDesc), ct.c_int, ct.c_int,
+                                _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
+}
+for _name, (_res, _args) in _SIGS.items():
+    _f = getattr(_lib, _name)
+    _f.restype = _res
+    _f.argtypes = _args
+
+
+def lib():
+    return _lib
+
+
+def _check(status, where):
+    if status != FC_OK:
+        raise FlashCartError(status, where)
+
+
+def _stream(stream=None):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return _vp(stream.cuda_stream)
+
+
+def _ptr(t):
+    return _vp(t.data_ptr()) if t is not None else None
+
+
+def _dev(t, dtype, name):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError("%s must be a CUDA tensor" % name)
+    if t.dtype != dtype:
+        raise TypeError("%s must be %s, got %s" % (name, dtype, t.dtype))
+    if not t.is_contiguous():
+        raise ValueError("%s must be contiguous" % name)
+    return t
+
+
+def conv_desc(lmax, channels, sum_paths=False):
+    return ConvDesc(lmax, lmax, lmax, channels, int(bool(sum_paths)))
+
+
+def num_paths(lmax, channels=4, sum_paths=False):
+    d = conv_desc(lmax, channels, sum_paths)
+    n = _lib.fc_conv_num_paths(ct.byref(d))
+    if n < 0:
+        raise FlashCartError(4, "fc_conv_num_paths")
+    return n
+
+
+def out_row(lmax, channels=4, sum_paths=False):
+    d = conv_desc(lmax, channels, sum_paths)
+    n = _lib.fc_conv_out_row(ct.byref(d))
+    if n < 0:
+        raise FlashCartError(4, "fc_conv_out_row")
+    return n
+
+
+def paths(lmax):
+    d = conv_desc(lmax, 4)
+    out = []
+    for p in range(num_paths(lmax)):
+        a, b, c = ct.c_int(), ct.c_int(), ct.c_int()
+        _check(_lib.fc_conv_path(ct.byref(d), p, ct.byref(a), ct.byref(b), ct.byref(c)),
+               "fc_conv_path")
+        out.append((a.value, b.value, c.value))
+    return out
+
+
+def build_rowptr(edge_index, edge_vec, n_nodes, stream=None):
+    """Receiver row pointer [n_nodes+1] of a receiver-sorted edge list; raises
+    FlashCartError(FC_ERR_CSR / FC_ERR_DEGENERATE_EDGE) on a bad graph."""
+    _dev(edge_index, torch.int32, "edge_index")
+    E = edge_index.shape[1]
+    if edge_vec is not None:
+        _dev(edge_vec, torch.float32, "edge_vec")
+        assert edge_vec.shape == (E, 3)
+    dev = edge_index.device
+    rowptr = torch.empty(n_nodes + 1, dtype=torch.int32, device=dev)
+    flag = torch.empty(1, dtype=torch.int32, device=dev)
+    _check(_lib.fc_build_rowptr(n_nodes, E, _ptr(edge_index), _ptr(edge_vec),
+                                _ptr(rowptr), _ptr(flag), _stream(stream)),
+           "fc_build_rowptr")
+    return rowptr
+
+
+def edge_conv(lmax, rowptr, edge_index, edge_vec, x, w, sum_paths=False,
+              out=None, stream=None):
+    """z of Sec. 4 Eq. (1): [N][out_row * C]."""
+    _dev(rowptr, torch.int32, "rowptr")
+    _dev(edge_index, torch.int32, "edge_index")
+    _dev(edge_vec, torch.float32, "edge_vec")
+    _dev(x, torch.float32, "x")
+    _dev(w, torch.float32, "w")
+    N = rowptr.shape[0] - 1
+    E = edge_index.shape[1]
+    C = x.shape[1] // ((lmax + 1) ** 2)
+    d = conv_desc(lmax, C, sum_paths)
+    zr = out_row(lmax, C, sum_paths)
+    if x.shape != (N, (lmax + 1) ** 2 * C):
+        raise ValueError("x shape %s" % (tuple(x.shape),))
+    if w.numel() != E * num_paths(lmax) * C:
+        raise ValueError("w shape %s" % (tuple(w.shape),))
+    if out is None:
+        out = torch.empty((N, zr * C), dtype=torch.float32, device=x.device)
+    else:
+        _dev(out, torch.float32, "out")
+        assert out.shape == (N, zr * C)
+    _check(_lib.fc_edge_conv(ct.byref(d), N, E, _ptr(rowptr), _ptr(edge_index),
+                             _ptr(edge_vec), _ptr(x), _ptr(w), _ptr(out),
+                             _stream(stream)), "fc_edge_conv")
+    return out

@@ -1,0 +1,140 @@
+/*
+ * flashcart.h -- C ABI of libflashcart: irreducible-Cartesian tensor
+ * products for equivariant interatomic potentials on NVIDIA B200 (sm_100a).
+ *
+ * The operations are those of "FlashCart: Fast Cartesian Tensor Products
+ * for Equivariant Interatomic Potentials" (arXiv 2610.06409):
+ *   - fc_edge_conv          receiver-sorted edge convolution, Sec. 4 Eq. (1)
+ *                           and Algorithm 1 (App. D "Receiver-sorted forward")
+ *   - fc_edge_conv_vjp      its vector-Jacobian product, App. C Eq. (C1)
+ *                           summed as in Algorithm 2, extended through the
+ *                           direction tensors to the edge vectors (App. C,
+ *                           last paragraph of "Symbolic derivatives")
+ *   - fc_product_ladder     node-local correlation ladder, Sec. 5 Eq. (2)
+ *                           with path-reduced products (App. E)
+ *   - fc_product_ladder_vjp its vector-Jacobian product
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * Tensors.  A rank-l feature is a symmetric trace-free (STF) Cartesian
+ * tensor stored by its 2l+1 independent components (Sec. 3): those with at
+ * most one z index, ordered p_z = 0 with p_x descending, then p_z = 1 with
+ * p_x descending (l=1: x,y,z; l=2: xx,xy,yy,xz,yz; l=3: xxx,xxy,xyy,yyy,
+ * xxz,xyz,yyz).
+ * Paths.  Admissible (l1, l2) -> l3 with |l1-l2| <= l3 <= l1+l2 and
+ * l1+l2+l3 even (Sec. 2), ordered by l3, then l1, then l2; eta is the
+ * position of a path among those with the same l3.  Path normalisation
+ * C_{l1 l2 l3} of Eq. (B1) is chosen so that T_l1(r) (x) T_l2(r) -> T_l3(r).
+ * Layout (App. D "Data layout").  Row per node or edge, rank blocks in
+ * increasing l; inside block l the component c, then the path eta, then the
+ * channel k is fastest: offset off(l) + (c P_l + eta) C + k with
+ * off(l) = sum_{l'<l} (2l'+1) P_l' C.  Node features have P_l = 1, so x is
+ * [N][(L+1)^2 C].  Weights are [E][P][C] (channel fastest).
+ * Edges.  edge_index is int32 [2][E]: row 0 receivers u_e, row 1 senders
+ * v_e, sorted by receiver (non-decreasing).  edge_vec is float [E][3] and
+ * points from the receiver to the sender, r_e = pos[v_e] - pos[u_e] (+ any
+ * periodic shift) (Sec. 2).  rowptr [N+1]: incoming edges of u are
+ * [rowptr[u], rowptr[u+1]) (Sec. 4, App. D).
+ * Memory.  Every pointer argument of a compute call is DEVICE memory owned
+ * by the caller, 16-byte aligned, and stays valid until the stream has
+ * executed the call.  The library allocates no device memory; scratch comes
+ * from a caller-provided workspace whose size a *_workspace_size call gives.
+ * Streams.  Compute calls are asynchronous on `stream` (NULL = the legacy
+ * default stream).  Host-side argument checks happen before anything is
+ * enqueued; a failing call enqueues nothing and returns an error status.
+ * Outputs are overwritten, never accumulated into.
+ * Precision.  FP32 inputs and outputs, FP32 arithmetic with fused
+ * multiply-adds.  Results that combine per-sender or per-edge gradient
+ * contributions are not bitwise reproducible run to run.
+ */
+#ifndef FLASHCART_H
+#define FLASHCART_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t. */
+typedef struct CUstream_st *fc_stream_t;
+
+typedef enum {
+  FC_OK = 0,
+  FC_ERR_ARG = 1,              /* NULL pointer, negative size, bad descriptor */
+  FC_ERR_CSR = 2,              /* receivers unsorted or out of range, senders out of range */
+  FC_ERR_DEGENERATE_EDGE = 3,  /* an edge vector of zero (or non-finite) length */
+  FC_ERR_UNSUPPORTED_RANK = 4, /* a rank combination this build has no kernel for */
+  FC_ERR_ALIGN = 5,            /* pointer not 16-byte aligned or channels not a multiple of 4 */
+  FC_ERR_CUDA = 6,             /* a CUDA runtime call failed (launch, copy) */
+  FC_ERR_WORKSPACE = 7         /* workspace NULL or smaller than required */
+} fc_status;
+
+/* Human-readable text of a status code; never NULL. */
+const char *fc_status_string(int status);
+
+/* Library version as 10000*major + 100*minor + patch. */
+int fc_version(void);
+
+/* Edge-convolution descriptor.  This build supports
+ * lmax_in == lmax_edge == lmax_out in {2, 3, 4}, channels >= 4 and a
+ * multiple of 4.  sum_paths = 0 keeps the P_l paths of each output rank
+ * separate (z row = sum_l (2l+1) P_l C); sum_paths = 1 sums them (z row =
+ * (lmax_out+1)^2 C, the node-feature layout). */
+typedef struct {
+  int lmax_in;    /* rank of node features x (l1)           */
+  int lmax_edge;  /* rank of direction tensors T_l2(r-hat) */
+  int lmax_out;   /* rank of outputs (l3)                   */
+  int channels;   /* C                                      */
+  int sum_paths;  /* 0 or 1                                 */
+} fc_conv_desc;
+
+/* Number of paths P of the descriptor, or -1 if it is not supported. */
+int fc_conv_num_paths(const fc_conv_desc *desc);
+
+/* Output components per channel of one z row (z row = this x C), or -1. */
+int fc_conv_out_row(const fc_conv_desc *desc);
+
+/* Path p of the descriptor: writes l1, l2, l3.  Returns FC_OK or FC_ERR_ARG. */
+int fc_conv_path(const fc_conv_desc *desc, int p, int *l1, int *l2, int *l3);
+
+/* Build the receiver row pointer of a receiver-sorted edge list and
+ * validate the graph (App. D "Receiver-sorted forward").
+ *   edge_index [2][n_edges] int32 (device), edge_vec [n_edges][3] float
+ *   (device, may be NULL to skip the length check), rowptr [n_nodes+1]
+ *   int32 (device, written), flag: one int32 of device scratch.
+ * Rejects receivers out of [0, n_nodes) or not sorted (FC_ERR_CSR),
+ * senders out of range (FC_ERR_CSR), and edge vectors of zero or
+ * non-finite length (FC_ERR_DEGENERATE_EDGE).  Synchronises `stream` to
+ * read the verdict; rowptr is only meaningful when FC_OK is returned.
+ * n_edges = 0 is valid (rowptr all zero). */
+int fc_build_rowptr(int n_nodes, int n_edges, const int32_t *edge_index,
+                    const float *edge_vec, int32_t *rowptr, int32_t *flag,
+                    fc_stream_t stream);
+
+/* Receiver-sorted edge convolution, Sec. 4 Eq. (1):
+ *   z[u, eta, k] = sum_{e: u_e = u} w[e, eta, k] f_eta(x[v_e, :, k], T(r-hat_e))
+ * with f_eta the Cartesian product of path eta (App. B Eq. (B1)) and
+ * T(r-hat) = (T_0, ..., T_lmax_edge) the direction tensors of App. B.
+ * Each receiver's sum is accumulated on chip and stored once (Algorithm 1:
+ * no atomics, no per-edge message tensor), except with sum_paths = 1, where
+ * path partial sums from different warps are added atomically into z after
+ * the call zeroes it.
+ *   rowptr [n_nodes+1] from fc_build_rowptr; edge_index, edge_vec as above;
+ *   x [n_nodes][(lmax_in+1)^2 C]; w [n_edges][P][C];
+ *   z [n_nodes][fc_conv_out_row() C] (written; receivers without edges get 0).
+ * The graph must have passed fc_build_rowptr: the kernel does not fault on
+ * a bad graph (rowptr is clamped to [0, n_edges], out-of-range senders
+ * contribute nothing) but its output is then meaningless.
+ * Returns FC_OK, FC_ERR_ARG, FC_ERR_UNSUPPORTED_RANK, FC_ERR_ALIGN or
+ * FC_ERR_CUDA. */
+int fc_edge_conv(const fc_conv_desc *desc, int n_nodes, int n_edges,
+                 const int32_t *rowptr, const int32_t *edge_index,
+                 const float *edge_vec, const float *x, const float *w,
+                 float *z, fc_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* FLASHCART_H */
