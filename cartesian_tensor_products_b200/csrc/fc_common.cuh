@@ -12,6 +12,12 @@ template <int L, int G, int g>
 struct FwdGroup;
 template <int L>
 struct FwdMeta;
+template <int L>
+struct Direction;
+template <int L, int G, int g>
+struct VjpGroup;
+template <int L>
+struct VjpMeta;
 
 inline bool aligned16(const void* p) {
   return (reinterpret_cast<uintptr_t>(p) & 15u) == 0;

@@ -5,17 +5,21 @@
 //   y_e = T(r-hat_e) shared by all channels.
 // Every receiver's sums are accumulated on chip and stored once.
 //
-// B200 design.  A CTA holds G warps; warp g owns a fixed group of output
-// rows (path, component), chosen offline so that every warp does the same
-// number of FMAs, and covers 128 channels of one receiver (4 per lane, so
-// every global access is a coalesced 16-byte vector).  The CTA walks a
-// strided list of (receiver, 128-channel tile) units.  For each chunk of up
-// to 32 incoming edges a warp first forms, lane-per-edge, the entries of
-// M_eta[a][b] = sum_b2 K_eta[a][b][b2] y_e,b2 its rows need and parks them
-// in a warp-private shared-memory row; then it walks the edges, loading the
-// sender's feature rows (L2-resident) and the edge's path weights
-// (streamed from HBM, one edge ahead in registers) and accumulating
-// w * (M x) with every M entry read as a shared-memory broadcast.
+// B200 design.  One CTA per (receiver, 128-channel tile); its G warps each
+// own a fixed group of output rows (path, component), cut offline so that
+// the warps do near-equal work.  A lane owns 4 consecutive channels, so
+// every global access is a coalesced 16-byte vector.  Per incoming edge a
+// warp needs the sender's x rows its rows touch and the edge's weight rows
+// of its paths: each lane streams its own 16-byte slices of those rows into
+// a 3-deep shared-memory ring with cp.async, three edges ahead of use, and
+// reads back only what it copied (no barrier on the data path).  Every 16
+// edges the warp forms, lane-per-edge, the entries
+// M[a][b] = sum_b2 K[a][b][b2] y_b2 (y = T(r-hat)) of its rows into a
+// warp-private shared-memory window; the per-edge loop then reads them as
+// broadcasts and applies them to the lane's 4 channels with packed FP32x2
+// FMAs.  Sender indices and edge vectors come from a 32-edge register
+// window (one per lane) read with warp shuffles.  With 4 groups every SMSP
+// runs one instruction stream (warp g of each resident CTA).
 #include "fc_common.cuh"
 #include "fc_device.cuh"
 #include "generated/fc_fwd_L2.cuh"
@@ -34,116 +38,152 @@ struct ConvArgs {
   int n_nodes, n_edges, C, ntiles, xrow, zrow, P, sum_paths;
 };
 
-template <class Grp>
-__device__ __forceinline__ void load_edge(const ConvArgs& a, int v, int e, int k0, bool act,
-                                          float4 (&xr)[Grp::NX], float4 (&wr)[Grp::NWP]) {
-  if (act && v >= 0) {
-    Grp::load_x(a.x + (size_t)v * a.xrow * a.C + k0, a.C, xr);
-    Grp::load_w(a.w + (size_t)e * a.P * a.C + k0, a.C, wr);
+// sender and edge vector of edge `e` for this lane's window slot
+struct EdgeWin {
+  int v;
+  float rx, ry, rz;
+};
+
+__device__ __forceinline__ EdgeWin load_win(const ConvArgs& a, int e, int e1) {
+  EdgeWin wv;
+  if (e < e1) {
+    wv.v = __ldg(a.send + e);
+    wv.rx = __ldg(a.vec + 3 * e);
+    wv.ry = __ldg(a.vec + 3 * e + 1);
+    wv.rz = __ldg(a.vec + 3 * e + 2);
   } else {
-#pragma unroll
-    for (int i = 0; i < Grp::NX; ++i) xr[i] = zero4();
-#pragma unroll
-    for (int i = 0; i < Grp::NWP; ++i) wr[i] = zero4();
+    wv.v = -1;
+    wv.rx = 1.0f;
+    wv.ry = 0.0f;
+    wv.rz = 0.0f;
   }
+  return wv;
 }
 
 template <class Grp>
-__device__ __forceinline__ void fwd_warp(const ConvArgs& a, float* __restrict__ mbuf,
-                                         int* __restrict__ sbuf, int lane) {
-  const int n_units = a.n_nodes * a.ntiles;
-  for (int unit = blockIdx.x; unit < n_units; unit += gridDim.x) {
-    const int u = unit / a.ntiles;
-    const int tile = unit - u * a.ntiles;
-    const int k0 = tile * 128 + lane * 4;
-    const bool act = k0 < a.C;
-    int e0 = a.rowptr[u], e1 = a.rowptr[u + 1];
-    e0 = e0 < 0 ? 0 : (e0 > a.n_edges ? a.n_edges : e0);
-    e1 = e1 < e0 ? e0 : (e1 > a.n_edges ? a.n_edges : e1);
-    float4 acc[Grp::NA];
-#pragma unroll
-    for (int i = 0; i < Grp::NA; ++i) acc[i] = zero4();
+__device__ __forceinline__ void issue_edge(const ConvArgs& a, int C, float* st, int q, int v,
+                                           int k0, bool act) {
+  const bool vok = act && v >= 0 && v < a.n_nodes;
+  const int kk = act ? k0 : 0;
+  const float* xv = a.x + (size_t)(vok ? v : 0) * a.xrow * C + kk;
+  const float* we = a.w + (size_t)q * a.P * C + kk;
+  Grp::issue(st, xv, we, C, vok, act);
+}
 
-    for (int cs = e0; cs < e1; cs += 32) {
-      const int n = (e1 - cs) < 32 ? (e1 - cs) : 32;
-      if (lane < n) {
-        const int e = cs + lane;
-        const float rx = a.vec[3 * e], ry = a.vec[3 * e + 1], rz = a.vec[3 * e + 2];
-        const float inv = 1.0f / sqrtf(rx * rx + ry * ry + rz * rz);
-        Grp::make_m(rx * inv, ry * inv, rz * inv, mbuf + lane * Grp::MSTRIDE);
-        const int v = a.send[e];
-        sbuf[lane] = (v >= 0 && v < a.n_nodes) ? v : -1;
-      }
+// CC > 0: the channel count is the compile-time constant CC (every row
+// offset becomes an immediate); CC == 0: runtime a.C.
+template <class Grp, int S, int MW, int CC>
+__device__ __forceinline__ void fwd_warp(const ConvArgs& a, float* smem, int lane) {
+  constexpr int STAGE = Grp::NROW * 128;  // floats per stage (all lanes)
+  const int C = CC > 0 ? CC : a.C;
+  const int unit = blockIdx.x;
+  const int u = CC == 128 ? unit : unit / a.ntiles;
+  const int tile = unit - u * (CC == 128 ? 1 : a.ntiles);
+  const int k0 = tile * 128 + lane * 4;
+  const bool act = k0 < C;
+  int e0 = __ldg(a.rowptr + u), e1 = __ldg(a.rowptr + u + 1);
+  e0 = e0 < 0 ? 0 : (e0 > a.n_edges ? a.n_edges : e0);
+  e1 = e1 < e0 ? e0 : (e1 > a.n_edges ? a.n_edges : e1);
+  float* st = smem + Grp::RING_OFF + lane * 4;
+  float* mwin = smem + Grp::MWIN_OFF;
+
+  float4 acc[Grp::NA];
+#pragma unroll
+  for (int i = 0; i < Grp::NA; ++i) acc[i] = zero4();
+
+  EdgeWin cur = load_win(a, e0 + lane, e1);
+  EdgeWin nxt = load_win(a, e0 + 32 + lane, e1);
+
+  // prefill S edges
+#pragma unroll
+  for (int s = 0; s < S; ++s) {
+    const int q = e0 + s;
+    const int v = __shfl_sync(0xffffffffu, cur.v, s);
+    if (q < e1) issue_edge<Grp>(a, C, st + s * STAGE, q, v, k0, act);
+    cp_async_commit();
+  }
+
+  for (int q = e0; q < e1; ++q) {
+    const int p = q - e0;
+    if (p > 0 && (p & 31) == 0) {
+      cur = nxt;
+      nxt = load_win(a, q + 32 + lane, e1);
+    }
+    if ((p % MW) == 0) {
+      // M entries of the next MW edges, lane-per-edge, into the warp's window
+      const int src = (p & 31) + (lane % MW);
+      const float rx = __shfl_sync(0xffffffffu, cur.rx, src);
+      const float ry = __shfl_sync(0xffffffffu, cur.ry, src);
+      const float rz = __shfl_sync(0xffffffffu, cur.rz, src);
       __syncwarp();
-      // ping-pong between two register buffers, one edge of look-ahead
-      float4 xa[Grp::NX], wa[Grp::NWP], xb[Grp::NX], wb[Grp::NWP];
-      load_edge<Grp>(a, sbuf[0], cs, k0, act, xa, wa);
-      for (int j = 0; j < n; j += 2) {
-        if (j + 1 < n) load_edge<Grp>(a, sbuf[j + 1], cs + j + 1, k0, act, xb, wb);
-        Grp::accum(acc, xa, wa, mbuf + j * Grp::MSTRIDE);
-        if (j + 1 >= n) break;
-        if (j + 2 < n) load_edge<Grp>(a, sbuf[j + 2], cs + j + 2, k0, act, xa, wa);
-        Grp::accum(acc, xb, wb, mbuf + (j + 1) * Grp::MSTRIDE);
+      if (lane < MW && q + lane < e1) {
+        const float inv = 1.0f / sqrtf(rx * rx + ry * ry + rz * rz);
+        Grp::make_m(rx * inv, ry * inv, rz * inv, mwin + lane * Grp::MSTRIDE);
       }
       __syncwarp();
     }
-    if (act) Grp::store(a.z + (size_t)u * a.zrow * a.C + k0, a.C, a.sum_paths, acc);
+    const int slot = p % S;
+    cp_async_wait<S - 1>();
+    Grp::accum(acc, st + slot * STAGE, mwin + (p % MW) * Grp::MSTRIDE);
+    // refill this slot with edge q + S
+    const int pn = p + S;
+    if (q + S < e1) {
+      int v;
+      if ((pn >> 5) == (p >> 5))
+        v = __shfl_sync(0xffffffffu, cur.v, pn & 31);
+      else
+        v = __shfl_sync(0xffffffffu, nxt.v, pn & 31);
+      issue_edge<Grp>(a, C, st + slot * STAGE, q + S, v, k0, act);
+    }
+    cp_async_commit();
   }
+  cp_async_wait<0>();
+  if (act) Grp::store(a.z + (size_t)u * a.zrow * C + k0, C, a.sum_paths, acc);
 }
 
-template <int L, int g>
-__device__ __forceinline__ void dispatch_fwd(int warp, const ConvArgs& a, float* mbuf,
-                                             int* sbuf, int lane) {
+template <int L, int CC, int g>
+__device__ __forceinline__ void dispatch_fwd(int warp, const ConvArgs& a, float* smem,
+                                             int lane) {
   if constexpr (g < FwdMeta<L>::G) {
+    using Grp = FwdGroup<L, FwdMeta<L>::G, g>;
     if (warp == g) {
-      fwd_warp<FwdGroup<L, FwdMeta<L>::G, g>>(a, mbuf, sbuf, lane);
+      fwd_warp<Grp, FwdMeta<L>::S, FwdMeta<L>::MWIN, CC>(a, smem, lane);
       return;
     }
-    dispatch_fwd<L, g + 1>(warp, a, mbuf, sbuf, lane);
+    dispatch_fwd<L, CC, g + 1>(warp, a, smem, lane);
   }
 }
 
-template <int L>
-__global__ void __launch_bounds__(FwdMeta<L>::G * 32, 1)
+template <int L, int CC>
+__global__ void __launch_bounds__(FwdMeta<L>::G * 32, (FwdMeta<L>::G <= 4 ? 2 : 1))
     edge_conv_fwd_kernel(const ConvArgs a) {
   extern __shared__ __align__(16) float smem[];
-  constexpr int MS = FwdMeta<L>::MAXSTRIDE;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  float* mbuf = smem + warp * 32 * MS;
-  int* sbuf = reinterpret_cast<int*>(smem + FwdMeta<L>::G * 32 * MS) + warp * 32;
-  dispatch_fwd<L, 0>(warp, a, mbuf, sbuf, lane);
+  dispatch_fwd<L, CC, 0>(warp, a, smem, lane);
 }
 
-template <int L>
-static size_t fwd_smem_bytes() {
-  return sizeof(float) * (size_t)FwdMeta<L>::G * 32 * FwdMeta<L>::MAXSTRIDE +
-         sizeof(int) * (size_t)FwdMeta<L>::G * 32;
+template <int L, int CC>
+static int launch_fwd_cc(const ConvArgs& a, cudaStream_t s) {
+  static_assert(sizeof(float) * FwdMeta<L>::SMEM_FLOATS <= 227 * 1024,
+                "forward kernel shared memory exceeds the 227 KB per-CTA limit of sm_100");
+  const size_t smem = sizeof(float) * (size_t)FwdMeta<L>::SMEM_FLOATS;
+  static int configured[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return FC_ERR_CUDA;
+  if (!configured[dev]) {
+    if (cudaFuncSetAttribute(edge_conv_fwd_kernel<L, CC>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+      return FC_ERR_CUDA;
+    configured[dev] = 1;
+  }
+  const long long units = (long long)a.n_nodes * a.ntiles;
+  edge_conv_fwd_kernel<L, CC><<<(unsigned)units, FwdMeta<L>::G * 32, smem, s>>>(a);
+  return cudaGetLastError() == cudaSuccess ? FC_OK : FC_ERR_CUDA;
 }
 
 template <int L>
 static int launch_fwd(const ConvArgs& a, cudaStream_t s) {
-  const size_t smem = fwd_smem_bytes<L>();
-  static int configured[64] = {0};
-  static int blocks_per_sm[64] = {0};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return FC_ERR_CUDA;
-  if (!configured[dev]) {
-    if (cudaFuncSetAttribute(edge_conv_fwd_kernel<L>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
-      return FC_ERR_CUDA;
-    int nb = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, edge_conv_fwd_kernel<L>,
-                                                      FwdMeta<L>::G * 32, smem) != cudaSuccess)
-      return FC_ERR_CUDA;
-    blocks_per_sm[dev] = nb > 0 ? nb : 1;
-    configured[dev] = 1;
-  }
-  const long long units = (long long)a.n_nodes * a.ntiles;
-  long long grid = (long long)device_sm_count() * blocks_per_sm[dev];
-  if (grid > units) grid = units;
-  if (grid < 1) grid = 1;
-  edge_conv_fwd_kernel<L><<<(int)grid, FwdMeta<L>::G * 32, smem, s>>>(a);
-  return cudaGetLastError() == cudaSuccess ? FC_OK : FC_ERR_CUDA;
+  return a.C == 128 ? launch_fwd_cc<L, 128>(a, s) : launch_fwd_cc<L, 0>(a, s);
 }
 
 }  // namespace fc

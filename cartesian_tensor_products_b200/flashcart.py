@@ -54,6 +54,8 @@ _SIGS = {
     "fc_build_rowptr": (ct.c_int, [ct.c_int, ct.c_int, _vp, _vp, _vp, _vp, _vp]),
     "fc_edge_conv": (ct.c_int, [ct.POINTER(ConvDesc), ct.c_int, ct.c_int,
                                 _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
+    "fc_edge_conv_vjp": (ct.c_int, [ct.POINTER(ConvDesc), ct.c_int, ct.c_int,
+                                    _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _f = getattr(_lib, _name)
@@ -164,3 +166,36 @@ def edge_conv(lmax, rowptr, edge_index, edge_vec, x, w, sum_paths=False,
                              _ptr(edge_vec), _ptr(x), _ptr(w), _ptr(out),
                              _stream(stream)), "fc_edge_conv")
     return out
+
+
+def edge_conv_vjp(lmax, rowptr, edge_index, edge_vec, x, w, g, sum_paths=False,
+                  want=("x", "w", "r"), out=None, stream=None):
+    """(x_bar, w_bar, r_bar) of App. C Eq. (C1); entries not in `want` are None."""
+    _dev(rowptr, torch.int32, "rowptr")
+    _dev(edge_index, torch.int32, "edge_index")
+    _dev(edge_vec, torch.float32, "edge_vec")
+    _dev(x, torch.float32, "x")
+    _dev(w, torch.float32, "w")
+    _dev(g, torch.float32, "g")
+    N = rowptr.shape[0] - 1
+    E = edge_index.shape[1]
+    C = x.shape[1] // ((lmax + 1) ** 2)
+    d = conv_desc(lmax, C, sum_paths)
+    P = num_paths(lmax)
+    if g.shape != (N, out_row(lmax, C, sum_paths) * C):
+        raise ValueError("g shape %s" % (tuple(g.shape),))
+    if out is None:
+        out = {}
+    xb = out.get("x") if "x" in want else None
+    wb = out.get("w") if "w" in want else None
+    rb = out.get("r") if "r" in want else None
+    if "x" in want and xb is None:
+        xb = torch.empty_like(x)
+    if "w" in want and wb is None:
+        wb = torch.empty((E, P, C), dtype=torch.float32, device=x.device)
+    if "r" in want and rb is None:
+        rb = torch.empty((E, 3), dtype=torch.float32, device=x.device)
+    _check(_lib.fc_edge_conv_vjp(ct.byref(d), N, E, _ptr(rowptr), _ptr(edge_index),
+                                 _ptr(edge_vec), _ptr(x), _ptr(w), _ptr(g), _ptr(xb),
+                                 _ptr(wb), _ptr(rb), _stream(stream)), "fc_edge_conv_vjp")
+    return xb, wb, rb

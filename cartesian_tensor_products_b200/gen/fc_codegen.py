@@ -94,12 +94,13 @@ class Tables:
 # partition of output rows into warp groups (forward kernel)
 # ---------------------------------------------------------------------------
 
-def partition_rows(T, G):
+def partition_rows(T, G, row_weight=0.0):
     """Rows (p, a) in order of l1 (descending), then path, then a; cut into
-    G contiguous groups of near-equal cost."""
+    G contiguous groups of near-equal cost (per-lane FMAs of the row plus
+    row_weight per accumulator)."""
     order = sorted(range(T.P), key=lambda p: (-T.paths[p][0], p))
     rows = [(p, a) for p in order for a in range(2 * T.paths[p][2] + 1)]
-    cost = [T.row_cost(p, a) + 0.25 for (p, a) in rows]
+    cost = [T.row_cost(p, a) + 0.25 + row_weight for (p, a) in rows]
     remaining = sum(cost)
     groups, cur, acc = [], [], 0.0
     target = remaining / G
@@ -148,8 +149,20 @@ def lincomb_expr(terms, var):
     return " + ".join(out).replace("+ -", "- ")
 
 
+def ycomp(l, c):
+    """index of component c of rank l in the stacked direction tensor"""
+    return l * l + c
+
+
 class GroupCode:
-    """Straight-line code of one warp group of the forward kernel."""
+    """Straight-line code of one warp group of the forward kernel.
+
+    A lane owns 4 channels (one float4).  Per edge the group needs the x
+    rows its M entries touch and the weight rows of its paths; both are
+    staged in a per-warp shared-memory ring, each lane copying and reading
+    only its own 16-byte slice.  M entries are formed in registers from the
+    direction tensor y of the edge (same value in every lane) and used for
+    the 4 channels of the lane."""
 
     def __init__(self, T, rows, gid):
         self.T, self.rows, self.gid = T, rows, gid
@@ -158,7 +171,6 @@ class GroupCode:
             if p not in self.paths:
                 self.paths.append(p)
         self.prow = {p: [a for (q, a) in rows if q == p] for p in self.paths}
-        # x rows (component index within node row) needed
         xr = []
         for p in self.paths:
             l1 = T.paths[p][0]
@@ -171,21 +183,48 @@ class GroupCode:
                     if l1 * l1 + b not in xr:
                         xr.append(l1 * l1 + b)
         self.xrows = sorted(xr)
-        # M entries (non-identity rows)
-        self.ment = []                        # (p, a, b1, {b2: coef})
+        self.ment = []                        # (p, a, b1, {b2: coef}) in use order
+        self.form = {}                        # path -> True: input side (t_b = w x_b)
         for p in self.paths:
             if T.is_identity(p):
                 continue
-            for a in self.prow[p]:
-                for b1, terms in T.mrow(p, a):
-                    self.ment.append((p, a, b1, terms))
+            ents = [(a, b1, terms) for a in self.prow[p] for b1, terms in T.mrow(p, a)]
+            bset = sorted(set(b for _, b, _ in ents))
+            self.form[p] = len(bset) <= len(self.prow[p])
+            if self.form[p]:
+                # b-major: consecutive FMAs update different accumulators
+                ents.sort(key=lambda e: (e[1], e[0]))
+            else:
+                # term-major over the rows of the path
+                per_row = {a: [e for e in ents if e[0] == a] for a in self.prow[p]}
+                ents = []
+                depth = max(len(v) for v in per_row.values())
+                for j in range(depth):
+                    for a in self.prow[p]:
+                        if j < len(per_row[a]):
+                            ents.append(per_row[a][j])
+            for (a, b1, terms) in ents:
+                self.ment.append((p, a, b1, terms))
         self.NM = len(self.ment)
-        self.NMP = (self.NM + 3) // 4 * 4     # padded to float4
-        s = self.NMP // 4
-        if s % 2 == 0:
-            s += 1                            # odd float4 stride: conflict-free
-        self.MSTRIDE = max(4, 4 * s)
         self.NA = len(rows)
+        self.NROW = len(self.xrows) + len(self.paths)
+        # entries equal up to sign share one stored value
+        self.uniq, self.usign, ukey = [], [], {}
+        for (p, a, b1, terms) in self.ment:
+            l2 = T.paths[p][1]
+            t = tuple(sorted(terms.items()))
+            neg = tuple((b, -c) for b, c in t)
+            key = (l2, min(t, neg))
+            sign = 1 if key[1] == t else -1
+            if key not in ukey:
+                ukey[key] = len(self.uniq)
+                self.uniq.append((l2, dict(key[1])))
+            self.usign.append((ukey[key], sign))
+        self.NU = len(self.uniq)
+        q = max(1, (self.NU + 3) // 4)
+        if q % 2 == 0:
+            q += 1                            # odd float4 stride: conflict-free stores
+        self.MSTRIDE = 4 * q
 
     def y_needed(self):
         need = set()
@@ -195,17 +234,21 @@ class GroupCode:
                 need.add((l2, b2))
         return sorted(need)
 
-    def emit(self, L):
+    def emit(self, L, G):
         T = self.T
         g = self.gid
+        comp = "xyzw"
         o = []
-        o.append("template <> struct FwdGroup<%d, %d, %d> {" % (L, NGROUPS[L], g))
-        o.append("  static constexpr int NA = %d;   // output rows (float4 accumulators)" % self.NA)
-        o.append("  static constexpr int NX = %d;   // x rows loaded per edge" % len(self.xrows))
-        o.append("  static constexpr int NWP = %d;  // weight paths loaded per edge" % len(self.paths))
-        o.append("  static constexpr int NM = %d;   // M entries per edge" % self.NM)
-        o.append("  static constexpr int MSTRIDE = %d;  // floats per edge row in smem" % self.MSTRIDE)
-        # ---- make_m
+        o.append("template <> struct FwdGroup<%d, %d, %d> {" % (L, G, g))
+        o.append("  static constexpr int NA = %d;    // output rows (float4 accumulators)" % self.NA)
+        o.append("  static constexpr int NX = %d;    // x rows staged per edge" % len(self.xrows))
+        o.append("  static constexpr int NWP = %d;   // weight rows staged per edge" % len(self.paths))
+        o.append("  static constexpr int NROW = %d;  // staged 512-byte rows per edge" % self.NROW)
+        o.append("  static constexpr int NM = %d;    // M entries per edge (%d distinct up to sign)" % (self.NM, self.NU))
+        o.append("  static constexpr int MSTRIDE = %d;  // floats per edge row of the M window" % self.MSTRIDE)
+        o.append("  static constexpr int RING_OFF = %d;  // staging ring (floats into shared memory)" % self.ring_off)
+        o.append("  static constexpr int MWIN_OFF = %d;  // M window (floats into shared memory)" % self.mwin_off)
+        # ---- M entries of one edge (lane-per-edge), from the unit direction
         o.append("  static __device__ __forceinline__ void make_m(float ux, float uy, float uz, float* __restrict__ mrow) {")
         if self.NM:
             for (l2, b2) in self.y_needed():
@@ -214,8 +257,7 @@ class GroupCode:
                 else:
                     o.append("    const float y_%d_%d = %s;" % (l2, b2, poly_expr(T.ypoly[l2][b2])))
             vals = []
-            for (p, a, b1, terms) in self.ment:
-                l2 = T.paths[p][1]
+            for k, (l2, terms) in enumerate(self.uniq):
                 vals.append(lincomb_expr(terms, lambda b, l2=l2: "y_%d_%d" % (l2, b)))
             while len(vals) % 4:
                 vals.append("0.0f")
@@ -224,61 +266,59 @@ class GroupCode:
         else:
             o.append("    (void)ux; (void)uy; (void)uz; (void)mrow;")
         o.append("  }")
-        # ---- loads
-        o.append("  static __device__ __forceinline__ void load_x(const float* __restrict__ xv, int C, float4 (&xr)[NX]) {")
+        # ---- issue the copies of one edge
+        o.append("  static __device__ __forceinline__ void issue(float* st, const float* __restrict__ xv, const float* __restrict__ we, int C, bool xok, bool ok) {")
         for i, r in enumerate(self.xrows):
-            o.append("    xr[%d] = ld_x4(xv + %d * C);" % (i, r))
-        o.append("  }")
-        o.append("  static __device__ __forceinline__ void load_w(const float* __restrict__ we, int C, float4 (&wr)[NWP]) {")
+            o.append("    cp_async16(st + %d, xv + %d * C, xok);" % (128 * i, r))
         for i, p in enumerate(self.paths):
-            o.append("    wr[%d] = ld_w4(we + %d * C);" % (i, p))
+            o.append("    cp_async16(st + %d, we + %d * C, ok);" % (128 * (len(self.xrows) + i), p))
         o.append("  }")
-        # ---- accumulate
-        o.append("  static __device__ __forceinline__ void accum(float4 (&acc)[NA], const float4 (&xr)[NX], const float4 (&wr)[NWP], const float* __restrict__ m) {")
-        if self.NM:
-            for q in range(self.NMP // 4):
-                o.append("    const float4 mq%d = ld_s4(m + %d);" % (q, 4 * q))
+        # ---- accumulate one edge
+        o.append("  static __device__ __forceinline__ void accum(float4 (&acc)[NA], const float* st, const float* __restrict__ m) {")
+        for i, r in enumerate(self.xrows):
+            o.append("    const float4 x%d = ld_s4(st + %d);" % (r, 128 * i))
+        for i, p in enumerate(self.paths):
+            o.append("    const float4 w%d = ld_s4(st + %d);" % (i, 128 * (len(self.xrows) + i)))
+        acc_of = {r: i for i, r in enumerate(self.rows)}
+        loaded = set()
         mi = 0
-        ai = 0
-        acc_of = {}
-        for (p, a) in self.rows:
-            acc_of[(p, a)] = ai
-            ai += 1
-        xidx = {r: i for i, r in enumerate(self.xrows)}
-        comp = "xyzw"
         for pi, p in enumerate(self.paths):
             l1, l2, l3 = T.paths[p]
             o.append("    // path (%d,%d)->%d rows %s" % (l1, l2, l3, self.prow[p]))
             if T.is_identity(p):
                 for a in self.prow[p]:
-                    o.append("    acc[%d] = fma4(wr[%d], xr[%d], acc[%d]);" % (acc_of[(p, a)], pi, xidx[l1 * l1 + a], acc_of[(p, a)]))
+                    i = acc_of[(p, a)]
+                    o.append("    acc[%d] = fma4(w%d, x%d, acc[%d]);" % (i, pi, l1 * l1 + a, i))
                 continue
             rows_p = self.prow[p]
-            # entries of this path in M order
             ents = [(a, b1) for (pp, a, b1, _) in self.ment if pp == p]
-            base = mi
+            names = []
+            for k in range(len(ents)):
+                ui, sign = self.usign[mi + k]
+                q, c = divmod(ui, 4)
+                if q not in loaded:
+                    o.append("    const float4 mq%d = ld_s4(m + %d);" % (q, 4 * q))
+                    loaded.add(q)
+                names.append(("" if sign > 0 else "-") + "mq%d.%s" % (q, comp[c]))
             mi += len(ents)
-            bset = sorted(set(b for _, b in ents))
-            input_side = len(bset) <= len(rows_p)
-            if input_side:
+            if self.form[p]:
+                bset = sorted(set(b for _, b in ents))
                 for b in bset:
-                    o.append("    const float4 t%d_%d = mul4(wr[%d], xr[%d]);" % (pi, b, pi, xidx[l1 * l1 + b]))
+                    o.append("    const float4 t%d_%d = mul4(w%d, x%d);" % (pi, b, pi, l1 * l1 + b))
                 for k, (a, b) in enumerate(ents):
-                    q, c = divmod(base + k, 4)
-                    o.append("    acc[%d] = fma4s(mq%d.%s, t%d_%d, acc[%d]);" % (acc_of[(p, a)], q, comp[c], pi, b, acc_of[(p, a)]))
+                    i = acc_of[(p, a)]
+                    o.append("    acc[%d] = fma4s(%s, t%d_%d, acc[%d]);" % (i, names[k], pi, b, i))
             else:
+                started = set()
+                for k, (a, b) in enumerate(ents):
+                    if a not in started:
+                        o.append("    float4 s%d_%d = mul4s(%s, x%d);" % (pi, a, names[k], l1 * l1 + b))
+                        started.add(a)
+                    else:
+                        o.append("    s%d_%d = fma4s(%s, x%d, s%d_%d);" % (pi, a, names[k], l1 * l1 + b, pi, a))
                 for a in rows_p:
-                    first = True
-                    for k, (aa, b) in enumerate(ents):
-                        if aa != a:
-                            continue
-                        q, c = divmod(base + k, 4)
-                        if first:
-                            o.append("    float4 s%d_%d = mul4s(mq%d.%s, xr[%d]);" % (pi, a, q, comp[c], xidx[l1 * l1 + b]))
-                            first = False
-                        else:
-                            o.append("    s%d_%d = fma4s(mq%d.%s, xr[%d], s%d_%d);" % (pi, a, q, comp[c], xidx[l1 * l1 + b], pi, a))
-                    o.append("    acc[%d] = fma4(wr[%d], s%d_%d, acc[%d]);" % (acc_of[(p, a)], pi, pi, a, acc_of[(p, a)]))
+                    i = acc_of[(p, a)]
+                    o.append("    acc[%d] = fma4(w%d, s%d_%d, acc[%d]);" % (i, pi, pi, a, i))
         o.append("  }")
         # ---- store
         o.append("  static __device__ __forceinline__ void store(float* __restrict__ zu, int C, int sum_paths, const float4 (&acc)[NA]) {")
@@ -294,31 +334,58 @@ class GroupCode:
         return "\n".join(o)
 
 
-NGROUPS = {2: 4, 3: 8, 4: 16}
+def emit_direction(L):
+    """T_l(u) for l <= L, stacked: y[l*l + c]"""
+    o = ["template <> struct Direction<%d> {" % L,
+         "  static constexpr int NY = %d;" % ((L + 1) ** 2),
+         "  static __device__ __forceinline__ void eval(float ux, float uy, float uz, float (&y)[NY]) {"]
+    T = Tables(L)
+    for l in range(L + 1):
+        for c in range(2 * l + 1):
+            o.append("    y[%d] = %s;" % (ycomp(l, c), poly_expr(T.ypoly[l][c]) if l else "1.0f"))
+    o.append("  }")
+    o.append("};")
+    return "\n".join(o)
+
+
+NGROUPS = {2: 4, 3: 4, 4: 8}
+ROW_WEIGHT = {2: 0.0, 3: 0.0, 4: 4.0}
+STAGES = {2: 3, 3: 3, 4: 2}
+MWIN = 16
 
 
 def emit_fwd(L, G):
     T = Tables(L)
-    groups = partition_rows(T, G)
+    groups = partition_rows(T, G, ROW_WEIGHT[L])
     codes = [GroupCode(T, rows, g) for g, rows in enumerate(groups)]
     out = []
     out.append("// Generated by gen/fc_codegen.py -- do not edit.")
     out.append("// Receiver-sorted forward, rank %d: %d paths, %d output rows, %d warp groups." % (L, T.P, T.zrow, G))
     for c in codes:
         cost = sum(T.row_cost(p, a) for p, a in c.rows)
-        out.append("//   group %d: %d rows, %d M entries, %d x rows, %d w paths, cost %d" %
+        out.append("//   group %d: %d rows, %d M entries, %d x rows, %d w rows, %d FMA/channel" %
                    (c.gid, c.NA, c.NM, len(c.xrows), len(c.paths), cost))
     out.append("#pragma once")
     out.append('#include "../fc_device.cuh"')
     out.append("namespace fc {")
     out.append("template <> struct FwdMeta<%d> {" % L)
     out.append("  static constexpr int G = %d;           // warp groups = warps per CTA" % G)
-    out.append("  static constexpr int MAXSTRIDE = %d;   // largest per-edge M row (floats)" % max(c.MSTRIDE for c in codes))
+    out.append("  static constexpr int S = %d;           // staging ring depth (edges)" % STAGES[L])
+    out.append("  static constexpr int MAXROW = %d;      // largest staged rows per edge of a group" % max(c.NROW for c in codes))
     out.append("  static constexpr int P = %d;           // paths" % T.P)
     out.append("  static constexpr int ZROW = %d;        // output components per channel" % T.zrow)
+    off = 0
+    for c in codes:
+        c.ring_off = off
+        off += STAGES[L] * 128 * c.NROW
+    for c in codes:
+        c.mwin_off = off
+        off += MWIN * c.MSTRIDE
+    out.append("  static constexpr int MWIN = %d;        // edges per M window" % MWIN)
+    out.append("  static constexpr int SMEM_FLOATS = %d; // staging rings + M windows of all warps" % off)
     out.append("};")
     for c in codes:
-        out.append(c.emit(L))
+        out.append(c.emit(L, G))
     out.append("}  // namespace fc")
     return "\n".join(out) + "\n", T, codes
 
@@ -352,6 +419,259 @@ def main():
     with open(path, "w") as f:
         f.write(emit_tables((2, 3, 4)))
     written.append(path)
+    return written
+
+
+
+# ---------------------------------------------------------------------------
+# receiver-sorted VJP (App. C Eq. C1 summed as in Algorithm 2)
+# ---------------------------------------------------------------------------
+
+def direction_derivative_polys(l):
+    """d T_l(u)_c / d u_j as polynomials (j = x, y, z), for every component."""
+    out = []
+    for poly in A.direction_polys(l):
+        out.append([A.p_diff(poly, j) for j in range(3)])
+    return out
+
+
+def partition_paths(T, G, cost):
+    """Whole paths (h = M^T g needs all rows of a path) in order of l1
+    (descending), cut into G contiguous groups of near-equal cost."""
+    order = sorted(range(T.P), key=lambda p: (-T.paths[p][0], p))
+    c = [cost(p) for p in order]
+    remaining = sum(c)
+    groups, cur, acc = [], [], 0.0
+    target = remaining / G
+    for i, p in enumerate(order):
+        if cur and acc + c[i] / 2 > target and len(groups) < G - 1:
+            groups.append(cur)
+            remaining -= acc
+            target = remaining / (G - len(groups))
+            cur, acc = [], 0.0
+        cur.append(p)
+        acc += c[i]
+    groups.append(cur)
+    while len(groups) < G:
+        groups.append([])
+    return groups
+
+
+def vjp_path_cost(T, p):
+    l1, l2, l3 = T.paths[p]
+    nm = sum(len(T.mrow(p, a)) for a in range(2 * l3 + 1)) if not T.is_identity(p) else 2 * l1 + 1
+    nk = sum(1 for a in range(2 * l3 + 1) for b1 in range(2 * l1 + 1)
+             for b2 in range(2 * l2 + 1) if T.K[p][a][b1][b2] != 0)
+    return 2 * nm + 4 * (2 * l1 + 1) + 2 * (2 * l1 + 1) + 3 * nm + nk
+
+
+class VjpGroupCode:
+    """Straight-line code of one warp group of the VJP kernel (whole paths)."""
+
+    def __init__(self, T, paths, gid):
+        self.T, self.gpaths, self.gid = T, paths, gid
+        L = T.L
+        self.rows = [(p, a) for p in paths for a in range(2 * T.paths[p][2] + 1)]
+        self.NA = len(self.rows)
+        xr = []
+        for p in paths:
+            l1 = T.paths[p][0]
+            for b in range(2 * l1 + 1):
+                if l1 * l1 + b not in xr:
+                    xr.append(l1 * l1 + b)
+        self.xrows = sorted(xr)
+        # M entries (row-major per path) and the (a, b1) -> {b2: K} terms
+        self.ment = []
+        for p in paths:
+            l1, l2, l3 = T.paths[p]
+            for a in range(2 * l3 + 1):
+                for b1, terms in T.mrow(p, a):
+                    self.ment.append((p, a, b1, terms))
+        self.NM = len(self.ment)
+        ycomps = sorted(set((T.paths[p][1], b2) for p in paths
+                            for b2 in range(2 * T.paths[p][1] + 1) if T.paths[p][1] > 0))
+        self.ycomps = ycomps                 # direction components with a gradient
+        self.NYD = len(ycomps)
+        self.NROW = len(self.xrows) + len(paths)
+        self.dbase = (self.NM + 3) // 4 * 4  # offset of d y / d u in a window row
+        n = self.dbase + 3 * self.NYD
+        q = max(1, (n + 3) // 4)
+        if q % 2 == 0:
+            q += 1
+        self.MSTRIDE = 4 * q
+
+    def emit(self, L, G):
+        T = self.T
+        g = self.gid
+        o = []
+        o.append("template <> struct VjpGroup<%d, %d, %d> {" % (L, G, g))
+        o.append("  static constexpr int NA = %d;    // g rows held in registers (float4)" % self.NA)
+        o.append("  static constexpr int NX = %d;    // x rows staged per edge (= x_bar rows)" % len(self.xrows))
+        o.append("  static constexpr int NWP = %d;   // weight rows staged per edge" % len(self.gpaths))
+        o.append("  static constexpr int NROW = %d;  // staged 512-byte rows per edge" % self.NROW)
+        o.append("  static constexpr int NM = %d;    // M entries per edge" % self.NM)
+        o.append("  static constexpr int NYD = %d;   // direction components with a gradient" % self.NYD)
+        o.append("  static constexpr int MSTRIDE = %d;  // floats per edge row of the window" % self.MSTRIDE)
+        o.append("  static constexpr int RING_OFF = %d;" % self.ring_off)
+        o.append("  static constexpr int MWIN_OFF = %d;" % self.mwin_off)
+        # ---- window row: M pairs, then d y / d u (3 per component)
+        o.append("  static __device__ __forceinline__ void make_row(float ux, float uy, float uz, float* __restrict__ mrow) {")
+        yneed = set()
+        for (p, a, b1, terms) in self.ment:
+            for b2 in terms:
+                yneed.add((T.paths[p][1], b2))
+        for (l2, b2) in sorted(yneed):
+            o.append("    const float y_%d_%d = %s;" % (l2, b2, poly_expr(T.ypoly[l2][b2]) if l2 else "1.0f"))
+        vals = []
+        for k, (p, a, b1, terms) in enumerate(self.ment):
+            l2 = T.paths[p][1]
+            vals.append(lincomb_expr(terms, lambda b, l2=l2: "y_%d_%d" % (l2, b)))
+        while len(vals) < self.dbase:
+            vals.append("0.0f")
+        for (l2, b2) in self.ycomps:
+            for j in range(3):
+                vals.append(poly_expr(direction_derivative_polys(l2)[b2][j]))
+        while len(vals) % 4:
+            vals.append("0.0f")
+        for q in range(len(vals) // 4):
+            o.append("    st_f4(mrow + %d, %s, %s, %s, %s);" % (4 * q, *vals[4 * q:4 * q + 4]))
+        o.append("  }")
+        # ---- staging
+        o.append("  static __device__ __forceinline__ void issue(float* st, const float* __restrict__ xv, const float* __restrict__ we, int C, bool xok, bool ok) {")
+        for i, r in enumerate(self.xrows):
+            o.append("    cp_async16(st + %d, xv + %d * C, xok);" % (128 * i, r))
+        for i, p in enumerate(self.gpaths):
+            o.append("    cp_async16(st + %d, we + %d * C, ok);" % (128 * (len(self.xrows) + i), p))
+        o.append("  }")
+        # ---- load g rows of the receiver
+        o.append("  static __device__ __forceinline__ void load_g(const float* __restrict__ gu, int C, int sum_paths, float4 (&gr)[NA]) {")
+        o.append("    if (!sum_paths) {")
+        for i, (p, a) in enumerate(self.rows):
+            o.append("      gr[%d] = ld_x4(gu + %d * C);" % (i, T.zslot(p, a)))
+        o.append("    } else {")
+        for i, (p, a) in enumerate(self.rows):
+            o.append("      gr[%d] = ld_x4(gu + %d * C);" % (i, T.zslot(p, a, True)))
+        o.append("    }")
+        o.append("  }")
+        # ---- one edge
+        xidx = {r: i for i, r in enumerate(self.xrows)}
+        gi = {r: i for i, r in enumerate(self.rows)}
+        o.append("  static __device__ __forceinline__ void edge(const float4 (&gr)[NA], const float* st, const float* __restrict__ m,")
+        o.append("      float4 (&xb)[NX], float (&yb)[%d], float* __restrict__ wbar_e, int C, bool act) {" % max(1, self.NYD))
+        for i, r in enumerate(self.xrows):
+            o.append("    const float4 x%d = ld_s4(st + %d);" % (r, 128 * i))
+        ycidx = {c: i for i, c in enumerate(self.ycomps)}
+        mi = 0
+        loaded = set()
+        for pi, p in enumerate(self.gpaths):
+            l1, l2, l3 = T.paths[p]
+            ents = [(a, b1, terms) for (pp, a, b1, terms) in self.ment if pp == p]
+            bset = sorted(set(b for _, b, _ in ents))
+            names = []
+            for k in range(len(ents)):
+                q, c = divmod(mi + k, 4)
+                if q not in loaded:
+                    o.append("    const float4 mq%d = ld_s4(m + %d);" % (q, 4 * q))
+                    loaded.add(q)
+                names.append("mq%d.%s" % (q, "xyzw"[c]))
+            mi += len(ents)
+            o.append("    { // path (%d,%d)->%d" % (l1, l2, l3))
+            o.append("      const float4 w = ld_s4(st + %d);" % (128 * (len(self.xrows) + pi)))
+            # h_b1 = sum_a M[a][b1] g_a  (row-major order keeps the chains apart)
+            started = set()
+            for k, (a, b, _) in enumerate(ents):
+                ga = "gr[%d]" % gi[(p, a)]
+                if b not in started:
+                    o.append("      float4 h%d = mul4s(%s, %s);" % (b, names[k], ga))
+                    started.add(b)
+                else:
+                    o.append("      h%d = fma4s(%s, %s, h%d);" % (b, names[k], ga, b))
+            # w_bar = <h, x>;  x_bar += w h
+            first = True
+            for b in bset:
+                xr = "x%d" % (l1 * l1 + b)
+                if first:
+                    o.append("      float4 wb = mul4(h%d, %s);" % (b, xr))
+                    first = False
+                else:
+                    o.append("      wb = fma4(h%d, %s, wb);" % (b, xr))
+                o.append("      xb[%d] = fma4(w, h%d, xb[%d]);" % (xidx[l1 * l1 + b], b, xidx[l1 * l1 + b]))
+            o.append("      if (act) st_z4(wbar_e + %d * C, wb);" % p)
+            # y_bar: d_(a,b1) = <g_a, w x_b1> over the lane's 4 channels, then K
+            if l2 > 0:
+                for b in bset:
+                    o.append("      const float4 t%d = mul4(w, x%d);" % (b, l1 * l1 + b))
+                for k, (a, b, terms) in enumerate(ents):
+                    o.append("      { const float d = dot4(gr[%d], t%d);" % (gi[(p, a)], b))
+                    for b2, c in sorted(terms.items()):
+                        o.append("        yb[%d] = fmaf(%s, d, yb[%d]);" % (ycidx[(l2, b2)], flit(c), ycidx[(l2, b2)]))
+                    o.append("      }")
+            o.append("    }")
+        o.append("  }")
+        # ---- u_bar = (d y / d u)^T y_bar  (uniform d y / d u from the window)
+        o.append("  static __device__ __forceinline__ void ubar(const float (&yb)[%d], const float* __restrict__ m, float& ux, float& uy, float& uz) {" % max(1, self.NYD))
+        o.append("    ux = 0.0f; uy = 0.0f; uz = 0.0f;")
+        for i in range(self.NYD):
+            base = self.dbase + 3 * i
+            o.append("    ux = fmaf(yb[%d], m[%d], ux); uy = fmaf(yb[%d], m[%d], uy); uz = fmaf(yb[%d], m[%d], uz);" %
+                     (i, base, i, base + 1, i, base + 2))
+        o.append("  }")
+        # ---- x_bar rows
+        o.append("  static __device__ __forceinline__ void flush_xbar(float* __restrict__ xbv, int C, float4 (&xb)[NX]) {")
+        for i, r in enumerate(self.xrows):
+            o.append("    red_add4(xbv + %d * C, xb[%d]); xb[%d] = zero4();" % (r, i, i))
+        o.append("  }")
+        o.append("};")
+        return "\n".join(o)
+
+
+VJP_NGROUPS = {2: 4, 3: 8, 4: 8}
+VJP_STAGES = {2: 3, 3: 3, 4: 2}
+VJP_MWIN = {2: 16, 3: 16, 4: 8}
+
+
+def emit_vjp(L, G):
+    T = Tables(L)
+    groups = partition_paths(T, G, lambda p: vjp_path_cost(T, p))
+    codes = [VjpGroupCode(T, ps, g) for g, ps in enumerate(groups)]
+    off = 0
+    for c in codes:
+        c.ring_off = off
+        off += VJP_STAGES[L] * 128 * c.NROW
+    for c in codes:
+        c.mwin_off = off
+        off += VJP_MWIN[L] * c.MSTRIDE
+    out = ["// Generated by gen/fc_codegen.py -- do not edit.",
+           "// Receiver-sorted VJP, rank %d: %d paths, %d warp groups (whole paths)." % (L, T.P, G)]
+    for c in codes:
+        out.append("//   group %d: paths %s, %d g rows, %d M entries, %d x rows, cost %d" %
+                   (c.gid, [T.paths[p] for p in c.gpaths], c.NA, c.NM, len(c.xrows),
+                    sum(vjp_path_cost(T, p) for p in c.gpaths)))
+    out += ["#pragma once", '#include "../fc_device.cuh"', "namespace fc {",
+            "template <> struct VjpMeta<%d> {" % L,
+            "  static constexpr int G = %d;" % G,
+            "  static constexpr int S = %d;" % VJP_STAGES[L],
+            "  static constexpr int MWIN = %d;" % VJP_MWIN[L],
+            "  static constexpr int P = %d;" % T.P,
+            "  static constexpr int SMEM_FLOATS = %d;" % off,
+            "};"]
+    for c in codes:
+        out.append(c.emit(L, G))
+    out.append("}  // namespace fc")
+    return "\n".join(out) + "\n", T, codes
+
+
+_main_fwd = main
+
+
+def main():
+    written = _main_fwd()
+    for L in (2, 3, 4):
+        src, _, _ = emit_vjp(L, VJP_NGROUPS[L])
+        path = os.path.join(OUTDIR, "fc_vjp_L%d.cuh" % L)
+        with open(path, "w") as f:
+            f.write(src)
+        written.append(path)
     return written
 
 

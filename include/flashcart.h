@@ -134,6 +134,27 @@ int fc_edge_conv(const fc_conv_desc *desc, int n_nodes, int n_edges,
                  const float *edge_vec, const float *x, const float *w,
                  float *z, fc_stream_t stream);
 
+/* Vector-Jacobian product of fc_edge_conv, App. C Eq. (C1) summed over the
+ * receiver-sorted edges as in Algorithm 2, with the direction-tensor
+ * gradient carried to the edge vectors (App. C "Symbolic derivatives"):
+ *   x_bar[v, :, k]  = sum_{e: v_e = v} sum_eta w[e,eta,k] (M_eta,e^T g[u_e,eta,k])
+ *   w_bar[e, eta, k] = <g[u_e, eta, k], f_eta(x[v_e, :, k], T(r-hat_e))>
+ *   r_bar[e]        = (d T(r_e/|r_e|) / d r_e)^T y_bar[e],
+ *   y_bar[e]        = sum_{eta,k} w[e,eta,k] d<g, f_eta(x, y)>/dy at y = T(r-hat_e)
+ * where M_eta,e[a][b] = d f_eta,a / d x_b and the gradients are taken with
+ * respect to the independent components as free variables (App. C).
+ *   g has the layout of z (fc_conv_out_row() x C per node);
+ *   x_bar [n_nodes][(lmax_in+1)^2 C], w_bar [n_edges][P][C], r_bar
+ *   [n_edges][3]: each may be NULL to skip it.  x_bar and r_bar are zeroed
+ *   on the stream and then accumulated with atomic additions (their bits
+ *   can differ run to run); w_bar is written once per entry.
+ * Same graph requirements and error returns as fc_edge_conv. */
+int fc_edge_conv_vjp(const fc_conv_desc *desc, int n_nodes, int n_edges,
+                     const int32_t *rowptr, const int32_t *edge_index,
+                     const float *edge_vec, const float *x, const float *w,
+                     const float *g, float *x_bar, float *w_bar, float *r_bar,
+                     fc_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif
