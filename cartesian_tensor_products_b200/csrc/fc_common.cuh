@@ -18,6 +18,8 @@ template <int L, int G, int g>
 struct VjpGroup;
 template <int L>
 struct VjpMeta;
+template <int L>
+struct LadderTP;
 
 inline bool aligned16(const void* p) {
   return (reinterpret_cast<uintptr_t>(p) & 15u) == 0;

@@ -1,0 +1,464 @@
+// libflashcart: node-local correlation ladder and its VJP.
+//
+// FlashCart (arXiv 2610.06409) Sec. 5 Eq. (2) with path-reduced products
+// (App. E "Path-reduced products") and a per-rank channel mix after every
+// product:
+//   B_v[n, l3, c, k] = sum_{paths (l1,l2)->l3} W_v[p, k] f_p(A_v[n,l1,:,k], A_1[n,l2,:,k])_c
+//   A_{v+1}[n, l, c, :] = M_{v,l} B_v[n, l, c, :]        (C x C per rank)
+//   z = A_1 + A_2 + ... + A_order
+// Every product couples channel k only with channel k (channel-diagonal,
+// Sec. 5), so the product kernel is one thread per channel walking a chunk
+// of nodes with the path weights of its channel in registers.  The mix is a
+// per-rank FP32 GEMM over the rows (node, component) of that rank, with the
+// new state and the running sum z written in its epilogue.  The VJP replays
+// the steps backwards: B_v is recomputed, B_bar = M^T-product of A_bar,
+// M_bar += A_bar^T B (split over row chunks, atomic tile adds), and the
+// product VJP (App. C Eq. C1 per path) adds into A_v_bar and A_1_bar and
+// accumulates W_bar over its node chunk before one atomic add per entry.
+#include "fc_common.cuh"
+#include "fc_device.cuh"
+#include "generated/fc_ladder_L2.cuh"
+#include "generated/fc_ladder_L3.cuh"
+#include "generated/fc_ladder_L4.cuh"
+
+namespace fc {
+
+constexpr int kLadderNodeChunk = 16;   // nodes per thread in the product kernels
+
+// ---------------------------------------------------------------------------
+// channel-diagonal products
+// ---------------------------------------------------------------------------
+template <int L>
+__global__ void __launch_bounds__(128) ladder_tp_kernel(int N, int C, const float* __restrict__ Av,
+                                                        const float* __restrict__ A1,
+                                                        const float* __restrict__ W,
+                                                        float* __restrict__ B) {
+  using TP = LadderTP<L>;
+  const int k = blockIdx.y * blockDim.x + threadIdx.x;
+  if (k >= C) return;
+  float w[TP::P];
+#pragma unroll
+  for (int p = 0; p < TP::P; ++p) w[p] = __ldg(W + (size_t)p * C + k);
+  const int n0 = blockIdx.x * kLadderNodeChunk;
+  const int n1 = min(N, n0 + kLadderNodeChunk);
+  for (int n = n0; n < n1; ++n) {
+    const size_t base = (size_t)n * TP::NY * C + k;
+    float a[TP::NY], b[TP::NY], o[TP::NY];
+#pragma unroll
+    for (int i = 0; i < TP::NY; ++i) {
+      a[i] = __ldg(Av + base + (size_t)i * C);
+      b[i] = __ldg(A1 + base + (size_t)i * C);
+    }
+    TP::fwd(a, b, w, o);
+#pragma unroll
+    for (int i = 0; i < TP::NY; ++i) B[base + (size_t)i * C] = o[i];
+  }
+}
+
+// Avbar += w VJP1, A1bar += w VJP2, Wbar += <g, f> (atomic, once per chunk).
+// Avbar may alias A1bar (first step: A_v = A_1).
+template <int L>
+__global__ void __launch_bounds__(128) ladder_tp_vjp_kernel(int N, int C, const float* __restrict__ Av,
+                                                            const float* __restrict__ A1,
+                                                            const float* __restrict__ W,
+                                                            const float* __restrict__ G,
+                                                            float* Avbar, float* A1bar,
+                                                            float* __restrict__ Wbar) {
+  using TP = LadderTP<L>;
+  const int k = blockIdx.y * blockDim.x + threadIdx.x;
+  if (k >= C) return;
+  float w[TP::P], wb[TP::P];
+#pragma unroll
+  for (int p = 0; p < TP::P; ++p) {
+    w[p] = __ldg(W + (size_t)p * C + k);
+    wb[p] = 0.0f;
+  }
+  const bool alias = (Avbar == A1bar);
+  const int n0 = blockIdx.x * kLadderNodeChunk;
+  const int n1 = min(N, n0 + kLadderNodeChunk);
+  for (int n = n0; n < n1; ++n) {
+    const size_t base = (size_t)n * TP::NY * C + k;
+    float a[TP::NY], b[TP::NY], g[TP::NY], ab[TP::NY], bb[TP::NY];
+#pragma unroll
+    for (int i = 0; i < TP::NY; ++i) {
+      a[i] = __ldg(Av + base + (size_t)i * C);
+      b[i] = __ldg(A1 + base + (size_t)i * C);
+      g[i] = __ldg(G + base + (size_t)i * C);
+      ab[i] = 0.0f;
+      bb[i] = 0.0f;
+    }
+    TP::vjp(a, b, w, g, ab, bb, wb);
+    if (alias) {
+#pragma unroll
+      for (int i = 0; i < TP::NY; ++i) A1bar[base + (size_t)i * C] += ab[i] + bb[i];
+    } else {
+#pragma unroll
+      for (int i = 0; i < TP::NY; ++i) {
+        Avbar[base + (size_t)i * C] += ab[i];
+        A1bar[base + (size_t)i * C] += bb[i];
+      }
+    }
+  }
+#pragma unroll
+  for (int p = 0; p < TP::P; ++p) atomicAdd(Wbar + (size_t)p * C + k, wb[p]);
+}
+
+// ---------------------------------------------------------------------------
+// per-rank channel mixing GEMMs (FP32, register-tiled)
+// ---------------------------------------------------------------------------
+// rows of rank l: i in [0, N(2l+1)) -> node n = i / (2l+1), component c.
+__device__ __forceinline__ size_t rank_row(int i, int l, int NY, int C) {
+  const int w = 2 * l + 1;
+  const int n = i / w;
+  const int c = i - n * w;
+  return ((size_t)n * NY + l * l + c) * C;
+}
+
+enum { kMixFwd = 0, kMixBar = 1 };
+
+constexpr int kBM = 64, kBN = 128, kBK = 32;
+
+// kMixFwd: out[r][j] = sum_t in[r][t] M[j][t]   (in x M^T), z[r][j] += out
+// kMixBar: out[r][j] = sum_t in[r][t] M[t][j]   (in x M)
+template <int MODE>
+__global__ void __launch_bounds__(256) ladder_mix_kernel(int N, int C, int NY,
+                                                         const float* __restrict__ in,
+                                                         const float* __restrict__ Mall,
+                                                         float* __restrict__ out, float* z) {
+  __shared__ __align__(16) float As[kBK][kBM + 4];
+  __shared__ __align__(16) float Bs[kBK][kBN + 4];
+  const int l = blockIdx.z;
+  const int R = N * (2 * l + 1);
+  const int r0 = blockIdx.x * kBM;
+  if (r0 >= R) return;
+  const int j0 = blockIdx.y * kBN;
+  const float* M = Mall + (size_t)l * C * C;
+  const int tid = threadIdx.x;
+  const int tx = tid & 15, ty = tid >> 4;  // 16 x 16 threads: 8 cols x 4 rows each
+  float acc[4][8];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc[i][j] = 0.0f;
+
+  for (int t0 = 0; t0 < C; t0 += kBK) {
+    // A tile: 64 rows x 32 t, two float4 per thread, stored t-major
+#pragma unroll
+    for (int s = 0; s < 2; ++s) {
+      const int idx = tid + s * 256;        // 0..511
+      const int rr = idx >> 3, tq = (idx & 7) * 4;
+      float4 v = zero4();
+      if (r0 + rr < R && t0 + tq < C)
+        v = __ldg(reinterpret_cast<const float4*>(in + rank_row(r0 + rr, l, NY, C) + t0 + tq));
+      As[tq + 0][rr] = v.x; As[tq + 1][rr] = v.y; As[tq + 2][rr] = v.z; As[tq + 3][rr] = v.w;
+    }
+    // B tile: 32 t x 128 j
+#pragma unroll
+    for (int s = 0; s < 4; ++s) {
+      const int idx = tid + s * 256;        // 0..1023
+      if (MODE == kMixFwd) {
+        const int jj = idx >> 3, tq = (idx & 7) * 4;   // M[j][t..t+3]
+        float4 v = zero4();
+        if (j0 + jj < C && t0 + tq < C)
+          v = __ldg(reinterpret_cast<const float4*>(M + (size_t)(j0 + jj) * C + t0 + tq));
+        Bs[tq + 0][jj] = v.x; Bs[tq + 1][jj] = v.y; Bs[tq + 2][jj] = v.z; Bs[tq + 3][jj] = v.w;
+      } else {
+        const int tt = idx >> 5, jq = (idx & 31) * 4;  // M[t][j..j+3]
+        float4 v = zero4();
+        if (t0 + tt < C && j0 + jq < C)
+          v = __ldg(reinterpret_cast<const float4*>(M + (size_t)(t0 + tt) * C + j0 + jq));
+        *reinterpret_cast<float4*>(&Bs[tt][jq]) = v;
+      }
+    }
+    __syncthreads();
+#pragma unroll 8
+    for (int t = 0; t < kBK; ++t) {
+      const float4 a = *reinterpret_cast<const float4*>(&As[t][ty * 4]);
+      const float4 b0 = *reinterpret_cast<const float4*>(&Bs[t][tx * 8]);
+      const float4 b1 = *reinterpret_cast<const float4*>(&Bs[t][tx * 8 + 4]);
+      const float av[4] = {a.x, a.y, a.z, a.w};
+      const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int r = r0 + ty * 4 + i;
+    if (r >= R) continue;
+    const size_t base = rank_row(r, l, NY, C);
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int j = j0 + tx * 8 + h * 4;
+      if (j >= C) continue;
+      const float4 v = make_float4(acc[i][h * 4], acc[i][h * 4 + 1], acc[i][h * 4 + 2], acc[i][h * 4 + 3]);
+      *reinterpret_cast<float4*>(out + base + j) = v;
+      if (MODE == kMixFwd) {
+        float4 zz = *reinterpret_cast<float4*>(z + base + j);
+        zz.x += v.x; zz.y += v.y; zz.z += v.z; zz.w += v.w;
+        *reinterpret_cast<float4*>(z + base + j) = zz;
+      }
+    }
+  }
+}
+
+constexpr int kWgradRows = 512;   // rows per CTA of the weight-gradient GEMM
+
+// Mbar_l[k][j] += sum_{rows i of rank l} Abar[i][k] B[i][j]
+__global__ void __launch_bounds__(256) ladder_wgrad_kernel(int N, int C, int NY,
+                                                           const float* __restrict__ Abar,
+                                                           const float* __restrict__ B,
+                                                           float* __restrict__ Mbar) {
+  __shared__ __align__(16) float As[kBK][kBM + 4];
+  __shared__ __align__(16) float Bs[kBK][kBN + 4];
+  const int l = blockIdx.z;
+  const int R = N * (2 * l + 1);
+  const int i0 = blockIdx.x * kWgradRows;
+  if (i0 >= R) return;
+  const int i1 = min(R, i0 + kWgradRows);
+  const int ktiles = (C + kBM - 1) / kBM;
+  const int k0 = (blockIdx.y % ktiles) * kBM;
+  const int j0 = (blockIdx.y / ktiles) * kBN;
+  const int tid = threadIdx.x;
+  const int tx = tid & 15, ty = tid >> 4;
+  float acc[4][8];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc[i][j] = 0.0f;
+  for (int t0 = i0; t0 < i1; t0 += kBK) {
+    // A: 32 rows x 64 k  (two float4 per thread)
+#pragma unroll
+    for (int s = 0; s < 2; ++s) {
+      const int idx = tid + s * 256;       // 0..511
+      const int tt = idx >> 4, kq = (idx & 15) * 4;
+      float4 v = zero4();
+      if (t0 + tt < i1 && k0 + kq < C)
+        v = __ldg(reinterpret_cast<const float4*>(Abar + rank_row(t0 + tt, l, NY, C) + k0 + kq));
+      *reinterpret_cast<float4*>(&As[tt][kq]) = v;
+    }
+    // B: 32 rows x 128 j
+#pragma unroll
+    for (int s = 0; s < 4; ++s) {
+      const int idx = tid + s * 256;       // 0..1023
+      const int tt = idx >> 5, jq = (idx & 31) * 4;
+      float4 v = zero4();
+      if (t0 + tt < i1 && j0 + jq < C)
+        v = __ldg(reinterpret_cast<const float4*>(B + rank_row(t0 + tt, l, NY, C) + j0 + jq));
+      *reinterpret_cast<float4*>(&Bs[tt][jq]) = v;
+    }
+    __syncthreads();
+#pragma unroll 8
+    for (int t = 0; t < kBK; ++t) {
+      const float4 a = *reinterpret_cast<const float4*>(&As[t][ty * 4]);
+      const float4 b0 = *reinterpret_cast<const float4*>(&Bs[t][tx * 8]);
+      const float4 b1 = *reinterpret_cast<const float4*>(&Bs[t][tx * 8 + 4]);
+      const float av[4] = {a.x, a.y, a.z, a.w};
+      const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+    }
+    __syncthreads();
+  }
+  float* Ml = Mbar + (size_t)l * C * C;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int k = k0 + ty * 4 + i;
+    if (k >= C) continue;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int jj = j0 + tx * 8 + j;
+      if (jj < C) atomicAdd(Ml + (size_t)k * C + jj, acc[i][j]);
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// orchestration
+// ---------------------------------------------------------------------------
+static int check_ladder_desc(const fc_ladder_desc* d) {
+  if (!d) return FC_ERR_ARG;
+  if (d->channels <= 0 || d->order < 1 || d->lmax < 0) return FC_ERR_ARG;
+  if (d->lmax < 2 || d->lmax > 4) return FC_ERR_UNSUPPORTED_RANK;
+  if (d->channels % 4) return FC_ERR_ALIGN;
+  return FC_OK;
+}
+
+template <int L>
+static int launch_tp(int N, int C, const float* Av, const float* A1, const float* W, float* B,
+                     cudaStream_t s) {
+  dim3 grid((N + kLadderNodeChunk - 1) / kLadderNodeChunk, (C + 127) / 128);
+  ladder_tp_kernel<L><<<grid, 128, 0, s>>>(N, C, Av, A1, W, B);
+  return cudaGetLastError() == cudaSuccess ? FC_OK : FC_ERR_CUDA;
+}
+
+template <int L>
+static int launch_tp_vjp(int N, int C, const float* Av, const float* A1, const float* W,
+                         const float* G, float* Avbar, float* A1bar, float* Wbar, cudaStream_t s) {
+  dim3 grid((N + kLadderNodeChunk - 1) / kLadderNodeChunk, (C + 127) / 128);
+  ladder_tp_vjp_kernel<L><<<grid, 128, 0, s>>>(N, C, Av, A1, W, G, Avbar, A1bar, Wbar);
+  return cudaGetLastError() == cudaSuccess ? FC_OK : FC_ERR_CUDA;
+}
+
+static int tp_dispatch(int L, int N, int C, const float* Av, const float* A1, const float* W,
+                       float* B, cudaStream_t s) {
+  switch (L) {
+    case 2: return launch_tp<2>(N, C, Av, A1, W, B, s);
+    case 3: return launch_tp<3>(N, C, Av, A1, W, B, s);
+    case 4: return launch_tp<4>(N, C, Av, A1, W, B, s);
+  }
+  return FC_ERR_UNSUPPORTED_RANK;
+}
+
+static int tp_vjp_dispatch(int L, int N, int C, const float* Av, const float* A1, const float* W,
+                           const float* G, float* Avbar, float* A1bar, float* Wbar, cudaStream_t s) {
+  switch (L) {
+    case 2: return launch_tp_vjp<2>(N, C, Av, A1, W, G, Avbar, A1bar, Wbar, s);
+    case 3: return launch_tp_vjp<3>(N, C, Av, A1, W, G, Avbar, A1bar, Wbar, s);
+    case 4: return launch_tp_vjp<4>(N, C, Av, A1, W, G, Avbar, A1bar, Wbar, s);
+  }
+  return FC_ERR_UNSUPPORTED_RANK;
+}
+
+template <int MODE>
+static int launch_mix(int L, int N, int C, const float* in, const float* M, float* out, float* z,
+                      cudaStream_t s) {
+  const int NY = (L + 1) * (L + 1);
+  const int Rmax = N * (2 * L + 1);
+  dim3 grid((Rmax + kBM - 1) / kBM, (C + kBN - 1) / kBN, L + 1);
+  ladder_mix_kernel<MODE><<<grid, 256, 0, s>>>(N, C, NY, in, M, out, z);
+  return cudaGetLastError() == cudaSuccess ? FC_OK : FC_ERR_CUDA;
+}
+
+static int launch_wgrad(int L, int N, int C, const float* Abar, const float* B, float* Mbar,
+                        cudaStream_t s) {
+  const int NY = (L + 1) * (L + 1);
+  const int Rmax = N * (2 * L + 1);
+  const int tiles = ((C + kBM - 1) / kBM) * ((C + kBN - 1) / kBN);
+  dim3 grid((Rmax + kWgradRows - 1) / kWgradRows, tiles, L + 1);
+  ladder_wgrad_kernel<<<grid, 256, 0, s>>>(N, C, NY, Abar, B, Mbar);
+  return cudaGetLastError() == cudaSuccess ? FC_OK : FC_ERR_CUDA;
+}
+
+}  // namespace fc
+
+using namespace fc;
+
+extern "C" {
+
+int fc_ladder_num_paths(const fc_ladder_desc* d) {
+  if (check_ladder_desc(d) != FC_OK) return -1;
+  return num_paths(d->lmax);
+}
+
+size_t fc_product_ladder_workspace_size(const fc_ladder_desc* d, int n_nodes) {
+  if (check_ladder_desc(d) != FC_OK || n_nodes < 0) return 0;
+  const int NY = (d->lmax + 1) * (d->lmax + 1);
+  return sizeof(float) * (size_t)n_nodes * NY * d->channels;
+}
+
+int fc_product_ladder(const fc_ladder_desc* d, int n_nodes, const float* A1, const float* path_w,
+                      const float* mix_w, float* states, float* z, void* workspace,
+                      size_t ws_bytes, fc_stream_t stream) {
+  int st = check_ladder_desc(d);
+  if (st != FC_OK) return st;
+  if (n_nodes < 0) return FC_ERR_ARG;
+  if (n_nodes == 0) return FC_OK;
+  const int L = d->lmax, C = d->channels, S = d->order - 1;
+  if (!A1 || !z || (S > 0 && (!path_w || !mix_w || !states))) return FC_ERR_ARG;
+  if (!aligned16(A1) || !aligned16(z) || (S > 0 && (!aligned16(mix_w) || !aligned4(path_w) ||
+                                                    !aligned16(states))))
+    return FC_ERR_ALIGN;
+  const size_t need = fc_product_ladder_workspace_size(d, n_nodes);
+  if (S > 0 && (!workspace || ws_bytes < need)) return FC_ERR_WORKSPACE;
+  if (S > 0 && !aligned16(workspace)) return FC_ERR_ALIGN;
+  cudaStream_t s = (cudaStream_t)stream;
+  const int NY = (L + 1) * (L + 1);
+  const size_t plane = (size_t)n_nodes * NY * C;
+  const int P = num_paths(L);
+  if (cudaMemcpyAsync(z, A1, sizeof(float) * plane, cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+    return FC_ERR_CUDA;
+  float* B = static_cast<float*>(workspace);
+  for (int v = 1; v <= S; ++v) {
+    const float* Av = v == 1 ? A1 : states + (size_t)(v - 2) * plane;
+    st = tp_dispatch(L, n_nodes, C, Av, A1, path_w + (size_t)(v - 1) * P * C, B, s);
+    if (st != FC_OK) return st;
+    st = launch_mix<kMixFwd>(L, n_nodes, C, B, mix_w + (size_t)(v - 1) * (L + 1) * C * C,
+                             states + (size_t)(v - 1) * plane, z, s);
+    if (st != FC_OK) return st;
+  }
+  return FC_OK;
+}
+
+size_t fc_product_ladder_vjp_workspace_size(const fc_ladder_desc* d, int n_nodes) {
+  if (check_ladder_desc(d) != FC_OK || n_nodes < 0) return 0;
+  const int NY = (d->lmax + 1) * (d->lmax + 1);
+  return 4 * sizeof(float) * (size_t)n_nodes * NY * d->channels;
+}
+
+int fc_product_ladder_vjp(const fc_ladder_desc* d, int n_nodes, const float* A1,
+                          const float* path_w, const float* mix_w, const float* states,
+                          const float* gz, float* A1_bar, float* path_w_bar, float* mix_w_bar,
+                          void* workspace, size_t ws_bytes, fc_stream_t stream) {
+  int st = check_ladder_desc(d);
+  if (st != FC_OK) return st;
+  if (n_nodes < 0) return FC_ERR_ARG;
+  const int L = d->lmax, C = d->channels, S = d->order - 1;
+  const int NY = (L + 1) * (L + 1);
+  const int P = num_paths(L);
+  cudaStream_t s = (cudaStream_t)stream;
+  if (!gz || !A1_bar || !A1) return FC_ERR_ARG;
+  if (S > 0 && (!path_w || !mix_w || !states || !path_w_bar || !mix_w_bar)) return FC_ERR_ARG;
+  if (!aligned16(A1) || !aligned16(gz) || !aligned16(A1_bar) ||
+      (S > 0 && (!aligned16(mix_w) || !aligned16(states) || !aligned4(path_w) ||
+                 !aligned4(path_w_bar) || !aligned4(mix_w_bar))))
+    return FC_ERR_ALIGN;
+  const size_t need = fc_product_ladder_vjp_workspace_size(d, n_nodes);
+  if (S > 0 && n_nodes > 0 && (!workspace || ws_bytes < need)) return FC_ERR_WORKSPACE;
+  if (S > 0 && n_nodes > 0 && !aligned16(workspace)) return FC_ERR_ALIGN;
+  const size_t plane = (size_t)n_nodes * NY * C;
+  if (S > 0) {
+    if (cudaMemsetAsync(path_w_bar, 0, sizeof(float) * (size_t)S * P * C, s) != cudaSuccess ||
+        cudaMemsetAsync(mix_w_bar, 0, sizeof(float) * (size_t)S * (L + 1) * C * C, s) != cudaSuccess)
+      return FC_ERR_CUDA;
+  }
+  if (n_nodes == 0) return FC_OK;
+  // every A_v feeds z directly
+  if (cudaMemcpyAsync(A1_bar, gz, sizeof(float) * plane, cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+    return FC_ERR_CUDA;
+  float* ws = static_cast<float*>(workspace);
+  float* B = ws;
+  float* Bbar = ws + plane;
+  float* Ab[2] = {ws + 2 * plane, ws + 3 * plane};
+  const float* Anext_bar = gz;           // gradient of A_{v+1}
+  for (int v = S; v >= 1; --v) {
+    const float* Av = v == 1 ? A1 : states + (size_t)(v - 2) * plane;
+    const float* W = path_w + (size_t)(v - 1) * P * C;
+    const float* M = mix_w + (size_t)(v - 1) * (L + 1) * C * C;
+    float* Avbar;
+    if (v == 1) {
+      Avbar = A1_bar;
+    } else {
+      Avbar = Ab[v & 1];
+      if (cudaMemcpyAsync(Avbar, gz, sizeof(float) * plane, cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+        return FC_ERR_CUDA;
+    }
+    if ((st = tp_dispatch(L, n_nodes, C, Av, A1, W, B, s)) != FC_OK) return st;
+    if ((st = launch_mix<kMixBar>(L, n_nodes, C, Anext_bar, M, Bbar, nullptr, s)) != FC_OK) return st;
+    if ((st = launch_wgrad(L, n_nodes, C, Anext_bar, B, mix_w_bar + (size_t)(v - 1) * (L + 1) * C * C,
+                           s)) != FC_OK)
+      return st;
+    if ((st = tp_vjp_dispatch(L, n_nodes, C, Av, A1, W, Bbar, Avbar, A1_bar,
+                              path_w_bar + (size_t)(v - 1) * P * C, s)) != FC_OK)
+      return st;
+    Anext_bar = Avbar;
+  }
+  return FC_OK;
+}
+
+}  // extern "C"

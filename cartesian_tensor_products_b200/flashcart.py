@@ -56,6 +56,13 @@ _SIGS = {
                                 _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
     "fc_edge_conv_vjp": (ct.c_int, [ct.POINTER(ConvDesc), ct.c_int, ct.c_int,
                                     _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
+    "fc_ladder_num_paths": (ct.c_int, [ct.POINTER(LadderDesc)]),
+    "fc_product_ladder_workspace_size": (ct.c_size_t, [ct.POINTER(LadderDesc), ct.c_int]),
+    "fc_product_ladder": (ct.c_int, [ct.POINTER(LadderDesc), ct.c_int, _vp, _vp, _vp, _vp,
+                                     _vp, _vp, ct.c_size_t, _vp]),
+    "fc_product_ladder_vjp_workspace_size": (ct.c_size_t, [ct.POINTER(LadderDesc), ct.c_int]),
+    "fc_product_ladder_vjp": (ct.c_int, [ct.POINTER(LadderDesc), ct.c_int, _vp, _vp, _vp, _vp,
+                                         _vp, _vp, _vp, _vp, _vp, ct.c_size_t, _vp]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _f = getattr(_lib, _name)
@@ -199,3 +206,58 @@ def edge_conv_vjp(lmax, rowptr, edge_index, edge_vec, x, w, g, sum_paths=False,
                                  _ptr(edge_vec), _ptr(x), _ptr(w), _ptr(g), _ptr(xb),
                                  _ptr(wb), _ptr(rb), _stream(stream)), "fc_edge_conv_vjp")
     return xb, wb, rb
+
+
+def _workspace(nbytes, device):
+    if nbytes == 0:
+        return None
+    return torch.empty((nbytes + 15) // 16 * 4, dtype=torch.float32, device=device)
+
+
+def product_ladder(lmax, order, A1, path_w, mix_w, workspace=None, stream=None):
+    """(states [order-1][N][...], z) of Sec. 5 Eq. (2), path-reduced products
+    followed by a per-rank channel mix."""
+    _dev(A1, torch.float32, "A1")
+    N = A1.shape[0]
+    NY = (lmax + 1) ** 2
+    C = A1.shape[1] // NY
+    d = LadderDesc(lmax, C, order)
+    S = order - 1
+    states = torch.empty((max(S, 0), N, NY * C), dtype=torch.float32, device=A1.device)
+    z = torch.empty_like(A1)
+    ws_bytes = _lib.fc_product_ladder_workspace_size(ct.byref(d), N)
+    if workspace is None:
+        workspace = _workspace(ws_bytes, A1.device)
+    if S > 0:
+        _dev(path_w, torch.float32, "path_w")
+        _dev(mix_w, torch.float32, "mix_w")
+    _check(_lib.fc_product_ladder(ct.byref(d), N, _ptr(A1), _ptr(path_w) if S > 0 else None,
+                                  _ptr(mix_w) if S > 0 else None, _ptr(states) if S > 0 else None,
+                                  _ptr(z), _ptr(workspace), ws_bytes if workspace is not None else 0,
+                                  _stream(stream)), "fc_product_ladder")
+    return states, z
+
+
+def product_ladder_vjp(lmax, order, A1, path_w, mix_w, states, gz, workspace=None,
+                       stream=None):
+    """(A1_bar, path_w_bar, mix_w_bar) of fc_product_ladder."""
+    _dev(A1, torch.float32, "A1")
+    _dev(gz, torch.float32, "gz")
+    N = A1.shape[0]
+    NY = (lmax + 1) ** 2
+    C = A1.shape[1] // NY
+    d = LadderDesc(lmax, C, order)
+    S = order - 1
+    A1b = torch.empty_like(A1)
+    pwb = torch.empty((max(S, 0),) + tuple(path_w.shape[1:]), dtype=torch.float32, device=A1.device)
+    mwb = torch.empty((max(S, 0),) + tuple(mix_w.shape[1:]), dtype=torch.float32, device=A1.device)
+    ws_bytes = _lib.fc_product_ladder_vjp_workspace_size(ct.byref(d), N)
+    if workspace is None:
+        workspace = _workspace(ws_bytes, A1.device)
+    _check(_lib.fc_product_ladder_vjp(
+        ct.byref(d), N, _ptr(A1), _ptr(path_w) if S > 0 else None,
+        _ptr(mix_w) if S > 0 else None, _ptr(states) if S > 0 else None, _ptr(gz),
+        _ptr(A1b), _ptr(pwb) if S > 0 else None, _ptr(mwb) if S > 0 else None,
+        _ptr(workspace), ws_bytes if workspace is not None else 0, _stream(stream)),
+        "fc_product_ladder_vjp")
+    return A1b, pwb, mwb

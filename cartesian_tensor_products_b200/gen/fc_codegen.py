@@ -675,6 +675,82 @@ def main():
     return written
 
 
+
+# ---------------------------------------------------------------------------
+# node-local product ladder (Sec. 5 Eq. 2, path-reduced products, App. E)
+# ---------------------------------------------------------------------------
+
+def emit_ladder(L):
+    """Channel-diagonal products of one node and one channel:
+       B[l3^2 + c] = sum_{paths -> l3} w_p f_p(a[l1 block], b[l2 block])_c
+    and their VJP (App. C Eq. C1 applied per path)."""
+    T = Tables(L)
+    NY = (L + 1) ** 2
+    o = ["// Generated by gen/fc_codegen.py -- do not edit.",
+         "// Node-local channel-diagonal products, rank %d, %d paths." % (L, T.P),
+         "#pragma once", "namespace fc {",
+         "template <> struct LadderTP<%d> {" % L,
+         "  static constexpr int NY = %d;" % NY,
+         "  static constexpr int P = %d;" % T.P]
+    # forward
+    o.append("  static __device__ __forceinline__ void fwd(const float (&a)[NY], const float (&b)[NY], const float (&w)[P], float (&B)[NY]) {")
+    o.append("#pragma unroll")
+    o.append("    for (int i = 0; i < NY; ++i) B[i] = 0.0f;")
+    for p, (l1, l2, l3) in enumerate(T.paths):
+        K = T.K[p]
+        for c in range(2 * l3 + 1):
+            terms = [(b1, b2, K[c][b1][b2]) for b1 in range(2 * l1 + 1)
+                     for b2 in range(2 * l2 + 1) if K[c][b1][b2] != 0]
+            if not terms:
+                continue
+            expr = " + ".join("%s*(a[%d]*b[%d])" % (flit(k), l1 * l1 + b1, l2 * l2 + b2)
+                              for b1, b2, k in terms)
+            o.append("    B[%d] = fmaf(w[%d], %s, B[%d]);" % (l3 * l3 + c, p, expr, l3 * l3 + c))
+    o.append("  }")
+    # VJP: g is the gradient of B
+    o.append("  static __device__ __forceinline__ void vjp(const float (&a)[NY], const float (&b)[NY], const float (&w)[P], const float (&g)[NY],")
+    o.append("                                             float (&abar)[NY], float (&bbar)[NY], float (&wbar)[P]) {")
+    for p, (l1, l2, l3) in enumerate(T.paths):
+        K = T.K[p]
+        o.append("    { // path (%d,%d)->%d" % (l1, l2, l3))
+        # w_bar = <g, f>
+        fterms = []
+        for c in range(2 * l3 + 1):
+            for b1 in range(2 * l1 + 1):
+                for b2 in range(2 * l2 + 1):
+                    if K[c][b1][b2] != 0:
+                        fterms.append("%s*(g[%d]*(a[%d]*b[%d]))" % (flit(K[c][b1][b2]), l3 * l3 + c, l1 * l1 + b1, l2 * l2 + b2))
+        o.append("      wbar[%d] += %s;" % (p, " + ".join(fterms)))
+        for b1 in range(2 * l1 + 1):
+            t = ["%s*(g[%d]*b[%d])" % (flit(K[c][b1][b2]), l3 * l3 + c, l2 * l2 + b2)
+                 for c in range(2 * l3 + 1) for b2 in range(2 * l2 + 1) if K[c][b1][b2] != 0]
+            if t:
+                o.append("      abar[%d] = fmaf(w[%d], %s, abar[%d]);" % (l1 * l1 + b1, p, " + ".join(t), l1 * l1 + b1))
+        for b2 in range(2 * l2 + 1):
+            t = ["%s*(g[%d]*a[%d])" % (flit(K[c][b1][b2]), l3 * l3 + c, l1 * l1 + b1)
+                 for c in range(2 * l3 + 1) for b1 in range(2 * l1 + 1) if K[c][b1][b2] != 0]
+            if t:
+                o.append("      bbar[%d] = fmaf(w[%d], %s, bbar[%d]);" % (l2 * l2 + b2, p, " + ".join(t), l2 * l2 + b2))
+        o.append("    }")
+    o.append("  }")
+    o.append("};")
+    o.append("}  // namespace fc")
+    return "\n".join(o) + "\n"
+
+
+_main_conv = main
+
+
+def main():
+    written = _main_conv()
+    for L in (2, 3, 4):
+        path = os.path.join(OUTDIR, "fc_ladder_L%d.cuh" % L)
+        with open(path, "w") as f:
+            f.write(emit_ladder(L))
+        written.append(path)
+    return written
+
+
 if __name__ == "__main__":
     for p in main():
         print(p)

@@ -155,6 +155,51 @@ int fc_edge_conv_vjp(const fc_conv_desc *desc, int n_nodes, int n_edges,
                      const float *g, float *x_bar, float *w_bar, float *r_bar,
                      fc_stream_t stream);
 
+/* Product-ladder descriptor: ranks 0..lmax for every state (lmax in
+ * {2,3,4}), channels a multiple of 4, order >= 1 (order-1 products). */
+typedef struct {
+  int lmax;
+  int channels;
+  int order;
+} fc_ladder_desc;
+
+/* Number of paths P of the ladder products (all l1, l2, l3 <= lmax), or -1. */
+int fc_ladder_num_paths(const fc_ladder_desc *desc);
+
+/* Node-local correlation ladder, Sec. 5 Eq. (2) with path-reduced products
+ * (App. E) and a per-rank channel mix after every product:
+ *   B_v[n,l3,c,k]   = sum_{p = (l1,l2)->l3} path_w[v-1][p][k]
+ *                       f_p(A_v[n,l1,:,k], A_1[n,l2,:,k])_c
+ *   A_{v+1}[n,l,c,k] = sum_k' mix_w[v-1][l][k][k'] B_v[n,l,c,k']
+ *   z = A_1 + A_2 + ... + A_order          (v = 1 .. order-1)
+ * Products couple equal channels only (channel-diagonal, Sec. 5).
+ *   A1 [n_nodes][(lmax+1)^2 C] (node layout), path_w [order-1][P][C],
+ *   mix_w [order-1][lmax+1][C][C] (row = output channel),
+ *   states [order-1][n_nodes][(lmax+1)^2 C] receives A_2 .. A_order,
+ *   z [n_nodes][(lmax+1)^2 C].
+ * workspace: fc_product_ladder_workspace_size() bytes of device scratch
+ * (one product state), 16-byte aligned; FC_ERR_WORKSPACE if too small.
+ * order = 1 copies A1 to z and needs no workspace. */
+size_t fc_product_ladder_workspace_size(const fc_ladder_desc *desc, int n_nodes);
+int fc_product_ladder(const fc_ladder_desc *desc, int n_nodes, const float *A1,
+                      const float *path_w, const float *mix_w, float *states,
+                      float *z, void *workspace, size_t ws_bytes,
+                      fc_stream_t stream);
+
+/* VJP of fc_product_ladder by reverse accumulation through its steps:
+ * given gz (gradient of z, node layout) and the states of the forward call,
+ * writes A1_bar (node layout), path_w_bar [order-1][P][C] and mix_w_bar
+ * [order-1][lmax+1][C][C].  The weight gradients sum over all nodes with
+ * atomic additions (not bitwise reproducible).  workspace:
+ * fc_product_ladder_vjp_workspace_size() bytes (four product states). */
+size_t fc_product_ladder_vjp_workspace_size(const fc_ladder_desc *desc, int n_nodes);
+int fc_product_ladder_vjp(const fc_ladder_desc *desc, int n_nodes,
+                          const float *A1, const float *path_w,
+                          const float *mix_w, const float *states,
+                          const float *gz, float *A1_bar, float *path_w_bar,
+                          float *mix_w_bar, void *workspace, size_t ws_bytes,
+                          fc_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif
