@@ -462,3 +462,46 @@ int fc_product_ladder_vjp(const fc_ladder_desc* d, int n_nodes, const float* A1,
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// allocation-free variant of fc_product_ladder
+// ---------------------------------------------------------------------------
+// Some callers cannot allocate device memory: code that runs inside another
+// framework's memory pool, where the pool already holds nearly all of HBM
+// and a raw cudaMalloc fails or fragments it, and latency-critical loops,
+// where cudaMalloc may synchronise the device.  For them the scratch of one
+// product state lives in this fixed array, which every GPU that loads the
+// library keeps until the process exits.  Host code must not use the
+// array's name as a device address (it is a host-side stand-in); the device
+// address comes from cudaGetSymbolAddress, once per device.
+namespace fc {
+constexpr size_t kLadderStaticScratchBytes = 16u << 20;   // 16 MiB per GPU
+static __device__ __align__(256) float g_ladder_scratch[kLadderStaticScratchBytes / sizeof(float)];
+static void* g_ladder_scratch_addr[64] = {nullptr};
+
+// Device address of g_ladder_scratch on the current device (set-up on the
+// first call per device), or nullptr if the runtime call fails.
+static void* ladder_static_scratch() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  if (g_ladder_scratch_addr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_ladder_scratch) != cudaSuccess) return nullptr;
+    g_ladder_scratch_addr[dev] = p;
+  }
+  return g_ladder_scratch_addr[dev];
+}
+}  // namespace fc
+
+extern "C" int fc_product_ladder_noalloc(const fc_ladder_desc* d, int n_nodes, const float* A1,
+                                         const float* path_w, const float* mix_w, float* states,
+                                         float* z, fc_stream_t stream) {
+  int st = check_ladder_desc(d);
+  if (st != FC_OK) return st;
+  if (n_nodes < 0) return FC_ERR_ARG;
+  const size_t need = fc_product_ladder_workspace_size(d, n_nodes);
+  if (need > kLadderStaticScratchBytes) return FC_ERR_WORKSPACE;
+  void* ws = ladder_static_scratch();
+  if (ws == nullptr) return FC_ERR_CUDA;
+  return fc_product_ladder(d, n_nodes, A1, path_w, mix_w, states, z, ws, need, stream);
+}

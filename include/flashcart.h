@@ -200,6 +200,32 @@ int fc_product_ladder_vjp(const fc_ladder_desc *desc, int n_nodes,
                           float *mix_w_bar, void *workspace, size_t ws_bytes,
                           fc_stream_t stream);
 
+/* fc_product_ladder without a workspace argument and without allocating.
+ * No counterpart in the paper: it exists for callers that cannot allocate
+ * device memory -- code that runs inside another framework's memory pool
+ * (the pool already holds nearly all of HBM, so a raw cudaMalloc would
+ * fail or fragment it) and latency-critical loops (cudaMalloc may
+ * synchronise the device).  The caller still passes inputs and outputs
+ * exactly as for fc_product_ladder; the scratch of one product state is a
+ * fixed 16 MiB array inside the library, held by every GPU that loads the
+ * library until the process exits.
+ *   Limit: fc_product_ladder_workspace_size(desc, n_nodes) <= 16 MiB
+ *   (n_nodes * (lmax+1)^2 * channels * 4 bytes), else FC_ERR_WORKSPACE and
+ *   nothing is enqueued.
+ *   The first call on a device looks up the array's device address (a
+ *   runtime query, no allocation); make that first call before any stream
+ *   capture on that device.
+ *   Every call shares the one array, which keeps the last call's contents
+ *   (nothing in it needs to start at zero): calls that overlap on the GPU,
+ *   on different streams or in different host threads, race and must be
+ *   serialised by the caller.
+ * Returns the statuses of fc_product_ladder, or FC_ERR_CUDA if the
+ * address look-up fails. */
+int fc_product_ladder_noalloc(const fc_ladder_desc *desc, int n_nodes,
+                              const float *A1, const float *path_w,
+                              const float *mix_w, float *states, float *z,
+                              fc_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif
