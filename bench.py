@@ -63,6 +63,23 @@ def algorithmic_flops(E, C, L):
     return per * E * C
 
 
+# DRAM bytes (read + write) of one edge_conv_fwd_kernel<3, 128> launch on
+# this workload from an ncu capture (profiles/edge_conv_fwd_microbench_r3.md),
+# valid only while the kernel sources hash to the value it was taken with.
+FWD_TRAFFIC = {"sha1": "fd73249bad71fbdc90bf9ab89880fab481d8e1e1", "bytes": 1594546000 + 50859520}
+FWD_SOURCES = ("cartesian_tensor_products_b200/csrc/fc_edge_conv.cu",
+               "cartesian_tensor_products_b200/csrc/generated/fc_fwd_L3.cuh")
+
+
+def fwd_sources_sha1():
+    import hashlib
+    h = hashlib.sha1()
+    for rel in FWD_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
 def fp32_peak_tflops(sm_count, mhz):
     return sm_count * 128 * 2 * mhz * 1e6 / 1e12
 
@@ -145,6 +162,138 @@ def cpu_baseline(wl, n_recv):
             "sample": "first %d receivers of the workload (%d edges x %d channels), FP64 dense 3^l oracle" % (
                 n_recv, len(sel), C),
             "seconds": dt}
+
+
+def time_events(fn, steps, warmup, stream, flush=None):
+    """Mean device time (ms) of fn over `steps` calls, CUDA events on the
+    launching stream; optional L2 flush before every call (not timed)."""
+    import torch
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    times = []
+    for _ in range(steps):
+        if flush is not None:
+            flush()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        fn()
+        b.record(stream)
+        b.synchronize()
+        times.append(a.elapsed_time(b))
+    return statistics.mean(times), min(times)
+
+
+def extra_rows(fc, W, dev, stream, peaks, fp32_peak, steps):
+    """Timed rows of the other hot-path steps (edge-conv VJP, rank 4, ladder)."""
+    import torch
+    rows = {}
+    flush_buf = torch.empty(64 * 1024 * 1024, dtype=torch.float32, device=dev)  # 256 MB > L2
+
+    def flush():
+        flush_buf.zero_()
+
+    # --- edge-conv VJP, rank 3, microbench graph
+    wl = W.microbench_grad(lmax=3)
+    L, C, N = 3, 128, wl["n_nodes"]
+    E = wl["edge_index"].shape[1]
+    P = fc.num_paths(L)
+    ei = torch.from_numpy(wl["edge_index"]).to(dev)
+    ev = torch.from_numpy(wl["edge_vec"]).to(dev)
+    x = torch.from_numpy(wl["x"]).to(dev)
+    w = torch.from_numpy(wl["w"]).to(dev)
+    g = torch.from_numpy(wl["g"]).to(dev)
+    rp = fc.build_rowptr(ei, ev, N)
+    out = {"x": torch.empty_like(x), "w": torch.empty_like(w),
+           "r": torch.empty((E, 3), device=dev)}
+    ms, mn = time_events(lambda: fc.edge_conv_vjp(L, rp, ei, ev, x, w, g, out=out),
+                         steps, 3, stream)
+    zr = fc.out_row(L)
+    byt = 4 * (2 * E * P * C + N * zr * C + 2 * N * 16 * C + 3 * E + 3 * E + E + N)
+    rows["edge_conv_vjp_r3"] = {
+        "workload": "microbench graph, rank 3, x_bar + w_bar + r_bar",
+        "ms": ms, "ms_min": mn, "edge_channels_per_s": E * C / (ms * 1e-3),
+        "roofline": {"bound": "hbm", "achieved": byt / (ms * 1e-3) / 1e9,
+                     "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": byt / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                     "algorithmic_bytes": byt}}
+    del out, w, g, x
+    torch.cuda.empty_cache()
+
+    # --- rank 4 on the microbench graph, forward and VJP
+    wl4 = W.microbench(lmax=4, weight_seed=32)
+    L4 = 4
+    P4 = fc.num_paths(L4)
+    x4 = torch.from_numpy(wl4["x"]).to(dev)
+    w4 = torch.from_numpy(wl4["w"]).to(dev)
+    z4 = torch.empty((N, fc.out_row(L4) * C), device=dev)
+    ms4, mn4 = time_events(lambda: fc.edge_conv(L4, rp, ei, ev, x4, w4, out=z4), steps, 3, stream)
+    byt4 = 4 * (E * P4 * C + N * 25 * C + N * fc.out_row(L4) * C + 4 * E + N)
+    fl4 = algorithmic_flops(E, C, 4)
+    rows["edge_conv_fwd_r4"] = {
+        "workload": "microbench graph, rank 4 (42 paths), forward",
+        "ms": ms4, "ms_min": mn4, "edge_channels_per_s": E * C / (ms4 * 1e-3),
+        "roofline": {"bound": "hbm", "achieved": byt4 / (ms4 * 1e-3) / 1e9,
+                     "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": byt4 / (ms4 * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                     "algorithmic_bytes": byt4,
+                     "fp32_frac": fl4 / (ms4 * 1e-3) / 1e12 / fp32_peak}}
+    g4 = torch.randn((N, fc.out_row(L4) * C), device=dev)
+    out4 = {"x": torch.empty_like(x4), "w": torch.empty_like(w4),
+            "r": torch.empty((E, 3), device=dev)}
+    ms4b, mn4b = time_events(lambda: fc.edge_conv_vjp(L4, rp, ei, ev, x4, w4, g4, out=out4),
+                             steps, 3, stream)
+    byt4b = 4 * (2 * E * P4 * C + N * fc.out_row(L4) * C + 2 * N * 25 * C + 7 * E + N)
+    rows["edge_conv_vjp_r4"] = {
+        "workload": "microbench graph, rank 4, x_bar + w_bar + r_bar",
+        "ms": ms4b, "ms_min": mn4b, "edge_channels_per_s": E * C / (ms4b * 1e-3),
+        "roofline": {"bound": "hbm", "achieved": byt4b / (ms4b * 1e-3) / 1e9,
+                     "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": byt4b / (ms4b * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                     "algorithmic_bytes": byt4b}}
+    del x4, w4, z4, g4, out4
+    torch.cuda.empty_cache()
+
+    # --- ladder, 4096 nodes x 128 channels, rank 3, order 4
+    lad = W.ladder()
+    Ll, Cl, order, Nl = lad["lmax"], lad["channels"], lad["order"], lad["n_nodes"]
+    A1 = torch.from_numpy(lad["A1"]).to(dev)
+    pw = torch.from_numpy(lad["path_w"]).to(dev)
+    mw = torch.from_numpy(lad["mix_w"]).to(dev)
+    gz = torch.from_numpy(lad["gz"]).to(dev)
+    ws = torch.empty(4 * Nl * 16 * Cl, device=dev)
+    res = {}
+
+    def lad_fwd():
+        res["s"], res["z"] = fc.product_ladder(Ll, order, A1, pw, mw, workspace=ws)
+    msl, mnl = time_events(lad_fwd, steps, 3, stream, flush=flush)
+    states = res["s"]
+
+    def lad_vjp():
+        fc.product_ladder_vjp(Ll, order, A1, pw, mw, states, gz, workspace=ws)
+    mslb, mnlb = time_events(lad_vjp, steps, 3, stream, flush=flush)
+    S = order - 1
+    mix_flops = S * 2 * Nl * 16 * Cl * Cl
+    tp_flops = S * Nl * Cl * 2 * 751
+    rows["ladder_fwd"] = {
+        "workload": "4096 nodes x 128 channels, rank 3, order 4 (3 products + 3 per-rank 128x128 mixes)",
+        "ms": msl, "ms_min": mnl,
+        "roofline": {"bound": "alu", "achieved": (mix_flops + tp_flops) / (msl * 1e-3) / 1e12,
+                     "peak": fp32_peak, "unit": "TFLOP/s",
+                     "frac": (mix_flops + tp_flops) / (msl * 1e-3) / 1e12 / fp32_peak,
+                     "algorithmic_flops": mix_flops + tp_flops},
+        "l2_flush": "256 MB written before every call"}
+    vjp_flops = 3 * mix_flops + 4 * tp_flops
+    rows["ladder_vjp"] = {
+        "workload": "same ladder, A1_bar + path_w_bar + mix_w_bar",
+        "ms": mslb, "ms_min": mnlb,
+        "roofline": {"bound": "alu", "achieved": vjp_flops / (mslb * 1e-3) / 1e12,
+                     "peak": fp32_peak, "unit": "TFLOP/s",
+                     "frac": vjp_flops / (mslb * 1e-3) / 1e12 / fp32_peak,
+                     "algorithmic_flops": vjp_flops},
+        "l2_flush": "256 MB written before every call"}
+    return rows
 
 
 def run_reference(args):
@@ -257,7 +406,8 @@ def run_ours(args):
     fp32_peak = fp32_peak_tflops(sm_count, peaks.get("sm_max_mhz", 1965.0))
     roof = {"bound": "hbm", "achieved": achieved_gbs, "peak": peaks["hbm_gbs"],
             "unit": "GB/s", "frac": achieved_gbs / peaks["hbm_gbs"],
-            "traffic": None, "peak_source": peak_kind + " (MEASURED_PEAKS.json hbm_gbs)",
+            "traffic": FWD_TRAFFIC["bytes"] if fwd_sources_sha1() == FWD_TRAFFIC["sha1"] else None,
+            "peak_source": peak_kind + " (MEASURED_PEAKS.json hbm_gbs)",
             "algorithmic_bytes": abytes,
             "fp32": {"achieved_tflops": flops / (kern_ms * 1e-3) / 1e12,
                      "peak_tflops": fp32_peak,
@@ -311,6 +461,10 @@ def run_ours(args):
                "steps": n_e2e, "ms_per_step": e_ms / n_e2e,
                "includes": "H2D of x, w, edge_index, edge_vec; fc_build_rowptr (validates, syncs); fc_edge_conv; D2H of z"}
 
+    rows = None
+    if rank == 0 and not args.no_rows:
+        rows = extra_rows(fc, W, dev, stream, peaks, fp32_peak, max(3, min(args.steps, 10)))
+
     line = None
     if rank == 0:
         cb = None
@@ -327,7 +481,7 @@ def run_ours(args):
                            "l2_flush": "none: the 1.54 GB weight stream exceeds the 126 MB L2",
                            "per_rank": "each rank runs its own copy (weak scaling)"},
                 "roofline": roof, "cpu_baseline": cb, "e2e": e2e,
-                "gpu_launches": args.steps, "clocks": clocks,
+                "gpu_launches": args.steps, "clocks": clocks, "rows": rows,
                 "kernel_ms": {"mean": kern_ms, "min": min(per), "max": max(per)}}
         print(json.dumps(line), flush=True)
     if world > 1:
