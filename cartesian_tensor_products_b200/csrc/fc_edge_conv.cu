@@ -73,10 +73,9 @@ __device__ __forceinline__ void issue_edge(const ConvArgs& a, int C, float* st, 
 // CC > 0: the channel count is the compile-time constant CC (every row
 // offset becomes an immediate); CC == 0: runtime a.C.
 template <class Grp, int S, int MW, int CC>
-__device__ __forceinline__ void fwd_warp(const ConvArgs& a, float* smem, int lane) {
+__device__ __forceinline__ void fwd_warp(const ConvArgs& a, float* smem, int lane, int unit) {
   constexpr int STAGE = Grp::NROW * 128;  // floats per stage (all lanes)
   const int C = CC > 0 ? CC : a.C;
-  const int unit = blockIdx.x;
   const int u = CC == 128 ? unit : unit / a.ntiles;
   const int tile = unit - u * (CC == 128 ? 1 : a.ntiles);
   const int k0 = tile * 128 + lane * 4;
@@ -142,24 +141,37 @@ __device__ __forceinline__ void fwd_warp(const ConvArgs& a, float* smem, int lan
 }
 
 template <int L, int CC, int g>
-__device__ __forceinline__ void dispatch_fwd(int warp, const ConvArgs& a, float* smem,
-                                             int lane) {
+__device__ __forceinline__ void dispatch_fwd(int grp, const ConvArgs& a, float* smem, int lane,
+                                             int unit) {
   if constexpr (g < FwdMeta<L>::G) {
     using Grp = FwdGroup<L, FwdMeta<L>::G, g>;
-    if (warp == g) {
-      fwd_warp<Grp, FwdMeta<L>::S, FwdMeta<L>::MWIN, CC>(a, smem, lane);
+    if (grp == g) {
+      fwd_warp<Grp, FwdMeta<L>::S, FwdMeta<L>::MWIN, CC>(a, smem, lane, unit);
       return;
     }
-    dispatch_fwd<L, CC, g + 1>(warp, a, smem, lane);
+    dispatch_fwd<L, CC, g + 1>(grp, a, smem, lane, unit);
   }
 }
 
+// Up to 4 groups: a CTA is the G groups of one receiver tile (warp g runs
+// group g, one warp per SMSP).  More groups: a CTA is one group for WARPS
+// consecutive receiver tiles, blocks ordered group-major, so an SMSP still
+// mostly runs one instruction stream.
 template <int L, int CC>
-__global__ void __launch_bounds__(FwdMeta<L>::G * 32, (FwdMeta<L>::G <= 4 ? 2 : 1))
-    edge_conv_fwd_kernel(const ConvArgs a) {
+__global__ void __launch_bounds__(FwdMeta<L>::WARPS * 32, 2) edge_conv_fwd_kernel(const ConvArgs a) {
   extern __shared__ __align__(16) float smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  dispatch_fwd<L, CC, 0>(warp, a, smem, lane);
+  if constexpr (!FwdMeta<L>::GROUP_MAJOR) {
+    dispatch_fwd<L, CC, 0>(warp, a, smem, lane, blockIdx.x);
+  } else {
+    constexpr int WARPS = FwdMeta<L>::WARPS;
+    const int units = a.n_nodes * a.ntiles;
+    const int nb = (units + WARPS - 1) / WARPS;
+    const int grp = blockIdx.x / nb;
+    const int unit = (blockIdx.x - grp * nb) * WARPS + warp;
+    if (unit >= units) return;
+    dispatch_fwd<L, CC, 0>(grp, a, smem + warp * FwdMeta<L>::WARP_FLOATS, lane, unit);
+  }
 }
 
 template <int L, int CC>
@@ -177,7 +189,11 @@ static int launch_fwd_cc(const ConvArgs& a, cudaStream_t s) {
     configured[dev] = 1;
   }
   const long long units = (long long)a.n_nodes * a.ntiles;
-  edge_conv_fwd_kernel<L, CC><<<(unsigned)units, FwdMeta<L>::G * 32, smem, s>>>(a);
+  constexpr int WARPS = FwdMeta<L>::WARPS;
+  const long long blocks =
+      FwdMeta<L>::GROUP_MAJOR ? (units + WARPS - 1) / WARPS * FwdMeta<L>::G : units;
+  if (blocks > 0x7fffffffLL) return FC_ERR_ARG;
+  edge_conv_fwd_kernel<L, CC><<<(unsigned)blocks, WARPS * 32, smem, s>>>(a);
   return cudaGetLastError() == cudaSuccess ? FC_OK : FC_ERR_CUDA;
 }
 

@@ -10,9 +10,12 @@
 // last paragraph of "Symbolic derivatives"):
 //   r_bar = (I - u u^T)/|r| (dT/du)^T y_bar,   u = r/|r|.
 //
-// B200 design.  One CTA per (receiver, 128-channel tile); its G warps each
-// own whole paths (h = M^T g needs every row of a path) and hold the
-// receiver's g rows of those paths in registers for all its edges.  Sender
+// B200 design.  Output paths are cut offline into G groups of whole paths
+// (h = M^T g needs every row of a path).  A CTA is (group, 4 consecutive
+// receiver tiles): its 4 warps run the same code, one receiver each, and
+// hold the receiver's g rows of the group's paths in registers for all its
+// edges; blocks are ordered group-major so an SMSP mostly runs one
+// instruction stream.  Sender
 // rows and edge weights are streamed through a per-warp cp.async ring as
 // in the forward kernel; M and dT/du are formed lane-per-edge into a
 // warp-private window.  Per edge a lane computes, for its 4 channels,
@@ -75,11 +78,10 @@ __device__ __forceinline__ void vissue_edge(const VjpArgs& a, int C, float* st, 
 }
 
 template <class Grp, int S, int MW, int CC>
-__device__ __forceinline__ void vjp_warp(const VjpArgs& a, float* smem, int lane) {
+__device__ __forceinline__ void vjp_warp(const VjpArgs& a, float* smem, int lane, int unit) {
   constexpr int STAGE = Grp::NROW * 128;
   constexpr int NYB = Grp::NYD > 0 ? Grp::NYD : 1;
   const int C = CC > 0 ? CC : a.C;
-  const int unit = blockIdx.x;
   const int u = CC == 128 ? unit : unit / a.ntiles;
   const int tile = unit - u * (CC == 128 ? 1 : a.ntiles);
   const int k0 = tile * 128 + lane * 4;
@@ -189,23 +191,32 @@ __device__ __forceinline__ void vjp_warp(const VjpArgs& a, float* smem, int lane
 }
 
 template <int L, int CC, int g>
-__device__ __forceinline__ void dispatch_vjp(int warp, const VjpArgs& a, float* smem, int lane) {
+__device__ __forceinline__ void dispatch_vjp(int grp, const VjpArgs& a, float* smem, int lane,
+                                             int unit) {
   if constexpr (g < VjpMeta<L>::G) {
     using Grp = VjpGroup<L, VjpMeta<L>::G, g>;
-    if (warp == g) {
-      vjp_warp<Grp, VjpMeta<L>::S, VjpMeta<L>::MWIN, CC>(a, smem, lane);
+    if (grp == g) {
+      vjp_warp<Grp, VjpMeta<L>::S, VjpMeta<L>::MWIN, CC>(a, smem, lane, unit);
       return;
     }
-    dispatch_vjp<L, CC, g + 1>(warp, a, smem, lane);
+    dispatch_vjp<L, CC, g + 1>(grp, a, smem, lane, unit);
   }
 }
 
+// CTA = (path group, WARPS consecutive receiver units): every warp of a CTA
+// runs the same code, and blocks are ordered group-major, so an SMSP mostly
+// executes one instruction stream.
 template <int L, int CC>
-__global__ void __launch_bounds__(VjpMeta<L>::G * 32, (VjpMeta<L>::G <= 4 ? 2 : 1))
-    edge_conv_vjp_kernel(const VjpArgs a) {
+__global__ void __launch_bounds__(VjpMeta<L>::WARPS * 32, 2) edge_conv_vjp_kernel(const VjpArgs a) {
   extern __shared__ __align__(16) float smem[];
+  constexpr int WARPS = VjpMeta<L>::WARPS;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  dispatch_vjp<L, CC, 0>(warp, a, smem, lane);
+  const int units = a.n_nodes * a.ntiles;
+  const int nb = (units + WARPS - 1) / WARPS;
+  const int grp = blockIdx.x / nb;
+  const int unit = (blockIdx.x - grp * nb) * WARPS + warp;
+  if (unit >= units) return;
+  dispatch_vjp<L, CC, 0>(grp, a, smem + warp * VjpMeta<L>::WARP_FLOATS, lane, unit);
 }
 
 template <int L, int CC>
@@ -223,7 +234,10 @@ static int launch_vjp_cc(const VjpArgs& a, cudaStream_t s) {
     configured[dev] = 1;
   }
   const long long units = (long long)a.n_nodes * a.ntiles;
-  edge_conv_vjp_kernel<L, CC><<<(unsigned)units, VjpMeta<L>::G * 32, smem, s>>>(a);
+  constexpr int WARPS = VjpMeta<L>::WARPS;
+  const long long blocks = (units + WARPS - 1) / WARPS * VjpMeta<L>::G;
+  if (blocks > 0x7fffffffLL) return FC_ERR_ARG;
+  edge_conv_vjp_kernel<L, CC><<<(unsigned)blocks, WARPS * 32, smem, s>>>(a);
   return cudaGetLastError() == cudaSuccess ? FC_OK : FC_ERR_CUDA;
 }
 

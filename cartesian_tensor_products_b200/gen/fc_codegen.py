@@ -352,6 +352,7 @@ NGROUPS = {2: 4, 3: 4, 4: 8}
 ROW_WEIGHT = {2: 0.0, 3: 0.0, 4: 4.0}
 STAGES = {2: 3, 3: 3, 4: 2}
 MWIN = 16
+FWD_WARPS = 2
 
 
 def emit_fwd(L, G):
@@ -374,15 +375,30 @@ def emit_fwd(L, G):
     out.append("  static constexpr int MAXROW = %d;      // largest staged rows per edge of a group" % max(c.NROW for c in codes))
     out.append("  static constexpr int P = %d;           // paths" % T.P)
     out.append("  static constexpr int ZROW = %d;        // output components per channel" % T.zrow)
-    off = 0
-    for c in codes:
-        c.ring_off = off
-        off += STAGES[L] * 128 * c.NROW
-    for c in codes:
-        c.mwin_off = off
-        off += MWIN * c.MSTRIDE
+    if G <= 4:
+        # one CTA = the G groups of one receiver (one warp per SMSP)
+        off = 0
+        for c in codes:
+            c.ring_off = off
+            off += STAGES[L] * 128 * c.NROW
+        for c in codes:
+            c.mwin_off = off
+            off += MWIN * c.MSTRIDE
+        warp_floats, warps, total = 0, G, off
+    else:
+        # one CTA = one group for FWD_WARPS receivers (group-major blocks)
+        nrow = max(c.NROW for c in codes)
+        mstride = max(c.MSTRIDE for c in codes)
+        for c in codes:
+            c.ring_off = 0
+            c.mwin_off = STAGES[L] * 128 * nrow
+        warp_floats = STAGES[L] * 128 * nrow + MWIN * mstride
+        warps, total = FWD_WARPS, FWD_WARPS * warp_floats
     out.append("  static constexpr int MWIN = %d;        // edges per M window" % MWIN)
-    out.append("  static constexpr int SMEM_FLOATS = %d; // staging rings + M windows of all warps" % off)
+    out.append("  static constexpr bool GROUP_MAJOR = %s;" % ("true" if G > 4 else "false"))
+    out.append("  static constexpr int WARPS = %d;       // warps per CTA" % warps)
+    out.append("  static constexpr int WARP_FLOATS = %d; // shared memory of one warp (group-major)" % warp_floats)
+    out.append("  static constexpr int SMEM_FLOATS = %d; // shared memory of a CTA" % total)
     out.append("};")
     for c in codes:
         out.append(c.emit(L, G))
@@ -634,13 +650,14 @@ def emit_vjp(L, G):
     T = Tables(L)
     groups = partition_paths(T, G, lambda p: vjp_path_cost(T, p))
     codes = [VjpGroupCode(T, ps, g) for g, ps in enumerate(groups)]
-    off = 0
+    # every warp of a CTA runs the same group (one instruction stream per
+    # SMSP), so all groups share one per-warp layout: ring, then M window
+    nrow = max(c.NROW for c in codes)
+    mstride = max(c.MSTRIDE for c in codes)
     for c in codes:
-        c.ring_off = off
-        off += VJP_STAGES[L] * 128 * c.NROW
-    for c in codes:
-        c.mwin_off = off
-        off += VJP_MWIN[L] * c.MSTRIDE
+        c.ring_off = 0
+        c.mwin_off = VJP_STAGES[L] * 128 * nrow
+    off = VJP_STAGES[L] * 128 * nrow + VJP_MWIN[L] * mstride
     out = ["// Generated by gen/fc_codegen.py -- do not edit.",
            "// Receiver-sorted VJP, rank %d: %d paths, %d warp groups (whole paths)." % (L, T.P, G)]
     for c in codes:
@@ -653,7 +670,9 @@ def emit_vjp(L, G):
             "  static constexpr int S = %d;" % VJP_STAGES[L],
             "  static constexpr int MWIN = %d;" % VJP_MWIN[L],
             "  static constexpr int P = %d;" % T.P,
-            "  static constexpr int SMEM_FLOATS = %d;" % off,
+            "  static constexpr int WARP_FLOATS = %d;   // shared memory of one warp" % off,
+            "  static constexpr int WARPS = 4;           // receivers per CTA (same group)",
+            "  static constexpr int SMEM_FLOATS = %d;" % (4 * off),
             "};"]
     for c in codes:
         out.append(c.emit(L, G))
