@@ -28,7 +28,39 @@ int check_conv_desc(const fc_conv_desc* d) {
   if (d->lmax_in != d->lmax_edge || d->lmax_in != d->lmax_out) return FC_ERR_UNSUPPORTED_RANK;
   if (d->lmax_in < 2 || d->lmax_in > 4) return FC_ERR_UNSUPPORTED_RANK;
   if (d->channels % 4) return FC_ERR_ALIGN;
+  if (d->envelope != 0 && d->envelope != 1) return FC_ERR_ARG;
+  if (d->envelope == 1 && !(d->r_cut > 0.0f && isfinite(d->r_cut) && isfinite(d->edge_scale)))
+    return FC_ERR_ARG;
   return FC_OK;
+}
+
+// E = sum of the rank-0 block; gz = indicator of the rank-0 block
+__global__ void readout_kernel(long long total, int NYC, int C, const float* __restrict__ z,
+                               float* __restrict__ energy, float* __restrict__ gz) {
+  float part = 0.0f;
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < total;
+       i += (long long)gridDim.x * blockDim.x) {
+    const bool r0 = (i % NYC) < C;
+    if (r0) part += z[i];
+    if (gz) gz[i] = r0 ? 1.0f : 0.0f;
+  }
+  for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+  if ((threadIdx.x & 31) == 0) atomicAdd(energy, part);
+}
+
+__global__ void forces_kernel(int N, int E, const int32_t* __restrict__ recv,
+                              const int32_t* __restrict__ send, const float* __restrict__ rbar,
+                              float* __restrict__ F) {
+  const int e = blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= E) return;
+  const int u = recv[e], v = send[e];
+  const float x = rbar[3 * e], y = rbar[3 * e + 1], zz = rbar[3 * e + 2];
+  if (v >= 0 && v < N) {
+    atomicAdd(F + 3 * v, -x); atomicAdd(F + 3 * v + 1, -y); atomicAdd(F + 3 * v + 2, -zz);
+  }
+  if (u >= 0 && u < N) {
+    atomicAdd(F + 3 * u, x); atomicAdd(F + 3 * u + 1, y); atomicAdd(F + 3 * u + 2, zz);
+  }
 }
 
 // Flags raised by the validation kernel.
@@ -110,6 +142,37 @@ int fc_conv_path(const fc_conv_desc* d, int p, int* l1, int* l2, int* l3) {
           ++n;
         }
   return FC_ERR_ARG;
+}
+
+int fc_scalar_readout(int n_nodes, int lmax, int channels, const float* z, float* energy,
+                      float* gz, fc_stream_t stream) {
+  if (n_nodes < 0 || lmax < 0 || lmax > 8 || channels <= 0 || !energy) return FC_ERR_ARG;
+  if (n_nodes > 0 && !z) return FC_ERR_ARG;
+  if (!aligned4(energy) || (z && !aligned4(z)) || (gz && !aligned4(gz))) return FC_ERR_ALIGN;
+  cudaStream_t s = (cudaStream_t)stream;
+  if (cudaMemsetAsync(energy, 0, sizeof(float), s) != cudaSuccess) return FC_ERR_CUDA;
+  if (n_nodes == 0) return FC_OK;
+  const int NYC = (lmax + 1) * (lmax + 1) * channels;
+  const long long total = (long long)n_nodes * NYC;
+  long long blocks = (total + 255) / 256;
+  if (blocks > 4 * 148) blocks = 4 * 148;
+  readout_kernel<<<(int)blocks, 256, 0, s>>>(total, NYC, channels, z, energy, gz);
+  return cudaGetLastError() == cudaSuccess ? FC_OK : FC_ERR_CUDA;
+}
+
+int fc_edge_forces(int n_nodes, int n_edges, const int32_t* edge_index, const float* r_bar,
+                   float* forces, fc_stream_t stream) {
+  if (n_nodes < 0 || n_edges < 0 || !forces) return FC_ERR_ARG;
+  if (n_edges > 0 && (!edge_index || !r_bar)) return FC_ERR_ARG;
+  if (!aligned4(forces) || (r_bar && !aligned4(r_bar)) || (edge_index && !aligned4(edge_index)))
+    return FC_ERR_ALIGN;
+  cudaStream_t s = (cudaStream_t)stream;
+  if (n_nodes > 0 && cudaMemsetAsync(forces, 0, sizeof(float) * 3 * (size_t)n_nodes, s) != cudaSuccess)
+    return FC_ERR_CUDA;
+  if (n_edges == 0) return FC_OK;
+  forces_kernel<<<(n_edges + 255) / 256, 256, 0, s>>>(n_nodes, n_edges, edge_index,
+                                                       edge_index + n_edges, r_bar, forces);
+  return cudaGetLastError() == cudaSuccess ? FC_OK : FC_ERR_CUDA;
 }
 
 int fc_build_rowptr(int n_nodes, int n_edges, const int32_t* edge_index,

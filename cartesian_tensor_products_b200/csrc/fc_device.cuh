@@ -67,6 +67,27 @@ __device__ __forceinline__ void red_add4(float* p, float4 v) {
   atomicAdd(reinterpret_cast<float4*>(p), v);
 }
 
+// ---- radial envelope of an edge of length r: s(r) and ds/dr --------------
+// env = 1: s = scale (cos(pi r / rc) + 1) / 2 for r < rc, 0 beyond;
+// env = 0: s = 1.
+__device__ __forceinline__ void edge_envelope(int env, float r, float rc, float scale, float& s,
+                                              float& sp) {
+  if (!env) {
+    s = 1.0f;
+    sp = 0.0f;
+    return;
+  }
+  if (!(r < rc)) {
+    s = 0.0f;
+    sp = 0.0f;
+    return;
+  }
+  float sn, cs;
+  sincospif(r / rc, &sn, &cs);
+  s = 0.5f * scale * (cs + 1.0f);
+  sp = -0.5f * scale * (3.14159265358979f / rc) * sn;
+}
+
 // ---- asynchronous global -> shared copies (one 16-byte slice per lane) --
 // ok == false writes 16 zero bytes and reads nothing from src.
 __device__ __forceinline__ void cp_async16(float* dst_smem, const float* src, bool ok) {

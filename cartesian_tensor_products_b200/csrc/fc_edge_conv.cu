@@ -36,6 +36,8 @@ struct ConvArgs {
   const float* w;
   float* z;
   int n_nodes, n_edges, C, ntiles, xrow, zrow, P, sum_paths;
+  int envelope;
+  float r_cut, edge_scale;
 };
 
 // sender and edge vector of edge `e` for this lane's window slot
@@ -72,7 +74,7 @@ __device__ __forceinline__ void issue_edge(const ConvArgs& a, int C, float* st, 
 
 // CC > 0: the channel count is the compile-time constant CC (every row
 // offset becomes an immediate); CC == 0: runtime a.C.
-template <class Grp, int S, int MW, int CC>
+template <class Grp, int S, int MW, int CC, bool ENV>
 __device__ __forceinline__ void fwd_warp(const ConvArgs& a, float* smem, int lane, int unit) {
   constexpr int STAGE = Grp::NROW * 128;  // floats per stage (all lanes)
   const int C = CC > 0 ? CC : a.C;
@@ -116,14 +118,17 @@ __device__ __forceinline__ void fwd_warp(const ConvArgs& a, float* smem, int lan
       const float rz = __shfl_sync(0xffffffffu, cur.rz, src);
       __syncwarp();
       if (lane < MW && q + lane < e1) {
-        const float inv = 1.0f / sqrtf(rx * rx + ry * ry + rz * rz);
-        Grp::make_m(rx * inv, ry * inv, rz * inv, mwin + lane * Grp::MSTRIDE);
+        const float r = sqrtf(rx * rx + ry * ry + rz * rz);
+        const float inv = 1.0f / r;
+        float es, esp;
+        edge_envelope(a.envelope, r, a.r_cut, a.edge_scale, es, esp);
+        Grp::make_m(rx * inv, ry * inv, rz * inv, es, mwin + lane * Grp::MSTRIDE);
       }
       __syncwarp();
     }
     const int slot = p % S;
     cp_async_wait<S - 1>();
-    Grp::accum(acc, st + slot * STAGE, mwin + (p % MW) * Grp::MSTRIDE);
+    Grp::template accum<ENV>(acc, st + slot * STAGE, mwin + (p % MW) * Grp::MSTRIDE);
     // refill this slot with edge q + S
     const int pn = p + S;
     if (q + S < e1) {
@@ -140,16 +145,16 @@ __device__ __forceinline__ void fwd_warp(const ConvArgs& a, float* smem, int lan
   if (act) Grp::store(a.z + (size_t)u * a.zrow * C + k0, C, a.sum_paths, acc);
 }
 
-template <int L, int CC, int g>
+template <int L, int CC, bool ENV, int g>
 __device__ __forceinline__ void dispatch_fwd(int grp, const ConvArgs& a, float* smem, int lane,
                                              int unit) {
   if constexpr (g < FwdMeta<L>::G) {
     using Grp = FwdGroup<L, FwdMeta<L>::G, g>;
     if (grp == g) {
-      fwd_warp<Grp, FwdMeta<L>::S, FwdMeta<L>::MWIN, CC>(a, smem, lane, unit);
+      fwd_warp<Grp, FwdMeta<L>::S, FwdMeta<L>::MWIN, CC, ENV>(a, smem, lane, unit);
       return;
     }
-    dispatch_fwd<L, CC, g + 1>(grp, a, smem, lane, unit);
+    dispatch_fwd<L, CC, ENV, g + 1>(grp, a, smem, lane, unit);
   }
 }
 
@@ -157,12 +162,12 @@ __device__ __forceinline__ void dispatch_fwd(int grp, const ConvArgs& a, float* 
 // group g, one warp per SMSP).  More groups: a CTA is one group for WARPS
 // consecutive receiver tiles, blocks ordered group-major, so an SMSP still
 // mostly runs one instruction stream.
-template <int L, int CC>
+template <int L, int CC, bool ENV>
 __global__ void __launch_bounds__(FwdMeta<L>::WARPS * 32, 2) edge_conv_fwd_kernel(const ConvArgs a) {
   extern __shared__ __align__(16) float smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if constexpr (!FwdMeta<L>::GROUP_MAJOR) {
-    dispatch_fwd<L, CC, 0>(warp, a, smem, lane, blockIdx.x);
+    dispatch_fwd<L, CC, ENV, 0>(warp, a, smem, lane, blockIdx.x);
   } else {
     constexpr int WARPS = FwdMeta<L>::WARPS;
     const int units = a.n_nodes * a.ntiles;
@@ -170,11 +175,11 @@ __global__ void __launch_bounds__(FwdMeta<L>::WARPS * 32, 2) edge_conv_fwd_kerne
     const int grp = blockIdx.x / nb;
     const int unit = (blockIdx.x - grp * nb) * WARPS + warp;
     if (unit >= units) return;
-    dispatch_fwd<L, CC, 0>(grp, a, smem + warp * FwdMeta<L>::WARP_FLOATS, lane, unit);
+    dispatch_fwd<L, CC, ENV, 0>(grp, a, smem + warp * FwdMeta<L>::WARP_FLOATS, lane, unit);
   }
 }
 
-template <int L, int CC>
+template <int L, int CC, bool ENV>
 static int launch_fwd_cc(const ConvArgs& a, cudaStream_t s) {
   static_assert(sizeof(float) * FwdMeta<L>::SMEM_FLOATS <= 227 * 1024,
                 "forward kernel shared memory exceeds the 227 KB per-CTA limit of sm_100");
@@ -183,7 +188,7 @@ static int launch_fwd_cc(const ConvArgs& a, cudaStream_t s) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return FC_ERR_CUDA;
   if (!configured[dev]) {
-    if (cudaFuncSetAttribute(edge_conv_fwd_kernel<L, CC>,
+    if (cudaFuncSetAttribute(edge_conv_fwd_kernel<L, CC, ENV>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
       return FC_ERR_CUDA;
     configured[dev] = 1;
@@ -193,13 +198,14 @@ static int launch_fwd_cc(const ConvArgs& a, cudaStream_t s) {
   const long long blocks =
       FwdMeta<L>::GROUP_MAJOR ? (units + WARPS - 1) / WARPS * FwdMeta<L>::G : units;
   if (blocks > 0x7fffffffLL) return FC_ERR_ARG;
-  edge_conv_fwd_kernel<L, CC><<<(unsigned)blocks, WARPS * 32, smem, s>>>(a);
+  edge_conv_fwd_kernel<L, CC, ENV><<<(unsigned)blocks, WARPS * 32, smem, s>>>(a);
   return cudaGetLastError() == cudaSuccess ? FC_OK : FC_ERR_CUDA;
 }
 
 template <int L>
 static int launch_fwd(const ConvArgs& a, cudaStream_t s) {
-  return a.C == 128 ? launch_fwd_cc<L, 128>(a, s) : launch_fwd_cc<L, 0>(a, s);
+  if (a.envelope) return a.C == 128 ? launch_fwd_cc<L, 128, true>(a, s) : launch_fwd_cc<L, 0, true>(a, s);
+  return a.C == 128 ? launch_fwd_cc<L, 128, false>(a, s) : launch_fwd_cc<L, 0, false>(a, s);
 }
 
 }  // namespace fc
@@ -236,6 +242,9 @@ extern "C" int fc_edge_conv(const fc_conv_desc* d, int n_nodes, int n_edges,
   a.zrow = out_row(L, d->sum_paths);
   a.P = num_paths(L);
   a.sum_paths = d->sum_paths;
+  a.envelope = d->envelope;
+  a.r_cut = d->r_cut;
+  a.edge_scale = d->edge_scale;
   if ((long long)n_nodes * a.ntiles > 0x7fffffffLL) return FC_ERR_ARG;
   cudaStream_t s = (cudaStream_t)stream;
   if (d->sum_paths) {

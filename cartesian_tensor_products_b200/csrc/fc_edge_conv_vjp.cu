@@ -44,6 +44,8 @@ struct VjpArgs {
   float* wbar;
   float* rbar;
   int n_nodes, n_edges, C, ntiles, xrow, zrow, P, sum_paths;
+  int envelope;
+  float r_cut, edge_scale;
 };
 
 struct VEdgeWin {
@@ -132,8 +134,11 @@ __device__ __forceinline__ void vjp_warp(const VjpArgs& a, float* smem, int lane
       const float rz = __shfl_sync(0xffffffffu, cur.rz, src);
       __syncwarp();
       if (lane < MW && q + lane < e1) {
-        const float inv = 1.0f / sqrtf(rx * rx + ry * ry + rz * rz);
-        Grp::make_row(rx * inv, ry * inv, rz * inv, mwin + lane * Grp::MSTRIDE);
+        const float r = sqrtf(rx * rx + ry * ry + rz * rz);
+        const float inv = 1.0f / r;
+        float es, esp;
+        edge_envelope(a.envelope, r, a.r_cut, a.edge_scale, es, esp);
+        Grp::make_row(rx * inv, ry * inv, rz * inv, es, esp, mwin + lane * Grp::MSTRIDE);
       }
       __syncwarp();
     }
@@ -153,13 +158,14 @@ __device__ __forceinline__ void vjp_warp(const VjpArgs& a, float* smem, int lane
     // edge-vector gradient
     if constexpr (Grp::NYD > 0) {
       if (a.rbar != nullptr) {
-        float ux, uy, uz;
-        Grp::ubar(yb, m, ux, uy, uz);
+        float ux, uy, uz, rho;
+        Grp::ubar(yb, m, ux, uy, uz, rho);
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) {
           ux += __shfl_xor_sync(0xffffffffu, ux, o);
           uy += __shfl_xor_sync(0xffffffffu, uy, o);
           uz += __shfl_xor_sync(0xffffffffu, uz, o);
+          rho += __shfl_xor_sync(0xffffffffu, rho, o);
         }
         const float rx = __shfl_sync(0xffffffffu, cur.rx, p & 31);
         const float ry = __shfl_sync(0xffffffffu, cur.ry, p & 31);
@@ -168,9 +174,11 @@ __device__ __forceinline__ void vjp_warp(const VjpArgs& a, float* smem, int lane
           const float inv = 1.0f / sqrtf(rx * rx + ry * ry + rz * rz);
           const float nx = rx * inv, ny = ry * inv, nz = rz * inv;
           const float dotu = ux * nx + uy * ny + uz * nz;
-          atomicAdd(a.rbar + 3 * (size_t)q + 0, (ux - nx * dotu) * inv);
-          atomicAdd(a.rbar + 3 * (size_t)q + 1, (uy - ny * dotu) * inv);
-          atomicAdd(a.rbar + 3 * (size_t)q + 2, (uz - nz * dotu) * inv);
+          // direction part (I - u u^T)/|r| u_bar plus the radial part of the
+          // envelope, s'(|r|) (y_bar . y) r-hat
+          atomicAdd(a.rbar + 3 * (size_t)q + 0, (ux - nx * dotu) * inv + rho * nx);
+          atomicAdd(a.rbar + 3 * (size_t)q + 1, (uy - ny * dotu) * inv + rho * ny);
+          atomicAdd(a.rbar + 3 * (size_t)q + 2, (uz - nz * dotu) * inv + rho * nz);
         }
       }
 #pragma unroll
@@ -285,6 +293,9 @@ extern "C" int fc_edge_conv_vjp(const fc_conv_desc* d, int n_nodes, int n_edges,
   a.zrow = out_row(L, d->sum_paths);
   a.P = num_paths(L);
   a.sum_paths = d->sum_paths;
+  a.envelope = d->envelope;
+  a.r_cut = d->r_cut;
+  a.edge_scale = d->edge_scale;
   if ((long long)n_nodes * a.ntiles > 0x7fffffffLL) return FC_ERR_ARG;
   cudaStream_t s = (cudaStream_t)stream;
   if (x_bar && cudaMemsetAsync(x_bar, 0, sizeof(float) * (size_t)n_nodes * a.xrow * C, s) != cudaSuccess)

@@ -36,7 +36,8 @@ class FlashCartError(RuntimeError):
 class ConvDesc(ct.Structure):
     _fields_ = [("lmax_in", ct.c_int), ("lmax_edge", ct.c_int),
                 ("lmax_out", ct.c_int), ("channels", ct.c_int),
-                ("sum_paths", ct.c_int)]
+                ("sum_paths", ct.c_int), ("envelope", ct.c_int),
+                ("r_cut", ct.c_float), ("edge_scale", ct.c_float)]
 
 
 class LadderDesc(ct.Structure):
@@ -56,6 +57,8 @@ _SIGS = {
                                 _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
     "fc_edge_conv_vjp": (ct.c_int, [ct.POINTER(ConvDesc), ct.c_int, ct.c_int,
                                     _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
+    "fc_scalar_readout": (ct.c_int, [ct.c_int, ct.c_int, ct.c_int, _vp, _vp, _vp, _vp]),
+    "fc_edge_forces": (ct.c_int, [ct.c_int, ct.c_int, _vp, _vp, _vp, _vp]),
     "fc_ladder_num_paths": (ct.c_int, [ct.POINTER(LadderDesc)]),
     "fc_product_ladder_workspace_size": (ct.c_size_t, [ct.POINTER(LadderDesc), ct.c_int]),
     "fc_product_ladder": (ct.c_int, [ct.POINTER(LadderDesc), ct.c_int, _vp, _vp, _vp, _vp,
@@ -99,8 +102,13 @@ def _dev(t, dtype, name):
     return t
 
 
-def conv_desc(lmax, channels, sum_paths=False):
-    return ConvDesc(lmax, lmax, lmax, channels, int(bool(sum_paths)))
+def conv_desc(lmax, channels, sum_paths=False, envelope=None):
+    """envelope: None, or (r_cut, edge_scale) for the cosine radial envelope."""
+    if envelope is None:
+        return ConvDesc(lmax, lmax, lmax, channels, int(bool(sum_paths)), 0, 0.0, 0.0)
+    r_cut, scale = envelope
+    return ConvDesc(lmax, lmax, lmax, channels, int(bool(sum_paths)), 1, float(r_cut),
+                    float(scale))
 
 
 def num_paths(lmax, channels=4, sum_paths=False):
@@ -148,7 +156,7 @@ def build_rowptr(edge_index, edge_vec, n_nodes, stream=None):
 
 
 def edge_conv(lmax, rowptr, edge_index, edge_vec, x, w, sum_paths=False,
-              out=None, stream=None):
+              out=None, stream=None, envelope=None):
     """z of Sec. 4 Eq. (1): [N][out_row * C]."""
     _dev(rowptr, torch.int32, "rowptr")
     _dev(edge_index, torch.int32, "edge_index")
@@ -158,7 +166,7 @@ def edge_conv(lmax, rowptr, edge_index, edge_vec, x, w, sum_paths=False,
     N = rowptr.shape[0] - 1
     E = edge_index.shape[1]
     C = x.shape[1] // ((lmax + 1) ** 2)
-    d = conv_desc(lmax, C, sum_paths)
+    d = conv_desc(lmax, C, sum_paths, envelope)
     zr = out_row(lmax, C, sum_paths)
     if x.shape != (N, (lmax + 1) ** 2 * C):
         raise ValueError("x shape %s" % (tuple(x.shape),))
@@ -176,7 +184,7 @@ def edge_conv(lmax, rowptr, edge_index, edge_vec, x, w, sum_paths=False,
 
 
 def edge_conv_vjp(lmax, rowptr, edge_index, edge_vec, x, w, g, sum_paths=False,
-                  want=("x", "w", "r"), out=None, stream=None):
+                  want=("x", "w", "r"), out=None, stream=None, envelope=None):
     """(x_bar, w_bar, r_bar) of App. C Eq. (C1); entries not in `want` are None."""
     _dev(rowptr, torch.int32, "rowptr")
     _dev(edge_index, torch.int32, "edge_index")
@@ -187,7 +195,7 @@ def edge_conv_vjp(lmax, rowptr, edge_index, edge_vec, x, w, g, sum_paths=False,
     N = rowptr.shape[0] - 1
     E = edge_index.shape[1]
     C = x.shape[1] // ((lmax + 1) ** 2)
-    d = conv_desc(lmax, C, sum_paths)
+    d = conv_desc(lmax, C, sum_paths, envelope)
     P = num_paths(lmax)
     if g.shape != (N, out_row(lmax, C, sum_paths) * C):
         raise ValueError("g shape %s" % (tuple(g.shape),))
@@ -261,3 +269,47 @@ def product_ladder_vjp(lmax, order, A1, path_w, mix_w, states, gz, workspace=Non
         _ptr(workspace), ws_bytes if workspace is not None else 0, _stream(stream)),
         "fc_product_ladder_vjp")
     return A1b, pwb, mwb
+
+
+def scalar_readout(lmax, z, want_grad=True, stream=None):
+    """(energy [1], gz) with energy = sum of the rank-0 block of z and
+    gz = d energy / d z."""
+    _dev(z, torch.float32, "z")
+    N = z.shape[0]
+    C = z.shape[1] // ((lmax + 1) ** 2)
+    energy = torch.empty(1, dtype=torch.float32, device=z.device)
+    gz = torch.empty_like(z) if want_grad else None
+    _check(_lib.fc_scalar_readout(N, lmax, C, _ptr(z), _ptr(energy), _ptr(gz),
+                                  _stream(stream)), "fc_scalar_readout")
+    return energy, gz
+
+
+def edge_forces(edge_index, r_bar, n_nodes, stream=None):
+    """forces [N][3] = -dE/dpos from per-edge gradients r_bar."""
+    _dev(edge_index, torch.int32, "edge_index")
+    _dev(r_bar, torch.float32, "r_bar")
+    F = torch.empty((n_nodes, 3), dtype=torch.float32, device=r_bar.device)
+    _check(_lib.fc_edge_forces(n_nodes, edge_index.shape[1], _ptr(edge_index), _ptr(r_bar),
+                               _ptr(F), _stream(stream)), "fc_edge_forces")
+    return F
+
+
+def interaction_block(lmax, order, rowptr, edge_index, edge_vec, x, omega, path_w, mix_w,
+                      r_cut, edge_scale, stream=None):
+    """Energy and forces of one interaction block, each step a library call:
+    edge convolution with paths summed per output rank and the cosine
+    envelope (App. E Eq. E1 with the 1/sqrt(mean neighbours) factor in
+    edge_scale), the product ladder (Sec. 5 Eq. 2), E = sum of its rank-0
+    outputs, then the ladder VJP, the convolution VJP (r_bar only) and the
+    force scatter.  Returns (energy [1], forces [N][3], z)."""
+    env = (r_cut, edge_scale)
+    N = rowptr.shape[0] - 1
+    A1 = edge_conv(lmax, rowptr, edge_index, edge_vec, x, omega, sum_paths=True,
+                   envelope=env, stream=stream)
+    states, z = product_ladder(lmax, order, A1, path_w, mix_w, stream=stream)
+    energy, gz = scalar_readout(lmax, z, stream=stream)
+    A1b, _, _ = product_ladder_vjp(lmax, order, A1, path_w, mix_w, states, gz, stream=stream)
+    _, _, rb = edge_conv_vjp(lmax, rowptr, edge_index, edge_vec, x, omega, A1b, sum_paths=True,
+                             want=("r",), envelope=env, stream=stream)
+    F = edge_forces(edge_index, rb, N, stream=stream)
+    return energy, F, z

@@ -220,6 +220,15 @@ class GroupCode:
                 ukey[key] = len(self.uniq)
                 self.uniq.append((l2, dict(key[1])))
             self.usign.append((ukey[key], sign))
+        # identity paths (l2 = 0) use the stored edge scale s when an
+        # envelope is on
+        self.sidx = None
+        if any(T.is_identity(p) for p in self.paths):
+            key = (0, ((0, 1),))
+            if key not in ukey:
+                ukey[key] = len(self.uniq)
+                self.uniq.append((0, {0: 1}))
+            self.sidx = ukey[key]
         self.NU = len(self.uniq)
         q = max(1, (self.NU + 3) // 4)
         if q % 2 == 0:
@@ -230,6 +239,9 @@ class GroupCode:
         need = set()
         for (p, a, b1, terms) in self.ment:
             l2 = self.T.paths[p][1]
+            for b2 in terms:
+                need.add((l2, b2))
+        for (l2, terms) in self.uniq:
             for b2 in terms:
                 need.add((l2, b2))
         return sorted(need)
@@ -249,7 +261,7 @@ class GroupCode:
         o.append("  static constexpr int RING_OFF = %d;  // staging ring (floats into shared memory)" % self.ring_off)
         o.append("  static constexpr int MWIN_OFF = %d;  // M window (floats into shared memory)" % self.mwin_off)
         # ---- M entries of one edge (lane-per-edge), from the unit direction
-        o.append("  static __device__ __forceinline__ void make_m(float ux, float uy, float uz, float* __restrict__ mrow) {")
+        o.append("  static __device__ __forceinline__ void make_m(float ux, float uy, float uz, float s, float* __restrict__ mrow) {")
         if self.NM:
             for (l2, b2) in self.y_needed():
                 if l2 == 0:
@@ -258,13 +270,13 @@ class GroupCode:
                     o.append("    const float y_%d_%d = %s;" % (l2, b2, poly_expr(T.ypoly[l2][b2])))
             vals = []
             for k, (l2, terms) in enumerate(self.uniq):
-                vals.append(lincomb_expr(terms, lambda b, l2=l2: "y_%d_%d" % (l2, b)))
+                vals.append("s*(%s)" % lincomb_expr(terms, lambda b, l2=l2: "y_%d_%d" % (l2, b)))
             while len(vals) % 4:
                 vals.append("0.0f")
             for q in range(len(vals) // 4):
                 o.append("    st_f4(mrow + %d, %s, %s, %s, %s);" % (4 * q, *vals[4 * q:4 * q + 4]))
         else:
-            o.append("    (void)ux; (void)uy; (void)uz; (void)mrow;")
+            o.append("    (void)ux; (void)uy; (void)uz; (void)s; (void)mrow;")
         o.append("  }")
         # ---- issue the copies of one edge
         o.append("  static __device__ __forceinline__ void issue(float* st, const float* __restrict__ xv, const float* __restrict__ we, int C, bool xok, bool ok) {")
@@ -274,6 +286,9 @@ class GroupCode:
             o.append("    cp_async16(st + %d, we + %d * C, ok);" % (128 * (len(self.xrows) + i), p))
         o.append("  }")
         # ---- accumulate one edge
+        o.append("  // ENV: an edge envelope scales every M entry; the identity paths")
+        o.append("  // (l2 = 0) then read the stored scale instead of using w x directly")
+        o.append("  template <bool ENV>")
         o.append("  static __device__ __forceinline__ void accum(float4 (&acc)[NA], const float* st, const float* __restrict__ m) {")
         for i, r in enumerate(self.xrows):
             o.append("    const float4 x%d = ld_s4(st + %d);" % (r, 128 * i))
@@ -286,9 +301,17 @@ class GroupCode:
             l1, l2, l3 = T.paths[p]
             o.append("    // path (%d,%d)->%d rows %s" % (l1, l2, l3, self.prow[p]))
             if T.is_identity(p):
+                q, c = divmod(self.sidx, 4)
+                o.append("    if constexpr (ENV) {")
+                o.append("      const float sc = m[%d];" % self.sidx)
                 for a in self.prow[p]:
                     i = acc_of[(p, a)]
-                    o.append("    acc[%d] = fma4(w%d, x%d, acc[%d]);" % (i, pi, l1 * l1 + a, i))
+                    o.append("      acc[%d] = fma4s(sc, mul4(w%d, x%d), acc[%d]);" % (i, pi, l1 * l1 + a, i))
+                o.append("    } else {")
+                for a in self.prow[p]:
+                    i = acc_of[(p, a)]
+                    o.append("      acc[%d] = fma4(w%d, x%d, acc[%d]);" % (i, pi, l1 * l1 + a, i))
+                o.append("    }")
                 continue
             rows_p = self.prow[p]
             ents = [(a, b1) for (pp, a, b1, _) in self.ment if pp == p]
@@ -504,13 +527,16 @@ class VjpGroupCode:
                 for b1, terms in T.mrow(p, a):
                     self.ment.append((p, a, b1, terms))
         self.NM = len(self.ment)
+        # every direction component the group touches, T_0 = 1 included: it has
+        # no angular derivative, but under a radial envelope s(|r|) T_0 does
         ycomps = sorted(set((T.paths[p][1], b2) for p in paths
-                            for b2 in range(2 * T.paths[p][1] + 1) if T.paths[p][1] > 0))
+                            for b2 in range(2 * T.paths[p][1] + 1)))
         self.ycomps = ycomps                 # direction components with a gradient
         self.NYD = len(ycomps)
         self.NROW = len(self.xrows) + len(paths)
         self.dbase = (self.NM + 3) // 4 * 4  # offset of d y / d u in a window row
-        n = self.dbase + 3 * self.NYD
+        self.ybase = self.dbase + 3 * self.NYD   # offset of s'(|r|) y
+        n = self.ybase + self.NYD
         q = max(1, (n + 3) // 4)
         if q % 2 == 0:
             q += 1
@@ -531,8 +557,8 @@ class VjpGroupCode:
         o.append("  static constexpr int RING_OFF = %d;" % self.ring_off)
         o.append("  static constexpr int MWIN_OFF = %d;" % self.mwin_off)
         # ---- window row: M pairs, then d y / d u (3 per component)
-        o.append("  static __device__ __forceinline__ void make_row(float ux, float uy, float uz, float* __restrict__ mrow) {")
-        yneed = set()
+        o.append("  static __device__ __forceinline__ void make_row(float ux, float uy, float uz, float s, float sp, float* __restrict__ mrow) {")
+        yneed = set(self.ycomps)
         for (p, a, b1, terms) in self.ment:
             for b2 in terms:
                 yneed.add((T.paths[p][1], b2))
@@ -541,12 +567,14 @@ class VjpGroupCode:
         vals = []
         for k, (p, a, b1, terms) in enumerate(self.ment):
             l2 = T.paths[p][1]
-            vals.append(lincomb_expr(terms, lambda b, l2=l2: "y_%d_%d" % (l2, b)))
+            vals.append("s*(%s)" % lincomb_expr(terms, lambda b, l2=l2: "y_%d_%d" % (l2, b)))
         while len(vals) < self.dbase:
             vals.append("0.0f")
         for (l2, b2) in self.ycomps:
             for j in range(3):
-                vals.append(poly_expr(direction_derivative_polys(l2)[b2][j]))
+                vals.append("s*(%s)" % poly_expr(direction_derivative_polys(l2)[b2][j]))
+        for (l2, b2) in self.ycomps:
+            vals.append("sp*y_%d_%d" % (l2, b2))
         while len(vals) % 4:
             vals.append("0.0f")
         for q in range(len(vals) // 4):
@@ -614,7 +642,7 @@ class VjpGroupCode:
                 o.append("      xb[%d] = fma4(w, h%d, xb[%d]);" % (xidx[l1 * l1 + b], b, xidx[l1 * l1 + b]))
             o.append("      if (act) st_z4(wbar_e + %d * C, wb);" % p)
             # y_bar: d_(a,b1) = <g_a, w x_b1> over the lane's 4 channels, then K
-            if l2 > 0:
+            if True:
                 for b in bset:
                     o.append("      const float4 t%d = mul4(w, x%d);" % (b, l1 * l1 + b))
                 for k, (a, b, terms) in enumerate(ents):
@@ -625,12 +653,13 @@ class VjpGroupCode:
             o.append("    }")
         o.append("  }")
         # ---- u_bar = (d y / d u)^T y_bar  (uniform d y / d u from the window)
-        o.append("  static __device__ __forceinline__ void ubar(const float (&yb)[%d], const float* __restrict__ m, float& ux, float& uy, float& uz) {" % max(1, self.NYD))
-        o.append("    ux = 0.0f; uy = 0.0f; uz = 0.0f;")
+        o.append("  static __device__ __forceinline__ void ubar(const float (&yb)[%d], const float* __restrict__ m, float& ux, float& uy, float& uz, float& rho) {" % max(1, self.NYD))
+        o.append("    ux = 0.0f; uy = 0.0f; uz = 0.0f; rho = 0.0f;")
         for i in range(self.NYD):
             base = self.dbase + 3 * i
             o.append("    ux = fmaf(yb[%d], m[%d], ux); uy = fmaf(yb[%d], m[%d], uy); uz = fmaf(yb[%d], m[%d], uz);" %
                      (i, base, i, base + 1, i, base + 2))
+            o.append("    rho = fmaf(yb[%d], m[%d], rho);" % (i, self.ybase + i))
         o.append("  }")
         # ---- x_bar rows
         o.append("  static __device__ __forceinline__ void flush_xbar(float* __restrict__ xbv, int C, float4 (&xb)[NX]) {")

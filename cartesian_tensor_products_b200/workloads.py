@@ -192,8 +192,12 @@ def periodic_neighbours(pos, box, cutoff):
     return ei, ev
 
 
-def diamond(seed=5, channels=128, lmax=3, order=5, cutoff=5.0):
-    pos, box = diamond_positions(seed=seed)
+def diamond(seed=5, channels=128, lmax=3, order=5, cutoff=5.0, cells=5):
+    """Full interaction block workload: diamond cell, periodic neighbour list,
+    node features, per-(edge, path, channel) weights omega ~ N(0,1)/sqrt(P)
+    (multiplied in the block by the cosine envelope and 1/sqrt(mean
+    neighbours)), ladder weights.  shift = edge_vec - (pos[v] - pos[u])."""
+    pos, box = diamond_positions(cells=cells, seed=seed)
     ei, ev = periodic_neighbours(pos, box, cutoff)
     n = pos.shape[0]
     g = rng(seed + 100)
@@ -202,7 +206,10 @@ def diamond(seed=5, channels=128, lmax=3, order=5, cutoff=5.0):
     x = normal(g, (n, (lmax + 1) ** 2 * channels))
     omega = normal(g, (E, P, channels), 1.0 / np.sqrt(P))
     lad = ladder_inputs(n, lmax, channels, order, seed + 200)
+    shift = (ev.astype(np.float64) - (pos[ei[1]] - pos[ei[0]]))
+    shift = box * np.round(shift / box)
     return dict(name="diamond", n_nodes=n, lmax=lmax, channels=channels,
                 order=order, cutoff=cutoff, box=box, pos=pos.astype(np.float32),
-                pos64=pos, edge_index=ei, edge_vec=ev, x=x, omega=omega,
-                path_w=lad["path_w"], mix_w=lad["mix_w"])
+                pos64=pos, edge_index=ei, edge_vec=ev, shift=shift, x=x, omega=omega,
+                path_w=lad["path_w"], mix_w=lad["mix_w"],
+                edge_scale=float(1.0 / np.sqrt(ei.shape[1] / n)))

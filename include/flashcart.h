@@ -81,13 +81,24 @@ int fc_version(void);
  * lmax_in == lmax_edge == lmax_out in {2, 3, 4}, channels >= 4 and a
  * multiple of 4.  sum_paths = 0 keeps the P_l paths of each output rank
  * separate (z row = sum_l (2l+1) P_l C); sum_paths = 1 sums them (z row =
- * (lmax_out+1)^2 C, the node-feature layout). */
+ * (lmax_out+1)^2 C, the node-feature layout).
+ * envelope = 1 multiplies the direction tensors of edge e by
+ *   s_e = edge_scale * (cos(pi |r_e| / r_cut) + 1) / 2   (|r_e| < r_cut, else 0),
+ * a smooth radial envelope that makes every edge contribution vanish at
+ * the cutoff (App. B, "A radial envelope makes every edge contribution
+ * vanish smoothly"); by bilinearity this equals scaling all weights of edge
+ * e by s_e, and edge_scale can carry a 1/sqrt(mean neighbours) factor (App.
+ * E Eq. E1).  The VJP's r_bar then includes the derivative of s_e.
+ * envelope = 0 (r_cut and edge_scale ignored) means s_e = 1. */
 typedef struct {
-  int lmax_in;    /* rank of node features x (l1)           */
-  int lmax_edge;  /* rank of direction tensors T_l2(r-hat) */
-  int lmax_out;   /* rank of outputs (l3)                   */
-  int channels;   /* C                                      */
-  int sum_paths;  /* 0 or 1                                 */
+  int lmax_in;      /* rank of node features x (l1)           */
+  int lmax_edge;    /* rank of direction tensors T_l2(r-hat) */
+  int lmax_out;     /* rank of outputs (l3)                   */
+  int channels;     /* C                                      */
+  int sum_paths;    /* 0 or 1                                 */
+  int envelope;     /* 0 or 1                                 */
+  float r_cut;      /* cutoff radius (envelope = 1), > 0      */
+  float edge_scale; /* global factor of s_e (envelope = 1)    */
 } fc_conv_desc;
 
 /* Number of paths P of the descriptor, or -1 if it is not supported. */
@@ -154,6 +165,21 @@ int fc_edge_conv_vjp(const fc_conv_desc *desc, int n_nodes, int n_edges,
                      const float *edge_vec, const float *x, const float *w,
                      const float *g, float *x_bar, float *w_bar, float *r_bar,
                      fc_stream_t stream);
+
+/* Scalar readout of a node-layout array z [n_nodes][(lmax+1)^2 C]:
+ *   energy[0] = sum_{n,k} z[n, rank 0, k]   (device float, overwritten)
+ *   gz[n, rank 0, k] = 1, every other entry 0  (device, may be NULL)
+ * i.e. E as the sum of the rank-0 outputs and dE/dz.  The sum uses atomic
+ * additions (not bitwise reproducible). */
+int fc_scalar_readout(int n_nodes, int lmax, int channels, const float *z,
+                      float *energy, float *gz, fc_stream_t stream);
+
+/* Forces from edge-vector gradients, for r_e = pos[v_e] - pos[u_e]
+ * (+ a fixed periodic shift):
+ *   forces[i] = -(sum_{e: v_e = i} r_bar[e] - sum_{e: u_e = i} r_bar[e])
+ * = -dE/dpos_i.  forces [n_nodes][3] (device, overwritten; atomic sums). */
+int fc_edge_forces(int n_nodes, int n_edges, const int32_t *edge_index,
+                   const float *r_bar, float *forces, fc_stream_t stream);
 
 /* Product-ladder descriptor: ranks 0..lmax for every state (lmax in
  * {2,3,4}), channels a multiple of 4, order >= 1 (order-1 products). */

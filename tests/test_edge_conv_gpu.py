@@ -154,3 +154,21 @@ def test_graph_validation(fc):
         fc.build_rowptr(ei, dev(bad), 3)
     assert e.value.status == 3
     assert fc.build_rowptr(dev(np.zeros((2, 0), np.int32)), None, 4).cpu().tolist() == [0] * 5
+
+
+@pytest.mark.parametrize("sum_paths", [False, True])
+def test_envelope_forward(fc, sum_paths):
+    """Cosine radial envelope: equal to scaling every weight of edge e by
+    s(|r_e|) (bilinearity); some edges lie beyond the cutoff."""
+    wl = W.tiny()
+    wl = dict(wl, lmax=3, **W.conv_inputs(wl["n_nodes"], wl["edge_index"], 3, 8, 91))
+    r_cut, scale = 2.5, 0.7
+    s, _, _ = O.envelope(wl["edge_vec"], r_cut, scale)
+    assert (s == 0).any() and (s > 0).any()
+    ei, ev = dev(wl["edge_index"]), dev(wl["edge_vec"])
+    rowptr = fc.build_rowptr(ei, ev, wl["n_nodes"])
+    z = fc.edge_conv(3, rowptr, ei, ev, dev(wl["x"]), dev(wl["w"]), sum_paths=sum_paths,
+                     envelope=(r_cut, scale)).cpu().numpy()
+    ref = O.edge_conv(3, 3, 3, 8, wl["edge_index"], wl["edge_vec"], wl["x"],
+                      wl["w"] * s[:, None, None], wl["n_nodes"], sum_paths=sum_paths)
+    assert rel_err(z, ref) <= FWD_TOL

@@ -132,3 +132,25 @@ def test_vjp_ragged_and_channel_tails(fc, L, C):
     wl = dict(n_nodes=N, lmax=L, channels=C, edge_index=ei, edge_vec=ev,
               **W.conv_inputs(N, ei, L, C, 31 + C, with_grad=True))
     check_all(gpu_vjp(fc, wl, wl["g"]), oracle_vjp(wl, wl["g"]))
+
+
+@pytest.mark.parametrize("sum_paths", [False, True])
+def test_envelope_vjp(fc, sum_paths):
+    """With the envelope s(|r|): x_bar as for weights w s, w_bar = s <g, f>,
+    and r_bar gains s'(|r|) r_hat sum_{p,k} w <g, f>."""
+    wl = W.tiny()
+    wl = dict(wl, lmax=3, **W.conv_inputs(wl["n_nodes"], wl["edge_index"], 3, 8, 92,
+                                         with_grad=True, sum_paths=sum_paths))
+    r_cut, scale = 2.5, 0.7
+    s, sp, r = O.envelope(wl["edge_vec"], r_cut, scale)
+    ei, ev = dev(wl["edge_index"]), dev(wl["edge_vec"])
+    rowptr = fc.build_rowptr(ei, ev, wl["n_nodes"])
+    xb, wb, rb = fc.edge_conv_vjp(3, rowptr, ei, ev, dev(wl["x"]), dev(wl["w"]), dev(wl["g"]),
+                                  sum_paths=sum_paths, envelope=(r_cut, scale))
+    w_eff = wl["w"] * s[:, None, None]
+    rxb, rwb, rrb = O.edge_conv_vjp(3, 3, 3, 8, wl["edge_index"], wl["edge_vec"], wl["x"], w_eff,
+                                    wl["g"], wl["n_nodes"], sum_paths=sum_paths)
+    ev64 = wl["edge_vec"].astype(np.float64)
+    rrb = rrb + ((rwb * wl["w"]).sum((1, 2)) * sp)[:, None] * ev64 / r[:, None]
+    check_all((xb.cpu().numpy(), wb.cpu().numpy(), rb.cpu().numpy()),
+              (rxb, rwb * s[:, None, None], rrb))
