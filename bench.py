@@ -293,6 +293,28 @@ def extra_rows(fc, W, dev, stream, peaks, fp32_peak, steps):
                      "frac": vjp_flops / (mslb * 1e-3) / 1e12 / fp32_peak,
                      "algorithmic_flops": vjp_flops},
         "l2_flush": "256 MB written before every call"}
+    del A1, pw, mw, gz, ws, res, states
+    torch.cuda.empty_cache()
+
+    # --- one interaction block on the 1000-atom diamond cell: energy + forces
+    dm = W.diamond()
+    Nd, Ed = dm["n_nodes"], dm["edge_index"].shape[1]
+    dei = torch.from_numpy(dm["edge_index"]).to(dev)
+    dev_ = torch.from_numpy(dm["edge_vec"]).to(dev)
+    dx = torch.from_numpy(dm["x"]).to(dev)
+    dom = torch.from_numpy(dm["omega"]).to(dev)
+    dpw = torch.from_numpy(dm["path_w"]).to(dev)
+    dmw = torch.from_numpy(dm["mix_w"]).to(dev)
+    drp = fc.build_rowptr(dei, dev_, Nd)
+    msb, mnb = time_events(lambda: fc.interaction_block(dm["lmax"], dm["order"], drp, dei, dev_, dx,
+                                                        dom, dpw, dmw, dm["cutoff"],
+                                                        dm["edge_scale"]),
+                           steps, 3, stream, flush=flush)
+    rows["block_energy_forces"] = {
+        "workload": "1000-atom diamond (5x5x5 cells, a = 3.567 A, 5 A cutoff, %d edges), C=128, rank 3: "
+                    "enveloped conv (paths summed) + order-5 ladder + E + ladder VJP + conv VJP + forces" % Ed,
+        "ms": msb, "ms_min": mnb, "us_per_atom": 1e3 * msb / Nd,
+        "l2_flush": "256 MB written before every call"}
     return rows
 
 

@@ -122,7 +122,7 @@ __device__ __forceinline__ void fwd_warp(const ConvArgs& a, float* smem, int lan
         const float inv = 1.0f / r;
         float es, esp;
         edge_envelope(a.envelope, r, a.r_cut, a.edge_scale, es, esp);
-        Grp::make_m(rx * inv, ry * inv, rz * inv, es, mwin + lane * Grp::MSTRIDE);
+        Grp::template make_m<ENV>(rx * inv, ry * inv, rz * inv, es, mwin + lane * Grp::MSTRIDE);
       }
       __syncwarp();
     }

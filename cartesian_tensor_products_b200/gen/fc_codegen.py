@@ -261,20 +261,27 @@ class GroupCode:
         o.append("  static constexpr int RING_OFF = %d;  // staging ring (floats into shared memory)" % self.ring_off)
         o.append("  static constexpr int MWIN_OFF = %d;  // M window (floats into shared memory)" % self.mwin_off)
         # ---- M entries of one edge (lane-per-edge), from the unit direction
+        o.append("  template <bool ENV>")
         o.append("  static __device__ __forceinline__ void make_m(float ux, float uy, float uz, float s, float* __restrict__ mrow) {")
-        if self.NM:
+        if self.NM or self.sidx is not None:
             for (l2, b2) in self.y_needed():
                 if l2 == 0:
                     o.append("    const float y_%d_%d = 1.0f;" % (l2, b2))
                 else:
                     o.append("    const float y_%d_%d = %s;" % (l2, b2, poly_expr(T.ypoly[l2][b2])))
-            vals = []
-            for k, (l2, terms) in enumerate(self.uniq):
-                vals.append("s*(%s)" % lincomb_expr(terms, lambda b, l2=l2: "y_%d_%d" % (l2, b)))
-            while len(vals) % 4:
-                vals.append("0.0f")
-            for q in range(len(vals) // 4):
-                o.append("    st_f4(mrow + %d, %s, %s, %s, %s);" % (4 * q, *vals[4 * q:4 * q + 4]))
+            for env in (True, False):
+                vals = []
+                for k, (l2, terms) in enumerate(self.uniq):
+                    e = lincomb_expr(terms, lambda b, l2=l2: "y_%d_%d" % (l2, b))
+                    if not env and k == self.sidx:
+                        e = "0.0f"          # the scale slot is read only under an envelope
+                    vals.append(("s*(%s)" % e) if env else e)
+                while len(vals) % 4:
+                    vals.append("0.0f")
+                o.append("    if constexpr (%sENV) {" % ("" if env else "!"))
+                for q in range(len(vals) // 4):
+                    o.append("      st_f4(mrow + %d, %s, %s, %s, %s);" % (4 * q, *vals[4 * q:4 * q + 4]))
+                o.append("    }")
         else:
             o.append("    (void)ux; (void)uy; (void)uz; (void)s; (void)mrow;")
         o.append("  }")
