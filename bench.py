@@ -164,6 +164,39 @@ def cpu_baseline(wl, n_recv):
             "seconds": dt}
 
 
+# ---------------------------------------------------------------------------
+# multi-rank plumbing (one process per GPU; no collective on the data path)
+# ---------------------------------------------------------------------------
+
+def rank_env():
+    """(world, rank, local_rank) from the torchrun environment."""
+    return (int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def rank_graph_seed(rank):
+    """Each rank runs its own copy of the workload (weak scaling): rank 0 the
+    reference graph, the others independent random graphs of the same shape."""
+    return 2 if rank == 0 else 2 + 1000 * rank
+
+
+def reduce_max(value, world, device):
+    """Max over ranks of a host float (collective on every rank alike)."""
+    if world <= 1:
+        return float(value)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def weak_throughput(world, units_per_rank, steps, max_ms):
+    """Whole-job units per second: every rank processed units_per_rank per
+    step, the job took max_ms (max over ranks) for `steps` steps."""
+    return world * units_per_rank * steps / (max_ms * 1e-3)
+
+
 def time_events(fn, steps, warmup, stream, flush=None):
     """Mean device time (ms) of fn over `steps` calls, CUDA events on the
     launching stream; optional L2 flush before every call (not timed)."""
@@ -349,9 +382,7 @@ def run_ours(args):
     import torch
     import torch.distributed as dist
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    world, rank, local = rank_env()
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     if world > 1:
@@ -364,7 +395,7 @@ def run_ours(args):
     from cartesian_tensor_products_b200 import flashcart as fc
     from cartesian_tensor_products_b200 import workloads as W
 
-    wl = W.microbench(seed=2 + 1000 * rank if rank else 2)
+    wl = W.microbench(seed=rank_graph_seed(rank))
     L, C, N = wl["lmax"], wl["channels"], wl["n_nodes"]
     E = wl["edge_index"].shape[1]
     P = fc.num_paths(L)
@@ -411,12 +442,9 @@ def run_ours(args):
     clocks = sampler.stop()
     total_ms = t_all0.elapsed_time(t_all1)
     per = [a.elapsed_time(b) for a, b in zip(ev_start, ev_end)]
-    if world > 1:
-        t = torch.tensor([total_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = reduce_max(total_ms, world, dev)
     ms_per_step = total_ms / args.steps
-    value = world * E * C * args.steps / (total_ms * 1e-3)
+    value = weak_throughput(world, E * C, args.steps, total_ms)
 
     # ---- roofline of the (single) kernel of the step
     peaks, peak_kind = load_peaks()
@@ -474,17 +502,14 @@ def run_ours(args):
         a1.record(stream)
         torch.cuda.synchronize()
         e_ms = a0.elapsed_time(a1)
-        if world > 1:
-            t = torch.tensor([e_ms], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e_ms = float(t.item())
-        e2e = {"value": world * E * C * n_e2e / (e_ms * 1e-3), "unit": UNIT,
+        e_ms = reduce_max(e_ms, world, dev)
+        e2e = {"value": weak_throughput(world, E * C, n_e2e, e_ms), "unit": UNIT,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "steps": n_e2e, "ms_per_step": e_ms / n_e2e,
                "includes": "H2D of x, w, edge_index, edge_vec; fc_build_rowptr (validates, syncs); fc_edge_conv; D2H of z"}
 
     rows = None
-    if rank == 0 and not args.no_rows:
+    if world == 1 and not args.no_rows:
         rows = extra_rows(fc, W, dev, stream, peaks, fp32_peak, max(3, min(args.steps, 10)))
 
     line = None
