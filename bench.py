@@ -45,6 +45,8 @@ def parse():
                     help="receivers per oracle sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-rows", action="store_true")
+    ap.add_argument("--rows", default=",".join(ROW_NAMES),
+                    help="comma-separated extra rows to time: " + ", ".join(ROW_NAMES))
     ap.add_argument("--no-e2e", action="store_true")
     return ap.parse_args()
 
@@ -66,7 +68,7 @@ def algorithmic_flops(E, C, L):
 # DRAM bytes (read + write) of one edge_conv_fwd_kernel<3, 128> launch on
 # this workload from an ncu capture (profiles/edge_conv_fwd_microbench_r3.md),
 # valid only while the kernel sources hash to the value it was taken with.
-FWD_TRAFFIC = {"sha1": "fd73249bad71fbdc90bf9ab89880fab481d8e1e1", "bytes": 1594546000 + 50859520}
+FWD_TRAFFIC = {"sha1": "09d510c3c39768669ff17afc07977537a44bf766", "bytes": 1594689000 + 48416512}
 FWD_SOURCES = ("cartesian_tensor_products_b200/csrc/fc_edge_conv.cu",
                "cartesian_tensor_products_b200/csrc/generated/fc_fwd_L3.cuh")
 
@@ -218,9 +220,17 @@ def time_events(fn, steps, warmup, stream, flush=None):
     return statistics.mean(times), min(times)
 
 
-def extra_rows(fc, W, dev, stream, peaks, fp32_peak, steps):
-    """Timed rows of the other hot-path steps (edge-conv VJP, rank 4, ladder)."""
+ROW_NAMES = ("edge_conv_vjp_r3", "edge_conv_fwd_r4", "edge_conv_vjp_r4", "ladder",
+             "block_energy_forces")
+
+
+def extra_rows(fc, W, dev, stream, peaks, fp32_peak, steps, select=ROW_NAMES):
+    """Timed rows of the other hot-path steps (edge-conv VJP, rank 4, ladder,
+    one interaction block); `select` names the ones to run."""
     import torch
+    unknown = set(select) - set(ROW_NAMES)
+    if unknown:
+        raise SystemExit("unknown rows: %s" % ", ".join(sorted(unknown)))
     rows = {}
     flush_buf = torch.empty(64 * 1024 * 1024, dtype=torch.float32, device=dev)  # 256 MB > L2
 
@@ -234,120 +244,127 @@ def extra_rows(fc, W, dev, stream, peaks, fp32_peak, steps):
     P = fc.num_paths(L)
     ei = torch.from_numpy(wl["edge_index"]).to(dev)
     ev = torch.from_numpy(wl["edge_vec"]).to(dev)
-    x = torch.from_numpy(wl["x"]).to(dev)
-    w = torch.from_numpy(wl["w"]).to(dev)
-    g = torch.from_numpy(wl["g"]).to(dev)
     rp = fc.build_rowptr(ei, ev, N)
-    out = {"x": torch.empty_like(x), "w": torch.empty_like(w),
-           "r": torch.empty((E, 3), device=dev)}
-    ms, mn = time_events(lambda: fc.edge_conv_vjp(L, rp, ei, ev, x, w, g, out=out),
-                         steps, 3, stream)
-    zr = fc.out_row(L)
-    byt = 4 * (2 * E * P * C + N * zr * C + 2 * N * 16 * C + 3 * E + 3 * E + E + N)
-    rows["edge_conv_vjp_r3"] = {
-        "workload": "microbench graph, rank 3, x_bar + w_bar + r_bar",
-        "ms": ms, "ms_min": mn, "edge_channels_per_s": E * C / (ms * 1e-3),
-        "roofline": {"bound": "hbm", "achieved": byt / (ms * 1e-3) / 1e9,
-                     "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                     "frac": byt / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
-                     "algorithmic_bytes": byt}}
-    del out, w, g, x
-    torch.cuda.empty_cache()
-
-    # --- rank 4 on the microbench graph, forward and VJP
-    wl4 = W.microbench(lmax=4, weight_seed=32)
-    L4 = 4
-    P4 = fc.num_paths(L4)
-    x4 = torch.from_numpy(wl4["x"]).to(dev)
-    w4 = torch.from_numpy(wl4["w"]).to(dev)
-    z4 = torch.empty((N, fc.out_row(L4) * C), device=dev)
-    ms4, mn4 = time_events(lambda: fc.edge_conv(L4, rp, ei, ev, x4, w4, out=z4), steps, 3, stream)
-    byt4 = 4 * (E * P4 * C + N * 25 * C + N * fc.out_row(L4) * C + 4 * E + N)
-    fl4 = algorithmic_flops(E, C, 4)
-    rows["edge_conv_fwd_r4"] = {
-        "workload": "microbench graph, rank 4 (42 paths), forward",
-        "ms": ms4, "ms_min": mn4, "edge_channels_per_s": E * C / (ms4 * 1e-3),
-        "roofline": {"bound": "hbm", "achieved": byt4 / (ms4 * 1e-3) / 1e9,
-                     "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                     "frac": byt4 / (ms4 * 1e-3) / 1e9 / peaks["hbm_gbs"],
-                     "algorithmic_bytes": byt4,
-                     "fp32_frac": fl4 / (ms4 * 1e-3) / 1e12 / fp32_peak}}
-    g4 = torch.randn((N, fc.out_row(L4) * C), device=dev)
-    out4 = {"x": torch.empty_like(x4), "w": torch.empty_like(w4),
-            "r": torch.empty((E, 3), device=dev)}
-    ms4b, mn4b = time_events(lambda: fc.edge_conv_vjp(L4, rp, ei, ev, x4, w4, g4, out=out4),
+    if "edge_conv_vjp_r3" in select:
+        x = torch.from_numpy(wl["x"]).to(dev)
+        w = torch.from_numpy(wl["w"]).to(dev)
+        g = torch.from_numpy(wl["g"]).to(dev)
+        out = {"x": torch.empty_like(x), "w": torch.empty_like(w),
+               "r": torch.empty((E, 3), device=dev)}
+        ms, mn = time_events(lambda: fc.edge_conv_vjp(L, rp, ei, ev, x, w, g, out=out),
                              steps, 3, stream)
-    byt4b = 4 * (2 * E * P4 * C + N * fc.out_row(L4) * C + 2 * N * 25 * C + 7 * E + N)
-    rows["edge_conv_vjp_r4"] = {
-        "workload": "microbench graph, rank 4, x_bar + w_bar + r_bar",
-        "ms": ms4b, "ms_min": mn4b, "edge_channels_per_s": E * C / (ms4b * 1e-3),
-        "roofline": {"bound": "hbm", "achieved": byt4b / (ms4b * 1e-3) / 1e9,
-                     "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                     "frac": byt4b / (ms4b * 1e-3) / 1e9 / peaks["hbm_gbs"],
-                     "algorithmic_bytes": byt4b}}
-    del x4, w4, z4, g4, out4
-    torch.cuda.empty_cache()
+        zr = fc.out_row(L)
+        byt = 4 * (2 * E * P * C + N * zr * C + 2 * N * 16 * C + 3 * E + 3 * E + E + N)
+        rows["edge_conv_vjp_r3"] = {
+            "workload": "microbench graph, rank 3, x_bar + w_bar + r_bar",
+            "ms": ms, "ms_min": mn, "edge_channels_per_s": E * C / (ms * 1e-3),
+            "roofline": {"bound": "hbm", "achieved": byt / (ms * 1e-3) / 1e9,
+                         "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": byt / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                         "algorithmic_bytes": byt}}
+        del out, w, g, x
+        torch.cuda.empty_cache()
 
-    # --- ladder, 4096 nodes x 128 channels, rank 3, order 4
-    lad = W.ladder()
-    Ll, Cl, order, Nl = lad["lmax"], lad["channels"], lad["order"], lad["n_nodes"]
-    A1 = torch.from_numpy(lad["A1"]).to(dev)
-    pw = torch.from_numpy(lad["path_w"]).to(dev)
-    mw = torch.from_numpy(lad["mix_w"]).to(dev)
-    gz = torch.from_numpy(lad["gz"]).to(dev)
-    ws = torch.empty(4 * Nl * 16 * Cl, device=dev)
-    res = {}
+    if "edge_conv_fwd_r4" in select or "edge_conv_vjp_r4" in select:
+        # --- rank 4 on the microbench graph, forward and VJP
+        wl4 = W.microbench(lmax=4, weight_seed=32)
+        L4 = 4
+        P4 = fc.num_paths(L4)
+        x4 = torch.from_numpy(wl4["x"]).to(dev)
+        w4 = torch.from_numpy(wl4["w"]).to(dev)
+        if "edge_conv_fwd_r4" in select:
+            z4 = torch.empty((N, fc.out_row(L4) * C), device=dev)
+            ms4, mn4 = time_events(lambda: fc.edge_conv(L4, rp, ei, ev, x4, w4, out=z4), steps, 3, stream)
+            byt4 = 4 * (E * P4 * C + N * 25 * C + N * fc.out_row(L4) * C + 4 * E + N)
+            fl4 = algorithmic_flops(E, C, 4)
+            rows["edge_conv_fwd_r4"] = {
+                "workload": "microbench graph, rank 4 (42 paths), forward",
+                "ms": ms4, "ms_min": mn4, "edge_channels_per_s": E * C / (ms4 * 1e-3),
+                "roofline": {"bound": "hbm", "achieved": byt4 / (ms4 * 1e-3) / 1e9,
+                             "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                             "frac": byt4 / (ms4 * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                             "algorithmic_bytes": byt4,
+                             "fp32_frac": fl4 / (ms4 * 1e-3) / 1e12 / fp32_peak}}
+        if "edge_conv_vjp_r4" in select:
+            g4 = torch.randn((N, fc.out_row(L4) * C), device=dev)
+            out4 = {"x": torch.empty_like(x4), "w": torch.empty_like(w4),
+                    "r": torch.empty((E, 3), device=dev)}
+            ms4b, mn4b = time_events(lambda: fc.edge_conv_vjp(L4, rp, ei, ev, x4, w4, g4, out=out4),
+                                     steps, 3, stream)
+            byt4b = 4 * (2 * E * P4 * C + N * fc.out_row(L4) * C + 2 * N * 25 * C + 7 * E + N)
+            rows["edge_conv_vjp_r4"] = {
+                "workload": "microbench graph, rank 4, x_bar + w_bar + r_bar",
+                "ms": ms4b, "ms_min": mn4b, "edge_channels_per_s": E * C / (ms4b * 1e-3),
+                "roofline": {"bound": "hbm", "achieved": byt4b / (ms4b * 1e-3) / 1e9,
+                             "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                             "frac": byt4b / (ms4b * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                             "algorithmic_bytes": byt4b}}
+        z4 = g4 = out4 = None
+        del x4, w4
+        torch.cuda.empty_cache()
 
-    def lad_fwd():
-        res["s"], res["z"] = fc.product_ladder(Ll, order, A1, pw, mw, workspace=ws)
-    msl, mnl = time_events(lad_fwd, steps, 3, stream, flush=flush)
-    states = res["s"]
+    if "ladder" in select:
+        # --- ladder, 4096 nodes x 128 channels, rank 3, order 4
+        lad = W.ladder()
+        Ll, Cl, order, Nl = lad["lmax"], lad["channels"], lad["order"], lad["n_nodes"]
+        A1 = torch.from_numpy(lad["A1"]).to(dev)
+        pw = torch.from_numpy(lad["path_w"]).to(dev)
+        mw = torch.from_numpy(lad["mix_w"]).to(dev)
+        gz = torch.from_numpy(lad["gz"]).to(dev)
+        ws = torch.empty(4 * Nl * 16 * Cl, device=dev)
+        res = {}
 
-    def lad_vjp():
-        fc.product_ladder_vjp(Ll, order, A1, pw, mw, states, gz, workspace=ws)
-    mslb, mnlb = time_events(lad_vjp, steps, 3, stream, flush=flush)
-    S = order - 1
-    mix_flops = S * 2 * Nl * 16 * Cl * Cl
-    tp_flops = S * Nl * Cl * 2 * 751
-    rows["ladder_fwd"] = {
-        "workload": "4096 nodes x 128 channels, rank 3, order 4 (3 products + 3 per-rank 128x128 mixes)",
-        "ms": msl, "ms_min": mnl,
-        "roofline": {"bound": "alu", "achieved": (mix_flops + tp_flops) / (msl * 1e-3) / 1e12,
-                     "peak": fp32_peak, "unit": "TFLOP/s",
-                     "frac": (mix_flops + tp_flops) / (msl * 1e-3) / 1e12 / fp32_peak,
-                     "algorithmic_flops": mix_flops + tp_flops},
-        "l2_flush": "256 MB written before every call"}
-    vjp_flops = 3 * mix_flops + 4 * tp_flops
-    rows["ladder_vjp"] = {
-        "workload": "same ladder, A1_bar + path_w_bar + mix_w_bar",
-        "ms": mslb, "ms_min": mnlb,
-        "roofline": {"bound": "alu", "achieved": vjp_flops / (mslb * 1e-3) / 1e12,
-                     "peak": fp32_peak, "unit": "TFLOP/s",
-                     "frac": vjp_flops / (mslb * 1e-3) / 1e12 / fp32_peak,
-                     "algorithmic_flops": vjp_flops},
-        "l2_flush": "256 MB written before every call"}
-    del A1, pw, mw, gz, ws, res, states
-    torch.cuda.empty_cache()
+        def lad_fwd():
+            res["s"], res["z"] = fc.product_ladder(Ll, order, A1, pw, mw, workspace=ws)
+        msl, mnl = time_events(lad_fwd, steps, 3, stream, flush=flush)
+        states = res["s"]
 
-    # --- one interaction block on the 1000-atom diamond cell: energy + forces
-    dm = W.diamond()
-    Nd, Ed = dm["n_nodes"], dm["edge_index"].shape[1]
-    dei = torch.from_numpy(dm["edge_index"]).to(dev)
-    dev_ = torch.from_numpy(dm["edge_vec"]).to(dev)
-    dx = torch.from_numpy(dm["x"]).to(dev)
-    dom = torch.from_numpy(dm["omega"]).to(dev)
-    dpw = torch.from_numpy(dm["path_w"]).to(dev)
-    dmw = torch.from_numpy(dm["mix_w"]).to(dev)
-    drp = fc.build_rowptr(dei, dev_, Nd)
-    msb, mnb = time_events(lambda: fc.interaction_block(dm["lmax"], dm["order"], drp, dei, dev_, dx,
-                                                        dom, dpw, dmw, dm["cutoff"],
-                                                        dm["edge_scale"]),
-                           steps, 3, stream, flush=flush)
-    rows["block_energy_forces"] = {
-        "workload": "1000-atom diamond (5x5x5 cells, a = 3.567 A, 5 A cutoff, %d edges), C=128, rank 3: "
-                    "enveloped conv (paths summed) + order-5 ladder + E + ladder VJP + conv VJP + forces" % Ed,
-        "ms": msb, "ms_min": mnb, "us_per_atom": 1e3 * msb / Nd,
-        "l2_flush": "256 MB written before every call"}
+        def lad_vjp():
+            fc.product_ladder_vjp(Ll, order, A1, pw, mw, states, gz, workspace=ws)
+        mslb, mnlb = time_events(lad_vjp, steps, 3, stream, flush=flush)
+        S = order - 1
+        mix_flops = S * 2 * Nl * 16 * Cl * Cl
+        tp_flops = S * Nl * Cl * 2 * 751
+        rows["ladder_fwd"] = {
+            "workload": "4096 nodes x 128 channels, rank 3, order 4 (3 products + 3 per-rank 128x128 mixes)",
+            "ms": msl, "ms_min": mnl,
+            "roofline": {"bound": "alu", "achieved": (mix_flops + tp_flops) / (msl * 1e-3) / 1e12,
+                         "peak": fp32_peak, "unit": "TFLOP/s",
+                         "frac": (mix_flops + tp_flops) / (msl * 1e-3) / 1e12 / fp32_peak,
+                         "algorithmic_flops": mix_flops + tp_flops},
+            "l2_flush": "256 MB written before every call"}
+        vjp_flops = 3 * mix_flops + 4 * tp_flops
+        rows["ladder_vjp"] = {
+            "workload": "same ladder, A1_bar + path_w_bar + mix_w_bar",
+            "ms": mslb, "ms_min": mnlb,
+            "roofline": {"bound": "alu", "achieved": vjp_flops / (mslb * 1e-3) / 1e12,
+                         "peak": fp32_peak, "unit": "TFLOP/s",
+                         "frac": vjp_flops / (mslb * 1e-3) / 1e12 / fp32_peak,
+                         "algorithmic_flops": vjp_flops},
+            "l2_flush": "256 MB written before every call"}
+        del A1, pw, mw, gz, ws, res, states
+        torch.cuda.empty_cache()
+
+    if "block_energy_forces" in select:
+        # --- one interaction block on the 1000-atom diamond cell: energy + forces
+        dm = W.diamond()
+        Nd, Ed = dm["n_nodes"], dm["edge_index"].shape[1]
+        dei = torch.from_numpy(dm["edge_index"]).to(dev)
+        dev_ = torch.from_numpy(dm["edge_vec"]).to(dev)
+        dx = torch.from_numpy(dm["x"]).to(dev)
+        dom = torch.from_numpy(dm["omega"]).to(dev)
+        dpw = torch.from_numpy(dm["path_w"]).to(dev)
+        dmw = torch.from_numpy(dm["mix_w"]).to(dev)
+        drp = fc.build_rowptr(dei, dev_, Nd)
+        msb, mnb = time_events(lambda: fc.interaction_block(dm["lmax"], dm["order"], drp, dei, dev_, dx,
+                                                            dom, dpw, dmw, dm["cutoff"],
+                                                            dm["edge_scale"]),
+                               steps, 3, stream, flush=flush)
+        rows["block_energy_forces"] = {
+            "workload": "1000-atom diamond (5x5x5 cells, a = 3.567 A, 5 A cutoff, %d edges), C=128, rank 3: "
+                        "enveloped conv (paths summed) + order-5 ladder + E + ladder VJP + conv VJP + forces" % Ed,
+            "ms": msb, "ms_min": mnb, "us_per_atom": 1e3 * msb / Nd,
+            "l2_flush": "256 MB written before every call"}
     return rows
 
 
@@ -510,7 +527,8 @@ def run_ours(args):
 
     rows = None
     if world == 1 and not args.no_rows:
-        rows = extra_rows(fc, W, dev, stream, peaks, fp32_peak, max(3, min(args.steps, 10)))
+        rows = extra_rows(fc, W, dev, stream, peaks, fp32_peak, max(3, min(args.steps, 10)),
+                          select=[r for r in args.rows.split(",") if r])
 
     line = None
     if rank == 0:
