@@ -58,4 +58,10 @@ int device_sm_count();
 // validates the parts of a convolution descriptor this build supports
 int check_conv_desc(const fc_conv_desc* d);
 
+// tensor-core per-rank channel mix of the ladder (fc_mix_tc.cu), C = 128:
+// mode 0: out = in M^T per rank; mode 1: out = in M per rank
+bool mix_tc_supported(int L, int C);
+int launch_mix_tc(int mode, int L, int N, const float* in, const float* M, float* out,
+                  cudaStream_t s);
+
 }  // namespace fc

@@ -9,8 +9,11 @@
 // Every product couples channel k only with channel k (channel-diagonal,
 // Sec. 5), so the product kernel is one thread per channel walking a chunk
 // of nodes with the path weights of its channel in registers.  The mix is a
-// per-rank FP32 GEMM over the rows (node, component) of that rank, with the
-// new state and the running sum z written in its epilogue.  The VJP replays
+// per-rank GEMM over the rows (node, component) of that rank: at C = 128 on
+// the tcgen05 tensor cores with a three-term TF32 split (fc_mix_tc.cu),
+// which writes the new state and leaves z to one summing pass at the end;
+// else the register-tiled FP32 kernel below, which also adds the new state
+// into z in its epilogue.  The VJP replays
 // the steps backwards: B_v is recomputed, B_bar = M^T-product of A_bar,
 // M_bar += A_bar^T B (split over row chunks, atomic tile adds), and the
 // product VJP (App. C Eq. C1 per path) adds into A_v_bar and A_1_bar and
@@ -278,6 +281,35 @@ __global__ void __launch_bounds__(256) ladder_wgrad_kernel(int N, int C, int NY,
   }
 }
 
+// z = A_1 + sum_v states[v], float4 per thread (plane % 4 == 0)
+__global__ void __launch_bounds__(256) ladder_sum_kernel(size_t plane4, int S,
+                                                         const float4* __restrict__ A1,
+                                                         const float4* __restrict__ states,
+                                                         float4* __restrict__ z) {
+  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < plane4;
+       i += (size_t)gridDim.x * blockDim.x) {
+    float4 acc = __ldg(A1 + i);
+    for (int v = 0; v < S; ++v) {
+      const float4 a = __ldcs(states + (size_t)v * plane4 + i);
+      acc.x += a.x;
+      acc.y += a.y;
+      acc.z += a.z;
+      acc.w += a.w;
+    }
+    __stcs(z + i, acc);
+  }
+}
+
+static int launch_ladder_sum(size_t plane, int S, const float* A1, const float* states, float* z,
+                             cudaStream_t s) {
+  const size_t plane4 = plane / 4;
+  const int grid = 8 * device_sm_count();
+  ladder_sum_kernel<<<grid, 256, 0, s>>>(plane4, S, reinterpret_cast<const float4*>(A1),
+                                         reinterpret_cast<const float4*>(states),
+                                         reinterpret_cast<float4*>(z));
+  return cudaGetLastError() == cudaSuccess ? FC_OK : FC_ERR_CUDA;
+}
+
 // ---------------------------------------------------------------------------
 // orchestration
 // ---------------------------------------------------------------------------
@@ -381,17 +413,22 @@ int fc_product_ladder(const fc_ladder_desc* d, int n_nodes, const float* A1, con
   const int NY = (L + 1) * (L + 1);
   const size_t plane = (size_t)n_nodes * NY * C;
   const int P = num_paths(L);
-  if (cudaMemcpyAsync(z, A1, sizeof(float) * plane, cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+  // tensor-core mix: states only, then z = A_1 + sum of the states in one pass
+  const bool tc = S > 0 && mix_tc_supported(L, C);
+  if (!tc && cudaMemcpyAsync(z, A1, sizeof(float) * plane, cudaMemcpyDeviceToDevice, s) != cudaSuccess)
     return FC_ERR_CUDA;
   float* B = static_cast<float*>(workspace);
   for (int v = 1; v <= S; ++v) {
     const float* Av = v == 1 ? A1 : states + (size_t)(v - 2) * plane;
     st = tp_dispatch(L, n_nodes, C, Av, A1, path_w + (size_t)(v - 1) * P * C, B, s);
     if (st != FC_OK) return st;
-    st = launch_mix<kMixFwd>(L, n_nodes, C, B, mix_w + (size_t)(v - 1) * (L + 1) * C * C,
-                             states + (size_t)(v - 1) * plane, z, s);
+    const float* Mv = mix_w + (size_t)(v - 1) * (L + 1) * C * C;
+    float* Anext = states + (size_t)(v - 1) * plane;
+    st = tc ? launch_mix_tc(0, L, n_nodes, B, Mv, Anext, s)
+            : launch_mix<kMixFwd>(L, n_nodes, C, B, Mv, Anext, z, s);
     if (st != FC_OK) return st;
   }
+  if (tc) return launch_ladder_sum(plane, S, A1, states, z, s);
   return FC_OK;
 }
 
@@ -449,7 +486,9 @@ int fc_product_ladder_vjp(const fc_ladder_desc* d, int n_nodes, const float* A1,
         return FC_ERR_CUDA;
     }
     if ((st = tp_dispatch(L, n_nodes, C, Av, A1, W, B, s)) != FC_OK) return st;
-    if ((st = launch_mix<kMixBar>(L, n_nodes, C, Anext_bar, M, Bbar, nullptr, s)) != FC_OK) return st;
+    st = mix_tc_supported(L, C) ? launch_mix_tc(1, L, n_nodes, Anext_bar, M, Bbar, s)
+                                : launch_mix<kMixBar>(L, n_nodes, C, Anext_bar, M, Bbar, nullptr, s);
+    if (st != FC_OK) return st;
     if ((st = launch_wgrad(L, n_nodes, C, Anext_bar, B, mix_w_bar + (size_t)(v - 1) * (L + 1) * C * C,
                            s)) != FC_OK)
       return st;

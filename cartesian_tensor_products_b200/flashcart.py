@@ -66,6 +66,7 @@ _SIGS = {
     "fc_product_ladder_vjp_workspace_size": (ct.c_size_t, [ct.POINTER(LadderDesc), ct.c_int]),
     "fc_product_ladder_vjp": (ct.c_int, [ct.POINTER(LadderDesc), ct.c_int, _vp, _vp, _vp, _vp,
                                          _vp, _vp, _vp, _vp, _vp, ct.c_size_t, _vp]),
+    "fc_device_error": (ct.c_int, [ct.POINTER(ct.c_int), _vp]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _f = getattr(_lib, _name)
@@ -269,6 +270,14 @@ def product_ladder_vjp(lmax, order, A1, path_w, mix_w, states, gz, workspace=Non
         _ptr(workspace), ws_bytes if workspace is not None else 0, _stream(stream)),
         "fc_product_ladder_vjp")
     return A1b, pwb, mwb
+
+
+def device_error(stream=None):
+    """Sticky error word of the kernels with bounded barrier waits (0 = none
+    gave up since the last call); synchronises the stream and clears it."""
+    flag = ct.c_int(0)
+    _check(_lib.fc_device_error(ct.byref(flag), _stream(stream)), "fc_device_error")
+    return flag.value
 
 
 def scalar_readout(lmax, z, want_grad=True, stream=None):

@@ -252,6 +252,13 @@ int fc_product_ladder_noalloc(const fc_ladder_desc *desc, int n_nodes,
                               const float *mix_w, float *states, float *z,
                               fc_stream_t stream);
 
+/* Sticky device-side error word of the kernels that wait on barriers (the
+ * tensor-core ladder mix): each wait gives up after a bounded number of
+ * polls, skips the rest of its work and sets the word instead of hanging.
+ * Synchronises `stream`, writes the word to *flag (0 = no wait gave up
+ * since the last call) and clears it.  FC_ERR_ARG if flag is NULL. */
+int fc_device_error(int *flag, fc_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -53,6 +53,26 @@ def test_small_ladder_full(fc, L, C, order, N):
         assert rel_err(mwb[v], rm[v]) <= VJP_TOL
 
 
+@pytest.mark.parametrize("L,order,N", [(2, 3, 50), (3, 4, 37), (4, 3, 21), (3, 3, 1200)])
+def test_tensor_core_mix_c128(fc, L, order, N):
+    """C = 128 takes the tcgen05 mix (three-term TF32 split): ragged last
+    tiles of every rank; N = 1200 at rank 3 gives 152 tiles, so some CTAs
+    walk two tiles and cross a rank boundary."""
+    C = 128
+    wl = dict(lmax=L, channels=C, order=order, **W.ladder_inputs(N, L, C, order, 2000 + L + N))
+    states, z, a1b, pwb, mwb = run_gpu(fc, wl, wl["gz"])
+    assert fc.device_error() == 0
+    rs, rz = O.ladder(L, C, order, wl["A1"], wl["path_w"], wl["mix_w"])
+    assert rel_err(z, rz) <= FWD_TOL
+    for v in range(order - 1):
+        assert rel_err(states[v], rs[v]) <= FWD_TOL
+    ra, rp, rm = O.ladder_vjp(L, C, order, wl["A1"], wl["path_w"], wl["mix_w"], wl["gz"])
+    assert rel_err(a1b, ra) <= VJP_TOL
+    for v in range(order - 1):
+        assert rel_err(pwb[v], rp[v]) <= VJP_TOL
+        assert rel_err(mwb[v], rm[v]) <= VJP_TOL
+
+
 def test_order_one_is_copy(fc):
     wl = dict(lmax=3, channels=8, order=1, **W.ladder_inputs(6, 3, 8, 1, 5))
     wl["path_w"] = np.zeros((1, 23, 8), np.float32)
@@ -89,3 +109,4 @@ def test_ladder_4096_sampled_nodes(fc, lad):
     assert rel_err(pwb, rp) <= VJP_TOL
     assert rel_err(mwb, rm) <= VJP_TOL
     assert np.isfinite(z).all()
+    assert fc.device_error() == 0
