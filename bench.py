@@ -311,7 +311,9 @@ def extra_rows(fc, W, dev, stream, peaks, fp32_peak, steps, select=ROW_NAMES):
         pw = torch.from_numpy(lad["path_w"]).to(dev)
         mw = torch.from_numpy(lad["mix_w"]).to(dev)
         gz = torch.from_numpy(lad["gz"]).to(dev)
-        ws = torch.empty(4 * Nl * 16 * Cl, device=dev)
+        ws_bytes = max(fc.ladder_workspace_bytes(Ll, Cl, order, Nl),
+                       fc.ladder_workspace_bytes(Ll, Cl, order, Nl, vjp=True))
+        ws = torch.empty(ws_bytes // 4, device=dev)
         res = {}
 
         def lad_fwd():

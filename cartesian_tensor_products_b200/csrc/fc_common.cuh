@@ -58,10 +58,23 @@ int device_sm_count();
 // validates the parts of a convolution descriptor this build supports
 int check_conv_desc(const fc_conv_desc* d);
 
-// tensor-core per-rank channel mix of the ladder (fc_mix_tc.cu), C = 128:
-// mode 0: out = in M^T per rank; mode 1: out = in M per rank
+// tensor-core per-rank channel mix of the ladder (fc_mix_tc.cu), C = 128.
+// Operands in the tiled split layout: rows of rank l in 128-row tiles
+// ts[l] .. ts[l+1] - 1, each tile 4 K chunks x (hi, lo) x 4096 floats in the
+// core-matrix layout; matrices [L+1][hi, lo][16384].
+struct MixTiles {
+  int ts[8];   // first tile of rank l (ts[l] = total for l > L)
+  int total;
+};
 bool mix_tc_supported(int L, int C);
-int launch_mix_tc(int mode, int L, int N, const float* in, const float* M, float* out,
-                  cudaStream_t s);
+MixTiles mix_tc_tiles(int L, int N);
+size_t mix_tc_operand_floats(int L, int N);
+size_t mix_tc_matrix_floats(int L);
+// natural [N][(L+1)^2][128] -> tiled split layout (rows past each rank's end = 0)
+int launch_mix_tc_split_rows(int L, int N, const float* in, float* xs, cudaStream_t s);
+// mode 0: A(j, t) = M[j][t] (forward); mode 1: A(j, t) = M[t][j] (VJP)
+int launch_mix_tc_split_matrix(int mode, int L, const float* M, float* ws, cudaStream_t s);
+// out[n][l^2 + c][j] = sum_t A_l(j, t) x[n][l^2 + c][t] for every rank l
+int launch_mix_tc(int L, int N, const float* xs, const float* ws, float* out, cudaStream_t s);
 
 }  // namespace fc

@@ -10,16 +10,17 @@
 // Sec. 5), so the product kernel is one thread per channel walking a chunk
 // of nodes with the path weights of its channel in registers.  The mix is a
 // per-rank GEMM over the rows (node, component) of that rank: at C = 128 on
-// the tcgen05 tensor cores with a three-term TF32 split (fc_mix_tc.cu),
-// which writes the new state and leaves z to one summing pass at the end;
-// else the register-tiled FP32 kernel below, which also adds the new state
-// into z in its epilogue.  The VJP replays
+// the tcgen05 tensor cores with a three-term TF32 split (fc_mix_tc.cu), fed
+// by a product kernel that writes its output pre-split in the mix's tiled
+// layout, with z summed in one pass at the end; else the register-tiled FP32
+// kernel below, which also adds the new state into z in its epilogue.  The VJP replays
 // the steps backwards: B_v is recomputed, B_bar = M^T-product of A_bar,
 // M_bar += A_bar^T B (split over row chunks, atomic tile adds), and the
 // product VJP (App. C Eq. C1 per path) adds into A_v_bar and A_1_bar and
 // accumulates W_bar over its node chunk before one atomic add per entry.
 #include "fc_common.cuh"
 #include "fc_device.cuh"
+#include "fc_tc.cuh"
 #include "generated/fc_ladder_L2.cuh"
 #include "generated/fc_ladder_L3.cuh"
 #include "generated/fc_ladder_L4.cuh"
@@ -58,6 +59,48 @@ __global__ void __launch_bounds__(128) ladder_tp_kernel(int N, int C, const floa
   }
 }
 
+// The same product written straight into the tiled split layout of the
+// tensor-core mix (C = 128): component i of node n is row n (2l+1) + i - l^2
+// of rank l, tile ts[l] + row / 128, in the tile's TF32 hi and lo blocks.
+template <int L>
+__global__ void __launch_bounds__(128) ladder_tp_tiled_kernel(int N, const float* __restrict__ Av,
+                                                              const float* __restrict__ A1,
+                                                              const float* __restrict__ W,
+                                                              MixTiles tiles,
+                                                              float* __restrict__ xs) {
+  using TP = LadderTP<L>;
+  constexpr int C = 128;
+  const int k = threadIdx.x;
+  float w[TP::P];
+#pragma unroll
+  for (int p = 0; p < TP::P; ++p) w[p] = __ldg(W + (size_t)p * C + k);
+  const int n0 = blockIdx.x * kLadderNodeChunk;
+  const int n1 = min(N, n0 + kLadderNodeChunk);
+  for (int n = n0; n < n1; ++n) {
+    const size_t base = (size_t)n * TP::NY * C + k;
+    float a[TP::NY], b[TP::NY], o[TP::NY];
+#pragma unroll
+    for (int i = 0; i < TP::NY; ++i) {
+      a[i] = __ldg(Av + base + (size_t)i * C);
+      b[i] = __ldg(A1 + base + (size_t)i * C);
+    }
+    TP::fwd(a, b, w, o);
+#pragma unroll
+    for (int l = 0; l <= L; ++l) {
+#pragma unroll
+      for (int c = 0; c < 2 * l + 1; ++c) {
+        const int row = n * (2 * l + 1) + c;
+        const int t = tiles.ts[l] + (row >> 7);
+        float* hi = xs + (size_t)t * 32768 + tc::core_offset(row & 127, k, 128);
+        uint32_t h, lo;
+        tc::split_tf32(o[l * l + c], h, lo);
+        hi[0] = __uint_as_float(h);
+        hi[16384] = __uint_as_float(lo);
+      }
+    }
+  }
+}
+
 // Avbar += w VJP1, A1bar += w VJP2, Wbar += <g, f> (atomic, once per chunk).
 // Avbar may alias A1bar (first step: A_v = A_1).
 template <int L>
@@ -81,24 +124,26 @@ __global__ void __launch_bounds__(128) ladder_tp_vjp_kernel(int N, int C, const 
   const int n1 = min(N, n0 + kLadderNodeChunk);
   for (int n = n0; n < n1; ++n) {
     const size_t base = (size_t)n * TP::NY * C + k;
+    // the running gradients are loaded with the inputs (one memory round trip
+    // per node) and the products accumulate onto them
     float a[TP::NY], b[TP::NY], g[TP::NY], ab[TP::NY], bb[TP::NY];
 #pragma unroll
     for (int i = 0; i < TP::NY; ++i) {
       a[i] = __ldg(Av + base + (size_t)i * C);
       b[i] = __ldg(A1 + base + (size_t)i * C);
       g[i] = __ldg(G + base + (size_t)i * C);
-      ab[i] = 0.0f;
-      bb[i] = 0.0f;
+      bb[i] = A1bar[base + (size_t)i * C];
+      ab[i] = alias ? 0.0f : Avbar[base + (size_t)i * C];
     }
     TP::vjp(a, b, w, g, ab, bb, wb);
     if (alias) {
 #pragma unroll
-      for (int i = 0; i < TP::NY; ++i) A1bar[base + (size_t)i * C] += ab[i] + bb[i];
+      for (int i = 0; i < TP::NY; ++i) A1bar[base + (size_t)i * C] = ab[i] + bb[i];
     } else {
 #pragma unroll
       for (int i = 0; i < TP::NY; ++i) {
-        Avbar[base + (size_t)i * C] += ab[i];
-        A1bar[base + (size_t)i * C] += bb[i];
+        Avbar[base + (size_t)i * C] = ab[i];
+        A1bar[base + (size_t)i * C] = bb[i];
       }
     }
   }
@@ -347,6 +392,18 @@ static int tp_dispatch(int L, int N, int C, const float* Av, const float* A1, co
   return FC_ERR_UNSUPPORTED_RANK;
 }
 
+static int tp_tiled_dispatch(int L, int N, const float* Av, const float* A1, const float* W,
+                             const MixTiles& tiles, float* xs, cudaStream_t s) {
+  const dim3 grid((N + kLadderNodeChunk - 1) / kLadderNodeChunk);
+  switch (L) {
+    case 2: ladder_tp_tiled_kernel<2><<<grid, 128, 0, s>>>(N, Av, A1, W, tiles, xs); break;
+    case 3: ladder_tp_tiled_kernel<3><<<grid, 128, 0, s>>>(N, Av, A1, W, tiles, xs); break;
+    case 4: ladder_tp_tiled_kernel<4><<<grid, 128, 0, s>>>(N, Av, A1, W, tiles, xs); break;
+    default: return FC_ERR_UNSUPPORTED_RANK;
+  }
+  return cudaGetLastError() == cudaSuccess ? FC_OK : FC_ERR_CUDA;
+}
+
 static int tp_vjp_dispatch(int L, int N, int C, const float* Av, const float* A1, const float* W,
                            const float* G, float* Avbar, float* A1bar, float* Wbar, cudaStream_t s) {
   switch (L) {
@@ -388,9 +445,16 @@ int fc_ladder_num_paths(const fc_ladder_desc* d) {
   return num_paths(d->lmax);
 }
 
+// Tensor-core path scratch: the product in the tiled split layout plus one
+// step's split mixing matrices.
+static size_t tc_scratch_floats(int L, int N) {
+  return mix_tc_operand_floats(L, N) + mix_tc_matrix_floats(L);
+}
+
 size_t fc_product_ladder_workspace_size(const fc_ladder_desc* d, int n_nodes) {
   if (check_ladder_desc(d) != FC_OK || n_nodes < 0) return 0;
   const int NY = (d->lmax + 1) * (d->lmax + 1);
+  if (mix_tc_supported(d->lmax, d->channels)) return sizeof(float) * tc_scratch_floats(d->lmax, n_nodes);
   return sizeof(float) * (size_t)n_nodes * NY * d->channels;
 }
 
@@ -413,29 +477,47 @@ int fc_product_ladder(const fc_ladder_desc* d, int n_nodes, const float* A1, con
   const int NY = (L + 1) * (L + 1);
   const size_t plane = (size_t)n_nodes * NY * C;
   const int P = num_paths(L);
-  // tensor-core mix: states only, then z = A_1 + sum of the states in one pass
-  const bool tc = S > 0 && mix_tc_supported(L, C);
-  if (!tc && cudaMemcpyAsync(z, A1, sizeof(float) * plane, cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+  if (S > 0 && mix_tc_supported(L, C)) {
+    // tensor cores: the product is written pre-split into the mix's tiled
+    // layout; the mix writes the states; z = A_1 + sum of the states at the end
+    const MixTiles tiles = mix_tc_tiles(L, n_nodes);
+    float* xs = static_cast<float*>(workspace);
+    float* wsm = xs + mix_tc_operand_floats(L, n_nodes);
+    for (int l = 0; l <= L; ++l)   // rows past each rank's end stay zero
+      if (cudaMemsetAsync(xs + (size_t)(tiles.ts[l + 1] - 1) * 32768, 0, 32768 * sizeof(float), s) !=
+          cudaSuccess)
+        return FC_ERR_CUDA;
+    for (int v = 1; v <= S; ++v) {
+      const float* Av = v == 1 ? A1 : states + (size_t)(v - 2) * plane;
+      if ((st = tp_tiled_dispatch(L, n_nodes, Av, A1, path_w + (size_t)(v - 1) * P * C, tiles, xs, s)) !=
+              FC_OK ||
+          (st = launch_mix_tc_split_matrix(0, L, mix_w + (size_t)(v - 1) * (L + 1) * C * C, wsm, s)) !=
+              FC_OK ||
+          (st = launch_mix_tc(L, n_nodes, xs, wsm, states + (size_t)(v - 1) * plane, s)) != FC_OK)
+        return st;
+    }
+    return launch_ladder_sum(plane, S, A1, states, z, s);
+  }
+  if (cudaMemcpyAsync(z, A1, sizeof(float) * plane, cudaMemcpyDeviceToDevice, s) != cudaSuccess)
     return FC_ERR_CUDA;
   float* B = static_cast<float*>(workspace);
   for (int v = 1; v <= S; ++v) {
     const float* Av = v == 1 ? A1 : states + (size_t)(v - 2) * plane;
     st = tp_dispatch(L, n_nodes, C, Av, A1, path_w + (size_t)(v - 1) * P * C, B, s);
     if (st != FC_OK) return st;
-    const float* Mv = mix_w + (size_t)(v - 1) * (L + 1) * C * C;
-    float* Anext = states + (size_t)(v - 1) * plane;
-    st = tc ? launch_mix_tc(0, L, n_nodes, B, Mv, Anext, s)
-            : launch_mix<kMixFwd>(L, n_nodes, C, B, Mv, Anext, z, s);
+    st = launch_mix<kMixFwd>(L, n_nodes, C, B, mix_w + (size_t)(v - 1) * (L + 1) * C * C,
+                             states + (size_t)(v - 1) * plane, z, s);
     if (st != FC_OK) return st;
   }
-  if (tc) return launch_ladder_sum(plane, S, A1, states, z, s);
   return FC_OK;
 }
 
 size_t fc_product_ladder_vjp_workspace_size(const fc_ladder_desc* d, int n_nodes) {
   if (check_ladder_desc(d) != FC_OK || n_nodes < 0) return 0;
   const int NY = (d->lmax + 1) * (d->lmax + 1);
-  return 4 * sizeof(float) * (size_t)n_nodes * NY * d->channels;
+  size_t f = 4 * (size_t)n_nodes * NY * d->channels;
+  if (mix_tc_supported(d->lmax, d->channels)) f += tc_scratch_floats(d->lmax, n_nodes);
+  return sizeof(float) * f;
 }
 
 int fc_product_ladder_vjp(const fc_ladder_desc* d, int n_nodes, const float* A1,
@@ -472,6 +554,9 @@ int fc_product_ladder_vjp(const fc_ladder_desc* d, int n_nodes, const float* A1,
   float* B = ws;
   float* Bbar = ws + plane;
   float* Ab[2] = {ws + 2 * plane, ws + 3 * plane};
+  const bool tc = mix_tc_supported(L, C);
+  float* xs = ws + 4 * plane;                                   // tensor-core path only
+  float* wsm = tc ? xs + mix_tc_operand_floats(L, n_nodes) : nullptr;
   const float* Anext_bar = gz;           // gradient of A_{v+1}
   for (int v = S; v >= 1; --v) {
     const float* Av = v == 1 ? A1 : states + (size_t)(v - 2) * plane;
@@ -486,9 +571,14 @@ int fc_product_ladder_vjp(const fc_ladder_desc* d, int n_nodes, const float* A1,
         return FC_ERR_CUDA;
     }
     if ((st = tp_dispatch(L, n_nodes, C, Av, A1, W, B, s)) != FC_OK) return st;
-    st = mix_tc_supported(L, C) ? launch_mix_tc(1, L, n_nodes, Anext_bar, M, Bbar, s)
-                                : launch_mix<kMixBar>(L, n_nodes, C, Anext_bar, M, Bbar, nullptr, s);
-    if (st != FC_OK) return st;
+    if (tc) {
+      if ((st = launch_mix_tc_split_rows(L, n_nodes, Anext_bar, xs, s)) != FC_OK ||
+          (st = launch_mix_tc_split_matrix(1, L, M, wsm, s)) != FC_OK ||
+          (st = launch_mix_tc(L, n_nodes, xs, wsm, Bbar, s)) != FC_OK)
+        return st;
+    } else if ((st = launch_mix<kMixBar>(L, n_nodes, C, Anext_bar, M, Bbar, nullptr, s)) != FC_OK) {
+      return st;
+    }
     if ((st = launch_wgrad(L, n_nodes, C, Anext_bar, B, mix_w_bar + (size_t)(v - 1) * (L + 1) * C * C,
                            s)) != FC_OK)
       return st;

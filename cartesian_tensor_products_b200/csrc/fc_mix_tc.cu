@@ -9,20 +9,28 @@
 // up to a relative 2^-21, so three TF32 MMAs per K step keep the 1e-5
 // forward tolerance of FP32 arithmetic while running on the tensor pipe.
 //
-// One persistent CTA per SM walks a contiguous range of 128-row tiles (tiles
-// never straddle two ranks), warp-specialised:
-//  * warps 0-7 (producers) hold the next tile's rows in registers (64 KB per
-//    SM in flight, coalesced 64-byte row segments), split them into TF32 hi
-//    and lo and write them in the core-matrix layout into one of three
-//    shared-memory stages, one K chunk (32 channels) at a time.  The rank's
-//    matrix, split likewise, stays in shared memory (128 KB) until the rank
-//    changes.  Thread 0 issues the 12 MMAs of a chunk (128 x 128 x 8 each,
-//    the matrix as operand A, the rows as operand B) and commits them to the
-//    stage's mbarrier, which frees the stage;
-//  * warps 8-11 (epilogue) drain the accumulator D[channel][row] from TMEM,
-//    two tiles deep (256 columns), so the stores of one tile overlap the
-//    MMAs of the next: lane = output channel, so every store of a warp is
-//    one 128-byte row segment, and the epilogue issues no loads at all.
+// Operands arrive pre-split in the "tiled" layout the MMA reads (written by
+// the product kernel, or by ladder_split_rows_kernel / ladder_split_mix_kernel
+// below): rows of rank l form 128-row tiles (tile_start[l] .. tile_start[l+1]),
+// each tile a 64 KB hi block and a 64 KB lo block of 128 rows x 128 channels
+// in the core-matrix layout of fc_tc.cuh, so K chunk c (32 channels) is the
+// contiguous 16 KB at c * 16 KB of either block; rows past the last row of a
+// rank are zeros.  The matrix of rank l is a 64 KB hi and a 64 KB lo block.
+//
+// The mix kernel moves no data through the SM's load path.  One persistent
+// CTA per SM walks a contiguous range of tiles with warp-specialised roles:
+//  * warp 0, one thread: bulk copies (TMA engine) of each chunk (hi and lo,
+//    32 KB) into one of three shared-memory stages, and of the 128 KB matrix
+//    whenever the rank changes, each completing on an mbarrier;
+//  * warp 1, one thread: the 12 MMAs of a chunk (128 x 128 x 8 each, the
+//    matrix as operand A, the rows as operand B) into a TMEM accumulator
+//    D[channel][row], two tiles deep (256 columns); commits free the stage
+//    and publish the tile;
+//  * warps 4-7: drain D from TMEM (lane = output channel, so every store of a
+//    warp is one 128-byte row segment) into the new state while the next
+//    tile's MMAs run.  (Staging the drain in shared memory and writing each
+//    node's run of rows with bulk stores from one thread measured slower.)
+//
 // C = 128 only (the tile is the whole channel range); other widths use the
 // FP32 SIMT kernels.
 #include "fc_common.cuh"
@@ -38,25 +46,55 @@ constexpr int kTcRows = 128;           // rows per tile = N of every MMA
 constexpr int kTcChunk = 32;           // channels per K chunk
 constexpr int kTcChunks = kTcC / kTcChunk;
 constexpr int kTcStages = 3;           // shared-memory stages of the row operand
-constexpr int kTcProducers = 256;      // warps 0..7 load, split and issue
-constexpr int kTcThreads = 384;        // + warps 8..11 drain the accumulator
-constexpr int kTcStageFloats = kTcRows * kTcChunk;   // 4096 (one of hi / lo)
-constexpr int kTcWFloats = kTcC * kTcC;              // 16384 (one of hi / lo)
+constexpr int kTcThreads = 256;        // warp 0 copies, warp 1 issues, warps 4..7 drain
+constexpr int kTcBlockFloats = kTcRows * kTcChunk;   // 4096: one hi or lo chunk block
+constexpr int kTcChunkFloats = 2 * kTcBlockFloats;   // hi + lo of one chunk
+constexpr int kTcWFloats = kTcC * kTcC;              // 16384: one hi or lo block (tile or matrix)
+constexpr int kTcTileFloats = 2 * kTcWFloats;        // hi + lo of a tile
 constexpr uint32_t kTcWaitPolls = 1u << 22;
-constexpr int kTcBars = kTcStages + 4;               // stage_free[3], acc_full[2], acc_free[2]
+constexpr int kTcBars = 2 * kTcStages + 5;   // stage_full[3], stage_free[3], w_full, acc_full[2], acc_free[2]
 constexpr size_t kTcSmemBytes =
-    sizeof(float) * (2 * kTcWFloats + 2 * kTcStages * kTcStageFloats) + 8 * kTcBars + 8;
+    sizeof(float) * (2 * kTcWFloats + kTcStages * kTcChunkFloats) + 8 * kTcBars + 8;
 static_assert(kTcSmemBytes <= 232448, "shared memory per CTA");
 
-struct MixTcArgs {
+__device__ int g_tc_error = 0;
+
+// Launch geometry in registers (scalar fields only, so the argument block is
+// never copied to local memory).
+struct Geom {
   int N, NY, L;
-  const float* in;          // [N][NY][C]
-  const float* M;           // [L+1][C][C] of this ladder step
-  float* out;               // [N][NY][C]
-  int tile_start[8];        // first tile of rank l; tile_start[L+1] = total
+  int t1, t2, t3, t4, t5, t6, t7;   // tile_start[1..7] (tile_start[0] = 0)
 };
 
-__device__ int g_tc_error = 0;
+__host__ __device__ __forceinline__ int tile_rank(const Geom& g, int t) {
+  return (g.L >= 1 && t >= g.t1) + (g.L >= 2 && t >= g.t2) + (g.L >= 3 && t >= g.t3) +
+         (g.L >= 4 && t >= g.t4) + (g.L >= 5 && t >= g.t5) + (g.L >= 6 && t >= g.t6);
+}
+
+__host__ __device__ __forceinline__ int tile_first(const Geom& g, int l) {
+  return l == 0 ? 0 : l == 1 ? g.t1 : l == 2 ? g.t2 : l == 3 ? g.t3 : l == 4 ? g.t4
+       : l == 5 ? g.t5 : g.t6;
+}
+
+__host__ __device__ __forceinline__ int tile_count(const Geom& g) {
+  return g.L == 0 ? g.t1 : g.L == 1 ? g.t2 : g.L == 2 ? g.t3 : g.L == 3 ? g.t4
+       : g.L == 4 ? g.t5 : g.L == 5 ? g.t6 : g.t7;
+}
+
+Geom make_geom(int L, int N) {
+  Geom g{};
+  g.N = N;
+  g.NY = (L + 1) * (L + 1);
+  g.L = L;
+  int ts[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+  int T = 0;
+  for (int l = 0; l <= 7; ++l) {
+    ts[l] = T;
+    if (l <= L) T += (N * (2 * l + 1) + kTcRows - 1) / kTcRows;
+  }
+  g.t1 = ts[1]; g.t2 = ts[2]; g.t3 = ts[3]; g.t4 = ts[4]; g.t5 = ts[5]; g.t6 = ts[6]; g.t7 = ts[7];
+  return g;
+}
 
 __device__ __forceinline__ size_t tc_rank_row(int i, int l, int NY) {
   const int w = 2 * l + 1;
@@ -64,111 +102,104 @@ __device__ __forceinline__ size_t tc_rank_row(int i, int l, int NY) {
   return ((size_t)n * NY + l * l + (i - n * w)) * kTcC;
 }
 
-__device__ __forceinline__ int tile_rank(const MixTcArgs& a, int t) {
-  int l = 0;
-  while (l < a.L && t >= a.tile_start[l + 1]) ++l;
-  return l;
+__device__ __forceinline__ void split4(const float4 v, uint4& h, uint4& w) {
+  tc::split_tf32(v.x, h.x, w.x);
+  tc::split_tf32(v.y, h.y, w.y);
+  tc::split_tf32(v.z, h.z, w.z);
+  tc::split_tf32(v.w, h.w, w.w);
 }
 
-// Producer thread p's share of K chunk c of tile t: 4 float4 at (row r, K group q)
-// with r = 16 (p/32) + 8 (it/2) + p%8, q = (p%32)/8 + 4 (it%2).  One warp
-// instruction reads 8 rows x 64 contiguous bytes; zeros past the last row.
-__device__ __forceinline__ void load_chunk(const MixTcArgs& a, int t, int t_end, int c,
-                                           float4 (&v)[4]) {
-  if (t >= t_end) return;
+// ---------------------------------------------------------------------------
+// natural layout [N][NY][128] -> tiled split layout (one CTA per tile chunk)
+// ---------------------------------------------------------------------------
+// Thread p moves 4 float4 of chunk c of tile t: (row r, K group q) with
+// r = 16 (p/32) + 8 (it/2) + p%8, q = (p%32)/8 + 4 (it%2): a warp reads 8 rows
+// x 64 contiguous bytes and eight consecutive threads fill one 128-byte core
+// matrix.  Rows past the rank's last row are written as zeros.
+__global__ void __launch_bounds__(256) ladder_split_rows_kernel(Geom g, const float* __restrict__ in,
+                                                                float* __restrict__ xs) {
+  const int t = blockIdx.x, c = blockIdx.y;
   const int p = threadIdx.x, lane = p & 31;
-  const int l = tile_rank(a, t);
-  const int R = a.N * (2 * l + 1);
-#pragma unroll
-  for (int h = 0; h < 2; ++h) {
-    const int i = (t - a.tile_start[l]) * kTcRows + 16 * (p >> 5) + 8 * h + (lane & 7);
-    if (i < R) {
-      const float4* src = reinterpret_cast<const float4*>(a.in + tc_rank_row(i, l, a.NY) + c * kTcChunk);
-      v[2 * h] = __ldg(src + (lane >> 3));
-      v[2 * h + 1] = __ldg(src + (lane >> 3) + 4);
-    } else {
-      v[2 * h] = zero4();
-      v[2 * h + 1] = zero4();
-    }
-  }
-}
-
-// The same elements into one stage, split into TF32 hi and lo, core-matrix
-// layout (eight consecutive threads fill one 128-byte core matrix).
-__device__ __forceinline__ void store_chunk(const float4 (&v)[4], float* hi, float* lo) {
-  const int p = threadIdx.x, lane = p & 31;
+  const int l = tile_rank(g, t);
+  const int R = g.N * (2 * l + 1);
+  const int row0 = (t - tile_first(g, l)) * kTcRows;
+  float* hi = xs + (size_t)t * kTcTileFloats + c * kTcBlockFloats;
+  float* lo = hi + kTcWFloats;
 #pragma unroll
   for (int it = 0; it < 4; ++it) {
     const int r = 16 * (p >> 5) + 8 * (it >> 1) + (lane & 7);
     const int q = (lane >> 3) + 4 * (it & 1);
+    const int i = row0 + r;
+    float4 v = zero4();
+    if (i < R) v = __ldg(reinterpret_cast<const float4*>(in + tc_rank_row(i, l, g.NY) + c * kTcChunk) + q);
     uint4 h, w;
-    tc::split_tf32(v[it].x, h.x, w.x);
-    tc::split_tf32(v[it].y, h.y, w.y);
-    tc::split_tf32(v[it].z, h.z, w.z);
-    tc::split_tf32(v[it].w, h.w, w.w);
+    split4(v, h, w);
     const int off = tc::core_offset(r, 4 * q, kTcRows);
     *reinterpret_cast<uint4*>(hi + off) = h;
     *reinterpret_cast<uint4*>(lo + off) = w;
   }
 }
 
-// A operand (row = output channel j, K = input channel t): forward M[j][t],
-// VJP M[t][j]; split into hi and lo by the 256 producer threads.
+// Mixing matrices [L+1][128][128] -> [L+1][hi, lo][16384] in the core layout
+// of operand A (row = output channel j, K = input channel t): forward
+// A(j, t) = M[j][t], VJP A(j, t) = M[t][j].
 template <int MODE>
-__device__ __forceinline__ void load_weights(const float* Ml, float* hi, float* lo) {
-  const int p = threadIdx.x;
-  const int j = p & (kTcC - 1);
-#pragma unroll 4
-  for (int it = 0; it < kTcWFloats / 4 / kTcProducers; ++it) {
-    const int q = 2 * it + (p >> 7);
-    float4 v;
-    if (MODE == 0) {
-      v = __ldg(reinterpret_cast<const float4*>(Ml + (size_t)j * kTcC) + q);
-    } else {
-      v.x = __ldg(Ml + (size_t)(4 * q + 0) * kTcC + j);
-      v.y = __ldg(Ml + (size_t)(4 * q + 1) * kTcC + j);
-      v.z = __ldg(Ml + (size_t)(4 * q + 2) * kTcC + j);
-      v.w = __ldg(Ml + (size_t)(4 * q + 3) * kTcC + j);
-    }
-    uint4 h, w;
-    tc::split_tf32(v.x, h.x, w.x);
-    tc::split_tf32(v.y, h.y, w.y);
-    tc::split_tf32(v.z, h.z, w.z);
-    tc::split_tf32(v.w, h.w, w.w);
-    const int off = tc::core_offset(j, 4 * q, kTcC);
-    *reinterpret_cast<uint4*>(hi + off) = h;
-    *reinterpret_cast<uint4*>(lo + off) = w;
+__global__ void __launch_bounds__(256) ladder_split_mix_kernel(const float* __restrict__ M,
+                                                               float* __restrict__ ws) {
+  const int l = blockIdx.y;
+  const int idx = blockIdx.x * blockDim.x + threadIdx.x;   // 0 .. 4095
+  const int j = idx & (kTcC - 1), q = idx >> 7;            // output channel, K group
+  const float* Ml = M + (size_t)l * kTcC * kTcC;
+  float4 v;
+  if (MODE == 0) {
+    v = __ldg(reinterpret_cast<const float4*>(Ml + (size_t)j * kTcC) + q);
+  } else {
+    v.x = __ldg(Ml + (size_t)(4 * q + 0) * kTcC + j);
+    v.y = __ldg(Ml + (size_t)(4 * q + 1) * kTcC + j);
+    v.z = __ldg(Ml + (size_t)(4 * q + 2) * kTcC + j);
+    v.w = __ldg(Ml + (size_t)(4 * q + 3) * kTcC + j);
   }
+  uint4 h, w;
+  split4(v, h, w);
+  float* hi = ws + (size_t)l * 2 * kTcWFloats;
+  const int off = tc::core_offset(j, 4 * q, kTcC);
+  *reinterpret_cast<uint4*>(hi + off) = h;
+  *reinterpret_cast<uint4*>(hi + kTcWFloats + off) = w;
 }
 
-// MODE 0: out[r][j] = sum_t in[r][t] M_l[j][t].
-// MODE 1: out[r][j] = sum_t in[r][t] M_l[t][j].
-// The accumulator of a tile is D[j][r] (TMEM lane = output channel, column =
-// tile row), two tiles deep (256 columns).
-template <int MODE>
-__global__ void __launch_bounds__(kTcThreads, 1) ladder_mix_tc_kernel(const MixTcArgs a) {
+// ---------------------------------------------------------------------------
+// the mix: out[row][j] = sum_t A(j, t) x[row][t] over the tiles of every rank
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(kTcThreads, 1) ladder_mix_tc_kernel(Geom geo,
+                                                                      const float* __restrict__ xs,
+                                                                      const float* __restrict__ ws,
+                                                                      float* __restrict__ out) {
   extern __shared__ __align__(1024) unsigned char smem[];
-  float* w_hi = reinterpret_cast<float*>(smem);
-  float* w_lo = w_hi + kTcWFloats;
-  float* x_hi = w_lo + kTcWFloats;                       // kTcStages stages
-  float* x_lo = x_hi + kTcStages * kTcStageFloats;       // kTcStages stages
-  uint64_t* stage_free = reinterpret_cast<uint64_t*>(x_lo + kTcStages * kTcStageFloats);
-  uint64_t* acc_full = stage_free + kTcStages;
+  float* w_s = reinterpret_cast<float*>(smem);                // hi, lo: 2 x 16384
+  float* x_s = w_s + 2 * kTcWFloats;                          // stages of (hi, lo): 3 x 8192
+  uint64_t* stage_full = reinterpret_cast<uint64_t*>(x_s + kTcStages * kTcChunkFloats);
+  uint64_t* stage_free = stage_full + kTcStages;
+  uint64_t* w_full = stage_free + kTcStages;
+  uint64_t* acc_full = w_full + 1;
   uint64_t* acc_free = acc_full + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_free + 2);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int T = a.tile_start[a.L + 1];
+  const int T = tile_count(geo);
   const int t_begin = (int)((long long)blockIdx.x * T / gridDim.x);
   const int t_end = (int)((long long)(blockIdx.x + 1) * T / gridDim.x);
 
   if (warp == 0) tc::tmem_alloc(tmem_slot, 2 * kTcRows);
   if (tid == 0) {
-    for (int s = 0; s < kTcStages; ++s) tc::bar_init(&stage_free[s], 1);
+    for (int s = 0; s < kTcStages; ++s) {
+      tc::bar_init(&stage_full[s], 1);
+      tc::bar_init(&stage_free[s], 1);
+    }
+    tc::bar_init(w_full, 1);
     tc::bar_init(&acc_full[0], 1);
     tc::bar_init(&acc_full[1], 1);
-    tc::bar_init(&acc_free[0], kTcThreads - kTcProducers);
-    tc::bar_init(&acc_free[1], kTcThreads - kTcProducers);
+    tc::bar_init(&acc_free[0], 128);
+    tc::bar_init(&acc_free[1], 128);
     tc::fence_bar_init();
   }
   tc::fence_before_sync();
@@ -177,84 +208,110 @@ __global__ void __launch_bounds__(kTcThreads, 1) ladder_mix_tc_kernel(const MixT
   const uint32_t tmem = *tmem_slot;
   bool fail = false;
 
-  if (tid < kTcProducers) {
-    // ---------------- producers (and the MMA issuer, thread 0) ----------------
-    constexpr uint32_t idesc = tc::idesc_tf32(kTcC, kTcRows);
-    constexpr uint32_t kLbo = kTcRows * 16, kSbo = 128;   // both operands are 128-row tiles
-    float4 buf[kTcChunks][4];
-#pragma unroll
-    for (int c = 0; c < kTcChunks; ++c) load_chunk(a, t_begin, t_end, c, buf[c]);
-    int cur_l = -1;
-    for (int t = t_begin; t < t_end && !fail; ++t) {
-      const int ti = t - t_begin;
-      const int l = tile_rank(a, t);
-      const uint32_t d_tmem = tmem + (uint32_t)(ti & 1) * kTcRows;
-      if (l != cur_l) {
-        if (ti > 0) {   // every MMA of the previous tile has read the old matrix
-          const int gl = kTcChunks * ti - 1;
-          if (!tc::bar_wait(&stage_free[gl % kTcStages], (gl / kTcStages) & 1, kTcWaitPolls))
-            fail = true;
-          if (tc::named_bar_or(1, kTcProducers, fail)) {
+  if (warp == 0) {
+    // ---------------- bulk-copy producer ----------------
+    if (lane == 0) {
+      int cur_l = -1, w_loads = 0, g = 0;
+      for (int t = t_begin; t < t_end && !fail; ++t) {
+        const int ti = t - t_begin;
+        const int l = tile_rank(geo, t);
+        if (l != cur_l) {
+          if (ti > 0) {   // the MMAs of the previous tile have read the old matrix
+            const int gl = g - 1;
+            if (!tc::bar_wait(&stage_free[gl % kTcStages], (gl / kTcStages) & 1, kTcWaitPolls)) {
+              fail = true;
+              break;
+            }
+          }
+          tc::bar_arrive_expect_tx(w_full, 2 * kTcWFloats * sizeof(float));
+          tc::bulk_load(w_s, ws + (size_t)l * 2 * kTcWFloats, 2 * kTcWFloats * sizeof(float), w_full);
+          ++w_loads;
+          cur_l = l;
+        }
+        for (int c = 0; c < kTcChunks; ++c, ++g) {
+          const int s = g % kTcStages;
+          if (g >= kTcStages &&
+              !tc::bar_wait(&stage_free[s], ((g - kTcStages) / kTcStages) & 1, kTcWaitPolls)) {
             fail = true;
             break;
           }
+          const float* src = xs + (size_t)t * kTcTileFloats + c * kTcBlockFloats;
+          tc::bar_arrive_expect_tx(&stage_full[s], kTcChunkFloats * sizeof(float));
+          tc::bulk_load(x_s + s * kTcChunkFloats, src, kTcBlockFloats * sizeof(float), &stage_full[s]);
+          tc::bulk_load(x_s + s * kTcChunkFloats + kTcBlockFloats, src + kTcWFloats,
+                        kTcBlockFloats * sizeof(float), &stage_full[s]);
         }
-        load_weights<MODE>(a.M + (size_t)l * kTcC * kTcC, w_hi, w_lo);
-        cur_l = l;
       }
-#pragma unroll
-      for (int c = 0; c < kTcChunks; ++c) {
-        const int g = kTcChunks * ti + c;
-        const int s = g % kTcStages;
-        bool bad = false;
-        if (g >= kTcStages &&
-            !tc::bar_wait(&stage_free[s], ((g - kTcStages) / kTcStages) & 1, kTcWaitPolls))
-          bad = true;
-        store_chunk(buf[c], x_hi + s * kTcStageFloats, x_lo + s * kTcStageFloats);
-        load_chunk(a, t + 1, t_end, c, buf[c]);
-        tc::fence_proxy_async();
-        if (tc::named_bar_or(1, kTcProducers, bad || fail)) {
+      if (fail) {
+        // let the copies already issued land before the CTA can exit
+        for (int k = 1; k <= kTcStages && g - k >= 0; ++k)
+          tc::bar_wait(&stage_full[(g - k) % kTcStages], ((g - k) / kTcStages) & 1, kTcWaitPolls);
+        if (w_loads > 0) tc::bar_wait(w_full, (w_loads - 1) & 1, kTcWaitPolls);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0) {
+      constexpr uint32_t idesc = tc::idesc_tf32(kTcC, kTcRows);
+      constexpr uint32_t kLbo = kTcRows * 16, kSbo = 128;   // both operands are 128-row blocks
+      const uint32_t wh = tc::smem_addr(w_s), wl = tc::smem_addr(w_s + kTcWFloats);
+      int cur_l = -1, w_loads = 0, g = 0;
+      for (int t = t_begin; t < t_end && !fail; ++t) {
+        const int ti = t - t_begin;
+        const int l = tile_rank(geo, t);
+        const uint32_t d_tmem = tmem + (uint32_t)(ti & 1) * kTcRows;
+        if (l != cur_l) {
+          if (!tc::bar_wait(w_full, w_loads & 1, kTcWaitPolls)) {
+            fail = true;
+            break;
+          }
+          ++w_loads;
+          cur_l = l;
+        }
+        // the epilogue has drained this accumulator (tile ti - 2)
+        if (ti >= 2 && !tc::bar_wait(&acc_free[ti & 1], ((ti - 2) >> 1) & 1, kTcWaitPolls)) {
           fail = true;
           break;
         }
-        if (tid == 0) {
-          // the epilogue has drained this accumulator buffer (tile ti - 2)
-          if (c == 0 && ti >= 2 &&
-              !tc::bar_wait(&acc_free[ti & 1], ((ti - 2) >> 1) & 1, kTcWaitPolls)) {
+        tc::fence_after_sync();
+        for (int c = 0; c < kTcChunks; ++c, ++g) {
+          const int s = g % kTcStages;
+          if (!tc::bar_wait(&stage_full[s], (g / kTcStages) & 1, kTcWaitPolls)) {
             fail = true;
-          } else {
-            tc::fence_after_sync();
-            const uint32_t xh = tc::smem_addr(x_hi + s * kTcStageFloats);
-            const uint32_t xl = tc::smem_addr(x_lo + s * kTcStageFloats);
-            const uint32_t wh = tc::smem_addr(w_hi), wl = tc::smem_addr(w_lo);
-#pragma unroll
-            for (int j = 0; j < kTcChunk / 8; ++j) {
-              const uint32_t kx = 2 * j * kLbo;                          // K group 2j of the stage
-              const uint32_t kw = (c * (kTcChunk / 4) + 2 * j) * kLbo;   // same K group of M
-              const uint64_t dwh = tc::smem_desc(wh + kw, kLbo, kSbo);
-              const uint64_t dwl = tc::smem_desc(wl + kw, kLbo, kSbo);
-              const uint64_t dxh = tc::smem_desc(xh + kx, kLbo, kSbo);
-              const uint64_t dxl = tc::smem_desc(xl + kx, kLbo, kSbo);
-              tc::mma_tf32(d_tmem, dwh, dxh, idesc, (c | j) != 0);
-              tc::mma_tf32(d_tmem, dwh, dxl, idesc, 1u);
-              tc::mma_tf32(d_tmem, dwl, dxh, idesc, 1u);
-            }
-            tc::commit(&stage_free[s]);
-            if (c == kTcChunks - 1) tc::commit(&acc_full[ti & 1]);
+            break;
           }
+          tc::fence_after_sync();
+          const uint32_t xh = tc::smem_addr(x_s + s * kTcChunkFloats);
+          const uint32_t xl = xh + kTcBlockFloats * sizeof(float);
+#pragma unroll
+          for (int j = 0; j < kTcChunk / 8; ++j) {
+            const uint32_t kx = 2 * j * kLbo;                          // K group 2j of the chunk
+            const uint32_t kw = (c * (kTcChunk / 4) + 2 * j) * kLbo;   // same K group of A
+            const uint64_t dwh = tc::smem_desc(wh + kw, kLbo, kSbo);
+            const uint64_t dwl = tc::smem_desc(wl + kw, kLbo, kSbo);
+            const uint64_t dxh = tc::smem_desc(xh + kx, kLbo, kSbo);
+            const uint64_t dxl = tc::smem_desc(xl + kx, kLbo, kSbo);
+            tc::mma_tf32(d_tmem, dwh, dxh, idesc, (c | j) != 0);
+            tc::mma_tf32(d_tmem, dwh, dxl, idesc, 1u);
+            tc::mma_tf32(d_tmem, dwl, dxh, idesc, 1u);
+          }
+          tc::commit(&stage_free[s]);
+          if (c == kTcChunks - 1) tc::commit(&acc_full[ti & 1]);
         }
       }
     }
-  } else {
-    // ---------------- epilogue: TMEM -> new state (and z) ----------------
-    const int ew = warp - kTcProducers / 32;        // 0..3 = TMEM lane quarter
+    __syncwarp();
+  } else if (warp >= 4) {
+    // ---------------- epilogue: TMEM -> new state ----------------
+    const int ew = warp - 4;                         // TMEM lane quarter
     const int j = 32 * ew + lane;                    // output channel
     for (int t = t_begin; t < t_end; ++t) {
       const int ti = t - t_begin;
-      const int l = tile_rank(a, t);
+      const int l = tile_rank(geo, t);
       const int w = 2 * l + 1;
-      const int R = a.N * w;
-      const int row0 = (t - a.tile_start[l]) * kTcRows;
+      const int R = geo.N * w;
+      const int row0 = (t - tile_first(geo, l)) * kTcRows;
       const uint32_t d_tmem = tmem + (uint32_t)(ti & 1) * kTcRows + ((uint32_t)(32 * ew) << 16);
       if (!tc::bar_wait(&acc_full[ti & 1], (ti >> 1) & 1, kTcWaitPolls)) {
         fail = true;
@@ -269,7 +326,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) ladder_mix_tc_kernel(const MixT
         int n = i0 / w, cc = i0 - (i0 / w) * w;
 #pragma unroll
         for (int r = 0; r < 32; ++r) {
-          if (i0 + r < R) a.out[((size_t)n * a.NY + l * l + cc) * kTcC + j] = v[r];
+          if (i0 + r < R) out[((size_t)n * geo.NY + l * l + cc) * kTcC + j] = v[r];
           if (++cc == w) { cc = 0; ++n; }
         }
       }
@@ -278,7 +335,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) ladder_mix_tc_kernel(const MixT
     }
   }
   if (fail) atomicExch(&g_tc_error, 1);
-  // every MMA completed before its tile's accumulator was read; release TMEM
+  // every MMA completed before its tile was drained; release TMEM
   tc::fence_before_sync();
   __syncthreads();
   if (warp == 0) {
@@ -288,50 +345,61 @@ __global__ void __launch_bounds__(kTcThreads, 1) ladder_mix_tc_kernel(const MixT
 }
 
 int g_tc_smem_set[64] = {0};
-int g_sm_count[64] = {0};
-
-template <int MODE>
-int launch_mix_tc_mode(int L, int N, const float* in, const float* M, float* out,
-                       cudaStream_t s) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return FC_ERR_CUDA;
-  if (!(g_tc_smem_set[dev] & (1 << MODE))) {
-    if (cudaFuncSetAttribute(ladder_mix_tc_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)kTcSmemBytes) != cudaSuccess)
-      return FC_ERR_CUDA;
-    g_tc_smem_set[dev] |= 1 << MODE;
-  }
-  if (g_sm_count[dev] == 0 &&
-      cudaDeviceGetAttribute(&g_sm_count[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-    return FC_ERR_CUDA;
-  MixTcArgs a{};
-  a.N = N;
-  a.NY = (L + 1) * (L + 1);
-  a.L = L;
-  a.in = in;
-  a.M = M;
-  a.out = out;
-  int T = 0;
-  for (int l = 0; l <= L; ++l) {
-    a.tile_start[l] = T;
-    T += (N * (2 * l + 1) + kTcRows - 1) / kTcRows;
-  }
-  a.tile_start[L + 1] = T;
-  if (T == 0) return FC_OK;
-  const int grid = T < g_sm_count[dev] ? T : g_sm_count[dev];
-  ladder_mix_tc_kernel<MODE><<<grid, kTcThreads, kTcSmemBytes, s>>>(a);
-  return cudaGetLastError() == cudaSuccess ? FC_OK : FC_ERR_CUDA;
-}
 
 }  // namespace
 
 bool mix_tc_supported(int L, int C) { return C == kTcC && L >= 0 && L <= 6; }
 
-int launch_mix_tc(int mode, int L, int N, const float* in, const float* M, float* out,
-                  cudaStream_t s) {
+MixTiles mix_tc_tiles(int L, int N) {
+  const Geom g = make_geom(L, N);
+  MixTiles m{};
+  m.ts[0] = 0;
+  m.ts[1] = g.t1; m.ts[2] = g.t2; m.ts[3] = g.t3; m.ts[4] = g.t4;
+  m.ts[5] = g.t5; m.ts[6] = g.t6; m.ts[7] = g.t7;
+  m.total = tile_count(g);
+  return m;
+}
+
+size_t mix_tc_operand_floats(int L, int N) {
+  return (size_t)mix_tc_tiles(L, N).total * kTcTileFloats;
+}
+
+size_t mix_tc_matrix_floats(int L) { return (size_t)(L + 1) * 2 * kTcWFloats; }
+
+int launch_mix_tc_split_rows(int L, int N, const float* in, float* xs, cudaStream_t s) {
+  const Geom g = make_geom(L, N);
+  const int T = tile_count(g);
+  if (T == 0) return FC_OK;
+  ladder_split_rows_kernel<<<dim3(T, kTcChunks), 256, 0, s>>>(g, in, xs);
+  return cudaGetLastError() == cudaSuccess ? FC_OK : FC_ERR_CUDA;
+}
+
+int launch_mix_tc_split_matrix(int mode, int L, const float* M, float* ws, cudaStream_t s) {
+  const dim3 grid(kTcWFloats / 4 / 256, L + 1);
+  if (mode == 0)
+    ladder_split_mix_kernel<0><<<grid, 256, 0, s>>>(M, ws);
+  else
+    ladder_split_mix_kernel<1><<<grid, 256, 0, s>>>(M, ws);
+  return cudaGetLastError() == cudaSuccess ? FC_OK : FC_ERR_CUDA;
+}
+
+int launch_mix_tc(int L, int N, const float* xs, const float* ws, float* out, cudaStream_t s) {
   if (!mix_tc_supported(L, kTcC)) return FC_ERR_UNSUPPORTED_RANK;
-  return mode == 0 ? launch_mix_tc_mode<0>(L, N, in, M, out, s)
-                   : launch_mix_tc_mode<1>(L, N, in, M, out, s);
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return FC_ERR_CUDA;
+  if (!g_tc_smem_set[dev]) {
+    if (cudaFuncSetAttribute(ladder_mix_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)kTcSmemBytes) != cudaSuccess)
+      return FC_ERR_CUDA;
+    g_tc_smem_set[dev] = 1;
+  }
+  const Geom g = make_geom(L, N);
+  const int T = tile_count(g);
+  if (T == 0) return FC_OK;
+  const int sms = device_sm_count();
+  const int grid = T < sms ? T : sms;
+  ladder_mix_tc_kernel<<<grid, kTcThreads, kTcSmemBytes, s>>>(g, xs, ws, out);
+  return cudaGetLastError() == cudaSuccess ? FC_OK : FC_ERR_CUDA;
 }
 
 }  // namespace fc

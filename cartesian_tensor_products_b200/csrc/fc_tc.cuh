@@ -97,24 +97,30 @@ __device__ __forceinline__ bool bar_wait(uint64_t* bar, uint32_t parity, uint32_
   return false;
 }
 
+// Arrival that also expects `bytes` of asynchronous-copy data on the barrier.
+__device__ __forceinline__ void bar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;"
+               :
+               : "r"(smem_addr(bar)), "r"(bytes)
+               : "memory");
+}
+
+// Bulk copy (TMA engine, no tensor map) of `bytes` contiguous bytes from
+// global memory into this CTA's shared memory; completion is signalled on the
+// mbarrier as transaction bytes.  Both addresses 16-byte aligned, bytes a
+// multiple of 16.
+__device__ __forceinline__ void bulk_load(void* smem_dst, const void* gmem_src, uint32_t bytes,
+                                          uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+      :
+      : "r"(smem_addr(smem_dst)), "l"(gmem_src), "r"(bytes), "r"(smem_addr(bar))
+      : "memory");
+}
+
 // Plain arrival on an mbarrier (counted in its expected arrivals).
 __device__ __forceinline__ void bar_arrive(uint64_t* bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" : : "r"(smem_addr(bar)) : "memory");
-}
-
-// Named barrier among `count` threads (a multiple of 32) of the CTA; returns
-// whether any of them passed pred = true.
-__device__ __forceinline__ bool named_bar_or(int id, int count, bool pred) {
-  uint32_t r;
-  asm volatile(
-      "{\n\t.reg .pred p, q;\n\t"
-      "setp.ne.u32 q, %1, 0;\n\t"
-      "bar.red.or.pred p, %2, %3, q;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}\n"
-      : "=r"(r)
-      : "r"((uint32_t)pred), "r"(id), "r"(count)
-      : "memory");
-  return r != 0;
 }
 
 // Whole warp: allocate ncols TMEM columns (power of two >= 32); the TMEM
@@ -151,12 +157,12 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
-// Round to the nearest TF32 value (ties away from zero); the result is an
-// FP32 bit pattern whose 13 low mantissa bits are zero.
+// Round a finite FP32 value to the nearest TF32 value (ties away from zero):
+// add half a TF32 unit in the last place to the sign-magnitude bit pattern
+// and clear the 13 low mantissa bits (a carry into the exponent is the
+// correct rounding up to the next binade).  Two integer operations.
 __device__ __forceinline__ uint32_t to_tf32(float x) {
-  uint32_t r;
-  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
-  return r;
+  return (__float_as_uint(x) + 0x1000u) & 0xFFFFE000u;
 }
 
 // x = hi + lo with hi and lo both TF32 values: |x - hi - lo| <= 2^-22 |x|.

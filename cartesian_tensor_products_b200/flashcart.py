@@ -223,6 +223,23 @@ def _workspace(nbytes, device):
     return torch.empty((nbytes + 15) // 16 * 4, dtype=torch.float32, device=device)
 
 
+def _scratch(workspace, need, device):
+    """(buffer, its size in bytes): a new buffer of `need` bytes, or the
+    caller's tensor with its actual size, which the library checks."""
+    if workspace is None:
+        return _workspace(need, device), need
+    if not (workspace.is_cuda and workspace.is_contiguous()):
+        raise ValueError("workspace must be a contiguous CUDA tensor")
+    return workspace, workspace.numel() * workspace.element_size()
+
+
+def ladder_workspace_bytes(lmax, channels, order, n_nodes, vjp=False):
+    """Scratch bytes fc_product_ladder (or, with vjp=True, its VJP) needs."""
+    d = LadderDesc(lmax, channels, order)
+    f = _lib.fc_product_ladder_vjp_workspace_size if vjp else _lib.fc_product_ladder_workspace_size
+    return f(ct.byref(d), n_nodes)
+
+
 def product_ladder(lmax, order, A1, path_w, mix_w, workspace=None, stream=None):
     """(states [order-1][N][...], z) of Sec. 5 Eq. (2), path-reduced products
     followed by a per-rank channel mix."""
@@ -235,8 +252,7 @@ def product_ladder(lmax, order, A1, path_w, mix_w, workspace=None, stream=None):
     states = torch.empty((max(S, 0), N, NY * C), dtype=torch.float32, device=A1.device)
     z = torch.empty_like(A1)
     ws_bytes = _lib.fc_product_ladder_workspace_size(ct.byref(d), N)
-    if workspace is None:
-        workspace = _workspace(ws_bytes, A1.device)
+    workspace, ws_bytes = _scratch(workspace, ws_bytes, A1.device)
     if S > 0:
         _dev(path_w, torch.float32, "path_w")
         _dev(mix_w, torch.float32, "mix_w")
@@ -261,8 +277,7 @@ def product_ladder_vjp(lmax, order, A1, path_w, mix_w, states, gz, workspace=Non
     pwb = torch.empty((max(S, 0),) + tuple(path_w.shape[1:]), dtype=torch.float32, device=A1.device)
     mwb = torch.empty((max(S, 0),) + tuple(mix_w.shape[1:]), dtype=torch.float32, device=A1.device)
     ws_bytes = _lib.fc_product_ladder_vjp_workspace_size(ct.byref(d), N)
-    if workspace is None:
-        workspace = _workspace(ws_bytes, A1.device)
+    workspace, ws_bytes = _scratch(workspace, ws_bytes, A1.device)
     _check(_lib.fc_product_ladder_vjp(
         ct.byref(d), N, _ptr(A1), _ptr(path_w) if S > 0 else None,
         _ptr(mix_w) if S > 0 else None, _ptr(states) if S > 0 else None, _ptr(gz),

@@ -203,8 +203,14 @@ int fc_ladder_num_paths(const fc_ladder_desc *desc);
  *   mix_w [order-1][lmax+1][C][C] (row = output channel),
  *   states [order-1][n_nodes][(lmax+1)^2 C] receives A_2 .. A_order,
  *   z [n_nodes][(lmax+1)^2 C].
- * workspace: fc_product_ladder_workspace_size() bytes of device scratch
- * (one product state), 16-byte aligned; FC_ERR_WORKSPACE if too small.
+ * At C = 128 the per-rank mix runs on the tcgen05 tensor cores (FP32
+ * accuracy through a three-term TF32 split) and z is summed in one pass at
+ * the end; other widths use FP32 SIMT kernels.
+ * workspace: fc_product_ladder_workspace_size() bytes of device scratch,
+ * 16-byte aligned, ws_bytes = its real size; FC_ERR_WORKSPACE if NULL or
+ * smaller.  At C = 128 that is the product in the mix's tiled split layout
+ * (128-row tiles per rank, TF32 hi and lo: about two product states) plus
+ * one step's split matrices; otherwise one product state.
  * order = 1 copies A1 to z and needs no workspace. */
 size_t fc_product_ladder_workspace_size(const fc_ladder_desc *desc, int n_nodes);
 int fc_product_ladder(const fc_ladder_desc *desc, int n_nodes, const float *A1,
@@ -217,7 +223,9 @@ int fc_product_ladder(const fc_ladder_desc *desc, int n_nodes, const float *A1,
  * writes A1_bar (node layout), path_w_bar [order-1][P][C] and mix_w_bar
  * [order-1][lmax+1][C][C].  The weight gradients sum over all nodes with
  * atomic additions (not bitwise reproducible).  workspace:
- * fc_product_ladder_vjp_workspace_size() bytes (four product states). */
+ * fc_product_ladder_vjp_workspace_size() bytes (four product states, plus
+ * the tensor-core scratch of fc_product_ladder at C = 128); ws_bytes = its
+ * real size, FC_ERR_WORKSPACE if smaller. */
 size_t fc_product_ladder_vjp_workspace_size(const fc_ladder_desc *desc, int n_nodes);
 int fc_product_ladder_vjp(const fc_ladder_desc *desc, int n_nodes,
                           const float *A1, const float *path_w,
@@ -232,12 +240,12 @@ int fc_product_ladder_vjp(const fc_ladder_desc *desc, int n_nodes,
  * (the pool already holds nearly all of HBM, so a raw cudaMalloc would
  * fail or fragment it) and latency-critical loops (cudaMalloc may
  * synchronise the device).  The caller still passes inputs and outputs
- * exactly as for fc_product_ladder; the scratch of one product state is a
- * fixed 16 MiB array inside the library, held by every GPU that loads the
- * library until the process exits.
- *   Limit: fc_product_ladder_workspace_size(desc, n_nodes) <= 16 MiB
- *   (n_nodes * (lmax+1)^2 * channels * 4 bytes), else FC_ERR_WORKSPACE and
- *   nothing is enqueued.
+ * exactly as for fc_product_ladder; its scratch is a fixed 16 MiB array
+ * inside the library, held by every GPU that loads the library until the
+ * process exits.
+ *   Limit: fc_product_ladder_workspace_size(desc, n_nodes) <= 16 MiB (at
+ *   rank 3, C = 128: about 990 nodes), else FC_ERR_WORKSPACE and nothing is
+ *   enqueued.
  *   The first call on a device looks up the array's device address (a
  *   runtime query, no allocation); make that first call before any stream
  *   capture on that device.

@@ -73,6 +73,26 @@ def test_tensor_core_mix_c128(fc, L, order, N):
         assert rel_err(mwb[v], rm[v]) <= VJP_TOL
 
 
+def test_caller_workspace_too_small_is_refused(fc):
+    """A caller-provided scratch buffer is passed with its real size; one
+    byte short of the query is refused on the host (FC_ERR_WORKSPACE)."""
+    L, C, order, N = 3, 128, 3, 40
+    wl = W.ladder_inputs(N, L, C, order, 77)
+    A1, pw, mw = dev(wl["A1"]), dev(wl["path_w"]), dev(wl["mix_w"])
+    need = fc.ladder_workspace_bytes(L, C, order, N)
+    short = torch.empty(need // 4 - 1, device="cuda")
+    with pytest.raises(fc.FlashCartError) as e:
+        fc.product_ladder(L, order, A1, pw, mw, workspace=short)
+    assert e.value.status == 7
+    states, z = fc.product_ladder(L, order, A1, pw, mw, workspace=torch.empty(need // 4, device="cuda"))
+    need_v = fc.ladder_workspace_bytes(L, C, order, N, vjp=True)
+    with pytest.raises(fc.FlashCartError) as e:
+        fc.product_ladder_vjp(L, order, A1, pw, mw, states, dev(wl["gz"]),
+                              workspace=torch.empty(need_v // 4 - 1, device="cuda"))
+    assert e.value.status == 7
+    torch.cuda.synchronize()
+
+
 def test_order_one_is_copy(fc):
     wl = dict(lmax=3, channels=8, order=1, **W.ladder_inputs(6, 3, 8, 1, 5))
     wl["path_w"] = np.zeros((1, 23, 8), np.float32)

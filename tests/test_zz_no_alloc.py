@@ -28,7 +28,7 @@ def test_noalloc_ladder_matches_workspace_entry_twice():
     f.restype = ct.c_int
     f.argtypes = [ct.POINTER(fc.LadderDesc), ct.c_int] + [ct.c_void_p] * 6
 
-    L, C, order, N = 3, 128, 4, 512          # 4 MiB of scratch
+    L, C, order, N = 3, 128, 4, 512          # 8.5 MiB of scratch (tensor-core path)
     wl = W.ladder_inputs(N, L, C, order, 2024)
     dev = torch.device("cuda:0")
     A1 = torch.from_numpy(wl["A1"]).to(dev)
