@@ -96,6 +96,21 @@ def conv_inputs(n_nodes, edge_index, lmax, channels, seed, with_grad=False,
     return out
 
 
+def cotangents(n_nodes, n_edges, lmax, channels, seed, edge_vec=None):
+    """Cotangents of the VJP outputs for the VJP-of-VJP (App. C Eq. C2):
+    vx like x_bar (N(0,1)), vw like w_bar (N(0,1)/sqrt(#paths)) and vr like
+    r_bar (N(0,1) per edge, scaled by |r| when edge vectors are given, so a
+    unit relative step along vr is a unit relative step of the edge)."""
+    g = rng(seed)
+    P = path_count(lmax, lmax, lmax)
+    vx = normal(g, (n_nodes, (lmax + 1) ** 2 * channels))
+    vw = normal(g, (n_edges, P, channels), 1.0 / np.sqrt(P))
+    vr = normal(g, (n_edges, 3))
+    if edge_vec is not None:
+        vr = (vr * np.linalg.norm(np.asarray(edge_vec, np.float64), axis=1)[:, None]).astype(np.float32)
+    return {"vx": vx, "vw": vw, "vr": vr}
+
+
 def tiny(seed=1):
     pos, ei, ev = random_graph(32, 4, 4.0, seed)
     d = conv_inputs(32, ei, 2, 8, seed + 100)

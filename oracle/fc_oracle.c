@@ -22,6 +22,8 @@
  *   - Cartesian product, distinct placements       App. B Eq. (B1)
  *   - permutation average vs distinct placements   App. C "Symbolic construction"
  *   - weighted product VJP                         App. C Eq. (C1)
+ *   - VJP-of-VJP of the weighted product           App. C Eq. (C2), Algorithm 3
+ *   - derivatives of the direction tensors         App. C, paragraph after Eq. (C2)
  *   - receiver-sorted convolution                  Sec. 4 Eq. (1)
  *   - array layout off(l) + (c P_l + eta) d + k    App. D "Data layout"
  *   - ladder product + channel mixing              Sec. 5 Eq. (2), App. E
@@ -315,55 +317,112 @@ void orc_direction(int l, const double *r, double *comps) {
   orc_stf_extract(l, d, comps);
 }
 
+/* Partial derivatives of the components of T_l(u), u taken as free (not
+ * normalised): order 1 gives d T_c / d u_i in d1[i][c]; order 2 gives
+ * d^2 T_c / d u_i d u_j in d2[3 i + j][c].  Product rule on the outer
+ * powers of each term of the direction-tensor sum: a slot holding u_i is
+ * replaced by 1 (and for order 2 a second, different slot holding u_j). */
+static void direction_du(int l, const double *u, int order,
+                         double d1[3][2 * ORC_MAXL + 1],
+                         double d2[9][2 * ORC_MAXL + 1]) {
+  int D = pow3(l), idx[ORC_MAXL];
+  int nd = order == 1 ? 3 : 9;
+  double acc[9][ORC_MAXD];
+  double Pw[ORC_MAXD], P[ORC_MAXD], A[ORC_MAXD];
+  double pre = dfact(2 * l - 1) / fact(l);
+  for (int j = 0; j < nd; ++j)
+    for (int f = 0; f < D; ++f) acc[j][f] = 0.0;
+  for (int m = 0; 2 * m <= l; ++m) {
+    int k = l - 2 * m;
+    double c = pre * ((m & 1) ? -1.0 : 1.0) * dfact(2 * l - 2 * m - 1) /
+               dfact(2 * l - 1) * count_delta_placements(l, m);
+    for (int j = 0; j < nd; ++j) {
+      int di = order == 1 ? j : j / 3, dj = order == 1 ? -1 : j % 3;
+      int Dk = pow3(k);
+      for (int f = 0; f < Dk; ++f) {
+        unflat(k, f, idx);
+        double s = 0.0;
+        for (int s1 = 0; s1 < k; ++s1) {
+          if (idx[s1] != di) continue;
+          if (order == 1) {
+            double p = 1.0;
+            for (int t = 0; t < k; ++t)
+              if (t != s1) p *= u[idx[t]];
+            s += p;
+          } else {
+            for (int s2 = 0; s2 < k; ++s2) {
+              if (s2 == s1 || idx[s2] != dj) continue;
+              double p = 1.0;
+              for (int t = 0; t < k; ++t)
+                if (t != s1 && t != s2) p *= u[idx[t]];
+              s += p;
+            }
+          }
+        }
+        Pw[f] = s;
+      }
+      outer_delta(k, Pw, m, P);
+      orc_permavg(l, P, A);
+      for (int f = 0; f < D; ++f) acc[j][f] += c * A[f];
+    }
+  }
+  for (int j = 0; j < nd; ++j) orc_stf_extract(l, acc[j], order == 1 ? d1[j] : d2[j]);
+}
+
 /* d T_l(r/|r|) / d r as a (2l+1) x 3 matrix, by the product rule on the
  * outer powers and the chain rule through u = r/|r|:
  * du/dr = (I - u u^T)/|r|. */
 void orc_direction_jac(int l, const double *r, double *jac) {
   double u[3], nr = sqrt(r[0] * r[0] + r[1] * r[1] + r[2] * r[2]);
   unit(r, u);
-  int D = pow3(l), idx[ORC_MAXL];
-  double dT[3][ORC_MAXD];
-  double Pw[ORC_MAXD], P[ORC_MAXD], A[ORC_MAXD];
-  double pre = dfact(2 * l - 1) / fact(l);
-  for (int j = 0; j < 3; ++j)
-    for (int f = 0; f < D; ++f) dT[j][f] = 0.0;
-  for (int m = 0; 2 * m <= l; ++m) {
-    int k = l - 2 * m;
-    double c = pre * ((m & 1) ? -1.0 : 1.0) * dfact(2 * l - 2 * m - 1) /
-               dfact(2 * l - 1) * count_delta_placements(l, m);
-    for (int j = 0; j < 3; ++j) {
-      /* derivative of prod_t u[idx_t] w.r.t. u_j */
-      int Dk = pow3(k);
-      for (int f = 0; f < Dk; ++f) {
-        unflat(k, f, idx);
-        double s = 0.0;
-        for (int sl = 0; sl < k; ++sl) {
-          if (idx[sl] != j) continue;
-          double p = 1.0;
-          for (int t = 0; t < k; ++t)
-            if (t != sl) p *= u[idx[t]];
-          s += p;
-        }
-        Pw[f] = s;
-      }
-      outer_delta(k, Pw, m, P);
-      orc_permavg(l, P, A);
-      for (int f = 0; f < D; ++f) dT[j][f] += c * A[f];
-    }
-  }
-  /* chain rule */
+  double comps[3][2 * ORC_MAXL + 1];
+  direction_du(l, u, 1, comps, NULL);
   double proj[3][3];
   for (int a = 0; a < 3; ++a)
     for (int b = 0; b < 3; ++b)
       proj[a][b] = ((a == b) ? 1.0 : 0.0) - u[a] * u[b];
-  double comps[3][2 * ORC_MAXL + 1];
-  for (int j = 0; j < 3; ++j) orc_stf_extract(l, dT[j], comps[j]);
   for (int c = 0; c < 2 * l + 1; ++c)
     for (int b = 0; b < 3; ++b) {
       double s = 0.0;
       for (int j = 0; j < 3; ++j) s += comps[j][c] * proj[j][b];
       jac[c * 3 + b] = s / nr;
     }
+}
+
+/* Hessian-vector product of F(r) = <ybar, T_l(r/|r|)> (ybar: 2l+1 weights of
+ * the components): out = (d^2 F / dr dr) v.  With u = r/|r|, P = I - u u^T,
+ * G = dF/du, H_u = d^2 F / du du and the gradient dF/dr = P G / |r|,
+ * differentiating along r + t v (du/dt = P v/|r| =: w, d|r|/dt = u.v,
+ * dP/dt = -(w u^T + u w^T)) gives
+ *   out = [-(w (u.G) + u (w.G)) + P H_u w] / |r| - P G (u.v) / |r|^2. */
+void orc_direction_hvp(int l, const double *r, const double *ybar,
+                       const double *v, double *out) {
+  double u[3], nr = sqrt(r[0] * r[0] + r[1] * r[1] + r[2] * r[2]);
+  unit(r, u);
+  double d1[3][2 * ORC_MAXL + 1], d2[9][2 * ORC_MAXL + 1];
+  direction_du(l, u, 1, d1, NULL);
+  direction_du(l, u, 2, NULL, d2);
+  double G[3], Hu[3][3];
+  for (int i = 0; i < 3; ++i) {
+    G[i] = 0.0;
+    for (int c = 0; c < 2 * l + 1; ++c) G[i] += ybar[c] * d1[i][c];
+    for (int j = 0; j < 3; ++j) {
+      Hu[i][j] = 0.0;
+      for (int c = 0; c < 2 * l + 1; ++c) Hu[i][j] += ybar[c] * d2[3 * i + j][c];
+    }
+  }
+  double uv = u[0] * v[0] + u[1] * v[1] + u[2] * v[2];
+  double w[3], PG[3], Hw[3];
+  for (int i = 0; i < 3; ++i) w[i] = (v[i] - u[i] * uv) / nr;
+  double uG = u[0] * G[0] + u[1] * G[1] + u[2] * G[2];
+  double wG = w[0] * G[0] + w[1] * G[1] + w[2] * G[2];
+  for (int i = 0; i < 3; ++i) {
+    PG[i] = G[i] - u[i] * uG;
+    Hw[i] = Hu[i][0] * w[0] + Hu[i][1] * w[1] + Hu[i][2] * w[2];
+  }
+  double uHw = u[0] * Hw[0] + u[1] * Hw[1] + u[2] * Hw[2];
+  for (int i = 0; i < 3; ++i)
+    out[i] = (-(w[i] * uG + u[i] * wG) + Hw[i] - u[i] * uHw) / nr - PG[i] * uv / (nr * nr);
 }
 
 /* ------------------------------------------------------------------ */
@@ -724,6 +783,171 @@ int orc_edge_conv_vjp(int lin, int ledge, int lout, int C, int sum_paths,
   }
   for (int p = 0; p < ps.P; ++p) free(K[p]);
   free(y);
+  return 0;
+}
+
+/* ------------------------------------------------------------------ */
+/* VJP-of-VJP of the edge convolution (App. C Eq. C2, Algorithm 3)       */
+/* ------------------------------------------------------------------ */
+
+/* Gradients of  Lv = <vx, x_bar> + <vw, w_bar> + <vr, r_bar>  (x_bar, w_bar,
+ * r_bar the VJP of orc_edge_conv_vjp for the incoming gradient g) with
+ * respect to g, x, w and the edge vectors.  Per edge, path and channel, with
+ * y the direction tensors and vy = (d y / d r) vr their derivative along vr
+ * (the cotangent of y_bar):
+ *   g_hat  += w [f(vx, y) + f(x, vy)] + vw f(x, y)      (summed per receiver)
+ *   x_hat  += VJP1(g, w vy + vw y)                      (summed per sender)
+ *   w_hat   = <g, f(vx, y) + f(x, vy)>
+ *   y_hat  += VJP2(g, w vx + vw x)
+ * and, through the direction tensors,
+ *   r_hat   = (d y / d r)^T y_hat + (d^2 <y_bar, y> / dr dr) vr
+ * with y_bar = sum w VJP2(g, x) the edge's first-order direction gradient.
+ * vx, vw, vr may be NULL (zero cotangent); outputs may be NULL (skipped).
+ * With edge_mask only the listed edges contribute (others' w_hat, r_hat 0). */
+int orc_edge_conv_vjp2(int lin, int ledge, int lout, int C, int sum_paths,
+                       int N, int E, const int32_t *recv, const int32_t *send,
+                       const double *vec, const double *x, const double *w,
+                       const double *g, const double *vx, const double *vw,
+                       const double *vr, const unsigned char *edge_mask,
+                       double *g_hat, double *x_hat, double *w_hat,
+                       double *r_hat) {
+  if (lin > 4 || ledge > 4 || lout > 4) return 1;
+  path_set ps;
+  make_paths(lin, ledge, lout, sum_paths, &ps);
+  int xrow = (lin + 1) * (lin + 1);
+  int yrow = (ledge + 1) * (ledge + 1);
+  double *K[ORC_MAXP];
+  for (int p = 0; p < ps.P; ++p) {
+    int n1 = 2 * ps.l1[p] + 1, n2 = 2 * ps.l2[p] + 1, n3 = 2 * ps.l3[p] + 1;
+    K[p] = (double *)malloc(sizeof(double) * n1 * n2 * n3);
+    orc_path_coeffs(ps.l1[p], ps.l2[p], ps.l3[p], K[p]);
+  }
+  /* direction tensors and their derivative along vr, per edge */
+  size_t En = (size_t)(E > 0 ? E : 1);
+  double *y = (double *)malloc(sizeof(double) * En * yrow);
+  double *vy = (double *)malloc(sizeof(double) * En * yrow);
+  for (int e = 0; e < E; ++e)
+    for (int l = 0; l <= ledge; ++l) {
+      orc_direction(l, vec + 3 * e, y + (size_t)e * yrow + l * l);
+      double jac[(2 * ORC_MAXL + 1) * 3];
+      orc_direction_jac(l, vec + 3 * e, jac);
+      for (int c = 0; c < 2 * l + 1; ++c) {
+        double t = 0.0;
+        if (vr)
+          for (int b = 0; b < 3; ++b) t += jac[c * 3 + b] * vr[3 * e + b];
+        vy[(size_t)e * yrow + l * l + c] = t;
+      }
+    }
+  if (g_hat) memset(g_hat, 0, sizeof(double) * (size_t)N * ps.zrow * C);
+  if (x_hat) memset(x_hat, 0, sizeof(double) * (size_t)N * xrow * C);
+  if (w_hat) memset(w_hat, 0, sizeof(double) * (size_t)E * ps.P * C);
+
+  /* g_hat, x_hat, w_hat: channels are independent */
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int k = 0; k < C; ++k) {
+    double gc[2 * ORC_MAXL + 1], xc[2 * ORC_MAXL + 1], vxc[2 * ORC_MAXL + 1];
+    double fxy[2 * ORC_MAXL + 1], sv[2 * ORC_MAXL + 1], zc[2 * ORC_MAXL + 1];
+    for (int e = 0; e < E; ++e) {
+      if (edge_mask && !edge_mask[e]) continue;
+      int u = recv[e], v = send[e];
+      for (int p = 0; p < ps.P; ++p) {
+        int l1 = ps.l1[p], l2 = ps.l2[p], l3 = ps.l3[p];
+        int n1 = 2 * l1 + 1, n2 = 2 * l2 + 1, n3 = 2 * l3 + 1;
+        int slot[2 * ORC_MAXL + 1];
+        for (int c = 0; c < n3; ++c) {
+          slot[c] = sum_paths ? ps.zoff[l3] + c : ps.zoff[l3] + c * ps.Pl[l3] + ps.eta[p];
+          gc[c] = g[((size_t)u * ps.zrow + slot[c]) * C + k];
+        }
+        for (int c = 0; c < n1; ++c) {
+          xc[c] = x[((size_t)v * xrow + l1 * l1 + c) * C + k];
+          vxc[c] = vx ? vx[((size_t)v * xrow + l1 * l1 + c) * C + k] : 0.0;
+        }
+        const double *ye = y + (size_t)e * yrow + l2 * l2;
+        const double *vye = vy + (size_t)e * yrow + l2 * l2;
+        size_t wi = ((size_t)e * ps.P + p) * C + k;
+        double wk = w[wi], vwk = vw ? vw[wi] : 0.0;
+        const double *Kp = K[p];
+        /* f(x, y) and s = f(vx, y) + f(x, vy) */
+        for (int a = 0; a < n3; ++a) {
+          double t0 = 0.0, t1 = 0.0;
+          for (int b1 = 0; b1 < n1; ++b1)
+            for (int b2 = 0; b2 < n2; ++b2) {
+              double kk = Kp[(a * n1 + b1) * n2 + b2];
+              t0 += kk * xc[b1] * ye[b2];
+              t1 += kk * (vxc[b1] * ye[b2] + xc[b1] * vye[b2]);
+            }
+          fxy[a] = t0;
+          sv[a] = t1;
+        }
+        if (g_hat)
+          for (int a = 0; a < n3; ++a)
+            g_hat[((size_t)u * ps.zrow + slot[a]) * C + k] += wk * sv[a] + vwk * fxy[a];
+        if (w_hat) {
+          double t = 0.0;
+          for (int a = 0; a < n3; ++a) t += gc[a] * sv[a];
+          w_hat[wi] = t;
+        }
+        if (x_hat) {
+          for (int b2 = 0; b2 < n2; ++b2) zc[b2] = wk * vye[b2] + vwk * ye[b2];
+          for (int b1 = 0; b1 < n1; ++b1) {
+            double t = 0.0;
+            for (int a = 0; a < n3; ++a)
+              for (int b2 = 0; b2 < n2; ++b2)
+                t += gc[a] * Kp[(a * n1 + b1) * n2 + b2] * zc[b2];
+            x_hat[((size_t)v * xrow + l1 * l1 + b1) * C + k] += t;
+          }
+        }
+      }
+    }
+  }
+
+  /* r_hat: edges are independent */
+  if (r_hat) {
+#pragma omp parallel for schedule(dynamic, 16)
+    for (int e = 0; e < E; ++e) {
+      r_hat[3 * e] = r_hat[3 * e + 1] = r_hat[3 * e + 2] = 0.0;
+      if (edge_mask && !edge_mask[e]) continue;
+      int u = recv[e], v = send[e];
+      double yh[(ORC_MAXL + 1) * (ORC_MAXL + 1)], yb[(ORC_MAXL + 1) * (ORC_MAXL + 1)];
+      for (int i = 0; i < yrow; ++i) yh[i] = yb[i] = 0.0;
+      for (int k = 0; k < C; ++k)
+        for (int p = 0; p < ps.P; ++p) {
+          int l1 = ps.l1[p], l2 = ps.l2[p], l3 = ps.l3[p];
+          int n1 = 2 * l1 + 1, n2 = 2 * l2 + 1, n3 = 2 * l3 + 1;
+          size_t wi = ((size_t)e * ps.P + p) * C + k;
+          double wk = w[wi], vwk = vw ? vw[wi] : 0.0;
+          const double *Kp = K[p];
+          for (int b2 = 0; b2 < n2; ++b2) {
+            double th = 0.0, tb = 0.0;
+            for (int a = 0; a < n3; ++a) {
+              int slot = sum_paths ? ps.zoff[l3] + a : ps.zoff[l3] + a * ps.Pl[l3] + ps.eta[p];
+              double ga = g[((size_t)u * ps.zrow + slot) * C + k];
+              for (int b1 = 0; b1 < n1; ++b1) {
+                size_t xi = ((size_t)v * xrow + l1 * l1 + b1) * C + k;
+                double kg = ga * Kp[(a * n1 + b1) * n2 + b2];
+                th += kg * (wk * (vx ? vx[xi] : 0.0) + vwk * x[xi]);
+                tb += kg * wk * x[xi];
+              }
+            }
+            yh[l2 * l2 + b2] += th;
+            yb[l2 * l2 + b2] += tb;
+          }
+        }
+      for (int l = 0; l <= ledge; ++l) {
+        double jac[(2 * ORC_MAXL + 1) * 3], hv[3];
+        orc_direction_jac(l, vec + 3 * e, jac);
+        for (int c = 0; c < 2 * l + 1; ++c)
+          for (int b = 0; b < 3; ++b) r_hat[3 * e + b] += yh[l * l + c] * jac[c * 3 + b];
+        if (vr && l > 0) {
+          orc_direction_hvp(l, vec + 3 * e, yb + l * l, vr + 3 * e, hv);
+          for (int b = 0; b < 3; ++b) r_hat[3 * e + b] += hv[b];
+        }
+      }
+    }
+  }
+  for (int p = 0; p < ps.P; ++p) free(K[p]);
+  free(y);
+  free(vy);
   return 0;
 }
 

@@ -40,6 +40,9 @@ def lib():
             "orc_paths": (ct.c_int, [ct.c_int] * 3 + [ip, ip, ip]),
             "orc_edge_conv": (ct.c_int, [ct.c_int] * 7 + [i32, i32, d, d, d, u8, d]),
             "orc_edge_conv_vjp": (ct.c_int, [ct.c_int] * 7 + [i32, i32, d, d, d, d, u8, d, d, d]),
+            "orc_edge_conv_vjp2": (ct.c_int, [ct.c_int] * 7 + [i32, i32, d, d, d, d, d, d, d, u8,
+                                                               d, d, d, d]),
+            "orc_direction_hvp": (None, [ct.c_int, d, d, d, d]),
             "orc_ladder": (ct.c_int, [ct.c_int] * 4 + [d, d, d, u8, d, d]),
             "orc_ladder_vjp": (ct.c_int, [ct.c_int] * 4 + [d, d, d, d, u8, d, d, d]),
             "orc_max_rank": (ct.c_int, []),
@@ -139,6 +142,14 @@ def direction_jac(l, r):
     out = np.empty((2 * l + 1) * 3)
     lib().orc_direction_jac(l, _pd(r), _pd(out))
     return out.reshape(2 * l + 1, 3)
+
+
+def direction_hvp(l, r, ybar, v):
+    """(d^2 <ybar, T_l(r/|r|)> / dr dr) v, exact (App. C, derivatives of the
+    direction tensors used in force training)."""
+    out = np.empty(3)
+    lib().orc_direction_hvp(l, _pd(_d(r)), _pd(_d(ybar)), _pd(_d(v)), _pd(out))
+    return out
 
 
 def admissible(l1, l2, l3):
@@ -257,6 +268,52 @@ def edge_conv_vjp(lin, ledge, lout, C, edge_index, edge_vec, x, w, g, n_nodes,
         if rb is not None:
             full = np.zeros((E_full, 3)); full[sel] = rb; rb = full
     return xb, wb, rb
+
+
+def edge_conv_vjp_vjp(lin, ledge, lout, C, edge_index, edge_vec, x, w, g, vx, vw, vr,
+                      n_nodes, sum_paths=False, edge_mask=None, want=("g", "x", "w", "r")):
+    """VJP-of-VJP (App. C Eq. C2, Algorithm 3): gradients of
+    <vx, x_bar> + <vw, w_bar> + <vr, r_bar> with respect to (g, x, w, edge
+    vectors), where (x_bar, w_bar, r_bar) = edge_conv_vjp(...).  vx, vw, vr
+    may be None (zero cotangent).  With edge_mask only the listed edges
+    contribute; w_hat / r_hat rows of the other edges are zero."""
+    ei_full = np.asarray(edge_index)
+    E_full = ei_full.shape[1]
+    P = len(paths(lin, ledge, lout))
+    sel = None
+    ei, ev, ww = ei_full, np.asarray(edge_vec), np.asarray(w)
+    vww = None if vw is None else np.asarray(vw)
+    vrr = None if vr is None else np.asarray(vr)
+    if edge_mask is not None:
+        sel = np.nonzero(_mask(edge_mask, E_full))[0]
+        ei, ev, ww = ei[:, sel], ev[sel], ww[sel]
+        vww = None if vww is None else vww[sel]
+        vrr = None if vrr is None else vrr[sel]
+    ei = np.ascontiguousarray(ei, dtype=np.int32)
+    E = ei.shape[1]
+    recv = np.ascontiguousarray(ei[0])
+    send = np.ascontiguousarray(ei[1])
+    vec = _d(ev).reshape(E, 3)
+    x, ww, g = _d(x), _d(ww).reshape(E, P, C), _d(g)
+    vx = None if vx is None else _d(vx)
+    vww = None if vww is None else _d(vww).reshape(E, P, C)
+    vrr = None if vrr is None else _d(vrr).reshape(E, 3)
+    zrow = g.shape[1] // C
+    gh = np.empty((n_nodes, zrow * C)) if "g" in want else None
+    xh = np.empty((n_nodes, (lin + 1) ** 2 * C)) if "x" in want else None
+    wh = np.empty((E, P, C)) if "w" in want else None
+    rh = np.empty((E, 3)) if "r" in want else None
+    rc = lib().orc_edge_conv_vjp2(lin, ledge, lout, C, int(sum_paths), n_nodes, E,
+                                  _pi32(recv), _pi32(send), _pd(vec), _pd(x), _pd(ww),
+                                  _pd(g), _pd(vx), _pd(vww), _pd(vrr), None,
+                                  _pd(gh), _pd(xh), _pd(wh), _pd(rh))
+    assert rc == 0
+    if sel is not None:
+        if wh is not None:
+            full = np.zeros((E_full, P, C)); full[sel] = wh; wh = full
+        if rh is not None:
+            full = np.zeros((E_full, 3)); full[sel] = rh; rh = full
+    return gh, xh, wh, rh
 
 
 # --------------------------------------------------------------------------
