@@ -18,6 +18,10 @@ template <int L, int G, int g>
 struct VjpGroup;
 template <int L>
 struct VjpMeta;
+template <int L, int G, int g>
+struct VvjpGroup;
+template <int L>
+struct VvjpMeta;
 template <int L>
 struct LadderTP;
 

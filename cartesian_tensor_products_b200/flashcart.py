@@ -67,6 +67,7 @@ _SIGS = {
     "fc_product_ladder_vjp": (ct.c_int, [ct.POINTER(LadderDesc), ct.c_int, _vp, _vp, _vp, _vp,
                                          _vp, _vp, _vp, _vp, _vp, ct.c_size_t, _vp]),
     "fc_device_error": (ct.c_int, [ct.POINTER(ct.c_int), _vp]),
+    "fc_edge_conv_vjp_vjp": (ct.c_int, [ct.POINTER(ConvDesc), ct.c_int, ct.c_int] + [_vp] * 14),
 }
 for _name, (_res, _args) in _SIGS.items():
     _f = getattr(_lib, _name)
@@ -215,6 +216,37 @@ def edge_conv_vjp(lmax, rowptr, edge_index, edge_vec, x, w, g, sum_paths=False,
                                  _ptr(edge_vec), _ptr(x), _ptr(w), _ptr(g), _ptr(xb),
                                  _ptr(wb), _ptr(rb), _stream(stream)), "fc_edge_conv_vjp")
     return xb, wb, rb
+
+
+def edge_conv_vjp_vjp(lmax, rowptr, edge_index, edge_vec, x, w, g, v_x=None, v_w=None,
+                      v_r=None, sum_paths=False, want=("g", "x", "w", "r"), stream=None):
+    """(g_hat, x_hat, w_hat, r_hat) of App. C Eq. C2 (Algorithm 3): the
+    gradients of <v_x, x_bar> + <v_w, w_bar> + <v_r, r_bar> with respect to
+    g, x, w and the edge vectors; None cotangents are zero, outputs not in
+    `want` are None."""
+    for t, n in ((x, "x"), (g, "g")):
+        _dev(t, torch.float32, n)
+    _dev(rowptr, torch.int32, "rowptr")
+    _dev(edge_index, torch.int32, "edge_index")
+    for t, n in ((v_x, "v_x"), (v_w, "v_w"), (v_r, "v_r")):
+        if t is not None:
+            _dev(t, torch.float32, n)
+    N = rowptr.shape[0] - 1
+    E = edge_index.shape[1]
+    C = x.shape[1] // ((lmax + 1) ** 2)
+    d = conv_desc(lmax, C, sum_paths)
+    P = num_paths(lmax)
+    if g.shape != (N, out_row(lmax, C, sum_paths) * C):
+        raise ValueError("g shape %s" % (tuple(g.shape),))
+    gh = torch.empty_like(g) if "g" in want else None
+    xh = torch.empty_like(x) if "x" in want else None
+    wh = torch.empty((E, P, C), dtype=torch.float32, device=x.device) if "w" in want else None
+    rh = torch.empty((E, 3), dtype=torch.float32, device=x.device) if "r" in want else None
+    _check(_lib.fc_edge_conv_vjp_vjp(ct.byref(d), N, E, _ptr(rowptr), _ptr(edge_index),
+                                     _ptr(edge_vec), _ptr(x), _ptr(w), _ptr(g), _ptr(v_x),
+                                     _ptr(v_w), _ptr(v_r), _ptr(gh), _ptr(xh), _ptr(wh),
+                                     _ptr(rh), _stream(stream)), "fc_edge_conv_vjp_vjp")
+    return gh, xh, wh, rh
 
 
 def _workspace(nbytes, device):

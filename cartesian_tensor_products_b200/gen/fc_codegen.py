@@ -716,6 +716,286 @@ def emit_vjp(L, G):
     return "\n".join(out) + "\n", T, codes
 
 
+# ---------------------------------------------------------------------------
+# receiver-sorted VJP-of-VJP (App. C Eq. C2, Algorithm 3)
+# ---------------------------------------------------------------------------
+
+D2_PAIRS = ((0, 0), (0, 1), (0, 2), (1, 1), (1, 2), (2, 2))
+
+
+def direction_second_derivative_polys(l):
+    """d^2 T_l(u)_c / d u_i d u_j for the symmetric pairs D2_PAIRS."""
+    return [[A.p_diff(A.p_diff(poly, i), j) for (i, j) in D2_PAIRS]
+            for poly in A.direction_polys(l)]
+
+
+def vvjp_path_cost(T, p):
+    l1, l2, l3 = T.paths[p]
+    nm = sum(len(T.mrow(p, a)) for a in range(2 * l3 + 1))
+    nk = sum(1 for a in range(2 * l3 + 1) for b1 in range(2 * l1 + 1)
+             for b2 in range(2 * l2 + 1) if T.K[p][a][b1][b2] != 0)
+    return 6 * nm + 8 * (2 * l1 + 1) + (4 * nk if l2 > 0 else 0)
+
+
+class VvjpGroupCode:
+    """Straight-line code of one warp group of the VJP-of-VJP kernel (whole
+    paths).  Per edge, path and lane (4 channels), with M = M(y) and
+    Mv = M(vy) the per-edge matrices of the direction tensors and of their
+    derivative along the edge-vector cotangent:
+      t = w vx + vw x,  s = w x
+      h = M^T g,  hv = Mv^T g
+      g_hat += M t + Mv s                      (= w[f(vx,y) + f(x,vy)] + vw f(x,y))
+      w_hat  = <h, vx> + <hv, x>               (= <g, f(vx,y) + f(x,vy)>)
+      x_hat += w hv + vw h                     (= VJP1(g, w vy + vw y))
+      y_hat += K-contraction of <g, t>          (= VJP2(g, w vx + vw x))
+      y_bar += K-contraction of <g, s>          (= VJP2(g, w x), for the Hessian term)."""
+
+    def __init__(self, T, paths, gid):
+        self.T, self.gpaths, self.gid = T, paths, gid
+        self.rows = [(p, a) for p in paths for a in range(2 * T.paths[p][2] + 1)]
+        self.NA = len(self.rows)
+        self.xrows = sorted(set(T.paths[p][0] ** 2 + b for p in paths
+                                for b in range(2 * T.paths[p][0] + 1)))
+        self.NX = len(self.xrows)
+        self.NP = len(paths)
+        self.ment = [(p, a, b1, terms) for p in paths for a in range(2 * T.paths[p][2] + 1)
+                     for b1, terms in T.mrow(p, a)]
+        self.NM = len(self.ment)
+        # direction components with an angular derivative (T_0 = 1 has none)
+        self.dcomps = sorted(set((T.paths[p][1], b2) for p in paths if T.paths[p][1] > 0
+                                 for b2 in range(2 * T.paths[p][1] + 1)))
+        self.ND = len(self.dcomps)
+        self.NROW = 2 * self.NX + 2 * self.NP
+        self.dbase = (2 * self.NM + 3) // 4 * 4      # d y / d u of dcomps (3 each)
+        self.d2base = self.dbase + 3 * self.ND      # d^2 y / du du (6 each)
+        self.sbase = self.d2base + 6 * self.ND      # ux uy uz wx wy wz inv_r u.vr
+        n = self.sbase + 8
+        q = max(1, (n + 3) // 4)
+        if q % 2 == 0:
+            q += 1
+        self.MSTRIDE = 4 * q
+
+    def emit(self, L, G):
+        T = self.T
+        o = []
+        o.append("template <> struct VvjpGroup<%d, %d, %d> {" % (L, G, self.gid))
+        o.append("  static constexpr int NA = %d;    // g rows (and g_hat rows) in registers" % self.NA)
+        o.append("  static constexpr int NX = %d;    // x rows (and vx rows) staged per edge" % self.NX)
+        o.append("  static constexpr int NP = %d;    // paths (w and vw rows staged per edge)" % self.NP)
+        o.append("  static constexpr int NROW = %d;  // staged 512-byte rows per edge" % self.NROW)
+        o.append("  static constexpr int NM = %d;    // entries of M (and of Mv) per edge" % self.NM)
+        o.append("  static constexpr int ND = %d;    // direction components with a derivative" % self.ND)
+        o.append("  static constexpr int SBASE = %d; // per-edge scalars in the window row" % self.sbase)
+        o.append("  static constexpr int MSTRIDE = %d;" % self.MSTRIDE)
+        o.append("  static constexpr int RING_OFF = %d;" % self.ring_off)
+        o.append("  static constexpr int MWIN_OFF = %d;" % self.mwin_off)
+        # ---- window row
+        o.append("  static __device__ __forceinline__ void make_row(float ux, float uy, float uz, float inv_r, float vrx, float vry, float vrz, float* __restrict__ mrow) {")
+        yneed = set()
+        for (p, a, b1, terms) in self.ment:
+            for b2 in terms:
+                yneed.add((T.paths[p][1], b2))
+        dneed = sorted(set(self.dcomps) | set(c for c in yneed if c[0] > 0))
+        for (l2, b2) in sorted(yneed):
+            o.append("    const float y_%d_%d = %s;" % (l2, b2, poly_expr(T.ypoly[l2][b2]) if l2 else "1.0f"))
+        for (l2, b2) in dneed:
+            d = direction_derivative_polys(l2)[b2]
+            for j in range(3):
+                o.append("    const float d_%d_%d_%d = %s;" % (l2, b2, j, poly_expr(d[j])))
+        o.append("    const float uv = ux * vrx + uy * vry + uz * vrz;")
+        o.append("    const float wx = (vrx - ux * uv) * inv_r, wy = (vry - uy * uv) * inv_r, wz = (vrz - uz * uv) * inv_r;")
+        for (l2, b2) in sorted(yneed):
+            if l2:
+                o.append("    const float vy_%d_%d = d_%d_%d_0 * wx + d_%d_%d_1 * wy + d_%d_%d_2 * wz;" %
+                         (l2, b2, l2, b2, l2, b2, l2, b2))
+            else:
+                o.append("    const float vy_%d_%d = 0.0f;" % (l2, b2))
+        vals = []
+        for (p, a, b1, terms) in self.ment:
+            l2 = T.paths[p][1]
+            vals.append(lincomb_expr(terms, lambda b, l2=l2: "y_%d_%d" % (l2, b)))
+        for (p, a, b1, terms) in self.ment:
+            l2 = T.paths[p][1]
+            vals.append(lincomb_expr(terms, lambda b, l2=l2: "vy_%d_%d" % (l2, b)))
+        while len(vals) < self.dbase:
+            vals.append("0.0f")
+        for (l2, b2) in self.dcomps:
+            for j in range(3):
+                vals.append("d_%d_%d_%d" % (l2, b2, j))
+        for (l2, b2) in self.dcomps:
+            for e in direction_second_derivative_polys(l2)[b2]:
+                vals.append(poly_expr(e))
+        vals += ["ux", "uy", "uz", "wx", "wy", "wz", "inv_r", "uv"]
+        while len(vals) % 4:
+            vals.append("0.0f")
+        for q in range(len(vals) // 4):
+            o.append("    st_f4(mrow + %d, %s, %s, %s, %s);" % (4 * q, *vals[4 * q:4 * q + 4]))
+        o.append("  }")
+        # ---- staging
+        o.append("  static __device__ __forceinline__ void issue(float* st, const float* __restrict__ xv, const float* __restrict__ vxv,")
+        o.append("      const float* __restrict__ we, const float* __restrict__ vwe, int C, bool xok, bool vxok, bool ok, bool vwok) {")
+        for i, r in enumerate(self.xrows):
+            o.append("    cp_async16(st + %d, xv + %d * C, xok);" % (128 * i, r))
+        for i, r in enumerate(self.xrows):
+            o.append("    cp_async16(st + %d, vxv + %d * C, vxok);" % (128 * (self.NX + i), r))
+        for i, p in enumerate(self.gpaths):
+            o.append("    cp_async16(st + %d, we + %d * C, ok);" % (128 * (2 * self.NX + i), p))
+        for i, p in enumerate(self.gpaths):
+            o.append("    cp_async16(st + %d, vwe + %d * C, vwok);" % (128 * (2 * self.NX + self.NP + i), p))
+        o.append("  }")
+        # ---- g rows of the receiver
+        o.append("  static __device__ __forceinline__ void load_g(const float* __restrict__ gu, int C, int sum_paths, float4 (&gr)[NA]) {")
+        o.append("    if (!sum_paths) {")
+        for i, (p, a) in enumerate(self.rows):
+            o.append("      gr[%d] = ld_x4(gu + %d * C);" % (i, T.zslot(p, a)))
+        o.append("    } else {")
+        for i, (p, a) in enumerate(self.rows):
+            o.append("      gr[%d] = ld_x4(gu + %d * C);" % (i, T.zslot(p, a, True)))
+        o.append("    }")
+        o.append("  }")
+        # ---- g_hat rows of the receiver (added: with summed paths several
+        # groups share a slot)
+        o.append("  static __device__ __forceinline__ void store_ghat(float* __restrict__ gu, int C, int sum_paths, const float4 (&gh)[NA]) {")
+        o.append("    if (!sum_paths) {")
+        for i, (p, a) in enumerate(self.rows):
+            o.append("      red_add4(gu + %d * C, gh[%d]);" % (T.zslot(p, a), i))
+        o.append("    } else {")
+        for i, (p, a) in enumerate(self.rows):
+            o.append("      red_add4(gu + %d * C, gh[%d]);" % (T.zslot(p, a, True), i))
+        o.append("    }")
+        o.append("  }")
+        # ---- one edge
+        xidx = {r: i for i, r in enumerate(self.xrows)}
+        gi = {r: i for i, r in enumerate(self.rows)}
+        dix = {c: i for i, c in enumerate(self.dcomps)}
+        NDm = max(1, self.ND)
+        o.append("  static __device__ __forceinline__ void edge(const float4 (&gr)[NA], float4 (&gh)[NA], const float* st,")
+        o.append("      const float* __restrict__ m, float4 (&xh)[NX], float (&yh)[%d], float (&yb)[%d]," % (NDm, NDm))
+        o.append("      float* __restrict__ what_e, int C, bool wstore) {")
+        for i, r in enumerate(self.xrows):
+            o.append("    const float4 x%d = ld_s4(st + %d);" % (r, 128 * i))
+            o.append("    const float4 vx%d = ld_s4(st + %d);" % (r, 128 * (self.NX + i)))
+        mi = 0
+        loaded = set()
+
+        def mname(k):
+            q, c = divmod(k, 4)
+            return "mq%d.%s" % (q, "xyzw"[c])
+
+        for pi, p in enumerate(self.gpaths):
+            l1, l2, l3 = T.paths[p]
+            ents = [(a, b1, terms) for (pp, a, b1, terms) in self.ment if pp == p]
+            bset = sorted(set(b for _, b, _ in ents))
+            # the path's window quads, loaded at function scope just before their
+            # first use (a quad can span two paths)
+            ks = list(range(mi, mi + len(ents))) + list(range(self.NM + mi, self.NM + mi + len(ents)))
+            for q in sorted(set(k // 4 for k in ks)):
+                if q not in loaded:
+                    o.append("    const float4 mq%d = ld_s4(m + %d);" % (q, 4 * q))
+                    loaded.add(q)
+            o.append("    { // path (%d,%d)->%d" % (l1, l2, l3))
+            names = [mname(mi + k) for k in range(len(ents))]
+            vnames = [mname(self.NM + mi + k) for k in range(len(ents))]
+            mi += len(ents)
+            o.append("      const float4 w = ld_s4(st + %d);" % (128 * (2 * self.NX + pi)))
+            o.append("      const float4 vw = ld_s4(st + %d);" % (128 * (2 * self.NX + self.NP + pi)))
+            for b in bset:
+                r = l1 * l1 + b
+                o.append("      const float4 t%d = fma4(w, vx%d, mul4(vw, x%d));" % (b, r, r))
+                o.append("      const float4 s%d = mul4(w, x%d);" % (b, r))
+            started = set()
+            for k, (a, b, _) in enumerate(ents):
+                ga = "gr[%d]" % gi[(p, a)]
+                if b not in started:
+                    o.append("      float4 h%d = mul4s(%s, %s);" % (b, names[k], ga))
+                    o.append("      float4 hv%d = mul4s(%s, %s);" % (b, vnames[k], ga))
+                    started.add(b)
+                else:
+                    o.append("      h%d = fma4s(%s, %s, h%d);" % (b, names[k], ga, b))
+                    o.append("      hv%d = fma4s(%s, %s, hv%d);" % (b, vnames[k], ga, b))
+                o.append("      gh[%d] = fma4s(%s, t%d, fma4s(%s, s%d, gh[%d]));" %
+                         (gi[(p, a)], names[k], b, vnames[k], b, gi[(p, a)]))
+            first = True
+            for b in bset:
+                r = l1 * l1 + b
+                if first:
+                    o.append("      float4 wh = fma4(hv%d, x%d, mul4(h%d, vx%d));" % (b, r, b, r))
+                    first = False
+                else:
+                    o.append("      wh = fma4(hv%d, x%d, fma4(h%d, vx%d, wh));" % (b, r, b, r))
+                o.append("      xh[%d] = fma4(w, hv%d, fma4(vw, h%d, xh[%d]));" % (xidx[r], b, b, xidx[r]))
+            o.append("      if (wstore) st_z4(what_e + %d * C, wh);" % p)
+            if l2 > 0:
+                for k, (a, b, terms) in enumerate(ents):
+                    o.append("      { const float dh = dot4(gr[%d], t%d), db = dot4(gr[%d], s%d);" %
+                             (gi[(p, a)], b, gi[(p, a)], b))
+                    for b2, c in sorted(terms.items()):
+                        i = dix[(l2, b2)]
+                        o.append("        yh[%d] = fmaf(%s, dh, yh[%d]); yb[%d] = fmaf(%s, db, yb[%d]);" %
+                                 (i, flit(c), i, i, flit(c), i))
+                    o.append("      }")
+            o.append("    }")
+        o.append("  }")
+        # ---- fold y_hat, y_bar into u-space: D^T y_hat (3), G = D^T y_bar (3),
+        # H_u = sum y_bar D2 (6)
+        o.append("  static __device__ __forceinline__ void fold(const float (&yh)[%d], const float (&yb)[%d], const float* __restrict__ m, float (&red)[12]) {" % (NDm, NDm))
+        o.append("#pragma unroll")
+        o.append("    for (int i = 0; i < 12; ++i) red[i] = 0.0f;")
+        for i in range(self.ND):
+            b1 = self.dbase + 3 * i
+            b2 = self.d2base + 6 * i
+            for j in range(3):
+                o.append("    red[%d] = fmaf(yh[%d], m[%d], red[%d]); red[%d] = fmaf(yb[%d], m[%d], red[%d]);" %
+                         (j, i, b1 + j, j, 3 + j, i, b1 + j, 3 + j))
+            for j in range(6):
+                o.append("    red[%d] = fmaf(yb[%d], m[%d], red[%d]);" % (6 + j, i, b2 + j, 6 + j))
+        o.append("  }")
+        # ---- x_hat rows
+        o.append("  static __device__ __forceinline__ void flush_xhat(float* __restrict__ xhv, int C, float4 (&xh)[NX]) {")
+        for i, r in enumerate(self.xrows):
+            o.append("    red_add4(xhv + %d * C, xh[%d]); xh[%d] = zero4();" % (r, i, i))
+        o.append("  }")
+        o.append("};")
+        return "\n".join(o)
+
+
+VVJP_NGROUPS = {2: 6, 3: 16, 4: 32}
+VVJP_STAGES = {2: 2, 3: 2, 4: 2}
+VVJP_MWIN = {2: 8, 3: 8, 4: 8}
+
+
+def emit_vvjp(L, G):
+    T = Tables(L)
+    groups = partition_paths(T, G, lambda p: vvjp_path_cost(T, p))
+    codes = [VvjpGroupCode(T, ps, g) for g, ps in enumerate(groups)]
+    nrow = max(c.NROW for c in codes)
+    mstride = max(c.MSTRIDE for c in codes)
+    for c in codes:
+        c.ring_off = 0
+        c.mwin_off = VVJP_STAGES[L] * 128 * nrow
+    off = VVJP_STAGES[L] * 128 * nrow + VVJP_MWIN[L] * mstride
+    out = ["// Generated by gen/fc_codegen.py -- do not edit.",
+           "// Receiver-sorted VJP-of-VJP, rank %d: %d paths, %d warp groups (whole paths)." % (L, T.P, G)]
+    for c in codes:
+        out.append("//   group %d: paths %s, %d g rows, %d M entries, %d x rows, cost %d" %
+                   (c.gid, [T.paths[p] for p in c.gpaths], c.NA, c.NM, c.NX,
+                    sum(vvjp_path_cost(T, p) for p in c.gpaths)))
+    out += ["#pragma once", '#include "../fc_device.cuh"', "namespace fc {",
+            "template <> struct VvjpMeta<%d> {" % L,
+            "  static constexpr int G = %d;" % G,
+            "  static constexpr int S = %d;" % VVJP_STAGES[L],
+            "  static constexpr int MWIN = %d;" % VVJP_MWIN[L],
+            "  static constexpr int P = %d;" % T.P,
+            "  static constexpr int WARP_FLOATS = %d;   // shared memory of one warp" % off,
+            "  static constexpr int WARPS = 4;           // receivers per CTA (same group)",
+            "  static constexpr int SMEM_FLOATS = %d;" % (4 * off),
+            "};"]
+    for c in codes:
+        out.append(c.emit(L, G))
+    out.append("}  // namespace fc")
+    return "\n".join(out) + "\n", T, codes
+
+
 _main_fwd = main
 
 
@@ -724,6 +1004,11 @@ def main():
     for L in (2, 3, 4):
         src, _, _ = emit_vjp(L, VJP_NGROUPS[L])
         path = os.path.join(OUTDIR, "fc_vjp_L%d.cuh" % L)
+        with open(path, "w") as f:
+            f.write(src)
+        written.append(path)
+        src, _, _ = emit_vvjp(L, VVJP_NGROUPS[L])
+        path = os.path.join(OUTDIR, "fc_vvjp_L%d.cuh" % L)
         with open(path, "w") as f:
             f.write(src)
         written.append(path)

@@ -166,6 +166,36 @@ int fc_edge_conv_vjp(const fc_conv_desc *desc, int n_nodes, int n_edges,
                      const float *g, float *x_bar, float *w_bar, float *r_bar,
                      fc_stream_t stream);
 
+/* VJP-of-VJP of fc_edge_conv (the derivative of fc_edge_conv_vjp), App. C
+ * Eq. (C2) summed over the receiver-sorted edges as in Algorithm 3, with the
+ * direction tensors differentiated twice (App. C, paragraph after Eq. C2).
+ * Given the incoming gradient g of fc_edge_conv and cotangents v_x, v_w,
+ * v_r of the VJP outputs x_bar, w_bar, r_bar, it returns the gradients of
+ *   <v_x, x_bar> + <v_w, w_bar> + <v_r, r_bar>
+ * with respect to g, x, w and the edge vectors:
+ *   g_hat[u,eta,k] = sum_{e: u_e = u} w (f(v_x, y) + f(x, v_y)) + v_w f(x, y)
+ *   x_hat[v, :, k] = sum_{e: v_e = v} sum_eta VJP1_eta(g, w v_y + v_w y)
+ *   w_hat[e,eta,k] = <g, f(v_x, y) + f(x, v_y)>
+ *   r_hat[e]       = (dy/dr)^T y_hat + (d^2 <y_bar, y> / dr dr) v_r,
+ *   y_hat[e]       = sum_{eta,k} VJP2_eta(g, w v_x + v_w x),
+ *   y_bar[e]       = sum_{eta,k} w VJP2_eta(g, x)   (the first VJP's y gradient)
+ * with y = T(r-hat_e), v_y = (dy/dr) v_r[e] and every f, x, v_x, g at the
+ * edge's sender, receiver and channel.
+ *   x, w, g as for fc_edge_conv_vjp; v_x like x, v_w like w, v_r
+ *   [n_edges][3]: each may be NULL for a zero cotangent.
+ *   g_hat (layout of z), x_hat (layout of x), w_hat (layout of w), r_hat
+ *   [n_edges][3]: each may be NULL to skip it.  g_hat, x_hat and r_hat are
+ *   zeroed on the stream and accumulated with atomic additions; w_hat is
+ *   written once per entry.
+ * The radial envelope is not supported here: FC_ERR_ARG if desc->envelope.
+ * Same graph requirements and other error returns as fc_edge_conv. */
+int fc_edge_conv_vjp_vjp(const fc_conv_desc *desc, int n_nodes, int n_edges,
+                         const int32_t *rowptr, const int32_t *edge_index,
+                         const float *edge_vec, const float *x, const float *w,
+                         const float *g, const float *v_x, const float *v_w,
+                         const float *v_r, float *g_hat, float *x_hat,
+                         float *w_hat, float *r_hat, fc_stream_t stream);
+
 /* Scalar readout of a node-layout array z [n_nodes][(lmax+1)^2 C]:
  *   energy[0] = sum_{n,k} z[n, rank 0, k]   (device float, overwritten)
  *   gz[n, rank 0, k] = 1, every other entry 0  (device, may be NULL)
