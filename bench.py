@@ -220,8 +220,8 @@ def time_events(fn, steps, warmup, stream, flush=None):
     return statistics.mean(times), min(times)
 
 
-ROW_NAMES = ("edge_conv_vjp_r3", "edge_conv_fwd_r4", "edge_conv_vjp_r4", "ladder",
-             "block_energy_forces")
+ROW_NAMES = ("edge_conv_vjp_r3", "edge_conv_vvjp_r3", "edge_conv_fwd_r4", "edge_conv_vjp_r4",
+             "ladder", "block_energy_forces")
 
 
 def extra_rows(fc, W, dev, stream, peaks, fp32_peak, steps, select=ROW_NAMES):
@@ -263,6 +263,32 @@ def extra_rows(fc, W, dev, stream, peaks, fp32_peak, steps, select=ROW_NAMES):
                          "frac": byt / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
                          "algorithmic_bytes": byt}}
         del out, w, g, x
+        torch.cuda.empty_cache()
+
+    if "edge_conv_vvjp_r3" in select:
+        # --- VJP-of-VJP, rank 3, microbench graph: all four outputs, all cotangents
+        wl = W.microbench_grad(lmax=3)
+        cot = W.cotangents(N, E, 3, C, 61, wl["edge_vec"])
+        x = torch.from_numpy(wl["x"]).to(dev)
+        w = torch.from_numpy(wl["w"]).to(dev)
+        g = torch.from_numpy(wl["g"]).to(dev)
+        vx = torch.from_numpy(cot["vx"]).to(dev)
+        vw = torch.from_numpy(cot["vw"]).to(dev)
+        vr = torch.from_numpy(cot["vr"]).to(dev)
+        ms, mn = time_events(lambda: fc.edge_conv_vjp_vjp(L, rp, ei, ev, x, w, g, v_x=vx, v_w=vw, v_r=vr),
+                             steps, 3, stream)
+        zr = fc.out_row(L)
+        # w, vw in; w_hat out; x, vx, g in; g_hat, x_hat out (+ zeroing); edges
+        byt = 4 * (3 * E * P * C + 2 * N * 16 * C + 2 * N * zr * C + N * 16 * C
+                   + 3 * E * 3 + E + N)
+        rows["edge_conv_vvjp_r3"] = {
+            "workload": "microbench graph, rank 3, g_hat + x_hat + w_hat + r_hat from vx, vw, vr",
+            "ms": ms, "ms_min": mn, "edge_channels_per_s": E * C / (ms * 1e-3),
+            "roofline": {"bound": "hbm", "achieved": byt / (ms * 1e-3) / 1e9,
+                         "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": byt / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                         "algorithmic_bytes": byt}}
+        del x, w, g, vx, vw, vr
         torch.cuda.empty_cache()
 
     if "edge_conv_fwd_r4" in select or "edge_conv_vjp_r4" in select:
@@ -327,22 +353,37 @@ def extra_rows(fc, W, dev, stream, peaks, fp32_peak, steps, select=ROW_NAMES):
         S = order - 1
         mix_flops = S * 2 * Nl * 16 * Cl * Cl
         tp_flops = S * Nl * Cl * 2 * 751
+        plane_b = 4 * Nl * 16 * Cl
+        tc = Cl == 128
+        # tcgen05 TF32 peak: the measured bf16 peak x the nominal tf32/bf16 ratio (1.1/2.25);
+        # the three-term split issues three TF32 products per mixing product
+        tf32_peak = peaks["bf16_tflops"] * 1.1 / 2.25
+
+        def bound(byts, fp32_fl, tf32_fl, ms):
+            t = {"hbm": byts / (peaks["hbm_gbs"] * 1e9), "fp32": fp32_fl / (fp32_peak * 1e12),
+                 "tf32": tf32_fl / (tf32_peak * 1e12)}
+            key = max(t, key=t.get)
+            return {"bound": "alu" if key != "hbm" else "hbm", "limit": key,
+                    "t_roof_us": 1e6 * t[key], "frac": t[key] / (ms * 1e-3),
+                    "terms_us": {k: 1e6 * v for k, v in t.items()},
+                    "peaks": {"hbm_gbs": peaks["hbm_gbs"], "fp32_tflops": fp32_peak,
+                              "tf32_tflops": tf32_peak},
+                    "algorithmic_flops": mix_flops + tp_flops,
+                    "algorithmic_bytes": byts}
+        # forward: A1 read, states written, z written; products FP32; mix TF32 x3 (or FP32)
+        fb = plane_b * (1 + S + 1)
         rows["ladder_fwd"] = {
             "workload": "4096 nodes x 128 channels, rank 3, order 4 (3 products + 3 per-rank 128x128 mixes)",
             "ms": msl, "ms_min": mnl,
-            "roofline": {"bound": "alu", "achieved": (mix_flops + tp_flops) / (msl * 1e-3) / 1e12,
-                         "peak": fp32_peak, "unit": "TFLOP/s",
-                         "frac": (mix_flops + tp_flops) / (msl * 1e-3) / 1e12 / fp32_peak,
-                         "algorithmic_flops": mix_flops + tp_flops},
+            "roofline": bound(fb, tp_flops + (0 if tc else mix_flops), 3 * mix_flops if tc else 0, msl),
             "l2_flush": "256 MB written before every call"}
-        vjp_flops = 3 * mix_flops + 4 * tp_flops
+        # VJP: states and A1 read, gz read, A1_bar written; products 4x, mixes 2x (B_bar, M_bar)
+        vb = plane_b * (1 + S + 1 + 1)
         rows["ladder_vjp"] = {
             "workload": "same ladder, A1_bar + path_w_bar + mix_w_bar",
             "ms": mslb, "ms_min": mnlb,
-            "roofline": {"bound": "alu", "achieved": vjp_flops / (mslb * 1e-3) / 1e12,
-                         "peak": fp32_peak, "unit": "TFLOP/s",
-                         "frac": vjp_flops / (mslb * 1e-3) / 1e12 / fp32_peak,
-                         "algorithmic_flops": vjp_flops},
+            "roofline": bound(vb, 4 * tp_flops + mix_flops + (0 if tc else mix_flops),
+                              3 * mix_flops if tc else 0, mslb),
             "l2_flush": "256 MB written before every call"}
         del A1, pw, mw, gz, ws, res, states
         torch.cuda.empty_cache()
