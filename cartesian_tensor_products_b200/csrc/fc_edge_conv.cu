@@ -22,6 +22,7 @@
 // runs one instruction stream (warp g of each resident CTA).
 #include "fc_common.cuh"
 #include "fc_device.cuh"
+#include "generated/fc_fwd_L1.cuh"
 #include "generated/fc_fwd_L2.cuh"
 #include "generated/fc_fwd_L3.cuh"
 #include "generated/fc_fwd_L4.cuh"
@@ -252,6 +253,7 @@ extern "C" int fc_edge_conv(const fc_conv_desc* d, int n_nodes, int n_edges,
       return FC_ERR_CUDA;
   }
   switch (L) {
+    case 1: return launch_fwd<1>(a, s);
     case 2: return launch_fwd<2>(a, s);
     case 3: return launch_fwd<3>(a, s);
     case 4: return launch_fwd<4>(a, s);

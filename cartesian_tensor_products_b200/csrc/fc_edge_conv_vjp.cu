@@ -27,6 +27,7 @@
 // added atomically (3 floats per warp and edge) into r_bar.
 #include "fc_common.cuh"
 #include "fc_device.cuh"
+#include "generated/fc_vjp_L1.cuh"
 #include "generated/fc_vjp_L2.cuh"
 #include "generated/fc_vjp_L3.cuh"
 #include "generated/fc_vjp_L4.cuh"
@@ -306,6 +307,7 @@ extern "C" int fc_edge_conv_vjp(const fc_conv_desc* d, int n_nodes, int n_edges,
   if (n_edges == 0) return FC_OK;
   if (!x_bar && !w_bar && !r_bar) return FC_OK;
   switch (L) {
+    case 1: return launch_vjp<1>(a, s);
     case 2: return launch_vjp<2>(a, s);
     case 3: return launch_vjp<3>(a, s);
     case 4: return launch_vjp<4>(a, s);

@@ -3,6 +3,7 @@
 #include "fc_edge_conv_vvjp.cuh"
 
 namespace fc {
+int launch_vvjp_rank1(const VvjpArgs& a, cudaStream_t s);
 int launch_vvjp_rank2(const VvjpArgs& a, cudaStream_t s);
 int launch_vvjp_rank3(const VvjpArgs& a, cudaStream_t s);
 int launch_vvjp_rank4(const VvjpArgs& a, cudaStream_t s);
@@ -68,6 +69,7 @@ extern "C" int fc_edge_conv_vjp_vjp(const fc_conv_desc* d, int n_nodes, int n_ed
   if (n_edges == 0) return FC_OK;
   if (!g_hat && !x_hat && !w_hat && !r_hat) return FC_OK;
   switch (L) {
+    case 1: return launch_vvjp_rank1(a, s);
     case 2: return launch_vvjp_rank2(a, s);
     case 3: return launch_vvjp_rank3(a, s);
     case 4: return launch_vvjp_rank4(a, s);

@@ -1,0 +1,9 @@
+// libflashcart: VJP-of-VJP of the edge convolution, rank 1 instantiation.
+#include "fc_edge_conv_vvjp.cuh"
+#include "generated/fc_vvjp_L1.cuh"
+
+namespace fc {
+int launch_vvjp_rank1(const VvjpArgs& a, cudaStream_t s) {
+  return launch_vvjp_cc<1, 0>(a, s);
+}
+}  // namespace fc

@@ -21,6 +21,7 @@
 #include "fc_common.cuh"
 #include "fc_device.cuh"
 #include "fc_tc.cuh"
+#include "generated/fc_ladder_L1.cuh"
 #include "generated/fc_ladder_L2.cuh"
 #include "generated/fc_ladder_L3.cuh"
 #include "generated/fc_ladder_L4.cuh"
@@ -361,7 +362,7 @@ static int launch_ladder_sum(size_t plane, int S, const float* A1, const float* 
 static int check_ladder_desc(const fc_ladder_desc* d) {
   if (!d) return FC_ERR_ARG;
   if (d->channels <= 0 || d->order < 1 || d->lmax < 0) return FC_ERR_ARG;
-  if (d->lmax < 2 || d->lmax > 4) return FC_ERR_UNSUPPORTED_RANK;
+  if (d->lmax < 1 || d->lmax > 4) return FC_ERR_UNSUPPORTED_RANK;
   if (d->channels % 4) return FC_ERR_ALIGN;
   return FC_OK;
 }
@@ -385,6 +386,7 @@ static int launch_tp_vjp(int N, int C, const float* Av, const float* A1, const f
 static int tp_dispatch(int L, int N, int C, const float* Av, const float* A1, const float* W,
                        float* B, cudaStream_t s) {
   switch (L) {
+    case 1: return launch_tp<1>(N, C, Av, A1, W, B, s);
     case 2: return launch_tp<2>(N, C, Av, A1, W, B, s);
     case 3: return launch_tp<3>(N, C, Av, A1, W, B, s);
     case 4: return launch_tp<4>(N, C, Av, A1, W, B, s);
@@ -396,6 +398,7 @@ static int tp_tiled_dispatch(int L, int N, const float* Av, const float* A1, con
                              const MixTiles& tiles, float* xs, cudaStream_t s) {
   const dim3 grid((N + kLadderNodeChunk - 1) / kLadderNodeChunk);
   switch (L) {
+    case 1: ladder_tp_tiled_kernel<1><<<grid, 128, 0, s>>>(N, Av, A1, W, tiles, xs); break;
     case 2: ladder_tp_tiled_kernel<2><<<grid, 128, 0, s>>>(N, Av, A1, W, tiles, xs); break;
     case 3: ladder_tp_tiled_kernel<3><<<grid, 128, 0, s>>>(N, Av, A1, W, tiles, xs); break;
     case 4: ladder_tp_tiled_kernel<4><<<grid, 128, 0, s>>>(N, Av, A1, W, tiles, xs); break;
@@ -407,6 +410,7 @@ static int tp_tiled_dispatch(int L, int N, const float* Av, const float* A1, con
 static int tp_vjp_dispatch(int L, int N, int C, const float* Av, const float* A1, const float* W,
                            const float* G, float* Avbar, float* A1bar, float* Wbar, cudaStream_t s) {
   switch (L) {
+    case 1: return launch_tp_vjp<1>(N, C, Av, A1, W, G, Avbar, A1bar, Wbar, s);
     case 2: return launch_tp_vjp<2>(N, C, Av, A1, W, G, Avbar, A1bar, Wbar, s);
     case 3: return launch_tp_vjp<3>(N, C, Av, A1, W, G, Avbar, A1bar, Wbar, s);
     case 4: return launch_tp_vjp<4>(N, C, Av, A1, W, G, Avbar, A1bar, Wbar, s);

@@ -378,9 +378,9 @@ def emit_direction(L):
     return "\n".join(o)
 
 
-NGROUPS = {2: 4, 3: 4, 4: 8}
-ROW_WEIGHT = {2: 0.0, 3: 0.0, 4: 4.0}
-STAGES = {2: 3, 3: 3, 4: 2}
+NGROUPS = {1: 2, 2: 4, 3: 4, 4: 8}
+ROW_WEIGHT = {1: 0.0, 2: 0.0, 3: 0.0, 4: 4.0}
+STAGES = {1: 3, 2: 3, 3: 3, 4: 2}
 MWIN = 16
 FWD_WARPS = 2
 
@@ -455,7 +455,7 @@ def emit_tables(Ls):
 def main():
     os.makedirs(OUTDIR, exist_ok=True)
     written = []
-    for L in (2, 3, 4):
+    for L in (1, 2, 3, 4):
         src, _, _ = emit_fwd(L, NGROUPS[L])
         path = os.path.join(OUTDIR, "fc_fwd_L%d.cuh" % L)
         with open(path, "w") as f:
@@ -463,7 +463,7 @@ def main():
         written.append(path)
     path = os.path.join(OUTDIR, "fc_tables.cuh")
     with open(path, "w") as f:
-        f.write(emit_tables((2, 3, 4)))
+        f.write(emit_tables((1, 2, 3, 4)))
     written.append(path)
     return written
 
@@ -677,9 +677,9 @@ class VjpGroupCode:
         return "\n".join(o)
 
 
-VJP_NGROUPS = {2: 4, 3: 8, 4: 8}
-VJP_STAGES = {2: 3, 3: 3, 4: 2}
-VJP_MWIN = {2: 16, 3: 16, 4: 8}
+VJP_NGROUPS = {1: 2, 2: 4, 3: 8, 4: 8}
+VJP_STAGES = {1: 3, 2: 3, 3: 3, 4: 2}
+VJP_MWIN = {1: 16, 2: 16, 3: 16, 4: 8}
 
 
 def emit_vjp(L, G):
@@ -959,9 +959,9 @@ class VvjpGroupCode:
         return "\n".join(o)
 
 
-VVJP_NGROUPS = {2: 6, 3: 16, 4: 32}
-VVJP_STAGES = {2: 2, 3: 2, 4: 2}
-VVJP_MWIN = {2: 8, 3: 8, 4: 8}
+VVJP_NGROUPS = {1: 2, 2: 6, 3: 16, 4: 32}
+VVJP_STAGES = {1: 2, 2: 2, 3: 2, 4: 2}
+VVJP_MWIN = {1: 8, 2: 8, 3: 8, 4: 8}
 
 
 def emit_vvjp(L, G):
@@ -1001,7 +1001,7 @@ _main_fwd = main
 
 def main():
     written = _main_fwd()
-    for L in (2, 3, 4):
+    for L in (1, 2, 3, 4):
         src, _, _ = emit_vjp(L, VJP_NGROUPS[L])
         path = os.path.join(OUTDIR, "fc_vjp_L%d.cuh" % L)
         with open(path, "w") as f:
@@ -1083,7 +1083,7 @@ _main_conv = main
 
 def main():
     written = _main_conv()
-    for L in (2, 3, 4):
+    for L in (1, 2, 3, 4):
         path = os.path.join(OUTDIR, "fc_ladder_L%d.cuh" % L)
         with open(path, "w") as f:
             f.write(emit_ladder(L))

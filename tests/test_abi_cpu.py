@@ -49,7 +49,7 @@ def test_status_strings(fc):
     assert lib.fc_version() >= 100
 
 
-@pytest.mark.parametrize("L", [2, 3, 4])
+@pytest.mark.parametrize("L", [1, 2, 3, 4])
 def test_descriptor_queries_match_oracle_paths(fc, L):
     from oracle import oracle as O
     assert fc.paths(L) == O.paths(L, L, L)
@@ -60,7 +60,8 @@ def test_descriptor_queries_match_oracle_paths(fc, L):
 
 def test_descriptor_rejections(fc):
     lib = fc.lib()
-    bad = [fc.ConvDesc(1, 1, 1, 8, 0),      # unsupported rank
+    bad = [fc.ConvDesc(0, 0, 0, 8, 0),      # unsupported rank (1..4 are built)
+           fc.ConvDesc(5, 5, 5, 8, 0),      # unsupported rank
            fc.ConvDesc(3, 2, 3, 8, 0),      # mixed ranks
            fc.ConvDesc(3, 3, 3, 6, 0),      # channels not multiple of 4
            fc.ConvDesc(3, 3, 3, 0, 0),      # no channels

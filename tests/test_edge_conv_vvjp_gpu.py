@@ -80,7 +80,7 @@ def test_single_cotangents(fc, use):
     check_all(gpu_vvjp(fc, wl, use=use), oracle_vvjp(wl, use=use))
 
 
-@pytest.mark.parametrize("L,C,sum_paths", [(3, 40, False), (3, 40, True), (2, 200, False),
+@pytest.mark.parametrize("L,C,sum_paths", [(1, 8, False), (1, 64, True), (3, 40, False), (3, 40, True), (2, 200, False),
                                            (4, 12, True)])
 def test_ragged_degrees_and_channel_tails(fc, L, C, sum_paths):
     degrees = [0, 1, 31, 32, 33, 64, 65, 0, 7, 70, 2, 0]

@@ -36,7 +36,7 @@ def run_gpu(fc, wl, gz=None):
     return out
 
 
-@pytest.mark.parametrize("L,C,order,N", [(2, 8, 4, 24), (3, 8, 4, 20), (3, 12, 3, 17),
+@pytest.mark.parametrize("L,C,order,N", [(1, 8, 5, 30), (2, 8, 4, 24), (3, 8, 4, 20), (3, 12, 3, 17),
                                          (4, 4, 3, 9), (3, 40, 5, 10)])
 def test_small_ladder_full(fc, L, C, order, N):
     wl = dict(lmax=L, channels=C, order=order,
@@ -53,7 +53,7 @@ def test_small_ladder_full(fc, L, C, order, N):
         assert rel_err(mwb[v], rm[v]) <= VJP_TOL
 
 
-@pytest.mark.parametrize("L,order,N", [(2, 3, 50), (3, 4, 37), (4, 3, 21), (3, 3, 1200)])
+@pytest.mark.parametrize("L,order,N", [(1, 4, 90), (2, 3, 50), (3, 4, 37), (4, 3, 21), (3, 3, 1200)])
 def test_tensor_core_mix_c128(fc, L, order, N):
     """C = 128 takes the tcgen05 mix (three-term TF32 split): ragged last
     tiles of every rank; N = 1200 at rank 3 gives 152 tiles, so some CTAs
