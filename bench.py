@@ -48,6 +48,10 @@ def parse():
     ap.add_argument("--rows", default=",".join(ROW_NAMES),
                     help="comma-separated extra rows to time: " + ", ".join(ROW_NAMES))
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--grid", action="store_true",
+                    help="time forward, VJP and VJP-of-VJP over the edge-convolution benchmark grid "
+                         "(1024 nodes; ranks 1-5 x 64/128 neighbours x 64/128/256 channels) and print "
+                         "one JSON line with a row per configuration")
     return ap.parse_args()
 
 
@@ -597,8 +601,89 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
+def run_grid(args):
+    """The pages' edge-convolution benchmark grid (1024 nodes, 64 or 128
+    random neighbours, 64/128/256 channels, ranks 1-5): forward, VJP (x_bar,
+    w_bar, r_bar) and VJP-of-VJP (all four outputs, all cotangents; ranks
+    1-4) per configuration, CUDA events, inputs resident on the device
+    (seeded, synthetic; drawn on the device)."""
+    import torch
+    from cartesian_tensor_products_b200 import flashcart as fc
+    from cartesian_tensor_products_b200 import workloads as W
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream()
+    peaks, peak_kind = load_peaks()
+    steps = max(3, min(args.steps, 10))
+    out = []
+    for k in (64, 128):
+        _, ei_np, ev_np = W.random_graph(1024, k, 20.0, 2 + k)
+        ei = torch.from_numpy(ei_np).to(dev)
+        ev = torch.from_numpy(ev_np).to(dev)
+        rp = fc.build_rowptr(ei, ev, 1024)
+        E = ei_np.shape[1]
+        for L in (1, 2, 3, 4, 5):
+            P = fc.num_paths(L)
+            for C in (64, 128, 256):
+                gen = torch.Generator(device=dev)
+                gen.manual_seed(1000 * L + C + k)
+                rnd = lambda *shape, s=1.0: torch.randn(*shape, device=dev, generator=gen) * s
+                x = rnd(1024, (L + 1) ** 2 * C)
+                w = rnd(E, P, C, s=P ** -0.5)
+                zr = fc.out_row(L)
+                g = rnd(1024, zr * C)
+                vx, vw, vr = rnd(1024, (L + 1) ** 2 * C), rnd(E, P, C, s=P ** -0.5), rnd(E, 3)
+                z = torch.empty((1024, zr * C), device=dev)
+                f_ms, _ = time_events(lambda: fc.edge_conv(L, rp, ei, ev, x, w, out=z), steps, 3, stream)
+                v_ms, _ = time_events(lambda: fc.edge_conv_vjp(L, rp, ei, ev, x, w, g), steps, 3, stream)
+                vv_ms = None
+                if L <= 4:      # the VJP-of-VJP is built up to rank 4
+                    vv_ms, _ = time_events(lambda: fc.edge_conv_vjp_vjp(L, rp, ei, ev, x, w, g, v_x=vx,
+                                                                        v_w=vw, v_r=vr), steps, 3, stream)
+                fb = algorithmic_bytes(1024, E, C, L, P, zr)
+                out.append({"lmax": L, "neighbours": k, "channels": C, "paths": P,
+                            "fwd_ms": f_ms, "vjp_ms": v_ms, "vvjp_ms": vv_ms,
+                            "fwd_edge_channels_per_s": E * C / (f_ms * 1e-3),
+                            "fwd_hbm_frac": fb / (f_ms * 1e-3) / 1e9 / peaks["hbm_gbs"]})
+                del x, w, g, vx, vw, vr, z
+                torch.cuda.empty_cache()
+    # node-local grid: 4096 nodes, ranks 1-4, orders 2-6, 64/128/256 channels
+    lad = []
+    for L in (1, 2, 3, 4):
+        P = fc.num_paths(L)
+        NY = (L + 1) ** 2
+        for C in (64, 128, 256):
+            for order in (2, 3, 4, 5, 6):
+                gen = torch.Generator(device=dev)
+                gen.manual_seed(7000 + 100 * L + 10 * order + C)
+                A1 = torch.randn(4096, NY * C, device=dev, generator=gen)
+                pw = torch.randn(order - 1, P, C, device=dev, generator=gen) * P ** -0.5
+                mw = torch.randn(order - 1, L + 1, C, C, device=dev, generator=gen) * C ** -0.5
+                gz = torch.randn(4096, NY * C, device=dev, generator=gen)
+                res = {}
+
+                def lf():
+                    res["s"], res["z"] = fc.product_ladder(L, order, A1, pw, mw)
+                f_ms, _ = time_events(lf, steps, 3, stream)
+                v_ms, _ = time_events(lambda: fc.product_ladder_vjp(L, order, A1, pw, mw, res["s"], gz),
+                                      steps, 3, stream)
+                lad.append({"lmax": L, "order": order, "channels": C, "fwd_ms": f_ms, "vjp_ms": v_ms,
+                            "mix": "tcgen05 TF32x3" if C == 128 else "FP32 SIMT"})
+                del A1, pw, mw, gz, res
+                torch.cuda.empty_cache()
+    print(json.dumps({"metric": "edge-conv grid: fwd / VJP / VJP-of-VJP ms per configuration",
+                      "unit": "ms", "n_gpus": 1, "dtype": "f32", "data": "synthetic",
+                      "peak_source": peak_kind, "steps": steps,
+                      "config": {"workload": "1024 nodes, random neighbours in a 20 A box; "
+                                             "ranks 1-5 x 64/128 neighbours x 64/128/256 channels"},
+                      "grid": out, "ladder_grid": lad}))
+
+
 def main():
     args = parse()
+    if args.grid:
+        run_grid(args)
+        return
     if args.impl == "reference":
         run_reference(args)
     else:

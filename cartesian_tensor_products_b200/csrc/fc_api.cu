@@ -26,7 +26,7 @@ int check_conv_desc(const fc_conv_desc* d) {
   if (d->sum_paths != 0 && d->sum_paths != 1) return FC_ERR_ARG;
   if (d->channels <= 0) return FC_ERR_ARG;
   if (d->lmax_in != d->lmax_edge || d->lmax_in != d->lmax_out) return FC_ERR_UNSUPPORTED_RANK;
-  if (d->lmax_in < 1 || d->lmax_in > 4) return FC_ERR_UNSUPPORTED_RANK;
+  if (d->lmax_in < 1 || d->lmax_in > 5) return FC_ERR_UNSUPPORTED_RANK;
   if (d->channels % 4) return FC_ERR_ALIGN;
   if (d->envelope != 0 && d->envelope != 1) return FC_ERR_ARG;
   if (d->envelope == 1 && !(d->r_cut > 0.0f && isfinite(d->r_cut) && isfinite(d->edge_scale)))

@@ -1,0 +1,209 @@
+// libflashcart: receiver-sorted edge convolution, forward.
+//
+// FlashCart (arXiv 2610.06409) Sec. 4 Eq. (1) and Algorithm 1:
+//   z_{u eta k} = sum_{e: u_e = u} w_{e eta k} f_eta(x_{v_e k}, y_e),
+//   y_e = T(r-hat_e) shared by all channels.
+// Every receiver's sums are accumulated on chip and stored once.
+//
+// B200 design.  One CTA per (receiver, 128-channel tile); its G warps each
+// own a fixed group of output rows (path, component), cut offline so that
+// the warps do near-equal work.  A lane owns 4 consecutive channels, so
+// every global access is a coalesced 16-byte vector.  Per incoming edge a
+// warp needs the sender's x rows its rows touch and the edge's weight rows
+// of its paths: each lane streams its own 16-byte slices of those rows into
+// a 3-deep shared-memory ring with cp.async, three edges ahead of use, and
+// reads back only what it copied (no barrier on the data path).  Every 16
+// edges the warp forms, lane-per-edge, the entries
+// M[a][b] = sum_b2 K[a][b][b2] y_b2 (y = T(r-hat)) of its rows into a
+// warp-private shared-memory window; the per-edge loop then reads them as
+// broadcasts and applies them to the lane's 4 channels with packed FP32x2
+// FMAs.  Sender indices and edge vectors come from a 32-edge register
+// window (one per lane) read with warp shuffles.  With 4 groups every SMSP
+// runs one instruction stream (warp g of each resident CTA).
+#pragma once
+#include "fc_common.cuh"
+#include "fc_device.cuh"
+
+namespace fc {
+
+struct ConvArgs {
+  const int32_t* rowptr;
+  const int32_t* send;
+  const float* vec;
+  const float* x;
+  const float* w;
+  float* z;
+  int n_nodes, n_edges, C, ntiles, xrow, zrow, P, sum_paths;
+  int envelope;
+  float r_cut, edge_scale;
+};
+
+// sender and edge vector of edge `e` for this lane's window slot
+struct EdgeWin {
+  int v;
+  float rx, ry, rz;
+};
+
+__device__ __forceinline__ EdgeWin load_win(const ConvArgs& a, int e, int e1) {
+  EdgeWin wv;
+  if (e < e1) {
+    wv.v = __ldg(a.send + e);
+    wv.rx = __ldg(a.vec + 3 * e);
+    wv.ry = __ldg(a.vec + 3 * e + 1);
+    wv.rz = __ldg(a.vec + 3 * e + 2);
+  } else {
+    wv.v = -1;
+    wv.rx = 1.0f;
+    wv.ry = 0.0f;
+    wv.rz = 0.0f;
+  }
+  return wv;
+}
+
+template <class Grp>
+__device__ __forceinline__ void issue_edge(const ConvArgs& a, int C, float* st, int q, int v,
+                                           int k0, bool act) {
+  const bool vok = act && v >= 0 && v < a.n_nodes;
+  const int kk = act ? k0 : 0;
+  const float* xv = a.x + (size_t)(vok ? v : 0) * a.xrow * C + kk;
+  const float* we = a.w + (size_t)q * a.P * C + kk;
+  Grp::issue(st, xv, we, C, vok, act);
+}
+
+// CC > 0: the channel count is the compile-time constant CC (every row
+// offset becomes an immediate); CC == 0: runtime a.C.
+template <class Grp, int S, int MW, int CC, bool ENV>
+__device__ __forceinline__ void fwd_warp(const ConvArgs& a, float* smem, int lane, int unit) {
+  constexpr int STAGE = Grp::NROW * 128;  // floats per stage (all lanes)
+  const int C = CC > 0 ? CC : a.C;
+  const int u = CC == 128 ? unit : unit / a.ntiles;
+  const int tile = unit - u * (CC == 128 ? 1 : a.ntiles);
+  const int k0 = tile * 128 + lane * 4;
+  const bool act = k0 < C;
+  int e0 = __ldg(a.rowptr + u), e1 = __ldg(a.rowptr + u + 1);
+  e0 = e0 < 0 ? 0 : (e0 > a.n_edges ? a.n_edges : e0);
+  e1 = e1 < e0 ? e0 : (e1 > a.n_edges ? a.n_edges : e1);
+  float* st = smem + Grp::RING_OFF + lane * 4;
+  float* mwin = smem + Grp::MWIN_OFF;
+
+  float4 acc[Grp::NA];
+#pragma unroll
+  for (int i = 0; i < Grp::NA; ++i) acc[i] = zero4();
+
+  EdgeWin cur = load_win(a, e0 + lane, e1);
+  EdgeWin nxt = load_win(a, e0 + 32 + lane, e1);
+
+  // prefill S edges
+#pragma unroll
+  for (int s = 0; s < S; ++s) {
+    const int q = e0 + s;
+    const int v = __shfl_sync(0xffffffffu, cur.v, s);
+    if (q < e1) issue_edge<Grp>(a, C, st + s * STAGE, q, v, k0, act);
+    cp_async_commit();
+  }
+
+  for (int q = e0; q < e1; ++q) {
+    const int p = q - e0;
+    if (p > 0 && (p & 31) == 0) {
+      cur = nxt;
+      nxt = load_win(a, q + 32 + lane, e1);
+    }
+    if ((p % MW) == 0) {
+      // M entries of the next MW edges, lane-per-edge, into the warp's window
+      const int src = (p & 31) + (lane % MW);
+      const float rx = __shfl_sync(0xffffffffu, cur.rx, src);
+      const float ry = __shfl_sync(0xffffffffu, cur.ry, src);
+      const float rz = __shfl_sync(0xffffffffu, cur.rz, src);
+      __syncwarp();
+      if (lane < MW && q + lane < e1) {
+        const float r = sqrtf(rx * rx + ry * ry + rz * rz);
+        const float inv = 1.0f / r;
+        float es, esp;
+        edge_envelope(a.envelope, r, a.r_cut, a.edge_scale, es, esp);
+        Grp::template make_m<ENV>(rx * inv, ry * inv, rz * inv, es, mwin + lane * Grp::MSTRIDE);
+      }
+      __syncwarp();
+    }
+    const int slot = p % S;
+    cp_async_wait<S - 1>();
+    Grp::template accum<ENV>(acc, st + slot * STAGE, mwin + (p % MW) * Grp::MSTRIDE);
+    // refill this slot with edge q + S
+    const int pn = p + S;
+    if (q + S < e1) {
+      int v;
+      if ((pn >> 5) == (p >> 5))
+        v = __shfl_sync(0xffffffffu, cur.v, pn & 31);
+      else
+        v = __shfl_sync(0xffffffffu, nxt.v, pn & 31);
+      issue_edge<Grp>(a, C, st + slot * STAGE, q + S, v, k0, act);
+    }
+    cp_async_commit();
+  }
+  cp_async_wait<0>();
+  if (act) Grp::store(a.z + (size_t)u * a.zrow * C + k0, C, a.sum_paths, acc);
+}
+
+template <int L, int CC, bool ENV, int g>
+__device__ __forceinline__ void dispatch_fwd(int grp, const ConvArgs& a, float* smem, int lane,
+                                             int unit) {
+  if constexpr (g < FwdMeta<L>::G) {
+    using Grp = FwdGroup<L, FwdMeta<L>::G, g>;
+    if (grp == g) {
+      fwd_warp<Grp, FwdMeta<L>::S, FwdMeta<L>::MWIN, CC, ENV>(a, smem, lane, unit);
+      return;
+    }
+    dispatch_fwd<L, CC, ENV, g + 1>(grp, a, smem, lane, unit);
+  }
+}
+
+// Up to 4 groups: a CTA is the G groups of one receiver tile (warp g runs
+// group g, one warp per SMSP).  More groups: a CTA is one group for WARPS
+// consecutive receiver tiles, blocks ordered group-major, so an SMSP still
+// mostly runs one instruction stream.
+template <int L, int CC, bool ENV>
+__global__ void __launch_bounds__(FwdMeta<L>::WARPS * 32, 2) edge_conv_fwd_kernel(const ConvArgs a) {
+  extern __shared__ __align__(16) float smem[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if constexpr (!FwdMeta<L>::GROUP_MAJOR) {
+    dispatch_fwd<L, CC, ENV, 0>(warp, a, smem, lane, blockIdx.x);
+  } else {
+    constexpr int WARPS = FwdMeta<L>::WARPS;
+    const int units = a.n_nodes * a.ntiles;
+    const int nb = (units + WARPS - 1) / WARPS;
+    const int grp = blockIdx.x / nb;
+    const int unit = (blockIdx.x - grp * nb) * WARPS + warp;
+    if (unit >= units) return;
+    dispatch_fwd<L, CC, ENV, 0>(grp, a, smem + warp * FwdMeta<L>::WARP_FLOATS, lane, unit);
+  }
+}
+
+template <int L, int CC, bool ENV>
+static int launch_fwd_cc(const ConvArgs& a, cudaStream_t s) {
+  static_assert(sizeof(float) * FwdMeta<L>::SMEM_FLOATS <= 227 * 1024,
+                "forward kernel shared memory exceeds the 227 KB per-CTA limit of sm_100");
+  const size_t smem = sizeof(float) * (size_t)FwdMeta<L>::SMEM_FLOATS;
+  static int configured[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return FC_ERR_CUDA;
+  if (!configured[dev]) {
+    if (cudaFuncSetAttribute(edge_conv_fwd_kernel<L, CC, ENV>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+      return FC_ERR_CUDA;
+    configured[dev] = 1;
+  }
+  const long long units = (long long)a.n_nodes * a.ntiles;
+  constexpr int WARPS = FwdMeta<L>::WARPS;
+  const long long blocks =
+      FwdMeta<L>::GROUP_MAJOR ? (units + WARPS - 1) / WARPS * FwdMeta<L>::G : units;
+  if (blocks > 0x7fffffffLL) return FC_ERR_ARG;
+  edge_conv_fwd_kernel<L, CC, ENV><<<(unsigned)blocks, WARPS * 32, smem, s>>>(a);
+  return cudaGetLastError() == cudaSuccess ? FC_OK : FC_ERR_CUDA;
+}
+
+template <int L>
+static int launch_fwd(const ConvArgs& a, cudaStream_t s) {
+  if (a.envelope) return a.C == 128 ? launch_fwd_cc<L, 128, true>(a, s) : launch_fwd_cc<L, 0, true>(a, s);
+  return a.C == 128 ? launch_fwd_cc<L, 128, false>(a, s) : launch_fwd_cc<L, 0, false>(a, s);
+}
+
+}  // namespace fc

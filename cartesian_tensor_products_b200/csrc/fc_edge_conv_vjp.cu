@@ -25,236 +25,14 @@
 // atomically), and y_bar through d_(a,b1) = <g_a, w x_b1>; y_bar is folded
 // into u_bar = (dT/du)^T y_bar, reduced over the warp with shuffles and
 // added atomically (3 floats per warp and edge) into r_bar.
-#include "fc_common.cuh"
-#include "fc_device.cuh"
+#include "fc_edge_conv_vjp.cuh"
 #include "generated/fc_vjp_L1.cuh"
 #include "generated/fc_vjp_L2.cuh"
 #include "generated/fc_vjp_L3.cuh"
 #include "generated/fc_vjp_L4.cuh"
 
 namespace fc {
-
-struct VjpArgs {
-  const int32_t* rowptr;
-  const int32_t* send;
-  const float* vec;
-  const float* x;
-  const float* w;
-  const float* g;
-  float* xbar;
-  float* wbar;
-  float* rbar;
-  int n_nodes, n_edges, C, ntiles, xrow, zrow, P, sum_paths;
-  int envelope;
-  float r_cut, edge_scale;
-};
-
-struct VEdgeWin {
-  int v;
-  float rx, ry, rz;
-};
-
-__device__ __forceinline__ VEdgeWin vload_win(const VjpArgs& a, int e, int e1) {
-  VEdgeWin wv;
-  if (e < e1) {
-    wv.v = __ldg(a.send + e);
-    wv.rx = __ldg(a.vec + 3 * e);
-    wv.ry = __ldg(a.vec + 3 * e + 1);
-    wv.rz = __ldg(a.vec + 3 * e + 2);
-  } else {
-    wv.v = -1;
-    wv.rx = 1.0f;
-    wv.ry = 0.0f;
-    wv.rz = 0.0f;
-  }
-  return wv;
-}
-
-template <class Grp>
-__device__ __forceinline__ void vissue_edge(const VjpArgs& a, int C, float* st, int q, int v,
-                                            int k0, bool act) {
-  const bool vok = act && v >= 0 && v < a.n_nodes;
-  const int kk = act ? k0 : 0;
-  const float* xv = a.x + (size_t)(vok ? v : 0) * a.xrow * C + kk;
-  const float* we = a.w + (size_t)q * a.P * C + kk;
-  Grp::issue(st, xv, we, C, vok, act);
-}
-
-template <class Grp, int S, int MW, int CC>
-__device__ __forceinline__ void vjp_warp(const VjpArgs& a, float* smem, int lane, int unit) {
-  constexpr int STAGE = Grp::NROW * 128;
-  constexpr int NYB = Grp::NYD > 0 ? Grp::NYD : 1;
-  const int C = CC > 0 ? CC : a.C;
-  const int u = CC == 128 ? unit : unit / a.ntiles;
-  const int tile = unit - u * (CC == 128 ? 1 : a.ntiles);
-  const int k0 = tile * 128 + lane * 4;
-  const bool act = k0 < C;
-  int e0 = __ldg(a.rowptr + u), e1 = __ldg(a.rowptr + u + 1);
-  e0 = e0 < 0 ? 0 : (e0 > a.n_edges ? a.n_edges : e0);
-  e1 = e1 < e0 ? e0 : (e1 > a.n_edges ? a.n_edges : e1);
-  if (e0 == e1) return;
-  float* st = smem + Grp::RING_OFF + lane * 4;
-  float* mwin = smem + Grp::MWIN_OFF;
-  const bool wstore = act && a.wbar != nullptr;
-  float* wbase = a.wbar != nullptr ? a.wbar : a.xbar;   // any valid pointer when unused
-
-  float4 gr[Grp::NA];
-  if (act) {
-    Grp::load_g(a.g + (size_t)u * a.zrow * C + k0, C, a.sum_paths, gr);
-  } else {
-#pragma unroll
-    for (int i = 0; i < Grp::NA; ++i) gr[i] = zero4();
-  }
-  float4 xb[Grp::NX];
-#pragma unroll
-  for (int i = 0; i < Grp::NX; ++i) xb[i] = zero4();
-  float yb[NYB];
-#pragma unroll
-  for (int i = 0; i < NYB; ++i) yb[i] = 0.0f;
-
-  VEdgeWin cur = vload_win(a, e0 + lane, e1);
-  VEdgeWin nxt = vload_win(a, e0 + 32 + lane, e1);
-#pragma unroll
-  for (int s = 0; s < S; ++s) {
-    const int q = e0 + s;
-    const int v = __shfl_sync(0xffffffffu, cur.v, s);
-    if (q < e1) vissue_edge<Grp>(a, C, st + s * STAGE, q, v, k0, act);
-    cp_async_commit();
-  }
-
-  for (int q = e0; q < e1; ++q) {
-    const int p = q - e0;
-    if (p > 0 && (p & 31) == 0) {
-      cur = nxt;
-      nxt = vload_win(a, q + 32 + lane, e1);
-    }
-    if ((p % MW) == 0) {
-      const int src = (p & 31) + (lane % MW);
-      const float rx = __shfl_sync(0xffffffffu, cur.rx, src);
-      const float ry = __shfl_sync(0xffffffffu, cur.ry, src);
-      const float rz = __shfl_sync(0xffffffffu, cur.rz, src);
-      __syncwarp();
-      if (lane < MW && q + lane < e1) {
-        const float r = sqrtf(rx * rx + ry * ry + rz * rz);
-        const float inv = 1.0f / r;
-        float es, esp;
-        edge_envelope(a.envelope, r, a.r_cut, a.edge_scale, es, esp);
-        Grp::make_row(rx * inv, ry * inv, rz * inv, es, esp, mwin + lane * Grp::MSTRIDE);
-      }
-      __syncwarp();
-    }
-    const int slot = p % S;
-    cp_async_wait<S - 1>();
-    const float* m = mwin + (p % MW) * Grp::MSTRIDE;
-    Grp::edge(gr, st + slot * STAGE, m, xb, yb,
-              wbase + (wstore ? (size_t)q * a.P * C + k0 : 0), C, wstore);
-    // sender gradient
-    const int v = __shfl_sync(0xffffffffu, cur.v, p & 31);
-    if (a.xbar != nullptr && act && v >= 0 && v < a.n_nodes) {
-      Grp::flush_xbar(a.xbar + (size_t)v * a.xrow * C + k0, C, xb);
-    } else {
-#pragma unroll
-      for (int i = 0; i < Grp::NX; ++i) xb[i] = zero4();
-    }
-    // edge-vector gradient
-    if constexpr (Grp::NYD > 0) {
-      if (a.rbar != nullptr) {
-        float ux, uy, uz, rho;
-        Grp::ubar(yb, m, ux, uy, uz, rho);
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-          ux += __shfl_xor_sync(0xffffffffu, ux, o);
-          uy += __shfl_xor_sync(0xffffffffu, uy, o);
-          uz += __shfl_xor_sync(0xffffffffu, uz, o);
-          rho += __shfl_xor_sync(0xffffffffu, rho, o);
-        }
-        const float rx = __shfl_sync(0xffffffffu, cur.rx, p & 31);
-        const float ry = __shfl_sync(0xffffffffu, cur.ry, p & 31);
-        const float rz = __shfl_sync(0xffffffffu, cur.rz, p & 31);
-        if (lane == 0) {
-          const float inv = 1.0f / sqrtf(rx * rx + ry * ry + rz * rz);
-          const float nx = rx * inv, ny = ry * inv, nz = rz * inv;
-          const float dotu = ux * nx + uy * ny + uz * nz;
-          // direction part (I - u u^T)/|r| u_bar plus the radial part of the
-          // envelope, s'(|r|) (y_bar . y) r-hat
-          atomicAdd(a.rbar + 3 * (size_t)q + 0, (ux - nx * dotu) * inv + rho * nx);
-          atomicAdd(a.rbar + 3 * (size_t)q + 1, (uy - ny * dotu) * inv + rho * ny);
-          atomicAdd(a.rbar + 3 * (size_t)q + 2, (uz - nz * dotu) * inv + rho * nz);
-        }
-      }
-#pragma unroll
-      for (int i = 0; i < NYB; ++i) yb[i] = 0.0f;
-    }
-    const int pn = p + S;
-    if (q + S < e1) {
-      int vn;
-      if ((pn >> 5) == (p >> 5))
-        vn = __shfl_sync(0xffffffffu, cur.v, pn & 31);
-      else
-        vn = __shfl_sync(0xffffffffu, nxt.v, pn & 31);
-      vissue_edge<Grp>(a, C, st + slot * STAGE, q + S, vn, k0, act);
-    }
-    cp_async_commit();
-  }
-  cp_async_wait<0>();
-}
-
-template <int L, int CC, int g>
-__device__ __forceinline__ void dispatch_vjp(int grp, const VjpArgs& a, float* smem, int lane,
-                                             int unit) {
-  if constexpr (g < VjpMeta<L>::G) {
-    using Grp = VjpGroup<L, VjpMeta<L>::G, g>;
-    if (grp == g) {
-      vjp_warp<Grp, VjpMeta<L>::S, VjpMeta<L>::MWIN, CC>(a, smem, lane, unit);
-      return;
-    }
-    dispatch_vjp<L, CC, g + 1>(grp, a, smem, lane, unit);
-  }
-}
-
-// CTA = (path group, WARPS consecutive receiver units): every warp of a CTA
-// runs the same code, and blocks are ordered group-major, so an SMSP mostly
-// executes one instruction stream.
-template <int L, int CC>
-__global__ void __launch_bounds__(VjpMeta<L>::WARPS * 32, 2) edge_conv_vjp_kernel(const VjpArgs a) {
-  extern __shared__ __align__(16) float smem[];
-  constexpr int WARPS = VjpMeta<L>::WARPS;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int units = a.n_nodes * a.ntiles;
-  const int nb = (units + WARPS - 1) / WARPS;
-  const int grp = blockIdx.x / nb;
-  const int unit = (blockIdx.x - grp * nb) * WARPS + warp;
-  if (unit >= units) return;
-  dispatch_vjp<L, CC, 0>(grp, a, smem + warp * VjpMeta<L>::WARP_FLOATS, lane, unit);
-}
-
-template <int L, int CC>
-static int launch_vjp_cc(const VjpArgs& a, cudaStream_t s) {
-  static_assert(sizeof(float) * VjpMeta<L>::SMEM_FLOATS <= 227 * 1024,
-                "VJP kernel shared memory exceeds the 227 KB per-CTA limit of sm_100");
-  const size_t smem = sizeof(float) * (size_t)VjpMeta<L>::SMEM_FLOATS;
-  static int configured[64] = {0};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return FC_ERR_CUDA;
-  if (!configured[dev]) {
-    if (cudaFuncSetAttribute(edge_conv_vjp_kernel<L, CC>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
-      return FC_ERR_CUDA;
-    configured[dev] = 1;
-  }
-  const long long units = (long long)a.n_nodes * a.ntiles;
-  constexpr int WARPS = VjpMeta<L>::WARPS;
-  const long long blocks = (units + WARPS - 1) / WARPS * VjpMeta<L>::G;
-  if (blocks > 0x7fffffffLL) return FC_ERR_ARG;
-  edge_conv_vjp_kernel<L, CC><<<(unsigned)blocks, WARPS * 32, smem, s>>>(a);
-  return cudaGetLastError() == cudaSuccess ? FC_OK : FC_ERR_CUDA;
-}
-
-template <int L>
-static int launch_vjp(const VjpArgs& a, cudaStream_t s) {
-  return a.C == 128 ? launch_vjp_cc<L, 128>(a, s) : launch_vjp_cc<L, 0>(a, s);
-}
-
+int launch_vjp_rank5(const VjpArgs& a, cudaStream_t s);
 }  // namespace fc
 
 using namespace fc;
@@ -311,6 +89,7 @@ extern "C" int fc_edge_conv_vjp(const fc_conv_desc* d, int n_nodes, int n_edges,
     case 2: return launch_vjp<2>(a, s);
     case 3: return launch_vjp<3>(a, s);
     case 4: return launch_vjp<4>(a, s);
+    case 5: return launch_vjp_rank5(a, s);
     default: return FC_ERR_UNSUPPORTED_RANK;
   }
 }

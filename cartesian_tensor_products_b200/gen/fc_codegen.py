@@ -378,9 +378,9 @@ def emit_direction(L):
     return "\n".join(o)
 
 
-NGROUPS = {1: 2, 2: 4, 3: 4, 4: 8}
-ROW_WEIGHT = {1: 0.0, 2: 0.0, 3: 0.0, 4: 4.0}
-STAGES = {1: 3, 2: 3, 3: 3, 4: 2}
+NGROUPS = {1: 2, 2: 4, 3: 4, 4: 8, 5: 24}
+ROW_WEIGHT = {1: 0.0, 2: 0.0, 3: 0.0, 4: 4.0, 5: 4.0}
+STAGES = {1: 3, 2: 3, 3: 3, 4: 2, 5: 2}
 MWIN = 16
 FWD_WARPS = 2
 
@@ -455,7 +455,7 @@ def emit_tables(Ls):
 def main():
     os.makedirs(OUTDIR, exist_ok=True)
     written = []
-    for L in (1, 2, 3, 4):
+    for L in (1, 2, 3, 4, 5):
         src, _, _ = emit_fwd(L, NGROUPS[L])
         path = os.path.join(OUTDIR, "fc_fwd_L%d.cuh" % L)
         with open(path, "w") as f:
@@ -463,7 +463,7 @@ def main():
         written.append(path)
     path = os.path.join(OUTDIR, "fc_tables.cuh")
     with open(path, "w") as f:
-        f.write(emit_tables((1, 2, 3, 4)))
+        f.write(emit_tables((1, 2, 3, 4, 5)))
     written.append(path)
     return written
 
@@ -677,9 +677,9 @@ class VjpGroupCode:
         return "\n".join(o)
 
 
-VJP_NGROUPS = {1: 2, 2: 4, 3: 8, 4: 8}
-VJP_STAGES = {1: 3, 2: 3, 3: 3, 4: 2}
-VJP_MWIN = {1: 16, 2: 16, 3: 16, 4: 8}
+VJP_NGROUPS = {1: 2, 2: 4, 3: 8, 4: 8, 5: 24}
+VJP_STAGES = {1: 3, 2: 3, 3: 3, 4: 2, 5: 2}
+VJP_MWIN = {1: 16, 2: 16, 3: 16, 4: 8, 5: 8}
 
 
 def emit_vjp(L, G):
@@ -1001,12 +1001,14 @@ _main_fwd = main
 
 def main():
     written = _main_fwd()
-    for L in (1, 2, 3, 4):
+    for L in (1, 2, 3, 4, 5):
         src, _, _ = emit_vjp(L, VJP_NGROUPS[L])
         path = os.path.join(OUTDIR, "fc_vjp_L%d.cuh" % L)
         with open(path, "w") as f:
             f.write(src)
         written.append(path)
+        if L == 5:          # the VJP-of-VJP is built up to rank 4
+            continue
         src, _, _ = emit_vvjp(L, VVJP_NGROUPS[L])
         path = os.path.join(OUTDIR, "fc_vvjp_L%d.cuh" % L)
         with open(path, "w") as f:

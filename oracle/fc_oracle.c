@@ -623,7 +623,7 @@ int orc_edge_conv(int lin, int ledge, int lout, int C, int sum_paths, int N,
                   int E, const int32_t *recv, const int32_t *send,
                   const double *vec, const double *x, const double *w,
                   const unsigned char *recv_mask, double *z) {
-  if (lin > 4 || ledge > 4 || lout > 4) return 1;
+  if (lin > 5 || ledge > 5 || lout > 5) return 1;
   path_set ps;
   make_paths(lin, ledge, lout, sum_paths, &ps);
   int xrow = (lin + 1) * (lin + 1);
@@ -682,7 +682,7 @@ int orc_edge_conv_vjp(int lin, int ledge, int lout, int C, int sum_paths,
                       const double *vec, const double *x, const double *w,
                       const double *g, const unsigned char *edge_mask,
                       double *x_bar, double *w_bar, double *r_bar) {
-  if (lin > 4 || ledge > 4 || lout > 4) return 1;
+  if (lin > 5 || ledge > 5 || lout > 5) return 1;
   path_set ps;
   make_paths(lin, ledge, lout, sum_paths, &ps);
   int xrow = (lin + 1) * (lin + 1);
@@ -811,7 +811,7 @@ int orc_edge_conv_vjp2(int lin, int ledge, int lout, int C, int sum_paths,
                        const double *vr, const unsigned char *edge_mask,
                        double *g_hat, double *x_hat, double *w_hat,
                        double *r_hat) {
-  if (lin > 4 || ledge > 4 || lout > 4) return 1;
+  if (lin > 5 || ledge > 5 || lout > 5) return 1;
   path_set ps;
   make_paths(lin, ledge, lout, sum_paths, &ps);
   int xrow = (lin + 1) * (lin + 1);

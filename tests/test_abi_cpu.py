@@ -49,7 +49,7 @@ def test_status_strings(fc):
     assert lib.fc_version() >= 100
 
 
-@pytest.mark.parametrize("L", [1, 2, 3, 4])
+@pytest.mark.parametrize("L", [1, 2, 3, 4, 5])
 def test_descriptor_queries_match_oracle_paths(fc, L):
     from oracle import oracle as O
     assert fc.paths(L) == O.paths(L, L, L)
@@ -61,7 +61,7 @@ def test_descriptor_queries_match_oracle_paths(fc, L):
 def test_descriptor_rejections(fc):
     lib = fc.lib()
     bad = [fc.ConvDesc(0, 0, 0, 8, 0),      # unsupported rank (1..4 are built)
-           fc.ConvDesc(5, 5, 5, 8, 0),      # unsupported rank
+           fc.ConvDesc(6, 6, 6, 8, 0),      # unsupported rank
            fc.ConvDesc(3, 2, 3, 8, 0),      # mixed ranks
            fc.ConvDesc(3, 3, 3, 6, 0),      # channels not multiple of 4
            fc.ConvDesc(3, 3, 3, 0, 0),      # no channels
@@ -72,7 +72,7 @@ def test_descriptor_rejections(fc):
     d = fc.ConvDesc(3, 3, 3, 6, 0)
     st = lib.fc_edge_conv(ct.byref(d), 4, 0, None, None, None, None, None, None, None)
     assert st == 5
-    d = fc.ConvDesc(5, 5, 5, 8, 0)
+    d = fc.ConvDesc(6, 6, 6, 8, 0)
     st = lib.fc_edge_conv(ct.byref(d), 4, 0, None, None, None, None, None, None, None)
     assert st == 4
     d = fc.ConvDesc(3, 3, 3, 8, 0)

@@ -112,7 +112,7 @@ def test_microbench_rank4_sampled(fc):
     assert rel_err(z[rows], ref[rows]) <= FWD_TOL
 
 
-@pytest.mark.parametrize("L,C", [(1, 8), (1, 64), (2, 4), (3, 40), (3, 200), (4, 12)])
+@pytest.mark.parametrize("L,C", [(1, 8), (1, 64), (2, 4), (3, 40), (3, 200), (4, 12), (5, 8)])
 def test_ragged_degrees_and_channel_tails(fc, L, C):
     degrees = [0, 1, 31, 32, 33, 64, 65, 0, 7, 70, 2, 0]
     ei, ev = ragged_graph(len(degrees) + 60, degrees + [3] * 60, 6.0, L * 1000 + C)

@@ -124,7 +124,7 @@ def test_microbench_vjp_dense_gradient_samples(fc, micro_grad):
     assert dots.max() < 1e-3
 
 
-@pytest.mark.parametrize("L,C", [(1, 8), (1, 64), (2, 4), (3, 40), (3, 200), (4, 12)])
+@pytest.mark.parametrize("L,C", [(1, 8), (1, 64), (2, 4), (3, 40), (3, 200), (4, 12), (5, 8)])
 def test_vjp_ragged_and_channel_tails(fc, L, C):
     degrees = [0, 1, 31, 32, 33, 40, 2, 0] + [3] * 40
     N = len(degrees)

@@ -125,6 +125,19 @@ def test_microbench_sampled_receivers(fc):
     assert np.all(np.isfinite(got[0]))
 
 
+def test_rank5_is_refused(fc):
+    """The VJP-of-VJP is built up to rank 4 (the pages split launches above
+    rank 4); rank 5 returns FC_ERR_UNSUPPORTED_RANK before any launch."""
+    t = W.tiny()
+    ei, ev = dev(t["edge_index"]), dev(t["edge_vec"])
+    rowptr = fc.build_rowptr(ei, ev, t["n_nodes"])
+    d = W.conv_inputs(t["n_nodes"], t["edge_index"], 5, 4, 3, with_grad=True)
+    with pytest.raises(fc.FlashCartError) as e:
+        fc.edge_conv_vjp_vjp(5, rowptr, ei, ev, dev(d["x"]), dev(d["w"]), dev(d["g"]),
+                             v_x=dev(d["x"]))
+    assert e.value.status == 4
+
+
 def test_envelope_is_refused_and_empty_graph(fc):
     t = W.tiny()
     wl = case(2, 8, t["edge_index"], t["edge_vec"], t["n_nodes"], 49)

@@ -31,7 +31,7 @@ def test_component_order_matches_oracle():
         assert G.components(l) == [O.comp_pxyz(l, c) for c in range(2 * l + 1)]
 
 
-@pytest.mark.parametrize("L", [1, 2, 3, 4])
+@pytest.mark.parametrize("L", [1, 2, 3, 4, 5])
 def test_forward_groups_cover_every_row_once(L):
     T = CG.Tables(L)
     groups = CG.partition_rows(T, CG.NGROUPS[L])
