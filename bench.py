@@ -74,6 +74,7 @@ def algorithmic_flops(E, C, L):
 # valid only while the kernel sources hash to the value it was taken with.
 FWD_TRAFFIC = {"sha1": "09d510c3c39768669ff17afc07977537a44bf766", "bytes": 1594689000 + 48416512}
 FWD_SOURCES = ("cartesian_tensor_products_b200/csrc/fc_edge_conv.cu",
+               "cartesian_tensor_products_b200/csrc/fc_edge_conv.cuh",
                "cartesian_tensor_products_b200/csrc/generated/fc_fwd_L3.cuh")
 
 

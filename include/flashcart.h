@@ -78,17 +78,18 @@ const char *fc_status_string(int status);
 int fc_version(void);
 
 /* Edge-convolution descriptor.  This build supports
- * lmax_in == lmax_edge == lmax_out in {2, 3, 4}, channels >= 4 and a
- * multiple of 4.  sum_paths = 0 keeps the P_l paths of each output rank
+ * lmax_in == lmax_edge == lmax_out in {1, 2, 3, 4, 5}, channels >= 4 and
+ * a multiple of 4 (rank 5: forward and VJP without the envelope; the
+ * VJP-of-VJP goes up to rank 4).  sum_paths = 0 keeps the P_l paths of each output rank
  * separate (z row = sum_l (2l+1) P_l C); sum_paths = 1 sums them (z row =
  * (lmax_out+1)^2 C, the node-feature layout).
  * envelope = 1 multiplies the direction tensors of edge e by
  *   s_e = edge_scale * (cos(pi |r_e| / r_cut) + 1) / 2   (|r_e| < r_cut, else 0),
- * a smooth radial envelope that makes every edge contribution vanish at
- * the cutoff (App. B, "A radial envelope makes every edge contribution
- * vanish smoothly"); by bilinearity this equals scaling all weights of edge
- * e by s_e, and edge_scale can carry a 1/sqrt(mean neighbours) factor (App.
- * E Eq. E1).  The VJP's r_bar then includes the derivative of s_e.
+ * a radial envelope that takes each edge's contribution smoothly to zero
+ * at the cutoff (Sec. 2, paragraph on equivariant convolution); by
+ * bilinearity this equals scaling all weights of edge e by s_e, and
+ * edge_scale can carry a 1/sqrt(mean neighbours) factor (App. E Eq. E1).
+ * The VJP's r_bar then includes the derivative of s_e.
  * envelope = 0 (r_cut and edge_scale ignored) means s_e = 1. */
 typedef struct {
   int lmax_in;      /* rank of node features x (l1)           */
@@ -212,7 +213,7 @@ int fc_edge_forces(int n_nodes, int n_edges, const int32_t *edge_index,
                    const float *r_bar, float *forces, fc_stream_t stream);
 
 /* Product-ladder descriptor: ranks 0..lmax for every state (lmax in
- * {2,3,4}), channels a multiple of 4, order >= 1 (order-1 products). */
+ * {1,2,3,4}), channels a multiple of 4, order >= 1 (order-1 products). */
 typedef struct {
   int lmax;
   int channels;
