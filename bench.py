@@ -72,7 +72,7 @@ def algorithmic_flops(E, C, L):
 # DRAM bytes (read + write) of one edge_conv_fwd_kernel<3, 128> launch on
 # this workload from an ncu capture (profiles/edge_conv_fwd_microbench_r3.md),
 # valid only while the kernel sources hash to the value it was taken with.
-FWD_TRAFFIC = {"sha1": "09d510c3c39768669ff17afc07977537a44bf766", "bytes": 1594689000 + 48416512}
+FWD_TRAFFIC = {"sha1": "909690aa9d2cf0b750751bc7bab142d350c8e724", "bytes": 1595942912 + 48170496}
 FWD_SOURCES = ("cartesian_tensor_products_b200/csrc/fc_edge_conv.cu",
                "cartesian_tensor_products_b200/csrc/fc_edge_conv.cuh",
                "cartesian_tensor_products_b200/csrc/generated/fc_fwd_L3.cuh")
