@@ -80,5 +80,9 @@ int launch_mix_tc_split_rows(int L, int N, const float* in, float* xs, cudaStrea
 int launch_mix_tc_split_matrix(int mode, int L, const float* M, float* ws, cudaStream_t s);
 // out[n][l^2 + c][j] = sum_t A_l(j, t) x[n][l^2 + c][t] for every rank l
 int launch_mix_tc(int L, int N, const float* xs, const float* ws, float* out, cudaStream_t s);
+// natural -> transposed split tiles (channels x rows, K-major along rows)
+int launch_mix_tc_split_cols(int L, int N, const float* in, float* xs, cudaStream_t s);
+// Mbar[l][k][j] += sum over the rows of rank l of a[row][k] b[row][j] (both transposed split)
+int launch_wgrad_tc(int L, int N, const float* as, const float* bs, float* Mbar, cudaStream_t s);
 
 }  // namespace fc

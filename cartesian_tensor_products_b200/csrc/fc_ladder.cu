@@ -520,7 +520,10 @@ size_t fc_product_ladder_vjp_workspace_size(const fc_ladder_desc* d, int n_nodes
   if (check_ladder_desc(d) != FC_OK || n_nodes < 0) return 0;
   const int NY = (d->lmax + 1) * (d->lmax + 1);
   size_t f = 4 * (size_t)n_nodes * NY * d->channels;
-  if (mix_tc_supported(d->lmax, d->channels)) f += tc_scratch_floats(d->lmax, n_nodes);
+  // tensor cores: the split gradient (for the mix), the matrices, and the
+  // transposed split gradient and recomputed product (for the weight gradient)
+  if (mix_tc_supported(d->lmax, d->channels))
+    f += tc_scratch_floats(d->lmax, n_nodes) + 2 * mix_tc_operand_floats(d->lmax, n_nodes);
   return sizeof(float) * f;
 }
 
@@ -561,6 +564,8 @@ int fc_product_ladder_vjp(const fc_ladder_desc* d, int n_nodes, const float* A1,
   const bool tc = mix_tc_supported(L, C);
   float* xs = ws + 4 * plane;                                   // tensor-core path only
   float* wsm = tc ? xs + mix_tc_operand_floats(L, n_nodes) : nullptr;
+  float* xta = tc ? wsm + mix_tc_matrix_floats(L) : nullptr;    // transposed split A_bar
+  float* xtb = tc ? xta + mix_tc_operand_floats(L, n_nodes) : nullptr;   // transposed split B
   const float* Anext_bar = gz;           // gradient of A_{v+1}
   for (int v = S; v >= 1; --v) {
     const float* Av = v == 1 ? A1 : states + (size_t)(v - 2) * plane;
@@ -574,18 +579,23 @@ int fc_product_ladder_vjp(const fc_ladder_desc* d, int n_nodes, const float* A1,
       if (cudaMemcpyAsync(Avbar, gz, sizeof(float) * plane, cudaMemcpyDeviceToDevice, s) != cudaSuccess)
         return FC_ERR_CUDA;
     }
-    if ((st = tp_dispatch(L, n_nodes, C, Av, A1, W, B, s)) != FC_OK) return st;
+    float* Mbar = mix_w_bar + (size_t)(v - 1) * (L + 1) * C * C;
     if (tc) {
-      if ((st = launch_mix_tc_split_rows(L, n_nodes, Anext_bar, xs, s)) != FC_OK ||
+      // B_bar = A_bar M and M_bar += A_bar^T B on the tensor cores; B is recomputed
+      if ((st = tp_dispatch(L, n_nodes, C, Av, A1, W, B, s)) != FC_OK ||
+          (st = launch_mix_tc_split_rows(L, n_nodes, Anext_bar, xs, s)) != FC_OK ||
           (st = launch_mix_tc_split_matrix(1, L, M, wsm, s)) != FC_OK ||
-          (st = launch_mix_tc(L, n_nodes, xs, wsm, Bbar, s)) != FC_OK)
+          (st = launch_mix_tc(L, n_nodes, xs, wsm, Bbar, s)) != FC_OK ||
+          (st = launch_mix_tc_split_cols(L, n_nodes, Anext_bar, xta, s)) != FC_OK ||
+          (st = launch_mix_tc_split_cols(L, n_nodes, B, xtb, s)) != FC_OK ||
+          (st = launch_wgrad_tc(L, n_nodes, xta, xtb, Mbar, s)) != FC_OK)
         return st;
-    } else if ((st = launch_mix<kMixBar>(L, n_nodes, C, Anext_bar, M, Bbar, nullptr, s)) != FC_OK) {
-      return st;
+    } else {
+      if ((st = tp_dispatch(L, n_nodes, C, Av, A1, W, B, s)) != FC_OK ||
+          (st = launch_mix<kMixBar>(L, n_nodes, C, Anext_bar, M, Bbar, nullptr, s)) != FC_OK ||
+          (st = launch_wgrad(L, n_nodes, C, Anext_bar, B, Mbar, s)) != FC_OK)
+        return st;
     }
-    if ((st = launch_wgrad(L, n_nodes, C, Anext_bar, B, mix_w_bar + (size_t)(v - 1) * (L + 1) * C * C,
-                           s)) != FC_OK)
-      return st;
     if ((st = tp_vjp_dispatch(L, n_nodes, C, Av, A1, W, Bbar, Avbar, A1_bar,
                               path_w_bar + (size_t)(v - 1) * P * C, s)) != FC_OK)
       return st;

@@ -344,7 +344,215 @@ __global__ void __launch_bounds__(kTcThreads, 1) ladder_mix_tc_kernel(Geom geo,
   }
 }
 
+// ---------------------------------------------------------------------------
+// weight gradient of the mix: Mbar_l[k][j] += sum_{rows of rank l} Abar[row][k] B[row][j]
+// ---------------------------------------------------------------------------
+// Here the tile rows are the K dimension, so both operands are taken
+// transposed: ladder_split_cols_kernel writes a tile as 128 channels x 128
+// rows in the K-major core-matrix layout (4 consecutive rows of one channel
+// per 16 bytes), so a K chunk of 32 rows is a contiguous 16 KB hi and 16 KB lo
+// block, exactly as the mix's chunks.  One persistent CTA per SM walks its
+// tiles: one thread bulk-copies each chunk of both operands (64 KB) into one
+// of three stages, one thread issues the 12 MMAs of a chunk (M = N = 128,
+// three TF32 products per K step), the accumulator D[k][j] sums every tile
+// of one rank, and at a rank change and at the end warps 4-7 add it to Mbar
+// with vector atomics (CTAs share Mbar_l).  (Reading the row-major tiles with
+// MN-major descriptors instead returned zeros on sm_100a.)
+
+// natural [N][NY][128] -> transposed split tiles: element (row r, channel k)
+// of tile t at core_offset(k, r, 128) of the tile's hi / lo block.  Thread p
+// moves a 4-row x 4-channel block: 4 row-wise float4 loads, 4 channel-wise
+// float4 stores.  Rows past the rank's last row are written as zeros.
+__global__ void __launch_bounds__(256) ladder_split_cols_kernel(Geom g, const float* __restrict__ in,
+                                                                float* __restrict__ xs) {
+  const int t = blockIdx.x;
+  const int l = tile_rank(g, t);
+  const int R = g.N * (2 * l + 1);
+  const int row0 = (t - tile_first(g, l)) * kTcRows;
+  float* hi = xs + (size_t)t * kTcTileFloats;
+#pragma unroll
+  for (int it = 0; it < 4; ++it) {
+    const int u = it * 256 + threadIdx.x;          // 0 .. 1023
+    const int k4 = u & 31, r4 = u >> 5;            // channel group (fastest), row group
+    float4 v[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int r = row0 + 4 * r4 + i;
+      v[i] = r < R ? __ldg(reinterpret_cast<const float4*>(in + tc_rank_row(r, l, g.NY)) + k4) : zero4();
+    }
+    const float c0[4] = {v[0].x, v[1].x, v[2].x, v[3].x};
+    const float c1[4] = {v[0].y, v[1].y, v[2].y, v[3].y};
+    const float c2[4] = {v[0].z, v[1].z, v[2].z, v[3].z};
+    const float c3[4] = {v[0].w, v[1].w, v[2].w, v[3].w};
+    const float* cs[4] = {c0, c1, c2, c3};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      uint4 h, w;
+      split4(make_float4(cs[j][0], cs[j][1], cs[j][2], cs[j][3]), h, w);
+      const int off = tc::core_offset(4 * k4 + j, 4 * r4, kTcRows);
+      *reinterpret_cast<uint4*>(hi + off) = h;
+      *reinterpret_cast<uint4*>(hi + kTcWFloats + off) = w;
+    }
+  }
+}
+
+constexpr int kWgThreads = 256;
+constexpr int kWgStageFloats = 2 * kTcChunkFloats;   // A and B chunks (hi + lo each)
+constexpr size_t kWgSmemBytes = sizeof(float) * kTcStages * kWgStageFloats + 8 * 16 + 8;
+static_assert(kWgSmemBytes <= 232448, "shared memory per CTA");
+
+__global__ void __launch_bounds__(kWgThreads, 1) ladder_wgrad_tc_kernel(Geom geo,
+                                                                        const float* __restrict__ as,
+                                                                        const float* __restrict__ bs,
+                                                                        float* __restrict__ Mbar) {
+  extern __shared__ __align__(1024) unsigned char smem[];
+  float* st = reinterpret_cast<float*>(smem);        // stages: A hi, A lo, B hi, B lo (4096 each)
+  uint64_t* stage_full = reinterpret_cast<uint64_t*>(st + kTcStages * kWgStageFloats);
+  uint64_t* stage_free = stage_full + kTcStages;
+  uint64_t* acc_full = stage_free + kTcStages;
+  uint64_t* acc_free = acc_full + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_free + 1);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int T = tile_count(geo);
+  const int t_begin = (int)((long long)blockIdx.x * T / gridDim.x);
+  const int t_end = (int)((long long)(blockIdx.x + 1) * T / gridDim.x);
+
+  if (warp == 0) tc::tmem_alloc(tmem_slot, kTcRows);
+  if (tid == 0) {
+    for (int s = 0; s < kTcStages; ++s) {
+      tc::bar_init(&stage_full[s], 1);
+      tc::bar_init(&stage_free[s], 1);
+    }
+    tc::bar_init(acc_full, 1);
+    tc::bar_init(acc_free, 128);
+    tc::fence_bar_init();
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = *tmem_slot;
+  bool fail = false;
+
+  if (warp == 0) {
+    // ---------------- bulk-copy producer ----------------
+    if (lane == 0) {
+      int g = 0;
+      for (int t = t_begin; t < t_end && !fail; ++t) {
+        for (int c = 0; c < kTcChunks; ++c, ++g) {
+          const int s = g % kTcStages;
+          if (g >= kTcStages &&
+              !tc::bar_wait(&stage_free[s], ((g - kTcStages) / kTcStages) & 1, kTcWaitPolls)) {
+            fail = true;
+            break;
+          }
+          float* dst = st + s * kWgStageFloats;
+          const float* sa = as + (size_t)t * kTcTileFloats + c * kTcBlockFloats;
+          const float* sb = bs + (size_t)t * kTcTileFloats + c * kTcBlockFloats;
+          tc::bar_arrive_expect_tx(&stage_full[s], kWgStageFloats * sizeof(float));
+          tc::bulk_load(dst, sa, kTcBlockFloats * sizeof(float), &stage_full[s]);
+          tc::bulk_load(dst + kTcBlockFloats, sa + kTcWFloats, kTcBlockFloats * sizeof(float), &stage_full[s]);
+          tc::bulk_load(dst + 2 * kTcBlockFloats, sb, kTcBlockFloats * sizeof(float), &stage_full[s]);
+          tc::bulk_load(dst + 3 * kTcBlockFloats, sb + kTcWFloats, kTcBlockFloats * sizeof(float),
+                        &stage_full[s]);
+        }
+      }
+      if (fail)   // let the copies already issued land
+        for (int k = 1; k <= kTcStages && g - k >= 0; ++k)
+          tc::bar_wait(&stage_full[(g - k) % kTcStages], ((g - k) / kTcStages) & 1, kTcWaitPolls);
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0) {
+      constexpr uint32_t idesc = tc::idesc_tf32(kTcC, kTcC);
+      constexpr uint32_t kLbo = kTcRows * 16, kSbo = 128;   // K group (4 rows), 8-channel group
+      int g = 0, seg = 0, cur_l = -1;
+      bool fresh = true;
+      for (int t = t_begin; t < t_end && !fail; ++t) {
+        const int l = tile_rank(geo, t);
+        if (l != cur_l) {
+          if (cur_l >= 0) {   // publish the finished rank, wait until it is drained
+            tc::commit(acc_full);
+            if (!tc::bar_wait(acc_free, seg & 1, kTcWaitPolls)) {
+              fail = true;
+              break;
+            }
+            ++seg;
+          }
+          cur_l = l;
+          fresh = true;
+        }
+        for (int c = 0; c < kTcChunks; ++c, ++g) {
+          const int s = g % kTcStages;
+          if (!tc::bar_wait(&stage_full[s], (g / kTcStages) & 1, kTcWaitPolls)) {
+            fail = true;
+            break;
+          }
+          tc::fence_after_sync();
+          const uint32_t a_h = tc::smem_addr(st + s * kWgStageFloats);
+          const uint32_t a_l = a_h + kTcBlockFloats * sizeof(float);
+          const uint32_t b_h = a_h + 2 * kTcBlockFloats * sizeof(float);
+          const uint32_t b_l = a_h + 3 * kTcBlockFloats * sizeof(float);
+#pragma unroll
+          for (int j = 0; j < kTcChunk / 8; ++j) {
+            const uint32_t kx = 2 * j * kLbo;
+            const uint64_t dah = tc::smem_desc(a_h + kx, kLbo, kSbo);
+            const uint64_t dal = tc::smem_desc(a_l + kx, kLbo, kSbo);
+            const uint64_t dbh = tc::smem_desc(b_h + kx, kLbo, kSbo);
+            const uint64_t dbl = tc::smem_desc(b_l + kx, kLbo, kSbo);
+            tc::mma_tf32(tmem, dah, dbh, idesc, (fresh && c == 0 && j == 0) ? 0u : 1u);
+            tc::mma_tf32(tmem, dal, dbh, idesc, 1u);
+            tc::mma_tf32(tmem, dah, dbl, idesc, 1u);
+          }
+          tc::commit(&stage_free[s]);
+        }
+        fresh = false;
+      }
+      if (!fail && cur_l >= 0) tc::commit(acc_full);   // the last rank of the range
+    }
+    __syncwarp();
+  } else if (warp >= 4) {
+    // ---------------- drain: D[k][j] -> Mbar_l at every rank change ----------------
+    const int ew = warp - 4;
+    const int k = 32 * ew + lane;
+    int seg = 0, cur_l = -1;
+    for (int t = t_begin; t <= t_end; ++t) {
+      const int l = t < t_end ? tile_rank(geo, t) : -1;
+      if (l == cur_l) continue;
+      if (cur_l >= 0) {
+        if (!tc::bar_wait(acc_full, seg & 1, kTcWaitPolls)) {
+          fail = true;
+          break;
+        }
+        tc::fence_after_sync();
+        float* Ml = Mbar + (size_t)cur_l * kTcC * kTcC + (size_t)k * kTcC;
+#pragma unroll 1
+        for (int q = 0; q < kTcC / 32; ++q) {
+          float v[32];
+          tc::tmem_ld32(tmem + ((uint32_t)(32 * ew) << 16) + 32 * q, v);
+#pragma unroll
+          for (int u = 0; u < 8; ++u)
+            red_add4(Ml + 32 * q + 4 * u, make_float4(v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3]));
+        }
+        tc::fence_before_sync();
+        tc::bar_arrive(acc_free);
+        ++seg;
+      }
+      cur_l = l;
+    }
+  }
+  if (fail) atomicExch(&g_tc_error, 1);
+  tc::fence_before_sync();
+  __syncthreads();
+  if (warp == 0) {
+    tc::fence_after_sync();
+    tc::tmem_dealloc(tmem, kTcRows);
+  }
+}
+
 int g_tc_smem_set[64] = {0};
+int g_wg_smem_set[64] = {0};
 
 }  // namespace
 
@@ -399,6 +607,33 @@ int launch_mix_tc(int L, int N, const float* xs, const float* ws, float* out, cu
   const int sms = device_sm_count();
   const int grid = T < sms ? T : sms;
   ladder_mix_tc_kernel<<<grid, kTcThreads, kTcSmemBytes, s>>>(g, xs, ws, out);
+  return cudaGetLastError() == cudaSuccess ? FC_OK : FC_ERR_CUDA;
+}
+
+int launch_mix_tc_split_cols(int L, int N, const float* in, float* xs, cudaStream_t s) {
+  const Geom g = make_geom(L, N);
+  const int T = tile_count(g);
+  if (T == 0) return FC_OK;
+  ladder_split_cols_kernel<<<T, 256, 0, s>>>(g, in, xs);
+  return cudaGetLastError() == cudaSuccess ? FC_OK : FC_ERR_CUDA;
+}
+
+int launch_wgrad_tc(int L, int N, const float* as, const float* bs, float* Mbar, cudaStream_t s) {
+  if (!mix_tc_supported(L, kTcC)) return FC_ERR_UNSUPPORTED_RANK;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return FC_ERR_CUDA;
+  if (!g_wg_smem_set[dev]) {
+    if (cudaFuncSetAttribute(ladder_wgrad_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)kWgSmemBytes) != cudaSuccess)
+      return FC_ERR_CUDA;
+    g_wg_smem_set[dev] = 1;
+  }
+  const Geom g = make_geom(L, N);
+  const int T = tile_count(g);
+  if (T == 0) return FC_OK;
+  const int sms = device_sm_count();
+  const int grid = T < sms ? T : sms;
+  ladder_wgrad_tc_kernel<<<grid, kWgThreads, kWgSmemBytes, s>>>(g, as, bs, Mbar);
   return cudaGetLastError() == cudaSuccess ? FC_OK : FC_ERR_CUDA;
 }
 
