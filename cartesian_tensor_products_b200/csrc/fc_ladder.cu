@@ -28,7 +28,11 @@
 
 namespace fc {
 
-constexpr int kLadderNodeChunk = 16;   // nodes per thread in the product kernels
+// nodes per thread: the forward products take short chunks (more CTAs in
+// flight to hide the memory latency); the product VJP keeps long ones because
+// it adds its path-weight gradients atomically once per chunk
+constexpr int kLadderFwdChunk = 4;
+constexpr int kLadderNodeChunk = 8;
 
 // ---------------------------------------------------------------------------
 // channel-diagonal products
@@ -44,8 +48,8 @@ __global__ void __launch_bounds__(128) ladder_tp_kernel(int N, int C, const floa
   float w[TP::P];
 #pragma unroll
   for (int p = 0; p < TP::P; ++p) w[p] = __ldg(W + (size_t)p * C + k);
-  const int n0 = blockIdx.x * kLadderNodeChunk;
-  const int n1 = min(N, n0 + kLadderNodeChunk);
+  const int n0 = blockIdx.x * kLadderFwdChunk;
+  const int n1 = min(N, n0 + kLadderFwdChunk);
   for (int n = n0; n < n1; ++n) {
     const size_t base = (size_t)n * TP::NY * C + k;
     float a[TP::NY], b[TP::NY], o[TP::NY];
@@ -75,8 +79,8 @@ __global__ void __launch_bounds__(128) ladder_tp_tiled_kernel(int N, const float
   float w[TP::P];
 #pragma unroll
   for (int p = 0; p < TP::P; ++p) w[p] = __ldg(W + (size_t)p * C + k);
-  const int n0 = blockIdx.x * kLadderNodeChunk;
-  const int n1 = min(N, n0 + kLadderNodeChunk);
+  const int n0 = blockIdx.x * kLadderFwdChunk;
+  const int n1 = min(N, n0 + kLadderFwdChunk);
   for (int n = n0; n < n1; ++n) {
     const size_t base = (size_t)n * TP::NY * C + k;
     float a[TP::NY], b[TP::NY], o[TP::NY];
@@ -370,7 +374,7 @@ static int check_ladder_desc(const fc_ladder_desc* d) {
 template <int L>
 static int launch_tp(int N, int C, const float* Av, const float* A1, const float* W, float* B,
                      cudaStream_t s) {
-  dim3 grid((N + kLadderNodeChunk - 1) / kLadderNodeChunk, (C + 127) / 128);
+  dim3 grid((N + kLadderFwdChunk - 1) / kLadderFwdChunk, (C + 127) / 128);
   ladder_tp_kernel<L><<<grid, 128, 0, s>>>(N, C, Av, A1, W, B);
   return cudaGetLastError() == cudaSuccess ? FC_OK : FC_ERR_CUDA;
 }
@@ -396,7 +400,7 @@ static int tp_dispatch(int L, int N, int C, const float* Av, const float* A1, co
 
 static int tp_tiled_dispatch(int L, int N, const float* Av, const float* A1, const float* W,
                              const MixTiles& tiles, float* xs, cudaStream_t s) {
-  const dim3 grid((N + kLadderNodeChunk - 1) / kLadderNodeChunk);
+  const dim3 grid((N + kLadderFwdChunk - 1) / kLadderFwdChunk);
   switch (L) {
     case 1: ladder_tp_tiled_kernel<1><<<grid, 128, 0, s>>>(N, Av, A1, W, tiles, xs); break;
     case 2: ladder_tp_tiled_kernel<2><<<grid, 128, 0, s>>>(N, Av, A1, W, tiles, xs); break;
