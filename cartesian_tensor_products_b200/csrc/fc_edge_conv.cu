@@ -1,25 +1,7 @@
-// libflashcart: receiver-sorted edge convolution, forward.
-//
-// FlashCart (arXiv 2610.06409) Sec. 4 Eq. (1) and Algorithm 1:
-//   z_{u eta k} = sum_{e: u_e = u} w_{e eta k} f_eta(x_{v_e k}, y_e),
-//   y_e = T(r-hat_e) shared by all channels.
-// Every receiver's sums are accumulated on chip and stored once.
-//
-// B200 design.  One CTA per (receiver, 128-channel tile); its G warps each
-// own a fixed group of output rows (path, component), cut offline so that
-// the warps do near-equal work.  A lane owns 4 consecutive channels, so
-// every global access is a coalesced 16-byte vector.  Per incoming edge a
-// warp needs the sender's x rows its rows touch and the edge's weight rows
-// of its paths: each lane streams its own 16-byte slices of those rows into
-// a 3-deep shared-memory ring with cp.async, three edges ahead of use, and
-// reads back only what it copied (no barrier on the data path).  Every 16
-// edges the warp forms, lane-per-edge, the entries
-// M[a][b] = sum_b2 K[a][b][b2] y_b2 (y = T(r-hat)) of its rows into a
-// warp-private shared-memory window; the per-edge loop then reads them as
-// broadcasts and applies them to the lane's 4 channels with packed FP32x2
-// FMAs.  Sender indices and edge vectors come from a 32-edge register
-// window (one per lane) read with warp shuffles.  With 4 groups every SMSP
-// runs one instruction stream (warp g of each resident CTA).
+// libflashcart: receiver-sorted edge convolution, forward (FlashCart
+// Sec. 4 Eq. (1), Algorithm 1): C ABI entry point and the rank 1-4
+// instantiations; the kernel templates and their design notes are in
+// fc_edge_conv.cuh, rank 5 is instantiated in fc_edge_conv_L5.cu.
 #include "fc_edge_conv.cuh"
 #include "generated/fc_fwd_L1.cuh"
 #include "generated/fc_fwd_L2.cuh"

@@ -1,30 +1,7 @@
-// libflashcart: receiver-sorted edge convolution, vector-Jacobian product.
-//
-// FlashCart (arXiv 2610.06409) App. C Eq. (C1) per edge, path and channel
-// (f bilinear, c = w f):
-//   x_bar_b1 = w sum_a g_a dF_a/dx_b1 = w (M^T g)_b1      -> sender v_e
-//   w_bar    = <g, f(x, y)> = <M^T g, x>                   -> stored per edge
-//   y_bar_b2 = w sum_a g_a dF_a/dy_b2                      -> edge e
-// summed as in Algorithm 2 (receiver-sorted, the receiver's g loaded once),
-// and carried through the direction tensors to the edge vector (App. C,
-// last paragraph of "Symbolic derivatives"):
-//   r_bar = (I - u u^T)/|r| (dT/du)^T y_bar,   u = r/|r|.
-//
-// B200 design.  Output paths are cut offline into G groups of whole paths
-// (h = M^T g needs every row of a path).  A CTA is (group, 4 consecutive
-// receiver tiles): its 4 warps run the same code, one receiver each, and
-// hold the receiver's g rows of the group's paths in registers for all its
-// edges; blocks are ordered group-major so an SMSP mostly runs one
-// instruction stream.  Sender
-// rows and edge weights are streamed through a per-warp cp.async ring as
-// in the forward kernel; M and dT/du are formed lane-per-edge into a
-// warp-private window.  Per edge a lane computes, for its 4 channels,
-// h = M^T g, w_bar = <h, x> (one coalesced 16-byte store per path), the
-// sender contribution w h (summed over the warp's paths, then one vector
-// atomic add per x_bar row, as Algorithm 2 adds sender gradients
-// atomically), and y_bar through d_(a,b1) = <g_a, w x_b1>; y_bar is folded
-// into u_bar = (dT/du)^T y_bar, reduced over the warp with shuffles and
-// added atomically (3 floats per warp and edge) into r_bar.
+// libflashcart: receiver-sorted edge convolution, vector-Jacobian product (FlashCart
+// App. C Eq. (C1), Algorithm 2): C ABI entry point and the rank 1-4
+// instantiations; the kernel templates and their design notes are in
+// fc_edge_conv_vjp.cuh, rank 5 is instantiated in fc_edge_conv_vjp_L5.cu.
 #include "fc_edge_conv_vjp.cuh"
 #include "generated/fc_vjp_L1.cuh"
 #include "generated/fc_vjp_L2.cuh"
