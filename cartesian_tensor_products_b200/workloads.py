@@ -164,6 +164,25 @@ def ladder_inputs(n_nodes, lmax, channels, order, seed):
     return dict(A1=A1, path_w=np.ascontiguousarray(path_w), mix_w=mix_w, gz=gz)
 
 
+def full_ladder_inputs(n_nodes, lmax, channels, order, seed):
+    """Full ladder (Sec. 5 Eq. 2): A ~ N(0,1); W1 ~ N(0, 1/C) per rank;
+    for each later step and rank l a [C][P_l C] map ~ N(0, 1/(P_l C)),
+    stored rank after rank; gz ~ N(0,1)."""
+    g = rng(seed)
+    ppr = paths_per_rank(lmax, lmax, lmax)
+    P = sum(ppr)
+    C = channels
+    A = normal(g, (n_nodes, (lmax + 1) ** 2 * C))
+    W1 = normal(g, (lmax + 1, C, C), 1.0 / np.sqrt(C))
+    blocks = []
+    for q in range(order - 1):
+        blocks.append(np.concatenate([normal(g, (C, p * C), 1.0 / np.sqrt(p * C)).ravel()
+                                      for p in ppr]))
+    Wq = np.stack(blocks) if blocks else np.zeros((0, C * P * C), np.float32)
+    gz = normal(g, (n_nodes, (lmax + 1) ** 2 * C))
+    return dict(A=A, W1=W1, Wq=np.ascontiguousarray(Wq, dtype=np.float32), gz=gz)
+
+
 def ladder(seed=4, n_nodes=4096, channels=128, lmax=3, order=4):
     d = ladder_inputs(n_nodes, lmax, channels, order, seed)
     return dict(name="ladder", n_nodes=n_nodes, lmax=lmax, channels=channels,

@@ -27,6 +27,7 @@
  *   - receiver-sorted convolution                  Sec. 4 Eq. (1)
  *   - array layout off(l) + (c P_l + eta) d + k    App. D "Data layout"
  *   - ladder product + channel mixing              Sec. 5 Eq. (2), App. E
+ *   - full ladder (paths kept, path+channel mix)   Sec. 5 Eq. (2)
  *
  * Readings where the pages are silent (each also listed in the design notes):
  *   - C_{l1 l2 l3} of Eq. (B1) is "defined elsewhere".  Here it is fixed so
@@ -1020,6 +1021,85 @@ int orc_ladder(int L, int C, int order, int N, const double *A1,
       for (size_t i = 0; i < nrow; ++i) z[(size_t)n * nrow + i] += An[i];
     }
     free(Av); free(B); free(An);
+  }
+  return 0;
+}
+
+/* Full correlation ladder, Sec. 5 Eq. (2): the products keep every path
+ * separate and a learned map mixes paths and channels per output rank.
+ *   phi_1[l,c,j] = sum_k W1[l][j][k] A[l,c,k]
+ *   B_q[eta,c,k] = f_eta(phi_{q-1}[l1,:,k], A[l2,:,k])_c          (q = 2 .. order)
+ *   phi_q[l,c,j] = sum_{eta -> l} sum_k Wq[l][j][eta_l C + k] B_q[eta,c,k]
+ *   z = phi_1 + ... + phi_order
+ * W1: [L+1][C][C]; Wq: [order-1] blocks of C*P*C, each the rank blocks
+ * [C][P_l C] one after the other (rank l at C * C * sum_{l'<l} P_l'), eta_l
+ * the path's position among the paths into rank l.
+ * states: [order][N][(L+1)^2 C] = phi_1 .. phi_order (may be NULL). */
+int orc_full_ladder(int L, int C, int order, int N, const double *A,
+                    const double *W1, const double *Wq,
+                    const unsigned char *node_mask, double *states, double *z) {
+  if (L > 4 || order < 1) return 1;
+  path_set ps;
+  make_paths(L, L, L, 0, &ps);
+  int row = (L + 1) * (L + 1);
+  size_t nrow = (size_t)row * C;
+  int rankoff[ORC_MAXL + 2];
+  rankoff[0] = 0;
+  for (int l = 0; l <= L; ++l) rankoff[l + 1] = rankoff[l] + ps.Pl[l];
+  if (states) memset(states, 0, sizeof(double) * (size_t)order * N * nrow);
+  memset(z, 0, sizeof(double) * (size_t)N * nrow);
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int n = 0; n < N; ++n) {
+    if (node_mask && !node_mask[n]) continue;
+    const double *a = A + (size_t)n * nrow;
+    double *phi = (double *)malloc(sizeof(double) * nrow);
+    double *nxt = (double *)malloc(sizeof(double) * nrow);
+    double *B = (double *)malloc(sizeof(double) * (size_t)ps.P * (2 * L + 1) * C);
+    double xc[2 * ORC_MAXL + 1], yc[2 * ORC_MAXL + 1], f[2 * ORC_MAXL + 1];
+    /* phi_1 */
+    for (int l = 0; l <= L; ++l)
+      for (int c = 0; c < 2 * l + 1; ++c)
+        for (int j = 0; j < C; ++j) {
+          double t = 0.0;
+          for (int k = 0; k < C; ++k)
+            t += W1[((size_t)l * C + j) * C + k] * a[(l * l + c) * C + k];
+          phi[(l * l + c) * C + j] = t;
+        }
+    for (int q = 1; q <= order; ++q) {
+      if (q > 1) {
+        /* B: per path p, component c, channel k at ((p * (2L+1)) + c) * C + k */
+        for (int p = 0; p < ps.P; ++p) {
+          int l1 = ps.l1[p], l2 = ps.l2[p], l3 = ps.l3[p];
+          for (int k = 0; k < C; ++k) {
+            for (int i = 0; i < 2 * l1 + 1; ++i) xc[i] = phi[(l1 * l1 + i) * C + k];
+            for (int i = 0; i < 2 * l2 + 1; ++i) yc[i] = a[(l2 * l2 + i) * C + k];
+            orc_product(l1, l2, l3, xc, yc, f);
+            for (int c = 0; c < 2 * l3 + 1; ++c)
+              B[((size_t)p * (2 * L + 1) + c) * C + k] = f[c];
+          }
+        }
+        const double *Wqq = Wq + (size_t)(q - 2) * C * ps.P * C;
+        for (int l = 0; l <= L; ++l) {
+          int K = ps.Pl[l] * C;
+          const double *Wl = Wqq + (size_t)C * C * rankoff[l];
+          for (int c = 0; c < 2 * l + 1; ++c)
+            for (int j = 0; j < C; ++j) {
+              double t = 0.0;
+              for (int p = 0; p < ps.P; ++p) {
+                if (ps.l3[p] != l) continue;
+                for (int k = 0; k < C; ++k)
+                  t += Wl[(size_t)j * K + ps.eta[p] * C + k] *
+                       B[((size_t)p * (2 * L + 1) + c) * C + k];
+              }
+              nxt[(l * l + c) * C + j] = t;
+            }
+        }
+        memcpy(phi, nxt, sizeof(double) * nrow);
+      }
+      if (states) memcpy(states + ((size_t)(q - 1) * N + n) * nrow, phi, sizeof(double) * nrow);
+      for (size_t i = 0; i < nrow; ++i) z[(size_t)n * nrow + i] += phi[i];
+    }
+    free(phi); free(nxt); free(B);
   }
   return 0;
 }

@@ -43,6 +43,7 @@ def lib():
             "orc_edge_conv_vjp2": (ct.c_int, [ct.c_int] * 7 + [i32, i32, d, d, d, d, d, d, d, u8,
                                                                d, d, d, d]),
             "orc_direction_hvp": (None, [ct.c_int, d, d, d, d]),
+            "orc_full_ladder": (ct.c_int, [ct.c_int] * 4 + [d, d, d, u8, d, d]),
             "orc_ladder": (ct.c_int, [ct.c_int] * 4 + [d, d, d, u8, d, d]),
             "orc_ladder_vjp": (ct.c_int, [ct.c_int] * 4 + [d, d, d, d, u8, d, d, d]),
             "orc_max_rank": (ct.c_int, []),
@@ -397,3 +398,24 @@ def block_energy_forces(L, C, order, edge_index, edge_vec, x, omega, path_w, mix
     np.add.at(F, ei[1], -dEdr)
     np.add.at(F, ei[0], dEdr)
     return e_node, dEdr, F
+
+
+def full_ladder(L, C, order, A, W1, Wq, node_mask=None):
+    """Full correlation ladder (Sec. 5 Eq. 2): per-path products, each step's
+    paths and channels mixed per output rank by Wq; returns (states
+    [order][N][(L+1)^2 C] = phi_1..phi_order, z = their sum).  W1:
+    [L+1][C][C]; Wq: [order-1][C*P*C], rank blocks [C][P_l C] in rank order."""
+    A = _d(A)
+    N = A.shape[0]
+    P = len(paths(L, L, L))
+    W1 = _d(W1).reshape(L + 1, C, C)
+    Wq = _d(Wq).reshape(order - 1, C * P * C) if order > 1 else np.zeros((1, C * P * C))
+    states = np.empty((order, N, (L + 1) ** 2 * C))
+    z = np.empty((N, (L + 1) ** 2 * C))
+    m = None if node_mask is None else _mask(node_mask, N)
+    rc = lib().orc_full_ladder(L, C, order, N, _pd(A), _pd(W1), _pd(np.ascontiguousarray(Wq)),
+                               None if m is None else m.ctypes.data_as(ct.POINTER(ct.c_uint8)),
+                               _pd(states), _pd(z))
+    assert rc == 0
+    return states, z
+
