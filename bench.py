@@ -16,6 +16,7 @@ time is the max over ranks.  --impl reference times the FP64 CPU oracle on a
 bounded sample of the same workload (rank 0 only).
 """
 import argparse
+import ctypes
 import json
 import os
 import statistics
@@ -227,7 +228,7 @@ def time_events(fn, steps, warmup, stream, flush=None):
 
 
 ROW_NAMES = ("edge_conv_vjp_r3", "edge_conv_vvjp_r3", "edge_conv_fwd_r4", "edge_conv_vjp_r4",
-             "ladder", "block_energy_forces")
+             "ladder", "full_ladder", "block_energy_forces")
 
 
 def extra_rows(fc, W, dev, stream, peaks, fp32_peak, steps, select=ROW_NAMES):
@@ -392,6 +393,34 @@ def extra_rows(fc, W, dev, stream, peaks, fp32_peak, steps, select=ROW_NAMES):
                               3 * mix_flops if tc else 0, mslb),
             "l2_flush": "256 MB written before every call"}
         del A1, pw, mw, gz, ws, res, states
+        torch.cuda.empty_cache()
+
+    if "full_ladder" in select:
+        # --- full ladder (path-separated products + per-rank path/channel maps), forward
+        Lf, Cf, of, Nf = 3, 128, 4, 4096
+        fd = W.full_ladder_inputs(Nf, Lf, Cf, of, 44)
+        A = torch.from_numpy(fd["A"]).to(dev)
+        W1 = torch.from_numpy(fd["W1"]).to(dev)
+        Wq = torch.from_numpy(fd["Wq"]).to(dev)
+        wsf = torch.empty(fc.lib().fc_full_ladder_workspace_size(
+            ctypes.byref(fc.LadderDesc(Lf, Cf, of)), Nf) // 4, device=dev)
+        msf, mnf = time_events(lambda: fc.full_ladder(Lf, of, A, W1, Wq, workspace=wsf), steps, 3, stream,
+                               flush=flush)
+        P = fc.num_paths(Lf)
+        rows_l = Nf * 16
+        mix_fl = 2 * rows_l * Cf * Cf + (of - 1) * 2 * Nf * sum(
+            (2 * l + 1) * p for l, p in enumerate(W.paths_per_rank(Lf, Lf, Lf))) * Cf * Cf
+        tp_fl = (of - 1) * Nf * Cf * 2 * 751
+        rows["full_ladder_fwd"] = {
+            "workload": "4096 nodes x 128 channels, rank 3, order 4: path-separated products, "
+                        "per-rank (P_l x 128) -> 128 maps (FP32 SIMT GEMMs)",
+            "ms": msf, "ms_min": mnf,
+            "roofline": {"bound": "alu", "achieved": (mix_fl + tp_fl) / (msf * 1e-3) / 1e12,
+                         "peak": fp32_peak, "unit": "TFLOP/s",
+                         "frac": (mix_fl + tp_fl) / (msf * 1e-3) / 1e12 / fp32_peak,
+                         "algorithmic_flops": mix_fl + tp_fl},
+            "l2_flush": "256 MB written before every call"}
+        del A, W1, Wq, wsf
         torch.cuda.empty_cache()
 
     if "block_energy_forces" in select:

@@ -68,6 +68,9 @@ _SIGS = {
                                          _vp, _vp, _vp, _vp, _vp, ct.c_size_t, _vp]),
     "fc_device_error": (ct.c_int, [ct.POINTER(ct.c_int), _vp]),
     "fc_edge_conv_vjp_vjp": (ct.c_int, [ct.POINTER(ConvDesc), ct.c_int, ct.c_int] + [_vp] * 14),
+    "fc_full_ladder_workspace_size": (ct.c_size_t, [ct.POINTER(LadderDesc), ct.c_int]),
+    "fc_full_ladder": (ct.c_int, [ct.POINTER(LadderDesc), ct.c_int, _vp, _vp, _vp, _vp, _vp, _vp,
+                                  ct.c_size_t, _vp]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _f = getattr(_lib, _name)
@@ -317,6 +320,28 @@ def product_ladder_vjp(lmax, order, A1, path_w, mix_w, states, gz, workspace=Non
         _ptr(workspace), ws_bytes if workspace is not None else 0, _stream(stream)),
         "fc_product_ladder_vjp")
     return A1b, pwb, mwb
+
+
+def full_ladder(lmax, order, A, W1, Wq, workspace=None, stream=None):
+    """(states [order][N][...] = phi_1..phi_order, z) of the full ladder
+    (Sec. 5 Eq. 2): path-separated products, per-rank path+channel maps."""
+    _dev(A, torch.float32, "A")
+    _dev(W1, torch.float32, "W1")
+    N = A.shape[0]
+    NY = (lmax + 1) ** 2
+    C = A.shape[1] // NY
+    d = LadderDesc(lmax, C, order)
+    states = torch.empty((order, N, NY * C), dtype=torch.float32, device=A.device)
+    z = torch.empty_like(A)
+    if order > 1:
+        _dev(Wq, torch.float32, "Wq")
+    ws_bytes = _lib.fc_full_ladder_workspace_size(ct.byref(d), N)
+    workspace, ws_bytes = _scratch(workspace, ws_bytes, A.device)
+    _check(_lib.fc_full_ladder(ct.byref(d), N, _ptr(A), _ptr(W1), _ptr(Wq) if order > 1 else None,
+                               _ptr(states), _ptr(z), _ptr(workspace),
+                               ws_bytes if workspace is not None else 0, _stream(stream)),
+           "fc_full_ladder")
+    return states, z
 
 
 def device_error(stream=None):

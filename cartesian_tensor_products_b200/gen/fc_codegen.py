@@ -1049,6 +1049,19 @@ def emit_ladder(L):
                               for b1, b2, k in terms)
             o.append("    B[%d] = fmaf(w[%d], %s, B[%d]);" % (l3 * l3 + c, p, expr, l3 * l3 + c))
     o.append("  }")
+    # full ladder: every path kept, written at its output slot
+    # zoff[l3] + c P_l3 + eta of a [ZROW][C] row (stride C)
+    o.append("  static constexpr int ZROW = %d;" % T.zrow)
+    o.append("  static __device__ __forceinline__ void fwd_paths(const float (&a)[NY], const float (&b)[NY], float* __restrict__ o, int C) {")
+    for p, (l1, l2, l3) in enumerate(T.paths):
+        K = T.K[p]
+        for c in range(2 * l3 + 1):
+            terms = [(b1, b2, K[c][b1][b2]) for b1 in range(2 * l1 + 1)
+                     for b2 in range(2 * l2 + 1) if K[c][b1][b2] != 0]
+            expr = " + ".join("%s*(a[%d]*b[%d])" % (flit(k), l1 * l1 + b1, l2 * l2 + b2)
+                              for b1, b2, k in terms) or "0.0f"
+            o.append("    o[(size_t)%d * C] = %s;" % (T.zslot(p, c), expr))
+    o.append("  }")
     # VJP: g is the gradient of B
     o.append("  static __device__ __forceinline__ void vjp(const float (&a)[NY], const float (&b)[NY], const float (&w)[P], const float (&g)[NY],")
     o.append("                                             float (&abar)[NY], float (&bbar)[NY], float (&wbar)[P]) {")

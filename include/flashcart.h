@@ -291,6 +291,26 @@ int fc_product_ladder_noalloc(const fc_ladder_desc *desc, int n_nodes,
                               const float *mix_w, float *states, float *z,
                               fc_stream_t stream);
 
+/* The full correlation ladder, forward: Sec. 5 Eq. (2) with every coupling
+ * path kept and a learned map that mixes paths and channels per output rank:
+ *   phi_1[l,c,:] = W1_l A[l,c,:]                              (C x C per rank)
+ *   B_q[eta,c,k] = f_eta(phi_{q-1}[l1,:,k], A[l2,:,k])_c      (q = 2 .. order)
+ *   phi_q[l,c,j] = sum_{eta -> l} sum_k Wq_l[j][eta_l C + k] B_q[eta,c,k]
+ *   z = phi_1 + ... + phi_order
+ * with eta_l the path's position among the paths into rank l (paths ordered
+ * by l3, then l1, then l2).  Ranks 1..4, channels a multiple of 4.
+ *   A [n_nodes][(lmax+1)^2 C]; W1 [lmax+1][C][C] (row = output channel);
+ *   Wq [order-1][C P C]: per step the rank blocks [C][P_l C] one after the
+ *   other (rank l at C C sum_{l'<l} P_l'); states [order][n_nodes][(lmax+1)^2 C]
+ *   receives phi_1 .. phi_order; z [n_nodes][(lmax+1)^2 C].
+ * workspace: fc_full_ladder_workspace_size() bytes (one path-separated
+ * product, n_nodes x fc_conv_out_row x C floats), 16-byte aligned; none for
+ * order 1.  Returns the statuses of fc_product_ladder. */
+size_t fc_full_ladder_workspace_size(const fc_ladder_desc *desc, int n_nodes);
+int fc_full_ladder(const fc_ladder_desc *desc, int n_nodes, const float *A,
+                   const float *W1, const float *Wq, float *states, float *z,
+                   void *workspace, size_t ws_bytes, fc_stream_t stream);
+
 /* Sticky device-side error word of the kernels that wait on barriers (the
  * tensor-core ladder mix): each wait gives up after a bounded number of
  * polls, skips the rest of its work and sets the word instead of hanging.
