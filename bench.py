@@ -206,6 +206,22 @@ def weak_throughput(world, units_per_rank, steps, max_ms):
     return world * units_per_rank * steps / (max_ms * 1e-3)
 
 
+def composite_bound(peaks, fp32_peak, byts, fp32_fl, tf32_fl, ms, algo_flops):
+    """Roofline of a chain of kernels: the largest of HBM time for the
+    algorithmic bytes, FP32 time for the SIMT flops and tensor time for the
+    TF32 products (tcgen05 TF32 peak = the measured bf16 peak x the nominal
+    tf32/bf16 ratio 1.1/2.25; the three-term split counts three products)."""
+    tf32_peak = peaks["bf16_tflops"] * 1.1 / 2.25
+    t = {"hbm": byts / (peaks["hbm_gbs"] * 1e9), "fp32": fp32_fl / (fp32_peak * 1e12),
+         "tf32": tf32_fl / (tf32_peak * 1e12)}
+    key = max(t, key=t.get)
+    return {"bound": "alu" if key != "hbm" else "hbm", "limit": key,
+            "t_roof_us": 1e6 * t[key], "frac": t[key] / (ms * 1e-3),
+            "terms_us": {k: 1e6 * v for k, v in t.items()},
+            "peaks": {"hbm_gbs": peaks["hbm_gbs"], "fp32_tflops": fp32_peak, "tf32_tflops": tf32_peak},
+            "algorithmic_flops": algo_flops, "algorithmic_bytes": byts}
+
+
 def time_events(fn, steps, warmup, stream, flush=None):
     """Mean device time (ms) of fn over `steps` calls, CUDA events on the
     launching stream; optional L2 flush before every call (not timed)."""
@@ -362,21 +378,9 @@ def extra_rows(fc, W, dev, stream, peaks, fp32_peak, steps, select=ROW_NAMES):
         tp_flops = S * Nl * Cl * 2 * 751
         plane_b = 4 * Nl * 16 * Cl
         tc = Cl == 128
-        # tcgen05 TF32 peak: the measured bf16 peak x the nominal tf32/bf16 ratio (1.1/2.25);
-        # the three-term split issues three TF32 products per mixing product
-        tf32_peak = peaks["bf16_tflops"] * 1.1 / 2.25
 
         def bound(byts, fp32_fl, tf32_fl, ms):
-            t = {"hbm": byts / (peaks["hbm_gbs"] * 1e9), "fp32": fp32_fl / (fp32_peak * 1e12),
-                 "tf32": tf32_fl / (tf32_peak * 1e12)}
-            key = max(t, key=t.get)
-            return {"bound": "alu" if key != "hbm" else "hbm", "limit": key,
-                    "t_roof_us": 1e6 * t[key], "frac": t[key] / (ms * 1e-3),
-                    "terms_us": {k: 1e6 * v for k, v in t.items()},
-                    "peaks": {"hbm_gbs": peaks["hbm_gbs"], "fp32_tflops": fp32_peak,
-                              "tf32_tflops": tf32_peak},
-                    "algorithmic_flops": mix_flops + tp_flops,
-                    "algorithmic_bytes": byts}
+            return composite_bound(peaks, fp32_peak, byts, fp32_fl, tf32_fl, ms, mix_flops + tp_flops)
         # forward: A1 read, states written, z written; products FP32; mix TF32 x3 (or FP32)
         fb = plane_b * (1 + S + 1)
         rows["ladder_fwd"] = {
@@ -411,14 +415,13 @@ def extra_rows(fc, W, dev, stream, peaks, fp32_peak, steps, select=ROW_NAMES):
         mix_fl = 2 * rows_l * Cf * Cf + (of - 1) * 2 * Nf * sum(
             (2 * l + 1) * p for l, p in enumerate(W.paths_per_rank(Lf, Lf, Lf))) * Cf * Cf
         tp_fl = (of - 1) * Nf * Cf * 2 * 751
+        # A read, order states and z written; products FP32; maps TF32 x3 on the tensor cores
+        fbf = 4 * Nf * 16 * Cf * (1 + of + 1)
         rows["full_ladder_fwd"] = {
             "workload": "4096 nodes x 128 channels, rank 3, order 4: path-separated products, "
-                        "per-rank (P_l x 128) -> 128 maps (FP32 SIMT GEMMs)",
+                        "per-rank (P_l x 128) -> 128 maps on tcgen05 (three-term TF32)",
             "ms": msf, "ms_min": mnf,
-            "roofline": {"bound": "alu", "achieved": (mix_fl + tp_fl) / (msf * 1e-3) / 1e12,
-                         "peak": fp32_peak, "unit": "TFLOP/s",
-                         "frac": (mix_fl + tp_fl) / (msf * 1e-3) / 1e12 / fp32_peak,
-                         "algorithmic_flops": mix_fl + tp_fl},
+            "roofline": composite_bound(peaks, fp32_peak, fbf, tp_fl, 3 * mix_fl, msf, mix_fl + tp_fl),
             "l2_flush": "256 MB written before every call"}
         del A, W1, Wq, wsf
         torch.cuda.empty_cache()

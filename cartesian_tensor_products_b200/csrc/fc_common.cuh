@@ -85,4 +85,52 @@ int launch_mix_tc_split_cols(int L, int N, const float* in, float* xs, cudaStrea
 // Mbar[l][k][j] += sum over the rows of rank l of a[row][k] b[row][j] (both transposed split)
 int launch_wgrad_tc(int L, int N, const float* as, const float* bs, float* Mbar, cudaStream_t s);
 
+// Tensor-core path + channel map of the full ladder (fc_mix_tc.cu), C = 128.
+// Rows of rank l (node n, component c) carry K = 32 k_l inputs (k_l = 4 P_l:
+// P_l paths x 128 channels).  They form 128-row tiles t_l .. t_{l+1} - 1,
+// component-major: tile t_l + c nb + n / 128 holds component c of nodes
+// 128 (n / 128) + 0..127 (nb = ceil(N / 128); rows past node N - 1 unused).
+// A tile is k_l hi blocks then k_l lo blocks of 4096 floats (128 rows x 32
+// inputs, core-matrix layout), and rank l's tiles start at float
+// pg_xbase(l) of the operand buffer.  The map of rank l ([128][K]) is split
+// the same way: k_l hi then k_l lo blocks from float pg_wbase(l).
+struct PathGeom {
+  int N, NY, L, nb;
+  int t1, t2, t3, t4, t5;   // first tile of ranks 1..5 (t_{L+1} = all tiles)
+  int k0, k1, k2, k3, k4;   // K chunks per row of ranks 0..4
+};
+__host__ __device__ __forceinline__ int pg_ts(const PathGeom& g, int l) {
+  return l <= 0 ? 0 : l == 1 ? g.t1 : l == 2 ? g.t2 : l == 3 ? g.t3 : l == 4 ? g.t4 : g.t5;
+}
+__host__ __device__ __forceinline__ int pg_kc(const PathGeom& g, int l) {
+  return l == 0 ? g.k0 : l == 1 ? g.k1 : l == 2 ? g.k2 : l == 3 ? g.k3 : g.k4;
+}
+__host__ __device__ __forceinline__ int pg_rank(const PathGeom& g, int t) {
+  return (g.L >= 1 && t >= g.t1) + (g.L >= 2 && t >= g.t2) + (g.L >= 3 && t >= g.t3) +
+         (g.L >= 4 && t >= g.t4);
+}
+__host__ __device__ __forceinline__ long long pg_xbase(const PathGeom& g, int l) {
+  long long b = 0;
+#pragma unroll
+  for (int r = 0; r < 5; ++r)
+    if (r < l) b += (long long)(pg_ts(g, r + 1) - pg_ts(g, r)) * pg_kc(g, r) * 8192;
+  return b;
+}
+__host__ __device__ __forceinline__ long long pg_wbase(const PathGeom& g, int l) {
+  long long b = 0;
+#pragma unroll
+  for (int r = 0; r < 5; ++r)
+    if (r < l) b += (long long)pg_kc(g, r) * 8192;
+  return b;
+}
+// kc[l] = K chunks per row of rank l (l <= L <= 4)
+PathGeom path_geom(int L, int N, const int* kc);
+// natural [N][(L+1)^2][128] -> operand tiles with k_l = 4 (the map of phi_1)
+int launch_path_split_rows(const PathGeom& g, const float* in, float* xs, cudaStream_t s);
+// the maps, rank l's ([128][32 k_l] row-major) at W + 4096 sum_{l'<l} k_l',
+// -> split blocks at ws + pg_wbase(l)
+int launch_path_split_map(const PathGeom& g, const float* W, float* ws, cudaStream_t s);
+// out[n][l^2 + c][j] = sum_k W_l[j][k] x_l[(n, c)][k]
+int launch_path_mix_tc(const PathGeom& g, const float* xs, const float* ws, float* out, cudaStream_t s);
+
 }  // namespace fc

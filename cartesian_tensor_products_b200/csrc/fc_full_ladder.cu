@@ -13,8 +13,17 @@
 // per CTA, 4 x 8 outputs per thread) with z += phi_q in its epilogue.  The
 // products are channel-diagonal: one thread per channel, generated
 // straight-line code per path (exact coefficients).
+//
+// At C = 128 the maps run on the tcgen05 tensor cores (fc_mix_tc.cu,
+// three-term TF32 split): the product kernel writes B_q straight into the
+// split tile layout the MMAs read (input k of a rank-l row = eta_l C +
+// channel), phi_1 reads A split into the same tiles; z is summed
+// from the states at the end.  Rows past the last node of a tile are never
+// written: the MMA column of such a row depends on that row alone and is not
+// stored.
 #include "fc_common.cuh"
 #include "fc_device.cuh"
+#include "fc_tc.cuh"
 #include "generated/fc_ladder_L1.cuh"
 #include "generated/fc_ladder_L2.cuh"
 #include "generated/fc_ladder_L3.cuh"
@@ -44,6 +53,56 @@ __global__ void __launch_bounds__(128) full_tp_paths_kernel(int N, int C, const 
       b[i] = __ldg(A + base + (size_t)i * C);
     }
     TP::fwd_paths(a, b, Bz + (size_t)n * TP::ZROW * C + k, C);
+  }
+}
+
+// The same products at C = 128, written as the TF32 hi / lo split of the
+// path-mix operand (component-major PathGeom tiles, k_l = 4 P_l).
+// A warp takes 8 consecutive nodes x 4 consecutive channels: for one output
+// (path, component) its 32 values are exactly one 128-byte core matrix
+// (8 rows x 4 inputs), so every store instruction writes one full line.
+template <int L>
+__global__ void __launch_bounds__(256, 2) full_tp_tiled_kernel(PathGeom g, const float* __restrict__ phi,
+                                                            const float* __restrict__ A,
+                                                            float* __restrict__ xs) {
+  using TP = LadderTP<L>;
+  constexpr int C = 128;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int n = 8 * blockIdx.x + (lane >> 2);
+  const int k = 32 * blockIdx.y + 4 * warp + (lane & 3);
+  if (n >= g.N) return;
+  const int kq = k >> 5, kk = k & 31;   // chunk within a path, input within the chunk
+  const int r = n & 127, nblk = n >> 7;
+  const size_t base = (size_t)n * TP::NY * C + k;
+  float a[TP::NY], b[TP::NY];
+#pragma unroll
+  for (int i = 0; i < TP::NY; ++i) {
+    a[i] = __ldg(phi + base + (size_t)i * C);
+    b[i] = __ldg(A + base + (size_t)i * C);
+  }
+  const int cofs = tc::core_offset(r, kk, 128);
+  TP::fwd_paths_to(a, b, [&](int l3, int c, int eta, float v) {
+    const int kc = pg_kc(g, l3);
+    float* hi = xs + pg_xbase(g, l3) + (long long)(c * g.nb + nblk) * kc * 8192 + (eta * 4 + kq) * 4096 + cofs;
+    uint32_t h, lo;
+    tc::split_tf32(v, h, lo);
+    hi[0] = __uint_as_float(h);
+    hi[(size_t)kc * 4096] = __uint_as_float(lo);
+  });
+}
+
+// z = sum of the order states
+__global__ void __launch_bounds__(256) full_sum_kernel(size_t plane4, int order,
+                                                       const float4* __restrict__ states,
+                                                       float4* __restrict__ z) {
+  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < plane4;
+       i += (size_t)gridDim.x * blockDim.x) {
+    float4 acc = __ldg(states + i);
+    for (int q = 1; q < order; ++q) {
+      const float4 v = __ldg(states + (size_t)q * plane4 + i);
+      acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+    }
+    z[i] = acc;
   }
 }
 
@@ -159,6 +218,19 @@ int tp_paths_dispatch(int L, int N, int C, const float* phi, const float* A, flo
   return FC_ERR_UNSUPPORTED_RANK;
 }
 
+int tp_tiled_dispatch(int L, const PathGeom& g, const float* phi, const float* A, float* xs,
+                      cudaStream_t s) {
+  const dim3 grid((g.N + 7) / 8, 4);
+  switch (L) {
+    case 1: full_tp_tiled_kernel<1><<<grid, 256, 0, s>>>(g, phi, A, xs); break;
+    case 2: full_tp_tiled_kernel<2><<<grid, 256, 0, s>>>(g, phi, A, xs); break;
+    case 3: full_tp_tiled_kernel<3><<<grid, 256, 0, s>>>(g, phi, A, xs); break;
+    case 4: full_tp_tiled_kernel<4><<<grid, 256, 0, s>>>(g, phi, A, xs); break;
+    default: return FC_ERR_UNSUPPORTED_RANK;
+  }
+  return cudaGetLastError() == cudaSuccess ? FC_OK : FC_ERR_CUDA;
+}
+
 // paths into each output rank (all l1, l2 <= L)
 void rank_paths(int L, int* Pl) {
   for (int l3 = 0; l3 <= L; ++l3) {
@@ -168,6 +240,21 @@ void rank_paths(int L, int* Pl) {
         if (l3 >= (l1 > l2 ? l1 - l2 : l2 - l1) && l3 <= l1 + l2 && ((l1 + l2 + l3) & 1) == 0) ++Pl[l3];
   }
 }
+
+// tile geometries of the tensor-core path: phi_1 (K = C per rank) and the
+// path-separated steps (K = P_l C)
+void tc_geoms(int L, int N, PathGeom& g1, PathGeom& gq) {
+  int Pl[6] = {0, 0, 0, 0, 0, 0}, k1[5] = {0, 0, 0, 0, 0}, kq[5] = {0, 0, 0, 0, 0};
+  rank_paths(L, Pl);
+  for (int l = 0; l <= L; ++l) {
+    k1[l] = 4;
+    kq[l] = 4 * Pl[l];
+  }
+  g1 = path_geom(L, N, k1);
+  gq = path_geom(L, N, kq);
+}
+
+size_t tc_operand_floats(const PathGeom& gq) { return (size_t)pg_xbase(gq, gq.L + 1); }
 
 int check_full_desc(const fc_ladder_desc* d) {
   if (!d) return FC_ERR_ARG;
@@ -183,7 +270,13 @@ int check_full_desc(const fc_ladder_desc* d) {
 using namespace fc;
 
 extern "C" size_t fc_full_ladder_workspace_size(const fc_ladder_desc* d, int n_nodes) {
-  if (check_full_desc(d) != FC_OK || n_nodes < 0 || d->order < 2) return 0;
+  if (check_full_desc(d) != FC_OK || n_nodes < 0) return 0;
+  if (mix_tc_supported(d->lmax, d->channels)) {
+    PathGeom g1, gq;
+    tc_geoms(d->lmax, n_nodes, g1, gq);
+    return sizeof(float) * (tc_operand_floats(gq) + (size_t)pg_wbase(gq, gq.L + 1));
+  }
+  if (d->order < 2) return 0;
   return sizeof(float) * (size_t)n_nodes * out_row(d->lmax, 0) * d->channels;
 }
 
@@ -200,9 +293,32 @@ extern "C" int fc_full_ladder(const fc_ladder_desc* d, int n_nodes, const float*
       (order > 1 && !aligned16(Wq)))
     return FC_ERR_ALIGN;
   const size_t need = fc_full_ladder_workspace_size(d, n_nodes);
-  if (order > 1 && (!workspace || ws_bytes < need)) return FC_ERR_WORKSPACE;
-  if (order > 1 && !aligned16(workspace)) return FC_ERR_ALIGN;
+  if (need > 0 && (!workspace || ws_bytes < need)) return FC_ERR_WORKSPACE;
+  if (need > 0 && !aligned16(workspace)) return FC_ERR_ALIGN;
   cudaStream_t s = (cudaStream_t)stream;
+  if (mix_tc_supported(L, C)) {
+    // tensor-core maps, then z = phi_1 + ... + phi_order
+    PathGeom g1, gq;
+    tc_geoms(L, n_nodes, g1, gq);
+    float* xs = static_cast<float*>(workspace);
+    float* wsm = xs + tc_operand_floats(gq);
+    const size_t plane = (size_t)n_nodes * (L + 1) * (L + 1) * C;
+    const size_t wq_step = (size_t)C * num_paths(L) * C;
+    if ((st = launch_path_split_rows(g1, A, xs, s)) != FC_OK ||
+        (st = launch_path_split_map(g1, W1, wsm, s)) != FC_OK ||
+        (st = launch_path_mix_tc(g1, xs, wsm, states, s)) != FC_OK)
+      return st;
+    for (int q = 2; q <= order; ++q) {
+      if ((st = tp_tiled_dispatch(L, gq, states + (size_t)(q - 2) * plane, A, xs, s)) != FC_OK ||
+          (st = launch_path_split_map(gq, Wq + (size_t)(q - 2) * wq_step, wsm, s)) != FC_OK ||
+          (st = launch_path_mix_tc(gq, xs, wsm, states + (size_t)(q - 1) * plane, s)) != FC_OK)
+        return st;
+    }
+    full_sum_kernel<<<8 * device_sm_count(), 256, 0, s>>>(plane / 4, order,
+                                                         reinterpret_cast<const float4*>(states),
+                                                         reinterpret_cast<float4*>(z));
+    return cudaGetLastError() == cudaSuccess ? FC_OK : FC_ERR_CUDA;
+  }
   const int NY = (L + 1) * (L + 1);
   const size_t plane = (size_t)n_nodes * NY * C;
   int Pl[6] = {0, 0, 0, 0, 0, 0};

@@ -551,8 +551,261 @@ __global__ void __launch_bounds__(kWgThreads, 1) ladder_wgrad_tc_kernel(Geom geo
   }
 }
 
+// ---------------------------------------------------------------------------
+// path + channel map of the full ladder: out[row][j] = sum_k W_l[j][k] x[row][k]
+// ---------------------------------------------------------------------------
+// A row of rank l has K = 32 k_l inputs (P_l paths x 128 channels), more than
+// one stage holds, so each stage carries a K chunk of both operands: the
+// tile's 128 rows x 32 inputs and the map's 128 outputs x 32 inputs (hi and
+// lo of each, 64 KB), three stages deep.  The map chunks are re-read from L2
+// by every tile of the rank (a map is at most 1.3 MB split).  CTAs take
+// contiguous tile ranges of equal K-chunk count (tiles of different ranks
+// differ in length).  Roles as in the mix above, with one change for
+// accuracy: the tensor core's FP32 accumulation loses a little at every
+// MMA, and over K = P_l 128 inputs (up to 336 MMAs) that loss builds up past
+// the forward tolerance.  So each path (4 chunks, the K of the plain mix)
+// goes to its own TMEM accumulator, two alternating, and the epilogue adds
+// the partial sums in FP32 registers (round-to-nearest) before it writes
+// the tile out.  The epilogue only stores (a read-modify-write of a running
+// sum here serialised on load latency and starved the tensor pipe).
+constexpr int kPmGroup = 4;   // chunks per accumulator: one path of 128 inputs
+
+constexpr int kPmStageFloats = 4 * kTcBlockFloats;   // x hi, x lo, W hi, W lo
+constexpr size_t kPmSmemBytes = sizeof(float) * kTcStages * kPmStageFloats + 8 * 16 + 8;
+static_assert(kPmSmemBytes <= 232448, "shared memory per CTA");
+
+__device__ __forceinline__ long long pg_chunks_before(const PathGeom& g, int l) {
+  long long c = 0;
+#pragma unroll
+  for (int r = 0; r < 5; ++r)
+    if (r < l) c += (long long)(pg_ts(g, r + 1) - pg_ts(g, r)) * pg_kc(g, r);
+  return c;
+}
+
+// first tile that starts at or after K chunk P of the whole operand
+__device__ __forceinline__ int pg_tile_at(const PathGeom& g, long long P) {
+  long long cum = 0;
+  for (int l = 0; l <= g.L; ++l) {
+    const int nt = pg_ts(g, l + 1) - pg_ts(g, l), kc = pg_kc(g, l);
+    const long long cl = (long long)nt * kc;
+    if (P < cum + cl) return pg_ts(g, l) + (int)((P - cum + kc - 1) / kc);
+    cum += cl;
+  }
+  return pg_ts(g, g.L + 1);
+}
+
+// natural [N][NY][128] -> component-major operand tiles with k_l = 4 (one
+// CTA per tile chunk; thread mapping as in ladder_split_rows_kernel).
+__global__ void __launch_bounds__(256) path_split_rows_kernel(PathGeom g, const float* __restrict__ in,
+                                                              float* __restrict__ xs) {
+  const int t = blockIdx.x, c = blockIdx.y;
+  const int p = threadIdx.x, lane = p & 31;
+  const int l = pg_rank(g, t);
+  const int tr = t - pg_ts(g, l);
+  const int comp = tr / g.nb, n0 = (tr - comp * g.nb) * kTcRows;
+  float* hi = xs + pg_xbase(g, l) + (size_t)tr * 4 * 2 * kTcBlockFloats + c * kTcBlockFloats;
+#pragma unroll
+  for (int it = 0; it < 4; ++it) {
+    const int r = 16 * (p >> 5) + 8 * (it >> 1) + (lane & 7);
+    const int q = (lane >> 3) + 4 * (it & 1);
+    const int n = n0 + r;
+    float4 v = zero4();
+    if (n < g.N)
+      v = __ldg(reinterpret_cast<const float4*>(in + ((size_t)n * g.NY + l * l + comp) * kTcC + c * kTcChunk) + q);
+    uint4 h, w;
+    split4(v, h, w);
+    const int off = tc::core_offset(r, 4 * q, kTcRows);
+    *reinterpret_cast<uint4*>(hi + off) = h;
+    *reinterpret_cast<uint4*>(hi + 4 * kTcBlockFloats + off) = w;
+  }
+}
+
+__global__ void __launch_bounds__(256) path_split_map_kernel(PathGeom g, const float* __restrict__ W,
+                                                             float* __restrict__ ws) {
+  const int l = blockIdx.y, c = blockIdx.x;
+  if (l > g.L) return;
+  const int kc = pg_kc(g, l);
+  if (c >= kc) return;
+  const int K = 32 * kc;
+  long long woff = 0;
+  for (int r = 0; r < l; ++r) woff += 4096LL * pg_kc(g, r);
+  const float* Wl = W + woff;
+  float* hi = ws + pg_wbase(g, l) + (size_t)c * kTcBlockFloats;
+#pragma unroll
+  for (int it = 0; it < 4; ++it) {
+    const int idx = it * 256 + threadIdx.x;   // 0 .. 1023
+    const int j = idx >> 3, q = idx & 7;      // output channel, group of 4 inputs
+    const float4 v = __ldg(reinterpret_cast<const float4*>(Wl + (size_t)j * K + 32 * c) + q);
+    uint4 h, w;
+    split4(v, h, w);
+    const int off = tc::core_offset(j, 4 * q, kTcC);
+    *reinterpret_cast<uint4*>(hi + off) = h;
+    *reinterpret_cast<uint4*>(hi + (size_t)kc * kTcBlockFloats + off) = w;
+  }
+}
+
+__global__ void __launch_bounds__(kTcThreads, 1) path_mix_tc_kernel(PathGeom geo,
+                                                                    const float* __restrict__ xs,
+                                                                    const float* __restrict__ ws,
+                                                                    float* __restrict__ out) {
+  extern __shared__ __align__(1024) unsigned char smem[];
+  float* st = reinterpret_cast<float*>(smem);
+  uint64_t* stage_full = reinterpret_cast<uint64_t*>(st + kTcStages * kPmStageFloats);
+  uint64_t* stage_free = stage_full + kTcStages;
+  uint64_t* acc_full = stage_free + kTcStages;
+  uint64_t* acc_free = acc_full + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_free + 2);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const long long total = pg_chunks_before(geo, geo.L + 1);
+  const int t_begin = pg_tile_at(geo, (long long)blockIdx.x * total / gridDim.x);
+  const int t_end = pg_tile_at(geo, (long long)(blockIdx.x + 1) * total / gridDim.x);
+
+  if (warp == 0) tc::tmem_alloc(tmem_slot, 2 * kTcRows);
+  if (tid == 0) {
+    for (int s = 0; s < kTcStages; ++s) {
+      tc::bar_init(&stage_full[s], 1);
+      tc::bar_init(&stage_free[s], 1);
+    }
+    tc::bar_init(&acc_full[0], 1);
+    tc::bar_init(&acc_full[1], 1);
+    tc::bar_init(&acc_free[0], 128);
+    tc::bar_init(&acc_free[1], 128);
+    tc::fence_bar_init();
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = *tmem_slot;
+  bool fail = false;
+
+  if (warp == 0) {
+    // ---------------- bulk-copy producer ----------------
+    if (lane == 0) {
+      int g = 0;
+      for (int t = t_begin; t < t_end && !fail; ++t) {
+        const int l = pg_rank(geo, t), kc = pg_kc(geo, l);
+        const float* xt = xs + pg_xbase(geo, l) + (long long)(t - pg_ts(geo, l)) * kc * 2 * kTcBlockFloats;
+        const float* wt = ws + pg_wbase(geo, l);
+        const size_t lo = (size_t)kc * kTcBlockFloats;
+        for (int c = 0; c < kc; ++c, ++g) {
+          const int s = g % kTcStages;
+          if (g >= kTcStages &&
+              !tc::bar_wait(&stage_free[s], ((g - kTcStages) / kTcStages) & 1, kTcWaitPolls)) {
+            fail = true;
+            break;
+          }
+          float* dst = st + s * kPmStageFloats;
+          const size_t co = (size_t)c * kTcBlockFloats;
+          constexpr uint32_t kB = kTcBlockFloats * sizeof(float);
+          tc::bar_arrive_expect_tx(&stage_full[s], kPmStageFloats * sizeof(float));
+          tc::bulk_load(dst, xt + co, kB, &stage_full[s]);
+          tc::bulk_load(dst + kTcBlockFloats, xt + lo + co, kB, &stage_full[s]);
+          tc::bulk_load(dst + 2 * kTcBlockFloats, wt + co, kB, &stage_full[s]);
+          tc::bulk_load(dst + 3 * kTcBlockFloats, wt + lo + co, kB, &stage_full[s]);
+        }
+      }
+      if (fail)   // let the copies already issued land
+        for (int k = 1; k <= kTcStages && g - k >= 0; ++k)
+          tc::bar_wait(&stage_full[(g - k) % kTcStages], ((g - k) / kTcStages) & 1, kTcWaitPolls);
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0) {
+      constexpr uint32_t idesc = tc::idesc_tf32(kTcC, kTcRows);
+      constexpr uint32_t kLbo = kTcRows * 16, kSbo = 128;
+      int g = 0, h = 0;   // chunks and accumulator groups issued
+      for (int t = t_begin; t < t_end && !fail; ++t) {
+        const int kc = pg_kc(geo, pg_rank(geo, t));
+        for (int c = 0; c < kc; ++c, ++g) {
+          const uint32_t d_tmem = tmem + (uint32_t)(h & 1) * kTcRows;
+          if (c % kPmGroup == 0) {   // the epilogue has added group h - 2
+            if (h >= 2 && !tc::bar_wait(&acc_free[h & 1], ((h - 2) >> 1) & 1, kTcWaitPolls)) {
+              fail = true;
+              break;
+            }
+            tc::fence_after_sync();
+          }
+          const int s = g % kTcStages;
+          if (!tc::bar_wait(&stage_full[s], (g / kTcStages) & 1, kTcWaitPolls)) {
+            fail = true;
+            break;
+          }
+          tc::fence_after_sync();
+          const uint32_t xh = tc::smem_addr(st + s * kPmStageFloats);
+          const uint32_t xl = xh + kTcBlockFloats * sizeof(float);
+          const uint32_t wh = xh + 2 * kTcBlockFloats * sizeof(float);
+          const uint32_t wl = xh + 3 * kTcBlockFloats * sizeof(float);
+#pragma unroll
+          for (int j = 0; j < kTcChunk / 8; ++j) {
+            const uint32_t kx = 2 * j * kLbo;
+            const uint64_t dwh = tc::smem_desc(wh + kx, kLbo, kSbo);
+            const uint64_t dwl = tc::smem_desc(wl + kx, kLbo, kSbo);
+            const uint64_t dxh = tc::smem_desc(xh + kx, kLbo, kSbo);
+            const uint64_t dxl = tc::smem_desc(xl + kx, kLbo, kSbo);
+            tc::mma_tf32(d_tmem, dwh, dxh, idesc, ((c % kPmGroup) | j) != 0);
+            tc::mma_tf32(d_tmem, dwh, dxl, idesc, 1u);
+            tc::mma_tf32(d_tmem, dwl, dxh, idesc, 1u);
+          }
+          tc::commit(&stage_free[s]);
+          if (c % kPmGroup == kPmGroup - 1 || c == kc - 1) tc::commit(&acc_full[(h++) & 1]);
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp >= 4) {
+    // ---------------- epilogue: sum the groups of a tile, write out and z ----------------
+    const int ew = warp - 4;
+    const int j = 32 * ew + lane;
+    int h = 0;
+    for (int t = t_begin; t < t_end && !fail; ++t) {
+      const int l = pg_rank(geo, t);
+      const int kc = pg_kc(geo, l);
+      const int tr = t - pg_ts(geo, l);
+      const int cmc = tr / geo.nb;                     // the tile's component
+      const int cmn = (tr - cmc * geo.nb) * kTcRows;   // and its first node
+      float acc[kTcRows];
+      for (int gi = 0; gi < (kc + kPmGroup - 1) / kPmGroup; ++gi, ++h) {
+        if (!tc::bar_wait(&acc_full[h & 1], (h >> 1) & 1, kTcWaitPolls)) {
+          fail = true;
+          break;
+        }
+        tc::fence_after_sync();
+        const uint32_t d_tmem = tmem + (uint32_t)(h & 1) * kTcRows + ((uint32_t)(32 * ew) << 16);
+#pragma unroll
+        for (int q = 0; q < kTcRows / 32; ++q) {
+          float v[32];
+          tc::tmem_ld32(d_tmem + 32 * q, v);
+#pragma unroll
+          for (int r = 0; r < 32; ++r) acc[32 * q + r] = gi ? acc[32 * q + r] + v[r] : v[r];
+        }
+        tc::fence_before_sync();
+        tc::bar_arrive(&acc_free[h & 1]);
+      }
+      if (fail) break;
+      float* o = out + ((size_t)cmn * geo.NY + l * l + cmc) * kTcC + j;
+      const size_t step = (size_t)geo.NY * kTcC;
+      const int nr = min(kTcRows, geo.N - cmn);
+#pragma unroll
+      for (int r = 0; r < kTcRows; ++r) {
+        if (r < nr) *o = acc[r];
+        o += step;
+      }
+    }
+  }
+  if (fail) atomicExch(&g_tc_error, 1);
+  tc::fence_before_sync();
+  __syncthreads();
+  if (warp == 0) {
+    tc::fence_after_sync();
+    tc::tmem_dealloc(tmem, 2 * kTcRows);
+  }
+}
+
 int g_tc_smem_set[64] = {0};
 int g_wg_smem_set[64] = {0};
+int g_pm_smem_set[64] = {0};
 
 }  // namespace
 
@@ -634,6 +887,61 @@ int launch_wgrad_tc(int L, int N, const float* as, const float* bs, float* Mbar,
   const int sms = device_sm_count();
   const int grid = T < sms ? T : sms;
   ladder_wgrad_tc_kernel<<<grid, kWgThreads, kWgSmemBytes, s>>>(g, as, bs, Mbar);
+  return cudaGetLastError() == cudaSuccess ? FC_OK : FC_ERR_CUDA;
+}
+
+PathGeom path_geom(int L, int N, const int* kc) {
+  PathGeom g{};
+  g.N = N;
+  g.NY = (L + 1) * (L + 1);
+  g.L = L;
+  g.nb = (N + kTcRows - 1) / kTcRows;
+  int ts[6] = {0, 0, 0, 0, 0, 0}, k[5] = {0, 0, 0, 0, 0};
+  int T = 0;
+  for (int l = 0; l <= 5; ++l) {
+    ts[l] = T;
+    if (l <= L && l < 5) {
+      T += (2 * l + 1) * g.nb;
+      k[l] = kc[l];
+    }
+  }
+  g.t1 = ts[1]; g.t2 = ts[2]; g.t3 = ts[3]; g.t4 = ts[4]; g.t5 = ts[5];
+  g.k0 = k[0]; g.k1 = k[1]; g.k2 = k[2]; g.k3 = k[3]; g.k4 = k[4];
+  return g;
+}
+
+int launch_path_split_rows(const PathGeom& g, const float* in, float* xs, cudaStream_t s) {
+  for (int l = 0; l <= g.L; ++l)
+    if (pg_kc(g, l) != 4) return FC_ERR_ARG;
+  const int T = pg_ts(g, g.L + 1);
+  if (T == 0) return FC_OK;
+  path_split_rows_kernel<<<dim3(T, kTcChunks), 256, 0, s>>>(g, in, xs);
+  return cudaGetLastError() == cudaSuccess ? FC_OK : FC_ERR_CUDA;
+}
+
+int launch_path_split_map(const PathGeom& g, const float* W, float* ws, cudaStream_t s) {
+  int kmax = 0;
+  for (int l = 0; l <= g.L; ++l) kmax = pg_kc(g, l) > kmax ? pg_kc(g, l) : kmax;
+  if (kmax == 0) return FC_OK;
+  path_split_map_kernel<<<dim3(kmax, g.L + 1), 256, 0, s>>>(g, W, ws);
+  return cudaGetLastError() == cudaSuccess ? FC_OK : FC_ERR_CUDA;
+}
+
+int launch_path_mix_tc(const PathGeom& g, const float* xs, const float* ws, float* out, cudaStream_t s) {
+  if (g.L < 0 || g.L > 4) return FC_ERR_UNSUPPORTED_RANK;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return FC_ERR_CUDA;
+  if (!g_pm_smem_set[dev]) {
+    if (cudaFuncSetAttribute(path_mix_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)kPmSmemBytes) != cudaSuccess)
+      return FC_ERR_CUDA;
+    g_pm_smem_set[dev] = 1;
+  }
+  const int T = pg_ts(g, g.L + 1);
+  if (T == 0) return FC_OK;
+  const int sms = device_sm_count();
+  const int grid = T < sms ? T : sms;
+  path_mix_tc_kernel<<<grid, kTcThreads, kPmSmemBytes, s>>>(g, xs, ws, out);
   return cudaGetLastError() == cudaSuccess ? FC_OK : FC_ERR_CUDA;
 }
 

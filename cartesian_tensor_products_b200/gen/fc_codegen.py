@@ -1062,6 +1062,18 @@ def emit_ladder(L):
                               for b1, b2, k in terms) or "0.0f"
             o.append("    o[(size_t)%d * C] = %s;" % (T.zslot(p, c), expr))
     o.append("  }")
+    # the same products handed to a writer: put(l3, c, eta_l3, value)
+    o.append("  template <class Put>")
+    o.append("  static __device__ __forceinline__ void fwd_paths_to(const float (&a)[NY], const float (&b)[NY], Put&& put) {")
+    for p, (l1, l2, l3) in enumerate(T.paths):
+        K = T.K[p]
+        for c in range(2 * l3 + 1):
+            terms = [(b1, b2, K[c][b1][b2]) for b1 in range(2 * l1 + 1)
+                     for b2 in range(2 * l2 + 1) if K[c][b1][b2] != 0]
+            expr = " + ".join("%s*(a[%d]*b[%d])" % (flit(k), l1 * l1 + b1, l2 * l2 + b2)
+                              for b1, b2, k in terms) or "0.0f"
+            o.append("    put(%d, %d, %d, %s);" % (l3, c, T.eta[p], expr))
+    o.append("  }")
     # VJP: g is the gradient of B
     o.append("  static __device__ __forceinline__ void vjp(const float (&a)[NY], const float (&b)[NY], const float (&w)[P], const float (&g)[NY],")
     o.append("                                             float (&abar)[NY], float (&bbar)[NY], float (&wbar)[P]) {")

@@ -303,9 +303,15 @@ int fc_product_ladder_noalloc(const fc_ladder_desc *desc, int n_nodes,
  *   Wq [order-1][C P C]: per step the rank blocks [C][P_l C] one after the
  *   other (rank l at C C sum_{l'<l} P_l'); states [order][n_nodes][(lmax+1)^2 C]
  *   receives phi_1 .. phi_order; z [n_nodes][(lmax+1)^2 C].
- * workspace: fc_full_ladder_workspace_size() bytes (one path-separated
- * product, n_nodes x fc_conv_out_row x C floats), 16-byte aligned; none for
- * order 1.  Returns the statuses of fc_product_ladder. */
+ * C = 128 runs the maps on the tensor cores (three-term TF32 split, FP32
+ * accuracy); the workspace then holds one path-separated product and the
+ * maps of one step as hi / lo TF32 tiles (about 2 n_nodes x
+ * fc_conv_out_row x C + 8 C P C floats), order 1 included.  Other widths use
+ * FP32 SIMT maps: one path-separated product (n_nodes x fc_conv_out_row x C
+ * floats), none for order 1.
+ * workspace: fc_full_ladder_workspace_size() bytes, 16-byte aligned (0 means
+ * none is needed).  Returns the statuses of fc_product_ladder; a wait of the
+ * tensor-core kernel that gives up sets the fc_device_error word. */
 size_t fc_full_ladder_workspace_size(const fc_ladder_desc *desc, int n_nodes);
 int fc_full_ladder(const fc_ladder_desc *desc, int n_nodes, const float *A,
                    const float *W1, const float *Wq, float *states, float *z,

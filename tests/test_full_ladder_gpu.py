@@ -24,8 +24,12 @@ def dev(a):
     return torch.from_numpy(np.ascontiguousarray(a)).cuda()
 
 
+# C = 128 runs the tensor-core maps: node counts whose rank blocks span
+# several 128-row tiles and end in a ragged tile, order 1 (phi_1 alone)
 @pytest.mark.parametrize("L,C,order,N", [(1, 8, 4, 33), (2, 8, 3, 20), (3, 12, 4, 13),
-                                         (3, 128, 3, 9), (4, 4, 3, 7), (3, 40, 1, 11)])
+                                         (3, 128, 3, 9), (4, 4, 3, 7), (3, 40, 1, 11),
+                                         (1, 128, 4, 70), (2, 128, 3, 100), (3, 128, 2, 150),
+                                         (4, 128, 3, 40), (3, 128, 1, 50)])
 def test_full_ladder_small(fc, L, C, order, N):
     d = W.full_ladder_inputs(N, L, C, order, 300 + 10 * L + C)
     st, z = fc.full_ladder(L, order, dev(d["A"]), dev(d["W1"]), dev(d["Wq"]))
