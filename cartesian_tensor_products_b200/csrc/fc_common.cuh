@@ -90,10 +90,10 @@ int launch_wgrad_tc(int L, int N, const float* as, const float* bs, float* Mbar,
 // P_l paths x 128 channels).  They form 128-row tiles t_l .. t_{l+1} - 1,
 // component-major: tile t_l + c nb + n / 128 holds component c of nodes
 // 128 (n / 128) + 0..127 (nb = ceil(N / 128); rows past node N - 1 unused).
-// A tile is k_l hi blocks then k_l lo blocks of 4096 floats (128 rows x 32
-// inputs, core-matrix layout), and rank l's tiles start at float
-// pg_xbase(l) of the operand buffer.  The map of rank l ([128][K]) is split
-// the same way: k_l hi then k_l lo blocks from float pg_wbase(l).
+// A tile is k_l FP32 blocks of 4096 floats (128 rows x 32 inputs,
+// core-matrix layout), and rank l's tiles start at float pg_xbase(l) of the
+// operand buffer.  The map of rank l ([128][K]) is split into TF32: k_l hi
+// then k_l lo blocks of the same layout from float pg_wbase(l).
 struct PathGeom {
   int N, NY, L, nb;
   int t1, t2, t3, t4, t5;   // first tile of ranks 1..5 (t_{L+1} = all tiles)
@@ -113,7 +113,7 @@ __host__ __device__ __forceinline__ long long pg_xbase(const PathGeom& g, int l)
   long long b = 0;
 #pragma unroll
   for (int r = 0; r < 5; ++r)
-    if (r < l) b += (long long)(pg_ts(g, r + 1) - pg_ts(g, r)) * pg_kc(g, r) * 8192;
+    if (r < l) b += (long long)(pg_ts(g, r + 1) - pg_ts(g, r)) * pg_kc(g, r) * 4096;
   return b;
 }
 __host__ __device__ __forceinline__ long long pg_wbase(const PathGeom& g, int l) {
@@ -125,7 +125,7 @@ __host__ __device__ __forceinline__ long long pg_wbase(const PathGeom& g, int l)
 }
 // kc[l] = K chunks per row of rank l (l <= L <= 4)
 PathGeom path_geom(int L, int N, const int* kc);
-// natural [N][(L+1)^2][128] -> operand tiles with k_l = 4 (the map of phi_1)
+// natural [N][(L+1)^2][128] -> FP32 operand tiles with k_l = 4 (the map of phi_1)
 int launch_path_split_rows(const PathGeom& g, const float* in, float* xs, cudaStream_t s);
 // the maps, rank l's ([128][32 k_l] row-major) at W + 4096 sum_{l'<l} k_l',
 // -> split blocks at ws + pg_wbase(l)

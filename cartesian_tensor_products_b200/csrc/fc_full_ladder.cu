@@ -16,8 +16,8 @@
 //
 // At C = 128 the maps run on the tcgen05 tensor cores (fc_mix_tc.cu,
 // three-term TF32 split): the product kernel writes B_q straight into the
-// split tile layout the MMAs read (input k of a rank-l row = eta_l C +
-// channel), phi_1 reads A split into the same tiles; z is summed
+// FP32 tile layout the map kernel stages (input k of a rank-l row = eta_l C +
+// channel), phi_1 reads A copied into the same tiles; z is summed
 // from the states at the end.  Rows past the last node of a tile are never
 // written: the MMA column of such a row depends on that row alone and is not
 // stored.
@@ -56,8 +56,8 @@ __global__ void __launch_bounds__(128) full_tp_paths_kernel(int N, int C, const 
   }
 }
 
-// The same products at C = 128, written as the TF32 hi / lo split of the
-// path-mix operand (component-major PathGeom tiles, k_l = 4 P_l).
+// The same products at C = 128, written as the FP32 path-mix operand
+// (component-major PathGeom tiles, k_l = 4 P_l).
 // A warp takes 8 consecutive nodes x 4 consecutive channels: for one output
 // (path, component) its 32 values are exactly one 128-byte core matrix
 // (8 rows x 4 inputs), so every store instruction writes one full line.
@@ -83,11 +83,7 @@ __global__ void __launch_bounds__(256, 2) full_tp_tiled_kernel(PathGeom g, const
   const int cofs = tc::core_offset(r, kk, 128);
   TP::fwd_paths_to(a, b, [&](int l3, int c, int eta, float v) {
     const int kc = pg_kc(g, l3);
-    float* hi = xs + pg_xbase(g, l3) + (long long)(c * g.nb + nblk) * kc * 8192 + (eta * 4 + kq) * 4096 + cofs;
-    uint32_t h, lo;
-    tc::split_tf32(v, h, lo);
-    hi[0] = __uint_as_float(h);
-    hi[(size_t)kc * 4096] = __uint_as_float(lo);
+    xs[pg_xbase(g, l3) + (long long)(c * g.nb + nblk) * kc * 4096 + (eta * 4 + kq) * 4096 + cofs] = v;
   });
 }
 

@@ -556,9 +556,12 @@ __global__ void __launch_bounds__(kWgThreads, 1) ladder_wgrad_tc_kernel(Geom geo
 // ---------------------------------------------------------------------------
 // A row of rank l has K = 32 k_l inputs (P_l paths x 128 channels), more than
 // one stage holds, so each stage carries a K chunk of both operands: the
-// tile's 128 rows x 32 inputs and the map's 128 outputs x 32 inputs (hi and
-// lo of each, 64 KB), three stages deep.  The map chunks are re-read from L2
-// by every tile of the rank (a map is at most 1.3 MB split).  CTAs take
+// tile's 128 rows x 32 inputs in FP32 and the map's 128 outputs x 32 inputs
+// as TF32 hi and lo (48 KB), three stages deep.  The row operand crosses HBM
+// once in FP32 (half the bytes of a pre-split operand): two converter warps
+// split each chunk into hi / lo blocks in shared memory (two buffers) for the
+// MMAs, with a proxy fence before they publish it.  The map chunks are
+// re-read from L2 by every tile of the rank (a map is at most 1.3 MB split).  CTAs take
 // contiguous tile ranges of equal K-chunk count (tiles of different ranks
 // differ in length).  Roles as in the mix above, with one change for
 // accuracy: the tensor core's FP32 accumulation loses a little at every
@@ -570,8 +573,11 @@ __global__ void __launch_bounds__(kWgThreads, 1) ladder_wgrad_tc_kernel(Geom geo
 // sum here serialised on load latency and starved the tensor pipe).
 constexpr int kPmGroup = 4;   // chunks per accumulator: one path of 128 inputs
 
-constexpr int kPmStageFloats = 4 * kTcBlockFloats;   // x hi, x lo, W hi, W lo
-constexpr size_t kPmSmemBytes = sizeof(float) * kTcStages * kPmStageFloats + 8 * 16 + 8;
+constexpr int kPmStageFloats = 3 * kTcBlockFloats;   // x (FP32), W hi, W lo
+constexpr int kPmCvtFloats = 2 * kTcBlockFloats;     // x hi, x lo
+constexpr int kPmCvtThreads = 64;                    // warps 2 and 3
+constexpr size_t kPmSmemBytes =
+    sizeof(float) * (kTcStages * kPmStageFloats + 2 * kPmCvtFloats) + 8 * 16 + 8;
 static_assert(kPmSmemBytes <= 232448, "shared memory per CTA");
 
 __device__ __forceinline__ long long pg_chunks_before(const PathGeom& g, int l) {
@@ -594,8 +600,8 @@ __device__ __forceinline__ int pg_tile_at(const PathGeom& g, long long P) {
   return pg_ts(g, g.L + 1);
 }
 
-// natural [N][NY][128] -> component-major operand tiles with k_l = 4 (one
-// CTA per tile chunk; thread mapping as in ladder_split_rows_kernel).
+// natural [N][NY][128] -> component-major FP32 operand tiles with k_l = 4
+// (one CTA per tile chunk; thread mapping as in ladder_split_rows_kernel).
 __global__ void __launch_bounds__(256) path_split_rows_kernel(PathGeom g, const float* __restrict__ in,
                                                               float* __restrict__ xs) {
   const int t = blockIdx.x, c = blockIdx.y;
@@ -603,7 +609,7 @@ __global__ void __launch_bounds__(256) path_split_rows_kernel(PathGeom g, const 
   const int l = pg_rank(g, t);
   const int tr = t - pg_ts(g, l);
   const int comp = tr / g.nb, n0 = (tr - comp * g.nb) * kTcRows;
-  float* hi = xs + pg_xbase(g, l) + (size_t)tr * 4 * 2 * kTcBlockFloats + c * kTcBlockFloats;
+  float* dst = xs + pg_xbase(g, l) + (size_t)tr * 4 * kTcBlockFloats + c * kTcBlockFloats;
 #pragma unroll
   for (int it = 0; it < 4; ++it) {
     const int r = 16 * (p >> 5) + 8 * (it >> 1) + (lane & 7);
@@ -612,11 +618,7 @@ __global__ void __launch_bounds__(256) path_split_rows_kernel(PathGeom g, const 
     float4 v = zero4();
     if (n < g.N)
       v = __ldg(reinterpret_cast<const float4*>(in + ((size_t)n * g.NY + l * l + comp) * kTcC + c * kTcChunk) + q);
-    uint4 h, w;
-    split4(v, h, w);
-    const int off = tc::core_offset(r, 4 * q, kTcRows);
-    *reinterpret_cast<uint4*>(hi + off) = h;
-    *reinterpret_cast<uint4*>(hi + 4 * kTcBlockFloats + off) = w;
+    *reinterpret_cast<float4*>(dst + tc::core_offset(r, 4 * q, kTcRows)) = v;
   }
 }
 
@@ -650,9 +652,12 @@ __global__ void __launch_bounds__(kTcThreads, 1) path_mix_tc_kernel(PathGeom geo
                                                                     float* __restrict__ out) {
   extern __shared__ __align__(1024) unsigned char smem[];
   float* st = reinterpret_cast<float*>(smem);
-  uint64_t* stage_full = reinterpret_cast<uint64_t*>(st + kTcStages * kPmStageFloats);
+  float* cv = st + kTcStages * kPmStageFloats;   // converted x: 2 buffers of (hi, lo)
+  uint64_t* stage_full = reinterpret_cast<uint64_t*>(cv + 2 * kPmCvtFloats);
   uint64_t* stage_free = stage_full + kTcStages;
-  uint64_t* acc_full = stage_free + kTcStages;
+  uint64_t* cvt_full = stage_free + kTcStages;
+  uint64_t* cvt_free = cvt_full + 2;
+  uint64_t* acc_full = cvt_free + 2;
   uint64_t* acc_free = acc_full + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_free + 2);
 
@@ -665,12 +670,14 @@ __global__ void __launch_bounds__(kTcThreads, 1) path_mix_tc_kernel(PathGeom geo
   if (tid == 0) {
     for (int s = 0; s < kTcStages; ++s) {
       tc::bar_init(&stage_full[s], 1);
-      tc::bar_init(&stage_free[s], 1);
+      tc::bar_init(&stage_free[s], kPmCvtThreads + 1);   // converter threads + the MMA commit
     }
-    tc::bar_init(&acc_full[0], 1);
-    tc::bar_init(&acc_full[1], 1);
-    tc::bar_init(&acc_free[0], 128);
-    tc::bar_init(&acc_free[1], 128);
+    for (int b = 0; b < 2; ++b) {
+      tc::bar_init(&cvt_full[b], kPmCvtThreads);
+      tc::bar_init(&cvt_free[b], 1);
+      tc::bar_init(&acc_full[b], 1);
+      tc::bar_init(&acc_free[b], 128);
+    }
     tc::fence_bar_init();
   }
   tc::fence_before_sync();
@@ -685,7 +692,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) path_mix_tc_kernel(PathGeom geo
       int g = 0;
       for (int t = t_begin; t < t_end && !fail; ++t) {
         const int l = pg_rank(geo, t), kc = pg_kc(geo, l);
-        const float* xt = xs + pg_xbase(geo, l) + (long long)(t - pg_ts(geo, l)) * kc * 2 * kTcBlockFloats;
+        const float* xt = xs + pg_xbase(geo, l) + (long long)(t - pg_ts(geo, l)) * kc * kTcBlockFloats;
         const float* wt = ws + pg_wbase(geo, l);
         const size_t lo = (size_t)kc * kTcBlockFloats;
         for (int c = 0; c < kc; ++c, ++g) {
@@ -700,9 +707,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) path_mix_tc_kernel(PathGeom geo
           constexpr uint32_t kB = kTcBlockFloats * sizeof(float);
           tc::bar_arrive_expect_tx(&stage_full[s], kPmStageFloats * sizeof(float));
           tc::bulk_load(dst, xt + co, kB, &stage_full[s]);
-          tc::bulk_load(dst + kTcBlockFloats, xt + lo + co, kB, &stage_full[s]);
-          tc::bulk_load(dst + 2 * kTcBlockFloats, wt + co, kB, &stage_full[s]);
-          tc::bulk_load(dst + 3 * kTcBlockFloats, wt + lo + co, kB, &stage_full[s]);
+          tc::bulk_load(dst + kTcBlockFloats, wt + co, kB, &stage_full[s]);
+          tc::bulk_load(dst + 2 * kTcBlockFloats, wt + lo + co, kB, &stage_full[s]);
         }
       }
       if (fail)   // let the copies already issued land
@@ -727,16 +733,17 @@ __global__ void __launch_bounds__(kTcThreads, 1) path_mix_tc_kernel(PathGeom geo
             }
             tc::fence_after_sync();
           }
-          const int s = g % kTcStages;
-          if (!tc::bar_wait(&stage_full[s], (g / kTcStages) & 1, kTcWaitPolls)) {
+          const int s = g % kTcStages, b = g & 1;
+          if (!tc::bar_wait(&stage_full[s], (g / kTcStages) & 1, kTcWaitPolls) ||
+              !tc::bar_wait(&cvt_full[b], (g >> 1) & 1, kTcWaitPolls)) {
             fail = true;
             break;
           }
           tc::fence_after_sync();
-          const uint32_t xh = tc::smem_addr(st + s * kPmStageFloats);
+          const uint32_t wh = tc::smem_addr(st + s * kPmStageFloats) + kTcBlockFloats * sizeof(float);
+          const uint32_t wl = wh + kTcBlockFloats * sizeof(float);
+          const uint32_t xh = tc::smem_addr(cv + b * kPmCvtFloats);
           const uint32_t xl = xh + kTcBlockFloats * sizeof(float);
-          const uint32_t wh = xh + 2 * kTcBlockFloats * sizeof(float);
-          const uint32_t wl = xh + 3 * kTcBlockFloats * sizeof(float);
 #pragma unroll
           for (int j = 0; j < kTcChunk / 8; ++j) {
             const uint32_t kx = 2 * j * kLbo;
@@ -749,13 +756,43 @@ __global__ void __launch_bounds__(kTcThreads, 1) path_mix_tc_kernel(PathGeom geo
             tc::mma_tf32(d_tmem, dwl, dxh, idesc, 1u);
           }
           tc::commit(&stage_free[s]);
+          tc::commit(&cvt_free[b]);
           if (c % kPmGroup == kPmGroup - 1 || c == kc - 1) tc::commit(&acc_full[(h++) & 1]);
         }
       }
     }
     __syncwarp();
-  } else if (warp >= 4) {
-    // ---------------- epilogue: sum the groups of a tile, write out and z ----------------
+  } else if (warp < 4) {
+    // ---------------- converter: FP32 chunk -> TF32 hi / lo blocks ----------------
+    const int ct = tid - 64;   // 0 .. 63
+    int g = 0;
+    for (int t = t_begin; t < t_end && !fail; ++t) {
+      const int kc = pg_kc(geo, pg_rank(geo, t));
+      for (int c = 0; c < kc; ++c, ++g) {
+        const int s = g % kTcStages, b = g & 1;
+        if (!tc::bar_wait(&stage_full[s], (g / kTcStages) & 1, kTcWaitPolls) ||
+            (g >= 2 && !tc::bar_wait(&cvt_free[b], ((g - 2) >> 1) & 1, kTcWaitPolls))) {
+          fail = true;
+          break;
+        }
+        const float4* src = reinterpret_cast<const float4*>(st + s * kPmStageFloats);
+        uint4* hi = reinterpret_cast<uint4*>(cv + b * kPmCvtFloats);
+        uint4* lo = hi + kTcBlockFloats / 4;
+#pragma unroll 4
+        for (int i = 0; i < kTcBlockFloats / 4 / kPmCvtThreads; ++i) {
+          const int q = i * kPmCvtThreads + ct;
+          uint4 h, w;
+          split4(src[q], h, w);
+          hi[q] = h;
+          lo[q] = w;
+        }
+        tc::fence_proxy_async();   // the generic-proxy writes, visible to the MMAs
+        tc::bar_arrive(&cvt_full[b]);
+        tc::bar_arrive(&stage_free[s]);
+      }
+    }
+  } else {
+    // ---------------- epilogue: sum the groups of a tile, write out ----------------
     const int ew = warp - 4;
     const int j = 32 * ew + lane;
     int h = 0;
