@@ -775,16 +775,24 @@ __global__ void __launch_bounds__(kTcThreads, 1) path_mix_tc_kernel(PathGeom geo
           fail = true;
           break;
         }
-        const float4* src = reinterpret_cast<const float4*>(st + s * kPmStageFloats);
-        uint4* hi = reinterpret_cast<uint4*>(cv + b * kPmCvtFloats);
-        uint4* lo = hi + kTcBlockFloats / 4;
-#pragma unroll 4
-        for (int i = 0; i < kTcBlockFloats / 4 / kPmCvtThreads; ++i) {
-          const int q = i * kPmCvtThreads + ct;
+        const uint32_t src = tc::smem_addr(st + s * kPmStageFloats) + 16 * ct;
+        const uint32_t hi = tc::smem_addr(cv + b * kPmCvtFloats) + 16 * ct;
+        constexpr uint32_t kLo = kTcBlockFloats * sizeof(float), kStep = 16 * kPmCvtThreads;
+        constexpr int kIters = kTcBlockFloats / 4 / kPmCvtThreads;   // 16
+        float4 v[kIters];
+#pragma unroll
+        for (int i = 0; i < kIters; ++i)
+          asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+                       : "=f"(v[i].x), "=f"(v[i].y), "=f"(v[i].z), "=f"(v[i].w)
+                       : "r"(src + i * kStep));
+#pragma unroll
+        for (int i = 0; i < kIters; ++i) {
           uint4 h, w;
-          split4(src[q], h, w);
-          hi[q] = h;
-          lo[q] = w;
+          split4(v[i], h, w);
+          asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(hi + i * kStep), "r"(h.x),
+                       "r"(h.y), "r"(h.z), "r"(h.w) : "memory");
+          asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(hi + kLo + i * kStep), "r"(w.x),
+                       "r"(w.y), "r"(w.z), "r"(w.w) : "memory");
         }
         tc::fence_proxy_async();   // the generic-proxy writes, visible to the MMAs
         tc::bar_arrive(&cvt_full[b]);
