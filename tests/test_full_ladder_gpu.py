@@ -55,3 +55,34 @@ def test_full_ladder_4096_sampled_nodes(fc):
     for q in range(order):
         assert rel_err(st[q].cpu().numpy()[nodes], rs[q][nodes]) <= FWD_TOL
     assert np.isfinite(z.cpu().numpy()).all()
+
+
+@pytest.mark.parametrize("L,C,order,N", [(3, 128, 3, 40), (3, 128, 1, 40), (2, 8, 3, 20)])
+def test_workspace_refusal_and_error_word(fc, L, C, order, N):
+    """One float short of the queried workspace is refused on the host
+    (FC_ERR_WORKSPACE = 7), on the tensor-core path (C = 128, which needs
+    scratch at order 1 too) and on the SIMT path; a run with the exact size
+    matches the oracle and leaves the bounded-wait error word clear."""
+    import ctypes as ct
+    d = W.full_ladder_inputs(N, L, C, order, 90 + C + order)
+    A, W1, Wq = dev(d["A"]), dev(d["W1"]), dev(d["Wq"])
+    need = fc.lib().fc_full_ladder_workspace_size(ct.byref(fc.LadderDesc(L, C, order)), N)
+    assert need > 0 and need % 4 == 0
+    with pytest.raises(fc.FlashCartError) as e:
+        fc.full_ladder(L, order, A, W1, Wq, workspace=torch.empty(need // 4 - 1, device="cuda"))
+    assert e.value.status == 7
+    st, z = fc.full_ladder(L, order, A, W1, Wq, workspace=torch.empty(need // 4, device="cuda"))
+    torch.cuda.synchronize()
+    assert fc.device_error() == 0
+    _, rz = O.full_ladder(L, C, order, d["A"], d["W1"], d["Wq"])
+    assert rel_err(z.cpu().numpy(), rz) <= FWD_TOL
+
+
+def test_no_nodes(fc):
+    """Zero nodes: FC_OK, nothing launched, empty outputs."""
+    d = W.full_ladder_inputs(3, 3, 128, 3, 5)
+    A = dev(d["A"])[:0]
+    st, z = fc.full_ladder(3, 3, A, dev(d["W1"]), dev(d["Wq"]))
+    torch.cuda.synchronize()
+    assert st.shape == (3, 0, 16 * 128) and z.shape == (0, 16 * 128)
+    assert fc.device_error() == 0
