@@ -304,9 +304,10 @@ int fc_product_ladder_noalloc(const fc_ladder_desc *desc, int n_nodes,
  *   other (rank l at C C sum_{l'<l} P_l'); states [order][n_nodes][(lmax+1)^2 C]
  *   receives phi_1 .. phi_order; z [n_nodes][(lmax+1)^2 C].
  * C = 128 runs the maps on the tensor cores (three-term TF32 split, FP32
- * accuracy); the workspace then holds one path-separated product and the
- * maps of one step as hi / lo TF32 tiles (about 2 n_nodes x
- * fc_conv_out_row x C + 8 C P C floats), order 1 included.  Other widths use
+ * accuracy); the workspace then holds one path-separated product as FP32
+ * tiles (about n_nodes x fc_conv_out_row x C floats, node count rounded up
+ * to 128) and the maps of one step as hi / lo TF32 tiles (2 C P C floats),
+ * order 1 included.  Other widths use
  * FP32 SIMT maps: one path-separated product (n_nodes x fc_conv_out_row x C
  * floats), none for order 1.
  * workspace: fc_full_ladder_workspace_size() bytes, 16-byte aligned (0 means
