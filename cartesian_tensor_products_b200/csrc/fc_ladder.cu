@@ -64,45 +64,39 @@ __global__ void __launch_bounds__(128) ladder_tp_kernel(int N, int C, const floa
   }
 }
 
-// The same product written straight into the tiled split layout of the
-// tensor-core mix (C = 128): component i of node n is row n (2l+1) + i - l^2
-// of rank l, tile ts[l] + row / 128, in the tile's TF32 hi and lo blocks.
+// The same product written straight into the FP32 component-major tiles of
+// the tensor-core map (PathGeom with k_l = 4, C = 128): component c of rank
+// l of node n is row n mod 128 of tile c nb + n / 128 of that rank.  A warp
+// takes 8 consecutive nodes x 4 consecutive channels, so each store of one
+// component is one full 128-byte core matrix.
 template <int L>
-__global__ void __launch_bounds__(128) ladder_tp_tiled_kernel(int N, const float* __restrict__ Av,
+__global__ void __launch_bounds__(256, 2) ladder_tp_cm_kernel(PathGeom g, const float* __restrict__ Av,
                                                               const float* __restrict__ A1,
                                                               const float* __restrict__ W,
-                                                              MixTiles tiles,
                                                               float* __restrict__ xs) {
   using TP = LadderTP<L>;
   constexpr int C = 128;
-  const int k = threadIdx.x;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int n = 8 * blockIdx.x + (lane >> 2);
+  const int k = 32 * blockIdx.y + 4 * warp + (lane & 3);
+  if (n >= g.N) return;
   float w[TP::P];
 #pragma unroll
   for (int p = 0; p < TP::P; ++p) w[p] = __ldg(W + (size_t)p * C + k);
-  const int n0 = blockIdx.x * kLadderFwdChunk;
-  const int n1 = min(N, n0 + kLadderFwdChunk);
-  for (int n = n0; n < n1; ++n) {
-    const size_t base = (size_t)n * TP::NY * C + k;
-    float a[TP::NY], b[TP::NY], o[TP::NY];
+  const size_t base = (size_t)n * TP::NY * C + k;
+  float a[TP::NY], b[TP::NY], o[TP::NY];
 #pragma unroll
-    for (int i = 0; i < TP::NY; ++i) {
-      a[i] = __ldg(Av + base + (size_t)i * C);
-      b[i] = __ldg(A1 + base + (size_t)i * C);
-    }
-    TP::fwd(a, b, w, o);
+  for (int i = 0; i < TP::NY; ++i) {
+    a[i] = __ldg(Av + base + (size_t)i * C);
+    b[i] = __ldg(A1 + base + (size_t)i * C);
+  }
+  TP::fwd(a, b, w, o);
+  const int cofs = (k >> 5) * 4096 + tc::core_offset(n & 127, k & 31, 128);
 #pragma unroll
-    for (int l = 0; l <= L; ++l) {
+  for (int l = 0; l <= L; ++l) {
 #pragma unroll
-      for (int c = 0; c < 2 * l + 1; ++c) {
-        const int row = n * (2 * l + 1) + c;
-        const int t = tiles.ts[l] + (row >> 7);
-        float* hi = xs + (size_t)t * 32768 + tc::core_offset(row & 127, k, 128);
-        uint32_t h, lo;
-        tc::split_tf32(o[l * l + c], h, lo);
-        hi[0] = __uint_as_float(h);
-        hi[16384] = __uint_as_float(lo);
-      }
-    }
+    for (int c = 0; c < 2 * l + 1; ++c)
+      xs[pg_xbase(g, l) + (long long)(c * g.nb + (n >> 7)) * 4 * 4096 + cofs] = o[l * l + c];
   }
 }
 
@@ -398,14 +392,14 @@ static int tp_dispatch(int L, int N, int C, const float* Av, const float* A1, co
   return FC_ERR_UNSUPPORTED_RANK;
 }
 
-static int tp_tiled_dispatch(int L, int N, const float* Av, const float* A1, const float* W,
-                             const MixTiles& tiles, float* xs, cudaStream_t s) {
-  const dim3 grid((N + kLadderFwdChunk - 1) / kLadderFwdChunk);
+static int tp_cm_dispatch(int L, const PathGeom& g, const float* Av, const float* A1, const float* W,
+                          float* xs, cudaStream_t s) {
+  const dim3 grid((g.N + 7) / 8, 4);
   switch (L) {
-    case 1: ladder_tp_tiled_kernel<1><<<grid, 128, 0, s>>>(N, Av, A1, W, tiles, xs); break;
-    case 2: ladder_tp_tiled_kernel<2><<<grid, 128, 0, s>>>(N, Av, A1, W, tiles, xs); break;
-    case 3: ladder_tp_tiled_kernel<3><<<grid, 128, 0, s>>>(N, Av, A1, W, tiles, xs); break;
-    case 4: ladder_tp_tiled_kernel<4><<<grid, 128, 0, s>>>(N, Av, A1, W, tiles, xs); break;
+    case 1: ladder_tp_cm_kernel<1><<<grid, 256, 0, s>>>(g, Av, A1, W, xs); break;
+    case 2: ladder_tp_cm_kernel<2><<<grid, 256, 0, s>>>(g, Av, A1, W, xs); break;
+    case 3: ladder_tp_cm_kernel<3><<<grid, 256, 0, s>>>(g, Av, A1, W, xs); break;
+    case 4: ladder_tp_cm_kernel<4><<<grid, 256, 0, s>>>(g, Av, A1, W, xs); break;
     default: return FC_ERR_UNSUPPORTED_RANK;
   }
   return cudaGetLastError() == cudaSuccess ? FC_OK : FC_ERR_CUDA;
@@ -453,16 +447,25 @@ int fc_ladder_num_paths(const fc_ladder_desc* d) {
   return num_paths(d->lmax);
 }
 
-// Tensor-core path scratch: the product in the tiled split layout plus one
+// Tensor-core VJP scratch: a gradient in the tiled split layout plus one
 // step's split mixing matrices.
 static size_t tc_scratch_floats(int L, int N) {
   return mix_tc_operand_floats(L, N) + mix_tc_matrix_floats(L);
 }
 
+// Tensor-core forward: the product as FP32 component-major tiles (k_l = 4)
+static PathGeom fwd_geom(int L, int N) {
+  const int kc[5] = {4, 4, 4, 4, 4};
+  return path_geom(L, N, kc);
+}
+
 size_t fc_product_ladder_workspace_size(const fc_ladder_desc* d, int n_nodes) {
   if (check_ladder_desc(d) != FC_OK || n_nodes < 0) return 0;
   const int NY = (d->lmax + 1) * (d->lmax + 1);
-  if (mix_tc_supported(d->lmax, d->channels)) return sizeof(float) * tc_scratch_floats(d->lmax, n_nodes);
+  if (mix_tc_supported(d->lmax, d->channels)) {
+    const PathGeom g = fwd_geom(d->lmax, n_nodes);
+    return sizeof(float) * (size_t)(pg_xbase(g, g.L + 1) + pg_wbase(g, g.L + 1));
+  }
   return sizeof(float) * (size_t)n_nodes * NY * d->channels;
 }
 
@@ -486,22 +489,19 @@ int fc_product_ladder(const fc_ladder_desc* d, int n_nodes, const float* A1, con
   const size_t plane = (size_t)n_nodes * NY * C;
   const int P = num_paths(L);
   if (S > 0 && mix_tc_supported(L, C)) {
-    // tensor cores: the product is written pre-split into the mix's tiled
-    // layout; the mix writes the states; z = A_1 + sum of the states at the end
-    const MixTiles tiles = mix_tc_tiles(L, n_nodes);
+    // tensor cores: the product is written as FP32 component-major tiles,
+    // the map kernel (K = 128 per rank, split to TF32 hi / lo in shared
+    // memory) writes the states; z = A_1 + sum of the states at the end.
+    // Rows past the last node of a tile are never written: the MMA column of
+    // such a row depends on that row alone and is not stored.
+    const PathGeom g = fwd_geom(L, n_nodes);
     float* xs = static_cast<float*>(workspace);
-    float* wsm = xs + mix_tc_operand_floats(L, n_nodes);
-    for (int l = 0; l <= L; ++l)   // rows past each rank's end stay zero
-      if (cudaMemsetAsync(xs + (size_t)(tiles.ts[l + 1] - 1) * 32768, 0, 32768 * sizeof(float), s) !=
-          cudaSuccess)
-        return FC_ERR_CUDA;
+    float* wsm = xs + pg_xbase(g, L + 1);
     for (int v = 1; v <= S; ++v) {
       const float* Av = v == 1 ? A1 : states + (size_t)(v - 2) * plane;
-      if ((st = tp_tiled_dispatch(L, n_nodes, Av, A1, path_w + (size_t)(v - 1) * P * C, tiles, xs, s)) !=
-              FC_OK ||
-          (st = launch_mix_tc_split_matrix(0, L, mix_w + (size_t)(v - 1) * (L + 1) * C * C, wsm, s)) !=
-              FC_OK ||
-          (st = launch_mix_tc(L, n_nodes, xs, wsm, states + (size_t)(v - 1) * plane, s)) != FC_OK)
+      if ((st = tp_cm_dispatch(L, g, Av, A1, path_w + (size_t)(v - 1) * P * C, xs, s)) != FC_OK ||
+          (st = launch_path_split_map(g, mix_w + (size_t)(v - 1) * (L + 1) * C * C, wsm, s)) != FC_OK ||
+          (st = launch_path_mix_tc(g, xs, wsm, states + (size_t)(v - 1) * plane, s)) != FC_OK)
         return st;
     }
     return launch_ladder_sum(plane, S, A1, states, z, s);
