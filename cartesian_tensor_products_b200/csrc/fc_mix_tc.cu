@@ -33,6 +33,13 @@
 //
 // C = 128 only (the tile is the whole channel range); other widths use the
 // FP32 SIMT kernels.
+//
+// This file holds three tensor-core kernels:
+//  * ladder_mix_tc_kernel: the mix above.  It is the VJP's B_bar = A_bar M.
+//  * ladder_wgrad_tc_kernel: the VJP's weight gradient.
+//  * path_mix_tc_kernel (further down): the per-rank maps with any K = 32 k_l
+//    over FP32 component-major tiles, split in shared memory.  It serves the
+//    full ladder's (P_l C -> C) maps and the ladder's forward mix (k_l = 4).
 #include "fc_common.cuh"
 #include "fc_device.cuh"
 #include "fc_tc.cuh"
