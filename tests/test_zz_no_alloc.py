@@ -28,7 +28,7 @@ def test_noalloc_ladder_matches_workspace_entry_twice():
     f.restype = ct.c_int
     f.argtypes = [ct.POINTER(fc.LadderDesc), ct.c_int] + [ct.c_void_p] * 6
 
-    L, C, order, N = 3, 128, 4, 512          # 8.5 MiB of scratch (tensor-core path)
+    L, C, order, N = 3, 128, 4, 512          # 4.5 MiB of scratch (tensor-core path)
     wl = W.ladder_inputs(N, L, C, order, 2024)
     dev = torch.device("cuda:0")
     A1 = torch.from_numpy(wl["A1"]).to(dev)
@@ -53,7 +53,7 @@ def test_noalloc_ladder_matches_workspace_entry_twice():
             assert rel_err(states[v].cpu().numpy(), ref_states[v]) <= FWD_TOL
 
     # beyond the 16 MiB array: refused on the host (FC_ERR_WORKSPACE)
-    big = 4096                               # 32 MiB of scratch
+    big = 4096                               # 32.5 MiB of scratch
     st = f(ct.byref(d), big, ct.c_void_p(A1.data_ptr()), ct.c_void_p(pw.data_ptr()),
            ct.c_void_p(mw.data_ptr()), ct.c_void_p(states.data_ptr()),
            ct.c_void_p(z.data_ptr()), stream)
