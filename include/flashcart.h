@@ -239,9 +239,9 @@ int fc_ladder_num_paths(const fc_ladder_desc *desc);
  * the end; other widths use FP32 SIMT kernels.
  * workspace: fc_product_ladder_workspace_size() bytes of device scratch,
  * 16-byte aligned, ws_bytes = its real size; FC_ERR_WORKSPACE if NULL or
- * smaller.  At C = 128 that is the product in the mix's tiled split layout
- * (128-row tiles per rank, TF32 hi and lo: about two product states) plus
- * one step's split matrices; otherwise one product state.
+ * smaller.  At C = 128 that is the product as FP32 128-node tiles per rank
+ * and component (about one product state, node count rounded up to 128)
+ * plus one step's TF32 hi / lo matrices; otherwise one product state.
  * order = 1 copies A1 to z and needs no workspace. */
 size_t fc_product_ladder_workspace_size(const fc_ladder_desc *desc, int n_nodes);
 int fc_product_ladder(const fc_ladder_desc *desc, int n_nodes, const float *A1,
@@ -275,8 +275,8 @@ int fc_product_ladder_vjp(const fc_ladder_desc *desc, int n_nodes,
  * inside the library, held by every GPU that loads the library until the
  * process exits.
  *   Limit: fc_product_ladder_workspace_size(desc, n_nodes) <= 16 MiB (at
- *   rank 3, C = 128: about 990 nodes), else FC_ERR_WORKSPACE and nothing is
- *   enqueued.
+ *   rank 3, C = 128: up to 1,920 nodes), else FC_ERR_WORKSPACE and nothing
+ *   is enqueued.
  *   The first call on a device looks up the array's device address (a
  *   runtime query, no allocation); make that first call before any stream
  *   capture on that device.
