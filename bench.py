@@ -71,8 +71,8 @@ def algorithmic_flops(E, C, L):
 
 
 # DRAM bytes (read + write) of one edge_conv_fwd_kernel<3, 128> launch on
-# this workload from an ncu capture (profiles/edge_conv_fwd_microbench_r3.md),
-# valid only while the kernel sources hash to the value it was taken with.
+# this workload from an ncu capture of the same command, valid only while
+# the kernel sources hash to the value it was taken with.
 FWD_TRAFFIC = {"sha1": "2a7bed009b4741f5c1c7e549431201dec8d0beda", "bytes": 1595942912 + 48170496}
 # the files that define the timed kernel's code (the .cu only dispatches)
 FWD_SOURCES = ("cartesian_tensor_products_b200/csrc/fc_edge_conv.cuh",
@@ -388,13 +388,15 @@ def extra_rows(fc, W, dev, stream, peaks, fp32_peak, steps, select=ROW_NAMES):
             "ms": msl, "ms_min": mnl,
             "roofline": bound(fb, tp_flops + (0 if tc else mix_flops), 3 * mix_flops if tc else 0, msl),
             "l2_flush": "256 MB written before every call"}
-        # VJP: states and A1 read, gz read, A1_bar written; products 4x, mixes 2x (B_bar, M_bar)
+        # VJP: states and A1 read, gz read, A1_bar written; products 4x (FP32
+        # SIMT); two mixes per step, B_bar = A_bar M and M_bar = A_bar^T B, both
+        # on the tensor cores at C = 128 (three TF32 products each), else FP32
         vb = plane_b * (1 + S + 1 + 1)
         rows["ladder_vjp"] = {
             "workload": "same ladder, A1_bar + path_w_bar + mix_w_bar",
             "ms": mslb, "ms_min": mnlb,
-            "roofline": bound(vb, 4 * tp_flops + mix_flops + (0 if tc else mix_flops),
-                              3 * mix_flops if tc else 0, mslb),
+            "roofline": bound(vb, 4 * tp_flops + (0 if tc else 2 * mix_flops),
+                              6 * mix_flops if tc else 0, mslb),
             "l2_flush": "256 MB written before every call"}
         del A1, pw, mw, gz, ws, res, states
         torch.cuda.empty_cache()

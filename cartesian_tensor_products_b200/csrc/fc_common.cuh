@@ -4,9 +4,31 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "flashcart.h"
 
 namespace fc {
+
+// Host-side per-device set-up flags (kernel attributes, cached queries).
+// Concurrent first calls from several host threads may each run the set-up
+// (the CUDA runtime calls involved are thread-safe and idempotent); the flag
+// itself is an atomic, so there is no data race.
+constexpr int kMaxDevices = 64;
+using DeviceFlags = std::atomic<int>[kMaxDevices];
+
+// Raises a kernel's dynamic shared-memory limit to `bytes` once per device.
+template <class Kernel>
+inline int set_smem_once(DeviceFlags& done, Kernel kernel, size_t bytes) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return FC_ERR_CUDA;
+  if (done[dev].load(std::memory_order_acquire)) return FC_OK;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) !=
+      cudaSuccess)
+    return FC_ERR_CUDA;
+  done[dev].store(1, std::memory_order_release);
+  return FC_OK;
+}
 
 template <int L, int G, int g>
 struct FwdGroup;

@@ -182,15 +182,8 @@ static int launch_fwd_cc(const ConvArgs& a, cudaStream_t s) {
   static_assert(sizeof(float) * FwdMeta<L>::SMEM_FLOATS <= 227 * 1024,
                 "forward kernel shared memory exceeds the 227 KB per-CTA limit of sm_100");
   const size_t smem = sizeof(float) * (size_t)FwdMeta<L>::SMEM_FLOATS;
-  static int configured[64] = {0};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return FC_ERR_CUDA;
-  if (!configured[dev]) {
-    if (cudaFuncSetAttribute(edge_conv_fwd_kernel<L, CC, ENV>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
-      return FC_ERR_CUDA;
-    configured[dev] = 1;
-  }
+  static DeviceFlags configured;
+  if (set_smem_once(configured, edge_conv_fwd_kernel<L, CC, ENV>, smem) != FC_OK) return FC_ERR_CUDA;
   const long long units = (long long)a.n_nodes * a.ntiles;
   constexpr int WARPS = FwdMeta<L>::WARPS;
   const long long blocks =

@@ -230,15 +230,8 @@ static int launch_vjp_cc(const VjpArgs& a, cudaStream_t s) {
   static_assert(sizeof(float) * VjpMeta<L>::SMEM_FLOATS <= 227 * 1024,
                 "VJP kernel shared memory exceeds the 227 KB per-CTA limit of sm_100");
   const size_t smem = sizeof(float) * (size_t)VjpMeta<L>::SMEM_FLOATS;
-  static int configured[64] = {0};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return FC_ERR_CUDA;
-  if (!configured[dev]) {
-    if (cudaFuncSetAttribute(edge_conv_vjp_kernel<L, CC>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
-      return FC_ERR_CUDA;
-    configured[dev] = 1;
-  }
+  static DeviceFlags configured;
+  if (set_smem_once(configured, edge_conv_vjp_kernel<L, CC>, smem) != FC_OK) return FC_ERR_CUDA;
   const long long units = (long long)a.n_nodes * a.ntiles;
   constexpr int WARPS = VjpMeta<L>::WARPS;
   const long long blocks = (units + WARPS - 1) / WARPS * VjpMeta<L>::G;

@@ -624,19 +624,19 @@ int fc_product_ladder_vjp(const fc_ladder_desc* d, int n_nodes, const float* A1,
 namespace fc {
 constexpr size_t kLadderStaticScratchBytes = 16u << 20;   // 16 MiB per GPU
 static __device__ __align__(256) float g_ladder_scratch[kLadderStaticScratchBytes / sizeof(float)];
-static void* g_ladder_scratch_addr[64] = {nullptr};
+static std::atomic<void*> g_ladder_scratch_addr[kMaxDevices];
 
 // Device address of g_ladder_scratch on the current device (set-up on the
 // first call per device), or nullptr if the runtime call fails.
 static void* ladder_static_scratch() {
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-  if (g_ladder_scratch_addr[dev] == nullptr) {
-    void* p = nullptr;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  void* p = g_ladder_scratch_addr[dev].load(std::memory_order_acquire);
+  if (p == nullptr) {
     if (cudaGetSymbolAddress(&p, g_ladder_scratch) != cudaSuccess) return nullptr;
-    g_ladder_scratch_addr[dev] = p;
+    g_ladder_scratch_addr[dev].store(p, std::memory_order_release);
   }
-  return g_ladder_scratch_addr[dev];
+  return p;
 }
 }  // namespace fc
 

@@ -58,13 +58,21 @@ constexpr int kTcBlockFloats = kTcRows * kTcChunk;   // 4096: one hi or lo chunk
 constexpr int kTcChunkFloats = 2 * kTcBlockFloats;   // hi + lo of one chunk
 constexpr int kTcWFloats = kTcC * kTcC;              // 16384: one hi or lo block (tile or matrix)
 constexpr int kTcTileFloats = 2 * kTcWFloats;        // hi + lo of a tile
-constexpr uint32_t kTcWaitPolls = 1u << 22;
-constexpr int kTcBars = 2 * kTcStages + 5;   // stage_full[3], stage_free[3], w_full, acc_full[2], acc_free[2]
+// Bounds of the mbarrier waits (global-timer nanoseconds).  A wait that runs
+// out skips the rest of the CTA's work and sets g_tc_error instead of
+// hanging; g_tc_wait_ns is the bound of every ordinary wait (settable per
+// device through fc_set_wait_timeout), kTcDrainNs the fixed, longer bound of
+// the waits on work already in flight (bulk copies, MMAs) that a CTA must
+// see finish before it releases TMEM and exits.
+constexpr uint64_t kTcDrainNs = 2000000000ull;
+constexpr unsigned long long kTcDefaultWaitNs = 500000000ull;
+constexpr int kTcBars = 2 * kTcStages + 6;   // stage_full[3], stage_free[3], w_full, acc_full[2], acc_free[2], drain
 constexpr size_t kTcSmemBytes =
     sizeof(float) * (2 * kTcWFloats + kTcStages * kTcChunkFloats) + 8 * kTcBars + 8;
 static_assert(kTcSmemBytes <= 232448, "shared memory per CTA");
 
 __device__ int g_tc_error = 0;
+__device__ unsigned long long g_tc_wait_ns = kTcDefaultWaitNs;
 
 // Launch geometry in registers (scalar fields only, so the argument block is
 // never copied to local memory).
@@ -189,7 +197,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) ladder_mix_tc_kernel(Geom geo,
   uint64_t* w_full = stage_free + kTcStages;
   uint64_t* acc_full = w_full + 1;
   uint64_t* acc_free = acc_full + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_free + 2);
+  uint64_t* drain = acc_free + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int T = tile_count(geo);
@@ -207,12 +216,14 @@ __global__ void __launch_bounds__(kTcThreads, 1) ladder_mix_tc_kernel(Geom geo,
     tc::bar_init(&acc_full[1], 1);
     tc::bar_init(&acc_free[0], 128);
     tc::bar_init(&acc_free[1], 128);
+    tc::bar_init(drain, 1);
     tc::fence_bar_init();
   }
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();
   const uint32_t tmem = *tmem_slot;
+  const uint64_t lim = g_tc_wait_ns;
   bool fail = false;
 
   if (warp == 0) {
@@ -225,7 +236,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) ladder_mix_tc_kernel(Geom geo,
         if (l != cur_l) {
           if (ti > 0) {   // the MMAs of the previous tile have read the old matrix
             const int gl = g - 1;
-            if (!tc::bar_wait(&stage_free[gl % kTcStages], (gl / kTcStages) & 1, kTcWaitPolls)) {
+            if (!tc::bar_wait(&stage_free[gl % kTcStages], (gl / kTcStages) & 1, lim)) {
               fail = true;
               break;
             }
@@ -238,7 +249,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) ladder_mix_tc_kernel(Geom geo,
         for (int c = 0; c < kTcChunks; ++c, ++g) {
           const int s = g % kTcStages;
           if (g >= kTcStages &&
-              !tc::bar_wait(&stage_free[s], ((g - kTcStages) / kTcStages) & 1, kTcWaitPolls)) {
+              !tc::bar_wait(&stage_free[s], ((g - kTcStages) / kTcStages) & 1, lim)) {
             fail = true;
             break;
           }
@@ -252,8 +263,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) ladder_mix_tc_kernel(Geom geo,
       if (fail) {
         // let the copies already issued land before the CTA can exit
         for (int k = 1; k <= kTcStages && g - k >= 0; ++k)
-          tc::bar_wait(&stage_full[(g - k) % kTcStages], ((g - k) / kTcStages) & 1, kTcWaitPolls);
-        if (w_loads > 0) tc::bar_wait(w_full, (w_loads - 1) & 1, kTcWaitPolls);
+          tc::bar_wait(&stage_full[(g - k) % kTcStages], ((g - k) / kTcStages) & 1, kTcDrainNs);
+        if (w_loads > 0) tc::bar_wait(w_full, (w_loads - 1) & 1, kTcDrainNs);
       }
     }
     __syncwarp();
@@ -269,7 +280,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) ladder_mix_tc_kernel(Geom geo,
         const int l = tile_rank(geo, t);
         const uint32_t d_tmem = tmem + (uint32_t)(ti & 1) * kTcRows;
         if (l != cur_l) {
-          if (!tc::bar_wait(w_full, w_loads & 1, kTcWaitPolls)) {
+          if (!tc::bar_wait(w_full, w_loads & 1, lim)) {
             fail = true;
             break;
           }
@@ -277,14 +288,14 @@ __global__ void __launch_bounds__(kTcThreads, 1) ladder_mix_tc_kernel(Geom geo,
           cur_l = l;
         }
         // the epilogue has drained this accumulator (tile ti - 2)
-        if (ti >= 2 && !tc::bar_wait(&acc_free[ti & 1], ((ti - 2) >> 1) & 1, kTcWaitPolls)) {
+        if (ti >= 2 && !tc::bar_wait(&acc_free[ti & 1], ((ti - 2) >> 1) & 1, lim)) {
           fail = true;
           break;
         }
         tc::fence_after_sync();
         for (int c = 0; c < kTcChunks; ++c, ++g) {
           const int s = g % kTcStages;
-          if (!tc::bar_wait(&stage_full[s], (g / kTcStages) & 1, kTcWaitPolls)) {
+          if (!tc::bar_wait(&stage_full[s], (g / kTcStages) & 1, lim)) {
             fail = true;
             break;
           }
@@ -307,6 +318,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) ladder_mix_tc_kernel(Geom geo,
           if (c == kTcChunks - 1) tc::commit(&acc_full[ti & 1]);
         }
       }
+      // every MMA issued above has finished (also after a wait gave up)
+      // before the CTA releases TMEM and its shared memory
+      tc::commit(drain);
+      if (!tc::bar_wait(drain, 0, kTcDrainNs)) fail = true;
     }
     __syncwarp();
   } else if (warp >= 4) {
@@ -320,7 +335,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) ladder_mix_tc_kernel(Geom geo,
       const int R = geo.N * w;
       const int row0 = (t - tile_first(geo, l)) * kTcRows;
       const uint32_t d_tmem = tmem + (uint32_t)(ti & 1) * kTcRows + ((uint32_t)(32 * ew) << 16);
-      if (!tc::bar_wait(&acc_full[ti & 1], (ti >> 1) & 1, kTcWaitPolls)) {
+      if (!tc::bar_wait(&acc_full[ti & 1], (ti >> 1) & 1, lim)) {
         fail = true;
         break;
       }
@@ -418,7 +433,8 @@ __global__ void __launch_bounds__(kWgThreads, 1) ladder_wgrad_tc_kernel(Geom geo
   uint64_t* stage_free = stage_full + kTcStages;
   uint64_t* acc_full = stage_free + kTcStages;
   uint64_t* acc_free = acc_full + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_free + 1);
+  uint64_t* drain = acc_free + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int T = tile_count(geo);
@@ -433,12 +449,14 @@ __global__ void __launch_bounds__(kWgThreads, 1) ladder_wgrad_tc_kernel(Geom geo
     }
     tc::bar_init(acc_full, 1);
     tc::bar_init(acc_free, 128);
+    tc::bar_init(drain, 1);
     tc::fence_bar_init();
   }
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();
   const uint32_t tmem = *tmem_slot;
+  const uint64_t lim = g_tc_wait_ns;
   bool fail = false;
 
   if (warp == 0) {
@@ -449,7 +467,7 @@ __global__ void __launch_bounds__(kWgThreads, 1) ladder_wgrad_tc_kernel(Geom geo
         for (int c = 0; c < kTcChunks; ++c, ++g) {
           const int s = g % kTcStages;
           if (g >= kTcStages &&
-              !tc::bar_wait(&stage_free[s], ((g - kTcStages) / kTcStages) & 1, kTcWaitPolls)) {
+              !tc::bar_wait(&stage_free[s], ((g - kTcStages) / kTcStages) & 1, lim)) {
             fail = true;
             break;
           }
@@ -466,7 +484,7 @@ __global__ void __launch_bounds__(kWgThreads, 1) ladder_wgrad_tc_kernel(Geom geo
       }
       if (fail)   // let the copies already issued land
         for (int k = 1; k <= kTcStages && g - k >= 0; ++k)
-          tc::bar_wait(&stage_full[(g - k) % kTcStages], ((g - k) / kTcStages) & 1, kTcWaitPolls);
+          tc::bar_wait(&stage_full[(g - k) % kTcStages], ((g - k) / kTcStages) & 1, kTcDrainNs);
     }
     __syncwarp();
   } else if (warp == 1) {
@@ -481,7 +499,7 @@ __global__ void __launch_bounds__(kWgThreads, 1) ladder_wgrad_tc_kernel(Geom geo
         if (l != cur_l) {
           if (cur_l >= 0) {   // publish the finished rank, wait until it is drained
             tc::commit(acc_full);
-            if (!tc::bar_wait(acc_free, seg & 1, kTcWaitPolls)) {
+            if (!tc::bar_wait(acc_free, seg & 1, lim)) {
               fail = true;
               break;
             }
@@ -492,7 +510,7 @@ __global__ void __launch_bounds__(kWgThreads, 1) ladder_wgrad_tc_kernel(Geom geo
         }
         for (int c = 0; c < kTcChunks; ++c, ++g) {
           const int s = g % kTcStages;
-          if (!tc::bar_wait(&stage_full[s], (g / kTcStages) & 1, kTcWaitPolls)) {
+          if (!tc::bar_wait(&stage_full[s], (g / kTcStages) & 1, lim)) {
             fail = true;
             break;
           }
@@ -517,6 +535,10 @@ __global__ void __launch_bounds__(kWgThreads, 1) ladder_wgrad_tc_kernel(Geom geo
         fresh = false;
       }
       if (!fail && cur_l >= 0) tc::commit(acc_full);   // the last rank of the range
+      // every MMA issued above has finished (also after a wait gave up)
+      // before the CTA releases TMEM and its shared memory
+      tc::commit(drain);
+      if (!tc::bar_wait(drain, 0, kTcDrainNs)) fail = true;
     }
     __syncwarp();
   } else if (warp >= 4) {
@@ -528,7 +550,7 @@ __global__ void __launch_bounds__(kWgThreads, 1) ladder_wgrad_tc_kernel(Geom geo
       const int l = t < t_end ? tile_rank(geo, t) : -1;
       if (l == cur_l) continue;
       if (cur_l >= 0) {
-        if (!tc::bar_wait(acc_full, seg & 1, kTcWaitPolls)) {
+        if (!tc::bar_wait(acc_full, seg & 1, lim)) {
           fail = true;
           break;
         }
@@ -666,7 +688,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) path_mix_tc_kernel(PathGeom geo
   uint64_t* cvt_free = cvt_full + 2;
   uint64_t* acc_full = cvt_free + 2;
   uint64_t* acc_free = acc_full + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_free + 2);
+  uint64_t* drain = acc_free + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const long long total = pg_chunks_before(geo, geo.L + 1);
@@ -685,12 +708,14 @@ __global__ void __launch_bounds__(kTcThreads, 1) path_mix_tc_kernel(PathGeom geo
       tc::bar_init(&acc_full[b], 1);
       tc::bar_init(&acc_free[b], 128);
     }
+    tc::bar_init(drain, 1);
     tc::fence_bar_init();
   }
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();
   const uint32_t tmem = *tmem_slot;
+  const uint64_t lim = g_tc_wait_ns;
   bool fail = false;
 
   if (warp == 0) {
@@ -705,7 +730,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) path_mix_tc_kernel(PathGeom geo
         for (int c = 0; c < kc; ++c, ++g) {
           const int s = g % kTcStages;
           if (g >= kTcStages &&
-              !tc::bar_wait(&stage_free[s], ((g - kTcStages) / kTcStages) & 1, kTcWaitPolls)) {
+              !tc::bar_wait(&stage_free[s], ((g - kTcStages) / kTcStages) & 1, lim)) {
             fail = true;
             break;
           }
@@ -720,7 +745,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) path_mix_tc_kernel(PathGeom geo
       }
       if (fail)   // let the copies already issued land
         for (int k = 1; k <= kTcStages && g - k >= 0; ++k)
-          tc::bar_wait(&stage_full[(g - k) % kTcStages], ((g - k) / kTcStages) & 1, kTcWaitPolls);
+          tc::bar_wait(&stage_full[(g - k) % kTcStages], ((g - k) / kTcStages) & 1, kTcDrainNs);
     }
     __syncwarp();
   } else if (warp == 1) {
@@ -734,15 +759,15 @@ __global__ void __launch_bounds__(kTcThreads, 1) path_mix_tc_kernel(PathGeom geo
         for (int c = 0; c < kc; ++c, ++g) {
           const uint32_t d_tmem = tmem + (uint32_t)(h & 1) * kTcRows;
           if (c % kPmGroup == 0) {   // the epilogue has added group h - 2
-            if (h >= 2 && !tc::bar_wait(&acc_free[h & 1], ((h - 2) >> 1) & 1, kTcWaitPolls)) {
+            if (h >= 2 && !tc::bar_wait(&acc_free[h & 1], ((h - 2) >> 1) & 1, lim)) {
               fail = true;
               break;
             }
             tc::fence_after_sync();
           }
           const int s = g % kTcStages, b = g & 1;
-          if (!tc::bar_wait(&stage_full[s], (g / kTcStages) & 1, kTcWaitPolls) ||
-              !tc::bar_wait(&cvt_full[b], (g >> 1) & 1, kTcWaitPolls)) {
+          if (!tc::bar_wait(&stage_full[s], (g / kTcStages) & 1, lim) ||
+              !tc::bar_wait(&cvt_full[b], (g >> 1) & 1, lim)) {
             fail = true;
             break;
           }
@@ -767,6 +792,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) path_mix_tc_kernel(PathGeom geo
           if (c % kPmGroup == kPmGroup - 1 || c == kc - 1) tc::commit(&acc_full[(h++) & 1]);
         }
       }
+      // every MMA issued above has finished (also after a wait gave up)
+      // before the CTA releases TMEM and its shared memory
+      tc::commit(drain);
+      if (!tc::bar_wait(drain, 0, kTcDrainNs)) fail = true;
     }
     __syncwarp();
   } else if (warp < 4) {
@@ -777,8 +806,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) path_mix_tc_kernel(PathGeom geo
       const int kc = pg_kc(geo, pg_rank(geo, t));
       for (int c = 0; c < kc; ++c, ++g) {
         const int s = g % kTcStages, b = g & 1;
-        if (!tc::bar_wait(&stage_full[s], (g / kTcStages) & 1, kTcWaitPolls) ||
-            (g >= 2 && !tc::bar_wait(&cvt_free[b], ((g - 2) >> 1) & 1, kTcWaitPolls))) {
+        if (!tc::bar_wait(&stage_full[s], (g / kTcStages) & 1, lim) ||
+            (g >= 2 && !tc::bar_wait(&cvt_free[b], ((g - 2) >> 1) & 1, lim))) {
           fail = true;
           break;
         }
@@ -819,7 +848,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) path_mix_tc_kernel(PathGeom geo
       const int cmn = (tr - cmc * geo.nb) * kTcRows;   // and its first node
       float acc[kTcRows];
       for (int gi = 0; gi < (kc + kPmGroup - 1) / kPmGroup; ++gi, ++h) {
-        if (!tc::bar_wait(&acc_full[h & 1], (h >> 1) & 1, kTcWaitPolls)) {
+        if (!tc::bar_wait(&acc_full[h & 1], (h >> 1) & 1, lim)) {
           fail = true;
           break;
         }
@@ -855,9 +884,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) path_mix_tc_kernel(PathGeom geo
   }
 }
 
-int g_tc_smem_set[64] = {0};
-int g_wg_smem_set[64] = {0};
-int g_pm_smem_set[64] = {0};
+DeviceFlags g_tc_smem_set;
+DeviceFlags g_wg_smem_set;
+DeviceFlags g_pm_smem_set;
 
 }  // namespace
 
@@ -898,14 +927,7 @@ int launch_mix_tc_split_matrix(int mode, int L, const float* M, float* ws, cudaS
 
 int launch_mix_tc(int L, int N, const float* xs, const float* ws, float* out, cudaStream_t s) {
   if (!mix_tc_supported(L, kTcC)) return FC_ERR_UNSUPPORTED_RANK;
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return FC_ERR_CUDA;
-  if (!g_tc_smem_set[dev]) {
-    if (cudaFuncSetAttribute(ladder_mix_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)kTcSmemBytes) != cudaSuccess)
-      return FC_ERR_CUDA;
-    g_tc_smem_set[dev] = 1;
-  }
+  if (set_smem_once(g_tc_smem_set, ladder_mix_tc_kernel, kTcSmemBytes) != FC_OK) return FC_ERR_CUDA;
   const Geom g = make_geom(L, N);
   const int T = tile_count(g);
   if (T == 0) return FC_OK;
@@ -925,14 +947,7 @@ int launch_mix_tc_split_cols(int L, int N, const float* in, float* xs, cudaStrea
 
 int launch_wgrad_tc(int L, int N, const float* as, const float* bs, float* Mbar, cudaStream_t s) {
   if (!mix_tc_supported(L, kTcC)) return FC_ERR_UNSUPPORTED_RANK;
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return FC_ERR_CUDA;
-  if (!g_wg_smem_set[dev]) {
-    if (cudaFuncSetAttribute(ladder_wgrad_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)kWgSmemBytes) != cudaSuccess)
-      return FC_ERR_CUDA;
-    g_wg_smem_set[dev] = 1;
-  }
+  if (set_smem_once(g_wg_smem_set, ladder_wgrad_tc_kernel, kWgSmemBytes) != FC_OK) return FC_ERR_CUDA;
   const Geom g = make_geom(L, N);
   const int T = tile_count(g);
   if (T == 0) return FC_OK;
@@ -981,14 +996,7 @@ int launch_path_split_map(const PathGeom& g, const float* W, float* ws, cudaStre
 
 int launch_path_mix_tc(const PathGeom& g, const float* xs, const float* ws, float* out, cudaStream_t s) {
   if (g.L < 0 || g.L > 4) return FC_ERR_UNSUPPORTED_RANK;
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return FC_ERR_CUDA;
-  if (!g_pm_smem_set[dev]) {
-    if (cudaFuncSetAttribute(path_mix_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)kPmSmemBytes) != cudaSuccess)
-      return FC_ERR_CUDA;
-    g_pm_smem_set[dev] = 1;
-  }
+  if (set_smem_once(g_pm_smem_set, path_mix_tc_kernel, kPmSmemBytes) != FC_OK) return FC_ERR_CUDA;
   const int T = pg_ts(g, g.L + 1);
   if (T == 0) return FC_OK;
   const int sms = device_sm_count();
@@ -1015,5 +1023,11 @@ extern "C" int fc_device_error(int* flag, fc_stream_t stream) {
         cudaStreamSynchronize(s) != cudaSuccess)
       return FC_ERR_CUDA;
   }
+  return FC_OK;
+}
+
+extern "C" int fc_set_wait_timeout(uint64_t ns) {
+  const unsigned long long v = ns ? (unsigned long long)ns : fc::kTcDefaultWaitNs;
+  if (cudaMemcpyToSymbol(fc::g_tc_wait_ns, &v, sizeof(v)) != cudaSuccess) return FC_ERR_CUDA;
   return FC_OK;
 }

@@ -79,11 +79,20 @@ __device__ __forceinline__ void fence_bar_init() {
   asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
 }
 
+// Nanoseconds of the GPU's global timer.
+__device__ __forceinline__ uint64_t global_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
 // Waits for the completion of the barrier phase with the given parity; gives
-// up after max_iter polls and returns false.
-__device__ __forceinline__ bool bar_wait(uint64_t* bar, uint32_t parity, uint32_t max_iter) {
+// up and returns false once limit_ns nanoseconds of the global timer have
+// passed since the first poll (the timer is read every 16 polls).
+__device__ __forceinline__ bool bar_wait(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
   const uint32_t a = smem_addr(bar);
-  for (uint32_t i = 0; i < max_iter; ++i) {
+  uint64_t t0 = 0;
+  for (uint32_t i = 0;; ++i) {
     uint32_t done;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
@@ -93,8 +102,11 @@ __device__ __forceinline__ bool bar_wait(uint64_t* bar, uint32_t parity, uint32_
         : "r"(a), "r"(parity)
         : "memory");
     if (done) return true;
+    if (i == 0)
+      t0 = global_ns();
+    else if ((i & 15) == 0 && global_ns() - t0 > limit_ns)
+      return false;
   }
-  return false;
 }
 
 // Arrival that also expects `bytes` of asynchronous-copy data on the barrier.

@@ -67,6 +67,8 @@ _SIGS = {
     "fc_product_ladder_vjp": (ct.c_int, [ct.POINTER(LadderDesc), ct.c_int, _vp, _vp, _vp, _vp,
                                          _vp, _vp, _vp, _vp, _vp, ct.c_size_t, _vp]),
     "fc_device_error": (ct.c_int, [ct.POINTER(ct.c_int), _vp]),
+    "fc_set_wait_timeout": (ct.c_int, [ct.c_uint64]),
+    "fc_edge_conv_workspace_size": (ct.c_size_t, [ct.POINTER(ConvDesc), ct.c_int, ct.c_int]),
     "fc_edge_conv_vjp_vjp": (ct.c_int, [ct.POINTER(ConvDesc), ct.c_int, ct.c_int] + [_vp] * 14),
     "fc_full_ladder_workspace_size": (ct.c_size_t, [ct.POINTER(LadderDesc), ct.c_int]),
     "fc_full_ladder": (ct.c_int, [ct.POINTER(LadderDesc), ct.c_int, _vp, _vp, _vp, _vp, _vp, _vp,
@@ -350,6 +352,12 @@ def device_error(stream=None):
     flag = ct.c_int(0)
     _check(_lib.fc_device_error(ct.byref(flag), _stream(stream)), "fc_device_error")
     return flag.value
+
+
+def set_wait_timeout(ns=0):
+    """Bound (ns) of the tensor-core kernels' barrier waits on the current
+    device; 0 restores the default."""
+    _check(_lib.fc_set_wait_timeout(int(ns)), "fc_set_wait_timeout")
 
 
 def scalar_readout(lmax, z, want_grad=True, stream=None):

@@ -111,6 +111,13 @@ int fc_conv_out_row(const fc_conv_desc *desc);
 /* Path p of the descriptor: writes l1, l2, l3.  Returns FC_OK or FC_ERR_ARG. */
 int fc_conv_path(const fc_conv_desc *desc, int p, int *l1, int *l2, int *l3);
 
+/* Scratch bytes the convolution calls need: always 0.  Every receiver's sums
+ * are accumulated on chip and stored once (Algorithm 1), so fc_edge_conv,
+ * fc_edge_conv_vjp and fc_edge_conv_vjp_vjp take no workspace argument; the
+ * query exists for callers written against a workspace-size convention.
+ * The descriptor and sizes are not inspected. */
+size_t fc_edge_conv_workspace_size(const fc_conv_desc *desc, int n_nodes, int n_edges);
+
 /* Build the receiver row pointer of a receiver-sorted edge list and
  * validate the graph (App. D "Receiver-sorted forward").
  *   edge_index [2][n_edges] int32 (device), edge_vec [n_edges][3] float
@@ -319,11 +326,23 @@ int fc_full_ladder(const fc_ladder_desc *desc, int n_nodes, const float *A,
                    void *workspace, size_t ws_bytes, fc_stream_t stream);
 
 /* Sticky device-side error word of the kernels that wait on barriers (the
- * tensor-core ladder mix): each wait gives up after a bounded number of
- * polls, skips the rest of its work and sets the word instead of hanging.
+ * tensor-core mixes and maps of the ladders): each wait gives up after a
+ * bounded time (fc_set_wait_timeout), skips the rest of its CTA's work --
+ * after letting the copies and MMAs it already started finish -- and sets
+ * the word instead of hanging; that call's outputs are then meaningless.
  * Synchronises `stream`, writes the word to *flag (0 = no wait gave up
  * since the last call) and clears it.  FC_ERR_ARG if flag is NULL. */
 int fc_device_error(int *flag, fc_stream_t stream);
+
+/* Bound, in nanoseconds of the GPU's global timer, of every barrier wait in
+ * the tensor-core kernels on the current device (ns = 0 restores the
+ * default of 500 ms; a healthy wait lasts microseconds).  A synchronous
+ * copy to the device: it applies to kernels launched after it returns, so
+ * call it while none of this library's kernels runs on the device.  A
+ * very small bound makes the waits give up (fc_device_error then reports
+ * 1), which is how the give-up path can be exercised.  Returns FC_OK or
+ * FC_ERR_CUDA. */
+int fc_set_wait_timeout(uint64_t ns);
 
 #ifdef __cplusplus
 }

@@ -67,9 +67,12 @@ def test_diamond_1000_sampled(fc):
                                         recv_mask=mask)
     rows = np.nonzero(mask)[0]
     assert rel_err(e_node[rows], re[rows]) <= FWD_TOL
+    # normwise against the whole force tensor: max over the sampled atoms of
+    # |F_i - ref_i| <= 1e-4 max|F| (the full reference is not formed)
+    fmax = np.abs(F).max()
     for i in atoms:
         ref = -(dEdr[send == i].sum(0) - dEdr[recv == i].sum(0))
-        assert rel_err(F[i], ref) <= VJP_TOL * np.abs(F).max() / np.abs(ref).max() + VJP_TOL
+        assert np.abs(F[i] - ref).max() <= VJP_TOL * fmax
     # translation invariance at full size
     assert np.abs(F.sum(0)).max() <= 1e-3 * np.abs(F).max()
     assert np.isfinite(E)
