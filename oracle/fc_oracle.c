@@ -1104,6 +1104,174 @@ int orc_full_ladder(int L, int C, int order, int N, const double *A,
   return 0;
 }
 
+/* Reverse accumulation through the full ladder (orc_full_ladder above).
+ * gz: [N][(L+1)^2 C], the gradient of z.  Every phi_q feeds z directly, so
+ * its gradient starts at gz; going down from q = order:
+ *   Wq_bar[l][j][eta C + k] += sum_c phibar_q[l,c,j] B_q[eta,c,k]
+ *   Bbar_q[eta,c,k]          = sum_j Wq[l][j][eta C + k] phibar_q[l,c,j]
+ *   phibar_{q-1}[l1,b1,k]   += sum_{a,b2} Bbar_q[eta,a,k] K[a][b1][b2] A[l2,b2,k]
+ *   A_bar[l2,b2,k]          += sum_{a,b1} Bbar_q[eta,a,k] K[a][b1][b2] phi_{q-1}[l1,b1,k]
+ * with K the path's coefficient tensor (f_a = sum K[a][b1][b2] x_b1 y_b2,
+ * bilinear, App. C Eq. C1), and at the first map
+ *   W1_bar[l][j][k] += sum_c phibar_1[l,c,j] A[l,c,k],
+ *   A_bar[l,c,k]    += sum_j W1[l][j][k] phibar_1[l,c,j].
+ * Weight gradients sum over the nodes that node_mask selects (NULL = all);
+ * A_bar rows of other nodes are 0.  W1_bar like W1, Wq_bar like Wq. */
+int orc_full_ladder_vjp(int L, int C, int order, int N, const double *A,
+                        const double *W1, const double *Wq, const double *gz,
+                        const unsigned char *node_mask, double *A_bar,
+                        double *W1_bar, double *Wq_bar) {
+  if (L > 4 || order < 1) return 1;
+  path_set ps;
+  make_paths(L, L, L, 0, &ps);
+  int row = (L + 1) * (L + 1);
+  size_t nrow = (size_t)row * C;
+  int rankoff[ORC_MAXL + 2];
+  rankoff[0] = 0;
+  for (int l = 0; l <= L; ++l) rankoff[l + 1] = rankoff[l] + ps.Pl[l];
+  double *K[ORC_MAXP];
+  for (int p = 0; p < ps.P; ++p) {
+    int n1 = 2 * ps.l1[p] + 1, n2 = 2 * ps.l2[p] + 1, n3 = 2 * ps.l3[p] + 1;
+    K[p] = (double *)malloc(sizeof(double) * n1 * n2 * n3);
+    orc_path_coeffs(ps.l1[p], ps.l2[p], ps.l3[p], K[p]);
+  }
+  size_t w1_n = (size_t)(L + 1) * C * C;
+  size_t wq_n = (size_t)(order > 1 ? order - 1 : 1) * C * ps.P * C;
+  size_t bsz = (size_t)ps.P * (2 * L + 1) * C;
+  memset(A_bar, 0, sizeof(double) * (size_t)N * nrow);
+  if (W1_bar) memset(W1_bar, 0, sizeof(double) * w1_n);
+  if (Wq_bar && order > 1) memset(Wq_bar, 0, sizeof(double) * (size_t)(order - 1) * C * ps.P * C);
+
+#pragma omp parallel
+  {
+    double *w1b = (double *)calloc(w1_n, sizeof(double));
+    double *wqb = (double *)calloc(wq_n, sizeof(double));
+    double *phi = (double *)malloc(sizeof(double) * (size_t)order * nrow);
+    double *B = (double *)malloc(sizeof(double) * (size_t)order * bsz);
+    double *pb = (double *)malloc(sizeof(double) * nrow);
+    double *pbn = (double *)malloc(sizeof(double) * nrow);
+    double *Bb = (double *)malloc(sizeof(double) * bsz);
+    double xc[2 * ORC_MAXL + 1], yc[2 * ORC_MAXL + 1], f[2 * ORC_MAXL + 1];
+#pragma omp for schedule(dynamic, 1)
+    for (int n = 0; n < N; ++n) {
+      if (node_mask && !node_mask[n]) continue;
+      const double *a = A + (size_t)n * nrow;
+      double *ab = A_bar + (size_t)n * nrow;
+      /* forward, keeping phi_q (index q-1) and B_q (index q-1, q >= 2) */
+      for (int l = 0; l <= L; ++l)
+        for (int c = 0; c < 2 * l + 1; ++c)
+          for (int j = 0; j < C; ++j) {
+            double t = 0.0;
+            for (int k = 0; k < C; ++k)
+              t += W1[((size_t)l * C + j) * C + k] * a[(l * l + c) * C + k];
+            phi[(l * l + c) * C + j] = t;
+          }
+      for (int q = 2; q <= order; ++q) {
+        const double *prev = phi + (size_t)(q - 2) * nrow;
+        double *Bq = B + (size_t)(q - 1) * bsz;
+        double *cur = phi + (size_t)(q - 1) * nrow;
+        for (int p = 0; p < ps.P; ++p) {
+          int l1 = ps.l1[p], l2 = ps.l2[p], l3 = ps.l3[p];
+          for (int k = 0; k < C; ++k) {
+            for (int i = 0; i < 2 * l1 + 1; ++i) xc[i] = prev[(l1 * l1 + i) * C + k];
+            for (int i = 0; i < 2 * l2 + 1; ++i) yc[i] = a[(l2 * l2 + i) * C + k];
+            orc_product(l1, l2, l3, xc, yc, f);
+            for (int c = 0; c < 2 * l3 + 1; ++c) Bq[((size_t)p * (2 * L + 1) + c) * C + k] = f[c];
+          }
+        }
+        const double *Wqq = Wq + (size_t)(q - 2) * C * ps.P * C;
+        for (int l = 0; l <= L; ++l) {
+          int Kl = ps.Pl[l] * C;
+          const double *Wl = Wqq + (size_t)C * C * rankoff[l];
+          for (int c = 0; c < 2 * l + 1; ++c)
+            for (int j = 0; j < C; ++j) {
+              double t = 0.0;
+              for (int p = 0; p < ps.P; ++p) {
+                if (ps.l3[p] != l) continue;
+                for (int k = 0; k < C; ++k)
+                  t += Wl[(size_t)j * Kl + ps.eta[p] * C + k] * Bq[((size_t)p * (2 * L + 1) + c) * C + k];
+              }
+              cur[(l * l + c) * C + j] = t;
+            }
+        }
+      }
+      /* reverse */
+      memcpy(pb, gz + (size_t)n * nrow, sizeof(double) * nrow);
+      for (int q = order; q >= 2; --q) {
+        const double *prev = phi + (size_t)(q - 2) * nrow;
+        const double *Bq = B + (size_t)(q - 1) * bsz;
+        const double *Wqq = Wq + (size_t)(q - 2) * C * ps.P * C;
+        double *wqg = wqb + (size_t)(q - 2) * C * ps.P * C;
+        for (int p = 0; p < ps.P; ++p) {
+          int l = ps.l3[p];
+          int Kl = ps.Pl[l] * C;
+          const double *Wl = Wqq + (size_t)C * C * rankoff[l];
+          double *Wg = wqg + (size_t)C * C * rankoff[l];
+          for (int j = 0; j < C; ++j)
+            for (int k = 0; k < C; ++k) {
+              double s = 0.0;
+              for (int c = 0; c < 2 * l + 1; ++c)
+                s += pb[(l * l + c) * C + j] * Bq[((size_t)p * (2 * L + 1) + c) * C + k];
+              Wg[(size_t)j * Kl + ps.eta[p] * C + k] += s;
+            }
+          for (int c = 0; c < 2 * l + 1; ++c)
+            for (int k = 0; k < C; ++k) {
+              double s = 0.0;
+              for (int j = 0; j < C; ++j)
+                s += Wl[(size_t)j * Kl + ps.eta[p] * C + k] * pb[(l * l + c) * C + j];
+              Bb[((size_t)p * (2 * L + 1) + c) * C + k] = s;
+            }
+        }
+        /* phi_{q-1} feeds z and step q */
+        memcpy(pbn, gz + (size_t)n * nrow, sizeof(double) * nrow);
+        for (int p = 0; p < ps.P; ++p) {
+          int l1 = ps.l1[p], l2 = ps.l2[p], l3 = ps.l3[p];
+          int n1 = 2 * l1 + 1, n2 = 2 * l2 + 1, n3 = 2 * l3 + 1;
+          const double *Kp = K[p];
+          for (int k = 0; k < C; ++k)
+            for (int aa = 0; aa < n3; ++aa) {
+              double g = Bb[((size_t)p * (2 * L + 1) + aa) * C + k];
+              for (int b1 = 0; b1 < n1; ++b1)
+                for (int b2 = 0; b2 < n2; ++b2) {
+                  double kk = Kp[(aa * n1 + b1) * n2 + b2];
+                  pbn[(l1 * l1 + b1) * C + k] += g * kk * a[(l2 * l2 + b2) * C + k];
+                  ab[(l2 * l2 + b2) * C + k] += g * kk * prev[(l1 * l1 + b1) * C + k];
+                }
+            }
+        }
+        memcpy(pb, pbn, sizeof(double) * nrow);
+      }
+      /* the first map */
+      for (int l = 0; l <= L; ++l)
+        for (int j = 0; j < C; ++j)
+          for (int k = 0; k < C; ++k) {
+            double s = 0.0;
+            for (int c = 0; c < 2 * l + 1; ++c)
+              s += pb[(l * l + c) * C + j] * a[(l * l + c) * C + k];
+            w1b[((size_t)l * C + j) * C + k] += s;
+          }
+      for (int l = 0; l <= L; ++l)
+        for (int c = 0; c < 2 * l + 1; ++c)
+          for (int k = 0; k < C; ++k) {
+            double s = 0.0;
+            for (int j = 0; j < C; ++j)
+              s += W1[((size_t)l * C + j) * C + k] * pb[(l * l + c) * C + j];
+            ab[(l * l + c) * C + k] += s;
+          }
+    }
+#pragma omp critical(orc_full_ladder_reduce)
+    {
+      if (W1_bar)
+        for (size_t i = 0; i < w1_n; ++i) W1_bar[i] += w1b[i];
+      if (Wq_bar && order > 1)
+        for (size_t i = 0; i < (size_t)(order - 1) * C * ps.P * C; ++i) Wq_bar[i] += wqb[i];
+    }
+    free(w1b); free(wqb); free(phi); free(B); free(pb); free(pbn); free(Bb);
+  }
+  for (int p = 0; p < ps.P; ++p) free(K[p]);
+  return 0;
+}
+
 /* Reverse accumulation through the ladder above.  gz: [N][(L+1)^2 C].
  * A1_bar like A1; path_w_bar like path_w; mix_bar like mix.  Weight
  * gradients sum over the nodes that node_mask selects (NULL = all). */

@@ -44,6 +44,7 @@ def lib():
                                                                d, d, d, d]),
             "orc_direction_hvp": (None, [ct.c_int, d, d, d, d]),
             "orc_full_ladder": (ct.c_int, [ct.c_int] * 4 + [d, d, d, u8, d, d]),
+            "orc_full_ladder_vjp": (ct.c_int, [ct.c_int] * 4 + [d, d, d, d, u8, d, d, d]),
             "orc_ladder": (ct.c_int, [ct.c_int] * 4 + [d, d, d, u8, d, d]),
             "orc_ladder_vjp": (ct.c_int, [ct.c_int] * 4 + [d, d, d, d, u8, d, d, d]),
             "orc_max_rank": (ct.c_int, []),
@@ -419,3 +420,22 @@ def full_ladder(L, C, order, A, W1, Wq, node_mask=None):
     assert rc == 0
     return states, z
 
+
+def full_ladder_vjp(L, C, order, A, W1, Wq, gz, node_mask=None):
+    """Gradients (A_bar, W1_bar, Wq_bar) of <gz, z> for the full ladder, by
+    reverse accumulation through its steps (Sec. 5 Eq. 2; App. C Eq. C1 for
+    each bilinear product).  Weight gradients sum over the selected nodes."""
+    A = _d(A)
+    N = A.shape[0]
+    P = len(paths(L, L, L))
+    W1 = _d(W1).reshape(L + 1, C, C)
+    Wq = _d(Wq).reshape(order - 1, C * P * C) if order > 1 else np.zeros((1, C * P * C))
+    gz = _d(gz)
+    Ab = np.empty_like(A)
+    W1b = np.zeros_like(W1)
+    Wqb = np.zeros_like(Wq)
+    m = None if node_mask is None else _mask(node_mask, N)
+    rc = lib().orc_full_ladder_vjp(L, C, order, N, _pd(A), _pd(W1), _pd(np.ascontiguousarray(Wq)),
+                                   _pd(gz), _pu8(m), _pd(Ab), _pd(W1b), _pd(Wqb))
+    assert rc == 0
+    return Ab, W1b, (Wqb if order > 1 else Wqb[:0])
