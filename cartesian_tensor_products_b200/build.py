@@ -7,6 +7,7 @@ Usage: python -m cartesian_tensor_products_b200.build [--force] [--verbose]
 """
 import glob
 import os
+import re
 import subprocess
 import sys
 
@@ -28,6 +29,33 @@ def _deps():
     return (_sources() + glob.glob(os.path.join(CSRC, "*.cuh"))
             + glob.glob(os.path.join(GEN, "*.py"))
             + glob.glob(os.path.join(INCLUDE, "*.h")))
+
+
+_INCLUDE_RE = re.compile(r'^\s*#\s*include\s+"([^"]+)"', re.M)
+
+
+def _headers(path, seen=None):
+    """Local headers a source includes, followed recursively (quoted
+    includes resolved next to the including file, in csrc/ or in include/)."""
+    seen = set() if seen is None else seen
+    with open(path) as f:
+        src = f.read()
+    for name in _INCLUDE_RE.findall(src):
+        for d in (os.path.dirname(path), CSRC, INCLUDE):
+            h = os.path.normpath(os.path.join(d, name))
+            if os.path.exists(h):
+                if h not in seen:
+                    seen.add(h)
+                    _headers(h, seen)
+                break
+    return seen
+
+
+def _stale(src, obj):
+    if not os.path.exists(obj):
+        return True
+    t = os.path.getmtime(obj)
+    return any(os.path.getmtime(p) > t for p in [src, __file__] + sorted(_headers(src)))
 
 
 def generate():
@@ -57,6 +85,8 @@ def build(force=False, verbose=False, jobs=None):
     for src in _sources():
         obj = os.path.join(objdir, os.path.basename(src)[:-3] + ".o")
         objs.append(obj)
+        if not force and not _stale(src, obj):
+            continue
         cmd = [NVCC, "-c", src, "-o", obj] + flags
         procs.append((cmd, subprocess.Popen(cmd, stdout=subprocess.PIPE,
                                             stderr=subprocess.STDOUT)))

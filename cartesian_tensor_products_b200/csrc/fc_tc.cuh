@@ -88,23 +88,27 @@ __device__ __forceinline__ uint64_t global_ns() {
 
 // Waits for the completion of the barrier phase with the given parity; gives
 // up and returns false once limit_ns nanoseconds of the global timer have
-// passed since the first poll (the timer is read every 16 polls).
+// passed since the first poll.  Each poll may suspend the thread until the
+// phase completes, for at most min(limit_ns, 1 ms) (the try_wait time hint),
+// so a small limit gives up promptly.
 __device__ __forceinline__ bool bar_wait(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
   const uint32_t a = smem_addr(bar);
+  const uint32_t hint = limit_ns < 1000000ull ? (uint32_t)limit_ns : 1000000u;
   uint64_t t0 = 0;
   for (uint32_t i = 0;; ++i) {
     uint32_t done;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}\n"
         : "=r"(done)
-        : "r"(a), "r"(parity)
+        : "r"(a), "r"(parity), "r"(hint)
         : "memory");
     if (done) return true;
+    const uint64_t now = global_ns();
     if (i == 0)
-      t0 = global_ns();
-    else if ((i & 15) == 0 && global_ns() - t0 > limit_ns)
+      t0 = now;
+    else if (now - t0 > limit_ns)
       return false;
   }
 }

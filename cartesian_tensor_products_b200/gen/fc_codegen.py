@@ -27,6 +27,18 @@ import fc_algebra as A  # noqa: E402
 OUTDIR = os.path.join(os.path.dirname(HERE), "csrc", "generated")
 
 
+
+def write_if_changed(path, src):
+    """Write src to path unless the file already holds it (keeps the mtime,
+    so the incremental build recompiles only what a change touches)."""
+    if os.path.exists(path):
+        with open(path) as f:
+            if f.read() == src:
+                return
+    with open(path, "w") as f:
+        f.write(src)
+
+
 def flit(x):
     """float literal of an exact rational"""
     v = float(x)
@@ -458,12 +470,10 @@ def main():
     for L in (1, 2, 3, 4, 5):
         src, _, _ = emit_fwd(L, NGROUPS[L])
         path = os.path.join(OUTDIR, "fc_fwd_L%d.cuh" % L)
-        with open(path, "w") as f:
-            f.write(src)
+        write_if_changed(path, src)
         written.append(path)
     path = os.path.join(OUTDIR, "fc_tables.cuh")
-    with open(path, "w") as f:
-        f.write(emit_tables((1, 2, 3, 4, 5)))
+    write_if_changed(path, emit_tables((1, 2, 3, 4, 5)))
     written.append(path)
     return written
 
@@ -1004,15 +1014,13 @@ def main():
     for L in (1, 2, 3, 4, 5):
         src, _, _ = emit_vjp(L, VJP_NGROUPS[L])
         path = os.path.join(OUTDIR, "fc_vjp_L%d.cuh" % L)
-        with open(path, "w") as f:
-            f.write(src)
+        write_if_changed(path, src)
         written.append(path)
         if L == 5:          # the VJP-of-VJP is built up to rank 4
             continue
         src, _, _ = emit_vvjp(L, VVJP_NGROUPS[L])
         path = os.path.join(OUTDIR, "fc_vvjp_L%d.cuh" % L)
-        with open(path, "w") as f:
-            f.write(src)
+        write_if_changed(path, src)
         written.append(path)
     return written
 
@@ -1112,8 +1120,7 @@ def main():
     written = _main_conv()
     for L in (1, 2, 3, 4):
         path = os.path.join(OUTDIR, "fc_ladder_L%d.cuh" % L)
-        with open(path, "w") as f:
-            f.write(emit_ladder(L))
+        write_if_changed(path, emit_ladder(L))
         written.append(path)
     return written
 
