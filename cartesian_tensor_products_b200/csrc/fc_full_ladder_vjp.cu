@@ -1,0 +1,464 @@
+// libflashcart: VJP of the full correlation ladder.
+//
+// FlashCart (arXiv 2610.06409) Sec. 5 Eq. (2), the full ladder of
+// fc_full_ladder (every coupling path kept, a learned per-rank map mixing
+// paths and channels), differentiated by reverse accumulation through its
+// steps.  Every phi_q feeds z, so the running gradient pbar of phi_q starts
+// at gz; going down from q = order:
+//   Wq_bar_l[j][eta C + k] += sum_rows pbar[row][j] B_q[row][eta C + k]    (rows of rank l)
+//   Bbar_q[row][eta C + k]  = sum_j pbar[row][j] Wq_l[j][eta C + k]
+//   pbar_{q-1} = gz + the product VJP of B_q = f(phi_{q-1}, A) applied to Bbar_q,
+//   A_bar     += the product VJP's A side
+// (App. C Eq. C1 per path, with B_q recomputed from the saved phi_{q-1});
+// then the first map: W1_bar_l += pbar_1^T A, A_bar += pbar_1 W1_l.
+//
+// Layouts.  B_q and Bbar_q use the convolution's output layout
+// ([N][sum_l (2l+1) P_l][C], slot zoff(l) + c P_l + eta), where the P_l C
+// inputs of one (node, component) row of rank l form one contiguous run, so
+// every map is a GEMM over the rows of a rank: the register-tiled FP32
+// kernels below (64 rows x 128 columns per CTA; 4 x 8 outputs per thread).
+// The weight gradients reduce over the rows (512-row chunks per CTA, one
+// atomic add per entry per chunk; not bitwise reproducible).  The products
+// are channel-diagonal: one thread per channel walks a chunk of nodes with
+// generated straight-line code (exact coefficients).
+#include "fc_common.cuh"
+#include "fc_device.cuh"
+#include "generated/fc_ladder_L1.cuh"
+#include "generated/fc_ladder_L2.cuh"
+#include "generated/fc_ladder_L3.cuh"
+#include "generated/fc_ladder_L4.cuh"
+
+namespace fc {
+
+namespace {
+
+// Rows of rank l are i in [0, N(2l+1)): node n = i / (2l+1), component c;
+// the row starts at float (n stride + off[l] + c cmul[l]) C of its array and
+// holds wid[l] values (a multiple of 4).
+struct RowLayout {
+  int stride;
+  int off[5], cmul[5], wid[5];
+};
+
+__device__ __forceinline__ size_t row_at(const RowLayout& g, int i, int l, int C) {
+  const int w = 2 * l + 1;
+  const int n = i / w;
+  const int c = i - n * w;
+  return ((size_t)n * g.stride + g.off[l] + (size_t)c * g.cmul[l]) * C;
+}
+
+constexpr int kVBM = 64, kVBN = 128, kVBK = 32;
+constexpr int kVRows = 512;          // rows per CTA of the weight-gradient GEMMs
+constexpr int kVChunk = 8;           // nodes per thread of the product VJP
+
+// out_l[row][m] (+)= sum_{t < C} in[row][t] Bm_l[t][m]
+// in: layout `ai` (width C), out: layout `ao` (width ao.wid[l]),
+// Bm_l: [C][ao.wid[l]] row-major at Bm + boff[l].
+template <bool ACC>
+__global__ void __launch_bounds__(256) rows_gemm_kernel(int N, int C, int L, RowLayout ai, RowLayout ao,
+                                                        const float* __restrict__ in,
+                                                        const float* __restrict__ Bm, long long boff0,
+                                                        long long boff1, long long boff2,
+                                                        long long boff3, long long boff4,
+                                                        float* __restrict__ out) {
+  __shared__ __align__(16) float As[kVBK][kVBM + 4];
+  __shared__ __align__(16) float Bs[kVBK][kVBN + 4];
+  const int l = blockIdx.z;
+  if (l > L) return;
+  const int R = N * (2 * l + 1);
+  const int r0 = blockIdx.x * kVBM;
+  const int W = ao.wid[l];
+  const int m0 = blockIdx.y * kVBN;
+  if (r0 >= R || m0 >= W) return;
+  const long long boff = l == 0 ? boff0 : l == 1 ? boff1 : l == 2 ? boff2 : l == 3 ? boff3 : boff4;
+  const float* Bl = Bm + boff;
+  const int tid = threadIdx.x;
+  const int tx = tid & 15, ty = tid >> 4;   // 16 x 16 threads: 8 columns x 4 rows each
+  float acc[4][8];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc[i][j] = 0.0f;
+  for (int t0 = 0; t0 < C; t0 += kVBK) {
+#pragma unroll
+    for (int s = 0; s < 2; ++s) {   // in: 64 rows x 32 t, stored t-major
+      const int idx = tid + s * 256;
+      const int rr = idx >> 3, tq = (idx & 7) * 4;
+      float4 v = zero4();
+      if (r0 + rr < R && t0 + tq < C)
+        v = __ldg(reinterpret_cast<const float4*>(in + row_at(ai, r0 + rr, l, C) + t0 + tq));
+      As[tq + 0][rr] = v.x; As[tq + 1][rr] = v.y; As[tq + 2][rr] = v.z; As[tq + 3][rr] = v.w;
+    }
+#pragma unroll
+    for (int s = 0; s < 4; ++s) {   // Bm: 32 t x 128 m
+      const int idx = tid + s * 256;
+      const int tt = idx >> 5, mq = (idx & 31) * 4;
+      float4 v = zero4();
+      if (t0 + tt < C && m0 + mq < W)
+        v = __ldg(reinterpret_cast<const float4*>(Bl + (size_t)(t0 + tt) * W + m0 + mq));
+      *reinterpret_cast<float4*>(&Bs[tt][mq]) = v;
+    }
+    __syncthreads();
+#pragma unroll 8
+    for (int t = 0; t < kVBK; ++t) {
+      const float4 a = *reinterpret_cast<const float4*>(&As[t][ty * 4]);
+      const float4 b0 = *reinterpret_cast<const float4*>(&Bs[t][tx * 8]);
+      const float4 b1 = *reinterpret_cast<const float4*>(&Bs[t][tx * 8 + 4]);
+      const float av[4] = {a.x, a.y, a.z, a.w};
+      const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int r = r0 + ty * 4 + i;
+    if (r >= R) continue;
+    float* o = out + row_at(ao, r, l, C);
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int m = m0 + tx * 8 + h * 4;
+      if (m >= W) continue;
+      float4 v = make_float4(acc[i][h * 4], acc[i][h * 4 + 1], acc[i][h * 4 + 2], acc[i][h * 4 + 3]);
+      if (ACC) {
+        const float4 p = *reinterpret_cast<const float4*>(o + m);
+        v.x += p.x; v.y += p.y; v.z += p.z; v.w += p.w;
+      }
+      *reinterpret_cast<float4*>(o + m) = v;
+    }
+  }
+}
+
+// Wb_l[j][m] += sum_{rows of rank l} a[row][j] b[row][m]
+// a: layout `la` (width C), b: layout `lb` (width lb.wid[l]),
+// Wb_l: [C][lb.wid[l]] row-major at Wb + woff[l].
+__global__ void __launch_bounds__(256) rows_wgrad_kernel(int N, int C, int L, RowLayout la, RowLayout lb,
+                                                         const float* __restrict__ a,
+                                                         const float* __restrict__ b, float* __restrict__ Wb,
+                                                         long long woff0, long long woff1, long long woff2,
+                                                         long long woff3, long long woff4) {
+  __shared__ __align__(16) float As[kVBK][kVBM + 4];
+  __shared__ __align__(16) float Bs[kVBK][kVBN + 4];
+  const int l = blockIdx.z;
+  if (l > L) return;
+  const int R = N * (2 * l + 1);
+  const int i0 = blockIdx.x * kVRows;
+  if (i0 >= R) return;
+  const int i1 = min(R, i0 + kVRows);
+  const int W = lb.wid[l];
+  const int jt = (C + kVBM - 1) / kVBM;
+  const int j0 = (blockIdx.y % jt) * kVBM;
+  const int m0 = (blockIdx.y / jt) * kVBN;
+  if (m0 >= W) return;
+  const long long woff = l == 0 ? woff0 : l == 1 ? woff1 : l == 2 ? woff2 : l == 3 ? woff3 : woff4;
+  const int tid = threadIdx.x;
+  const int tx = tid & 15, ty = tid >> 4;
+  float acc[4][8];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc[i][j] = 0.0f;
+  for (int t0 = i0; t0 < i1; t0 += kVBK) {
+#pragma unroll
+    for (int s = 0; s < 2; ++s) {   // a: 32 rows x 64 j
+      const int idx = tid + s * 256;
+      const int tt = idx >> 4, jq = (idx & 15) * 4;
+      float4 v = zero4();
+      if (t0 + tt < i1 && j0 + jq < C)
+        v = __ldg(reinterpret_cast<const float4*>(a + row_at(la, t0 + tt, l, C) + j0 + jq));
+      *reinterpret_cast<float4*>(&As[tt][jq]) = v;
+    }
+#pragma unroll
+    for (int s = 0; s < 4; ++s) {   // b: 32 rows x 128 m
+      const int idx = tid + s * 256;
+      const int tt = idx >> 5, mq = (idx & 31) * 4;
+      float4 v = zero4();
+      if (t0 + tt < i1 && m0 + mq < W)
+        v = __ldg(reinterpret_cast<const float4*>(b + row_at(lb, t0 + tt, l, C) + m0 + mq));
+      *reinterpret_cast<float4*>(&Bs[tt][mq]) = v;
+    }
+    __syncthreads();
+#pragma unroll 8
+    for (int t = 0; t < kVBK; ++t) {
+      const float4 av4 = *reinterpret_cast<const float4*>(&As[t][ty * 4]);
+      const float4 b0 = *reinterpret_cast<const float4*>(&Bs[t][tx * 8]);
+      const float4 b1 = *reinterpret_cast<const float4*>(&Bs[t][tx * 8 + 4]);
+      const float av[4] = {av4.x, av4.y, av4.z, av4.w};
+      const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+    }
+    __syncthreads();
+  }
+  float* Wl = Wb + woff;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int j = j0 + ty * 4 + i;
+    if (j >= C) continue;
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int m = m0 + tx * 8 + u;
+      if (m < W) atomicAdd(Wl + (size_t)j * W + m, acc[i][u]);
+    }
+  }
+}
+
+// Product VJP of one step, channel-diagonal, every path with its own output
+// gradient (Bbar in the convolution's output layout):
+//   pbn[n,:,k]  = gz[n,:,k] + d<Bbar, f(phi, A)>/dphi
+//   Abar[n,:,k] +=            d<Bbar, f(phi, A)>/dA
+template <int L>
+__global__ void __launch_bounds__(128) full_tp_vjp_kernel(int N, int C, const float* __restrict__ phi,
+                                                          const float* __restrict__ A,
+                                                          const float* __restrict__ Bbar,
+                                                          const float* __restrict__ gz,
+                                                          float* __restrict__ pbn, float* __restrict__ Abar) {
+  using TP = LadderTP<L>;
+  const int k = blockIdx.y * blockDim.x + threadIdx.x;
+  if (k >= C) return;
+  int zoff[L + 1], Pl[L + 1];
+  {
+    int o = 0;
+#pragma unroll
+    for (int l3 = 0; l3 <= L; ++l3) {
+      int p = 0;
+#pragma unroll
+      for (int l1 = 0; l1 <= L; ++l1)
+#pragma unroll
+        for (int l2 = 0; l2 <= L; ++l2)
+          if (l3 >= (l1 > l2 ? l1 - l2 : l2 - l1) && l3 <= l1 + l2 && ((l1 + l2 + l3) & 1) == 0) ++p;
+      Pl[l3] = p;
+      zoff[l3] = o;
+      o += (2 * l3 + 1) * p;
+    }
+  }
+  const int n0 = blockIdx.x * kVChunk;
+  const int n1 = min(N, n0 + kVChunk);
+  for (int n = n0; n < n1; ++n) {
+    const size_t base = (size_t)n * TP::NY * C + k;
+    const float* gb = Bbar + (size_t)n * TP::ZROW * C + k;
+    float a[TP::NY], b[TP::NY], ab[TP::NY], bb[TP::NY];
+#pragma unroll
+    for (int i = 0; i < TP::NY; ++i) {
+      a[i] = __ldg(phi + base + (size_t)i * C);
+      b[i] = __ldg(A + base + (size_t)i * C);
+      ab[i] = __ldg(gz + base + (size_t)i * C);
+      bb[i] = Abar[base + (size_t)i * C];
+    }
+    TP::vjp_paths(a, b, [&](int l3, int c, int eta) {
+      return __ldg(gb + (size_t)(zoff[l3] + c * Pl[l3] + eta) * C);
+    }, ab, bb);
+#pragma unroll
+    for (int i = 0; i < TP::NY; ++i) {
+      pbn[base + (size_t)i * C] = ab[i];
+      Abar[base + (size_t)i * C] = bb[i];
+    }
+  }
+}
+
+template <int L>
+int launch_full_tp_vjp(int N, int C, const float* phi, const float* A, const float* Bbar,
+                       const float* gz, float* pbn, float* Abar, cudaStream_t s) {
+  dim3 grid((N + kVChunk - 1) / kVChunk, (C + 127) / 128);
+  full_tp_vjp_kernel<L><<<grid, 128, 0, s>>>(N, C, phi, A, Bbar, gz, pbn, Abar);
+  return cudaGetLastError() == cudaSuccess ? FC_OK : FC_ERR_CUDA;
+}
+
+int full_tp_vjp_dispatch(int L, int N, int C, const float* phi, const float* A, const float* Bbar,
+                         const float* gz, float* pbn, float* Abar, cudaStream_t s) {
+  switch (L) {
+    case 1: return launch_full_tp_vjp<1>(N, C, phi, A, Bbar, gz, pbn, Abar, s);
+    case 2: return launch_full_tp_vjp<2>(N, C, phi, A, Bbar, gz, pbn, Abar, s);
+    case 3: return launch_full_tp_vjp<3>(N, C, phi, A, Bbar, gz, pbn, Abar, s);
+    case 4: return launch_full_tp_vjp<4>(N, C, phi, A, Bbar, gz, pbn, Abar, s);
+  }
+  return FC_ERR_UNSUPPORTED_RANK;
+}
+
+// products of one step in the convolution's output layout (fc_full_ladder.cu)
+template <int L>
+__global__ void __launch_bounds__(128) full_tp_zrow_kernel(int N, int C, const float* __restrict__ phi,
+                                                           const float* __restrict__ A,
+                                                           float* __restrict__ Bz) {
+  using TP = LadderTP<L>;
+  const int k = blockIdx.y * blockDim.x + threadIdx.x;
+  if (k >= C) return;
+  const int n0 = blockIdx.x * kVChunk;
+  const int n1 = min(N, n0 + kVChunk);
+  for (int n = n0; n < n1; ++n) {
+    const size_t base = (size_t)n * TP::NY * C + k;
+    float a[TP::NY], b[TP::NY];
+#pragma unroll
+    for (int i = 0; i < TP::NY; ++i) {
+      a[i] = __ldg(phi + base + (size_t)i * C);
+      b[i] = __ldg(A + base + (size_t)i * C);
+    }
+    TP::fwd_paths(a, b, Bz + (size_t)n * TP::ZROW * C + k, C);
+  }
+}
+
+int full_tp_zrow_dispatch(int L, int N, int C, const float* phi, const float* A, float* Bz,
+                          cudaStream_t s) {
+  dim3 grid((N + kVChunk - 1) / kVChunk, (C + 127) / 128);
+  switch (L) {
+    case 1: full_tp_zrow_kernel<1><<<grid, 128, 0, s>>>(N, C, phi, A, Bz); break;
+    case 2: full_tp_zrow_kernel<2><<<grid, 128, 0, s>>>(N, C, phi, A, Bz); break;
+    case 3: full_tp_zrow_kernel<3><<<grid, 128, 0, s>>>(N, C, phi, A, Bz); break;
+    case 4: full_tp_zrow_kernel<4><<<grid, 128, 0, s>>>(N, C, phi, A, Bz); break;
+    default: return FC_ERR_UNSUPPORTED_RANK;
+  }
+  return cudaGetLastError() == cudaSuccess ? FC_OK : FC_ERR_CUDA;
+}
+
+void rank_path_counts(int L, int* Pl) {
+  for (int l3 = 0; l3 <= L; ++l3) {
+    Pl[l3] = 0;
+    for (int l1 = 0; l1 <= L; ++l1)
+      for (int l2 = 0; l2 <= L; ++l2)
+        if (l3 >= (l1 > l2 ? l1 - l2 : l2 - l1) && l3 <= l1 + l2 && ((l1 + l2 + l3) & 1) == 0) ++Pl[l3];
+  }
+}
+
+RowLayout node_layout(int L) {
+  RowLayout g{};
+  g.stride = (L + 1) * (L + 1);
+  for (int l = 0; l <= L && l < 5; ++l) {
+    g.off[l] = l * l;
+    g.cmul[l] = 1;
+  }
+  return g;
+}
+
+RowLayout path_layout(int L, const int* Pl) {
+  RowLayout g{};
+  g.stride = out_row(L, 0);
+  int o = 0;
+  for (int l = 0; l <= L && l < 5; ++l) {
+    g.off[l] = o;
+    g.cmul[l] = Pl[l];
+    o += (2 * l + 1) * Pl[l];
+  }
+  return g;
+}
+
+template <bool ACC>
+int launch_rows_gemm(int N, int C, int L, const RowLayout& ai, const RowLayout& ao, const float* in,
+                     const float* Bm, const long long* boff, float* out, cudaStream_t s) {
+  int wmax = 0;
+  for (int l = 0; l <= L; ++l) wmax = ao.wid[l] > wmax ? ao.wid[l] : wmax;
+  const int Rmax = N * (2 * L + 1);
+  dim3 grid((Rmax + kVBM - 1) / kVBM, (wmax + kVBN - 1) / kVBN, L + 1);
+  rows_gemm_kernel<ACC><<<grid, 256, 0, s>>>(N, C, L, ai, ao, in, Bm, boff[0], boff[1],
+                                             boff[2], boff[3], boff[4], out);
+  return cudaGetLastError() == cudaSuccess ? FC_OK : FC_ERR_CUDA;
+}
+
+int launch_rows_wgrad(int N, int C, int L, const RowLayout& la, const RowLayout& lb, const float* a,
+                      const float* b, float* Wb, const long long* woff, cudaStream_t s) {
+  int wmax = 0;
+  for (int l = 0; l <= L; ++l) wmax = lb.wid[l] > wmax ? lb.wid[l] : wmax;
+  const int Rmax = N * (2 * L + 1);
+  const int tiles = ((C + kVBM - 1) / kVBM) * ((wmax + kVBN - 1) / kVBN);
+  dim3 grid((Rmax + kVRows - 1) / kVRows, tiles, L + 1);
+  rows_wgrad_kernel<<<grid, 256, 0, s>>>(N, C, L, la, lb, a, b, Wb, woff[0], woff[1], woff[2],
+                                         woff[3], woff[4]);
+  return cudaGetLastError() == cudaSuccess ? FC_OK : FC_ERR_CUDA;
+}
+
+int check_full_vjp_desc(const fc_ladder_desc* d) {
+  if (!d) return FC_ERR_ARG;
+  if (d->channels <= 0 || d->order < 1 || d->lmax < 0) return FC_ERR_ARG;
+  if (d->lmax < 1 || d->lmax > 4) return FC_ERR_UNSUPPORTED_RANK;
+  if (d->channels % 4) return FC_ERR_ALIGN;
+  return FC_OK;
+}
+
+}  // namespace
+}  // namespace fc
+
+using namespace fc;
+
+extern "C" size_t fc_full_ladder_vjp_workspace_size(const fc_ladder_desc* d, int n_nodes) {
+  if (check_full_vjp_desc(d) != FC_OK || n_nodes < 0) return 0;
+  const size_t plane = (size_t)n_nodes * (d->lmax + 1) * (d->lmax + 1) * d->channels;
+  const size_t zplane = (size_t)n_nodes * out_row(d->lmax, 0) * d->channels;
+  // two running gradients; one step's products and their gradient
+  return sizeof(float) * (2 * plane + (d->order > 1 ? 2 * zplane : 0));
+}
+
+extern "C" int fc_full_ladder_vjp(const fc_ladder_desc* d, int n_nodes, const float* A, const float* W1,
+                                  const float* Wq, const float* states, const float* gz, float* A_bar,
+                                  float* W1_bar, float* Wq_bar, void* workspace, size_t ws_bytes,
+                                  fc_stream_t stream) {
+  int st = check_full_vjp_desc(d);
+  if (st != FC_OK) return st;
+  if (n_nodes < 0) return FC_ERR_ARG;
+  const int L = d->lmax, C = d->channels, order = d->order;
+  if (!W1 || !W1_bar || (order > 1 && (!Wq || !Wq_bar))) return FC_ERR_ARG;
+  if (!aligned16(W1) || !aligned16(W1_bar) || (order > 1 && (!aligned16(Wq) || !aligned16(Wq_bar))))
+    return FC_ERR_ALIGN;
+  const int P = num_paths(L);
+  cudaStream_t s = (cudaStream_t)stream;
+  if (cudaMemsetAsync(W1_bar, 0, sizeof(float) * (size_t)(L + 1) * C * C, s) != cudaSuccess ||
+      (order > 1 &&
+       cudaMemsetAsync(Wq_bar, 0, sizeof(float) * (size_t)(order - 1) * C * P * C, s) != cudaSuccess))
+    return FC_ERR_CUDA;
+  if (n_nodes == 0) return FC_OK;
+  if (!A || !states || !gz || !A_bar) return FC_ERR_ARG;
+  if (!aligned16(A) || !aligned16(states) || !aligned16(gz) || !aligned16(A_bar)) return FC_ERR_ALIGN;
+  const size_t need = fc_full_ladder_vjp_workspace_size(d, n_nodes);
+  if (!workspace || ws_bytes < need) return FC_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return FC_ERR_ALIGN;
+
+  const int NY = (L + 1) * (L + 1);
+  const size_t plane = (size_t)n_nodes * NY * C;
+  const size_t zplane = (size_t)n_nodes * out_row(L, 0) * C;
+  float* pb = static_cast<float*>(workspace);
+  float* pbn = pb + plane;
+  float* Bq = pbn + plane;
+  float* Bbar = Bq + zplane;
+  int Pl[6] = {0, 0, 0, 0, 0, 0};
+  rank_path_counts(L, Pl);
+  RowLayout nl = node_layout(L), pl = path_layout(L, Pl);
+  for (int l = 0; l <= L; ++l) {
+    nl.wid[l] = C;
+    pl.wid[l] = Pl[l] * C;
+  }
+  // per-rank offsets of the [C][P_l C] blocks of one step's map, and of W1's [C][C]
+  long long qoff[5] = {0, 0, 0, 0, 0}, w1off[5] = {0, 0, 0, 0, 0};
+  {
+    long long o = 0;
+    for (int l = 0; l <= L; ++l) {
+      qoff[l] = o;
+      o += (long long)C * Pl[l] * C;
+      w1off[l] = (long long)l * C * C;
+    }
+  }
+  if (cudaMemsetAsync(A_bar, 0, sizeof(float) * plane, s) != cudaSuccess ||
+      cudaMemcpyAsync(pb, gz, sizeof(float) * plane, cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+    return FC_ERR_CUDA;
+  const size_t wq_step = (size_t)C * P * C;
+  for (int q = order; q >= 2; --q) {
+    const float* phi_prev = states + (size_t)(q - 2) * plane;
+    const float* Wqq = Wq + (size_t)(q - 2) * wq_step;
+    float* Wqb = Wq_bar + (size_t)(q - 2) * wq_step;
+    if ((st = full_tp_zrow_dispatch(L, n_nodes, C, phi_prev, A, Bq, s)) != FC_OK ||
+        (st = launch_rows_wgrad(n_nodes, C, L, nl, pl, pb, Bq, Wqb, qoff, s)) != FC_OK ||
+        (st = launch_rows_gemm<false>(n_nodes, C, L, nl, pl, pb, Wqq, qoff, Bbar, s)) != FC_OK ||
+        (st = full_tp_vjp_dispatch(L, n_nodes, C, phi_prev, A, Bbar, gz, pbn, A_bar, s)) != FC_OK)
+      return st;
+    float* t = pb;
+    pb = pbn;
+    pbn = t;
+  }
+  // the first map: W1_bar_l += pbar^T A, A_bar += pbar W1_l
+  if ((st = launch_rows_wgrad(n_nodes, C, L, nl, nl, pb, A, W1_bar, w1off, s)) != FC_OK ||
+      (st = launch_rows_gemm<true>(n_nodes, C, L, nl, nl, pb, W1, w1off, A_bar, s)) != FC_OK)
+    return st;
+  return FC_OK;
+}

@@ -73,6 +73,9 @@ _SIGS = {
     "fc_full_ladder_workspace_size": (ct.c_size_t, [ct.POINTER(LadderDesc), ct.c_int]),
     "fc_full_ladder": (ct.c_int, [ct.POINTER(LadderDesc), ct.c_int, _vp, _vp, _vp, _vp, _vp, _vp,
                                   ct.c_size_t, _vp]),
+    "fc_full_ladder_vjp_workspace_size": (ct.c_size_t, [ct.POINTER(LadderDesc), ct.c_int]),
+    "fc_full_ladder_vjp": (ct.c_int, [ct.POINTER(LadderDesc), ct.c_int] + [_vp] * 9
+                           + [ct.c_size_t, _vp]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _f = getattr(_lib, _name)
@@ -344,6 +347,31 @@ def full_ladder(lmax, order, A, W1, Wq, workspace=None, stream=None):
                                ws_bytes if workspace is not None else 0, _stream(stream)),
            "fc_full_ladder")
     return states, z
+
+
+def full_ladder_vjp(lmax, order, A, W1, Wq, states, gz, workspace=None, stream=None):
+    """(A_bar, W1_bar, Wq_bar): gradients of <gz, z> for fc_full_ladder,
+    given the states phi_1..phi_order it returned."""
+    for t, n in ((A, "A"), (W1, "W1"), (states, "states"), (gz, "gz")):
+        _dev(t, torch.float32, n)
+    N = A.shape[0]
+    NY = (lmax + 1) ** 2
+    C = A.shape[1] // NY
+    d = LadderDesc(lmax, C, order)
+    Ab = torch.empty_like(A)
+    W1b = torch.empty_like(W1)
+    if order > 1:
+        _dev(Wq, torch.float32, "Wq")
+        Wqb = torch.empty_like(Wq)
+    else:
+        Wqb = None
+    ws_bytes = _lib.fc_full_ladder_vjp_workspace_size(ct.byref(d), N)
+    workspace, ws_bytes = _scratch(workspace, ws_bytes, A.device)
+    _check(_lib.fc_full_ladder_vjp(ct.byref(d), N, _ptr(A), _ptr(W1), _ptr(Wq) if order > 1 else None,
+                                   _ptr(states), _ptr(gz), _ptr(Ab), _ptr(W1b), _ptr(Wqb),
+                                   _ptr(workspace), ws_bytes if workspace is not None else 0,
+                                   _stream(stream)), "fc_full_ladder_vjp")
+    return Ab, W1b, Wqb
 
 
 def device_error(stream=None):

@@ -1108,6 +1108,28 @@ def emit_ladder(L):
                 o.append("      bbar[%d] = fmaf(w[%d], %s, bbar[%d]);" % (l2 * l2 + b2, p, " + ".join(t), l2 * l2 + b2))
         o.append("    }")
     o.append("  }")
+    # full ladder VJP: every path has its own output gradient, get(l3, c, eta)
+    o.append("  template <class Get>")
+    o.append("  static __device__ __forceinline__ void vjp_paths(const float (&a)[NY], const float (&b)[NY], Get&& get,")
+    o.append("                                                   float (&abar)[NY], float (&bbar)[NY]) {")
+    for p, (l1, l2, l3) in enumerate(T.paths):
+        K = T.K[p]
+        o.append("    { // path (%d,%d)->%d" % (l1, l2, l3))
+        o.append("      float g[%d];" % (2 * l3 + 1))
+        for c in range(2 * l3 + 1):
+            o.append("      g[%d] = get(%d, %d, %d);" % (c, l3, c, T.eta[p]))
+        for b1 in range(2 * l1 + 1):
+            t = ["%s*(g[%d]*b[%d])" % (flit(K[c][b1][b2]), c, l2 * l2 + b2)
+                 for c in range(2 * l3 + 1) for b2 in range(2 * l2 + 1) if K[c][b1][b2] != 0]
+            if t:
+                o.append("      abar[%d] += %s;" % (l1 * l1 + b1, " + ".join(t)))
+        for b2 in range(2 * l2 + 1):
+            t = ["%s*(g[%d]*a[%d])" % (flit(K[c][b1][b2]), c, l1 * l1 + b1)
+                 for c in range(2 * l3 + 1) for b1 in range(2 * l1 + 1) if K[c][b1][b2] != 0]
+            if t:
+                o.append("      bbar[%d] += %s;" % (l2 * l2 + b2, " + ".join(t)))
+        o.append("    }")
+    o.append("  }")
     o.append("};")
     o.append("}  // namespace fc")
     return "\n".join(o) + "\n"

@@ -325,6 +325,30 @@ int fc_full_ladder(const fc_ladder_desc *desc, int n_nodes, const float *A,
                    const float *W1, const float *Wq, float *states, float *z,
                    void *workspace, size_t ws_bytes, fc_stream_t stream);
 
+/* VJP of fc_full_ladder by reverse accumulation through its steps (Sec. 5
+ * Eq. (2); each bilinear product differentiated as in App. C Eq. (C1)):
+ * given gz (gradient of z) and the states phi_1 .. phi_order of the forward
+ * call, writes the gradients of <gz, z>
+ *   A_bar [n_nodes][(lmax+1)^2 C], W1_bar like W1 ([lmax+1][C][C]),
+ *   Wq_bar like Wq ([order-1][C P C]; unused for order 1).
+ * Going down from q = order, the running gradient pbar of phi_q (gz plus
+ * what step q+1 sends back) gives Wq_bar_l += pbar^T B_q and
+ * Bbar_q = pbar Wq_l per rank, and the product VJP of B_q = f(phi_{q-1}, A)
+ * sends Bbar_q to phi_{q-1} and A; the first map gives W1_bar_l += pbar^T A
+ * and A_bar += pbar W1_l.  B_q is recomputed from the saved phi_{q-1}.
+ * Outputs are overwritten; the weight gradients sum over all nodes with
+ * atomic additions (not bitwise reproducible).  FP32 throughout.
+ * workspace: fc_full_ladder_vjp_workspace_size() bytes (two node-layout
+ * gradients plus one step's path-separated product and its gradient,
+ * n_nodes x fc_conv_out_row x C floats each), 16-byte aligned; ws_bytes its
+ * real size, FC_ERR_WORKSPACE if smaller.  Returns the statuses of
+ * fc_full_ladder. */
+size_t fc_full_ladder_vjp_workspace_size(const fc_ladder_desc *desc, int n_nodes);
+int fc_full_ladder_vjp(const fc_ladder_desc *desc, int n_nodes, const float *A,
+                       const float *W1, const float *Wq, const float *states,
+                       const float *gz, float *A_bar, float *W1_bar, float *Wq_bar,
+                       void *workspace, size_t ws_bytes, fc_stream_t stream);
+
 /* Sticky device-side error word of the kernels that wait on barriers (the
  * tensor-core mixes and maps of the ladders): each wait gives up after a
  * bounded time (fc_set_wait_timeout), skips the rest of its CTA's work --
