@@ -10,10 +10,11 @@ and its fraction of the HBM roofline.
 
 One step = one fc_edge_conv call over the whole graph with inputs resident
 in HBM.  The 1.54 GB weight tensor is larger than the 126 MB L2, so no L2
-flush is needed between steps.  Under torchrun (N > 1) every rank runs its
-own copy of the workload (weak scaling, no collective on the data path);
-time is the max over ranks.  --impl reference times the FP64 CPU oracle on a
+flush is needed between steps.  Time is the max over ranks.  --impl reference times the FP64 CPU oracle on a
 bounded sample of the same workload (rank 0 only).
+Under torchrun the ranks share ONE graph of N x 1024 nodes, cut by receiver
+range (cartesian_tensor_products_b200/shard.py): each step all-gathers the
+node features over NCCL and convolves the rank's own 1024 receivers.
 """
 import argparse
 import ctypes
@@ -222,6 +223,29 @@ def composite_bound(peaks, fp32_peak, byts, fp32_fl, tf32_fl, ms, algo_flops):
             "algorithmic_flops": algo_flops, "algorithmic_bytes": byts}
 
 
+def oracle_row(fn, units, unit, sample):
+    """The FP64 oracle timed once on a bounded sample of a row's workload
+    (host cores of this machine): units processed per second."""
+    from oracle import oracle as O
+    t0 = time.perf_counter()
+    fn()
+    dt = time.perf_counter() - t0
+    return {"value": units / dt, "unit": unit, "cores": O.num_threads(), "kind": "oracle",
+            "sample": sample, "seconds": dt}
+
+
+def peak_alloc(fn):
+    """Device memory the call adds at its peak (torch allocator: outputs and
+    workspace the binding allocates; the library itself allocates nothing)."""
+    import torch
+    torch.cuda.synchronize()
+    base = torch.cuda.memory_allocated()
+    torch.cuda.reset_peak_memory_stats()
+    fn()
+    torch.cuda.synchronize()
+    return torch.cuda.max_memory_allocated() - base
+
+
 def time_events(fn, steps, warmup, stream, flush=None):
     """Mean device time (ms) of fn over `steps` calls, CUDA events on the
     launching stream; optional L2 flush before every call (not timed)."""
@@ -278,8 +302,18 @@ def extra_rows(fc, W, dev, stream, peaks, fp32_peak, steps, select=ROW_NAMES):
                              steps, 3, stream)
         zr = fc.out_row(L)
         byt = 4 * (2 * E * P * C + N * zr * C + 2 * N * 16 * C + 3 * E + 3 * E + E + N)
+        from oracle import oracle as O
+        m4 = np.zeros(N, np.uint8)
+        m4[:4] = 1
+        em = m4[wl["edge_index"][0]]
+        cb = oracle_row(lambda: O.edge_conv_vjp(L, L, L, C, wl["edge_index"], wl["edge_vec"], wl["x"],
+                                                wl["w"], wl["g"] * m4[:, None], N, edge_mask=em),
+                        int(em.sum()) * C, "edge*channel/s",
+                        "edges of the first 4 receivers (%d x %d channels), FP64 oracle" % (em.sum(), C))
         rows["edge_conv_vjp_r3"] = {
             "workload": "microbench graph, rank 3, x_bar + w_bar + r_bar",
+            "cpu_baseline": cb,
+            "peak_alloc_bytes": peak_alloc(lambda: fc.edge_conv_vjp(L, rp, ei, ev, x, w, g)),
             "ms": ms, "ms_min": mn, "edge_channels_per_s": E * C / (ms * 1e-3),
             "roofline": {"bound": "hbm", "achieved": byt / (ms * 1e-3) / 1e9,
                          "peak": peaks["hbm_gbs"], "unit": "GB/s",
@@ -304,8 +338,20 @@ def extra_rows(fc, W, dev, stream, peaks, fp32_peak, steps, select=ROW_NAMES):
         # w, vw in; w_hat out; x, vx, g in; g_hat, x_hat out (+ zeroing); edges
         byt = 4 * (3 * E * P * C + 2 * N * 16 * C + 2 * N * zr * C + N * 16 * C
                    + 3 * E * 3 + E + N)
+        from oracle import oracle as O
+        m2 = np.zeros(N, np.uint8)
+        m2[:2] = 1
+        em = m2[wl["edge_index"][0]]
+        cb = oracle_row(lambda: O.edge_conv_vjp_vjp(3, 3, 3, C, wl["edge_index"], wl["edge_vec"], wl["x"],
+                                                    wl["w"], wl["g"] * m2[:, None], cot["vx"], cot["vw"],
+                                                    cot["vr"], N, edge_mask=em),
+                        int(em.sum()) * C, "edge*channel/s",
+                        "edges of the first 2 receivers (%d x %d channels), FP64 oracle" % (em.sum(), C))
         rows["edge_conv_vvjp_r3"] = {
             "workload": "microbench graph, rank 3, g_hat + x_hat + w_hat + r_hat from vx, vw, vr",
+            "cpu_baseline": cb,
+            "peak_alloc_bytes": peak_alloc(lambda: fc.edge_conv_vjp_vjp(L, rp, ei, ev, x, w, g, v_x=vx,
+                                                                        v_w=vw, v_r=vr)),
             "ms": ms, "ms_min": mn, "edge_channels_per_s": E * C / (ms * 1e-3),
             "roofline": {"bound": "hbm", "achieved": byt / (ms * 1e-3) / 1e9,
                          "peak": peaks["hbm_gbs"], "unit": "GB/s",
@@ -381,9 +427,21 @@ def extra_rows(fc, W, dev, stream, peaks, fp32_peak, steps, select=ROW_NAMES):
 
         def bound(byts, fp32_fl, tf32_fl, ms):
             return composite_bound(peaks, fp32_peak, byts, fp32_fl, tf32_fl, ms, mix_flops + tp_flops)
+        from oracle import oracle as O
+        ns = 64
+        lm = np.zeros(Nl, np.uint8)
+        lm[:ns] = 1
+        cbf = oracle_row(lambda: O.ladder(Ll, Cl, order, lad["A1"], lad["path_w"], lad["mix_w"], node_mask=lm),
+                         ns, "nodes/s", "first %d nodes, FP64 oracle" % ns)
+        cbv = oracle_row(lambda: O.ladder_vjp(Ll, Cl, order, lad["A1"], lad["path_w"], lad["mix_w"],
+                                              lad["gz"] * lm[:, None], node_mask=lm),
+                         ns, "nodes/s", "first %d nodes, FP64 oracle" % ns)
+        pa_f = peak_alloc(lambda: fc.product_ladder(Ll, order, A1, pw, mw))
+        pa_v = peak_alloc(lambda: fc.product_ladder_vjp(Ll, order, A1, pw, mw, states, gz))
         # forward: A1 read, states written, z written; products FP32; mix TF32 x3 (or FP32)
         fb = plane_b * (1 + S + 1)
         rows["ladder_fwd"] = {
+            "nodes_per_s": Nl / (msl * 1e-3), "cpu_baseline": cbf, "peak_alloc_bytes": pa_f,
             "workload": "4096 nodes x 128 channels, rank 3, order 4 (3 products + 3 per-rank 128x128 mixes)",
             "ms": msl, "ms_min": mnl,
             "roofline": bound(fb, tp_flops + (0 if tc else mix_flops), 3 * mix_flops if tc else 0, msl),
@@ -393,6 +451,7 @@ def extra_rows(fc, W, dev, stream, peaks, fp32_peak, steps, select=ROW_NAMES):
         # on the tensor cores at C = 128 (three TF32 products each), else FP32
         vb = plane_b * (1 + S + 1 + 1)
         rows["ladder_vjp"] = {
+            "nodes_per_s": Nl / (mslb * 1e-3), "cpu_baseline": cbv, "peak_alloc_bytes": pa_v,
             "workload": "same ladder, A1_bar + path_w_bar + mix_w_bar",
             "ms": mslb, "ms_min": mnlb,
             "roofline": bound(vb, 4 * tp_flops + (0 if tc else 2 * mix_flops),
@@ -419,7 +478,18 @@ def extra_rows(fc, W, dev, stream, peaks, fp32_peak, steps, select=ROW_NAMES):
         tp_fl = (of - 1) * Nf * Cf * 2 * 751
         # A read, order states and z written; products FP32; maps TF32 x3 on the tensor cores
         fbf = 4 * Nf * 16 * Cf * (1 + of + 1)
+        from oracle import oracle as O
+        ns = 16
+        fm = np.zeros(Nf, np.uint8)
+        fm[:ns] = 1
+        cbff = oracle_row(lambda: O.full_ladder(Lf, Cf, of, fd["A"], fd["W1"], fd["Wq"], node_mask=fm),
+                          ns, "nodes/s", "first %d nodes, FP64 oracle" % ns)
+        cbfv = oracle_row(lambda: O.full_ladder_vjp(Lf, Cf, of, fd["A"], fd["W1"], fd["Wq"],
+                                                    fd["gz"] * fm[:, None], node_mask=fm),
+                          ns, "nodes/s", "first %d nodes, FP64 oracle" % ns)
         rows["full_ladder_fwd"] = {
+            "nodes_per_s": Nf / (msf * 1e-3), "cpu_baseline": cbff,
+            "peak_alloc_bytes": peak_alloc(lambda: fc.full_ladder(Lf, of, A, W1, Wq)),
             "workload": "4096 nodes x 128 channels, rank 3, order 4: path-separated products, "
                         "per-rank (P_l x 128) -> 128 maps on tcgen05 (three-term TF32)",
             "ms": msf, "ms_min": mnf,
@@ -437,6 +507,8 @@ def extra_rows(fc, W, dev, stream, peaks, fp32_peak, steps, select=ROW_NAMES):
                                steps, 3, stream, flush=flush)
         vbf = 4 * Nf * 16 * Cf * (1 + (of - 1) + 1 + 1)
         rows["full_ladder_vjp"] = {
+            "nodes_per_s": Nf / (msv * 1e-3), "cpu_baseline": cbfv,
+            "peak_alloc_bytes": peak_alloc(lambda: fc.full_ladder_vjp(Lf, of, A, W1, Wq, st_f, gzf)),
             "workload": "same full ladder, A_bar + W1_bar + Wq_bar (maps and their gradients FP32 SIMT)",
             "ms": msv, "ms_min": mnv,
             "roofline": composite_bound(peaks, fp32_peak, vbf, 2 * mix_fl + 3 * tp_fl, 0, msv,
@@ -460,7 +532,19 @@ def extra_rows(fc, W, dev, stream, peaks, fp32_peak, steps, select=ROW_NAMES):
                                                             dom, dpw, dmw, dm["cutoff"],
                                                             dm["edge_scale"]),
                                steps, 3, stream, flush=flush)
+        from oracle import oracle as O
+        bm = np.zeros(Nd, np.uint8)
+        bm[:2] = 1
+        cbb = oracle_row(lambda: O.block_energy_forces(dm["lmax"], dm["channels"], dm["order"],
+                                                       dm["edge_index"], dm["edge_vec"], dm["x"],
+                                                       dm["omega"], dm["path_w"], dm["mix_w"], Nd,
+                                                       dm["cutoff"], dm["edge_scale"], recv_mask=bm),
+                         2, "atoms/s", "energies and incoming-edge gradients of the first 2 atoms, "
+                         "FP64 oracle")
         rows["block_energy_forces"] = {
+            "atoms_per_s": Nd / (msb * 1e-3), "cpu_baseline": cbb,
+            "peak_alloc_bytes": peak_alloc(lambda: fc.interaction_block(
+                dm["lmax"], dm["order"], drp, dei, dev_, dx, dom, dpw, dmw, dm["cutoff"], dm["edge_scale"])),
             "workload": "1000-atom diamond (5x5x5 cells, a = 3.567 A, 5 A cutoff, %d edges), C=128, rank 3: "
                         "enveloped conv (paths summed) + order-5 ladder + E + ladder VJP + conv VJP + forces" % Ed,
             "ms": msb, "ms_min": mnb, "us_per_atom": 1e3 * msb / Nd,
@@ -512,23 +596,58 @@ def run_ours(args):
     from cartesian_tensor_products_b200 import flashcart as fc
     from cartesian_tensor_products_b200 import workloads as W
 
-    wl = W.microbench(seed=rank_graph_seed(rank))
-    L, C, N = wl["lmax"], wl["channels"], wl["n_nodes"]
-    E = wl["edge_index"].shape[1]
+    stream = torch.cuda.current_stream()
+    sh = None
+    if world == 1:
+        wl = W.microbench(seed=rank_graph_seed(rank))
+        h_ei, h_ev, h_x, h_w = wl["edge_index"], wl["edge_vec"], wl["x"], wl["w"]
+        N = N_send = wl["n_nodes"]
+    else:
+        # one graph of world x 1024 nodes cut by receiver range: this rank's
+        # 1024 receivers take their 128 senders from all nodes; the step
+        # all-gathers the node features, then convolves the local edges
+        from cartesian_tensor_products_b200 import shard
+        wl = W.sharded_microbench(rank, world)
+        sh = shard.GraphShard(wl["edge_index"], wl["n_nodes"], rank, world, bounds=wl["bounds"])
+        h_ei, h_ev, h_x, h_w = sh.edge_index, wl["edge_vec_local"], wl["x_local"], wl["w_local"]
+        N, N_send = sh.n_local, wl["n_nodes"]
+    L, C = wl["lmax"], wl["channels"]
+    E = h_ei.shape[1]
     P = fc.num_paths(L)
     zrow = fc.out_row(L)
-    stream = torch.cuda.current_stream()
 
     # ---- inputs resident in HBM
-    ei = torch.from_numpy(wl["edge_index"]).to(dev)
-    ev = torch.from_numpy(wl["edge_vec"]).to(dev)
-    x = torch.from_numpy(wl["x"]).to(dev)
-    w = torch.from_numpy(wl["w"]).to(dev)
-    rowptr = fc.build_rowptr(ei, ev, N)
+    ei = torch.from_numpy(h_ei).to(dev)
+    ev = torch.from_numpy(h_ev).to(dev)
+    x = torch.from_numpy(h_x).to(dev)
+    w = torch.from_numpy(h_w).to(dev)
+    rowptr = fc.build_rowptr(ei, ev, N, n_send=N_send)
     z = torch.empty((N, zrow * C), dtype=torch.float32, device=dev)
+    x_all = torch.empty((N_send, x.shape[1]), dtype=torch.float32, device=dev) if sh else x
+    # receiver row pointer and graph validation, timed on its own (it reads
+    # its verdict back, so it synchronises)
+    torch.cuda.synchronize()
+    csr0 = torch.cuda.Event(enable_timing=True)
+    csr1 = torch.cuda.Event(enable_timing=True)
+    csr0.record(stream)
+    for _ in range(5):
+        fc.build_rowptr(ei, ev, N, n_send=N_send)
+    csr1.record(stream)
+    csr1.synchronize()
+    csr_ms = csr0.elapsed_time(csr1) / 5
+    conv_peak = peak_alloc(lambda: fc.edge_conv(L, rowptr, ei, ev, x_all, w))
+    k_start = torch.cuda.Event(enable_timing=True)
+    k_end = torch.cuda.Event(enable_timing=True)
+    k_ms = []
 
-    def step():
-        fc.edge_conv(L, rowptr, ei, ev, x, w, out=z)
+    def step(timed=False):
+        if sh is not None:
+            sh.gather_rows(x, out=x_all)
+        if timed:
+            k_start.record(stream)
+        fc.edge_conv(L, rowptr, ei, ev, x_all, w, out=z)
+        if timed:
+            k_end.record(stream)
 
     for _ in range(max(args.warmup, 3)):
         step()
@@ -554,6 +673,12 @@ def run_ours(args):
         ev_end[i].record(stream)
     t_all1.record(stream)
     torch.cuda.synchronize()
+    if sh is not None:
+        # the convolution kernel alone (the steps above include the all-gather)
+        for _ in range(args.steps):
+            step(timed=True)
+            k_end.synchronize()
+            k_ms.append(k_start.elapsed_time(k_end))
     if world > 1:
         dist.barrier()
     clocks = sampler.stop()
@@ -566,7 +691,7 @@ def run_ours(args):
     # ---- roofline of the (single) kernel of the step
     peaks, peak_kind = load_peaks()
     abytes = algorithmic_bytes(N, E, C, L, P, zrow)
-    kern_ms = statistics.mean(per)
+    kern_ms = statistics.mean(k_ms if k_ms else per)
     achieved_gbs = abytes / (kern_ms * 1e-3) / 1e9
     flops = algorithmic_flops(E, C, L)
     sm_count = props.multi_processor_count
@@ -588,10 +713,10 @@ def run_ours(args):
     # ---- end to end through the C ABI from pinned host buffers
     e2e = None
     if not args.no_e2e:
-        hx = torch.from_numpy(wl["x"]).pin_memory()
-        hw = torch.from_numpy(wl["w"]).pin_memory()
-        hei = torch.from_numpy(wl["edge_index"]).pin_memory()
-        hev = torch.from_numpy(wl["edge_vec"]).pin_memory()
+        hx = torch.from_numpy(h_x).pin_memory()
+        hw = torch.from_numpy(h_w).pin_memory()
+        hei = torch.from_numpy(h_ei).pin_memory()
+        hev = torch.from_numpy(h_ev).pin_memory()
         hz = torch.empty((N, zrow * C), dtype=torch.float32).pin_memory()
         dx, dw = torch.empty_like(x), torch.empty_like(w)
         dei, dev_ = torch.empty_like(ei), torch.empty_like(ev)
@@ -603,8 +728,9 @@ def run_ours(args):
             dw.copy_(hw, non_blocking=True)
             dei.copy_(hei, non_blocking=True)
             dev_.copy_(hev, non_blocking=True)
-            rp = fc.build_rowptr(dei, dev_, N)
-            fc.edge_conv(L, rp, dei, dev_, dx, dw, out=z)
+            rp = fc.build_rowptr(dei, dev_, N, n_send=N_send)
+            xa = sh.gather_rows(dx, out=x_all) if sh is not None else dx
+            fc.edge_conv(L, rp, dei, dev_, xa, dw, out=z)
             hz.copy_(z, non_blocking=True)
         e2e_step()
         torch.cuda.synchronize()
@@ -623,7 +749,9 @@ def run_ours(args):
         e2e = {"value": weak_throughput(world, E * C, n_e2e, e_ms), "unit": UNIT,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "steps": n_e2e, "ms_per_step": e_ms / n_e2e,
-               "includes": "H2D of x, w, edge_index, edge_vec; fc_build_rowptr (validates, syncs); fc_edge_conv; D2H of z"}
+               "includes": "H2D of x, w, edge_index, edge_vec; fc_build_rowptr (validates, syncs); "
+                           + ("all-gather of x; " if sh is not None else "")
+                           + "fc_edge_conv; D2H of z"}
 
     rows = None
     if world == 1 and not args.no_rows:
@@ -644,9 +772,13 @@ def run_ours(args):
                 "config": {"workload": WORKLOAD, "n_nodes": N, "n_edges": E,
                            "channels": C, "lmax": L, "paths": P,
                            "l2_flush": "none: the 1.54 GB weight stream exceeds the 126 MB L2",
-                           "per_rank": "each rank runs its own copy (weak scaling)"},
+                           "per_rank": ("one graph of %d nodes cut by receiver range: per step an "
+                                        "NCCL all-gather of the node features, then this rank's "
+                                        "1024 receivers (weak scaling)" % N_send) if sh is not None
+                           else "the whole graph on one GPU"},
                 "roofline": roof, "cpu_baseline": cb, "e2e": e2e,
                 "gpu_launches": args.steps, "clocks": clocks, "rows": rows,
+                "csr_build_ms": csr_ms, "peak_alloc_bytes": conv_peak,
                 "kernel_ms": {"mean": kern_ms, "min": min(per), "max": max(per)}}
         print(json.dumps(line), flush=True)
     if world > 1:

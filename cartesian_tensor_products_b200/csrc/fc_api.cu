@@ -69,7 +69,7 @@ enum : int { kBadRecv = 1, kUnsorted = 2, kBadSend = 4, kDegenerate = 8 };
 // Thread e (0 <= e <= E) validates edge e and fills the row pointers of the
 // receivers in (recv[e-1], recv[e]] with e (recv[-1] = -1, recv[E] = N),
 // so each entry of a valid receiver-sorted list is written exactly once.
-__global__ void build_rowptr_kernel(int N, int E, const int32_t* __restrict__ recv,
+__global__ void build_rowptr_kernel(int N, int NS, int E, const int32_t* __restrict__ recv,
                                     const int32_t* __restrict__ send,
                                     const float* __restrict__ vec,
                                     int32_t* __restrict__ rowptr, int32_t* __restrict__ flag) {
@@ -81,7 +81,7 @@ __global__ void build_rowptr_kernel(int N, int E, const int32_t* __restrict__ re
     cur = recv[e];
     if (cur < 0 || cur >= N) { bad |= kBadRecv; cur = cur < 0 ? 0 : N - 1; }
     const int s = send[e];
-    if (s < 0 || s >= N) bad |= kBadSend;
+    if (s < 0 || s >= NS) bad |= kBadSend;
     if (vec) {
       const float x = vec[3 * e], y = vec[3 * e + 1], z = vec[3 * e + 2];
       const float r2 = x * x + y * y + z * z;
@@ -175,10 +175,10 @@ int fc_edge_forces(int n_nodes, int n_edges, const int32_t* edge_index, const fl
   return cudaGetLastError() == cudaSuccess ? FC_OK : FC_ERR_CUDA;
 }
 
-int fc_build_rowptr(int n_nodes, int n_edges, const int32_t* edge_index,
-                    const float* edge_vec, int32_t* rowptr, int32_t* flag,
-                    fc_stream_t stream) {
-  if (n_nodes < 0 || n_edges < 0 || !rowptr || !flag) return FC_ERR_ARG;
+int fc_build_rowptr_rect(int n_nodes, int n_send, int n_edges, const int32_t* edge_index,
+                         const float* edge_vec, int32_t* rowptr, int32_t* flag,
+                         fc_stream_t stream) {
+  if (n_nodes < 0 || n_send < 0 || n_edges < 0 || !rowptr || !flag) return FC_ERR_ARG;
   if (n_edges > 0 && !edge_index) return FC_ERR_ARG;
   if (!aligned4(rowptr) || !aligned4(flag) || (edge_index && !aligned4(edge_index)) ||
       (edge_vec && !aligned4(edge_vec)))
@@ -193,7 +193,7 @@ int fc_build_rowptr(int n_nodes, int n_edges, const int32_t* edge_index,
     const int block = 256;
     const int grid = (int)((threads + block - 1) / block);
     build_rowptr_kernel<<<grid, block, 0, s>>>(
-        n_nodes, n_edges, edge_index, edge_index ? edge_index + n_edges : nullptr,
+        n_nodes, n_send, n_edges, edge_index, edge_index ? edge_index + n_edges : nullptr,
         edge_vec, rowptr, flag);
     if (cudaGetLastError() != cudaSuccess) return FC_ERR_CUDA;
   }
@@ -204,6 +204,12 @@ int fc_build_rowptr(int n_nodes, int n_edges, const int32_t* edge_index,
   if (h & (kBadRecv | kUnsorted | kBadSend)) return FC_ERR_CSR;
   if (h & kDegenerate) return FC_ERR_DEGENERATE_EDGE;
   return FC_OK;
+}
+
+int fc_build_rowptr(int n_nodes, int n_edges, const int32_t* edge_index,
+                    const float* edge_vec, int32_t* rowptr, int32_t* flag,
+                    fc_stream_t stream) {
+  return fc_build_rowptr_rect(n_nodes, n_nodes, n_edges, edge_index, edge_vec, rowptr, flag, stream);
 }
 
 }  // extern "C"

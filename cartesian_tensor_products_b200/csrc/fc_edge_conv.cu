@@ -14,13 +14,13 @@ int launch_fwd_rank5(const ConvArgs& a, cudaStream_t s);
 
 using namespace fc;
 
-extern "C" int fc_edge_conv(const fc_conv_desc* d, int n_nodes, int n_edges,
-                            const int32_t* rowptr, const int32_t* edge_index,
-                            const float* edge_vec, const float* x, const float* w, float* z,
-                            fc_stream_t stream) {
+extern "C" int fc_edge_conv_rect(const fc_conv_desc* d, int n_nodes, int n_send, int n_edges,
+                                 const int32_t* rowptr, const int32_t* edge_index,
+                                 const float* edge_vec, const float* x, const float* w, float* z,
+                                 fc_stream_t stream) {
   int st = check_conv_desc(d);
   if (st != FC_OK) return st;
-  if (n_nodes < 0 || n_edges < 0) return FC_ERR_ARG;
+  if (n_nodes < 0 || n_send < 0 || n_edges < 0) return FC_ERR_ARG;
   if (n_nodes == 0) return n_edges == 0 ? FC_OK : FC_ERR_ARG;
   if (!rowptr || !x || !z) return FC_ERR_ARG;
   if (n_edges > 0 && (!edge_index || !edge_vec || !w)) return FC_ERR_ARG;
@@ -37,6 +37,7 @@ extern "C" int fc_edge_conv(const fc_conv_desc* d, int n_nodes, int n_edges,
   a.w = w;
   a.z = z;
   a.n_nodes = n_nodes;
+  a.n_send = n_send;
   a.n_edges = n_edges;
   a.C = C;
   a.ntiles = (C + 127) / 128;
@@ -61,6 +62,14 @@ extern "C" int fc_edge_conv(const fc_conv_desc* d, int n_nodes, int n_edges,
     case 5: return launch_fwd_rank5(a, s);
     default: return FC_ERR_UNSUPPORTED_RANK;
   }
+}
+
+extern "C" int fc_edge_conv(const fc_conv_desc* d, int n_nodes, int n_edges,
+                            const int32_t* rowptr, const int32_t* edge_index,
+                            const float* edge_vec, const float* x, const float* w, float* z,
+                            fc_stream_t stream) {
+  return fc_edge_conv_rect(d, n_nodes, n_nodes, n_edges, rowptr, edge_index, edge_vec, x, w, z,
+                           stream);
 }
 
 extern "C" size_t fc_edge_conv_workspace_size(const fc_conv_desc* d, int n_nodes, int n_edges) {

@@ -34,6 +34,7 @@ struct ConvArgs {
   const float* w;
   float* z;
   int n_nodes, n_edges, C, ntiles, xrow, zrow, P, sum_paths;
+  int n_send;   // rows of x (senders index x); n_nodes = receivers = rows of rowptr - 1 and z
   int envelope;
   float r_cut, edge_scale;
 };
@@ -63,7 +64,7 @@ __device__ __forceinline__ EdgeWin load_win(const ConvArgs& a, int e, int e1) {
 template <class Grp>
 __device__ __forceinline__ void issue_edge(const ConvArgs& a, int C, float* st, int q, int v,
                                            int k0, bool act) {
-  const bool vok = act && v >= 0 && v < a.n_nodes;
+  const bool vok = act && v >= 0 && v < a.n_send;
   const int kk = act ? k0 : 0;
   const float* xv = a.x + (size_t)(vok ? v : 0) * a.xrow * C + kk;
   const float* we = a.w + (size_t)q * a.P * C + kk;

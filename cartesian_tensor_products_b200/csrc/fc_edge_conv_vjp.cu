@@ -14,14 +14,14 @@ int launch_vjp_rank5(const VjpArgs& a, cudaStream_t s);
 
 using namespace fc;
 
-extern "C" int fc_edge_conv_vjp(const fc_conv_desc* d, int n_nodes, int n_edges,
-                                const int32_t* rowptr, const int32_t* edge_index,
-                                const float* edge_vec, const float* x, const float* w,
-                                const float* g, float* x_bar, float* w_bar, float* r_bar,
-                                fc_stream_t stream) {
+extern "C" int fc_edge_conv_vjp_rect(const fc_conv_desc* d, int n_nodes, int n_send, int n_edges,
+                                     const int32_t* rowptr, const int32_t* edge_index,
+                                     const float* edge_vec, const float* x, const float* w,
+                                     const float* g, float* x_bar, float* w_bar, float* r_bar,
+                                     fc_stream_t stream) {
   int st = check_conv_desc(d);
   if (st != FC_OK) return st;
-  if (n_nodes < 0 || n_edges < 0) return FC_ERR_ARG;
+  if (n_nodes < 0 || n_send < 0 || n_edges < 0) return FC_ERR_ARG;
   if (n_nodes == 0) return n_edges == 0 ? FC_OK : FC_ERR_ARG;
   if (!rowptr || !x || !g) return FC_ERR_ARG;
   if (n_edges > 0 && (!edge_index || !edge_vec || !w)) return FC_ERR_ARG;
@@ -42,6 +42,7 @@ extern "C" int fc_edge_conv_vjp(const fc_conv_desc* d, int n_nodes, int n_edges,
   a.wbar = w_bar;
   a.rbar = r_bar;
   a.n_nodes = n_nodes;
+  a.n_send = n_send;
   a.n_edges = n_edges;
   a.C = C;
   a.ntiles = (C + 127) / 128;
@@ -54,7 +55,7 @@ extern "C" int fc_edge_conv_vjp(const fc_conv_desc* d, int n_nodes, int n_edges,
   a.edge_scale = d->edge_scale;
   if ((long long)n_nodes * a.ntiles > 0x7fffffffLL) return FC_ERR_ARG;
   cudaStream_t s = (cudaStream_t)stream;
-  if (x_bar && cudaMemsetAsync(x_bar, 0, sizeof(float) * (size_t)n_nodes * a.xrow * C, s) != cudaSuccess)
+  if (x_bar && cudaMemsetAsync(x_bar, 0, sizeof(float) * (size_t)n_send * a.xrow * C, s) != cudaSuccess)
     return FC_ERR_CUDA;
   if (r_bar && n_edges > 0 &&
       cudaMemsetAsync(r_bar, 0, sizeof(float) * 3 * (size_t)n_edges, s) != cudaSuccess)
@@ -69,4 +70,13 @@ extern "C" int fc_edge_conv_vjp(const fc_conv_desc* d, int n_nodes, int n_edges,
     case 5: return launch_vjp_rank5(a, s);
     default: return FC_ERR_UNSUPPORTED_RANK;
   }
+}
+
+extern "C" int fc_edge_conv_vjp(const fc_conv_desc* d, int n_nodes, int n_edges,
+                                const int32_t* rowptr, const int32_t* edge_index,
+                                const float* edge_vec, const float* x, const float* w,
+                                const float* g, float* x_bar, float* w_bar, float* r_bar,
+                                fc_stream_t stream) {
+  return fc_edge_conv_vjp_rect(d, n_nodes, n_nodes, n_edges, rowptr, edge_index, edge_vec, x, w, g,
+                               x_bar, w_bar, r_bar, stream);
 }

@@ -42,6 +42,7 @@ struct VjpArgs {
   float* wbar;
   float* rbar;
   int n_nodes, n_edges, C, ntiles, xrow, zrow, P, sum_paths;
+  int n_send;   // rows of x (senders index x); n_nodes = receivers = rows of rowptr - 1 and z
   int envelope;
   float r_cut, edge_scale;
 };
@@ -70,7 +71,7 @@ __device__ __forceinline__ VEdgeWin vload_win(const VjpArgs& a, int e, int e1) {
 template <class Grp>
 __device__ __forceinline__ void vissue_edge(const VjpArgs& a, int C, float* st, int q, int v,
                                             int k0, bool act) {
-  const bool vok = act && v >= 0 && v < a.n_nodes;
+  const bool vok = act && v >= 0 && v < a.n_send;
   const int kk = act ? k0 : 0;
   const float* xv = a.x + (size_t)(vok ? v : 0) * a.xrow * C + kk;
   const float* we = a.w + (size_t)q * a.P * C + kk;
@@ -147,7 +148,7 @@ __device__ __forceinline__ void vjp_warp(const VjpArgs& a, float* smem, int lane
               wbase + (wstore ? (size_t)q * a.P * C + k0 : 0), C, wstore);
     // sender gradient
     const int v = __shfl_sync(0xffffffffu, cur.v, p & 31);
-    if (a.xbar != nullptr && act && v >= 0 && v < a.n_nodes) {
+    if (a.xbar != nullptr && act && v >= 0 && v < a.n_send) {
       Grp::flush_xbar(a.xbar + (size_t)v * a.xrow * C + k0, C, xb);
     } else {
 #pragma unroll

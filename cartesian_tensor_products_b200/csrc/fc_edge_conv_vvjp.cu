@@ -47,6 +47,7 @@ extern "C" int fc_edge_conv_vjp_vjp(const fc_conv_desc* d, int n_nodes, int n_ed
   a.what = w_hat;
   a.rhat = r_hat;
   a.n_nodes = n_nodes;
+  a.n_send = n_nodes;
   a.n_edges = n_edges;
   a.C = C;
   a.ntiles = (C + 127) / 128;

@@ -49,6 +49,7 @@ struct VvjpArgs {
   float* what;
   float* rhat;
   int n_nodes, n_edges, C, ntiles, xrow, zrow, P, sum_paths;
+  int n_send;   // rows of x (senders index x); n_nodes = receivers = rows of rowptr - 1 and z
 };
 
 struct VvEdgeWin {
@@ -82,7 +83,7 @@ __device__ __forceinline__ VvEdgeWin vvload_win(const VvjpArgs& a, int e, int e1
 template <class Grp>
 __device__ __forceinline__ void vvissue_edge(const VvjpArgs& a, int C, float* st, int q, int v,
                                              int k0, bool act) {
-  const bool vok = act && v >= 0 && v < a.n_nodes;
+  const bool vok = act && v >= 0 && v < a.n_send;
   const int kk = act ? k0 : 0;
   const size_t xo = (size_t)(vok ? v : 0) * a.xrow * C + kk;
   const size_t wo = (size_t)q * a.P * C + kk;
@@ -162,7 +163,7 @@ __device__ __forceinline__ void vvjp_warp(const VvjpArgs& a, float* smem, int la
               wbase + (wstore ? (size_t)q * a.P * C + k0 : 0), C, wstore);
     // sender gradient
     const int v = __shfl_sync(0xffffffffu, cur.v, p & 31);
-    if (a.xhat != nullptr && act && v >= 0 && v < a.n_nodes) {
+    if (a.xhat != nullptr && act && v >= 0 && v < a.n_send) {
       Grp::flush_xhat(a.xhat + (size_t)v * a.xrow * C + k0, C, xh);
     } else {
 #pragma unroll

@@ -53,10 +53,15 @@ _SIGS = {
     "fc_conv_path": (ct.c_int, [ct.POINTER(ConvDesc), ct.c_int, ct.POINTER(ct.c_int),
                                 ct.POINTER(ct.c_int), ct.POINTER(ct.c_int)]),
     "fc_build_rowptr": (ct.c_int, [ct.c_int, ct.c_int, _vp, _vp, _vp, _vp, _vp]),
+    "fc_build_rowptr_rect": (ct.c_int, [ct.c_int, ct.c_int, ct.c_int, _vp, _vp, _vp, _vp, _vp]),
     "fc_edge_conv": (ct.c_int, [ct.POINTER(ConvDesc), ct.c_int, ct.c_int,
                                 _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
+    "fc_edge_conv_rect": (ct.c_int, [ct.POINTER(ConvDesc), ct.c_int, ct.c_int, ct.c_int,
+                                     _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
     "fc_edge_conv_vjp": (ct.c_int, [ct.POINTER(ConvDesc), ct.c_int, ct.c_int,
                                     _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
+    "fc_edge_conv_vjp_rect": (ct.c_int, [ct.POINTER(ConvDesc), ct.c_int, ct.c_int, ct.c_int,
+                                         _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
     "fc_scalar_readout": (ct.c_int, [ct.c_int, ct.c_int, ct.c_int, _vp, _vp, _vp, _vp]),
     "fc_edge_forces": (ct.c_int, [ct.c_int, ct.c_int, _vp, _vp, _vp, _vp]),
     "fc_ladder_num_paths": (ct.c_int, [ct.POINTER(LadderDesc)]),
@@ -148,9 +153,11 @@ def paths(lmax):
     return out
 
 
-def build_rowptr(edge_index, edge_vec, n_nodes, stream=None):
+def build_rowptr(edge_index, edge_vec, n_nodes, stream=None, n_send=None):
     """Receiver row pointer [n_nodes+1] of a receiver-sorted edge list; raises
-    FlashCartError(FC_ERR_CSR / FC_ERR_DEGENERATE_EDGE) on a bad graph."""
+    FlashCartError(FC_ERR_CSR / FC_ERR_DEGENERATE_EDGE) on a bad graph.
+    n_send: sender count when it differs from the receiver count (a
+    receiver range of a larger graph)."""
     _dev(edge_index, torch.int32, "edge_index")
     E = edge_index.shape[1]
     if edge_vec is not None:
@@ -159,9 +166,9 @@ def build_rowptr(edge_index, edge_vec, n_nodes, stream=None):
     dev = edge_index.device
     rowptr = torch.empty(n_nodes + 1, dtype=torch.int32, device=dev)
     flag = torch.empty(1, dtype=torch.int32, device=dev)
-    _check(_lib.fc_build_rowptr(n_nodes, E, _ptr(edge_index), _ptr(edge_vec),
-                                _ptr(rowptr), _ptr(flag), _stream(stream)),
-           "fc_build_rowptr")
+    _check(_lib.fc_build_rowptr_rect(n_nodes, n_nodes if n_send is None else n_send, E,
+                                     _ptr(edge_index), _ptr(edge_vec), _ptr(rowptr), _ptr(flag),
+                                     _stream(stream)), "fc_build_rowptr")
     return rowptr
 
 
@@ -178,7 +185,8 @@ def edge_conv(lmax, rowptr, edge_index, edge_vec, x, w, sum_paths=False,
     C = x.shape[1] // ((lmax + 1) ** 2)
     d = conv_desc(lmax, C, sum_paths, envelope)
     zr = out_row(lmax, C, sum_paths)
-    if x.shape != (N, (lmax + 1) ** 2 * C):
+    NS = x.shape[0]     # senders: N, or all nodes of the graph for a receiver range
+    if x.dim() != 2 or x.shape[1] != (lmax + 1) ** 2 * C:
         raise ValueError("x shape %s" % (tuple(x.shape),))
     if w.numel() != E * num_paths(lmax) * C:
         raise ValueError("w shape %s" % (tuple(w.shape),))
@@ -187,9 +195,9 @@ def edge_conv(lmax, rowptr, edge_index, edge_vec, x, w, sum_paths=False,
     else:
         _dev(out, torch.float32, "out")
         assert out.shape == (N, zr * C)
-    _check(_lib.fc_edge_conv(ct.byref(d), N, E, _ptr(rowptr), _ptr(edge_index),
-                             _ptr(edge_vec), _ptr(x), _ptr(w), _ptr(out),
-                             _stream(stream)), "fc_edge_conv")
+    _check(_lib.fc_edge_conv_rect(ct.byref(d), N, NS, E, _ptr(rowptr), _ptr(edge_index),
+                                  _ptr(edge_vec), _ptr(x), _ptr(w), _ptr(out),
+                                  _stream(stream)), "fc_edge_conv")
     return out
 
 
@@ -220,9 +228,9 @@ def edge_conv_vjp(lmax, rowptr, edge_index, edge_vec, x, w, g, sum_paths=False,
         wb = torch.empty((E, P, C), dtype=torch.float32, device=x.device)
     if "r" in want and rb is None:
         rb = torch.empty((E, 3), dtype=torch.float32, device=x.device)
-    _check(_lib.fc_edge_conv_vjp(ct.byref(d), N, E, _ptr(rowptr), _ptr(edge_index),
-                                 _ptr(edge_vec), _ptr(x), _ptr(w), _ptr(g), _ptr(xb),
-                                 _ptr(wb), _ptr(rb), _stream(stream)), "fc_edge_conv_vjp")
+    _check(_lib.fc_edge_conv_vjp_rect(ct.byref(d), N, x.shape[0], E, _ptr(rowptr), _ptr(edge_index),
+                                      _ptr(edge_vec), _ptr(x), _ptr(w), _ptr(g), _ptr(xb),
+                                      _ptr(wb), _ptr(rb), _stream(stream)), "fc_edge_conv_vjp")
     return xb, wb, rb
 
 

@@ -128,6 +128,38 @@ def microbench(seed=2, lmax=3, weight_seed=None):
                 edge_index=ei, edge_vec=ev, **d)
 
 
+def sharded_microbench(rank, world, n_per_rank=1024, k=128, channels=128, lmax=3, seed=2):
+    """One graph of world x n_per_rank nodes spread over `world` ranks by
+    receiver range (weak scaling: every rank owns n_per_rank receivers with
+    k random distinct senders among ALL nodes, the microbenchmark's per-rank
+    shape).  Positions are uniform in a cube that keeps the microbenchmark's
+    density; receiver block b draws its senders from seed + 1000 b, so every
+    rank builds the same global edge list.  Returns the global edge_index
+    and bounds, and this rank's own node features, edge vectors and weights
+    (rank-seeded)."""
+    n = world * n_per_rank
+    box = 20.0 * world ** (1.0 / 3.0)
+    pos = rng(seed).uniform(0.0, box, size=(n, 3))
+    recv = np.repeat(np.arange(n, dtype=np.int64), k)
+    send = np.empty(n * k, dtype=np.int64)
+    for b in range(world):
+        g = rng(seed + 1000 * b)
+        for u in range(b * n_per_rank, (b + 1) * n_per_rank):
+            s = g.choice(n - 1, size=k, replace=False)
+            s = np.where(s >= u, s + 1, s)
+            send[u * k:(u + 1) * k] = np.sort(s)
+    edge_index = np.stack([recv, send]).astype(np.int32)
+    e0, e1 = rank * n_per_rank * k, (rank + 1) * n_per_rank * k
+    ev = (pos[send[e0:e1]] - pos[recv[e0:e1]]).astype(np.float32)
+    g = rng(seed + 100 + 7919 * rank)
+    P = path_count(lmax, lmax, lmax)
+    x = normal(g, (n_per_rank, (lmax + 1) ** 2 * channels))
+    w = normal(g, (e1 - e0, P, channels), 1.0 / np.sqrt(P))
+    return dict(name="microbench_sharded", n_nodes=n, lmax=lmax, channels=channels,
+                edge_index=edge_index, bounds=[b * n_per_rank for b in range(world + 1)],
+                x_local=x, w_local=w, edge_vec_local=ev)
+
+
 def microbench_grad(seed=2, lmax=3, weight_seed=None):
     """The microbenchmark graph with an upstream gradient (VJP rows)."""
     pos, ei, ev = random_graph(1024, 128, 20.0, seed)

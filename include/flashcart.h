@@ -132,6 +132,12 @@ int fc_build_rowptr(int n_nodes, int n_edges, const int32_t *edge_index,
                     const float *edge_vec, int32_t *rowptr, int32_t *flag,
                     fc_stream_t stream);
 
+/* fc_build_rowptr for a receiver range (see fc_edge_conv_rect): receivers
+ * in [0, n_nodes), senders in [0, n_send). */
+int fc_build_rowptr_rect(int n_nodes, int n_send, int n_edges, const int32_t *edge_index,
+                         const float *edge_vec, int32_t *rowptr, int32_t *flag,
+                         fc_stream_t stream);
+
 /* Receiver-sorted edge convolution, Sec. 4 Eq. (1):
  *   z[u, eta, k] = sum_{e: u_e = u} w[e, eta, k] f_eta(x[v_e, :, k], T(r-hat_e))
  * with f_eta the Cartesian product of path eta (App. B Eq. (B1)) and
@@ -153,6 +159,19 @@ int fc_edge_conv(const fc_conv_desc *desc, int n_nodes, int n_edges,
                  const float *edge_vec, const float *x, const float *w,
                  float *z, fc_stream_t stream);
 
+/* fc_edge_conv with separate receiver and sender counts, for a graph cut
+ * into contiguous receiver ranges (one per GPU): the n_nodes receivers of
+ * this range (rowptr [n_nodes+1], z [n_nodes][...], receivers numbered
+ * from 0) take their edges from any of the n_send senders of the whole
+ * graph (x [n_send][(lmax_in+1)^2 C], senders < n_send).  Everything else
+ * as fc_edge_conv, which is this call with n_send = n_nodes.  The
+ * convolution is a sum over each receiver's own edges (Sec. 4 Eq. (1)), so
+ * the ranges' outputs are disjoint rows of the whole graph's z. */
+int fc_edge_conv_rect(const fc_conv_desc *desc, int n_nodes, int n_send, int n_edges,
+                      const int32_t *rowptr, const int32_t *edge_index,
+                      const float *edge_vec, const float *x, const float *w,
+                      float *z, fc_stream_t stream);
+
 /* Vector-Jacobian product of fc_edge_conv, App. C Eq. (C1) summed over the
  * receiver-sorted edges as in Algorithm 2, with the direction-tensor
  * gradient carried to the edge vectors (App. C "Symbolic derivatives"):
@@ -173,6 +192,19 @@ int fc_edge_conv_vjp(const fc_conv_desc *desc, int n_nodes, int n_edges,
                      const float *edge_vec, const float *x, const float *w,
                      const float *g, float *x_bar, float *w_bar, float *r_bar,
                      fc_stream_t stream);
+
+/* fc_edge_conv_vjp with separate receiver and sender counts (see
+ * fc_edge_conv_rect): g [n_nodes][...] for this range's receivers, x and
+ * x_bar [n_send][...] over all senders of the graph.  x_bar is then this
+ * range's partial sum of the sender gradients; the ranges' partials add up
+ * to the whole graph's x_bar (a reduce-scatter to the sender owners when
+ * the graph is spread over GPUs).  w_bar and r_bar are per edge, local to
+ * the range. */
+int fc_edge_conv_vjp_rect(const fc_conv_desc *desc, int n_nodes, int n_send, int n_edges,
+                          const int32_t *rowptr, const int32_t *edge_index,
+                          const float *edge_vec, const float *x, const float *w,
+                          const float *g, float *x_bar, float *w_bar, float *r_bar,
+                          fc_stream_t stream);
 
 /* VJP-of-VJP of fc_edge_conv (the derivative of fc_edge_conv_vjp), App. C
  * Eq. (C2) summed over the receiver-sorted edges as in Algorithm 3, with the
