@@ -571,6 +571,102 @@ void orc_path_coeffs(int l1, int l2, int l3, double *K) {
 }
 
 /* ------------------------------------------------------------------ */
+/* odd-J (parity-changing) products: App. B, paragraph after Eq. (B1),  */
+/* and Sec. 7 "Limitations" -- the same construction with one          */
+/* Levi-Civita contraction, the output a pseudo-tensor                  */
+/* ------------------------------------------------------------------ */
+
+/* (l1, l2) -> l3 with l1, l2 >= 1, |l1 - l2| <= l3 <= l1 + l2 - 1 and
+ * l1 + l2 + l3 odd: n = (l1 + l2 - l3 - 1)/2 index pairs contracted, one
+ * index of each input through the Levi-Civita symbol. */
+int orc_odd_admissible(int l1, int l2, int l3) {
+  if (l1 < 1 || l2 < 1 || l3 < 0) return 0;
+  if (l3 < abs(l1 - l2) || l3 > l1 + l2 - 1) return 0;
+  if (!((l1 + l2 + l3) & 1)) return 0;
+  if (l1 > ORC_MAXL || l2 > ORC_MAXL || l3 + 1 > ORC_MAXL) return 0;
+  return 1;
+}
+
+/* epsilon_{abc} for a, b, c in {0, 1, 2} */
+static double levi_civita(int a, int b, int c) {
+  return 0.5 * (double)((a - b) * (b - c) * (c - a));
+}
+
+/* Contract n pairs (x's last n slots with y's first n), then x's last free
+ * slot p and y's first free slot q through epsilon_{p q c}, c the new last
+ * slot; symmetrise over the l3 free slots (permutation average) and remove
+ * the traces.  No further factor: the plain symmetric trace-free part. */
+static void product_odd(int l1, int l2, int l3, const double *xd, const double *yd,
+                        double *out) {
+  int n = (l1 + l2 - l3 - 1) / 2;
+  int a = l1 - n, b = l2 - n;   /* free slots of x and of y after the pairs */
+  double Q[ORC_MAXD], Z[ORC_MAXD], S[ORC_MAXD];
+  contract(l1, xd, l2, yd, n, Q);   /* rank a + b = l3 + 1 */
+  int D = pow3(l3), idx[ORC_MAXL], qi[ORC_MAXL];
+  for (int f = 0; f < D; ++f) {
+    unflat(l3, f, idx);
+    double sum = 0.0;
+    for (int pp = 0; pp < 3; ++pp)
+      for (int qq = 0; qq < 3; ++qq) {
+        double e = levi_civita(pp, qq, idx[l3 - 1]);
+        if (e == 0.0) continue;
+        for (int j = 0; j < a - 1; ++j) qi[j] = idx[j];
+        qi[a - 1] = pp;
+        qi[a] = qq;
+        for (int j = 0; j < b - 1; ++j) qi[a + 1 + j] = idx[a - 1 + j];
+        sum += e * Q[flat(a + b, qi)];
+      }
+    Z[f] = sum;
+  }
+  orc_permavg(l3, Z, S);
+  orc_detrace(l3, S, out);
+}
+
+/* dense odd product from independent components */
+int orc_product_odd_dense(int l1, int l2, int l3, const double *xc, const double *yc,
+                          double *out) {
+  if (!orc_odd_admissible(l1, l2, l3)) return 1;
+  double xd[ORC_MAXD], yd[ORC_MAXD];
+  orc_stf_dense(l1, xc, xd);
+  orc_stf_dense(l2, yc, yd);
+  product_odd(l1, l2, l3, xd, yd, out);
+  return 0;
+}
+
+int orc_product_odd(int l1, int l2, int l3, const double *xc, const double *yc, double *out) {
+  double d[ORC_MAXD];
+  if (orc_product_odd_dense(l1, l2, l3, xc, yc, d)) return 1;
+  orc_stf_extract(l3, d, out);
+  return 0;
+}
+
+/* K[a][b1][b2] = f_a(e_b1, e_b2) of an odd path (bilinear, as above) */
+void orc_path_coeffs_odd(int l1, int l2, int l3, double *K) {
+  int n1 = 2 * l1 + 1, n2 = 2 * l2 + 1, n3 = 2 * l3 + 1;
+  double e1[2 * ORC_MAXL + 1], e2[2 * ORC_MAXL + 1], f[2 * ORC_MAXL + 1];
+  for (int b1 = 0; b1 < n1; ++b1)
+    for (int b2 = 0; b2 < n2; ++b2) {
+      for (int i = 0; i < n1; ++i) e1[i] = (i == b1);
+      for (int i = 0; i < n2; ++i) e2[i] = (i == b2);
+      orc_product_odd(l1, l2, l3, e1, e2, f);
+      for (int a = 0; a < n3; ++a) K[(a * n1 + b1) * n2 + b2] = f[a];
+    }
+}
+
+/* odd paths ordered by l3, then l1, then l2 */
+int orc_paths_odd(int lin, int ledge, int lout, int *l1s, int *l2s, int *l3s) {
+  int n = 0;
+  for (int l3 = 0; l3 <= lout; ++l3)
+    for (int l1 = 0; l1 <= lin; ++l1)
+      for (int l2 = 0; l2 <= ledge; ++l2)
+        if (orc_odd_admissible(l1, l2, l3)) {
+          if (l1s) { l1s[n] = l1; l2s[n] = l2; l3s[n] = l3; }
+          ++n;
+        }
+  return n;
+}
+
+/* ------------------------------------------------------------------ */
 /* path lists                                                           */
 /* ------------------------------------------------------------------ */
 
@@ -591,6 +687,7 @@ int orc_paths(int lin, int ledge, int lout, int *l1s, int *l2s, int *l3s) {
 #define ORC_MAXP 128
 
 typedef struct {
+  int odd;                  /* 1: the odd-J paths, 0: the natural-parity ones */
   int P, l1[ORC_MAXP], l2[ORC_MAXP], l3[ORC_MAXP];
   int eta[ORC_MAXP];        /* position of the path within its l3 */
   int Pl[ORC_MAXL + 1];     /* paths per output rank */
@@ -598,9 +695,11 @@ typedef struct {
   int zrow;                 /* output row length / C */
 } path_set;
 
-static void make_paths(int lin, int ledge, int lout, int sum_paths,
-                       path_set *ps) {
-  ps->P = orc_paths(lin, ledge, lout, ps->l1, ps->l2, ps->l3);
+static void make_paths_par(int lin, int ledge, int lout, int sum_paths, int odd,
+                           path_set *ps) {
+  ps->odd = odd;
+  ps->P = odd ? orc_paths_odd(lin, ledge, lout, ps->l1, ps->l2, ps->l3)
+              : orc_paths(lin, ledge, lout, ps->l1, ps->l2, ps->l3);
   for (int l = 0; l <= ORC_MAXL; ++l) ps->Pl[l] = 0;
   for (int p = 0; p < ps->P; ++p) ps->eta[p] = ps->Pl[ps->l3[p]]++;
   int off = 0;
@@ -609,6 +708,17 @@ static void make_paths(int lin, int ledge, int lout, int sum_paths,
     off += (2 * l + 1) * (sum_paths ? 1 : ps->Pl[l]);
   }
   ps->zrow = off;
+}
+
+static void make_paths(int lin, int ledge, int lout, int sum_paths, path_set *ps) {
+  make_paths_par(lin, ledge, lout, sum_paths, 0, ps);
+}
+
+static void path_coeffs_of(const path_set *ps, int p, double *K) {
+  if (ps->odd)
+    orc_path_coeffs_odd(ps->l1[p], ps->l2[p], ps->l3[p], K);
+  else
+    orc_path_coeffs(ps->l1[p], ps->l2[p], ps->l3[p], K);
 }
 
 /* ------------------------------------------------------------------ */
@@ -620,13 +730,13 @@ static void make_paths(int lin, int ledge, int lout, int sum_paths,
  * C*(zoff(l3) + c) + k when paths are summed.
  * Only edges whose receiver has recv_mask != 0 contribute (NULL = all);
  * z rows of other receivers are left at zero. */
-int orc_edge_conv(int lin, int ledge, int lout, int C, int sum_paths, int N,
-                  int E, const int32_t *recv, const int32_t *send,
-                  const double *vec, const double *x, const double *w,
-                  const unsigned char *recv_mask, double *z) {
+static int edge_conv_par(int odd, int lin, int ledge, int lout, int C, int sum_paths, int N,
+                         int E, const int32_t *recv, const int32_t *send,
+                         const double *vec, const double *x, const double *w,
+                         const unsigned char *recv_mask, double *z) {
   if (lin > 5 || ledge > 5 || lout > 5) return 1;
   path_set ps;
-  make_paths(lin, ledge, lout, sum_paths, &ps);
+  make_paths_par(lin, ledge, lout, sum_paths, odd, &ps);
   int xrow = (lin + 1) * (lin + 1);
   memset(z, 0, sizeof(double) * (size_t)N * ps.zrow * C);
   /* direction tensors per edge, dense (shared by every channel) */
@@ -653,8 +763,14 @@ int orc_edge_conv(int lin, int ledge, int lout, int C, int sum_paths, int N,
         int l1 = ps.l1[p], l2 = ps.l2[p], l3 = ps.l3[p];
         for (int c = 0; c < 2 * l1 + 1; ++c)
           xc[c] = x[((size_t)v * xrow + l1 * l1 + c) * C + k];
-        product_xc_yd(l1, l2, l3, xc,
-                      yd + (size_t)e * ystride + yoff[l2], f);
+        if (odd) {
+          double xd[ORC_MAXD], d[ORC_MAXD];
+          orc_stf_dense(l1, xc, xd);
+          product_odd(l1, l2, l3, xd, yd + (size_t)e * ystride + yoff[l2], d);
+          orc_stf_extract(l3, d, f);
+        } else {
+          product_xc_yd(l1, l2, l3, xc, yd + (size_t)e * ystride + yoff[l2], f);
+        }
         double wk = w[((size_t)e * ps.P + p) * C + k];
         for (int c = 0; c < 2 * l3 + 1; ++c) {
           int slot = sum_paths ? ps.zoff[l3] + c
@@ -668,6 +784,24 @@ int orc_edge_conv(int lin, int ledge, int lout, int C, int sum_paths, int N,
   return 0;
 }
 
+int orc_edge_conv(int lin, int ledge, int lout, int C, int sum_paths, int N,
+                  int E, const int32_t *recv, const int32_t *send,
+                  const double *vec, const double *x, const double *w,
+                  const unsigned char *recv_mask, double *z) {
+  return edge_conv_par(0, lin, ledge, lout, C, sum_paths, N, E, recv, send, vec, x, w,
+                       recv_mask, z);
+}
+
+/* the same sum over the odd-J paths (pseudo-tensor outputs), same layouts
+ * with the odd path list */
+int orc_edge_conv_odd(int lin, int ledge, int lout, int C, int sum_paths, int N,
+                      int E, const int32_t *recv, const int32_t *send,
+                      const double *vec, const double *x, const double *w,
+                      const unsigned char *recv_mask, double *z) {
+  return edge_conv_par(1, lin, ledge, lout, C, sum_paths, N, E, recv, send, vec, x, w,
+                       recv_mask, z);
+}
+
 /* ------------------------------------------------------------------ */
 /* its vector-Jacobian product, Eq. (C1) summed as in Sec. 4            */
 /* ------------------------------------------------------------------ */
@@ -678,14 +812,14 @@ int orc_edge_conv(int lin, int ledge, int lout, int C, int sum_paths, int N,
  * to the independent components as free variables (App. C).
  * Only edges with edge_mask != 0 contribute (NULL = all); any output pointer
  * may be NULL. */
-int orc_edge_conv_vjp(int lin, int ledge, int lout, int C, int sum_paths,
-                      int N, int E, const int32_t *recv, const int32_t *send,
-                      const double *vec, const double *x, const double *w,
-                      const double *g, const unsigned char *edge_mask,
-                      double *x_bar, double *w_bar, double *r_bar) {
+static int edge_conv_vjp_par(int odd, int lin, int ledge, int lout, int C, int sum_paths,
+                             int N, int E, const int32_t *recv, const int32_t *send,
+                             const double *vec, const double *x, const double *w,
+                             const double *g, const unsigned char *edge_mask,
+                             double *x_bar, double *w_bar, double *r_bar) {
   if (lin > 5 || ledge > 5 || lout > 5) return 1;
   path_set ps;
-  make_paths(lin, ledge, lout, sum_paths, &ps);
+  make_paths_par(lin, ledge, lout, sum_paths, odd, &ps);
   int xrow = (lin + 1) * (lin + 1);
   int yrow = (ledge + 1) * (ledge + 1);
   /* per-path coefficient tensors */
@@ -693,7 +827,7 @@ int orc_edge_conv_vjp(int lin, int ledge, int lout, int C, int sum_paths,
   for (int p = 0; p < ps.P; ++p) {
     int n1 = 2 * ps.l1[p] + 1, n2 = 2 * ps.l2[p] + 1, n3 = 2 * ps.l3[p] + 1;
     K[p] = (double *)malloc(sizeof(double) * n1 * n2 * n3);
-    orc_path_coeffs(ps.l1[p], ps.l2[p], ps.l3[p], K[p]);
+    path_coeffs_of(&ps, p, K[p]);
   }
   /* direction tensor components per edge */
   double *y = (double *)malloc(sizeof(double) * (size_t)(E > 0 ? E : 1) * yrow);
@@ -785,6 +919,25 @@ int orc_edge_conv_vjp(int lin, int ledge, int lout, int C, int sum_paths,
   for (int p = 0; p < ps.P; ++p) free(K[p]);
   free(y);
   return 0;
+}
+
+int orc_edge_conv_vjp(int lin, int ledge, int lout, int C, int sum_paths,
+                      int N, int E, const int32_t *recv, const int32_t *send,
+                      const double *vec, const double *x, const double *w,
+                      const double *g, const unsigned char *edge_mask,
+                      double *x_bar, double *w_bar, double *r_bar) {
+  return edge_conv_vjp_par(0, lin, ledge, lout, C, sum_paths, N, E, recv, send, vec, x, w, g,
+                           edge_mask, x_bar, w_bar, r_bar);
+}
+
+/* the VJP of orc_edge_conv_odd (same formulas, odd-path coefficients) */
+int orc_edge_conv_odd_vjp(int lin, int ledge, int lout, int C, int sum_paths,
+                          int N, int E, const int32_t *recv, const int32_t *send,
+                          const double *vec, const double *x, const double *w,
+                          const double *g, const unsigned char *edge_mask,
+                          double *x_bar, double *w_bar, double *r_bar) {
+  return edge_conv_vjp_par(1, lin, ledge, lout, C, sum_paths, N, E, recv, send, vec, x, w, g,
+                           edge_mask, x_bar, w_bar, r_bar);
 }
 
 /* ------------------------------------------------------------------ */

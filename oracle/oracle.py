@@ -40,6 +40,14 @@ def lib():
             "orc_paths": (ct.c_int, [ct.c_int] * 3 + [ip, ip, ip]),
             "orc_edge_conv": (ct.c_int, [ct.c_int] * 7 + [i32, i32, d, d, d, u8, d]),
             "orc_edge_conv_vjp": (ct.c_int, [ct.c_int] * 7 + [i32, i32, d, d, d, d, u8, d, d, d]),
+            "orc_edge_conv_odd": (ct.c_int, [ct.c_int] * 7 + [i32, i32, d, d, d, u8, d]),
+            "orc_edge_conv_odd_vjp": (ct.c_int, [ct.c_int] * 7 + [i32, i32, d, d, d, d, u8, d, d,
+                                                                  d]),
+            "orc_odd_admissible": (ct.c_int, [ct.c_int] * 3),
+            "orc_product_odd_dense": (ct.c_int, [ct.c_int] * 3 + [d, d, d]),
+            "orc_product_odd": (ct.c_int, [ct.c_int] * 3 + [d, d, d]),
+            "orc_path_coeffs_odd": (None, [ct.c_int] * 3 + [d]),
+            "orc_paths_odd": (ct.c_int, [ct.c_int] * 3 + [ip, ip, ip]),
             "orc_edge_conv_vjp2": (ct.c_int, [ct.c_int] * 7 + [i32, i32, d, d, d, d, d, d, d, u8,
                                                                d, d, d, d]),
             "orc_direction_hvp": (None, [ct.c_int, d, d, d, d]),
@@ -186,13 +194,46 @@ def path_coeffs(l1, l2, l3):
     return out.reshape(2 * l3 + 1, 2 * l1 + 1, 2 * l2 + 1)
 
 
-def paths(lin, ledge, lout):
-    n = lib().orc_paths(lin, ledge, lout, None, None, None)
+def paths(lin, ledge, lout, odd=False):
+    """Admissible paths ordered by l3, then l1, then l2; odd=True lists the
+    odd-J (Levi-Civita) paths instead."""
+    f = lib().orc_paths_odd if odd else lib().orc_paths
+    n = f(lin, ledge, lout, None, None, None)
     a = (ct.c_int * max(n, 1))()
     b = (ct.c_int * max(n, 1))()
     c = (ct.c_int * max(n, 1))()
-    lib().orc_paths(lin, ledge, lout, a, b, c)
+    f(lin, ledge, lout, a, b, c)
     return [(a[i], b[i], c[i]) for i in range(n)]
+
+
+# --------------------------------------------------------------------------
+# odd-J products (App. B after Eq. B1; Sec. 7): one Levi-Civita contraction
+# --------------------------------------------------------------------------
+
+def odd_admissible(l1, l2, l3):
+    return bool(lib().orc_odd_admissible(l1, l2, l3))
+
+
+def product_odd_dense(l1, l2, l3, x, y):
+    x, y = _d(x), _d(y)
+    out = np.empty(3 ** l3)
+    if lib().orc_product_odd_dense(l1, l2, l3, _pd(x), _pd(y), _pd(out)):
+        raise ValueError("path (%d,%d)->%d is not an odd-J path" % (l1, l2, l3))
+    return out.reshape((3,) * l3)
+
+
+def product_odd(l1, l2, l3, x, y):
+    x, y = _d(x), _d(y)
+    out = np.empty(2 * l3 + 1)
+    if lib().orc_product_odd(l1, l2, l3, _pd(x), _pd(y), _pd(out)):
+        raise ValueError("path (%d,%d)->%d is not an odd-J path" % (l1, l2, l3))
+    return out
+
+
+def path_coeffs_odd(l1, l2, l3):
+    out = np.empty((2 * l3 + 1) * (2 * l1 + 1) * (2 * l2 + 1))
+    lib().orc_path_coeffs_odd(l1, l2, l3, _pd(out))
+    return out.reshape(2 * l3 + 1, 2 * l1 + 1, 2 * l2 + 1)
 
 
 def num_threads():
@@ -203,20 +244,21 @@ def num_threads():
 # edge convolution (Sec. 4 Eq. 1) and its VJP (App. C Eq. C1)
 # --------------------------------------------------------------------------
 
-def zrow(lin, ledge, lout, sum_paths=False):
+def zrow(lin, ledge, lout, sum_paths=False, odd=False):
     """Output row length / C for the edge convolution."""
-    ps = paths(lin, ledge, lout)
+    ps = paths(lin, ledge, lout, odd)
     if sum_paths:
         return (lout + 1) ** 2
     return sum(2 * l3 + 1 for (_, _, l3) in ps)
 
 
 def edge_conv(lin, ledge, lout, C, edge_index, edge_vec, x, w, n_nodes,
-              sum_paths=False, recv_mask=None):
+              sum_paths=False, recv_mask=None, odd=False):
     """z = Eq. (1).  With recv_mask, only the listed receivers' rows are
-    computed (their edges are selected here; other rows stay zero)."""
+    computed (their edges are selected here; other rows stay zero).
+    odd=True: over the odd-J paths (pseudo-tensor outputs)."""
     ei = np.asarray(edge_index)
-    P = len(paths(lin, ledge, lout))
+    P = len(paths(lin, ledge, lout, odd))
     if recv_mask is not None:
         m = _mask(recv_mask, n_nodes)
         sel = np.nonzero(m[ei[0]])[0]
@@ -229,9 +271,10 @@ def edge_conv(lin, ledge, lout, C, edge_index, edge_vec, x, w, n_nodes,
     x = _d(x)
     w = _d(w).reshape(E, P, C)
     assert x.shape == (n_nodes, (lin + 1) ** 2 * C)
-    zr = zrow(lin, ledge, lout, sum_paths)
+    zr = zrow(lin, ledge, lout, sum_paths, odd)
     z = np.empty((n_nodes, zr * C))
-    rc = lib().orc_edge_conv(lin, ledge, lout, C, int(sum_paths), n_nodes, E,
+    f = lib().orc_edge_conv_odd if odd else lib().orc_edge_conv
+    rc = f(lin, ledge, lout, C, int(sum_paths), n_nodes, E,
                              _pi32(recv), _pi32(send), _pd(vec), _pd(x), _pd(w),
                              None, _pd(z))
     assert rc == 0
@@ -239,13 +282,13 @@ def edge_conv(lin, ledge, lout, C, edge_index, edge_vec, x, w, n_nodes,
 
 
 def edge_conv_vjp(lin, ledge, lout, C, edge_index, edge_vec, x, w, g, n_nodes,
-                  sum_paths=False, edge_mask=None, want=("x", "w", "r")):
+                  sum_paths=False, edge_mask=None, want=("x", "w", "r"), odd=False):
     """Eq. (C1) summed over edges.  With edge_mask, only the listed edges
     contribute (they are selected here); w_bar / r_bar rows of the other
-    edges are zero."""
+    edges are zero.  odd=True: the VJP of the odd-J convolution."""
     ei_full = np.asarray(edge_index)
     E_full = ei_full.shape[1]
-    P = len(paths(lin, ledge, lout))
+    P = len(paths(lin, ledge, lout, odd))
     sel = None
     ei, ev, ww = ei_full, np.asarray(edge_vec), np.asarray(w)
     if edge_mask is not None:
@@ -260,7 +303,8 @@ def edge_conv_vjp(lin, ledge, lout, C, edge_index, edge_vec, x, w, g, n_nodes,
     xb = np.empty(((n_nodes, (lin + 1) ** 2 * C))) if "x" in want else None
     wb = np.empty((E, P, C)) if "w" in want else None
     rb = np.empty((E, 3)) if "r" in want else None
-    rc = lib().orc_edge_conv_vjp(lin, ledge, lout, C, int(sum_paths), n_nodes, E,
+    f = lib().orc_edge_conv_odd_vjp if odd else lib().orc_edge_conv_vjp
+    rc = f(lin, ledge, lout, C, int(sum_paths), n_nodes, E,
                                  _pi32(recv), _pi32(send), _pd(vec), _pd(x),
                                  _pd(ww), _pd(g), None, _pd(xb), _pd(wb), _pd(rb))
     assert rc == 0
