@@ -268,7 +268,7 @@ def time_events(fn, steps, warmup, stream, flush=None):
 
 
 ROW_NAMES = ("edge_conv_vjp_r3", "edge_conv_vvjp_r3", "edge_conv_fwd_r4", "edge_conv_vjp_r4",
-             "ladder", "full_ladder", "block_energy_forces")
+             "edge_conv_odd_r3", "ladder", "full_ladder", "block_energy_forces")
 
 
 def extra_rows(fc, W, dev, stream, peaks, fp32_peak, steps, select=ROW_NAMES):
@@ -396,6 +396,37 @@ def extra_rows(fc, W, dev, stream, peaks, fp32_peak, steps, select=ROW_NAMES):
                              "algorithmic_bytes": byt4b}}
         z4 = g4 = out4 = None
         del x4, w4
+        torch.cuda.empty_cache()
+
+    if "edge_conv_odd_r3" in select:
+        # --- odd-J (Levi-Civita) paths, rank 3, microbench graph: forward and VJP
+        Po = fc.odd_num_paths(3)
+        zro = fc.odd_out_row(3)
+        gen = torch.Generator(device=dev)
+        gen.manual_seed(77)
+        xo = torch.randn(N, 16 * C, device=dev, generator=gen)
+        wo = torch.randn(E, Po, C, device=dev, generator=gen) * Po ** -0.5
+        go = torch.randn(N, zro * C, device=dev, generator=gen)
+        zo = torch.empty((N, zro * C), device=dev)
+        mso, mno = time_events(lambda: fc.edge_conv(3, rp, ei, ev, xo, wo, out=zo, odd=True), steps, 3, stream)
+        outo = {"x": torch.empty_like(xo), "w": torch.empty_like(wo), "r": torch.empty((E, 3), device=dev)}
+        msov, mnov = time_events(lambda: fc.edge_conv_vjp(3, rp, ei, ev, xo, wo, go, out=outo, odd=True),
+                                 steps, 3, stream)
+        bo = 4 * (E * Po * C + N * 16 * C + N * zro * C + 4 * E + N)
+        bov = 4 * (2 * E * Po * C + N * zro * C + 2 * N * 16 * C + 7 * E + N)
+        rows["edge_conv_odd_fwd_r3"] = {
+            "workload": "microbench graph, rank 3, the %d odd-J (Levi-Civita) paths, forward" % Po,
+            "ms": mso, "ms_min": mno, "edge_channels_per_s": E * C / (mso * 1e-3),
+            "roofline": {"bound": "hbm", "achieved": bo / (mso * 1e-3) / 1e9, "peak": peaks["hbm_gbs"],
+                         "unit": "GB/s", "frac": bo / (mso * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                         "algorithmic_bytes": bo}}
+        rows["edge_conv_odd_vjp_r3"] = {
+            "workload": "same odd-J convolution, x_bar + w_bar + r_bar",
+            "ms": msov, "ms_min": mnov, "edge_channels_per_s": E * C / (msov * 1e-3),
+            "roofline": {"bound": "hbm", "achieved": bov / (msov * 1e-3) / 1e9, "peak": peaks["hbm_gbs"],
+                         "unit": "GB/s", "frac": bov / (msov * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                         "algorithmic_bytes": bov}}
+        del xo, wo, go, zo, outo
         torch.cuda.empty_cache()
 
     if "ladder" in select:

@@ -78,6 +78,33 @@ inline int out_row(int L, int sum_paths) {
   return n;
 }
 
+// Odd-J (Levi-Civita) paths: l1, l2 >= 1, |l1 - l2| <= l3 <= l1 + l2 - 1,
+// l1 + l2 + l3 odd.  Their kernels are instantiated under rank key L + kOddKey.
+constexpr int kOddKey = 16;
+
+inline bool odd_admissible(int l1, int l2, int l3) {
+  return l1 >= 1 && l2 >= 1 && l3 >= (l1 > l2 ? l1 - l2 : l2 - l1) && l3 <= l1 + l2 - 1 &&
+         ((l1 + l2 + l3) & 1) == 1;
+}
+
+inline int num_odd_paths(int L) {
+  int n = 0;
+  for (int l3 = 0; l3 <= L; ++l3)
+    for (int l1 = 0; l1 <= L; ++l1)
+      for (int l2 = 0; l2 <= L; ++l2) n += odd_admissible(l1, l2, l3);
+  return n;
+}
+
+inline int odd_out_row(int L, int sum_paths) {
+  if (sum_paths) return (L + 1) * (L + 1);
+  int n = 0;
+  for (int l3 = 0; l3 <= L; ++l3)
+    for (int l1 = 0; l1 <= L; ++l1)
+      for (int l2 = 0; l2 <= L; ++l2)
+        if (odd_admissible(l1, l2, l3)) n += 2 * l3 + 1;
+  return n;
+}
+
 // SM count and occupancy are cached per device
 int device_sm_count();
 

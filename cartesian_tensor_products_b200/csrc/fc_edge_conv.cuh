@@ -194,6 +194,54 @@ static int launch_fwd_cc(const ConvArgs& a, cudaStream_t s) {
   return cudaGetLastError() == cudaSuccess ? FC_OK : FC_ERR_CUDA;
 }
 
+// Host checks and kernel arguments shared by the forward entry points
+// (natural-parity paths, odd = 0, or odd-J paths, odd = 1).  Returns FC_OK
+// with *launch = false when there is nothing to launch; with sum_paths the
+// output is zeroed on the stream (the kernels then add path sums into it).
+inline int conv_setup(const fc_conv_desc* d, int n_nodes, int n_send, int n_edges,
+                      const int32_t* rowptr, const int32_t* edge_index, const float* edge_vec,
+                      const float* x, const float* w, float* z, int odd, cudaStream_t s,
+                      ConvArgs& a, bool* launch) {
+  *launch = false;
+  int st = check_conv_desc(d);
+  if (st != FC_OK) return st;
+  if (odd && d->lmax_in > 4) return FC_ERR_UNSUPPORTED_RANK;
+  if (n_nodes < 0 || n_send < 0 || n_edges < 0) return FC_ERR_ARG;
+  if (n_nodes == 0) return n_edges == 0 ? FC_OK : FC_ERR_ARG;
+  if (!rowptr || !x || !z) return FC_ERR_ARG;
+  if (n_edges > 0 && (!edge_index || !edge_vec || !w)) return FC_ERR_ARG;
+  if (!aligned16(x) || !aligned16(z) || (w && !aligned16(w)) || !aligned4(rowptr) ||
+      (edge_index && !aligned4(edge_index)) || (edge_vec && !aligned4(edge_vec)))
+    return FC_ERR_ALIGN;
+  const int L = d->lmax_in;
+  const int C = d->channels;
+  a.rowptr = rowptr;
+  a.send = edge_index ? edge_index + n_edges : nullptr;
+  a.vec = edge_vec;
+  a.x = x;
+  a.w = w;
+  a.z = z;
+  a.n_nodes = n_nodes;
+  a.n_send = n_send;
+  a.n_edges = n_edges;
+  a.C = C;
+  a.ntiles = (C + 127) / 128;
+  a.xrow = (L + 1) * (L + 1);
+  a.zrow = odd ? odd_out_row(L, d->sum_paths) : out_row(L, d->sum_paths);
+  a.P = odd ? num_odd_paths(L) : num_paths(L);
+  a.sum_paths = d->sum_paths;
+  a.envelope = d->envelope;
+  a.r_cut = d->r_cut;
+  a.edge_scale = d->edge_scale;
+  if ((long long)n_nodes * a.ntiles > 0x7fffffffLL) return FC_ERR_ARG;
+  if (d->sum_paths) {
+    if (cudaMemsetAsync(z, 0, sizeof(float) * (size_t)n_nodes * a.zrow * C, s) != cudaSuccess)
+      return FC_ERR_CUDA;
+  }
+  *launch = true;
+  return FC_OK;
+}
+
 template <int L>
 static int launch_fwd(const ConvArgs& a, cudaStream_t s) {
   if (a.envelope) return a.C == 128 ? launch_fwd_cc<L, 128, true>(a, s) : launch_fwd_cc<L, 0, true>(a, s);

@@ -241,6 +241,61 @@ static int launch_vjp_cc(const VjpArgs& a, cudaStream_t s) {
   return cudaGetLastError() == cudaSuccess ? FC_OK : FC_ERR_CUDA;
 }
 
+// Host checks and kernel arguments shared by the VJP entry points
+// (natural-parity paths, odd = 0, or odd-J paths, odd = 1).  Zeroes x_bar
+// and r_bar on the stream (they are accumulated atomically); *launch is
+// false when there is nothing to launch.
+inline int vjp_setup(const fc_conv_desc* d, int n_nodes, int n_send, int n_edges,
+                     const int32_t* rowptr, const int32_t* edge_index, const float* edge_vec,
+                     const float* x, const float* w, const float* g, float* x_bar, float* w_bar,
+                     float* r_bar, int odd, cudaStream_t s, VjpArgs& a, bool* launch) {
+  *launch = false;
+  int st = check_conv_desc(d);
+  if (st != FC_OK) return st;
+  if (odd && d->lmax_in > 4) return FC_ERR_UNSUPPORTED_RANK;
+  if (n_nodes < 0 || n_send < 0 || n_edges < 0) return FC_ERR_ARG;
+  if (n_nodes == 0) return n_edges == 0 ? FC_OK : FC_ERR_ARG;
+  if (!rowptr || !x || !g) return FC_ERR_ARG;
+  if (n_edges > 0 && (!edge_index || !edge_vec || !w)) return FC_ERR_ARG;
+  if (!aligned16(x) || !aligned16(g) || (w && !aligned16(w)) || (x_bar && !aligned16(x_bar)) ||
+      (w_bar && !aligned16(w_bar)) || (r_bar && !aligned4(r_bar)) || !aligned4(rowptr) ||
+      (edge_index && !aligned4(edge_index)) || (edge_vec && !aligned4(edge_vec)))
+    return FC_ERR_ALIGN;
+  const int L = d->lmax_in;
+  const int C = d->channels;
+  a.rowptr = rowptr;
+  a.send = edge_index ? edge_index + n_edges : nullptr;
+  a.vec = edge_vec;
+  a.x = x;
+  a.w = w;
+  a.g = g;
+  a.xbar = x_bar;
+  a.wbar = w_bar;
+  a.rbar = r_bar;
+  a.n_nodes = n_nodes;
+  a.n_send = n_send;
+  a.n_edges = n_edges;
+  a.C = C;
+  a.ntiles = (C + 127) / 128;
+  a.xrow = (L + 1) * (L + 1);
+  a.zrow = odd ? odd_out_row(L, d->sum_paths) : out_row(L, d->sum_paths);
+  a.P = odd ? num_odd_paths(L) : num_paths(L);
+  a.sum_paths = d->sum_paths;
+  a.envelope = d->envelope;
+  a.r_cut = d->r_cut;
+  a.edge_scale = d->edge_scale;
+  if ((long long)n_nodes * a.ntiles > 0x7fffffffLL) return FC_ERR_ARG;
+  if (x_bar && cudaMemsetAsync(x_bar, 0, sizeof(float) * (size_t)n_send * a.xrow * C, s) != cudaSuccess)
+    return FC_ERR_CUDA;
+  if (r_bar && n_edges > 0 &&
+      cudaMemsetAsync(r_bar, 0, sizeof(float) * 3 * (size_t)n_edges, s) != cudaSuccess)
+    return FC_ERR_CUDA;
+  if (n_edges == 0) return FC_OK;
+  if (!x_bar && !w_bar && !r_bar) return FC_OK;
+  *launch = true;
+  return FC_OK;
+}
+
 template <int L>
 static int launch_vjp(const VjpArgs& a, cudaStream_t s) {
   return a.C == 128 ? launch_vjp_cc<L, 128>(a, s) : launch_vjp_cc<L, 0>(a, s);

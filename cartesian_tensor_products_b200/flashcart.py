@@ -62,6 +62,14 @@ _SIGS = {
                                     _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
     "fc_edge_conv_vjp_rect": (ct.c_int, [ct.POINTER(ConvDesc), ct.c_int, ct.c_int, ct.c_int,
                                          _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
+    "fc_conv_odd_num_paths": (ct.c_int, [ct.POINTER(ConvDesc)]),
+    "fc_conv_odd_out_row": (ct.c_int, [ct.POINTER(ConvDesc)]),
+    "fc_conv_odd_path": (ct.c_int, [ct.POINTER(ConvDesc), ct.c_int, ct.POINTER(ct.c_int),
+                                    ct.POINTER(ct.c_int), ct.POINTER(ct.c_int)]),
+    "fc_edge_conv_odd": (ct.c_int, [ct.POINTER(ConvDesc), ct.c_int, ct.c_int,
+                                    _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
+    "fc_edge_conv_odd_vjp": (ct.c_int, [ct.POINTER(ConvDesc), ct.c_int, ct.c_int,
+                                        _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
     "fc_scalar_readout": (ct.c_int, [ct.c_int, ct.c_int, ct.c_int, _vp, _vp, _vp, _vp]),
     "fc_edge_forces": (ct.c_int, [ct.c_int, ct.c_int, _vp, _vp, _vp, _vp]),
     "fc_ladder_num_paths": (ct.c_int, [ct.POINTER(LadderDesc)]),
@@ -153,6 +161,34 @@ def paths(lmax):
     return out
 
 
+def odd_num_paths(lmax, channels=4, sum_paths=False):
+    """Number of odd-J (Levi-Civita) paths at this rank."""
+    d = conv_desc(lmax, channels, sum_paths)
+    n = _lib.fc_conv_odd_num_paths(ct.byref(d))
+    if n < 0:
+        raise FlashCartError(4, "fc_conv_odd_num_paths")
+    return n
+
+
+def odd_out_row(lmax, channels=4, sum_paths=False):
+    d = conv_desc(lmax, channels, sum_paths)
+    n = _lib.fc_conv_odd_out_row(ct.byref(d))
+    if n < 0:
+        raise FlashCartError(4, "fc_conv_odd_out_row")
+    return n
+
+
+def odd_paths(lmax):
+    d = conv_desc(lmax, 4)
+    out = []
+    for p in range(odd_num_paths(lmax)):
+        a, b, c = ct.c_int(), ct.c_int(), ct.c_int()
+        _check(_lib.fc_conv_odd_path(ct.byref(d), p, ct.byref(a), ct.byref(b), ct.byref(c)),
+               "fc_conv_odd_path")
+        out.append((a.value, b.value, c.value))
+    return out
+
+
 def build_rowptr(edge_index, edge_vec, n_nodes, stream=None, n_send=None):
     """Receiver row pointer [n_nodes+1] of a receiver-sorted edge list; raises
     FlashCartError(FC_ERR_CSR / FC_ERR_DEGENERATE_EDGE) on a bad graph.
@@ -173,8 +209,9 @@ def build_rowptr(edge_index, edge_vec, n_nodes, stream=None, n_send=None):
 
 
 def edge_conv(lmax, rowptr, edge_index, edge_vec, x, w, sum_paths=False,
-              out=None, stream=None, envelope=None):
-    """z of Sec. 4 Eq. (1): [N][out_row * C]."""
+              out=None, stream=None, envelope=None, odd=False):
+    """z of Sec. 4 Eq. (1): [N][out_row * C].  odd=True: over the odd-J
+    (Levi-Civita) paths (fc_edge_conv_odd; senders = receivers)."""
     _dev(rowptr, torch.int32, "rowptr")
     _dev(edge_index, torch.int32, "edge_index")
     _dev(edge_vec, torch.float32, "edge_vec")
@@ -184,17 +221,24 @@ def edge_conv(lmax, rowptr, edge_index, edge_vec, x, w, sum_paths=False,
     E = edge_index.shape[1]
     C = x.shape[1] // ((lmax + 1) ** 2)
     d = conv_desc(lmax, C, sum_paths, envelope)
-    zr = out_row(lmax, C, sum_paths)
+    zr = odd_out_row(lmax, C, sum_paths) if odd else out_row(lmax, C, sum_paths)
     NS = x.shape[0]     # senders: N, or all nodes of the graph for a receiver range
     if x.dim() != 2 or x.shape[1] != (lmax + 1) ** 2 * C:
         raise ValueError("x shape %s" % (tuple(x.shape),))
-    if w.numel() != E * num_paths(lmax) * C:
+    if w.numel() != E * (odd_num_paths(lmax) if odd else num_paths(lmax)) * C:
         raise ValueError("w shape %s" % (tuple(w.shape),))
     if out is None:
         out = torch.empty((N, zr * C), dtype=torch.float32, device=x.device)
     else:
         _dev(out, torch.float32, "out")
         assert out.shape == (N, zr * C)
+    if odd:
+        if NS != N:
+            raise ValueError("the odd-J convolution takes senders = receivers")
+        _check(_lib.fc_edge_conv_odd(ct.byref(d), N, E, _ptr(rowptr), _ptr(edge_index),
+                                     _ptr(edge_vec), _ptr(x), _ptr(w), _ptr(out),
+                                     _stream(stream)), "fc_edge_conv_odd")
+        return out
     _check(_lib.fc_edge_conv_rect(ct.byref(d), N, NS, E, _ptr(rowptr), _ptr(edge_index),
                                   _ptr(edge_vec), _ptr(x), _ptr(w), _ptr(out),
                                   _stream(stream)), "fc_edge_conv")
@@ -202,8 +246,9 @@ def edge_conv(lmax, rowptr, edge_index, edge_vec, x, w, sum_paths=False,
 
 
 def edge_conv_vjp(lmax, rowptr, edge_index, edge_vec, x, w, g, sum_paths=False,
-                  want=("x", "w", "r"), out=None, stream=None, envelope=None):
-    """(x_bar, w_bar, r_bar) of App. C Eq. (C1); entries not in `want` are None."""
+                  want=("x", "w", "r"), out=None, stream=None, envelope=None, odd=False):
+    """(x_bar, w_bar, r_bar) of App. C Eq. (C1); entries not in `want` are None.
+    odd=True: the VJP of the odd-J path convolution."""
     _dev(rowptr, torch.int32, "rowptr")
     _dev(edge_index, torch.int32, "edge_index")
     _dev(edge_vec, torch.float32, "edge_vec")
@@ -214,8 +259,9 @@ def edge_conv_vjp(lmax, rowptr, edge_index, edge_vec, x, w, g, sum_paths=False,
     E = edge_index.shape[1]
     C = x.shape[1] // ((lmax + 1) ** 2)
     d = conv_desc(lmax, C, sum_paths, envelope)
-    P = num_paths(lmax)
-    if g.shape != (N, out_row(lmax, C, sum_paths) * C):
+    P = odd_num_paths(lmax) if odd else num_paths(lmax)
+    zr = odd_out_row(lmax, C, sum_paths) if odd else out_row(lmax, C, sum_paths)
+    if g.shape != (N, zr * C):
         raise ValueError("g shape %s" % (tuple(g.shape),))
     if out is None:
         out = {}
@@ -228,6 +274,11 @@ def edge_conv_vjp(lmax, rowptr, edge_index, edge_vec, x, w, g, sum_paths=False,
         wb = torch.empty((E, P, C), dtype=torch.float32, device=x.device)
     if "r" in want and rb is None:
         rb = torch.empty((E, 3), dtype=torch.float32, device=x.device)
+    if odd:
+        _check(_lib.fc_edge_conv_odd_vjp(ct.byref(d), N, E, _ptr(rowptr), _ptr(edge_index),
+                                         _ptr(edge_vec), _ptr(x), _ptr(w), _ptr(g), _ptr(xb),
+                                         _ptr(wb), _ptr(rb), _stream(stream)), "fc_edge_conv_odd_vjp")
+        return xb, wb, rb
     _check(_lib.fc_edge_conv_vjp_rect(ct.byref(d), N, x.shape[0], E, _ptr(rowptr), _ptr(edge_index),
                                       _ptr(edge_vec), _ptr(x), _ptr(w), _ptr(g), _ptr(xb),
                                       _ptr(wb), _ptr(rb), _stream(stream)), "fc_edge_conv_vjp")

@@ -26,6 +26,12 @@ How each step is written here:
   * C_{l1l2l3}: chosen so that (T_l1 (x) T_l2)_l3 = T_l3 (the reading used
     for the normalisation the pages leave to another paper); T_l(z-hat) has
     the polynomial |r|^l P_l(z/|r|) with P_l the Legendre polynomial.
+  * odd-J products (App. B, paragraph after Eq. (B1); Sec. 7): one index
+    of each input contracted through the Levi-Civita symbol after n pairs,
+    then the symmetric trace-free part with no further factor.  In
+    polynomial form the epsilon contraction is the triple product
+    r . (grad a x grad b) of the n-times paired derivatives a, b, scaled by
+    (l1-n-1)!(l2-n-1)!/(l1! l2!).
 """
 from fractions import Fraction
 from functools import lru_cache
@@ -264,3 +270,62 @@ def direction_component_poly(l, comp):
 
 def direction_polys(l):
     return [direction_component_poly(l, c) for c in components(l)]
+
+
+# --------------------------------------------------------------------------
+# odd-J (parity-changing) products
+# --------------------------------------------------------------------------
+
+def odd_admissible(l1, l2, l3):
+    return l1 >= 1 and l2 >= 1 and abs(l1 - l2) <= l3 <= l1 + l2 - 1 and (l1 + l2 + l3) % 2 == 1
+
+
+def odd_paths(lin, ledge, lout):
+    """Odd-J paths ordered by l3, then l1, then l2."""
+    return [(l1, l2, l3) for l3 in range(lout + 1) for l1 in range(lin + 1)
+            for l2 in range(ledge + 1) if odd_admissible(l1, l2, l3)]
+
+
+def triple_with_r(a, b):
+    """r . (grad a x grad b) as a polynomial."""
+    out = {}
+    for c in range(3):
+        i, j = (c + 1) % 3, (c + 2) % 3
+        rc = {tuple(1 if t == c else 0 for t in range(3)): Fraction(1)}
+        t = p_add(p_mul(p_diff(a, i), p_diff(b, j)), p_mul(p_diff(a, j), p_diff(b, i)), -1)
+        out = p_add(out, p_mul(rc, t))
+    return out
+
+
+def raw_odd_product_poly(l1, p1, l2, p2, l3):
+    n = (l1 + l2 - l3 - 1) // 2
+    pairs = [(p1, p2)]
+    for _ in range(n):
+        nxt = []
+        for a, b in pairs:
+            for k in range(3):
+                da, db = p_diff(a, k), p_diff(b, k)
+                if da and db:
+                    nxt.append((da, db))
+        pairs = nxt
+    out = {}
+    for a, b in pairs:
+        out = p_add(out, triple_with_r(a, b))
+    s = Fraction(factorial(l1 - n - 1) * factorial(l2 - n - 1), factorial(l1) * factorial(l2))
+    return harmonic_projection(l3, p_scale(out, s))
+
+
+@lru_cache(maxsize=None)
+def odd_path_coefficients(l1, l2, l3):
+    """K[a][b1][b2] (Fractions) of an odd-J path in independent components."""
+    n1, n2, n3 = 2 * l1 + 1, 2 * l2 + 1, 2 * l3 + 1
+    c1, c2 = components(l1), components(l2)
+    K = [[[Fraction(0)] * n2 for _ in range(n1)] for _ in range(n3)]
+    for b1 in range(n1):
+        p1 = poly_from_components(l1, {c1[b1]: Fraction(1)})
+        for b2 in range(n2):
+            p2 = poly_from_components(l2, {c2[b2]: Fraction(1)})
+            f = components_from_poly(l3, raw_odd_product_poly(l1, p1, l2, p2, l3))
+            for a in range(n3):
+                K[a][b1][b2] = f[a]
+    return K

@@ -51,10 +51,15 @@ def flit(x):
 # tables
 # ---------------------------------------------------------------------------
 
+# Odd-J (Levi-Civita) path sets are emitted under template key L + ODD_KEY.
+ODD_KEY = 16
+
+
 class Tables:
-    def __init__(self, L):
+    def __init__(self, L, odd=False):
         self.L = L
-        self.paths = A.paths(L, L, L)
+        self.odd = odd
+        self.paths = A.odd_paths(L, L, L) if odd else A.paths(L, L, L)
         self.P = len(self.paths)
         self.Pl = [sum(1 for p in self.paths if p[2] == l) for l in range(L + 1)]
         self.eta = []
@@ -68,7 +73,8 @@ class Tables:
             self.zoff.append(o)
             o += (2 * l + 1) * self.Pl[l]
         self.zrow = o
-        self.K = [A.path_coefficients(*p) for p in self.paths]
+        coeffs = A.odd_path_coefficients if odd else A.path_coefficients
+        self.K = [coeffs(*p) for p in self.paths]
         self.ypoly = {l: A.direction_polys(l) for l in range(L + 1)}
 
     def zslot(self, p, a, sum_paths=False):
@@ -397,13 +403,15 @@ MWIN = 16
 FWD_WARPS = 2
 
 
-def emit_fwd(L, G):
-    T = Tables(L)
+def emit_fwd(L, G, odd=False):
+    T = Tables(L, odd)
+    key = L + ODD_KEY if odd else L
     groups = partition_rows(T, G, ROW_WEIGHT[L])
     codes = [GroupCode(T, rows, g) for g, rows in enumerate(groups)]
     out = []
     out.append("// Generated by gen/fc_codegen.py -- do not edit.")
-    out.append("// Receiver-sorted forward, rank %d: %d paths, %d output rows, %d warp groups." % (L, T.P, T.zrow, G))
+    out.append("// Receiver-sorted forward, rank %d%s: %d paths, %d output rows, %d warp groups." %
+               (L, " odd-J paths (template key %d)" % key if odd else "", T.P, T.zrow, G))
     for c in codes:
         cost = sum(T.row_cost(p, a) for p, a in c.rows)
         out.append("//   group %d: %d rows, %d M entries, %d x rows, %d w rows, %d FMA/channel" %
@@ -411,7 +419,7 @@ def emit_fwd(L, G):
     out.append("#pragma once")
     out.append('#include "../fc_device.cuh"')
     out.append("namespace fc {")
-    out.append("template <> struct FwdMeta<%d> {" % L)
+    out.append("template <> struct FwdMeta<%d> {" % key)
     out.append("  static constexpr int G = %d;           // warp groups = warps per CTA" % G)
     out.append("  static constexpr int S = %d;           // staging ring depth (edges)" % STAGES[L])
     out.append("  static constexpr int MAXROW = %d;      // largest staged rows per edge of a group" % max(c.NROW for c in codes))
@@ -443,7 +451,7 @@ def emit_fwd(L, G):
     out.append("  static constexpr int SMEM_FLOATS = %d; // shared memory of a CTA" % total)
     out.append("};")
     for c in codes:
-        out.append(c.emit(L, G))
+        out.append(c.emit(key, G))
     out.append("}  // namespace fc")
     return "\n".join(out) + "\n", T, codes
 
@@ -692,8 +700,9 @@ VJP_STAGES = {1: 3, 2: 3, 3: 3, 4: 2, 5: 2}
 VJP_MWIN = {1: 16, 2: 16, 3: 16, 4: 8, 5: 8}
 
 
-def emit_vjp(L, G):
-    T = Tables(L)
+def emit_vjp(L, G, odd=False):
+    T = Tables(L, odd)
+    key = L + ODD_KEY if odd else L
     groups = partition_paths(T, G, lambda p: vjp_path_cost(T, p))
     codes = [VjpGroupCode(T, ps, g) for g, ps in enumerate(groups)]
     # every warp of a CTA runs the same group (one instruction stream per
@@ -705,13 +714,14 @@ def emit_vjp(L, G):
         c.mwin_off = VJP_STAGES[L] * 128 * nrow
     off = VJP_STAGES[L] * 128 * nrow + VJP_MWIN[L] * mstride
     out = ["// Generated by gen/fc_codegen.py -- do not edit.",
-           "// Receiver-sorted VJP, rank %d: %d paths, %d warp groups (whole paths)." % (L, T.P, G)]
+           "// Receiver-sorted VJP, rank %d%s: %d paths, %d warp groups (whole paths)." %
+           (L, " odd-J paths (template key %d)" % key if odd else "", T.P, G)]
     for c in codes:
         out.append("//   group %d: paths %s, %d g rows, %d M entries, %d x rows, cost %d" %
                    (c.gid, [T.paths[p] for p in c.gpaths], c.NA, c.NM, len(c.xrows),
                     sum(vjp_path_cost(T, p) for p in c.gpaths)))
     out += ["#pragma once", '#include "../fc_device.cuh"', "namespace fc {",
-            "template <> struct VjpMeta<%d> {" % L,
+            "template <> struct VjpMeta<%d> {" % key,
             "  static constexpr int G = %d;" % G,
             "  static constexpr int S = %d;" % VJP_STAGES[L],
             "  static constexpr int MWIN = %d;" % VJP_MWIN[L],
@@ -721,7 +731,7 @@ def emit_vjp(L, G):
             "  static constexpr int SMEM_FLOATS = %d;" % (4 * off),
             "};"]
     for c in codes:
-        out.append(c.emit(L, G))
+        out.append(c.emit(key, G))
     out.append("}  // namespace fc")
     return "\n".join(out) + "\n", T, codes
 
@@ -1009,8 +1019,22 @@ def emit_vvjp(L, G):
 _main_fwd = main
 
 
+# odd-J paths (ranks 1-4): 1, 4, 11, 23 paths
+ODD_NGROUPS = {1: 1, 2: 2, 3: 4, 4: 4}
+ODD_VJP_NGROUPS = {1: 1, 2: 2, 3: 4, 4: 8}
+
+
 def main():
     written = _main_fwd()
+    for L in (1, 2, 3, 4):
+        src, _, _ = emit_fwd(L, ODD_NGROUPS[L], odd=True)
+        path = os.path.join(OUTDIR, "fc_fwd_odd_L%d.cuh" % L)
+        write_if_changed(path, src)
+        written.append(path)
+        src, _, _ = emit_vjp(L, ODD_VJP_NGROUPS[L], odd=True)
+        path = os.path.join(OUTDIR, "fc_vjp_odd_L%d.cuh" % L)
+        write_if_changed(path, src)
+        written.append(path)
     for L in (1, 2, 3, 4, 5):
         src, _, _ = emit_vjp(L, VJP_NGROUPS[L])
         path = os.path.join(OUTDIR, "fc_vjp_L%d.cuh" % L)

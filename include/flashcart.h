@@ -206,6 +206,41 @@ int fc_edge_conv_vjp_rect(const fc_conv_desc *desc, int n_nodes, int n_send, int
                           const float *g, float *x_bar, float *w_bar, float *r_bar,
                           fc_stream_t stream);
 
+/* Edge convolution over the odd-J (Levi-Civita) paths: App. B, paragraph
+ * after Eq. (B1), and Sec. 7 ("Limitations") -- the same construction as
+ * Eq. (B1) with one index of each input contracted through the Levi-Civita
+ * symbol, so that parity is tracked explicitly.  An odd path (l1, l2) -> l3
+ * has l1, l2 >= 1, |l1 - l2| <= l3 <= l1 + l2 - 1 and l1 + l2 + l3 odd;
+ * with n = (l1 + l2 - l3 - 1) / 2,
+ *   f(x, y) = STF part of  eps_{pqc} x_{i.. p k1..kn} y_{k1..kn q j..}
+ * (n index pairs contracted, the free indices i.., j.., c symmetrised, the
+ * traces removed, no further factor: (1,1) -> 1 is the cross product x x y).
+ * The outputs are pseudo-tensors: under an improper rotation they pick up
+ * det(R) = -1 in addition to the rotation of a true tensor.
+ *   z[u, eta, k] = sum_{e: u_e = u} w[e, eta, k] f_eta(x[v_e, :, k], T(r-hat_e))
+ * over the odd paths, ordered by l3, then l1, then l2 (fc_conv_odd_path);
+ * output layout as for fc_edge_conv with the odd path counts P_l
+ * (fc_conv_odd_out_row components per channel; no odd path ends in rank 0,
+ * so the rank-0 block is empty, or zero with sum_paths = 1);
+ * w [n_edges][fc_conv_odd_num_paths()][C].  Ranks 1..4, otherwise the
+ * descriptor rules, graph requirements and error returns of fc_edge_conv. */
+int fc_conv_odd_num_paths(const fc_conv_desc *desc);
+int fc_conv_odd_out_row(const fc_conv_desc *desc);
+int fc_conv_odd_path(const fc_conv_desc *desc, int p, int *l1, int *l2, int *l3);
+int fc_edge_conv_odd(const fc_conv_desc *desc, int n_nodes, int n_edges,
+                     const int32_t *rowptr, const int32_t *edge_index,
+                     const float *edge_vec, const float *x, const float *w,
+                     float *z, fc_stream_t stream);
+
+/* VJP of fc_edge_conv_odd (App. C Eq. (C1) with the odd-path coefficients,
+ * summed as in Algorithm 2): x_bar, w_bar, r_bar exactly as documented for
+ * fc_edge_conv_vjp, g in the layout of fc_edge_conv_odd's output. */
+int fc_edge_conv_odd_vjp(const fc_conv_desc *desc, int n_nodes, int n_edges,
+                         const int32_t *rowptr, const int32_t *edge_index,
+                         const float *edge_vec, const float *x, const float *w,
+                         const float *g, float *x_bar, float *w_bar, float *r_bar,
+                         fc_stream_t stream);
+
 /* VJP-of-VJP of fc_edge_conv (the derivative of fc_edge_conv_vjp), App. C
  * Eq. (C2) summed over the receiver-sorted edges as in Algorithm 3, with the
  * direction tensors differentiated twice (App. C, paragraph after Eq. C2).

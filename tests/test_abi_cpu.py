@@ -82,3 +82,13 @@ def test_descriptor_rejections(fc):
     st = lib.fc_edge_conv(ct.byref(d), 1, 0, ct.c_void_p(16), None, None,
                           ct.c_void_p(20), None, ct.c_void_p(32), None)
     assert st == 5
+
+
+@pytest.mark.parametrize("L", [1, 2, 3, 4])
+def test_odd_path_queries_match_oracle(fc, L):
+    """Odd-J (Levi-Civita) path list and output row of the library against
+    the oracle's odd path rule (App. B, paragraph after Eq. B1)."""
+    from oracle import oracle as O
+    assert fc.odd_paths(L) == O.paths(L, L, L, odd=True)
+    assert fc.odd_out_row(L) == O.zrow(L, L, L, odd=True)
+    assert fc.odd_out_row(L, sum_paths=True) == (L + 1) ** 2

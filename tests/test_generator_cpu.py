@@ -43,3 +43,12 @@ def test_forward_groups_cover_every_row_once(L):
     nnz = sum(len(T.mrow(p, a)) for p in range(T.P) if not T.is_identity(p)
               for a in range(2 * T.paths[p][2] + 1))
     assert sum(c.NM for c in codes) == nnz
+
+
+@pytest.mark.parametrize("path", G.odd_paths(4, 4, 4))
+def test_odd_path_coefficients_match_oracle(path):
+    """Odd-J paths: r . (grad a x grad b) on polynomials (generator) against
+    the dense epsilon contraction (oracle)."""
+    K = np.array(G.odd_path_coefficients(*path), dtype=np.float64)
+    np.testing.assert_allclose(K, O.path_coeffs_odd(*path), atol=1e-14)
+    assert G.odd_paths(4, 4, 4) == O.paths(4, 4, 4, odd=True)
