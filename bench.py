@@ -820,8 +820,8 @@ def run_ours(args):
 def run_grid(args):
     """The pages' edge-convolution benchmark grid (1024 nodes, 64 or 128
     random neighbours, 64/128/256 channels, ranks 1-5): forward, VJP (x_bar,
-    w_bar, r_bar) and VJP-of-VJP (all four outputs, all cotangents; ranks
-    1-4) per configuration, CUDA events, inputs resident on the device
+    w_bar, r_bar) and VJP-of-VJP (all four outputs, all cotangents) per
+    configuration, CUDA events, inputs resident on the device
     (seeded, synthetic; drawn on the device)."""
     import torch
     from cartesian_tensor_products_b200 import flashcart as fc
@@ -852,10 +852,9 @@ def run_grid(args):
                 z = torch.empty((1024, zr * C), device=dev)
                 f_ms, _ = time_events(lambda: fc.edge_conv(L, rp, ei, ev, x, w, out=z), steps, 3, stream)
                 v_ms, _ = time_events(lambda: fc.edge_conv_vjp(L, rp, ei, ev, x, w, g), steps, 3, stream)
-                vv_ms = None
-                if L <= 4:      # the VJP-of-VJP is built up to rank 4
-                    vv_ms, _ = time_events(lambda: fc.edge_conv_vjp_vjp(L, rp, ei, ev, x, w, g, v_x=vx,
-                                                                        v_w=vw, v_r=vr), steps, 3, stream)
+                # rank 5 runs one launch per path group
+                vv_ms, _ = time_events(lambda: fc.edge_conv_vjp_vjp(L, rp, ei, ev, x, w, g, v_x=vx,
+                                                                    v_w=vw, v_r=vr), steps, 3, stream)
                 fb = algorithmic_bytes(1024, E, C, L, P, zr)
                 out.append({"lmax": L, "neighbours": k, "channels": C, "paths": P,
                             "fwd_ms": f_ms, "vjp_ms": v_ms, "vvjp_ms": vv_ms,

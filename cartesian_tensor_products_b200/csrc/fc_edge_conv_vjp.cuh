@@ -214,7 +214,7 @@ __device__ __forceinline__ void dispatch_vjp(int grp, const VjpArgs& a, float* s
 // runs the same code, and blocks are ordered group-major, so an SMSP mostly
 // executes one instruction stream.
 template <int L, int CC>
-__global__ void __launch_bounds__(VjpMeta<L>::WARPS * 32, 2) edge_conv_vjp_kernel(const VjpArgs a) {
+__global__ void __launch_bounds__(VjpMeta<L>::WARPS * 32, VjpMeta<L>::MINB) edge_conv_vjp_kernel(const VjpArgs a) {
   extern __shared__ __align__(16) float smem[];
   constexpr int WARPS = VjpMeta<L>::WARPS;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;

@@ -7,6 +7,19 @@ int launch_vvjp_rank1(const VvjpArgs& a, cudaStream_t s);
 int launch_vvjp_rank2(const VvjpArgs& a, cudaStream_t s);
 int launch_vvjp_rank3(const VvjpArgs& a, cudaStream_t s);
 int launch_vvjp_rank4(const VvjpArgs& a, cudaStream_t s);
+int launch_vvjp_rank5_part0(const VvjpArgs& a, cudaStream_t s);
+int launch_vvjp_rank5_part1(const VvjpArgs& a, cudaStream_t s);
+int launch_vvjp_rank5_part2(const VvjpArgs& a, cudaStream_t s);
+int launch_vvjp_rank5_part3(const VvjpArgs& a, cudaStream_t s);
+
+// rank 5: one launch per path group, in four ranges
+static int launch_vvjp_rank5(const VvjpArgs& a, cudaStream_t s) {
+  int st;
+  if ((st = launch_vvjp_rank5_part0(a, s)) != FC_OK || (st = launch_vvjp_rank5_part1(a, s)) != FC_OK ||
+      (st = launch_vvjp_rank5_part2(a, s)) != FC_OK)
+    return st;
+  return launch_vvjp_rank5_part3(a, s);
+}
 }  // namespace fc
 
 using namespace fc;
@@ -74,6 +87,7 @@ extern "C" int fc_edge_conv_vjp_vjp(const fc_conv_desc* d, int n_nodes, int n_ed
     case 2: return launch_vvjp_rank2(a, s);
     case 3: return launch_vvjp_rank3(a, s);
     case 4: return launch_vvjp_rank4(a, s);
+    case 5: return launch_vvjp_rank5(a, s);
     default: return FC_ERR_UNSUPPORTED_RANK;
   }
 }

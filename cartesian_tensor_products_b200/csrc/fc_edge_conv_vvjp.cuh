@@ -246,6 +246,42 @@ __global__ void __launch_bounds__(VvjpMeta<L>::WARPS * 32, 1) edge_conv_vvjp_ker
   dispatch_vvjp<L, CC, 0>(grp, a, smem + warp * VvjpMeta<L>::WARP_FLOATS, lane, unit);
 }
 
+// Split launches (ranks above 4, VvjpMeta<L>::SPLIT): path group g is a
+// kernel of its own, so its registers are allocated for that group alone
+// instead of for the largest group of one fused kernel; the launches of all
+// groups run back to back on the stream and add into the same outputs.
+template <int L, int CC, int g>
+__global__ void __launch_bounds__(VvjpMeta<L>::WARPS * 32, 1) edge_conv_vvjp_group_kernel(const VvjpArgs a) {
+  extern __shared__ __align__(16) float smem[];
+  using Grp = VvjpGroup<L, VvjpMeta<L>::G, g>;
+  constexpr int WARPS = VvjpMeta<L>::WARPS;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int unit = blockIdx.x * WARPS + warp;
+  if (unit >= a.n_nodes * a.ntiles) return;
+  vvjp_warp<Grp, VvjpMeta<L>::S, VvjpMeta<L>::MWIN, CC>(a, smem + warp * VvjpMeta<L>::WARP_FLOATS, lane,
+                                                          unit);
+}
+
+// launches of groups [g, G1)
+template <int L, int CC, int g, int G1>
+int launch_vvjp_groups(const VvjpArgs& a, cudaStream_t s) {
+  if constexpr (g < G1 && g < VvjpMeta<L>::G) {
+    static_assert(sizeof(float) * VvjpMeta<L>::SMEM_FLOATS <= 227 * 1024,
+                  "VJP-of-VJP kernel shared memory exceeds the 227 KB per-CTA limit of sm_100");
+    const size_t smem = sizeof(float) * (size_t)VvjpMeta<L>::SMEM_FLOATS;
+    static DeviceFlags configured;
+    if (set_smem_once(configured, edge_conv_vvjp_group_kernel<L, CC, g>, smem) != FC_OK)
+      return FC_ERR_CUDA;
+    constexpr int WARPS = VvjpMeta<L>::WARPS;
+    const long long blocks = ((long long)a.n_nodes * a.ntiles + WARPS - 1) / WARPS;
+    if (blocks > 0x7fffffffLL) return FC_ERR_ARG;
+    edge_conv_vvjp_group_kernel<L, CC, g><<<(unsigned)blocks, WARPS * 32, smem, s>>>(a);
+    if (cudaGetLastError() != cudaSuccess) return FC_ERR_CUDA;
+    return launch_vvjp_groups<L, CC, g + 1, G1>(a, s);
+  }
+  return FC_OK;
+}
+
 template <int L, int CC>
 int launch_vvjp_cc(const VvjpArgs& a, cudaStream_t s) {
   static_assert(sizeof(float) * VvjpMeta<L>::SMEM_FLOATS <= 227 * 1024,

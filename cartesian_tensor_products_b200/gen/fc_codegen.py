@@ -698,6 +698,7 @@ class VjpGroupCode:
 VJP_NGROUPS = {1: 2, 2: 4, 3: 8, 4: 8, 5: 24}
 VJP_STAGES = {1: 3, 2: 3, 3: 3, 4: 2, 5: 2}
 VJP_MWIN = {1: 16, 2: 16, 3: 16, 4: 8, 5: 8}
+VJP_MINB = {1: 2, 2: 2, 3: 2, 4: 2, 5: 2}     # resident CTAs per SM the launch bound asks for
 
 
 def emit_vjp(L, G, odd=False):
@@ -728,6 +729,7 @@ def emit_vjp(L, G, odd=False):
             "  static constexpr int P = %d;" % T.P,
             "  static constexpr int WARP_FLOATS = %d;   // shared memory of one warp" % off,
             "  static constexpr int WARPS = 4;           // receivers per CTA (same group)",
+            "  static constexpr int MINB = %d;            // CTAs per SM of the launch bound" % VJP_MINB[L],
             "  static constexpr int SMEM_FLOATS = %d;" % (4 * off),
             "};"]
     for c in codes:
@@ -980,13 +982,42 @@ class VvjpGroupCode:
 
 
 VVJP_NGROUPS = {1: 2, 2: 6, 3: 16, 4: 32}
-VVJP_STAGES = {1: 2, 2: 2, 3: 2, 4: 2}
-VVJP_MWIN = {1: 8, 2: 8, 3: 8, 4: 8}
+VVJP_STAGES = {1: 2, 2: 2, 3: 2, 4: 2, 5: 2}
+VVJP_MWIN = {1: 8, 2: 8, 3: 8, 4: 8, 5: 8}
+# Above rank 4 every path group is its own kernel launch (registers are then
+# allocated per group), and a group holds at most this many g rows.
+VVJP_SPLIT_MAX_ROWS = 12
+
+
+def partition_paths_capped(T, cost, max_rows, target):
+    """Whole paths in order of l1 (descending), cut into contiguous groups of
+    about `target` cost each, no group holding more than max_rows output rows
+    (a single path larger than that is a group of its own)."""
+    order = sorted(range(T.P), key=lambda p: (-T.paths[p][0], p))
+    groups, cur, acc, rows = [], [], 0.0, 0
+    for p in order:
+        r = 2 * T.paths[p][2] + 1
+        c = cost(p)
+        if cur and (rows + r > max_rows or acc + c / 2 > target):
+            groups.append(cur)
+            cur, acc, rows = [], 0.0, 0
+        cur.append(p)
+        acc += c
+        rows += r
+    if cur:
+        groups.append(cur)
+    return groups
 
 
 def emit_vvjp(L, G):
     T = Tables(L)
-    groups = partition_paths(T, G, lambda p: vvjp_path_cost(T, p))
+    if L > 4:
+        total = sum(vvjp_path_cost(T, p) for p in range(T.P))
+        groups = partition_paths_capped(T, lambda p: vvjp_path_cost(T, p), VVJP_SPLIT_MAX_ROWS,
+                                        total / G)
+        G = len(groups)
+    else:
+        groups = partition_paths(T, G, lambda p: vvjp_path_cost(T, p))
     codes = [VvjpGroupCode(T, ps, g) for g, ps in enumerate(groups)]
     nrow = max(c.NROW for c in codes)
     mstride = max(c.MSTRIDE for c in codes)
@@ -1003,6 +1034,7 @@ def emit_vvjp(L, G):
     out += ["#pragma once", '#include "../fc_device.cuh"', "namespace fc {",
             "template <> struct VvjpMeta<%d> {" % L,
             "  static constexpr int G = %d;" % G,
+            "  static constexpr bool SPLIT = %s;   // one launch per group" % ("true" if L > 4 else "false"),
             "  static constexpr int S = %d;" % VVJP_STAGES[L],
             "  static constexpr int MWIN = %d;" % VVJP_MWIN[L],
             "  static constexpr int P = %d;" % T.P,
@@ -1040,9 +1072,7 @@ def main():
         path = os.path.join(OUTDIR, "fc_vjp_L%d.cuh" % L)
         write_if_changed(path, src)
         written.append(path)
-        if L == 5:          # the VJP-of-VJP is built up to rank 4
-            continue
-        src, _, _ = emit_vvjp(L, VVJP_NGROUPS[L])
+        src, _, _ = emit_vvjp(L, VVJP_NGROUPS.get(L, 48))
         path = os.path.join(OUTDIR, "fc_vvjp_L%d.cuh" % L)
         write_if_changed(path, src)
         written.append(path)

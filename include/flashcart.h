@@ -79,8 +79,8 @@ int fc_version(void);
 
 /* Edge-convolution descriptor.  This build supports
  * lmax_in == lmax_edge == lmax_out in {1, 2, 3, 4, 5}, channels >= 4 and
- * a multiple of 4 (rank 5: forward and VJP without the envelope; the
- * VJP-of-VJP goes up to rank 4).  sum_paths = 0 keeps the P_l paths of each output rank
+ * a multiple of 4 (rank 5: without the envelope; its VJP-of-VJP runs one
+ * kernel launch per path group).  sum_paths = 0 keeps the P_l paths of each output rank
  * separate (z row = sum_l (2l+1) P_l C); sum_paths = 1 sums them (z row =
  * (lmax_out+1)^2 C, the node-feature layout).
  * envelope = 1 multiplies the direction tensors of edge e by

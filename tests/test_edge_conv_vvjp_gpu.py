@@ -125,17 +125,20 @@ def test_microbench_sampled_receivers(fc):
     assert np.all(np.isfinite(got[0]))
 
 
-def test_rank5_is_refused(fc):
-    """The VJP-of-VJP is built up to rank 4 (the pages split launches above
-    rank 4); rank 5 returns FC_ERR_UNSUPPORTED_RANK before any launch."""
-    t = W.tiny()
-    ei, ev = dev(t["edge_index"]), dev(t["edge_vec"])
-    rowptr = fc.build_rowptr(ei, ev, t["n_nodes"])
-    d = W.conv_inputs(t["n_nodes"], t["edge_index"], 5, 4, 3, with_grad=True)
-    with pytest.raises(fc.FlashCartError) as e:
-        fc.edge_conv_vjp_vjp(5, rowptr, ei, ev, dev(d["x"]), dev(d["w"]), dev(d["g"]),
-                             v_x=dev(d["x"]))
-    assert e.value.status == 4
+@pytest.mark.parametrize("C,degrees", [(4, None), (8, None), (128, [0, 1, 33, 2, 1, 1, 1, 1])])
+def test_rank5_split_launches(fc, C, degrees):
+    """Rank 5 runs one launch per path group (52 groups, each its own
+    kernel); every output against the oracle, on the tiny graph and, at
+    C = 128 (the compile-time-channel kernels), on a small ragged graph."""
+    if degrees is None:
+        t = W.tiny()
+        ei, ev, n = t["edge_index"], t["edge_vec"], t["n_nodes"]
+    else:
+        n = len(degrees) + 4
+        ei, ev = ragged_graph(n, degrees + [1] * 4, 6.0, 555)
+    wl = case(5, C, ei, ev, n, 57 + C)
+    got = gpu_vvjp(fc, wl)
+    check_all(got, oracle_vvjp(wl))
 
 
 def test_envelope_is_refused_and_empty_graph(fc):
