@@ -66,9 +66,15 @@ __global__ void __launch_bounds__(128) ladder_tp_kernel(int N, int C, const floa
 
 // The same product written straight into the FP32 component-major tiles of
 // the tensor-core map (PathGeom with k_l = 4, C = 128): component c of rank
-// l of node n is row n mod 128 of tile c nb + n / 128 of that rank.  A warp
-// takes 8 consecutive nodes x 4 consecutive channels, so each store of one
-// component is one full 128-byte core matrix.
+// l of node n is row n mod 128 of tile c nb + n / 128 of that rank.  A CTA
+// takes 8 consecutive nodes x 32 consecutive channels: it first stages both
+// operands (every component, as 16-byte cp.async copies: 8 per thread) in
+// shared memory, rows padded to 36 floats so that the reads below hit 32
+// distinct banks; then a warp takes the 8 nodes x 4 consecutive channels
+// (one channel per thread), so each store of one component is one full
+// 128-byte core matrix.
+constexpr int kCmPad = 36;   // floats per staged (node, component) row of 32 channels
+
 template <int L>
 __global__ void __launch_bounds__(256, 2) ladder_tp_cm_kernel(PathGeom g, const float* __restrict__ Av,
                                                               const float* __restrict__ A1,
@@ -76,19 +82,33 @@ __global__ void __launch_bounds__(256, 2) ladder_tp_cm_kernel(PathGeom g, const 
                                                               float* __restrict__ xs) {
   using TP = LadderTP<L>;
   constexpr int C = 128;
+  constexpr int NY = TP::NY;
+  extern __shared__ __align__(16) float sa[];   // [operand][component][node][kCmPad]
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int n = 8 * blockIdx.x + (lane >> 2);
-  const int k = 32 * blockIdx.y + 4 * warp + (lane & 3);
-  if (n >= g.N) return;
+  const int nb0 = 8 * blockIdx.x, k0 = 32 * blockIdx.y;
+  // stage: (operand, component, node, 16-byte chunk) of the CTA's tile
+  for (int q = threadIdx.x; q < 2 * NY * 8 * 8; q += 256) {
+    const int ch = q & 7, nn = (q >> 3) & 7, r = q >> 6;
+    const int op = r / NY, i = r - op * NY;
+    const int n = nb0 + nn;
+    const bool ok = n < g.N;
+    const float* src = (op ? A1 : Av) + ((size_t)(ok ? n : 0) * NY + i) * C + k0 + 4 * ch;
+    cp_async16(sa + ((op * NY + i) * 8 + nn) * kCmPad + 4 * ch, src, ok);
+  }
+  cp_async_commit();
   float w[TP::P];
+  const int nn = lane >> 2, kk = 4 * warp + (lane & 3);
+  const int n = nb0 + nn, k = k0 + kk;
 #pragma unroll
   for (int p = 0; p < TP::P; ++p) w[p] = __ldg(W + (size_t)p * C + k);
-  const size_t base = (size_t)n * TP::NY * C + k;
-  float a[TP::NY], b[TP::NY], o[TP::NY];
+  cp_async_wait<0>();
+  __syncthreads();
+  if (n >= g.N) return;
+  float a[NY], b[NY], o[NY];
 #pragma unroll
-  for (int i = 0; i < TP::NY; ++i) {
-    a[i] = __ldg(Av + base + (size_t)i * C);
-    b[i] = __ldg(A1 + base + (size_t)i * C);
+  for (int i = 0; i < NY; ++i) {
+    a[i] = sa[(i * 8 + nn) * kCmPad + kk];
+    b[i] = sa[((NY + i) * 8 + nn) * kCmPad + kk];
   }
   TP::fwd(a, b, w, o);
   const int cofs = (k >> 5) * 4096 + tc::core_offset(n & 127, k & 31, 128);
@@ -392,17 +412,25 @@ static int tp_dispatch(int L, int N, int C, const float* Av, const float* A1, co
   return FC_ERR_UNSUPPORTED_RANK;
 }
 
+template <int L>
+static int launch_tp_cm(const PathGeom& g, const float* Av, const float* A1, const float* W, float* xs,
+                        cudaStream_t s) {
+  const size_t smem = sizeof(float) * 2 * (L + 1) * (L + 1) * 8 * kCmPad;
+  static DeviceFlags configured;
+  if (set_smem_once(configured, ladder_tp_cm_kernel<L>, smem) != FC_OK) return FC_ERR_CUDA;
+  ladder_tp_cm_kernel<L><<<dim3((g.N + 7) / 8, 4), 256, smem, s>>>(g, Av, A1, W, xs);
+  return cudaGetLastError() == cudaSuccess ? FC_OK : FC_ERR_CUDA;
+}
+
 static int tp_cm_dispatch(int L, const PathGeom& g, const float* Av, const float* A1, const float* W,
                           float* xs, cudaStream_t s) {
-  const dim3 grid((g.N + 7) / 8, 4);
   switch (L) {
-    case 1: ladder_tp_cm_kernel<1><<<grid, 256, 0, s>>>(g, Av, A1, W, xs); break;
-    case 2: ladder_tp_cm_kernel<2><<<grid, 256, 0, s>>>(g, Av, A1, W, xs); break;
-    case 3: ladder_tp_cm_kernel<3><<<grid, 256, 0, s>>>(g, Av, A1, W, xs); break;
-    case 4: ladder_tp_cm_kernel<4><<<grid, 256, 0, s>>>(g, Av, A1, W, xs); break;
+    case 1: return launch_tp_cm<1>(g, Av, A1, W, xs, s);
+    case 2: return launch_tp_cm<2>(g, Av, A1, W, xs, s);
+    case 3: return launch_tp_cm<3>(g, Av, A1, W, xs, s);
+    case 4: return launch_tp_cm<4>(g, Av, A1, W, xs, s);
     default: return FC_ERR_UNSUPPORTED_RANK;
   }
-  return cudaGetLastError() == cudaSuccess ? FC_OK : FC_ERR_CUDA;
 }
 
 static int tp_vjp_dispatch(int L, int N, int C, const float* Av, const float* A1, const float* W,
