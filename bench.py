@@ -831,6 +831,12 @@ def run_grid(args):
     stream = torch.cuda.current_stream()
     peaks, peak_kind = load_peaks()
     steps = max(3, min(args.steps, 10))
+    props = torch.cuda.get_device_properties(dev)
+    gpu_id = str(getattr(props, "uuid", 0))
+    if gpu_id and not gpu_id.startswith("GPU-") and len(gpu_id) == 36:
+        gpu_id = "GPU-" + gpu_id
+    sampler = ClockSampler(gpu_id)
+    sampler.start()
     out = []
     for k in (64, 128):
         _, ei_np, ev_np = W.random_graph(1024, k, 20.0, 2 + k)
@@ -886,7 +892,9 @@ def run_grid(args):
                             "mix": "tcgen05 TF32x3" if C == 128 else "FP32 SIMT"})
                 del A1, pw, mw, gz, res
                 torch.cuda.empty_cache()
+    clocks = sampler.stop()
     print(json.dumps({"metric": "edge-conv grid: fwd / VJP / VJP-of-VJP ms per configuration",
+                      "clocks": clocks,
                       "unit": "ms", "n_gpus": 1, "dtype": "f32", "data": "synthetic",
                       "peak_source": peak_kind, "steps": steps,
                       "config": {"workload": "1024 nodes, random neighbours in a 20 A box; "
