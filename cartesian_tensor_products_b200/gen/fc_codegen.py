@@ -1142,19 +1142,18 @@ def emit_ladder(L):
     for p, (l1, l2, l3) in enumerate(T.paths):
         K = T.K[p]
         o.append("    { // path (%d,%d)->%d" % (l1, l2, l3))
-        # w_bar = <g, f>
-        fterms = []
-        for c in range(2 * l3 + 1):
-            for b1 in range(2 * l1 + 1):
-                for b2 in range(2 * l2 + 1):
-                    if K[c][b1][b2] != 0:
-                        fterms.append("%s*(g[%d]*(a[%d]*b[%d]))" % (flit(K[c][b1][b2]), l3 * l3 + c, l1 * l1 + b1, l2 * l2 + b2))
-        o.append("      wbar[%d] += %s;" % (p, " + ".join(fterms)))
+        # h_b1 = d<g, f>/da_b1 = sum K g_c b_b2; then abar += w h and, since f
+        # is linear in a, w_bar = <g, f> = sum_b1 a_b1 h_b1
+        hs = []
         for b1 in range(2 * l1 + 1):
             t = ["%s*(g[%d]*b[%d])" % (flit(K[c][b1][b2]), l3 * l3 + c, l2 * l2 + b2)
                  for c in range(2 * l3 + 1) for b2 in range(2 * l2 + 1) if K[c][b1][b2] != 0]
             if t:
-                o.append("      abar[%d] = fmaf(w[%d], %s, abar[%d]);" % (l1 * l1 + b1, p, " + ".join(t), l1 * l1 + b1))
+                o.append("      const float h%d = %s;" % (b1, " + ".join(t)))
+                o.append("      abar[%d] = fmaf(w[%d], h%d, abar[%d]);" % (l1 * l1 + b1, p, b1, l1 * l1 + b1))
+                hs.append(b1)
+        if hs:
+            o.append("      wbar[%d] += %s;" % (p, " + ".join("a[%d]*h%d" % (l1 * l1 + b1, b1) for b1 in hs)))
         for b2 in range(2 * l2 + 1):
             t = ["%s*(g[%d]*a[%d])" % (flit(K[c][b1][b2]), l3 * l3 + c, l1 * l1 + b1)
                  for c in range(2 * l3 + 1) for b1 in range(2 * l1 + 1) if K[c][b1][b2] != 0]
