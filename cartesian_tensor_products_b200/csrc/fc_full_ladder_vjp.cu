@@ -47,22 +47,54 @@ __device__ __forceinline__ size_t row_at(const RowLayout& g, int i, int l, int C
   return ((size_t)n * g.stride + g.off[l] + (size_t)c * g.cmul[l]) * C;
 }
 
-constexpr int kVBM = 64, kVBN = 128, kVBK = 32;
-constexpr int kVRows = 512;          // rows per CTA of the weight-gradient GEMMs
+constexpr int kVBM = 128, kVBN = 128, kVBK = 16;   // CTA tile of the row GEMMs
+constexpr int kVRows = 1024;         // rows per CTA of the weight-gradient GEMMs (split K)
 constexpr int kVChunk = 8;           // nodes per thread of the product VJP
+
+// Shared inner product of the row GEMMs: a 128 x 128 tile, 256 threads, each
+// thread 8 x 8 outputs (rows ty*4 + {0..3} and 64 + ty*4 + {0..3}, columns
+// likewise from tx), the column pairs in packed FP32x2 accumulators.  As is
+// k-major ([k][m]) and Bs is [k][n], so every thread reads two float4 of each
+// per k (broadcast within a row of the warp, consecutive across it).
+struct VTile {
+  float As[2][kVBK][kVBM];
+  float Bs[2][kVBK][kVBN];
+};
+
+__device__ __forceinline__ void vtile_mma(const VTile& sm, int buf, int tx, int ty, float2 (&acc)[8][4]) {
+#pragma unroll
+  for (int k = 0; k < kVBK; ++k) {
+    const float4 a0 = *reinterpret_cast<const float4*>(&sm.As[buf][k][ty * 4]);
+    const float4 a1 = *reinterpret_cast<const float4*>(&sm.As[buf][k][64 + ty * 4]);
+    const float4 b0 = *reinterpret_cast<const float4*>(&sm.Bs[buf][k][tx * 4]);
+    const float4 b1 = *reinterpret_cast<const float4*>(&sm.Bs[buf][k][64 + tx * 4]);
+    const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+    const float2 bv[4] = {make_float2(b0.x, b0.y), make_float2(b0.z, b0.w), make_float2(b1.x, b1.y),
+                          make_float2(b1.z, b1.w)};
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const float2 aa = make_float2(av[i], av[i]);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) acc[i][j] = __ffma2_rn(aa, bv[j], acc[i][j]);
+    }
+  }
+}
+
+// row index of accumulator i and column index of accumulator pair j
+__device__ __forceinline__ int vrow(int ty, int i) { return (i < 4 ? 0 : 64) + ty * 4 + (i & 3); }
+__device__ __forceinline__ int vcol(int tx, int j) { return (j < 2 ? 0 : 64) + tx * 4 + 2 * (j & 1); }
 
 // out_l[row][m] (+)= sum_{t < C} in[row][t] Bm_l[t][m]
 // in: layout `ai` (width C), out: layout `ao` (width ao.wid[l]),
 // Bm_l: [C][ao.wid[l]] row-major at Bm + boff[l].
 template <bool ACC>
-__global__ void __launch_bounds__(256) rows_gemm_kernel(int N, int C, int L, RowLayout ai, RowLayout ao,
-                                                        const float* __restrict__ in,
-                                                        const float* __restrict__ Bm, long long boff0,
-                                                        long long boff1, long long boff2,
-                                                        long long boff3, long long boff4,
-                                                        float* __restrict__ out) {
-  __shared__ __align__(16) float As[kVBK][kVBM + 4];
-  __shared__ __align__(16) float Bs[kVBK][kVBN + 4];
+__global__ void __launch_bounds__(256, 2) rows_gemm_kernel(int N, int C, int L, RowLayout ai, RowLayout ao,
+                                                           const float* __restrict__ in,
+                                                           const float* __restrict__ Bm, long long boff0,
+                                                           long long boff1, long long boff2,
+                                                           long long boff3, long long boff4,
+                                                           float* __restrict__ out) {
+  __shared__ __align__(16) VTile sm;
   const int l = blockIdx.z;
   if (l > L) return;
   const int R = N * (2 * l + 1);
@@ -72,57 +104,57 @@ __global__ void __launch_bounds__(256) rows_gemm_kernel(int N, int C, int L, Row
   if (r0 >= R || m0 >= W) return;
   const long long boff = l == 0 ? boff0 : l == 1 ? boff1 : l == 2 ? boff2 : l == 3 ? boff3 : boff4;
   const float* Bl = Bm + boff;
-  const int tid = threadIdx.x;
-  const int tx = tid & 15, ty = tid >> 4;   // 16 x 16 threads: 8 columns x 4 rows each
-  float acc[4][8];
+  const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
+  // global -> register prefetch of one K step: two float4 of each operand
+  const int ar0 = tid >> 2, aq = tid & 3;                 // A: rows ar0, ar0 + 64; k quad aq
+  const int bk = tid >> 5, bq = tid & 31;                 // B: k rows bk, bk + 8; n quad bq
+  const float* arow0 = r0 + ar0 < R ? in + row_at(ai, r0 + ar0, l, C) : nullptr;
+  const float* arow1 = r0 + ar0 + 64 < R ? in + row_at(ai, r0 + ar0 + 64, l, C) : nullptr;
+  float4 pa0, pa1, pb0, pb1;
+  auto fetch = [&](int t0) {
+    const int ka = t0 + 4 * aq;
+    pa0 = (arow0 && ka < C) ? __ldg(reinterpret_cast<const float4*>(arow0 + ka)) : zero4();
+    pa1 = (arow1 && ka < C) ? __ldg(reinterpret_cast<const float4*>(arow1 + ka)) : zero4();
+    const int n = m0 + 4 * bq;
+    pb0 = (t0 + bk < C && n < W) ? __ldg(reinterpret_cast<const float4*>(Bl + (size_t)(t0 + bk) * W + n)) : zero4();
+    pb1 = (t0 + bk + 8 < C && n < W) ? __ldg(reinterpret_cast<const float4*>(Bl + (size_t)(t0 + bk + 8) * W + n))
+                                     : zero4();
+  };
+  auto stash = [&](int buf) {
+    sm.As[buf][4 * aq + 0][ar0] = pa0.x; sm.As[buf][4 * aq + 1][ar0] = pa0.y;
+    sm.As[buf][4 * aq + 2][ar0] = pa0.z; sm.As[buf][4 * aq + 3][ar0] = pa0.w;
+    sm.As[buf][4 * aq + 0][ar0 + 64] = pa1.x; sm.As[buf][4 * aq + 1][ar0 + 64] = pa1.y;
+    sm.As[buf][4 * aq + 2][ar0 + 64] = pa1.z; sm.As[buf][4 * aq + 3][ar0 + 64] = pa1.w;
+    *reinterpret_cast<float4*>(&sm.Bs[buf][bk][4 * bq]) = pb0;
+    *reinterpret_cast<float4*>(&sm.Bs[buf][bk + 8][4 * bq]) = pb1;
+  };
+  float2 acc[8][4];
 #pragma unroll
-  for (int i = 0; i < 4; ++i)
+  for (int i = 0; i < 8; ++i)
 #pragma unroll
-    for (int j = 0; j < 8; ++j) acc[i][j] = 0.0f;
+    for (int j = 0; j < 4; ++j) acc[i][j] = make_float2(0.0f, 0.0f);
+  fetch(0);
+  stash(0);
+  __syncthreads();
+  int buf = 0;
   for (int t0 = 0; t0 < C; t0 += kVBK) {
-#pragma unroll
-    for (int s = 0; s < 2; ++s) {   // in: 64 rows x 32 t, stored t-major
-      const int idx = tid + s * 256;
-      const int rr = idx >> 3, tq = (idx & 7) * 4;
-      float4 v = zero4();
-      if (r0 + rr < R && t0 + tq < C)
-        v = __ldg(reinterpret_cast<const float4*>(in + row_at(ai, r0 + rr, l, C) + t0 + tq));
-      As[tq + 0][rr] = v.x; As[tq + 1][rr] = v.y; As[tq + 2][rr] = v.z; As[tq + 3][rr] = v.w;
-    }
-#pragma unroll
-    for (int s = 0; s < 4; ++s) {   // Bm: 32 t x 128 m
-      const int idx = tid + s * 256;
-      const int tt = idx >> 5, mq = (idx & 31) * 4;
-      float4 v = zero4();
-      if (t0 + tt < C && m0 + mq < W)
-        v = __ldg(reinterpret_cast<const float4*>(Bl + (size_t)(t0 + tt) * W + m0 + mq));
-      *reinterpret_cast<float4*>(&Bs[tt][mq]) = v;
-    }
+    const bool more = t0 + kVBK < C;
+    if (more) fetch(t0 + kVBK);
+    vtile_mma(sm, buf, tx, ty, acc);
+    if (more) stash(buf ^ 1);
     __syncthreads();
-#pragma unroll 8
-    for (int t = 0; t < kVBK; ++t) {
-      const float4 a = *reinterpret_cast<const float4*>(&As[t][ty * 4]);
-      const float4 b0 = *reinterpret_cast<const float4*>(&Bs[t][tx * 8]);
-      const float4 b1 = *reinterpret_cast<const float4*>(&Bs[t][tx * 8 + 4]);
-      const float av[4] = {a.x, a.y, a.z, a.w};
-      const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
-    }
-    __syncthreads();
+    buf ^= 1;
   }
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int r = r0 + ty * 4 + i;
+  for (int i = 0; i < 8; ++i) {
+    const int r = r0 + vrow(ty, i);
     if (r >= R) continue;
     float* o = out + row_at(ao, r, l, C);
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
-      const int m = m0 + tx * 8 + h * 4;
+      const int m = m0 + vcol(tx, 2 * h);
       if (m >= W) continue;
-      float4 v = make_float4(acc[i][h * 4], acc[i][h * 4 + 1], acc[i][h * 4 + 2], acc[i][h * 4 + 3]);
+      float4 v = make_float4(acc[i][2 * h].x, acc[i][2 * h].y, acc[i][2 * h + 1].x, acc[i][2 * h + 1].y);
       if (ACC) {
         const float4 p = *reinterpret_cast<const float4*>(o + m);
         v.x += p.x; v.y += p.y; v.z += p.z; v.w += p.w;
@@ -134,14 +166,14 @@ __global__ void __launch_bounds__(256) rows_gemm_kernel(int N, int C, int L, Row
 
 // Wb_l[j][m] += sum_{rows of rank l} a[row][j] b[row][m]
 // a: layout `la` (width C), b: layout `lb` (width lb.wid[l]),
-// Wb_l: [C][lb.wid[l]] row-major at Wb + woff[l].
-__global__ void __launch_bounds__(256) rows_wgrad_kernel(int N, int C, int L, RowLayout la, RowLayout lb,
-                                                         const float* __restrict__ a,
-                                                         const float* __restrict__ b, float* __restrict__ Wb,
-                                                         long long woff0, long long woff1, long long woff2,
-                                                         long long woff3, long long woff4) {
-  __shared__ __align__(16) float As[kVBK][kVBM + 4];
-  __shared__ __align__(16) float Bs[kVBK][kVBN + 4];
+// Wb_l: [C][lb.wid[l]] row-major at Wb + woff[l].  Each CTA reduces kVRows
+// rows (split K) and adds its tile with one atomic per entry.
+__global__ void __launch_bounds__(256, 2) rows_wgrad_kernel(int N, int C, int L, RowLayout la, RowLayout lb,
+                                                            const float* __restrict__ a,
+                                                            const float* __restrict__ b, float* __restrict__ Wb,
+                                                            long long woff0, long long woff1, long long woff2,
+                                                            long long woff3, long long woff4) {
+  __shared__ __align__(16) VTile sm;
   const int l = blockIdx.z;
   if (l > L) return;
   const int R = N * (2 * l + 1);
@@ -154,56 +186,52 @@ __global__ void __launch_bounds__(256) rows_wgrad_kernel(int N, int C, int L, Ro
   const int m0 = (blockIdx.y / jt) * kVBN;
   if (m0 >= W) return;
   const long long woff = l == 0 ? woff0 : l == 1 ? woff1 : l == 2 ? woff2 : l == 3 ? woff3 : woff4;
-  const int tid = threadIdx.x;
-  const int tx = tid & 15, ty = tid >> 4;
-  float acc[4][8];
+  const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
+  const int kr = tid >> 5, q = tid & 31;   // rows kr, kr + 8 of the K step; column quad q
+  float4 pa0, pa1, pb0, pb1;
+  auto fetch = [&](int t0) {
+    const int ra = t0 + kr, rb = t0 + kr + 8;
+    const int j = j0 + 4 * q, m = m0 + 4 * q;
+    pa0 = (ra < i1 && j < C) ? __ldg(reinterpret_cast<const float4*>(a + row_at(la, ra, l, C) + j)) : zero4();
+    pa1 = (rb < i1 && j < C) ? __ldg(reinterpret_cast<const float4*>(a + row_at(la, rb, l, C) + j)) : zero4();
+    pb0 = (ra < i1 && m < W) ? __ldg(reinterpret_cast<const float4*>(b + row_at(lb, ra, l, C) + m)) : zero4();
+    pb1 = (rb < i1 && m < W) ? __ldg(reinterpret_cast<const float4*>(b + row_at(lb, rb, l, C) + m)) : zero4();
+  };
+  auto stash = [&](int buf) {
+    *reinterpret_cast<float4*>(&sm.As[buf][kr][4 * q]) = pa0;
+    *reinterpret_cast<float4*>(&sm.As[buf][kr + 8][4 * q]) = pa1;
+    *reinterpret_cast<float4*>(&sm.Bs[buf][kr][4 * q]) = pb0;
+    *reinterpret_cast<float4*>(&sm.Bs[buf][kr + 8][4 * q]) = pb1;
+  };
+  float2 acc[8][4];
 #pragma unroll
-  for (int i = 0; i < 4; ++i)
+  for (int i = 0; i < 8; ++i)
 #pragma unroll
-    for (int j = 0; j < 8; ++j) acc[i][j] = 0.0f;
+    for (int j = 0; j < 4; ++j) acc[i][j] = make_float2(0.0f, 0.0f);
+  fetch(i0);
+  stash(0);
+  __syncthreads();
+  int buf = 0;
   for (int t0 = i0; t0 < i1; t0 += kVBK) {
-#pragma unroll
-    for (int s = 0; s < 2; ++s) {   // a: 32 rows x 64 j
-      const int idx = tid + s * 256;
-      const int tt = idx >> 4, jq = (idx & 15) * 4;
-      float4 v = zero4();
-      if (t0 + tt < i1 && j0 + jq < C)
-        v = __ldg(reinterpret_cast<const float4*>(a + row_at(la, t0 + tt, l, C) + j0 + jq));
-      *reinterpret_cast<float4*>(&As[tt][jq]) = v;
-    }
-#pragma unroll
-    for (int s = 0; s < 4; ++s) {   // b: 32 rows x 128 m
-      const int idx = tid + s * 256;
-      const int tt = idx >> 5, mq = (idx & 31) * 4;
-      float4 v = zero4();
-      if (t0 + tt < i1 && m0 + mq < W)
-        v = __ldg(reinterpret_cast<const float4*>(b + row_at(lb, t0 + tt, l, C) + m0 + mq));
-      *reinterpret_cast<float4*>(&Bs[tt][mq]) = v;
-    }
+    const bool more = t0 + kVBK < i1;
+    if (more) fetch(t0 + kVBK);
+    vtile_mma(sm, buf, tx, ty, acc);
+    if (more) stash(buf ^ 1);
     __syncthreads();
-#pragma unroll 8
-    for (int t = 0; t < kVBK; ++t) {
-      const float4 av4 = *reinterpret_cast<const float4*>(&As[t][ty * 4]);
-      const float4 b0 = *reinterpret_cast<const float4*>(&Bs[t][tx * 8]);
-      const float4 b1 = *reinterpret_cast<const float4*>(&Bs[t][tx * 8 + 4]);
-      const float av[4] = {av4.x, av4.y, av4.z, av4.w};
-      const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
-    }
-    __syncthreads();
+    buf ^= 1;
   }
   float* Wl = Wb + woff;
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int j = j0 + ty * 4 + i;
+  for (int i = 0; i < 8; ++i) {
+    const int j = j0 + vrow(ty, i);
     if (j >= C) continue;
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const int m = m0 + tx * 8 + u;
-      if (m < W) atomicAdd(Wl + (size_t)j * W + m, acc[i][u]);
+    for (int h = 0; h < 4; ++h) {
+      const int m = m0 + vcol(tx, h);
+      if (m < W) {
+        atomicAdd(Wl + (size_t)j * W + m, acc[i][h].x);
+        atomicAdd(Wl + (size_t)j * W + m + 1, acc[i][h].y);
+      }
     }
   }
 }
