@@ -143,10 +143,19 @@ int launch_wgrad_tc(int L, int N, const float* as, const float* bs, float* Mbar,
 // core-matrix layout), and rank l's tiles start at float pg_xbase(l) of the
 // operand buffer.  The map of rank l ([128][K]) is split into TF32: k_l hi
 // then k_l lo blocks of the same layout from float pg_wbase(l).
+//
+// A rank may carry several maps (e_l > 1: one per path into rank l, the
+// full-ladder VJP's B_bar = p_bar Wq_l, path by path): each (map, tile) pair
+// is a unit of work, the maps of rank l one after the other, and map e of
+// rank l writes row (node n, component c) at row n orow + ooff(l) + c e_l + e
+// of the output (orow = NY and e_l = 1: the node layout; e_l = P_l and orow =
+// the convolution's output row: one slot per path).
 struct PathGeom {
   int N, NY, L, nb;
   int t1, t2, t3, t4, t5;   // first tile of ranks 1..5 (t_{L+1} = all tiles)
   int k0, k1, k2, k3, k4;   // K chunks per row of ranks 0..4
+  int e0, e1, e2, e3, e4;   // maps of ranks 0..4
+  int orow;                 // output row length (in 128-channel rows)
 };
 __host__ __device__ __forceinline__ int pg_ts(const PathGeom& g, int l) {
   return l <= 0 ? 0 : l == 1 ? g.t1 : l == 2 ? g.t2 : l == 3 ? g.t3 : l == 4 ? g.t4 : g.t5;
@@ -165,20 +174,38 @@ __host__ __device__ __forceinline__ long long pg_xbase(const PathGeom& g, int l)
     if (r < l) b += (long long)(pg_ts(g, r + 1) - pg_ts(g, r)) * pg_kc(g, r) * 4096;
   return b;
 }
+__host__ __device__ __forceinline__ int pg_pe(const PathGeom& g, int l) {
+  return l == 0 ? g.e0 : l == 1 ? g.e1 : l == 2 ? g.e2 : l == 3 ? g.e3 : g.e4;
+}
+// maps of rank l start at float pg_wbase(l) (each map: k_l hi then k_l lo blocks)
 __host__ __device__ __forceinline__ long long pg_wbase(const PathGeom& g, int l) {
   long long b = 0;
 #pragma unroll
   for (int r = 0; r < 5; ++r)
-    if (r < l) b += (long long)pg_kc(g, r) * 8192;
+    if (r < l) b += (long long)pg_kc(g, r) * pg_pe(g, r) * 8192;
   return b;
 }
-// kc[l] = K chunks per row of rank l (l <= L <= 4)
+// first output row of rank l within a node's row
+__host__ __device__ __forceinline__ int pg_ooff(const PathGeom& g, int l) {
+  int o = 0;
+#pragma unroll
+  for (int r = 0; r < 5; ++r)
+    if (r < l) o += (2 * r + 1) * pg_pe(g, r);
+  return o;
+}
+// kc[l] = K chunks per row of rank l (l <= L <= 4); one map per rank, node-layout output
 PathGeom path_geom(int L, int N, const int* kc);
+// the same with pe[l] maps of rank l and path-slot output rows
+PathGeom path_geom_maps(int L, int N, const int* kc, const int* pe);
 // natural [N][(L+1)^2][128] -> FP32 operand tiles with k_l = 4 (the map of phi_1)
 int launch_path_split_rows(const PathGeom& g, const float* in, float* xs, cudaStream_t s);
 // the maps, rank l's ([128][32 k_l] row-major) at W + 4096 sum_{l'<l} k_l',
 // -> split blocks at ws + pg_wbase(l)
 int launch_path_split_map(const PathGeom& g, const float* W, float* ws, cudaStream_t s);
+// k_l = 4, e_l = P_l maps per rank: map e of rank l is the transposed block e
+// of Wq_l = [128][P_l 128] (rank l at Wq + 128 128 sum_{l'<l} P_l'):
+// A(j', t) = Wq_l[t][e 128 + j']
+int launch_path_split_map_t(const PathGeom& g, const float* Wq, float* ws, cudaStream_t s);
 // out[n][l^2 + c][j] = sum_k W_l[j][k] x_l[(n, c)][k]
 int launch_path_mix_tc(const PathGeom& g, const float* xs, const float* ws, float* out, cudaStream_t s);
 

@@ -16,8 +16,10 @@
 // ([N][sum_l (2l+1) P_l][C], slot zoff(l) + c P_l + eta), where the P_l C
 // inputs of one (node, component) row of rank l form one contiguous run, so
 // every map is a GEMM over the rows of a rank: the register-tiled FP32
-// kernels below (64 rows x 128 columns per CTA; 4 x 8 outputs per thread).
-// The weight gradients reduce over the rows (512-row chunks per CTA, one
+// kernels below (128 x 128 per CTA, 8 x 8 outputs per thread), except that at
+// C = 128 the transposed map B_bar = p_bar Wq_l runs on the tcgen05 tensor
+// cores (fc_mix_tc.cu's path map with one map per path).
+// The weight gradients reduce over the rows (1024-row chunks per CTA, one
 // atomic add per entry per chunk; not bitwise reproducible).  The products
 // are channel-diagonal: one thread per channel walks a chunk of nodes with
 // generated straight-line code (exact coefficients).
@@ -411,12 +413,28 @@ int check_full_vjp_desc(const fc_ladder_desc* d) {
 
 using namespace fc;
 
+// Tensor-core geometry of B_bar = p_bar Wq_l at C = 128: the rows of p_bar as
+// FP32 component-major tiles (K = 128, k_l = 4) and P_l maps per rank, one per
+// path, each writing its path's slot of the convolution's output layout.
+static PathGeom bbar_geom(int L, int N) {
+  int Pl[6] = {0, 0, 0, 0, 0, 0};
+  rank_path_counts(L, Pl);
+  const int kc[5] = {4, 4, 4, 4, 4};
+  return path_geom_maps(L, N, kc, Pl);
+}
+
 extern "C" size_t fc_full_ladder_vjp_workspace_size(const fc_ladder_desc* d, int n_nodes) {
   if (check_full_vjp_desc(d) != FC_OK || n_nodes < 0) return 0;
   const size_t plane = (size_t)n_nodes * (d->lmax + 1) * (d->lmax + 1) * d->channels;
   const size_t zplane = (size_t)n_nodes * out_row(d->lmax, 0) * d->channels;
   // two running gradients; one step's products and their gradient
-  return sizeof(float) * (2 * plane + (d->order > 1 ? 2 * zplane : 0));
+  size_t f = 2 * plane + (d->order > 1 ? 2 * zplane : 0);
+  // tensor cores: p_bar as operand tiles and one step's split maps
+  if (d->order > 1 && mix_tc_supported(d->lmax, d->channels)) {
+    const PathGeom g = bbar_geom(d->lmax, n_nodes);
+    f += (size_t)(pg_xbase(g, g.L + 1) + pg_wbase(g, g.L + 1));
+  }
+  return sizeof(float) * f;
 }
 
 extern "C" int fc_full_ladder_vjp(const fc_ladder_desc* d, int n_nodes, const float* A, const float* W1,
@@ -450,6 +468,10 @@ extern "C" int fc_full_ladder_vjp(const fc_ladder_desc* d, int n_nodes, const fl
   float* pbn = pb + plane;
   float* Bq = pbn + plane;
   float* Bbar = Bq + zplane;
+  const bool tc = order > 1 && mix_tc_supported(L, C);
+  const PathGeom gb = bbar_geom(L, n_nodes);
+  float* xs = Bbar + zplane;                      // tensor cores: p_bar tiles
+  float* wsm = tc ? xs + pg_xbase(gb, gb.L + 1) : nullptr;   // and the split maps
   int Pl[6] = {0, 0, 0, 0, 0, 0};
   rank_path_counts(L, Pl);
   RowLayout nl = node_layout(L), pl = path_layout(L, Pl);
@@ -476,9 +498,17 @@ extern "C" int fc_full_ladder_vjp(const fc_ladder_desc* d, int n_nodes, const fl
     const float* Wqq = Wq + (size_t)(q - 2) * wq_step;
     float* Wqb = Wq_bar + (size_t)(q - 2) * wq_step;
     if ((st = full_tp_zrow_dispatch(L, n_nodes, C, phi_prev, A, Bq, s)) != FC_OK ||
-        (st = launch_rows_wgrad(n_nodes, C, L, nl, pl, pb, Bq, Wqb, qoff, s)) != FC_OK ||
-        (st = launch_rows_gemm<false>(n_nodes, C, L, nl, pl, pb, Wqq, qoff, Bbar, s)) != FC_OK ||
-        (st = full_tp_vjp_dispatch(L, n_nodes, C, phi_prev, A, Bbar, gz, pbn, A_bar, s)) != FC_OK)
+        (st = launch_rows_wgrad(n_nodes, C, L, nl, pl, pb, Bq, Wqb, qoff, s)) != FC_OK)
+      return st;
+    if (tc) {   // B_bar on tcgen05, one map per path (three-term TF32 split)
+      if ((st = launch_path_split_rows(gb, pb, xs, s)) != FC_OK ||
+          (st = launch_path_split_map_t(gb, Wqq, wsm, s)) != FC_OK ||
+          (st = launch_path_mix_tc(gb, xs, wsm, Bbar, s)) != FC_OK)
+        return st;
+    } else if ((st = launch_rows_gemm<false>(n_nodes, C, L, nl, pl, pb, Wqq, qoff, Bbar, s)) != FC_OK) {
+      return st;
+    }
+    if ((st = full_tp_vjp_dispatch(L, n_nodes, C, phi_prev, A, Bbar, gz, pbn, A_bar, s)) != FC_OK)
       return st;
     float* t = pb;
     pb = pbn;

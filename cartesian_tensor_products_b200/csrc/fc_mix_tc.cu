@@ -609,24 +609,47 @@ constexpr size_t kPmSmemBytes =
     sizeof(float) * (kTcStages * kPmStageFloats + 2 * kPmCvtFloats) + 8 * 16 + 8;
 static_assert(kPmSmemBytes <= 232448, "shared memory per CTA");
 
+// Units of work: (map e, tile t) pairs, rank by rank, the maps of a rank one
+// after the other (a map is loaded once per run of the rank's tiles); a unit
+// of rank l is k_l K chunks.
+__host__ __device__ __forceinline__ int pg_units(const PathGeom& g, int l) {
+  return (pg_ts(g, l + 1) - pg_ts(g, l)) * pg_pe(g, l);
+}
+
 __device__ __forceinline__ long long pg_chunks_before(const PathGeom& g, int l) {
   long long c = 0;
 #pragma unroll
   for (int r = 0; r < 5; ++r)
-    if (r < l) c += (long long)(pg_ts(g, r + 1) - pg_ts(g, r)) * pg_kc(g, r);
+    if (r < l) c += (long long)pg_units(g, r) * pg_kc(g, r);
   return c;
 }
 
-// first tile that starts at or after K chunk P of the whole operand
-__device__ __forceinline__ int pg_tile_at(const PathGeom& g, long long P) {
+// first unit that starts at or after K chunk P of the whole run
+__device__ __forceinline__ int pg_unit_at(const PathGeom& g, long long P) {
   long long cum = 0;
+  int us = 0;
   for (int l = 0; l <= g.L; ++l) {
-    const int nt = pg_ts(g, l + 1) - pg_ts(g, l), kc = pg_kc(g, l);
-    const long long cl = (long long)nt * kc;
-    if (P < cum + cl) return pg_ts(g, l) + (int)((P - cum + kc - 1) / kc);
+    const int nu = pg_units(g, l), kc = pg_kc(g, l);
+    const long long cl = (long long)nu * kc;
+    if (P < cum + cl) return us + (int)((P - cum + kc - 1) / kc);
     cum += cl;
+    us += nu;
   }
-  return pg_ts(g, g.L + 1);
+  return us;
+}
+
+// unit u -> rank l, tile t, map e
+__device__ __forceinline__ void pg_unit(const PathGeom& g, int u, int& l, int& t, int& e) {
+  int us = 0;
+  l = 0;
+  while (l < g.L && u >= us + pg_units(g, l)) {
+    us += pg_units(g, l);
+    ++l;
+  }
+  const int nt = pg_ts(g, l + 1) - pg_ts(g, l);
+  const int v = u - us;
+  e = v / nt;
+  t = pg_ts(g, l) + (v - e * nt);
 }
 
 // natural [N][NY][128] -> component-major FP32 operand tiles with k_l = 4
@@ -675,6 +698,36 @@ __global__ void __launch_bounds__(256) path_split_map_kernel(PathGeom g, const f
   }
 }
 
+// Map e of rank l (k_l = 4): A(j', t) = Wq_l[t][e 128 + j'], the transposed
+// block e of Wq_l = [128][P_l 128] at Wq + 16384 sum_{l'<l} P_l', split to hi /
+// lo blocks at ws + pg_wbase(l) + e 8 4096.  One CTA per (K chunk, map, rank).
+__global__ void __launch_bounds__(256) path_split_map_t_kernel(PathGeom g, const float* __restrict__ Wq,
+                                                               float* __restrict__ ws) {
+  const int c = blockIdx.x, e = blockIdx.y, l = blockIdx.z;
+  if (l > g.L || e >= pg_pe(g, l)) return;
+  long long qoff = 0;
+  for (int r = 0; r < l; ++r) qoff += 16384LL * pg_pe(g, r);
+  const int row = kTcC * pg_pe(g, l);   // floats per row of Wq_l
+  const float* Wl = Wq + qoff;
+  float* hi = ws + pg_wbase(g, l) + (long long)e * 8 * kTcBlockFloats + (size_t)c * kTcBlockFloats;
+#pragma unroll
+  for (int it = 0; it < 4; ++it) {
+    const int idx = it * 256 + threadIdx.x;   // 0 .. 1023
+    const int j = idx & (kTcC - 1), q = idx >> 7;   // output column j', group of 4 inputs
+    const int t = 32 * c + 4 * q;
+    float4 v;
+    v.x = __ldg(Wl + (size_t)(t + 0) * row + e * kTcC + j);
+    v.y = __ldg(Wl + (size_t)(t + 1) * row + e * kTcC + j);
+    v.z = __ldg(Wl + (size_t)(t + 2) * row + e * kTcC + j);
+    v.w = __ldg(Wl + (size_t)(t + 3) * row + e * kTcC + j);
+    uint4 h, w;
+    split4(v, h, w);
+    const int off = tc::core_offset(j, 4 * q, kTcC);
+    *reinterpret_cast<uint4*>(hi + off) = h;
+    *reinterpret_cast<uint4*>(hi + 4 * kTcBlockFloats + off) = w;
+  }
+}
+
 __global__ void __launch_bounds__(kTcThreads, 1) path_mix_tc_kernel(PathGeom geo,
                                                                     const float* __restrict__ xs,
                                                                     const float* __restrict__ ws,
@@ -693,8 +746,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) path_mix_tc_kernel(PathGeom geo
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const long long total = pg_chunks_before(geo, geo.L + 1);
-  const int t_begin = pg_tile_at(geo, (long long)blockIdx.x * total / gridDim.x);
-  const int t_end = pg_tile_at(geo, (long long)(blockIdx.x + 1) * total / gridDim.x);
+  const int u_begin = pg_unit_at(geo, (long long)blockIdx.x * total / gridDim.x);
+  const int u_end = pg_unit_at(geo, (long long)(blockIdx.x + 1) * total / gridDim.x);
 
   if (warp == 0) tc::tmem_alloc(tmem_slot, 2 * kTcRows);
   if (tid == 0) {
@@ -722,10 +775,12 @@ __global__ void __launch_bounds__(kTcThreads, 1) path_mix_tc_kernel(PathGeom geo
     // ---------------- bulk-copy producer ----------------
     if (lane == 0) {
       int g = 0;
-      for (int t = t_begin; t < t_end && !fail; ++t) {
-        const int l = pg_rank(geo, t), kc = pg_kc(geo, l);
+      for (int u = u_begin; u < u_end && !fail; ++u) {
+        int l, t, e;
+        pg_unit(geo, u, l, t, e);
+        const int kc = pg_kc(geo, l);
         const float* xt = xs + pg_xbase(geo, l) + (long long)(t - pg_ts(geo, l)) * kc * kTcBlockFloats;
-        const float* wt = ws + pg_wbase(geo, l);
+        const float* wt = ws + pg_wbase(geo, l) + (long long)e * 2 * kc * kTcBlockFloats;
         const size_t lo = (size_t)kc * kTcBlockFloats;
         for (int c = 0; c < kc; ++c, ++g) {
           const int s = g % kTcStages;
@@ -754,8 +809,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) path_mix_tc_kernel(PathGeom geo
       constexpr uint32_t idesc = tc::idesc_tf32(kTcC, kTcRows);
       constexpr uint32_t kLbo = kTcRows * 16, kSbo = 128;
       int g = 0, h = 0;   // chunks and accumulator groups issued
-      for (int t = t_begin; t < t_end && !fail; ++t) {
-        const int kc = pg_kc(geo, pg_rank(geo, t));
+      for (int u = u_begin; u < u_end && !fail; ++u) {
+        int l, t, e;
+        pg_unit(geo, u, l, t, e);
+        const int kc = pg_kc(geo, l);
         for (int c = 0; c < kc; ++c, ++g) {
           const uint32_t d_tmem = tmem + (uint32_t)(h & 1) * kTcRows;
           if (c % kPmGroup == 0) {   // the epilogue has added group h - 2
@@ -802,8 +859,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) path_mix_tc_kernel(PathGeom geo
     // ---------------- converter: FP32 chunk -> TF32 hi / lo blocks ----------------
     const int ct = tid - 64;   // 0 .. 63
     int g = 0;
-    for (int t = t_begin; t < t_end && !fail; ++t) {
-      const int kc = pg_kc(geo, pg_rank(geo, t));
+    for (int u = u_begin; u < u_end && !fail; ++u) {
+      int l, t, e;
+      pg_unit(geo, u, l, t, e);
+      const int kc = pg_kc(geo, l);
       for (int c = 0; c < kc; ++c, ++g) {
         const int s = g % kTcStages, b = g & 1;
         if (!tc::bar_wait(&stage_full[s], (g / kTcStages) & 1, lim) ||
@@ -840,8 +899,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) path_mix_tc_kernel(PathGeom geo
     const int ew = warp - 4;
     const int j = 32 * ew + lane;
     int h = 0;
-    for (int t = t_begin; t < t_end && !fail; ++t) {
-      const int l = pg_rank(geo, t);
+    for (int u = u_begin; u < u_end && !fail; ++u) {
+      int l, t, e;
+      pg_unit(geo, u, l, t, e);
       const int kc = pg_kc(geo, l);
       const int tr = t - pg_ts(geo, l);
       const int cmc = tr / geo.nb;                     // the tile's component
@@ -865,8 +925,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) path_mix_tc_kernel(PathGeom geo
         tc::bar_arrive(&acc_free[h & 1]);
       }
       if (fail) break;
-      float* o = out + ((size_t)cmn * geo.NY + l * l + cmc) * kTcC + j;
-      const size_t step = (size_t)geo.NY * kTcC;
+      float* o = out + ((size_t)cmn * geo.orow + pg_ooff(geo, l) + (size_t)cmc * pg_pe(geo, l) + e) * kTcC + j;
+      const size_t step = (size_t)geo.orow * kTcC;
       const int nr = min(kTcRows, geo.N - cmn);
 #pragma unroll
       for (int r = 0; r < kTcRows; ++r) {
@@ -974,6 +1034,18 @@ PathGeom path_geom(int L, int N, const int* kc) {
   }
   g.t1 = ts[1]; g.t2 = ts[2]; g.t3 = ts[3]; g.t4 = ts[4]; g.t5 = ts[5];
   g.k0 = k[0]; g.k1 = k[1]; g.k2 = k[2]; g.k3 = k[3]; g.k4 = k[4];
+  g.e0 = g.e1 = g.e2 = g.e3 = g.e4 = 1;
+  g.orow = g.NY;
+  return g;
+}
+
+PathGeom path_geom_maps(int L, int N, const int* kc, const int* pe) {
+  PathGeom g = path_geom(L, N, kc);
+  int e[5] = {0, 0, 0, 0, 0};
+  for (int l = 0; l <= L && l < 5; ++l) e[l] = pe[l];
+  g.e0 = e[0]; g.e1 = e[1]; g.e2 = e[2]; g.e3 = e[3]; g.e4 = e[4];
+  g.orow = 0;
+  for (int l = 0; l <= L && l < 5; ++l) g.orow += (2 * l + 1) * e[l];
   return g;
 }
 
@@ -994,10 +1066,22 @@ int launch_path_split_map(const PathGeom& g, const float* W, float* ws, cudaStre
   return cudaGetLastError() == cudaSuccess ? FC_OK : FC_ERR_CUDA;
 }
 
+int launch_path_split_map_t(const PathGeom& g, const float* Wq, float* ws, cudaStream_t s) {
+  int emax = 0;
+  for (int l = 0; l <= g.L; ++l) {
+    if (pg_kc(g, l) != 4) return FC_ERR_ARG;
+    emax = pg_pe(g, l) > emax ? pg_pe(g, l) : emax;
+  }
+  if (emax == 0) return FC_OK;
+  path_split_map_t_kernel<<<dim3(4, emax, g.L + 1), 256, 0, s>>>(g, Wq, ws);
+  return cudaGetLastError() == cudaSuccess ? FC_OK : FC_ERR_CUDA;
+}
+
 int launch_path_mix_tc(const PathGeom& g, const float* xs, const float* ws, float* out, cudaStream_t s) {
   if (g.L < 0 || g.L > 4) return FC_ERR_UNSUPPORTED_RANK;
   if (set_smem_once(g_pm_smem_set, path_mix_tc_kernel, kPmSmemBytes) != FC_OK) return FC_ERR_CUDA;
-  const int T = pg_ts(g, g.L + 1);
+  int T = 0;   // units of work
+  for (int l = 0; l <= g.L; ++l) T += pg_units(g, l);
   if (T == 0) return FC_OK;
   const int sms = device_sm_count();
   const int grid = T < sms ? T : sms;
