@@ -526,11 +526,12 @@ def extra_rows(fc, W, dev, stream, peaks, fp32_peak, steps, select=ROW_NAMES):
             "ms": msf, "ms_min": mnf,
             "roofline": composite_bound(peaks, fp32_peak, fbf, tp_fl, 3 * mix_fl, msf, mix_fl + tp_fl),
             "l2_flush": "256 MB written before every call"}
-        # VJP: per step the map's weight gradient (FP32 SIMT) and the transposed
-        # map B_bar (tcgen05, three TF32 products; phi_1's transposed map FP32),
-        # each the forward map's flops; the products recomputed and
-        # differentiated (3 x the product flops); A, phi_1..phi_{order-1}, gz
-        # read, A_bar written
+        # VJP: per step the map's weight gradient and the transposed map B_bar,
+        # each the forward map's flops, on tcgen05 (three TF32 products each);
+        # phi_1's weight gradient on tcgen05 too, its transposed map (A_bar +=
+        # p_bar W1) FP32 SIMT; the products recomputed and differentiated
+        # (3 x the product flops); A, phi_1..phi_{order-1}, gz read, A_bar
+        # written
         st_f, _ = fc.full_ladder(Lf, of, A, W1, Wq, workspace=wsf)
         gzf = torch.from_numpy(fd["gz"]).to(dev)
         wsv = torch.empty(fc.lib().fc_full_ladder_vjp_workspace_size(
@@ -542,11 +543,11 @@ def extra_rows(fc, W, dev, stream, peaks, fp32_peak, steps, select=ROW_NAMES):
         rows["full_ladder_vjp"] = {
             "nodes_per_s": Nf / (msv * 1e-3), "cpu_baseline": cbfv,
             "peak_alloc_bytes": peak_alloc(lambda: fc.full_ladder_vjp(Lf, of, A, W1, Wq, st_f, gzf)),
-            "workload": "same full ladder, A_bar + W1_bar + Wq_bar (B_bar maps on tcgen05, "
-                        "weight gradients FP32 SIMT)",
+            "workload": "same full ladder, A_bar + W1_bar + Wq_bar (B_bar maps and weight "
+                        "gradients on tcgen05)",
             "ms": msv, "ms_min": mnv,
-            "roofline": composite_bound(peaks, fp32_peak, vbf, mix_fl + map1_fl + 3 * tp_fl,
-                                        3 * (mix_fl - map1_fl), msv, 2 * mix_fl + 3 * tp_fl),
+            "roofline": composite_bound(peaks, fp32_peak, vbf, map1_fl + 3 * tp_fl,
+                                        3 * mix_fl + 3 * (mix_fl - map1_fl), msv, 2 * mix_fl + 3 * tp_fl),
             "l2_flush": "256 MB written before every call"}
         del A, W1, Wq, wsf, wsv, st_f, gzf
         torch.cuda.empty_cache()

@@ -129,10 +129,6 @@ int launch_mix_tc_split_rows(int L, int N, const float* in, float* xs, cudaStrea
 int launch_mix_tc_split_matrix(int mode, int L, const float* M, float* ws, cudaStream_t s);
 // out[n][l^2 + c][j] = sum_t A_l(j, t) x[n][l^2 + c][t] for every rank l
 int launch_mix_tc(int L, int N, const float* xs, const float* ws, float* out, cudaStream_t s);
-// natural -> transposed split tiles (channels x rows, K-major along rows)
-int launch_mix_tc_split_cols(int L, int N, const float* in, float* xs, cudaStream_t s);
-// Mbar[l][k][j] += sum over the rows of rank l of a[row][k] b[row][j] (both transposed split)
-int launch_wgrad_tc(int L, int N, const float* as, const float* bs, float* Mbar, cudaStream_t s);
 
 // Tensor-core path + channel map of the full ladder (fc_mix_tc.cu), C = 128.
 // Rows of rank l (node n, component c) carry K = 32 k_l inputs (k_l = 4 P_l:
@@ -208,5 +204,34 @@ int launch_path_split_map(const PathGeom& g, const float* W, float* ws, cudaStre
 int launch_path_split_map_t(const PathGeom& g, const float* Wq, float* ws, cudaStream_t s);
 // out[n][l^2 + c][j] = sum_k W_l[j][k] x_l[(n, c)][k]
 int launch_path_mix_tc(const PathGeom& g, const float* xs, const float* ws, float* out, cudaStream_t s);
+
+// Weight gradient of a per-rank map from FP32 rows on tcgen05 (fc_mix_tc.cu):
+//   Wb_l[j][e 128 + k] += sum_{rows i = (n, c) of rank l} a[i][j] b_e[i][k]
+// C = 128.  Row (n, c) of a is at float (n sa + l^2 + c) 128 (node layout);
+// row (n, c) of b_e at (n sb + ob_l + c pe_l + e) 128 (e < pe_l: the node
+// layout with pe = 1, or the path slots of the convolution's output layout);
+// Wb_l is [128][pe_l 128] row-major at Wb + wo_l.  Adds atomically.
+struct WgGeom {
+  int N, L, sa, sb;
+  int ob0, ob1, ob2, ob3, ob4;
+  int pe0, pe1, pe2, pe3, pe4;
+  int wo0, wo1, wo2, wo3, wo4;
+};
+__host__ __device__ __forceinline__ int wg_ob(const WgGeom& g, int l) {
+  return l == 0 ? g.ob0 : l == 1 ? g.ob1 : l == 2 ? g.ob2 : l == 3 ? g.ob3 : g.ob4;
+}
+__host__ __device__ __forceinline__ int wg_pe(const WgGeom& g, int l) {
+  return l == 0 ? g.pe0 : l == 1 ? g.pe1 : l == 2 ? g.pe2 : l == 3 ? g.pe3 : g.pe4;
+}
+__host__ __device__ __forceinline__ int wg_wo(const WgGeom& g, int l) {
+  return l == 0 ? g.wo0 : l == 1 ? g.wo1 : l == 2 ? g.wo2 : l == 3 ? g.wo3 : g.wo4;
+}
+int launch_rows_wgrad_tc(const WgGeom& g, const float* a, const float* b, float* Wb, cudaStream_t s);
+// both operands in the node layout, one [128][128] block per rank at l 128^2
+inline WgGeom node_wg_geom(int L, int N) {
+  const int NY = (L + 1) * (L + 1);
+  WgGeom g{N, L, NY, NY, 0, 1, 4, 9, 16, 1, 1, 1, 1, 1, 0, 16384, 2 * 16384, 3 * 16384, 4 * 16384};
+  return g;
+}
 
 }  // namespace fc

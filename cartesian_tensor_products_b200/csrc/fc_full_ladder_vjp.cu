@@ -492,20 +492,25 @@ extern "C" int fc_full_ladder_vjp(const fc_ladder_desc* d, int n_nodes, const fl
   if (cudaMemsetAsync(A_bar, 0, sizeof(float) * plane, s) != cudaSuccess ||
       cudaMemcpyAsync(pb, gz, sizeof(float) * plane, cudaMemcpyDeviceToDevice, s) != cudaSuccess)
     return FC_ERR_CUDA;
+  // Wq_bar's operands for the tensor cores: p_bar in the node layout, B_q in the path slots
+  WgGeom wq{n_nodes, L, nl.stride, pl.stride};
+  wq.ob0 = pl.off[0], wq.ob1 = pl.off[1], wq.ob2 = pl.off[2], wq.ob3 = pl.off[3], wq.ob4 = pl.off[4];
+  wq.pe0 = Pl[0], wq.pe1 = Pl[1], wq.pe2 = Pl[2], wq.pe3 = Pl[3], wq.pe4 = Pl[4];
+  wq.wo0 = (int)qoff[0], wq.wo1 = (int)qoff[1], wq.wo2 = (int)qoff[2], wq.wo3 = (int)qoff[3], wq.wo4 = (int)qoff[4];
   const size_t wq_step = (size_t)C * P * C;
   for (int q = order; q >= 2; --q) {
     const float* phi_prev = states + (size_t)(q - 2) * plane;
     const float* Wqq = Wq + (size_t)(q - 2) * wq_step;
     float* Wqb = Wq_bar + (size_t)(q - 2) * wq_step;
-    if ((st = full_tp_zrow_dispatch(L, n_nodes, C, phi_prev, A, Bq, s)) != FC_OK ||
-        (st = launch_rows_wgrad(n_nodes, C, L, nl, pl, pb, Bq, Wqb, qoff, s)) != FC_OK)
-      return st;
-    if (tc) {   // B_bar on tcgen05, one map per path (three-term TF32 split)
-      if ((st = launch_path_split_rows(gb, pb, xs, s)) != FC_OK ||
+    if ((st = full_tp_zrow_dispatch(L, n_nodes, C, phi_prev, A, Bq, s)) != FC_OK) return st;
+    if (tc) {   // Wq_bar and B_bar on tcgen05 (three-term TF32 split), B_bar one map per path
+      if ((st = launch_rows_wgrad_tc(wq, pb, Bq, Wqb, s)) != FC_OK ||
+          (st = launch_path_split_rows(gb, pb, xs, s)) != FC_OK ||
           (st = launch_path_split_map_t(gb, Wqq, wsm, s)) != FC_OK ||
           (st = launch_path_mix_tc(gb, xs, wsm, Bbar, s)) != FC_OK)
         return st;
-    } else if ((st = launch_rows_gemm<false>(n_nodes, C, L, nl, pl, pb, Wqq, qoff, Bbar, s)) != FC_OK) {
+    } else if ((st = launch_rows_wgrad(n_nodes, C, L, nl, pl, pb, Bq, Wqb, qoff, s)) != FC_OK ||
+               (st = launch_rows_gemm<false>(n_nodes, C, L, nl, pl, pb, Wqq, qoff, Bbar, s)) != FC_OK) {
       return st;
     }
     if ((st = full_tp_vjp_dispatch(L, n_nodes, C, phi_prev, A, Bbar, gz, pbn, A_bar, s)) != FC_OK)
@@ -515,7 +520,8 @@ extern "C" int fc_full_ladder_vjp(const fc_ladder_desc* d, int n_nodes, const fl
     pbn = t;
   }
   // the first map: W1_bar_l += pbar^T A, A_bar += pbar W1_l
-  if ((st = launch_rows_wgrad(n_nodes, C, L, nl, nl, pb, A, W1_bar, w1off, s)) != FC_OK ||
+  if ((st = mix_tc_supported(L, C) ? launch_rows_wgrad_tc(node_wg_geom(L, n_nodes), pb, A, W1_bar, s)
+                                     : launch_rows_wgrad(n_nodes, C, L, nl, nl, pb, A, W1_bar, w1off, s)) != FC_OK ||
       (st = launch_rows_gemm<true>(n_nodes, C, L, nl, nl, pb, W1, w1off, A_bar, s)) != FC_OK)
     return st;
   return FC_OK;

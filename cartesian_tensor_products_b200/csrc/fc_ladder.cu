@@ -552,10 +552,9 @@ size_t fc_product_ladder_vjp_workspace_size(const fc_ladder_desc* d, int n_nodes
   if (check_ladder_desc(d) != FC_OK || n_nodes < 0) return 0;
   const int NY = (d->lmax + 1) * (d->lmax + 1);
   size_t f = 4 * (size_t)n_nodes * NY * d->channels;
-  // tensor cores: the split gradient (for the mix), the matrices, and the
-  // transposed split gradient and recomputed product (for the weight gradient)
-  if (mix_tc_supported(d->lmax, d->channels))
-    f += tc_scratch_floats(d->lmax, n_nodes) + 2 * mix_tc_operand_floats(d->lmax, n_nodes);
+  // tensor cores: the split gradient and the matrices (for B_bar = A_bar M;
+  // the weight gradient reads FP32 rows)
+  if (mix_tc_supported(d->lmax, d->channels)) f += tc_scratch_floats(d->lmax, n_nodes);
   return sizeof(float) * f;
 }
 
@@ -596,8 +595,6 @@ int fc_product_ladder_vjp(const fc_ladder_desc* d, int n_nodes, const float* A1,
   const bool tc = mix_tc_supported(L, C);
   float* xs = ws + 4 * plane;                                   // tensor-core path only
   float* wsm = tc ? xs + mix_tc_operand_floats(L, n_nodes) : nullptr;
-  float* xta = tc ? wsm + mix_tc_matrix_floats(L) : nullptr;    // transposed split A_bar
-  float* xtb = tc ? xta + mix_tc_operand_floats(L, n_nodes) : nullptr;   // transposed split B
   const float* Anext_bar = gz;           // gradient of A_{v+1}
   for (int v = S; v >= 1; --v) {
     const float* Av = v == 1 ? A1 : states + (size_t)(v - 2) * plane;
@@ -618,9 +615,7 @@ int fc_product_ladder_vjp(const fc_ladder_desc* d, int n_nodes, const float* A1,
           (st = launch_mix_tc_split_rows(L, n_nodes, Anext_bar, xs, s)) != FC_OK ||
           (st = launch_mix_tc_split_matrix(1, L, M, wsm, s)) != FC_OK ||
           (st = launch_mix_tc(L, n_nodes, xs, wsm, Bbar, s)) != FC_OK ||
-          (st = launch_mix_tc_split_cols(L, n_nodes, Anext_bar, xta, s)) != FC_OK ||
-          (st = launch_mix_tc_split_cols(L, n_nodes, B, xtb, s)) != FC_OK ||
-          (st = launch_wgrad_tc(L, n_nodes, xta, xtb, Mbar, s)) != FC_OK)
+          (st = launch_rows_wgrad_tc(node_wg_geom(L, n_nodes), Anext_bar, B, Mbar, s)) != FC_OK)
         return st;
     } else {
       if ((st = tp_dispatch(L, n_nodes, C, Av, A1, W, B, s)) != FC_OK ||

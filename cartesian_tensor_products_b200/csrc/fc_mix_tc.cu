@@ -36,10 +36,11 @@
 //
 // This file holds three tensor-core kernels:
 //  * ladder_mix_tc_kernel: the mix above.  It is the VJP's B_bar = A_bar M.
-//  * ladder_wgrad_tc_kernel: the VJP's weight gradient.
 //  * path_mix_tc_kernel (further down): the per-rank maps with any K = 32 k_l
 //    over FP32 component-major tiles, split in shared memory.  It serves the
 //    full ladder's (P_l C -> C) maps and the ladder's forward mix (k_l = 4).
+//  * rows_wgrad_tc_kernel (last): weight gradients sum_rows a^T b straight
+//    from FP32 rows, transposed and split in shared memory.
 #include "fc_common.cuh"
 #include "fc_device.cuh"
 #include "fc_tc.cuh"
@@ -363,220 +364,6 @@ __global__ void __launch_bounds__(kTcThreads, 1) ladder_mix_tc_kernel(Geom geo,
   if (warp == 0) {
     tc::fence_after_sync();
     tc::tmem_dealloc(tmem, 2 * kTcRows);
-  }
-}
-
-// ---------------------------------------------------------------------------
-// weight gradient of the mix: Mbar_l[k][j] += sum_{rows of rank l} Abar[row][k] B[row][j]
-// ---------------------------------------------------------------------------
-// Here the tile rows are the K dimension, so both operands are taken
-// transposed: ladder_split_cols_kernel writes a tile as 128 channels x 128
-// rows in the K-major core-matrix layout (4 consecutive rows of one channel
-// per 16 bytes), so a K chunk of 32 rows is a contiguous 16 KB hi and 16 KB lo
-// block, exactly as the mix's chunks.  One persistent CTA per SM walks its
-// tiles: one thread bulk-copies each chunk of both operands (64 KB) into one
-// of three stages, one thread issues the 12 MMAs of a chunk (M = N = 128,
-// three TF32 products per K step), the accumulator D[k][j] sums every tile
-// of one rank, and at a rank change and at the end warps 4-7 add it to Mbar
-// with vector atomics (CTAs share Mbar_l).  (Reading the row-major tiles with
-// MN-major descriptors instead returned zeros on sm_100a.)
-
-// natural [N][NY][128] -> transposed split tiles: element (row r, channel k)
-// of tile t at core_offset(k, r, 128) of the tile's hi / lo block.  Thread p
-// moves a 4-row x 4-channel block: 4 row-wise float4 loads, 4 channel-wise
-// float4 stores.  Rows past the rank's last row are written as zeros.
-__global__ void __launch_bounds__(256) ladder_split_cols_kernel(Geom g, const float* __restrict__ in,
-                                                                float* __restrict__ xs) {
-  const int t = blockIdx.x;
-  const int l = tile_rank(g, t);
-  const int R = g.N * (2 * l + 1);
-  const int row0 = (t - tile_first(g, l)) * kTcRows;
-  float* hi = xs + (size_t)t * kTcTileFloats;
-#pragma unroll
-  for (int it = 0; it < 4; ++it) {
-    const int u = it * 256 + threadIdx.x;          // 0 .. 1023
-    const int k4 = u & 31, r4 = u >> 5;            // channel group (fastest), row group
-    float4 v[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int r = row0 + 4 * r4 + i;
-      v[i] = r < R ? __ldg(reinterpret_cast<const float4*>(in + tc_rank_row(r, l, g.NY)) + k4) : zero4();
-    }
-    const float c0[4] = {v[0].x, v[1].x, v[2].x, v[3].x};
-    const float c1[4] = {v[0].y, v[1].y, v[2].y, v[3].y};
-    const float c2[4] = {v[0].z, v[1].z, v[2].z, v[3].z};
-    const float c3[4] = {v[0].w, v[1].w, v[2].w, v[3].w};
-    const float* cs[4] = {c0, c1, c2, c3};
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      uint4 h, w;
-      split4(make_float4(cs[j][0], cs[j][1], cs[j][2], cs[j][3]), h, w);
-      const int off = tc::core_offset(4 * k4 + j, 4 * r4, kTcRows);
-      *reinterpret_cast<uint4*>(hi + off) = h;
-      *reinterpret_cast<uint4*>(hi + kTcWFloats + off) = w;
-    }
-  }
-}
-
-constexpr int kWgThreads = 256;
-constexpr int kWgStageFloats = 2 * kTcChunkFloats;   // A and B chunks (hi + lo each)
-constexpr size_t kWgSmemBytes = sizeof(float) * kTcStages * kWgStageFloats + 8 * 16 + 8;
-static_assert(kWgSmemBytes <= 232448, "shared memory per CTA");
-
-__global__ void __launch_bounds__(kWgThreads, 1) ladder_wgrad_tc_kernel(Geom geo,
-                                                                        const float* __restrict__ as,
-                                                                        const float* __restrict__ bs,
-                                                                        float* __restrict__ Mbar) {
-  extern __shared__ __align__(1024) unsigned char smem[];
-  float* st = reinterpret_cast<float*>(smem);        // stages: A hi, A lo, B hi, B lo (4096 each)
-  uint64_t* stage_full = reinterpret_cast<uint64_t*>(st + kTcStages * kWgStageFloats);
-  uint64_t* stage_free = stage_full + kTcStages;
-  uint64_t* acc_full = stage_free + kTcStages;
-  uint64_t* acc_free = acc_full + 1;
-  uint64_t* drain = acc_free + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
-
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int T = tile_count(geo);
-  const int t_begin = (int)((long long)blockIdx.x * T / gridDim.x);
-  const int t_end = (int)((long long)(blockIdx.x + 1) * T / gridDim.x);
-
-  if (warp == 0) tc::tmem_alloc(tmem_slot, kTcRows);
-  if (tid == 0) {
-    for (int s = 0; s < kTcStages; ++s) {
-      tc::bar_init(&stage_full[s], 1);
-      tc::bar_init(&stage_free[s], 1);
-    }
-    tc::bar_init(acc_full, 1);
-    tc::bar_init(acc_free, 128);
-    tc::bar_init(drain, 1);
-    tc::fence_bar_init();
-  }
-  tc::fence_before_sync();
-  __syncthreads();
-  tc::fence_after_sync();
-  const uint32_t tmem = *tmem_slot;
-  const uint64_t lim = g_tc_wait_ns;
-  bool fail = false;
-
-  if (warp == 0) {
-    // ---------------- bulk-copy producer ----------------
-    if (lane == 0) {
-      int g = 0;
-      for (int t = t_begin; t < t_end && !fail; ++t) {
-        for (int c = 0; c < kTcChunks; ++c, ++g) {
-          const int s = g % kTcStages;
-          if (g >= kTcStages &&
-              !tc::bar_wait(&stage_free[s], ((g - kTcStages) / kTcStages) & 1, lim)) {
-            fail = true;
-            break;
-          }
-          float* dst = st + s * kWgStageFloats;
-          const float* sa = as + (size_t)t * kTcTileFloats + c * kTcBlockFloats;
-          const float* sb = bs + (size_t)t * kTcTileFloats + c * kTcBlockFloats;
-          tc::bar_arrive_expect_tx(&stage_full[s], kWgStageFloats * sizeof(float));
-          tc::bulk_load(dst, sa, kTcBlockFloats * sizeof(float), &stage_full[s]);
-          tc::bulk_load(dst + kTcBlockFloats, sa + kTcWFloats, kTcBlockFloats * sizeof(float), &stage_full[s]);
-          tc::bulk_load(dst + 2 * kTcBlockFloats, sb, kTcBlockFloats * sizeof(float), &stage_full[s]);
-          tc::bulk_load(dst + 3 * kTcBlockFloats, sb + kTcWFloats, kTcBlockFloats * sizeof(float),
-                        &stage_full[s]);
-        }
-      }
-      if (fail)   // let the copies already issued land
-        for (int k = 1; k <= kTcStages && g - k >= 0; ++k)
-          tc::bar_wait(&stage_full[(g - k) % kTcStages], ((g - k) / kTcStages) & 1, kTcDrainNs);
-    }
-    __syncwarp();
-  } else if (warp == 1) {
-    // ---------------- MMA issuer ----------------
-    if (lane == 0) {
-      constexpr uint32_t idesc = tc::idesc_tf32(kTcC, kTcC);
-      constexpr uint32_t kLbo = kTcRows * 16, kSbo = 128;   // K group (4 rows), 8-channel group
-      int g = 0, seg = 0, cur_l = -1;
-      bool fresh = true;
-      for (int t = t_begin; t < t_end && !fail; ++t) {
-        const int l = tile_rank(geo, t);
-        if (l != cur_l) {
-          if (cur_l >= 0) {   // publish the finished rank, wait until it is drained
-            tc::commit(acc_full);
-            if (!tc::bar_wait(acc_free, seg & 1, lim)) {
-              fail = true;
-              break;
-            }
-            ++seg;
-          }
-          cur_l = l;
-          fresh = true;
-        }
-        for (int c = 0; c < kTcChunks; ++c, ++g) {
-          const int s = g % kTcStages;
-          if (!tc::bar_wait(&stage_full[s], (g / kTcStages) & 1, lim)) {
-            fail = true;
-            break;
-          }
-          tc::fence_after_sync();
-          const uint32_t a_h = tc::smem_addr(st + s * kWgStageFloats);
-          const uint32_t a_l = a_h + kTcBlockFloats * sizeof(float);
-          const uint32_t b_h = a_h + 2 * kTcBlockFloats * sizeof(float);
-          const uint32_t b_l = a_h + 3 * kTcBlockFloats * sizeof(float);
-#pragma unroll
-          for (int j = 0; j < kTcChunk / 8; ++j) {
-            const uint32_t kx = 2 * j * kLbo;
-            const uint64_t dah = tc::smem_desc(a_h + kx, kLbo, kSbo);
-            const uint64_t dal = tc::smem_desc(a_l + kx, kLbo, kSbo);
-            const uint64_t dbh = tc::smem_desc(b_h + kx, kLbo, kSbo);
-            const uint64_t dbl = tc::smem_desc(b_l + kx, kLbo, kSbo);
-            tc::mma_tf32(tmem, dah, dbh, idesc, (fresh && c == 0 && j == 0) ? 0u : 1u);
-            tc::mma_tf32(tmem, dal, dbh, idesc, 1u);
-            tc::mma_tf32(tmem, dah, dbl, idesc, 1u);
-          }
-          tc::commit(&stage_free[s]);
-        }
-        fresh = false;
-      }
-      if (!fail && cur_l >= 0) tc::commit(acc_full);   // the last rank of the range
-      // every MMA issued above has finished (also after a wait gave up)
-      // before the CTA releases TMEM and its shared memory
-      tc::commit(drain);
-      if (!tc::bar_wait(drain, 0, kTcDrainNs)) fail = true;
-    }
-    __syncwarp();
-  } else if (warp >= 4) {
-    // ---------------- drain: D[k][j] -> Mbar_l at every rank change ----------------
-    const int ew = warp - 4;
-    const int k = 32 * ew + lane;
-    int seg = 0, cur_l = -1;
-    for (int t = t_begin; t <= t_end; ++t) {
-      const int l = t < t_end ? tile_rank(geo, t) : -1;
-      if (l == cur_l) continue;
-      if (cur_l >= 0) {
-        if (!tc::bar_wait(acc_full, seg & 1, lim)) {
-          fail = true;
-          break;
-        }
-        tc::fence_after_sync();
-        float* Ml = Mbar + (size_t)cur_l * kTcC * kTcC + (size_t)k * kTcC;
-#pragma unroll 1
-        for (int q = 0; q < kTcC / 32; ++q) {
-          float v[32];
-          tc::tmem_ld32(tmem + ((uint32_t)(32 * ew) << 16) + 32 * q, v);
-#pragma unroll
-          for (int u = 0; u < 8; ++u)
-            red_add4(Ml + 32 * q + 4 * u, make_float4(v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3]));
-        }
-        tc::fence_before_sync();
-        tc::bar_arrive(acc_free);
-        ++seg;
-      }
-      cur_l = l;
-    }
-  }
-  if (fail) atomicExch(&g_tc_error, 1);
-  tc::fence_before_sync();
-  __syncthreads();
-  if (warp == 0) {
-    tc::fence_after_sync();
-    tc::tmem_dealloc(tmem, kTcRows);
   }
 }
 
@@ -944,8 +731,293 @@ __global__ void __launch_bounds__(kTcThreads, 1) path_mix_tc_kernel(PathGeom geo
   }
 }
 
+// ---------------------------------------------------------------------------
+// weight gradient from FP32 rows: Wb_l[j][e 128 + k] += sum_i a[i][j] b_e[i][k]
+// ---------------------------------------------------------------------------
+// The contraction runs over the rows i of rank l (node n, component c), so
+// both operands must be K-major along the rows, i.e. transposed (the TF32
+// MMA reads K-major operands only).  Nothing is pre-split in global memory:
+// one warp copies the 32 rows of a K chunk of both operands (512 bytes per
+// row, any row layout) into one of two FP32 stages with cp.async, eight
+// converter warps transpose and split them into TF32 hi / lo K-major blocks
+// in shared memory (explicit shared-memory loads and stores, no predicates:
+// generic-pointer loads with a row mask left the converters waiting on
+// long-latency loads and the tensor pipe 15 % busy), one thread issues the
+// 12 MMAs of a chunk (M = N = 128: D[j][k], three TF32 products per K step)
+// and four warps add each finished accumulator into Wb with vector atomics.
+// The CTAs share the chunk list evenly; a segment (one accumulator chain) is
+// a run of at most kRwSeg chunks of one (rank, map), which bounds the chain
+// at 12 kRwSeg MMAs for FP32-level accuracy.  Two accumulators alternate in
+// TMEM so that a drain overlaps the next segment's MMAs.
+constexpr int kRwSeg = 32;                            // chunks per accumulator chain
+constexpr int kRwThreads = 448;                       // w0 copies, w1 issues, w2-9 convert, w10-13 drain
+constexpr int kRwCvtThreads = 256;
+constexpr int kRwStages = 2;   // FP32 stages (a third measured no faster: the converter-MMA handshake sets the pace)
+constexpr int kRwRowFloats = kTcChunk * kTcC;         // 4096: 32 rows x 128 channels
+constexpr int kRwStageFloats = 2 * kRwRowFloats;      // both operands, FP32
+constexpr int kRwCvtFloats = 4 * kTcBlockFloats;      // both operands, hi and lo
+constexpr size_t kRwSmemBytes =
+    sizeof(float) * (kRwStages * kRwStageFloats + 2 * kRwCvtFloats) + 8 * 16 + 8;
+static_assert(kRwSmemBytes <= 232448, "shared memory per CTA");
+
+// chunk list: rank by rank, the maps of a rank one after the other, a map's
+// chunks in row order
+__device__ __forceinline__ int wg_chunks(const WgGeom& g, int l) {
+  return (g.N * (2 * l + 1) + kTcChunk - 1) / kTcChunk;
+}
+__device__ __forceinline__ void wg_chunk(const WgGeom& g, int ch, int& l, int& e, int& q) {
+  l = 0;
+  int c0 = 0;
+  while (l < g.L && ch >= c0 + wg_pe(g, l) * wg_chunks(g, l)) {
+    c0 += wg_pe(g, l) * wg_chunks(g, l);
+    ++l;
+  }
+  const int nc = wg_chunks(g, l);
+  e = (ch - c0) / nc;
+  q = ch - c0 - e * nc;
+}
+
+__global__ void __launch_bounds__(kRwThreads, 1) rows_wgrad_tc_kernel(WgGeom geo, const float* __restrict__ a,
+                                                                      const float* __restrict__ b,
+                                                                      float* __restrict__ Wb) {
+  extern __shared__ __align__(1024) unsigned char smem[];
+  float* st = reinterpret_cast<float*>(smem);       // stages: a rows, b rows (FP32)
+  float* cv = st + kRwStages * kRwStageFloats;      // 2 buffers: a hi, a lo, b hi, b lo
+  uint64_t* stage_full = reinterpret_cast<uint64_t*>(cv + 2 * kRwCvtFloats);
+  uint64_t* stage_free = stage_full + kRwStages;
+  uint64_t* cvt_full = stage_free + kRwStages;
+  uint64_t* cvt_free = cvt_full + 2;
+  uint64_t* acc_full = cvt_free + 2;
+  uint64_t* acc_free = acc_full + 2;
+  uint64_t* drain = acc_free + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  int total = 0;
+  for (int l = 0; l <= geo.L; ++l) total += wg_pe(geo, l) * wg_chunks(geo, l);
+  const int c_begin = (int)((long long)blockIdx.x * total / gridDim.x);
+  const int c_end = (int)((long long)(blockIdx.x + 1) * total / gridDim.x);
+
+  if (warp == 0) tc::tmem_alloc(tmem_slot, 2 * kTcC);
+  if (tid == 0) {
+    for (int i = 0; i < kRwStages; ++i) {
+      tc::bar_init(&stage_full[i], 32);   // the producer's lanes, on their copies' completion
+      tc::bar_init(&stage_free[i], kRwCvtThreads / 32);   // one per converter warp
+    }
+    for (int i = 0; i < 2; ++i) {
+      tc::bar_init(&cvt_full[i], kRwCvtThreads / 32);
+      tc::bar_init(&cvt_free[i], 1);
+      tc::bar_init(&acc_full[i], 1);
+      tc::bar_init(&acc_free[i], 128);
+    }
+    tc::bar_init(drain, 1);
+    tc::fence_bar_init();
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = *tmem_slot;
+  const uint64_t lim = g_tc_wait_ns;
+  bool fail = false;
+
+  if (warp == 0) {
+    // ---------------- producer: cp.async, one 512-byte row per warp instruction ----------------
+    // The warp walks the chunk's rows (node n, component c) incrementally,
+    // 16 bytes a lane; rows past the rank's end are zero-filled, so the
+    // converters read every row unconditionally.
+    int g = 0;
+    for (int ch = c_begin; ch < c_end && !fail; ++ch, ++g) {
+      int l, e, q;
+      wg_chunk(geo, ch, l, e, q);
+      const int s = g % kRwStages;
+      bool ok = true;
+      if (lane == 0 && g >= kRwStages) ok = tc::bar_wait(&stage_free[s], ((g / kRwStages) - 1) & 1, lim);
+      if (!__shfl_sync(0xffffffffu, ok, 0)) {
+        fail = true;
+        break;
+      }
+      const int w = 2 * l + 1, R = geo.N * w;
+      const int i0 = q * kTcChunk;
+      const int nv = min(kTcChunk, R - i0);
+      const int pe = wg_pe(geo, l);
+      int n = i0 / w, c = i0 - n * w;
+      const float* ra = a + ((size_t)n * geo.sa + l * l + c) * kTcC + 4 * lane;
+      const float* rb = b + ((size_t)n * geo.sb + wg_ob(geo, l) + (size_t)c * pe + e) * kTcC + 4 * lane;
+      const long long na = (long long)(geo.sa - w + 1) * kTcC, nb = ((long long)geo.sb - (long long)(w - 1) * pe) * kTcC;
+      float* dst = st + s * kRwStageFloats + 4 * lane;
+      for (int r = 0; r < nv; ++r) {
+        cp_async16(dst + r * kTcC, ra, true);
+        cp_async16(dst + kRwRowFloats + r * kTcC, rb, true);
+        if (++c == w) {   // next node
+          c = 0;
+          ra += na;
+          rb += nb;
+        } else {
+          ra += kTcC;
+          rb += (size_t)pe * kTcC;
+        }
+      }
+      for (int r = nv; r < kTcChunk; ++r) {   // zero rows (reads nothing)
+        cp_async16(dst + r * kTcC, a, false);
+        cp_async16(dst + kRwRowFloats + r * kTcC, b, false);
+      }
+      tc::cp_async_bar_arrive(&stage_full[s]);   // one of the 32 expected arrivals
+    }
+    if (fail && lane == 0)   // let the copies already issued land
+      for (int k = 1; k <= kRwStages && g - k >= 0; ++k)
+        tc::bar_wait(&stage_full[(g - k) % kRwStages], ((g - k) / kRwStages) & 1, kTcDrainNs);
+    __syncwarp();
+  } else if (warp == 1) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0) {
+      constexpr uint32_t idesc = tc::idesc_tf32(kTcC, kTcC);
+      constexpr uint32_t kLbo = kTcC * 16, kSbo = 128;   // K group (4 rows), 8-channel group
+      int g = 0, h = -1, run = 0, pl = -1, pe = -1;
+      for (int ch = c_begin; ch < c_end && !fail; ++ch, ++g) {
+        int l, e, q;
+        wg_chunk(geo, ch, l, e, q);
+        const bool fresh = (l != pl || e != pe || run == kRwSeg);
+        if (fresh) {
+          if (h >= 0) tc::commit(&acc_full[h & 1]);   // the previous segment is complete
+          ++h;
+          run = 0;
+          pl = l;
+          pe = e;
+          if (h >= 2 && !tc::bar_wait(&acc_free[h & 1], ((h - 2) >> 1) & 1, lim)) {
+            fail = true;
+            break;
+          }
+          tc::fence_after_sync();
+        }
+        const int bb = g & 1;
+        if (!tc::bar_wait(&cvt_full[bb], (g >> 1) & 1, lim)) {
+          fail = true;
+          break;
+        }
+        tc::fence_after_sync();
+        const uint32_t d_tmem = tmem + (uint32_t)(h & 1) * kTcC;
+        const uint32_t ah = tc::smem_addr(cv + bb * kRwCvtFloats);
+        const uint32_t al = ah + kTcBlockFloats * sizeof(float);
+        const uint32_t bh = ah + 2 * kTcBlockFloats * sizeof(float);
+        const uint32_t bl = ah + 3 * kTcBlockFloats * sizeof(float);
+#pragma unroll
+        for (int j = 0; j < kTcChunk / 8; ++j) {
+          const uint32_t kx = 2 * j * kLbo;
+          const uint64_t dah = tc::smem_desc(ah + kx, kLbo, kSbo);
+          const uint64_t dal = tc::smem_desc(al + kx, kLbo, kSbo);
+          const uint64_t dbh = tc::smem_desc(bh + kx, kLbo, kSbo);
+          const uint64_t dbl = tc::smem_desc(bl + kx, kLbo, kSbo);
+          tc::mma_tf32(d_tmem, dah, dbh, idesc, (run | j) != 0);
+          tc::mma_tf32(d_tmem, dal, dbh, idesc, 1u);
+          tc::mma_tf32(d_tmem, dah, dbl, idesc, 1u);
+        }
+        tc::commit(&cvt_free[bb]);
+        ++run;
+      }
+      if (!fail && h >= 0) tc::commit(&acc_full[h & 1]);   // the last segment
+      // every MMA issued above has finished (also after a wait gave up)
+      // before the CTA releases TMEM and its shared memory
+      tc::commit(drain);
+      if (!tc::bar_wait(drain, 0, kTcDrainNs)) fail = true;
+    }
+    __syncwarp();
+  } else if (warp < 10) {
+    // ---------------- converters: FP32 rows -> transposed TF32 hi / lo ----------------
+    // Thread ct takes channel k = ct % 128 of rows 4 (h + 2 m) .. + 3 (h = ct / 128,
+    // m = 0..3) of both operands: 32 conflict-free scalar loads (a warp reads
+    // 32 consecutive channels of a row), then per 4 rows one 16-byte hi and
+    // one lo store (a warp fills 512 contiguous bytes).
+    const int ct = tid - 64;   // 0 .. 255
+    const int k = ct & (kTcC - 1), h = ct >> 7;
+    const uint32_t src0 = tc::smem_addr(st) + 4u * (uint32_t)(4 * h * kTcC + k);
+    const uint32_t dst0 = tc::smem_addr(cv) + 4u * (uint32_t)tc::core_offset(k, 4 * h, kTcC);
+    int g = 0;
+    for (int ch = c_begin; ch < c_end && !fail; ++ch, ++g) {
+      const int s = g % kRwStages, bb = g & 1;
+      if (!tc::bar_wait(&stage_full[s], (g / kRwStages) & 1, lim) ||
+          (g >= 2 && !tc::bar_wait(&cvt_free[bb], ((g - 2) >> 1) & 1, lim))) {
+        fail = true;
+        break;
+      }
+      const uint32_t src = src0 + 4u * s * kRwStageFloats;
+      const uint32_t dst = dst0 + 4u * bb * kRwCvtFloats;
+      float v[2][4][4];
+#pragma unroll
+      for (int op = 0; op < 2; ++op)
+#pragma unroll
+        for (int m = 0; m < 4; ++m)
+#pragma unroll
+          for (int r = 0; r < 4; ++r)
+            asm volatile("ld.shared.f32 %0, [%1];"
+                         : "=f"(v[op][m][r])
+                         : "r"(src + 4u * (op * kRwRowFloats + (8 * m + r) * kTcC)));
+#pragma unroll
+      for (int op = 0; op < 2; ++op)
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+          uint4 hv, lv;
+          split4(make_float4(v[op][m][0], v[op][m][1], v[op][m][2], v[op][m][3]), hv, lv);
+          const uint32_t d = dst + 4u * (op * 2 * kTcBlockFloats + m * 1024);
+          asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(d), "r"(hv.x), "r"(hv.y), "r"(hv.z),
+                       "r"(hv.w) : "memory");
+          asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(d + 4u * kTcBlockFloats), "r"(lv.x),
+                       "r"(lv.y), "r"(lv.z), "r"(lv.w) : "memory");
+        }
+      tc::fence_proxy_async();   // the generic-proxy writes, visible to the MMAs
+      __syncwarp();              // one arrival per warp (256 on one word serialise)
+      if (lane == 0) {
+        tc::bar_arrive(&cvt_full[bb]);
+        tc::bar_arrive(&stage_free[s]);
+      }
+    }
+  } else {
+    // ---------------- drain: D[j][k] -> Wb_l[j][e 128 + k] ----------------
+    const int ew = warp & 3;        // the TMEM lane quarter this warp may read
+    const int j = 32 * ew + lane;   // output row
+    int h = -1, run = 0, pl = -1, pe = -1;
+    for (int ch = c_begin; ch <= c_end && !fail; ++ch) {
+      int l = -1, e = -1, q = 0;
+      if (ch < c_end) wg_chunk(geo, ch, l, e, q);
+      const bool fresh = ch == c_end || l != pl || e != pe || run == kRwSeg;
+      if (fresh && h >= 0) {   // segment h (rank pl, map pe) is complete: add it
+        if (!tc::bar_wait(&acc_full[h & 1], (h >> 1) & 1, lim)) {
+          fail = true;
+          break;
+        }
+        tc::fence_after_sync();
+        float* Wr = Wb + wg_wo(geo, pl) + (size_t)j * (wg_pe(geo, pl) * kTcC) + pe * kTcC;
+#pragma unroll 1
+        for (int c = 0; c < kTcC / 32; ++c) {
+          float v[32];
+          tc::tmem_ld32(tmem + (uint32_t)(h & 1) * kTcC + ((uint32_t)(32 * ew) << 16) + 32 * c, v);
+#pragma unroll
+          for (int u = 0; u < 8; ++u)
+            red_add4(Wr + 32 * c + 4 * u, make_float4(v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3]));
+        }
+        tc::fence_before_sync();
+        tc::bar_arrive(&acc_free[h & 1]);
+      }
+      if (ch == c_end) break;
+      if (fresh) {
+        ++h;
+        run = 0;
+        pl = l;
+        pe = e;
+      }
+      ++run;
+    }
+  }
+  if (fail) atomicExch(&g_tc_error, 1);
+  tc::fence_before_sync();
+  __syncthreads();
+  if (warp == 0) {
+    tc::fence_after_sync();
+    tc::tmem_dealloc(tmem, 2 * kTcC);
+  }
+}
+
+DeviceFlags g_rw_smem_set;
 DeviceFlags g_tc_smem_set;
-DeviceFlags g_wg_smem_set;
 DeviceFlags g_pm_smem_set;
 
 }  // namespace
@@ -997,26 +1069,6 @@ int launch_mix_tc(int L, int N, const float* xs, const float* ws, float* out, cu
   return cudaGetLastError() == cudaSuccess ? FC_OK : FC_ERR_CUDA;
 }
 
-int launch_mix_tc_split_cols(int L, int N, const float* in, float* xs, cudaStream_t s) {
-  const Geom g = make_geom(L, N);
-  const int T = tile_count(g);
-  if (T == 0) return FC_OK;
-  ladder_split_cols_kernel<<<T, 256, 0, s>>>(g, in, xs);
-  return cudaGetLastError() == cudaSuccess ? FC_OK : FC_ERR_CUDA;
-}
-
-int launch_wgrad_tc(int L, int N, const float* as, const float* bs, float* Mbar, cudaStream_t s) {
-  if (!mix_tc_supported(L, kTcC)) return FC_ERR_UNSUPPORTED_RANK;
-  if (set_smem_once(g_wg_smem_set, ladder_wgrad_tc_kernel, kWgSmemBytes) != FC_OK) return FC_ERR_CUDA;
-  const Geom g = make_geom(L, N);
-  const int T = tile_count(g);
-  if (T == 0) return FC_OK;
-  const int sms = device_sm_count();
-  const int grid = T < sms ? T : sms;
-  ladder_wgrad_tc_kernel<<<grid, kWgThreads, kWgSmemBytes, s>>>(g, as, bs, Mbar);
-  return cudaGetLastError() == cudaSuccess ? FC_OK : FC_ERR_CUDA;
-}
-
 PathGeom path_geom(int L, int N, const int* kc) {
   PathGeom g{};
   g.N = N;
@@ -1063,6 +1115,18 @@ int launch_path_split_map(const PathGeom& g, const float* W, float* ws, cudaStre
   for (int l = 0; l <= g.L; ++l) kmax = pg_kc(g, l) > kmax ? pg_kc(g, l) : kmax;
   if (kmax == 0) return FC_OK;
   path_split_map_kernel<<<dim3(kmax, g.L + 1), 256, 0, s>>>(g, W, ws);
+  return cudaGetLastError() == cudaSuccess ? FC_OK : FC_ERR_CUDA;
+}
+
+int launch_rows_wgrad_tc(const WgGeom& g, const float* a, const float* b, float* Wb, cudaStream_t s) {
+  if (g.L < 0 || g.L > 4) return FC_ERR_UNSUPPORTED_RANK;
+  if (set_smem_once(g_rw_smem_set, rows_wgrad_tc_kernel, kRwSmemBytes) != FC_OK) return FC_ERR_CUDA;
+  long long total = 0;
+  for (int l = 0; l <= g.L; ++l) total += (long long)wg_pe(g, l) * ((g.N * (2 * l + 1) + kTcChunk - 1) / kTcChunk);
+  if (total == 0) return FC_OK;
+  const int sms = device_sm_count();
+  const int grid = total < sms ? (int)total : sms;
+  rows_wgrad_tc_kernel<<<grid, kRwThreads, kRwSmemBytes, s>>>(g, a, b, Wb);
   return cudaGetLastError() == cudaSuccess ? FC_OK : FC_ERR_CUDA;
 }
 

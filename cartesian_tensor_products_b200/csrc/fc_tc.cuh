@@ -134,6 +134,12 @@ __device__ __forceinline__ void bulk_load(void* smem_dst, const void* gmem_src, 
       : "memory");
 }
 
+// Arrival on an mbarrier once every cp.async this thread issued before it
+// has landed; .noinc: the arrival is one of the barrier's expected count.
+__device__ __forceinline__ void cp_async_bar_arrive(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" : : "r"(smem_addr(bar)) : "memory");
+}
+
 // Plain arrival on an mbarrier (counted in its expected arrivals).
 __device__ __forceinline__ void bar_arrive(uint64_t* bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" : : "r"(smem_addr(bar)) : "memory");

@@ -6,6 +6,8 @@ The sizes follow the scratch layouts the header states:
   rank and component, with K = 128 P_l inputs per row for the full ladder
   (Sec. 5 Eq. 2, every path kept) or K = 128 for the path-reduced ladder;
   plus one step's maps as TF32 hi and lo;
+* ladder VJP: four product states, plus at C = 128 the gradient as split
+  tiles and one step's split matrices;
 * SIMT path: one product state (full ladder: the convolution's output row
   of sum_l (2l+1) P_l slots; ladder: (L+1)^2 slots), none at order 1 for
   the full ladder;
@@ -61,6 +63,20 @@ def test_ladder_forward(fc, L, N):
     maps = (L + 1) * 2 * 128 * 128
     assert query(fc, "fc_product_ladder_workspace_size", L, 128, 4, N) == 4 * (product + maps)
     assert query(fc, "fc_product_ladder_workspace_size", L, 64, 4, N) == 4 * N * NY * 64
+
+
+@pytest.mark.parametrize("L", [1, 2, 3, 4])
+@pytest.mark.parametrize("N", [1, 128, 129, 4096])
+def test_ladder_vjp(fc, L, N):
+    """Four product states; at C = 128 also the gradient as split tiles of
+    128 rows per rank (rows n (2l+1) + c, hi and lo) and one step's split
+    matrices.  The weight gradient reads the FP32 rows and needs nothing."""
+    NY = (L + 1) ** 2
+    tiles = sum((N * (2 * l + 1) + 127) // 128 for l in range(L + 1))
+    states = 4 * N * NY * 128
+    split = tiles * 2 * 128 * 128 + (L + 1) * 2 * 128 * 128
+    assert query(fc, "fc_product_ladder_vjp_workspace_size", L, 128, 4, N) == 4 * (states + split)
+    assert query(fc, "fc_product_ladder_vjp_workspace_size", L, 64, 4, N) == 4 * 4 * N * NY * 64
 
 
 def test_unsupported_descriptors_need_nothing(fc):
