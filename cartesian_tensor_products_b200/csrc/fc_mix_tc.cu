@@ -41,6 +41,11 @@
 //    full ladder's (P_l C -> C) maps and the ladder's forward mix (k_l = 4).
 //  * rows_wgrad_tc_kernel (last): weight gradients sum_rows a^T b straight
 //    from FP32 rows, transposed and split in shared memory.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <cstring>
+
 #include "fc_common.cuh"
 #include "fc_device.cuh"
 #include "fc_tc.cuh"
@@ -734,36 +739,59 @@ __global__ void __launch_bounds__(kTcThreads, 1) path_mix_tc_kernel(PathGeom geo
 // ---------------------------------------------------------------------------
 // weight gradient from FP32 rows: Wb_l[j][e 128 + k] += sum_i a[i][j] b_e[i][k]
 // ---------------------------------------------------------------------------
-// The contraction runs over the rows i of rank l (node n, component c), so
-// both operands must be K-major along the rows, i.e. transposed (the TF32
-// MMA reads K-major operands only).  Nothing is pre-split in global memory:
-// one warp copies the 32 rows of a K chunk of both operands (512 bytes per
-// row, any row layout) into one of two FP32 stages with cp.async, eight
-// converter warps transpose and split them into TF32 hi / lo K-major blocks
-// in shared memory (explicit shared-memory loads and stores, no predicates:
-// generic-pointer loads with a row mask left the converters waiting on
-// long-latency loads and the tensor pipe 15 % busy), one thread issues the
-// 12 MMAs of a chunk (M = N = 128: D[j][k], three TF32 products per K step)
-// and four warps add each finished accumulator into Wb with vector atomics.
+// The contraction runs over the rows i of rank l (node n, component c): K is
+// the row index, so both operands enter the MMA transposed.  Nothing is
+// pre-split in global memory.  A K chunk is wg_nodes(l) = 32 / (2l+1) whole
+// nodes of rank l (32, 30, 30, 28, 27 rows for l = 0..4): one thread loads it
+// for both operands with two tiled TMA copies (operand a as a 3-D tensor:
+// channel, component, node; operand b as a 4-D tensor: channel, map e,
+// component, node; nodes past N are filled with zeros) into one of four FP32
+// stages.  Eight converter warps read a stage (one channel of all 32 rows per
+// thread, conflict-free), release it, and split the values into TF32 hi / lo:
+// operand a goes to tensor memory as the MMA's A operand (row j of A in TMEM
+// lane j, the K rows along columns: one 32-column store per thread), operand
+// b to K-major core-matrix blocks in shared memory.  One thread issues the 12
+// MMAs of a chunk (M = N = 128: D[j][k], three TF32 products per K step, A
+// from TMEM), three converted buffers deep, and four warps add each finished
+// accumulator into Wb with vector atomics.
+//
+// Measured on the way here (4096 nodes, rank 3, 2048 row chunks of 32):
+//  * a row per copy (cp.async from one warp, or one bulk copy per lane) took
+//    2300 and 4000 cycles per chunk to issue;
+//  * with both MMA operands in shared memory only two FP32 stages and two
+//    converted buffers (64 KB each) fit, about one chunk was in flight per SM,
+//    and a chunk cost about one loaded memory latency (2400 cycles);
+//  * A in TMEM halves the converted buffers and the MMA's shared-memory reads.
 // The CTAs share the chunk list evenly; a segment (one accumulator chain) is
 // a run of at most kRwSeg chunks of one (rank, map), which bounds the chain
 // at 12 kRwSeg MMAs for FP32-level accuracy.  Two accumulators alternate in
 // TMEM so that a drain overlaps the next segment's MMAs.
 constexpr int kRwSeg = 32;                            // chunks per accumulator chain
-constexpr int kRwThreads = 448;                       // w0 copies, w1 issues, w2-9 convert, w10-13 drain
-constexpr int kRwCvtThreads = 256;
-constexpr int kRwStages = 2;   // FP32 stages (a third measured no faster: the converter-MMA handshake sets the pace)
+constexpr int kRwThreads = 448;                       // w0 loads, w1 issues, w2-9 convert, w10-13 drain
+constexpr int kRwCvtWarps = 8;
+constexpr int kRwStages = 4;                          // FP32 stages
+constexpr int kRwBufs = 3;                            // converted buffers (B in smem, A in TMEM)
 constexpr int kRwRowFloats = kTcChunk * kTcC;         // 4096: 32 rows x 128 channels
 constexpr int kRwStageFloats = 2 * kRwRowFloats;      // both operands, FP32
-constexpr int kRwCvtFloats = 4 * kTcBlockFloats;      // both operands, hi and lo
+constexpr int kRwCvtFloats = 2 * kTcBlockFloats;      // operand b, hi and lo
+constexpr uint32_t kRwTmemCols = 512;                 // 2 accumulators + kRwBufs x (A hi, A lo)
+constexpr uint32_t kRwACol = 2 * kTcC;                // first A column
 constexpr size_t kRwSmemBytes =
-    sizeof(float) * (kRwStages * kRwStageFloats + 2 * kRwCvtFloats) + 8 * 16 + 8;
+    sizeof(float) * (kRwStages * kRwStageFloats + kRwBufs * kRwCvtFloats) + 8 * 24 + 8;
 static_assert(kRwSmemBytes <= 232448, "shared memory per CTA");
+static_assert(kRwACol + kRwBufs * 2 * kTcChunk <= kRwTmemCols, "tensor memory columns");
 
-// chunk list: rank by rank, the maps of a rank one after the other, a map's
-// chunks in row order
-__device__ __forceinline__ int wg_chunks(const WgGeom& g, int l) {
-  return (g.N * (2 * l + 1) + kTcChunk - 1) / kTcChunk;
+// Tensor maps of the two operands, one per rank (unused ranks zero).
+struct WgMaps {
+  CUtensorMap a[5];   // 3-D: 128 channels, 2l+1 components (row stride), N nodes (stride sa rows)
+  CUtensorMap b[5];   // 4-D: 128 channels, pe_l maps, 2l+1 components, N nodes (stride sb rows)
+};
+
+// nodes per K chunk of rank l, and the chunk list: rank by rank, the maps of
+// a rank one after the other, a map's chunks in node order
+__host__ __device__ __forceinline__ int wg_nodes(int l) { return kTcChunk / (2 * l + 1); }
+__host__ __device__ __forceinline__ int wg_chunks(const WgGeom& g, int l) {
+  return (g.N + wg_nodes(l) - 1) / wg_nodes(l);
 }
 __device__ __forceinline__ void wg_chunk(const WgGeom& g, int ch, int& l, int& e, int& q) {
   l = 0;
@@ -777,17 +805,17 @@ __device__ __forceinline__ void wg_chunk(const WgGeom& g, int ch, int& l, int& e
   q = ch - c0 - e * nc;
 }
 
-__global__ void __launch_bounds__(kRwThreads, 1) rows_wgrad_tc_kernel(WgGeom geo, const float* __restrict__ a,
-                                                                      const float* __restrict__ b,
+__global__ void __launch_bounds__(kRwThreads, 1) rows_wgrad_tc_kernel(WgGeom geo,
+                                                                      const __grid_constant__ WgMaps maps,
                                                                       float* __restrict__ Wb) {
   extern __shared__ __align__(1024) unsigned char smem[];
   float* st = reinterpret_cast<float*>(smem);       // stages: a rows, b rows (FP32)
-  float* cv = st + kRwStages * kRwStageFloats;      // 2 buffers: a hi, a lo, b hi, b lo
-  uint64_t* stage_full = reinterpret_cast<uint64_t*>(cv + 2 * kRwCvtFloats);
+  float* cv = st + kRwStages * kRwStageFloats;      // converted b: hi, lo
+  uint64_t* stage_full = reinterpret_cast<uint64_t*>(cv + kRwBufs * kRwCvtFloats);
   uint64_t* stage_free = stage_full + kRwStages;
   uint64_t* cvt_full = stage_free + kRwStages;
-  uint64_t* cvt_free = cvt_full + 2;
-  uint64_t* acc_full = cvt_free + 2;
+  uint64_t* cvt_free = cvt_full + kRwBufs;
+  uint64_t* acc_full = cvt_free + kRwBufs;
   uint64_t* acc_free = acc_full + 2;
   uint64_t* drain = acc_free + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
@@ -798,15 +826,17 @@ __global__ void __launch_bounds__(kRwThreads, 1) rows_wgrad_tc_kernel(WgGeom geo
   const int c_begin = (int)((long long)blockIdx.x * total / gridDim.x);
   const int c_end = (int)((long long)(blockIdx.x + 1) * total / gridDim.x);
 
-  if (warp == 0) tc::tmem_alloc(tmem_slot, 2 * kTcC);
+  if (warp == 0) tc::tmem_alloc(tmem_slot, kRwTmemCols);
   if (tid == 0) {
     for (int i = 0; i < kRwStages; ++i) {
-      tc::bar_init(&stage_full[i], 32);   // the producer's lanes, on their copies' completion
-      tc::bar_init(&stage_free[i], kRwCvtThreads / 32);   // one per converter warp
+      tc::bar_init(&stage_full[i], 1);
+      tc::bar_init(&stage_free[i], kRwCvtWarps);
+    }
+    for (int i = 0; i < kRwBufs; ++i) {
+      tc::bar_init(&cvt_full[i], kRwCvtWarps);
+      tc::bar_init(&cvt_free[i], 1);
     }
     for (int i = 0; i < 2; ++i) {
-      tc::bar_init(&cvt_full[i], kRwCvtThreads / 32);
-      tc::bar_init(&cvt_free[i], 1);
       tc::bar_init(&acc_full[i], 1);
       tc::bar_init(&acc_free[i], 128);
     }
@@ -821,47 +851,23 @@ __global__ void __launch_bounds__(kRwThreads, 1) rows_wgrad_tc_kernel(WgGeom geo
   bool fail = false;
 
   if (warp == 0) {
-    // ---------------- producer: cp.async, one 512-byte row per warp instruction ----------------
-    // The warp walks the chunk's rows (node n, component c) incrementally,
-    // 16 bytes a lane; rows past the rank's end are zero-filled, so the
-    // converters read every row unconditionally.
+    // ---------------- producer: two tiled TMA loads per chunk ----------------
     int g = 0;
-    for (int ch = c_begin; ch < c_end && !fail; ++ch, ++g) {
-      int l, e, q;
-      wg_chunk(geo, ch, l, e, q);
-      const int s = g % kRwStages;
-      bool ok = true;
-      if (lane == 0 && g >= kRwStages) ok = tc::bar_wait(&stage_free[s], ((g / kRwStages) - 1) & 1, lim);
-      if (!__shfl_sync(0xffffffffu, ok, 0)) {
-        fail = true;
-        break;
-      }
-      const int w = 2 * l + 1, R = geo.N * w;
-      const int i0 = q * kTcChunk;
-      const int nv = min(kTcChunk, R - i0);
-      const int pe = wg_pe(geo, l);
-      int n = i0 / w, c = i0 - n * w;
-      const float* ra = a + ((size_t)n * geo.sa + l * l + c) * kTcC + 4 * lane;
-      const float* rb = b + ((size_t)n * geo.sb + wg_ob(geo, l) + (size_t)c * pe + e) * kTcC + 4 * lane;
-      const long long na = (long long)(geo.sa - w + 1) * kTcC, nb = ((long long)geo.sb - (long long)(w - 1) * pe) * kTcC;
-      float* dst = st + s * kRwStageFloats + 4 * lane;
-      for (int r = 0; r < nv; ++r) {
-        cp_async16(dst + r * kTcC, ra, true);
-        cp_async16(dst + kRwRowFloats + r * kTcC, rb, true);
-        if (++c == w) {   // next node
-          c = 0;
-          ra += na;
-          rb += nb;
-        } else {
-          ra += kTcC;
-          rb += (size_t)pe * kTcC;
+    if (lane == 0) {
+      for (int ch = c_begin; ch < c_end && !fail; ++ch, ++g) {
+        int l, e, q;
+        wg_chunk(geo, ch, l, e, q);
+        const int s = g % kRwStages;
+        if (g >= kRwStages && !tc::bar_wait(&stage_free[s], ((g / kRwStages) - 1) & 1, lim)) {
+          fail = true;
+          break;
         }
+        const int nn = wg_nodes(l), rows = nn * (2 * l + 1);
+        float* dst = st + s * kRwStageFloats;
+        tc::bar_arrive_expect_tx(&stage_full[s], (uint32_t)(2 * rows * kTcC * sizeof(float)));
+        tc::tma_load_3d(dst, &maps.a[l], 0, 0, q * nn, &stage_full[s]);
+        tc::tma_load_4d(dst + kRwRowFloats, &maps.b[l], 0, e, 0, q * nn, &stage_full[s]);
       }
-      for (int r = nv; r < kTcChunk; ++r) {   // zero rows (reads nothing)
-        cp_async16(dst + r * kTcC, a, false);
-        cp_async16(dst + kRwRowFloats + r * kTcC, b, false);
-      }
-      tc::cp_async_bar_arrive(&stage_full[s]);   // one of the 32 expected arrivals
     }
     if (fail && lane == 0)   // let the copies already issued land
       for (int k = 1; k <= kRwStages && g - k >= 0; ++k)
@@ -889,27 +895,24 @@ __global__ void __launch_bounds__(kRwThreads, 1) rows_wgrad_tc_kernel(WgGeom geo
           }
           tc::fence_after_sync();
         }
-        const int bb = g & 1;
-        if (!tc::bar_wait(&cvt_full[bb], (g >> 1) & 1, lim)) {
+        const int bb = g % kRwBufs;
+        if (!tc::bar_wait(&cvt_full[bb], (g / kRwBufs) & 1, lim)) {
           fail = true;
           break;
         }
         tc::fence_after_sync();
         const uint32_t d_tmem = tmem + (uint32_t)(h & 1) * kTcC;
-        const uint32_t ah = tc::smem_addr(cv + bb * kRwCvtFloats);
-        const uint32_t al = ah + kTcBlockFloats * sizeof(float);
-        const uint32_t bh = ah + 2 * kTcBlockFloats * sizeof(float);
-        const uint32_t bl = ah + 3 * kTcBlockFloats * sizeof(float);
+        const uint32_t a_hi = tmem + kRwACol + (uint32_t)bb * 2 * kTcChunk;
+        const uint32_t bh = tc::smem_addr(cv + bb * kRwCvtFloats);
+        const uint32_t bl = bh + kTcBlockFloats * sizeof(float);
 #pragma unroll
         for (int j = 0; j < kTcChunk / 8; ++j) {
           const uint32_t kx = 2 * j * kLbo;
-          const uint64_t dah = tc::smem_desc(ah + kx, kLbo, kSbo);
-          const uint64_t dal = tc::smem_desc(al + kx, kLbo, kSbo);
           const uint64_t dbh = tc::smem_desc(bh + kx, kLbo, kSbo);
           const uint64_t dbl = tc::smem_desc(bl + kx, kLbo, kSbo);
-          tc::mma_tf32(d_tmem, dah, dbh, idesc, (run | j) != 0);
-          tc::mma_tf32(d_tmem, dal, dbh, idesc, 1u);
-          tc::mma_tf32(d_tmem, dah, dbl, idesc, 1u);
+          tc::mma_tf32_ts(d_tmem, a_hi + 8 * j, dbh, idesc, (run | j) != 0);
+          tc::mma_tf32_ts(d_tmem, a_hi + kTcChunk + 8 * j, dbh, idesc, 1u);
+          tc::mma_tf32_ts(d_tmem, a_hi + 8 * j, dbl, idesc, 1u);
         }
         tc::commit(&cvt_free[bb]);
         ++run;
@@ -922,53 +925,68 @@ __global__ void __launch_bounds__(kRwThreads, 1) rows_wgrad_tc_kernel(WgGeom geo
     }
     __syncwarp();
   } else if (warp < 10) {
-    // ---------------- converters: FP32 rows -> transposed TF32 hi / lo ----------------
-    // Thread ct takes channel k = ct % 128 of rows 4 (h + 2 m) .. + 3 (h = ct / 128,
-    // m = 0..3) of both operands: 32 conflict-free scalar loads (a warp reads
-    // 32 consecutive channels of a row), then per 4 rows one 16-byte hi and
-    // one lo store (a warp fills 512 contiguous bytes).
-    const int ct = tid - 64;   // 0 .. 255
-    const int k = ct & (kTcC - 1), h = ct >> 7;
-    const uint32_t src0 = tc::smem_addr(st) + 4u * (uint32_t)(4 * h * kTcC + k);
-    const uint32_t dst0 = tc::smem_addr(cv) + 4u * (uint32_t)tc::core_offset(k, 4 * h, kTcC);
+    // ---------------- converters: FP32 rows -> TF32 hi / lo ----------------
+    // Warps 4-7 take operand a: lane i of warp w converts channel
+    // 32 (w % 4) + i (its TMEM lane) and writes its 32 rows to 32 columns.
+    // Warps 2, 3, 8, 9 take operand b: thread t converts channel t and
+    // writes 4 rows per 16-byte store into the K-major blocks (a warp fills
+    // 512 contiguous bytes).
+    const bool op_a = warp >= 4 && warp < 8;
+    const int quarter = warp & 3;
+    const int chn = op_a ? 32 * quarter + lane : 32 * (warp < 4 ? warp - 2 : warp - 6) + lane;
+    const uint32_t src0 = tc::smem_addr(st) + 4u * (uint32_t)((op_a ? 0 : kRwRowFloats) + chn);
+    const uint32_t dstb = tc::smem_addr(cv) + 4u * (uint32_t)tc::core_offset(chn, 0, kTcC);
+    const uint32_t dsta = tmem + ((uint32_t)(32 * quarter) << 16) + kRwACol;
     int g = 0;
     for (int ch = c_begin; ch < c_end && !fail; ++ch, ++g) {
-      const int s = g % kRwStages, bb = g & 1;
-      if (!tc::bar_wait(&stage_full[s], (g / kRwStages) & 1, lim) ||
-          (g >= 2 && !tc::bar_wait(&cvt_free[bb], ((g - 2) >> 1) & 1, lim))) {
+      int l, e, q;
+      wg_chunk(geo, ch, l, e, q);
+      const int kv = wg_nodes(l) * (2 * l + 1);   // stage rows the loads wrote
+      const int s = g % kRwStages, bb = g % kRwBufs;
+      if (!tc::bar_wait(&stage_full[s], (g / kRwStages) & 1, lim)) {
         fail = true;
         break;
       }
       const uint32_t src = src0 + 4u * s * kRwStageFloats;
-      const uint32_t dst = dst0 + 4u * bb * kRwCvtFloats;
-      float v[2][4][4];
+      float v[kTcChunk];
 #pragma unroll
-      for (int op = 0; op < 2; ++op)
+      for (int r = 0; r < kTcChunk; ++r)
+        asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v[r]) : "r"(src + 4u * r * kTcC) : "memory");
 #pragma unroll
-        for (int m = 0; m < 4; ++m)
+      for (int r = 0; r < kTcChunk; ++r)
+        if (r >= kv) v[r] = 0.0f;
+      __syncwarp();   // the stage's values are in registers: release it
+      if (lane == 0) tc::bar_arrive(&stage_free[s]);
+      if (g >= kRwBufs && !tc::bar_wait(&cvt_free[bb], ((g / kRwBufs) - 1) & 1, lim)) {
+        fail = true;
+        break;
+      }
+      if (op_a) {
+        tc::fence_after_sync();
+        uint32_t hi[kTcChunk], lo[kTcChunk];
 #pragma unroll
-          for (int r = 0; r < 4; ++r)
-            asm volatile("ld.shared.f32 %0, [%1];"
-                         : "=f"(v[op][m][r])
-                         : "r"(src + 4u * (op * kRwRowFloats + (8 * m + r) * kTcC)));
+        for (int r = 0; r < kTcChunk; ++r) tc::split_tf32(v[r], hi[r], lo[r]);
+        const uint32_t ta = dsta + (uint32_t)bb * 2 * kTcChunk;
+        tc::tmem_st32(ta, hi);
+        tc::tmem_st32(ta + kTcChunk, lo);
+        tc::tmem_wait_st();
+        tc::fence_before_sync();
+      } else {
+        const uint32_t d = dstb + 4u * bb * kRwCvtFloats;
 #pragma unroll
-      for (int op = 0; op < 2; ++op)
-#pragma unroll
-        for (int m = 0; m < 4; ++m) {
+        for (int m = 0; m < kTcChunk / 4; ++m) {
           uint4 hv, lv;
-          split4(make_float4(v[op][m][0], v[op][m][1], v[op][m][2], v[op][m][3]), hv, lv);
-          const uint32_t d = dst + 4u * (op * 2 * kTcBlockFloats + m * 1024);
-          asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(d), "r"(hv.x), "r"(hv.y), "r"(hv.z),
+          split4(make_float4(v[4 * m], v[4 * m + 1], v[4 * m + 2], v[4 * m + 3]), hv, lv);
+          const uint32_t o = d + 4u * (m * (kTcC / 8) * 32);   // K group m
+          asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(o), "r"(hv.x), "r"(hv.y), "r"(hv.z),
                        "r"(hv.w) : "memory");
-          asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(d + 4u * kTcBlockFloats), "r"(lv.x),
+          asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(o + 4u * kTcBlockFloats), "r"(lv.x),
                        "r"(lv.y), "r"(lv.z), "r"(lv.w) : "memory");
         }
-      tc::fence_proxy_async();   // the generic-proxy writes, visible to the MMAs
-      __syncwarp();              // one arrival per warp (256 on one word serialise)
-      if (lane == 0) {
-        tc::bar_arrive(&cvt_full[bb]);
-        tc::bar_arrive(&stage_free[s]);
+        tc::fence_proxy_async();   // the generic-proxy writes, visible to the MMAs
       }
+      __syncwarp();
+      if (lane == 0) tc::bar_arrive(&cvt_full[bb]);
     }
   } else {
     // ---------------- drain: D[j][k] -> Wb_l[j][e 128 + k] ----------------
@@ -1012,7 +1030,7 @@ __global__ void __launch_bounds__(kRwThreads, 1) rows_wgrad_tc_kernel(WgGeom geo
   __syncthreads();
   if (warp == 0) {
     tc::fence_after_sync();
-    tc::tmem_dealloc(tmem, 2 * kTcC);
+    tc::tmem_dealloc(tmem, kRwTmemCols);
   }
 }
 
@@ -1118,15 +1136,59 @@ int launch_path_split_map(const PathGeom& g, const float* W, float* ws, cudaStre
   return cudaGetLastError() == cudaSuccess ? FC_OK : FC_ERR_CUDA;
 }
 
+// cuTensorMapEncodeTiled through the runtime's driver entry point (CUDA
+// 12.0 ABI), looked up once.
+static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static std::atomic<void*> fn{nullptr};
+  void* f = fn.load(std::memory_order_acquire);
+  if (!f) {
+    cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &f, 12000, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || !f)
+      return nullptr;
+    fn.store(f, std::memory_order_release);
+  }
+  return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+}
+
+// FP32 row tensor with `rank` dimensions: 128 channels (contiguous), then
+// dims[1..] with byte strides strides[0..]; box 128 x box[1..].
+static bool encode_rows(PFN_cuTensorMapEncodeTiled_v12000 enc, CUtensorMap* m, const float* base, int rank,
+                        const cuuint64_t* dims, const cuuint64_t* strides, const cuuint32_t* box) {
+  const cuuint32_t es[4] = {1, 1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, (cuuint32_t)rank, const_cast<float*>(base), dims, strides, box,
+             es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 int launch_rows_wgrad_tc(const WgGeom& g, const float* a, const float* b, float* Wb, cudaStream_t s) {
-  if (g.L < 0 || g.L > 4) return FC_ERR_UNSUPPORTED_RANK;
-  if (set_smem_once(g_rw_smem_set, rows_wgrad_tc_kernel, kRwSmemBytes) != FC_OK) return FC_ERR_CUDA;
+  if (g.L < 0 || g.L > 4 || g.N < 0) return FC_ERR_UNSUPPORTED_RANK;
   long long total = 0;
-  for (int l = 0; l <= g.L; ++l) total += (long long)wg_pe(g, l) * ((g.N * (2 * l + 1) + kTcChunk - 1) / kTcChunk);
+  for (int l = 0; l <= g.L; ++l) total += (long long)wg_pe(g, l) * wg_chunks(g, l);
   if (total == 0) return FC_OK;
+  if (set_smem_once(g_rw_smem_set, rows_wgrad_tc_kernel, kRwSmemBytes) != FC_OK) return FC_ERR_CUDA;
+  PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+  if (!enc) return FC_ERR_CUDA;
+  WgMaps maps;
+  memset(&maps, 0, sizeof(maps));
+  const cuuint64_t row = kTcC * sizeof(float);   // bytes per row
+  for (int l = 0; l <= g.L; ++l) {
+    const int pe = wg_pe(g, l), w = 2 * l + 1;
+    if (pe == 0) continue;
+    const cuuint64_t da[3] = {(cuuint64_t)kTcC, (cuuint64_t)w, (cuuint64_t)g.N};
+    const cuuint64_t sa[2] = {row, (cuuint64_t)g.sa * row};
+    const cuuint32_t ba[3] = {(cuuint32_t)kTcC, (cuuint32_t)w, (cuuint32_t)wg_nodes(l)};
+    const cuuint64_t db[4] = {(cuuint64_t)kTcC, (cuuint64_t)pe, (cuuint64_t)w, (cuuint64_t)g.N};
+    const cuuint64_t sb[3] = {row, (cuuint64_t)pe * row, (cuuint64_t)g.sb * row};
+    const cuuint32_t bb[4] = {(cuuint32_t)kTcC, 1u, (cuuint32_t)w, (cuuint32_t)wg_nodes(l)};
+    if (!encode_rows(enc, &maps.a[l], a + (size_t)l * l * kTcC, 3, da, sa, ba) ||
+        !encode_rows(enc, &maps.b[l], b + (size_t)wg_ob(g, l) * kTcC, 4, db, sb, bb))
+      return FC_ERR_CUDA;
+  }
   const int sms = device_sm_count();
   const int grid = total < sms ? (int)total : sms;
-  rows_wgrad_tc_kernel<<<grid, kRwThreads, kRwSmemBytes, s>>>(g, a, b, Wb);
+  rows_wgrad_tc_kernel<<<grid, kRwThreads, kRwSmemBytes, s>>>(g, maps, Wb);
   return cudaGetLastError() == cudaSuccess ? FC_OK : FC_ERR_CUDA;
 }
 
