@@ -396,7 +396,10 @@ constexpr int kPmGroup = 4;   // chunks per accumulator: one path of 128 inputs
 
 constexpr int kPmStageFloats = 3 * kTcBlockFloats;   // x (FP32), W hi, W lo
 constexpr int kPmCvtFloats = 2 * kTcBlockFloats;     // x hi, x lo
-constexpr int kPmCvtThreads = 64;                    // warps 2 and 3
+constexpr int kPmCvtThreads = 128;                   // warps 2, 3, 8 and 9
+constexpr int kPmThreads = 320;   // w0 copies, w1 issues, w2-3 and w8-9 convert, w4-7 drain
+constexpr uint32_t kPmTmemCols = 512;                 // 2 accumulators + the running sum of a tile
+constexpr uint32_t kPmSumCol = 2 * kTcRows;
 constexpr size_t kPmSmemBytes =
     sizeof(float) * (kTcStages * kPmStageFloats + 2 * kPmCvtFloats) + 8 * 16 + 8;
 static_assert(kPmSmemBytes <= 232448, "shared memory per CTA");
@@ -520,7 +523,7 @@ __global__ void __launch_bounds__(256) path_split_map_t_kernel(PathGeom g, const
   }
 }
 
-__global__ void __launch_bounds__(kTcThreads, 1) path_mix_tc_kernel(PathGeom geo,
+__global__ void __launch_bounds__(kPmThreads, 1) path_mix_tc_kernel(PathGeom geo,
                                                                     const float* __restrict__ xs,
                                                                     const float* __restrict__ ws,
                                                                     float* __restrict__ out) {
@@ -541,14 +544,14 @@ __global__ void __launch_bounds__(kTcThreads, 1) path_mix_tc_kernel(PathGeom geo
   const int u_begin = pg_unit_at(geo, (long long)blockIdx.x * total / gridDim.x);
   const int u_end = pg_unit_at(geo, (long long)(blockIdx.x + 1) * total / gridDim.x);
 
-  if (warp == 0) tc::tmem_alloc(tmem_slot, 2 * kTcRows);
+  if (warp == 0) tc::tmem_alloc(tmem_slot, kPmTmemCols);
   if (tid == 0) {
     for (int s = 0; s < kTcStages; ++s) {
       tc::bar_init(&stage_full[s], 1);
-      tc::bar_init(&stage_free[s], kPmCvtThreads + 1);   // converter threads + the MMA commit
+      tc::bar_init(&stage_free[s], kPmCvtThreads / 32 + 1);   // converter warps + the MMA commit
     }
     for (int b = 0; b < 2; ++b) {
-      tc::bar_init(&cvt_full[b], kPmCvtThreads);
+      tc::bar_init(&cvt_full[b], kPmCvtThreads / 32);
       tc::bar_init(&cvt_free[b], 1);
       tc::bar_init(&acc_full[b], 1);
       tc::bar_init(&acc_free[b], 128);
@@ -647,9 +650,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) path_mix_tc_kernel(PathGeom geo
       if (!tc::bar_wait(drain, 0, kTcDrainNs)) fail = true;
     }
     __syncwarp();
-  } else if (warp < 4) {
+  } else if (warp < 4 || warp >= 8) {
     // ---------------- converter: FP32 chunk -> TF32 hi / lo blocks ----------------
-    const int ct = tid - 64;   // 0 .. 63
+    const int ct = warp < 4 ? tid - 64 : tid - 192;   // 0 .. 127
     int g = 0;
     for (int u = u_begin; u < u_end && !fail; ++u) {
       int l, t, e;
@@ -665,7 +668,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) path_mix_tc_kernel(PathGeom geo
         const uint32_t src = tc::smem_addr(st + s * kPmStageFloats) + 16 * ct;
         const uint32_t hi = tc::smem_addr(cv + b * kPmCvtFloats) + 16 * ct;
         constexpr uint32_t kLo = kTcBlockFloats * sizeof(float), kStep = 16 * kPmCvtThreads;
-        constexpr int kIters = kTcBlockFloats / 4 / kPmCvtThreads;   // 16
+        constexpr int kIters = kTcBlockFloats / 4 / kPmCvtThreads;   // 8
         float4 v[kIters];
 #pragma unroll
         for (int i = 0; i < kIters; ++i)
@@ -682,14 +685,23 @@ __global__ void __launch_bounds__(kTcThreads, 1) path_mix_tc_kernel(PathGeom geo
                        "r"(w.y), "r"(w.z), "r"(w.w) : "memory");
         }
         tc::fence_proxy_async();   // the generic-proxy writes, visible to the MMAs
-        tc::bar_arrive(&cvt_full[b]);
-        tc::bar_arrive(&stage_free[s]);
+        __syncwarp();              // one arrival per warp
+        if (lane == 0) {
+          tc::bar_arrive(&cvt_full[b]);
+          tc::bar_arrive(&stage_free[s]);
+        }
       }
     }
   } else {
     // ---------------- epilogue: sum the groups of a tile, write out ----------------
+    // Group sums stay in TMEM (columns kPmSumCol..): the first group of a
+    // multi-group tile is copied there, later ones added; the last group is
+    // added on the way out.  A one-group tile is stored straight from its
+    // accumulator.  (128 running sums in registers capped the block at two
+    // converter warps.)
     const int ew = warp - 4;
     const int j = 32 * ew + lane;
+    const uint32_t lane_off = (uint32_t)(32 * ew) << 16;
     int h = 0;
     for (int u = u_begin; u < u_end && !fail; ++u) {
       int l, t, e;
@@ -698,32 +710,46 @@ __global__ void __launch_bounds__(kTcThreads, 1) path_mix_tc_kernel(PathGeom geo
       const int tr = t - pg_ts(geo, l);
       const int cmc = tr / geo.nb;                     // the tile's component
       const int cmn = (tr - cmc * geo.nb) * kTcRows;   // and its first node
-      float acc[kTcRows];
-      for (int gi = 0; gi < (kc + kPmGroup - 1) / kPmGroup; ++gi, ++h) {
+      const int ng = (kc + kPmGroup - 1) / kPmGroup;
+      float* o = out + ((size_t)cmn * geo.orow + pg_ooff(geo, l) + (size_t)cmc * pg_pe(geo, l) + e) * kTcC + j;
+      const size_t step = (size_t)geo.orow * kTcC;
+      const int nr = min(kTcRows, geo.N - cmn);
+      for (int gi = 0; gi < ng; ++gi, ++h) {
         if (!tc::bar_wait(&acc_full[h & 1], (h >> 1) & 1, lim)) {
           fail = true;
           break;
         }
         tc::fence_after_sync();
-        const uint32_t d_tmem = tmem + (uint32_t)(h & 1) * kTcRows + ((uint32_t)(32 * ew) << 16);
-#pragma unroll
+        const uint32_t d_tmem = tmem + (uint32_t)(h & 1) * kTcRows + lane_off;
+        const uint32_t s_tmem = tmem + kPmSumCol + lane_off;
+        const bool last = gi == ng - 1;
+#pragma unroll 1
         for (int q = 0; q < kTcRows / 32; ++q) {
           float v[32];
           tc::tmem_ld32(d_tmem + 32 * q, v);
+          if (gi > 0) {
+            float sv[32];
+            tc::tmem_ld32(s_tmem + 32 * q, sv);
 #pragma unroll
-          for (int r = 0; r < 32; ++r) acc[32 * q + r] = gi ? acc[32 * q + r] + v[r] : v[r];
+            for (int r = 0; r < 32; ++r) v[r] += sv[r];
+          }
+          if (last) {
+            float* oq = o + (size_t)(32 * q) * step;
+#pragma unroll
+            for (int r = 0; r < 32; ++r) {
+              if (32 * q + r < nr) *oq = v[r];
+              oq += step;
+            }
+          } else {
+            uint32_t w[32];
+#pragma unroll
+            for (int r = 0; r < 32; ++r) w[r] = __float_as_uint(v[r]);
+            tc::tmem_st32(s_tmem + 32 * q, w);
+          }
         }
+        if (!last) tc::tmem_wait_st();
         tc::fence_before_sync();
         tc::bar_arrive(&acc_free[h & 1]);
-      }
-      if (fail) break;
-      float* o = out + ((size_t)cmn * geo.orow + pg_ooff(geo, l) + (size_t)cmc * pg_pe(geo, l) + e) * kTcC + j;
-      const size_t step = (size_t)geo.orow * kTcC;
-      const int nr = min(kTcRows, geo.N - cmn);
-#pragma unroll
-      for (int r = 0; r < kTcRows; ++r) {
-        if (r < nr) *o = acc[r];
-        o += step;
       }
     }
   }
@@ -732,7 +758,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) path_mix_tc_kernel(PathGeom geo
   __syncthreads();
   if (warp == 0) {
     tc::fence_after_sync();
-    tc::tmem_dealloc(tmem, 2 * kTcRows);
+    tc::tmem_dealloc(tmem, kPmTmemCols);
   }
 }
 
@@ -1211,7 +1237,7 @@ int launch_path_mix_tc(const PathGeom& g, const float* xs, const float* ws, floa
   if (T == 0) return FC_OK;
   const int sms = device_sm_count();
   const int grid = T < sms ? T : sms;
-  path_mix_tc_kernel<<<grid, kTcThreads, kPmSmemBytes, s>>>(g, xs, ws, out);
+  path_mix_tc_kernel<<<grid, kPmThreads, kPmSmemBytes, s>>>(g, xs, ws, out);
   return cudaGetLastError() == cudaSuccess ? FC_OK : FC_ERR_CUDA;
 }
 
