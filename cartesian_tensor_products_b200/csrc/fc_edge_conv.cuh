@@ -19,7 +19,8 @@
 // broadcasts and applies them to the lane's 4 channels with packed FP32x2
 // FMAs.  Sender indices and edge vectors come from a 32-edge register
 // window (one per lane) read with warp shuffles.  With 4 groups every SMSP
-// runs one instruction stream (warp g of each resident CTA).
+// runs one instruction stream (warp g of each resident CTA).  At C = 64 a
+// warp runs two receivers, one per half-warp (fwd_warp_half).
 #pragma once
 #include "fc_common.cuh"
 #include "fc_device.cuh"
@@ -144,13 +145,94 @@ __device__ __forceinline__ void fwd_warp(const ConvArgs& a, float* smem, int lan
   if (act) Grp::store(a.z + (size_t)u * a.zrow * C + k0, C, a.sum_paths, acc);
 }
 
+// C = 64: a warp covers two receivers, half-warp h (lanes 16 h .. 16 h + 15,
+// 4 channels each) runs receiver 2 unit + h, so no lane idles.  Each half
+// keeps its own 16-edge register window of senders and edge vectors, and the
+// M window holds 8 edges per half (the same shared memory as the full warp's
+// 16); both halves walk their edges in step, a half whose receiver has fewer
+// edges (or none) sitting out the remaining iterations.
+template <class Grp, int S, int MW, bool ENV>
+__device__ __forceinline__ void fwd_warp_half(const ConvArgs& a, float* smem, int lane, int unit) {
+  constexpr int STAGE = Grp::NROW * 128;
+  constexpr int C = 64;
+  constexpr int HW = MW / 2;   // edges per half in one M window
+  static_assert(S <= 16 && HW >= 1, "ring depth within a 16-edge window");
+  const int h = lane >> 4, hl = lane & 15, hbase = lane & 16;
+  const int u = 2 * unit + h;
+  const bool has = u < a.n_nodes;
+  const int k0 = hl * 4;
+  int e0 = has ? __ldg(a.rowptr + u) : 0, e1 = has ? __ldg(a.rowptr + u + 1) : 0;
+  e0 = e0 < 0 ? 0 : (e0 > a.n_edges ? a.n_edges : e0);
+  e1 = e1 < e0 ? e0 : (e1 > a.n_edges ? a.n_edges : e1);
+  const int len = e1 - e0;
+  int lmax = len;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) lmax = max(lmax, __shfl_xor_sync(0xffffffffu, lmax, o));
+  float* st = smem + Grp::RING_OFF + lane * 4;
+  float* mwin = smem + Grp::MWIN_OFF + h * HW * Grp::MSTRIDE;
+
+  float4 acc[Grp::NA];
+#pragma unroll
+  for (int i = 0; i < Grp::NA; ++i) acc[i] = zero4();
+
+  // lane (h, i) holds edge e0 + 16 j + i of its half's receiver
+  EdgeWin cur = load_win(a, e0 + hl, e1);
+  EdgeWin nxt = load_win(a, e0 + 16 + hl, e1);
+
+#pragma unroll
+  for (int s = 0; s < S; ++s) {
+    const int v = __shfl_sync(0xffffffffu, cur.v, hbase + s);
+    if (s < len) issue_edge<Grp>(a, C, st + s * STAGE, e0 + s, v, k0, true);
+    cp_async_commit();
+  }
+
+  for (int p = 0; p < lmax; ++p) {
+    if (p > 0 && (p & 15) == 0) {
+      cur = nxt;
+      nxt = load_win(a, e0 + p + 16 + hl, e1);
+    }
+    if ((p % HW) == 0) {
+      // M entries of the next HW edges of each half, lanes (h, 0 .. HW-1)
+      const int src = hbase + (p & 15) + (hl % HW);
+      const float rx = __shfl_sync(0xffffffffu, cur.rx, src);
+      const float ry = __shfl_sync(0xffffffffu, cur.ry, src);
+      const float rz = __shfl_sync(0xffffffffu, cur.rz, src);
+      __syncwarp();
+      if (hl < HW && p + hl < len) {
+        const float r = sqrtf(rx * rx + ry * ry + rz * rz);
+        const float inv = 1.0f / r;
+        float es, esp;
+        edge_envelope(a.envelope, r, a.r_cut, a.edge_scale, es, esp);
+        Grp::template make_m<ENV>(rx * inv, ry * inv, rz * inv, es, mwin + hl * Grp::MSTRIDE);
+      }
+      __syncwarp();
+    }
+    const int slot = p % S;
+    cp_async_wait<S - 1>();
+    if (p < len) Grp::template accum<ENV>(acc, st + slot * STAGE, mwin + (p % HW) * Grp::MSTRIDE);
+    const int pn = p + S;
+    int v;
+    if ((pn >> 4) == (p >> 4))
+      v = __shfl_sync(0xffffffffu, cur.v, hbase + (pn & 15));
+    else
+      v = __shfl_sync(0xffffffffu, nxt.v, hbase + (pn & 15));
+    if (pn < len) issue_edge<Grp>(a, C, st + slot * STAGE, e0 + pn, v, k0, true);
+    cp_async_commit();
+  }
+  cp_async_wait<0>();
+  if (has) Grp::store(a.z + (size_t)u * a.zrow * C + k0, C, a.sum_paths, acc);
+}
+
 template <int L, int CC, bool ENV, int g>
 __device__ __forceinline__ void dispatch_fwd(int grp, const ConvArgs& a, float* smem, int lane,
                                              int unit) {
   if constexpr (g < FwdMeta<L>::G) {
     using Grp = FwdGroup<L, FwdMeta<L>::G, g>;
     if (grp == g) {
-      fwd_warp<Grp, FwdMeta<L>::S, FwdMeta<L>::MWIN, CC, ENV>(a, smem, lane, unit);
+      if constexpr (CC == 64)
+        fwd_warp_half<Grp, FwdMeta<L>::S, FwdMeta<L>::MWIN, ENV>(a, smem, lane, unit);
+      else
+        fwd_warp<Grp, FwdMeta<L>::S, FwdMeta<L>::MWIN, CC, ENV>(a, smem, lane, unit);
       return;
     }
     dispatch_fwd<L, CC, ENV, g + 1>(grp, a, smem, lane, unit);
@@ -169,7 +251,7 @@ __global__ void __launch_bounds__(FwdMeta<L>::WARPS * 32, 2) edge_conv_fwd_kerne
     dispatch_fwd<L, CC, ENV, 0>(warp, a, smem, lane, blockIdx.x);
   } else {
     constexpr int WARPS = FwdMeta<L>::WARPS;
-    const int units = a.n_nodes * a.ntiles;
+    const int units = CC == 64 ? (a.n_nodes + 1) / 2 : a.n_nodes * a.ntiles;
     const int nb = (units + WARPS - 1) / WARPS;
     const int grp = blockIdx.x / nb;
     const int unit = (blockIdx.x - grp * nb) * WARPS + warp;
@@ -185,7 +267,8 @@ static int launch_fwd_cc(const ConvArgs& a, cudaStream_t s) {
   const size_t smem = sizeof(float) * (size_t)FwdMeta<L>::SMEM_FLOATS;
   static DeviceFlags configured;
   if (set_smem_once(configured, edge_conv_fwd_kernel<L, CC, ENV>, smem) != FC_OK) return FC_ERR_CUDA;
-  const long long units = (long long)a.n_nodes * a.ntiles;
+  // CC = 64: a unit is a pair of receivers (one per half-warp)
+  const long long units = CC == 64 ? ((long long)a.n_nodes + 1) / 2 : (long long)a.n_nodes * a.ntiles;
   constexpr int WARPS = FwdMeta<L>::WARPS;
   const long long blocks =
       FwdMeta<L>::GROUP_MAJOR ? (units + WARPS - 1) / WARPS * FwdMeta<L>::G : units;
@@ -244,8 +327,12 @@ inline int conv_setup(const fc_conv_desc* d, int n_nodes, int n_send, int n_edge
 
 template <int L>
 static int launch_fwd(const ConvArgs& a, cudaStream_t s) {
-  if (a.envelope) return a.C == 128 ? launch_fwd_cc<L, 128, true>(a, s) : launch_fwd_cc<L, 0, true>(a, s);
-  return a.C == 128 ? launch_fwd_cc<L, 128, false>(a, s) : launch_fwd_cc<L, 0, false>(a, s);
+  if (a.envelope) {
+    if (a.C == 128) return launch_fwd_cc<L, 128, true>(a, s);
+    return a.C == 64 ? launch_fwd_cc<L, 64, true>(a, s) : launch_fwd_cc<L, 0, true>(a, s);
+  }
+  if (a.C == 128) return launch_fwd_cc<L, 128, false>(a, s);
+  return a.C == 64 ? launch_fwd_cc<L, 64, false>(a, s) : launch_fwd_cc<L, 0, false>(a, s);
 }
 
 }  // namespace fc

@@ -172,3 +172,43 @@ def test_envelope_forward(fc, sum_paths):
     ref = O.edge_conv(3, 3, 3, 8, wl["edge_index"], wl["edge_vec"], wl["x"],
                       wl["w"] * s[:, None, None], wl["n_nodes"], sum_paths=sum_paths)
     assert rel_err(z, ref) <= FWD_TOL
+
+
+@pytest.mark.parametrize("L", [1, 2, 3, 4, 5])
+def test_half_warp_pairs_c64(fc, L):
+    """C = 64 runs two receivers per warp, one per half-warp.  An odd receiver
+    count leaves the last warp's second half without a receiver; paired
+    receivers of different degree (0 beside 33, 64 beside 65, 16 beside 17,
+    ...) walk their edges in step, the shorter one sitting out.  Rank 5 is
+    checked on a receiver sample (the FP64 oracle is slow there)."""
+    degrees = [0, 33, 1, 0, 31, 64, 65, 2, 16, 17, 15, 0, 70, 3, 5]
+    N = len(degrees) + 60                                   # 75 receivers
+    ei, ev = ragged_graph(N, degrees + [4] * 60, 6.0, 500 + L)
+    wl = dict(n_nodes=N, lmax=L, channels=64, edge_index=ei, edge_vec=ev,
+              **W.conv_inputs(N, ei, L, 64, 64 + L))
+    z = gpu_conv(fc, wl)
+    rows = list(range(N)) if L <= 4 else [0, 1, 2, 7, 8, 9, N - 2, N - 1]
+    m = np.zeros(N, np.uint8)
+    m[rows] = 1
+    ref = oracle_conv(wl, recv_mask=m)
+    assert rel_err(z[rows], ref[rows]) <= FWD_TOL
+    zero_rows = [i for i, k in enumerate(degrees) if k == 0]
+    assert np.all(z[zero_rows] == 0)
+
+
+@pytest.mark.parametrize("sum_paths", [False, True])
+def test_half_warp_pairs_c64_envelope(fc, sum_paths):
+    """The C = 64 pairing with the cosine envelope and with path sums."""
+    degrees = [5, 0, 12, 40, 41, 3, 1] + [2] * 44
+    N = len(degrees)                                        # 51 receivers
+    ei, ev = ragged_graph(N, degrees, 3.0, 77)
+    inp = W.conv_inputs(N, ei, 3, 64, 78, sum_paths=sum_paths)
+    r_cut, scale = 2.5, 0.7
+    s, _, _ = O.envelope(ev, r_cut, scale)
+    assert (s == 0).any() and (s > 0).any()
+    rowptr = fc.build_rowptr(dev(ei), dev(ev), N)
+    z = fc.edge_conv(3, rowptr, dev(ei), dev(ev), dev(inp["x"]), dev(inp["w"]), sum_paths=sum_paths,
+                     envelope=(r_cut, scale)).cpu().numpy()
+    ref = O.edge_conv(3, 3, 3, 64, ei, ev, inp["x"], inp["w"] * s[:, None, None], N,
+                      sum_paths=sum_paths)
+    assert rel_err(z, ref) <= FWD_TOL
