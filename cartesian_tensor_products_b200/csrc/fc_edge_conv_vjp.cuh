@@ -24,7 +24,8 @@
 // atomic add per x_bar row, as Algorithm 2 adds sender gradients
 // atomically), and y_bar through d_(a,b1) = <g_a, w x_b1>; y_bar is folded
 // into u_bar = (dT/du)^T y_bar, reduced over the warp with shuffles and
-// added atomically (3 floats per warp and edge) into r_bar.
+// added atomically (3 floats per warp and edge) into r_bar.  At C = 64 a
+// warp runs two receivers, one per half-warp (vjp_warp_half).
 #pragma once
 #include "fc_common.cuh"
 #include "fc_device.cuh"
@@ -197,13 +198,144 @@ __device__ __forceinline__ void vjp_warp(const VjpArgs& a, float* smem, int lane
   cp_async_wait<0>();
 }
 
+// C = 64: two receivers per warp, half-warp h (lanes 16 h .. 16 h + 15, 4
+// channels each) runs receiver 2 unit + h.  As in the forward's pairing,
+// each half keeps its own 16-edge register window and 8 edges of the M
+// window, and the halves walk their edges in step; the per-edge reduction of
+// the edge-vector gradient runs over the 16 lanes of a half, whose first
+// lane adds it into r_bar.
+template <class Grp, int S, int MW>
+__device__ __forceinline__ void vjp_warp_half(const VjpArgs& a, float* smem, int lane, int unit) {
+  constexpr int STAGE = Grp::NROW * 128;
+  constexpr int NYB = Grp::NYD > 0 ? Grp::NYD : 1;
+  constexpr int C = 64;
+  constexpr int HW = MW / 2;
+  static_assert(S <= 16 && HW >= 1, "ring depth within a 16-edge window");
+  const int h = lane >> 4, hl = lane & 15, hbase = lane & 16;
+  const int u = 2 * unit + h;
+  const bool has = u < a.n_nodes;
+  const int k0 = hl * 4;
+  int e0 = has ? __ldg(a.rowptr + u) : 0, e1 = has ? __ldg(a.rowptr + u + 1) : 0;
+  e0 = e0 < 0 ? 0 : (e0 > a.n_edges ? a.n_edges : e0);
+  e1 = e1 < e0 ? e0 : (e1 > a.n_edges ? a.n_edges : e1);
+  const int len = e1 - e0;
+  int lmax = len;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) lmax = max(lmax, __shfl_xor_sync(0xffffffffu, lmax, o));
+  if (lmax == 0) return;
+  float* st = smem + Grp::RING_OFF + lane * 4;
+  float* mwin = smem + Grp::MWIN_OFF + h * HW * Grp::MSTRIDE;
+  const bool wstore = a.wbar != nullptr;
+  float* wbase = a.wbar != nullptr ? a.wbar : a.xbar;   // any valid pointer when unused
+
+  float4 gr[Grp::NA];
+  if (has) {
+    Grp::load_g(a.g + (size_t)u * a.zrow * C + k0, C, a.sum_paths, gr);
+  } else {
+#pragma unroll
+    for (int i = 0; i < Grp::NA; ++i) gr[i] = zero4();
+  }
+  float4 xb[Grp::NX];
+#pragma unroll
+  for (int i = 0; i < Grp::NX; ++i) xb[i] = zero4();
+  float yb[NYB];
+#pragma unroll
+  for (int i = 0; i < NYB; ++i) yb[i] = 0.0f;
+
+  VEdgeWin cur = vload_win(a, e0 + hl, e1);
+  VEdgeWin nxt = vload_win(a, e0 + 16 + hl, e1);
+#pragma unroll
+  for (int s = 0; s < S; ++s) {
+    const int v = __shfl_sync(0xffffffffu, cur.v, hbase + s);
+    if (s < len) vissue_edge<Grp>(a, C, st + s * STAGE, e0 + s, v, k0, true);
+    cp_async_commit();
+  }
+
+  for (int p = 0; p < lmax; ++p) {
+    const bool on = p < len;
+    const int q = e0 + p;
+    if (p > 0 && (p & 15) == 0) {
+      cur = nxt;
+      nxt = vload_win(a, q + 16 + hl, e1);
+    }
+    if ((p % HW) == 0) {
+      const int src = hbase + (p & 15) + (hl % HW);
+      const float rx = __shfl_sync(0xffffffffu, cur.rx, src);
+      const float ry = __shfl_sync(0xffffffffu, cur.ry, src);
+      const float rz = __shfl_sync(0xffffffffu, cur.rz, src);
+      __syncwarp();
+      if (hl < HW && p + hl < len) {
+        const float r = sqrtf(rx * rx + ry * ry + rz * rz);
+        const float inv = 1.0f / r;
+        float es, esp;
+        edge_envelope(a.envelope, r, a.r_cut, a.edge_scale, es, esp);
+        Grp::make_row(rx * inv, ry * inv, rz * inv, es, esp, mwin + hl * Grp::MSTRIDE);
+      }
+      __syncwarp();
+    }
+    const int slot = p % S;
+    cp_async_wait<S - 1>();
+    const float* m = mwin + (p % HW) * Grp::MSTRIDE;
+    if (on)
+      Grp::edge(gr, st + slot * STAGE, m, xb, yb, wbase + (wstore ? (size_t)q * a.P * C + k0 : 0), C,
+                wstore);
+    // sender gradient
+    const int v = __shfl_sync(0xffffffffu, cur.v, hbase + (p & 15));
+    if (on && a.xbar != nullptr && v >= 0 && v < a.n_send) {
+      Grp::flush_xbar(a.xbar + (size_t)v * a.xrow * C + k0, C, xb);
+    } else {
+#pragma unroll
+      for (int i = 0; i < Grp::NX; ++i) xb[i] = zero4();
+    }
+    // edge-vector gradient
+    if constexpr (Grp::NYD > 0) {
+      if (a.rbar != nullptr) {
+        float ux = 0.0f, uy = 0.0f, uz = 0.0f, rho = 0.0f;
+        if (on) Grp::ubar(yb, m, ux, uy, uz, rho);
+#pragma unroll
+        for (int o = 8; o > 0; o >>= 1) {
+          ux += __shfl_xor_sync(0xffffffffu, ux, o);
+          uy += __shfl_xor_sync(0xffffffffu, uy, o);
+          uz += __shfl_xor_sync(0xffffffffu, uz, o);
+          rho += __shfl_xor_sync(0xffffffffu, rho, o);
+        }
+        const float rx = __shfl_sync(0xffffffffu, cur.rx, hbase + (p & 15));
+        const float ry = __shfl_sync(0xffffffffu, cur.ry, hbase + (p & 15));
+        const float rz = __shfl_sync(0xffffffffu, cur.rz, hbase + (p & 15));
+        if (hl == 0 && on) {
+          const float inv = 1.0f / sqrtf(rx * rx + ry * ry + rz * rz);
+          const float nx = rx * inv, ny = ry * inv, nz = rz * inv;
+          const float dotu = ux * nx + uy * ny + uz * nz;
+          atomicAdd(a.rbar + 3 * (size_t)q + 0, (ux - nx * dotu) * inv + rho * nx);
+          atomicAdd(a.rbar + 3 * (size_t)q + 1, (uy - ny * dotu) * inv + rho * ny);
+          atomicAdd(a.rbar + 3 * (size_t)q + 2, (uz - nz * dotu) * inv + rho * nz);
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < NYB; ++i) yb[i] = 0.0f;
+    }
+    const int pn = p + S;
+    int vn;
+    if ((pn >> 4) == (p >> 4))
+      vn = __shfl_sync(0xffffffffu, cur.v, hbase + (pn & 15));
+    else
+      vn = __shfl_sync(0xffffffffu, nxt.v, hbase + (pn & 15));
+    if (pn < len) vissue_edge<Grp>(a, C, st + slot * STAGE, e0 + pn, vn, k0, true);
+    cp_async_commit();
+  }
+  cp_async_wait<0>();
+}
+
 template <int L, int CC, int g>
 __device__ __forceinline__ void dispatch_vjp(int grp, const VjpArgs& a, float* smem, int lane,
                                              int unit) {
   if constexpr (g < VjpMeta<L>::G) {
     using Grp = VjpGroup<L, VjpMeta<L>::G, g>;
     if (grp == g) {
-      vjp_warp<Grp, VjpMeta<L>::S, VjpMeta<L>::MWIN, CC>(a, smem, lane, unit);
+      if constexpr (CC == 64)
+        vjp_warp_half<Grp, VjpMeta<L>::S, VjpMeta<L>::MWIN>(a, smem, lane, unit);
+      else
+        vjp_warp<Grp, VjpMeta<L>::S, VjpMeta<L>::MWIN, CC>(a, smem, lane, unit);
       return;
     }
     dispatch_vjp<L, CC, g + 1>(grp, a, smem, lane, unit);
@@ -218,7 +350,7 @@ __global__ void __launch_bounds__(VjpMeta<L>::WARPS * 32, VjpMeta<L>::MINB) edge
   extern __shared__ __align__(16) float smem[];
   constexpr int WARPS = VjpMeta<L>::WARPS;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int units = a.n_nodes * a.ntiles;
+  const int units = CC == 64 ? (a.n_nodes + 1) / 2 : a.n_nodes * a.ntiles;   // CC = 64: receiver pairs
   const int nb = (units + WARPS - 1) / WARPS;
   const int grp = blockIdx.x / nb;
   const int unit = (blockIdx.x - grp * nb) * WARPS + warp;
@@ -233,7 +365,7 @@ static int launch_vjp_cc(const VjpArgs& a, cudaStream_t s) {
   const size_t smem = sizeof(float) * (size_t)VjpMeta<L>::SMEM_FLOATS;
   static DeviceFlags configured;
   if (set_smem_once(configured, edge_conv_vjp_kernel<L, CC>, smem) != FC_OK) return FC_ERR_CUDA;
-  const long long units = (long long)a.n_nodes * a.ntiles;
+  const long long units = CC == 64 ? ((long long)a.n_nodes + 1) / 2 : (long long)a.n_nodes * a.ntiles;
   constexpr int WARPS = VjpMeta<L>::WARPS;
   const long long blocks = (units + WARPS - 1) / WARPS * VjpMeta<L>::G;
   if (blocks > 0x7fffffffLL) return FC_ERR_ARG;
@@ -298,7 +430,8 @@ inline int vjp_setup(const fc_conv_desc* d, int n_nodes, int n_send, int n_edges
 
 template <int L>
 static int launch_vjp(const VjpArgs& a, cudaStream_t s) {
-  return a.C == 128 ? launch_vjp_cc<L, 128>(a, s) : launch_vjp_cc<L, 0>(a, s);
+  if (a.C == 128) return launch_vjp_cc<L, 128>(a, s);
+  return a.C == 64 ? launch_vjp_cc<L, 64>(a, s) : launch_vjp_cc<L, 0>(a, s);
 }
 
 }  // namespace fc

@@ -154,3 +154,36 @@ def test_envelope_vjp(fc, sum_paths):
     rrb = rrb + ((rwb * wl["w"]).sum((1, 2)) * sp)[:, None] * ev64 / r[:, None]
     check_all((xb.cpu().numpy(), wb.cpu().numpy(), rb.cpu().numpy()),
               (rxb, rwb * s[:, None, None], rrb))
+
+
+@pytest.mark.parametrize("L", [1, 2, 3, 4])
+def test_vjp_half_warp_pairs_c64(fc, L):
+    """C = 64 runs two receivers per warp, one per half-warp: an odd receiver
+    count leaves the last warp's second half without a receiver, and paired
+    receivers of unequal degree (0 beside 33, 64 beside 65, 16 beside 17)
+    walk their edges in step; the edge-vector gradient is reduced over each
+    half's 16 lanes."""
+    degrees = [0, 33, 1, 0, 31, 64, 65, 2, 16, 17, 15, 0, 70, 3, 5] + [3] * 60
+    N = len(degrees)                                        # 75 receivers
+    ei, ev = ragged_graph(N, degrees, 6.0, 900 + L)
+    wl = dict(n_nodes=N, lmax=L, channels=64, edge_index=ei, edge_vec=ev,
+              **W.conv_inputs(N, ei, L, 64, 910 + L, with_grad=True))
+    check_all(gpu_vjp(fc, wl, wl["g"]), oracle_vjp(wl, wl["g"]))
+
+
+def test_vjp_half_warp_pairs_c64_sum_paths_envelope(fc):
+    """The C = 64 pairing with path sums and the cosine envelope."""
+    degrees = [5, 0, 12, 40, 41, 3, 1] + [2] * 44
+    N = len(degrees)                                        # 51 receivers
+    ei, ev = ragged_graph(N, degrees, 3.0, 79)
+    inp = W.conv_inputs(N, ei, 3, 64, 80, with_grad=True, sum_paths=True)
+    r_cut, scale = 2.5, 0.7
+    s, sp, r = O.envelope(ev, r_cut, scale)
+    rowptr = fc.build_rowptr(dev(ei), dev(ev), N)
+    xb, wb, rb = fc.edge_conv_vjp(3, rowptr, dev(ei), dev(ev), dev(inp["x"]), dev(inp["w"]),
+                                  dev(inp["g"]), sum_paths=True, envelope=(r_cut, scale))
+    rxb, rwb, rrb = O.edge_conv_vjp(3, 3, 3, 64, ei, ev, inp["x"], inp["w"] * s[:, None, None],
+                                    inp["g"], N, sum_paths=True)
+    rrb = rrb + ((rwb * inp["w"]).sum((1, 2)) * sp)[:, None] * ev.astype(np.float64) / r[:, None]
+    check_all((xb.cpu().numpy(), wb.cpu().numpy(), rb.cpu().numpy()),
+              (rxb, rwb * s[:, None, None], rrb))
