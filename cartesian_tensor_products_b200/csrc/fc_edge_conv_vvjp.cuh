@@ -27,7 +27,8 @@
 // G = D^T y_bar, H_u = sum y_bar d^2y/du du), the warp reduces them and lane
 // 0 adds (I - u u^T) D^T y_hat / |r| plus the Hessian-vector product
 //   [-(w (u.G) + u (w.G)) + (I - u u^T) H_u w] / |r| - (I - u u^T) G (u.vr) / |r|^2,
-// w = (I - u u^T) vr / |r|, atomically into r_hat.
+// w = (I - u u^T) vr / |r|, atomically into r_hat.  At C = 64 (ranks 1-4)
+// a warp runs two receivers, one per half-warp (vvjp_warp_half).
 #pragma once
 #include "fc_common.cuh"
 #include "fc_device.cuh"
@@ -89,6 +90,32 @@ __device__ __forceinline__ void vvissue_edge(const VvjpArgs& a, int C, float* st
   const size_t wo = (size_t)q * a.P * C + kk;
   Grp::issue(st, a.x + xo, (a.vx ? a.vx : a.x) + xo, a.w + wo, (a.vw ? a.vw : a.w) + wo, C, vok,
              vok && a.vx != nullptr, act, act && a.vw != nullptr);
+}
+
+// Lane 0 of a reduced group: (I - u u^T) D^T y_hat / |r| plus the
+// Hessian-vector product, added into r_hat of edge q.
+template <class Grp>
+__device__ __forceinline__ void vvjp_rhat_add(const VvjpArgs& a, const float* m, const float (&red)[12],
+                                              int q) {
+  const float* sc = m + Grp::SBASE;
+  const float ux = sc[0], uy = sc[1], uz = sc[2];
+  const float wx = sc[3], wy = sc[4], wz = sc[5];
+  const float inv = sc[6], uv = sc[7];
+  const float ua = ux * red[0] + uy * red[1] + uz * red[2];
+  float ox = (red[0] - ux * ua) * inv, oy = (red[1] - uy * ua) * inv, oz = (red[2] - uz * ua) * inv;
+  const float Gx = red[3], Gy = red[4], Gz = red[5];
+  const float uG = ux * Gx + uy * Gy + uz * Gz, wG = wx * Gx + wy * Gy + wz * Gz;
+  const float Hwx = red[6] * wx + red[7] * wy + red[8] * wz;
+  const float Hwy = red[7] * wx + red[9] * wy + red[10] * wz;
+  const float Hwz = red[8] * wx + red[10] * wy + red[11] * wz;
+  const float uHw = ux * Hwx + uy * Hwy + uz * Hwz;
+  const float c2 = uv * inv * inv;
+  ox += (-(wx * uG + ux * wG) + Hwx - ux * uHw) * inv - (Gx - ux * uG) * c2;
+  oy += (-(wy * uG + uy * wG) + Hwy - uy * uHw) * inv - (Gy - uy * uG) * c2;
+  oz += (-(wz * uG + uz * wG) + Hwz - uz * uHw) * inv - (Gz - uz * uG) * c2;
+  atomicAdd(a.rhat + 3 * (size_t)q + 0, ox);
+  atomicAdd(a.rhat + 3 * (size_t)q + 1, oy);
+  atomicAdd(a.rhat + 3 * (size_t)q + 2, oz);
 }
 
 template <class Grp, int S, int MW, int CC>
@@ -178,29 +205,7 @@ __device__ __forceinline__ void vvjp_warp(const VvjpArgs& a, float* smem, int la
         for (int o = 16; o > 0; o >>= 1)
 #pragma unroll
           for (int i = 0; i < 12; ++i) red[i] += __shfl_xor_sync(0xffffffffu, red[i], o);
-        if (lane == 0) {
-          const float* sc = m + Grp::SBASE;
-          const float ux = sc[0], uy = sc[1], uz = sc[2];
-          const float wx = sc[3], wy = sc[4], wz = sc[5];
-          const float inv = sc[6], uv = sc[7];
-          // (I - u u^T) D^T y_hat / |r|
-          const float ua = ux * red[0] + uy * red[1] + uz * red[2];
-          float ox = (red[0] - ux * ua) * inv, oy = (red[1] - uy * ua) * inv, oz = (red[2] - uz * ua) * inv;
-          // Hessian-vector product of <y_bar, y(r)> along vr
-          const float Gx = red[3], Gy = red[4], Gz = red[5];
-          const float uG = ux * Gx + uy * Gy + uz * Gz, wG = wx * Gx + wy * Gy + wz * Gz;
-          const float Hwx = red[6] * wx + red[7] * wy + red[8] * wz;
-          const float Hwy = red[7] * wx + red[9] * wy + red[10] * wz;
-          const float Hwz = red[8] * wx + red[10] * wy + red[11] * wz;
-          const float uHw = ux * Hwx + uy * Hwy + uz * Hwz;
-          const float c2 = uv * inv * inv;
-          ox += (-(wx * uG + ux * wG) + Hwx - ux * uHw) * inv - (Gx - ux * uG) * c2;
-          oy += (-(wy * uG + uy * wG) + Hwy - uy * uHw) * inv - (Gy - uy * uG) * c2;
-          oz += (-(wz * uG + uz * wG) + Hwz - uz * uHw) * inv - (Gz - uz * uG) * c2;
-          atomicAdd(a.rhat + 3 * (size_t)q + 0, ox);
-          atomicAdd(a.rhat + 3 * (size_t)q + 1, oy);
-          atomicAdd(a.rhat + 3 * (size_t)q + 2, oz);
-        }
+        if (lane == 0) vvjp_rhat_add<Grp>(a, m, red, q);
       }
 #pragma unroll
       for (int i = 0; i < NDB; ++i) yh[i] = yb[i] = 0.0f;
@@ -220,13 +225,137 @@ __device__ __forceinline__ void vvjp_warp(const VvjpArgs& a, float* smem, int la
   if (a.ghat != nullptr && act) Grp::store_ghat(a.ghat + (size_t)u * a.zrow * C + k0, C, a.sum_paths, gh);
 }
 
+// C = 64: two receivers per warp, half-warp h (lanes 16 h .. 16 h + 15, 4
+// channels each) runs receiver 2 unit + h, as in the forward's and the VJP's
+// pairing: per half a 16-edge register window, 8 edges of the M window, and
+// the reduction of the 12 u-space numbers over the half's 16 lanes.
+template <class Grp, int S, int MW>
+__device__ __forceinline__ void vvjp_warp_half(const VvjpArgs& a, float* smem, int lane, int unit) {
+  constexpr int STAGE = Grp::NROW * 128;
+  constexpr int NDB = Grp::ND > 0 ? Grp::ND : 1;
+  constexpr int C = 64;
+  constexpr int HW = MW / 2;
+  static_assert(S <= 16 && HW >= 1, "ring depth within a 16-edge window");
+  const int h = lane >> 4, hl = lane & 15, hbase = lane & 16;
+  const int u = 2 * unit + h;
+  const bool has = u < a.n_nodes;
+  const int k0 = hl * 4;
+  int e0 = has ? __ldg(a.rowptr + u) : 0, e1 = has ? __ldg(a.rowptr + u + 1) : 0;
+  e0 = e0 < 0 ? 0 : (e0 > a.n_edges ? a.n_edges : e0);
+  e1 = e1 < e0 ? e0 : (e1 > a.n_edges ? a.n_edges : e1);
+  const int len = e1 - e0;
+  int lmax = len;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) lmax = max(lmax, __shfl_xor_sync(0xffffffffu, lmax, o));
+  if (lmax == 0) return;
+  float* st = smem + Grp::RING_OFF + lane * 4;
+  float* mwin = smem + Grp::MWIN_OFF + h * HW * Grp::MSTRIDE;
+  const bool wstore = a.what != nullptr;
+  float* wbase = a.what != nullptr ? a.what : a.ghat;   // any valid pointer when unused
+
+  float4 gr[Grp::NA], gh[Grp::NA];
+  if (has) {
+    Grp::load_g(a.g + (size_t)u * a.zrow * C + k0, C, a.sum_paths, gr);
+  } else {
+#pragma unroll
+    for (int i = 0; i < Grp::NA; ++i) gr[i] = zero4();
+  }
+#pragma unroll
+  for (int i = 0; i < Grp::NA; ++i) gh[i] = zero4();
+  float4 xh[Grp::NX];
+#pragma unroll
+  for (int i = 0; i < Grp::NX; ++i) xh[i] = zero4();
+  float yh[NDB], yb[NDB];
+#pragma unroll
+  for (int i = 0; i < NDB; ++i) yh[i] = yb[i] = 0.0f;
+
+  VvEdgeWin cur = vvload_win(a, e0 + hl, e1);
+  VvEdgeWin nxt = vvload_win(a, e0 + 16 + hl, e1);
+#pragma unroll
+  for (int s = 0; s < S; ++s) {
+    const int v = __shfl_sync(0xffffffffu, cur.v, hbase + s);
+    if (s < len) vvissue_edge<Grp>(a, C, st + s * STAGE, e0 + s, v, k0, true);
+    cp_async_commit();
+  }
+
+  for (int p = 0; p < lmax; ++p) {
+    const bool on = p < len;
+    const int q = e0 + p;
+    if (p > 0 && (p & 15) == 0) {
+      cur = nxt;
+      nxt = vvload_win(a, q + 16 + hl, e1);
+    }
+    if ((p % HW) == 0) {
+      const int src = hbase + (p & 15) + (hl % HW);
+      const float rx = __shfl_sync(0xffffffffu, cur.rx, src);
+      const float ry = __shfl_sync(0xffffffffu, cur.ry, src);
+      const float rz = __shfl_sync(0xffffffffu, cur.rz, src);
+      const float vrx = __shfl_sync(0xffffffffu, cur.vrx, src);
+      const float vry = __shfl_sync(0xffffffffu, cur.vry, src);
+      const float vrz = __shfl_sync(0xffffffffu, cur.vrz, src);
+      __syncwarp();
+      if (hl < HW && p + hl < len) {
+        const float inv = 1.0f / sqrtf(rx * rx + ry * ry + rz * rz);
+        Grp::make_row(rx * inv, ry * inv, rz * inv, inv, vrx, vry, vrz, mwin + hl * Grp::MSTRIDE);
+      }
+      __syncwarp();
+    }
+    const int slot = p % S;
+    cp_async_wait<S - 1>();
+    const float* m = mwin + (p % HW) * Grp::MSTRIDE;
+    if (on)
+      Grp::edge(gr, gh, st + slot * STAGE, m, xh, yh, yb,
+                wbase + (wstore ? (size_t)q * a.P * C + k0 : 0), C, wstore);
+    // sender gradient
+    const int v = __shfl_sync(0xffffffffu, cur.v, hbase + (p & 15));
+    if (on && a.xhat != nullptr && v >= 0 && v < a.n_send) {
+      Grp::flush_xhat(a.xhat + (size_t)v * a.xrow * C + k0, C, xh);
+    } else {
+#pragma unroll
+      for (int i = 0; i < Grp::NX; ++i) xh[i] = zero4();
+    }
+    // edge-vector gradient
+    if constexpr (Grp::ND > 0) {
+      if (a.rhat != nullptr) {
+        float red[12];
+        if (on) {
+          Grp::fold(yh, yb, m, red);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 12; ++i) red[i] = 0.0f;
+        }
+#pragma unroll
+        for (int o = 8; o > 0; o >>= 1)
+#pragma unroll
+          for (int i = 0; i < 12; ++i) red[i] += __shfl_xor_sync(0xffffffffu, red[i], o);
+        if (hl == 0 && on) vvjp_rhat_add<Grp>(a, m, red, q);
+      }
+#pragma unroll
+      for (int i = 0; i < NDB; ++i) yh[i] = yb[i] = 0.0f;
+    }
+    const int pn = p + S;
+    int vn;
+    if ((pn >> 4) == (p >> 4))
+      vn = __shfl_sync(0xffffffffu, cur.v, hbase + (pn & 15));
+    else
+      vn = __shfl_sync(0xffffffffu, nxt.v, hbase + (pn & 15));
+    if (pn < len) vvissue_edge<Grp>(a, C, st + slot * STAGE, e0 + pn, vn, k0, true);
+    cp_async_commit();
+  }
+  cp_async_wait<0>();
+  if (a.ghat != nullptr && has) Grp::store_ghat(a.ghat + (size_t)u * a.zrow * C + k0, C, a.sum_paths, gh);
+}
+
 template <int L, int CC, int g>
 __device__ __forceinline__ void dispatch_vvjp(int grp, const VvjpArgs& a, float* smem, int lane,
                                               int unit) {
   if constexpr (g < VvjpMeta<L>::G) {
     using Grp = VvjpGroup<L, VvjpMeta<L>::G, g>;
     if (grp == g) {
-      vvjp_warp<Grp, VvjpMeta<L>::S, VvjpMeta<L>::MWIN, CC>(a, smem, lane, unit);
+      if constexpr (CC == 64)
+        vvjp_warp_half<Grp, VvjpMeta<L>::S, VvjpMeta<L>::MWIN>(a, smem, lane, unit);
+      else
+        vvjp_warp<Grp, VvjpMeta<L>::S, VvjpMeta<L>::MWIN, CC>(a, smem, lane, unit);
       return;
     }
     dispatch_vvjp<L, CC, g + 1>(grp, a, smem, lane, unit);
@@ -238,7 +367,7 @@ __global__ void __launch_bounds__(VvjpMeta<L>::WARPS * 32, 1) edge_conv_vvjp_ker
   extern __shared__ __align__(16) float smem[];
   constexpr int WARPS = VvjpMeta<L>::WARPS;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int units = a.n_nodes * a.ntiles;
+  const int units = CC == 64 ? (a.n_nodes + 1) / 2 : a.n_nodes * a.ntiles;   // CC = 64: receiver pairs
   const int nb = (units + WARPS - 1) / WARPS;
   const int grp = blockIdx.x / nb;
   const int unit = (blockIdx.x - grp * nb) * WARPS + warp;
@@ -289,7 +418,7 @@ int launch_vvjp_cc(const VvjpArgs& a, cudaStream_t s) {
   const size_t smem = sizeof(float) * (size_t)VvjpMeta<L>::SMEM_FLOATS;
   static DeviceFlags configured;
   if (set_smem_once(configured, edge_conv_vvjp_kernel<L, CC>, smem) != FC_OK) return FC_ERR_CUDA;
-  const long long units = (long long)a.n_nodes * a.ntiles;
+  const long long units = CC == 64 ? ((long long)a.n_nodes + 1) / 2 : (long long)a.n_nodes * a.ntiles;
   constexpr int WARPS = VvjpMeta<L>::WARPS;
   const long long blocks = (units + WARPS - 1) / WARPS * VvjpMeta<L>::G;
   if (blocks > 0x7fffffffLL) return FC_ERR_ARG;

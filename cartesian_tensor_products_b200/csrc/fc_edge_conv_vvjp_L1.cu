@@ -4,6 +4,6 @@
 
 namespace fc {
 int launch_vvjp_rank1(const VvjpArgs& a, cudaStream_t s) {
-  return launch_vvjp_cc<1, 0>(a, s);
+  return a.C == 64 ? launch_vvjp_cc<1, 64>(a, s) : launch_vvjp_cc<1, 0>(a, s);
 }
 }  // namespace fc

@@ -4,6 +4,7 @@
 
 namespace fc {
 int launch_vvjp_rank3(const VvjpArgs& a, cudaStream_t s) {
-  return a.C == 128 ? launch_vvjp_cc<3, 128>(a, s) : launch_vvjp_cc<3, 0>(a, s);
+  if (a.C == 128) return launch_vvjp_cc<3, 128>(a, s);
+  return a.C == 64 ? launch_vvjp_cc<3, 64>(a, s) : launch_vvjp_cc<3, 0>(a, s);
 }
 }  // namespace fc

@@ -4,6 +4,6 @@
 
 namespace fc {
 int launch_vvjp_rank4(const VvjpArgs& a, cudaStream_t s) {
-  return launch_vvjp_cc<4, 0>(a, s);
+  return a.C == 64 ? launch_vvjp_cc<4, 64>(a, s) : launch_vvjp_cc<4, 0>(a, s);
 }
 }  // namespace fc

@@ -164,3 +164,17 @@ def test_envelope_is_refused_and_empty_graph(fc):
     gh, xh, wh, rh = fc.edge_conv_vjp_vjp(2, rp, e0, v0, x, w, g, v_x=x)
     torch.cuda.synchronize()
     assert torch.all(gh == 0) and torch.all(xh == 0) and wh.numel() == 0 and rh.numel() == 0
+
+
+@pytest.mark.parametrize("L,sum_paths", [(1, False), (2, True), (3, False), (3, True), (4, False)])
+def test_half_warp_pairs_c64(fc, L, sum_paths):
+    """C = 64 runs two receivers per warp, one per half-warp: an odd receiver
+    count leaves the last warp's second half without a receiver, and paired
+    receivers of unequal degree (0 beside 33, 16 beside 17, 40 beside 2) walk
+    their edges in step; the 12 u-space numbers of r_hat are reduced over each
+    half's 16 lanes."""
+    degrees = [0, 33, 1, 0, 31, 40, 2, 16, 17, 15, 0, 3] + [3] * 25
+    N = len(degrees)                                        # 37 receivers
+    ei, ev = ragged_graph(N, degrees, 6.0, 300 + L)
+    wl = case(L, 64, ei, ev, N, 310 + L, sum_paths=sum_paths)
+    check_all(gpu_vvjp(fc, wl, sum_paths=sum_paths), oracle_vvjp(wl, sum_paths=sum_paths))
