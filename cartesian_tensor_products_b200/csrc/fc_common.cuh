@@ -195,8 +195,8 @@ PathGeom path_geom(int L, int N, const int* kc);
 PathGeom path_geom_maps(int L, int N, const int* kc, const int* pe);
 // natural [N][(L+1)^2][128] -> FP32 operand tiles with k_l = 4 (the map of phi_1)
 int launch_path_split_rows(const PathGeom& g, const float* in, float* xs, cudaStream_t s);
-// the maps, rank l's ([128][32 k_l] row-major) at W + 4096 sum_{l'<l} k_l',
-// -> split blocks at ws + pg_wbase(l)
+// the maps, rank l's ([128 e_l][32 k_l] row-major, map e = rows 128 e ..) at
+// W + 4096 sum_{l'<l} k_l' e_l', -> split blocks at ws + pg_wbase(l)
 int launch_path_split_map(const PathGeom& g, const float* W, float* ws, cudaStream_t s);
 // k_l = 4, e_l = P_l maps per rank: map e of rank l is the transposed block e
 // of Wq_l = [128][P_l 128] (rank l at Wq + 128 128 sum_{l'<l} P_l'):

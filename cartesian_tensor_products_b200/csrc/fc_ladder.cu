@@ -65,8 +65,9 @@ __global__ void __launch_bounds__(128) ladder_tp_kernel(int N, int C, const floa
 }
 
 // The same product written straight into the FP32 component-major tiles of
-// the tensor-core map (PathGeom with k_l = 4, C = 128): component c of rank
-// l of node n is row n mod 128 of tile c nb + n / 128 of that rank.  A CTA
+// the tensor-core map (PathGeom with k_l = CW / 32, CW = 128 or 256 channels):
+// component c of rank l of node n is row n mod 128 of tile c nb + n / 128 of
+// that rank.  A CTA
 // takes 8 consecutive nodes x 32 consecutive channels: it first stages both
 // operands (every component, as 16-byte cp.async copies: 8 per thread) in
 // shared memory, rows padded to 36 floats so that the reads below hit 32
@@ -75,13 +76,13 @@ __global__ void __launch_bounds__(128) ladder_tp_kernel(int N, int C, const floa
 // 128-byte core matrix.
 constexpr int kCmPad = 36;   // floats per staged (node, component) row of 32 channels
 
-template <int L>
+template <int L, int CW>
 __global__ void __launch_bounds__(256, 2) ladder_tp_cm_kernel(PathGeom g, const float* __restrict__ Av,
                                                               const float* __restrict__ A1,
                                                               const float* __restrict__ W,
                                                               float* __restrict__ xs) {
   using TP = LadderTP<L>;
-  constexpr int C = 128;
+  constexpr int C = CW;
   constexpr int NY = TP::NY;
   extern __shared__ __align__(16) float sa[];   // [operand][component][node][kCmPad]
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -116,7 +117,7 @@ __global__ void __launch_bounds__(256, 2) ladder_tp_cm_kernel(PathGeom g, const 
   for (int l = 0; l <= L; ++l) {
 #pragma unroll
     for (int c = 0; c < 2 * l + 1; ++c)
-      xs[pg_xbase(g, l) + (long long)(c * g.nb + (n >> 7)) * 4 * 4096 + cofs] = o[l * l + c];
+      xs[pg_xbase(g, l) + (long long)(c * g.nb + (n >> 7)) * (CW / 32) * 4096 + cofs] = o[l * l + c];
   }
 }
 
@@ -412,23 +413,32 @@ static int tp_dispatch(int L, int N, int C, const float* Av, const float* A1, co
   return FC_ERR_UNSUPPORTED_RANK;
 }
 
-template <int L>
+template <int L, int CW>
 static int launch_tp_cm(const PathGeom& g, const float* Av, const float* A1, const float* W, float* xs,
                         cudaStream_t s) {
   const size_t smem = sizeof(float) * 2 * (L + 1) * (L + 1) * 8 * kCmPad;
   static DeviceFlags configured;
-  if (set_smem_once(configured, ladder_tp_cm_kernel<L>, smem) != FC_OK) return FC_ERR_CUDA;
-  ladder_tp_cm_kernel<L><<<dim3((g.N + 7) / 8, 4), 256, smem, s>>>(g, Av, A1, W, xs);
+  if (set_smem_once(configured, ladder_tp_cm_kernel<L, CW>, smem) != FC_OK) return FC_ERR_CUDA;
+  ladder_tp_cm_kernel<L, CW><<<dim3((g.N + 7) / 8, CW / 32), 256, smem, s>>>(g, Av, A1, W, xs);
   return cudaGetLastError() == cudaSuccess ? FC_OK : FC_ERR_CUDA;
 }
 
-static int tp_cm_dispatch(int L, const PathGeom& g, const float* Av, const float* A1, const float* W,
+static int tp_cm_dispatch(int L, int C, const PathGeom& g, const float* Av, const float* A1, const float* W,
                           float* xs, cudaStream_t s) {
+  if (C == 256) {
+    switch (L) {
+      case 1: return launch_tp_cm<1, 256>(g, Av, A1, W, xs, s);
+      case 2: return launch_tp_cm<2, 256>(g, Av, A1, W, xs, s);
+      case 3: return launch_tp_cm<3, 256>(g, Av, A1, W, xs, s);
+      case 4: return launch_tp_cm<4, 256>(g, Av, A1, W, xs, s);
+      default: return FC_ERR_UNSUPPORTED_RANK;
+    }
+  }
   switch (L) {
-    case 1: return launch_tp_cm<1>(g, Av, A1, W, xs, s);
-    case 2: return launch_tp_cm<2>(g, Av, A1, W, xs, s);
-    case 3: return launch_tp_cm<3>(g, Av, A1, W, xs, s);
-    case 4: return launch_tp_cm<4>(g, Av, A1, W, xs, s);
+    case 1: return launch_tp_cm<1, 128>(g, Av, A1, W, xs, s);
+    case 2: return launch_tp_cm<2, 128>(g, Av, A1, W, xs, s);
+    case 3: return launch_tp_cm<3, 128>(g, Av, A1, W, xs, s);
+    case 4: return launch_tp_cm<4, 128>(g, Av, A1, W, xs, s);
     default: return FC_ERR_UNSUPPORTED_RANK;
   }
 }
@@ -481,17 +491,26 @@ static size_t tc_scratch_floats(int L, int N) {
   return mix_tc_operand_floats(L, N) + mix_tc_matrix_floats(L);
 }
 
-// Tensor-core forward: the product as FP32 component-major tiles (k_l = 4)
-static PathGeom fwd_geom(int L, int N) {
-  const int kc[5] = {4, 4, 4, 4, 4};
-  return path_geom(L, N, kc);
+// Tensor-core forward at C = 128 or 256: the product as FP32 component-major
+// tiles of K = C inputs (k_l = C / 32); at C = 256 each rank's 256 x 256
+// matrix is two maps of 128 output channels (e_l = 2), and output row
+// (n, c, e) of the map kernel is channels 128 e .. 128 e + 127 of node n's
+// component c, the natural layout.
+static bool fwd_tc(int L, int C) { return mix_tc_supported(L, 128) && (C == 128 || C == 256); }
+
+static PathGeom fwd_geom(int L, int N, int C) {
+  const int k = C / 32;
+  const int kc[5] = {k, k, k, k, k};
+  if (C == 128) return path_geom(L, N, kc);
+  const int pe[5] = {2, 2, 2, 2, 2};
+  return path_geom_maps(L, N, kc, pe);
 }
 
 size_t fc_product_ladder_workspace_size(const fc_ladder_desc* d, int n_nodes) {
   if (check_ladder_desc(d) != FC_OK || n_nodes < 0) return 0;
   const int NY = (d->lmax + 1) * (d->lmax + 1);
-  if (mix_tc_supported(d->lmax, d->channels)) {
-    const PathGeom g = fwd_geom(d->lmax, n_nodes);
+  if (fwd_tc(d->lmax, d->channels)) {
+    const PathGeom g = fwd_geom(d->lmax, n_nodes, d->channels);
     return sizeof(float) * (size_t)(pg_xbase(g, g.L + 1) + pg_wbase(g, g.L + 1));
   }
   return sizeof(float) * (size_t)n_nodes * NY * d->channels;
@@ -516,18 +535,18 @@ int fc_product_ladder(const fc_ladder_desc* d, int n_nodes, const float* A1, con
   const int NY = (L + 1) * (L + 1);
   const size_t plane = (size_t)n_nodes * NY * C;
   const int P = num_paths(L);
-  if (S > 0 && mix_tc_supported(L, C)) {
+  if (S > 0 && fwd_tc(L, C)) {
     // tensor cores: the product is written as FP32 component-major tiles,
     // the map kernel (K = 128 per rank, split to TF32 hi / lo in shared
     // memory) writes the states; z = A_1 + sum of the states at the end.
     // Rows past the last node of a tile are never written: the MMA column of
     // such a row depends on that row alone and is not stored.
-    const PathGeom g = fwd_geom(L, n_nodes);
+    const PathGeom g = fwd_geom(L, n_nodes, C);
     float* xs = static_cast<float*>(workspace);
     float* wsm = xs + pg_xbase(g, L + 1);
     for (int v = 1; v <= S; ++v) {
       const float* Av = v == 1 ? A1 : states + (size_t)(v - 2) * plane;
-      if ((st = tp_cm_dispatch(L, g, Av, A1, path_w + (size_t)(v - 1) * P * C, xs, s)) != FC_OK ||
+      if ((st = tp_cm_dispatch(L, C, g, Av, A1, path_w + (size_t)(v - 1) * P * C, xs, s)) != FC_OK ||
           (st = launch_path_split_map(g, mix_w + (size_t)(v - 1) * (L + 1) * C * C, wsm, s)) != FC_OK ||
           (st = launch_path_mix_tc(g, xs, wsm, states + (size_t)(v - 1) * plane, s)) != FC_OK)
         return st;

@@ -469,17 +469,19 @@ __global__ void __launch_bounds__(256) path_split_rows_kernel(PathGeom g, const 
   }
 }
 
+// Map e of rank l is rows 128 e .. 128 e + 127 of the rank's [128 e_l][K]
+// matrix (e_l = 1: the whole [128][K] map).
 __global__ void __launch_bounds__(256) path_split_map_kernel(PathGeom g, const float* __restrict__ W,
                                                              float* __restrict__ ws) {
-  const int l = blockIdx.y, c = blockIdx.x;
+  const int l = blockIdx.y, c = blockIdx.x, e = blockIdx.z;
   if (l > g.L) return;
   const int kc = pg_kc(g, l);
-  if (c >= kc) return;
+  if (c >= kc || e >= pg_pe(g, l)) return;
   const int K = 32 * kc;
   long long woff = 0;
-  for (int r = 0; r < l; ++r) woff += 4096LL * pg_kc(g, r);
-  const float* Wl = W + woff;
-  float* hi = ws + pg_wbase(g, l) + (size_t)c * kTcBlockFloats;
+  for (int r = 0; r < l; ++r) woff += 4096LL * pg_kc(g, r) * pg_pe(g, r);
+  const float* Wl = W + woff + (long long)e * kTcC * K;
+  float* hi = ws + pg_wbase(g, l) + (long long)e * 2 * kc * kTcBlockFloats + (size_t)c * kTcBlockFloats;
 #pragma unroll
   for (int it = 0; it < 4; ++it) {
     const int idx = it * 256 + threadIdx.x;   // 0 .. 1023
@@ -1155,10 +1157,13 @@ int launch_path_split_rows(const PathGeom& g, const float* in, float* xs, cudaSt
 }
 
 int launch_path_split_map(const PathGeom& g, const float* W, float* ws, cudaStream_t s) {
-  int kmax = 0;
-  for (int l = 0; l <= g.L; ++l) kmax = pg_kc(g, l) > kmax ? pg_kc(g, l) : kmax;
-  if (kmax == 0) return FC_OK;
-  path_split_map_kernel<<<dim3(kmax, g.L + 1), 256, 0, s>>>(g, W, ws);
+  int kmax = 0, emax = 0;
+  for (int l = 0; l <= g.L; ++l) {
+    kmax = pg_kc(g, l) > kmax ? pg_kc(g, l) : kmax;
+    emax = pg_pe(g, l) > emax ? pg_pe(g, l) : emax;
+  }
+  if (kmax == 0 || emax == 0) return FC_OK;
+  path_split_map_kernel<<<dim3(kmax, g.L + 1, emax), 256, 0, s>>>(g, W, ws);
   return cudaGetLastError() == cudaSuccess ? FC_OK : FC_ERR_CUDA;
 }
 

@@ -73,6 +73,27 @@ def test_tensor_core_mix_c128(fc, L, order, N):
         assert rel_err(mwb[v], rm[v]) <= VJP_TOL
 
 
+@pytest.mark.parametrize("L,order,N", [(1, 3, 70), (2, 2, 33), (3, 4, 37), (3, 2, 300), (4, 3, 21)])
+def test_tensor_core_forward_c256(fc, L, order, N):
+    """C = 256: the forward's tcgen05 maps take K = 256 inputs per row and
+    split each rank's 256 x 256 matrix into two maps of 128 output channels
+    (ragged last tiles; N = 300 gives three tiles per component); the VJP
+    runs the FP32 kernels at this width."""
+    C = 256
+    wl = dict(lmax=L, channels=C, order=order, **W.ladder_inputs(N, L, C, order, 2500 + L + N))
+    states, z, a1b, pwb, mwb = run_gpu(fc, wl, wl["gz"])
+    assert fc.device_error() == 0
+    rs, rz = O.ladder(L, C, order, wl["A1"], wl["path_w"], wl["mix_w"])
+    assert rel_err(z, rz) <= FWD_TOL
+    for v in range(order - 1):
+        assert rel_err(states[v], rs[v]) <= FWD_TOL
+    ra, rp, rm = O.ladder_vjp(L, C, order, wl["A1"], wl["path_w"], wl["mix_w"], wl["gz"])
+    assert rel_err(a1b, ra) <= VJP_TOL
+    for v in range(order - 1):
+        assert rel_err(pwb[v], rp[v]) <= VJP_TOL
+        assert rel_err(mwb[v], rm[v]) <= VJP_TOL
+
+
 def test_caller_workspace_too_small_is_refused(fc):
     """A caller-provided scratch buffer is passed with its real size; one
     byte short of the query is refused on the host (FC_ERR_WORKSPACE)."""

@@ -5,7 +5,8 @@ The sizes follow the scratch layouts the header states:
 * tensor-core path (C = 128): the product as FP32 tiles of 128 nodes per
   rank and component, with K = 128 P_l inputs per row for the full ladder
   (Sec. 5 Eq. 2, every path kept) or K = 128 for the path-reduced ladder;
-  plus one step's maps as TF32 hi and lo;
+  plus one step's maps as TF32 hi and lo; the path-reduced ladder's forward
+  also at C = 256 (K = 256, two 128-row maps per rank);
 * ladder VJP: four product states, plus at C = 128 the gradient as split
   tiles and one step's split matrices;
 * SIMT path: one product state (full ladder: the convolution's output row
@@ -63,6 +64,10 @@ def test_ladder_forward(fc, L, N):
     maps = (L + 1) * 2 * 128 * 128
     assert query(fc, "fc_product_ladder_workspace_size", L, 128, 4, N) == 4 * (product + maps)
     assert query(fc, "fc_product_ladder_workspace_size", L, 64, 4, N) == 4 * N * NY * 64
+    # C = 256: K = 256 inputs per row, each rank's matrix as two 128-row maps
+    product = NY * blocks(N) * 128 * 256
+    maps = (L + 1) * 2 * 256 * 256
+    assert query(fc, "fc_product_ladder_workspace_size", L, 256, 4, N) == 4 * (product + maps)
 
 
 @pytest.mark.parametrize("L", [1, 2, 3, 4])
