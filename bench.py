@@ -893,7 +893,8 @@ def run_grid(args):
                 v_ms, _ = time_events(lambda: fc.product_ladder_vjp(L, order, A1, pw, mw, res["s"], gz),
                                       steps, 3, stream)
                 lad.append({"lmax": L, "order": order, "channels": C, "fwd_ms": f_ms, "vjp_ms": v_ms,
-                            "mix": "tcgen05 TF32x3" if C == 128 else "FP32 SIMT"})
+                            "mix": ("tcgen05 TF32x3" if C == 128 else
+                                    "tcgen05 TF32x3 fwd, FP32 SIMT VJP" if C == 256 else "FP32 SIMT")})
                 del A1, pw, mw, gz, res
                 torch.cuda.empty_cache()
     clocks = sampler.stop()
