@@ -193,14 +193,14 @@ __host__ __device__ __forceinline__ int pg_ooff(const PathGeom& g, int l) {
 PathGeom path_geom(int L, int N, const int* kc);
 // the same with pe[l] maps of rank l and path-slot output rows
 PathGeom path_geom_maps(int L, int N, const int* kc, const int* pe);
-// natural [N][(L+1)^2][128] -> FP32 operand tiles with k_l = 4 (the map of phi_1)
+// natural [N][(L+1)^2][32 k] -> FP32 operand tiles with k_l = k = 4 or 8 for every rank
 int launch_path_split_rows(const PathGeom& g, const float* in, float* xs, cudaStream_t s);
 // the maps, rank l's ([128 e_l][32 k_l] row-major, map e = rows 128 e ..) at
 // W + 4096 sum_{l'<l} k_l' e_l', -> split blocks at ws + pg_wbase(l)
 int launch_path_split_map(const PathGeom& g, const float* W, float* ws, cudaStream_t s);
-// k_l = 4, e_l = P_l maps per rank: map e of rank l is the transposed block e
-// of Wq_l = [128][P_l 128] (rank l at Wq + 128 128 sum_{l'<l} P_l'):
-// A(j', t) = Wq_l[t][e 128 + j']
+// e_l maps per rank: map e of rank l is the transposed block e of
+// Wq_l = [32 k_l][128 e_l] (rank l at Wq + 4096 sum_{l'<l} k_l' e_l'):
+// A(j', t) = Wq_l[t][e 128 + j'] (k_l = 4 or 8)
 int launch_path_split_map_t(const PathGeom& g, const float* Wq, float* ws, cudaStream_t s);
 // out[n][l^2 + c][j] = sum_k W_l[j][k] x_l[(n, c)][k]
 int launch_path_mix_tc(const PathGeom& g, const float* xs, const float* ws, float* out, cudaStream_t s);

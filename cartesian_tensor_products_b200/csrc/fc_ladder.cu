@@ -572,8 +572,14 @@ size_t fc_product_ladder_vjp_workspace_size(const fc_ladder_desc* d, int n_nodes
   const int NY = (d->lmax + 1) * (d->lmax + 1);
   size_t f = 4 * (size_t)n_nodes * NY * d->channels;
   // tensor cores: the split gradient and the matrices (for B_bar = A_bar M;
-  // the weight gradient reads FP32 rows)
-  if (mix_tc_supported(d->lmax, d->channels)) f += tc_scratch_floats(d->lmax, n_nodes);
+  // the weight gradient reads FP32 rows); at C = 256 the gradient as FP32
+  // tiles of K = 256 and one step's two transposed maps per rank
+  if (mix_tc_supported(d->lmax, d->channels)) {
+    f += tc_scratch_floats(d->lmax, n_nodes);
+  } else if (fwd_tc(d->lmax, d->channels)) {
+    const PathGeom g = fwd_geom(d->lmax, n_nodes, d->channels);
+    f += (size_t)(pg_xbase(g, g.L + 1) + pg_wbase(g, g.L + 1));
+  }
   return sizeof(float) * f;
 }
 
@@ -612,8 +618,12 @@ int fc_product_ladder_vjp(const fc_ladder_desc* d, int n_nodes, const float* A1,
   float* Bbar = ws + plane;
   float* Ab[2] = {ws + 2 * plane, ws + 3 * plane};
   const bool tc = mix_tc_supported(L, C);
-  float* xs = ws + 4 * plane;                                   // tensor-core path only
-  float* wsm = tc ? xs + mix_tc_operand_floats(L, n_nodes) : nullptr;
+  // C = 256: B_bar = A_bar M on the tcgen05 maps (the transposed matrix as two
+  // maps of 128 output channels, K = 256); the weight gradient stays FP32 SIMT
+  const bool tc256 = !tc && fwd_tc(L, C);
+  const PathGeom g256 = tc256 ? fwd_geom(L, n_nodes, C) : PathGeom{};
+  float* xs = ws + 4 * plane;                                   // tensor-core paths only
+  float* wsm = tc ? xs + mix_tc_operand_floats(L, n_nodes) : tc256 ? xs + pg_xbase(g256, L + 1) : nullptr;
   const float* Anext_bar = gz;           // gradient of A_{v+1}
   for (int v = S; v >= 1; --v) {
     const float* Av = v == 1 ? A1 : states + (size_t)(v - 2) * plane;
@@ -635,6 +645,13 @@ int fc_product_ladder_vjp(const fc_ladder_desc* d, int n_nodes, const float* A1,
           (st = launch_mix_tc_split_matrix(1, L, M, wsm, s)) != FC_OK ||
           (st = launch_mix_tc(L, n_nodes, xs, wsm, Bbar, s)) != FC_OK ||
           (st = launch_rows_wgrad_tc(node_wg_geom(L, n_nodes), Anext_bar, B, Mbar, s)) != FC_OK)
+        return st;
+    } else if (tc256) {
+      if ((st = tp_dispatch(L, n_nodes, C, Av, A1, W, B, s)) != FC_OK ||
+          (st = launch_path_split_rows(g256, Anext_bar, xs, s)) != FC_OK ||
+          (st = launch_path_split_map_t(g256, M, wsm, s)) != FC_OK ||
+          (st = launch_path_mix_tc(g256, xs, wsm, Bbar, s)) != FC_OK ||
+          (st = launch_wgrad(L, n_nodes, C, Anext_bar, B, Mbar, s)) != FC_OK)
         return st;
     } else {
       if ((st = tp_dispatch(L, n_nodes, C, Av, A1, W, B, s)) != FC_OK ||

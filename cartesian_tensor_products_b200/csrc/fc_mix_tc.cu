@@ -454,9 +454,11 @@ __global__ void __launch_bounds__(256) path_split_rows_kernel(PathGeom g, const 
   const int t = blockIdx.x, c = blockIdx.y;
   const int p = threadIdx.x, lane = p & 31;
   const int l = pg_rank(g, t);
+  const int kc = pg_kc(g, l);   // rows of 32 kc channels (128 or 256)
+  if (c >= kc) return;
   const int tr = t - pg_ts(g, l);
   const int comp = tr / g.nb, n0 = (tr - comp * g.nb) * kTcRows;
-  float* dst = xs + pg_xbase(g, l) + (size_t)tr * 4 * kTcBlockFloats + c * kTcBlockFloats;
+  float* dst = xs + pg_xbase(g, l) + (size_t)tr * kc * kTcBlockFloats + c * kTcBlockFloats;
 #pragma unroll
   for (int it = 0; it < 4; ++it) {
     const int r = 16 * (p >> 5) + 8 * (it >> 1) + (lane & 7);
@@ -464,7 +466,8 @@ __global__ void __launch_bounds__(256) path_split_rows_kernel(PathGeom g, const 
     const int n = n0 + r;
     float4 v = zero4();
     if (n < g.N)
-      v = __ldg(reinterpret_cast<const float4*>(in + ((size_t)n * g.NY + l * l + comp) * kTcC + c * kTcChunk) + q);
+      v = __ldg(reinterpret_cast<const float4*>(in + ((size_t)n * g.NY + l * l + comp) * (kTcChunk * kc) +
+                                                c * kTcChunk) + q);
     *reinterpret_cast<float4*>(dst + tc::core_offset(r, 4 * q, kTcRows)) = v;
   }
 }
@@ -495,18 +498,22 @@ __global__ void __launch_bounds__(256) path_split_map_kernel(PathGeom g, const f
   }
 }
 
-// Map e of rank l (k_l = 4): A(j', t) = Wq_l[t][e 128 + j'], the transposed
-// block e of Wq_l = [128][P_l 128] at Wq + 16384 sum_{l'<l} P_l', split to hi /
-// lo blocks at ws + pg_wbase(l) + e 8 4096.  One CTA per (K chunk, map, rank).
+// Map e of rank l: A(j', t) = Wq_l[t][e 128 + j'], the transposed block e of
+// Wq_l = [32 k_l][128 e_l] at Wq + 4096 sum_{l'<l} k_l' e_l' (the full
+// ladder: k_l = 4, e_l = P_l; the ladder VJP at 256 channels: k_l = 8, e_l = 2,
+// Wq_l = M_l), split to hi / lo blocks at ws + pg_wbase(l) + e 2 k_l 4096.
+// One CTA per (K chunk, map, rank).
 __global__ void __launch_bounds__(256) path_split_map_t_kernel(PathGeom g, const float* __restrict__ Wq,
                                                                float* __restrict__ ws) {
   const int c = blockIdx.x, e = blockIdx.y, l = blockIdx.z;
   if (l > g.L || e >= pg_pe(g, l)) return;
-  long long qoff = 0;
-  for (int r = 0; r < l; ++r) qoff += 16384LL * pg_pe(g, r);
+  const int kc = pg_kc(g, l);
+  if (c >= kc) return;
+  long long qoff = 0;   // Wq_r is [32 k_r][128 e_r]
+  for (int r = 0; r < l; ++r) qoff += 4096LL * pg_kc(g, r) * pg_pe(g, r);
   const int row = kTcC * pg_pe(g, l);   // floats per row of Wq_l
   const float* Wl = Wq + qoff;
-  float* hi = ws + pg_wbase(g, l) + (long long)e * 8 * kTcBlockFloats + (size_t)c * kTcBlockFloats;
+  float* hi = ws + pg_wbase(g, l) + (long long)e * 2 * kc * kTcBlockFloats + (size_t)c * kTcBlockFloats;
 #pragma unroll
   for (int it = 0; it < 4; ++it) {
     const int idx = it * 256 + threadIdx.x;   // 0 .. 1023
@@ -521,7 +528,7 @@ __global__ void __launch_bounds__(256) path_split_map_t_kernel(PathGeom g, const
     split4(v, h, w);
     const int off = tc::core_offset(j, 4 * q, kTcC);
     *reinterpret_cast<uint4*>(hi + off) = h;
-    *reinterpret_cast<uint4*>(hi + 4 * kTcBlockFloats + off) = w;
+    *reinterpret_cast<uint4*>(hi + (size_t)kc * kTcBlockFloats + off) = w;
   }
 }
 
@@ -1149,10 +1156,10 @@ PathGeom path_geom_maps(int L, int N, const int* kc, const int* pe) {
 
 int launch_path_split_rows(const PathGeom& g, const float* in, float* xs, cudaStream_t s) {
   for (int l = 0; l <= g.L; ++l)
-    if (pg_kc(g, l) != 4) return FC_ERR_ARG;
+    if (pg_kc(g, l) != pg_kc(g, 0) || (pg_kc(g, l) != 4 && pg_kc(g, l) != 8)) return FC_ERR_ARG;
   const int T = pg_ts(g, g.L + 1);
   if (T == 0) return FC_OK;
-  path_split_rows_kernel<<<dim3(T, kTcChunks), 256, 0, s>>>(g, in, xs);
+  path_split_rows_kernel<<<dim3(T, pg_kc(g, 0)), 256, 0, s>>>(g, in, xs);
   return cudaGetLastError() == cudaSuccess ? FC_OK : FC_ERR_CUDA;
 }
 
@@ -1224,13 +1231,14 @@ int launch_rows_wgrad_tc(const WgGeom& g, const float* a, const float* b, float*
 }
 
 int launch_path_split_map_t(const PathGeom& g, const float* Wq, float* ws, cudaStream_t s) {
-  int emax = 0;
+  int emax = 0, kmax = 0;
   for (int l = 0; l <= g.L; ++l) {
-    if (pg_kc(g, l) != 4) return FC_ERR_ARG;
+    if (pg_kc(g, l) != 4 && pg_kc(g, l) != 8) return FC_ERR_ARG;
     emax = pg_pe(g, l) > emax ? pg_pe(g, l) : emax;
+    kmax = pg_kc(g, l) > kmax ? pg_kc(g, l) : kmax;
   }
   if (emax == 0) return FC_OK;
-  path_split_map_t_kernel<<<dim3(4, emax, g.L + 1), 256, 0, s>>>(g, Wq, ws);
+  path_split_map_t_kernel<<<dim3(kmax, emax, g.L + 1), 256, 0, s>>>(g, Wq, ws);
   return cudaGetLastError() == cudaSuccess ? FC_OK : FC_ERR_CUDA;
 }
 

@@ -308,14 +308,14 @@ int fc_ladder_num_paths(const fc_ladder_desc *desc);
  *   mix_w [order-1][lmax+1][C][C] (row = output channel),
  *   states [order-1][n_nodes][(lmax+1)^2 C] receives A_2 .. A_order,
  *   z [n_nodes][(lmax+1)^2 C].
- * At C = 128 the per-rank mix runs on the tcgen05 tensor cores (FP32
- * accuracy through a three-term TF32 split) and z is summed in one pass at
- * the end; other widths use FP32 SIMT kernels.
+ * At C = 128 and 256 the per-rank mix runs on the tcgen05 tensor cores
+ * (FP32 accuracy through a three-term TF32 split) and z is summed in one
+ * pass at the end; other widths use FP32 SIMT kernels.
  * workspace: fc_product_ladder_workspace_size() bytes of device scratch,
  * 16-byte aligned, ws_bytes = its real size; FC_ERR_WORKSPACE if NULL or
- * smaller.  At C = 128 that is the product as FP32 128-node tiles per rank
- * and component (about one product state, node count rounded up to 128)
- * plus one step's TF32 hi / lo matrices; otherwise one product state.
+ * smaller.  At C = 128 and 256 that is the product as FP32 128-node tiles
+ * per rank and component (about one product state, node count rounded up to
+ * 128) plus one step's TF32 hi / lo matrices; otherwise one product state.
  * order = 1 copies A1 to z and needs no workspace. */
 size_t fc_product_ladder_workspace_size(const fc_ladder_desc *desc, int n_nodes);
 int fc_product_ladder(const fc_ladder_desc *desc, int n_nodes, const float *A1,
@@ -327,10 +327,12 @@ int fc_product_ladder(const fc_ladder_desc *desc, int n_nodes, const float *A1,
  * given gz (gradient of z, node layout) and the states of the forward call,
  * writes A1_bar (node layout), path_w_bar [order-1][P][C] and mix_w_bar
  * [order-1][lmax+1][C][C].  The weight gradients sum over all nodes with
- * atomic additions (not bitwise reproducible).  workspace:
- * fc_product_ladder_vjp_workspace_size() bytes (four product states, plus
- * the tensor-core scratch of fc_product_ladder at C = 128); ws_bytes = its
- * real size, FC_ERR_WORKSPACE if smaller. */
+ * atomic additions (not bitwise reproducible).  At C = 128 the mix
+ * B_bar = A_bar M and the weight gradient run on the tensor cores, at
+ * C = 256 the mix only.  workspace: fc_product_ladder_vjp_workspace_size()
+ * bytes (four product states, plus at C = 128 and 256 the gradient as
+ * TF32-split or FP32 128-row tiles and one step's split matrices); ws_bytes
+ * = its real size, FC_ERR_WORKSPACE if smaller. */
 size_t fc_product_ladder_vjp_workspace_size(const fc_ladder_desc *desc, int n_nodes);
 int fc_product_ladder_vjp(const fc_ladder_desc *desc, int n_nodes,
                           const float *A1, const float *path_w,

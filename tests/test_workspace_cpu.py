@@ -82,6 +82,10 @@ def test_ladder_vjp(fc, L, N):
     split = tiles * 2 * 128 * 128 + (L + 1) * 2 * 128 * 128
     assert query(fc, "fc_product_ladder_vjp_workspace_size", L, 128, 4, N) == 4 * (states + split)
     assert query(fc, "fc_product_ladder_vjp_workspace_size", L, 64, 4, N) == 4 * 4 * N * NY * 64
+    # C = 256: the gradient as FP32 tiles of K = 256 and the transposed maps
+    tiles256 = NY * ((N + 127) // 128) * 128 * 256
+    assert query(fc, "fc_product_ladder_vjp_workspace_size", L, 256, 4, N) == \
+        4 * (4 * N * NY * 256 + tiles256 + (L + 1) * 2 * 256 * 256)
 
 
 def test_unsupported_descriptors_need_nothing(fc):
