@@ -97,3 +97,23 @@ def test_odd_rank5_is_refused(fc):
     st = fc.lib().fc_edge_conv_odd(ct.byref(d), t["n_nodes"], ei.shape[1], fc._ptr(rp), fc._ptr(ei),
                                    fc._ptr(ev), fc._ptr(x), fc._ptr(x), fc._ptr(z), None)
     assert st == 4
+
+
+@pytest.mark.parametrize("L,sum_paths", [(1, False), (2, True), (3, False), (4, False)])
+def test_odd_conv_half_warp_pairs_c64(fc, L, sum_paths):
+    """C = 64 runs two receivers per warp, one per half-warp, for the odd-J
+    paths too: an odd receiver count and paired receivers of unequal degree
+    (0 beside 33, 40 beside 2, 16 beside 17), forward and VJP."""
+    degrees = [0, 33, 1, 0, 31, 40, 2, 16, 17] + [3] * 40
+    n = len(degrees)                                        # 49 receivers
+    C = 64
+    ei, ev = ragged_graph(n, degrees, 6.0, 950 + L)
+    x, w, gz = odd_inputs(n, ei, L, C, 960 + L, sum_paths)
+    z, (xb, wb, rb) = run(fc, L, ei, ev, n, x, w, gz, sum_paths)
+    ref = O.edge_conv(L, L, L, C, ei, ev, x, w, n, sum_paths=sum_paths, odd=True)
+    assert rel_err(z, ref) <= FWD_TOL
+    assert np.all(z[[i for i, k in enumerate(degrees) if k == 0]] == 0)
+    rx, rw, rr = O.edge_conv_vjp(L, L, L, C, ei, ev, x, w, gz, n, sum_paths=sum_paths, odd=True)
+    for name, a, b in (("x_bar", xb, rx), ("w_bar", wb, rw), ("r_bar", rb, rr)):
+        e = rel_err(a.reshape(b.shape), b)
+        assert e <= VJP_TOL, "%s rel err %g" % (name, e)
