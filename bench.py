@@ -894,7 +894,7 @@ def run_grid(args):
                                       steps, 3, stream)
                 lad.append({"lmax": L, "order": order, "channels": C, "fwd_ms": f_ms, "vjp_ms": v_ms,
                             "mix": ("tcgen05 TF32x3" if C == 128 else
-                                    "tcgen05 TF32x3 fwd, FP32 SIMT VJP" if C == 256 else "FP32 SIMT")})
+                                    "tcgen05 TF32x3, VJP weight gradient FP32 SIMT" if C == 256 else "FP32 SIMT")})
                 del A1, pw, mw, gz, res
                 torch.cuda.empty_cache()
     clocks = sampler.stop()
