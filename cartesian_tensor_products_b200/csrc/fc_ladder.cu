@@ -386,19 +386,26 @@ static int check_ladder_desc(const fc_ladder_desc* d) {
   return FC_OK;
 }
 
+// threads per block of the channel-diagonal kernels (one per channel): the
+// channel count rounded up to a warp, at most 128, so narrow widths idle no
+// more than a warp's remainder
+static int tp_threads(int C) { return C >= 128 ? 128 : (C + 31) / 32 * 32; }
+
 template <int L>
 static int launch_tp(int N, int C, const float* Av, const float* A1, const float* W, float* B,
                      cudaStream_t s) {
-  dim3 grid((N + kLadderFwdChunk - 1) / kLadderFwdChunk, (C + 127) / 128);
-  ladder_tp_kernel<L><<<grid, 128, 0, s>>>(N, C, Av, A1, W, B);
+  const int tb = tp_threads(C);
+  dim3 grid((N + kLadderFwdChunk - 1) / kLadderFwdChunk, (C + tb - 1) / tb);
+  ladder_tp_kernel<L><<<grid, tb, 0, s>>>(N, C, Av, A1, W, B);
   return cudaGetLastError() == cudaSuccess ? FC_OK : FC_ERR_CUDA;
 }
 
 template <int L>
 static int launch_tp_vjp(int N, int C, const float* Av, const float* A1, const float* W,
                          const float* G, float* Avbar, float* A1bar, float* Wbar, cudaStream_t s) {
-  dim3 grid((N + kLadderNodeChunk - 1) / kLadderNodeChunk, (C + 127) / 128);
-  ladder_tp_vjp_kernel<L><<<grid, 128, 0, s>>>(N, C, Av, A1, W, G, Avbar, A1bar, Wbar);
+  const int tb = tp_threads(C);
+  dim3 grid((N + kLadderNodeChunk - 1) / kLadderNodeChunk, (C + tb - 1) / tb);
+  ladder_tp_vjp_kernel<L><<<grid, tb, 0, s>>>(N, C, Av, A1, W, G, Avbar, A1bar, Wbar);
   return cudaGetLastError() == cudaSuccess ? FC_OK : FC_ERR_CUDA;
 }
 

@@ -37,7 +37,7 @@ def run_gpu(fc, wl, gz=None):
 
 
 @pytest.mark.parametrize("L,C,order,N", [(1, 8, 5, 30), (2, 8, 4, 24), (3, 8, 4, 20), (3, 12, 3, 17),
-                                         (4, 4, 3, 9), (3, 40, 5, 10)])
+                                         (4, 4, 3, 9), (3, 40, 5, 10), (3, 64, 4, 45), (2, 96, 3, 20)])
 def test_small_ladder_full(fc, L, C, order, N):
     wl = dict(lmax=L, channels=C, order=order,
               **W.ladder_inputs(N, L, C, order, 1000 + 10 * L + C))
